@@ -1,0 +1,331 @@
+"""Exact-budget LapSum soft top-k on the NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/lapsum_topk.h``: it only
+marshals tensors, sizes and the current CUDA stream into the native library
+``liblapsum_topk.so``; every step of the operator runs in that library's
+kernels.  There is no CPU path: CPU tensors are rejected and a missing or
+unbuildable library raises.
+
+Operator ("Fast LapSum: Exact Differentiable Top-k at Million Scale",
+technical summary section 2.1): p_i = F((r_i - b)/alpha) with F the Laplace
+CDF and b chosen so that sum_i p_i = k; backward grad_j = f_j (g_j - lambda),
+lambda = sum g f / sum f.
+
+    import torch, differentiable_soft_top_b200 as lt
+    p = lt.soft_topk(scores, k=1000.0, alpha=0.1)       # autograd-aware
+    res = lt.forward(scores, 1000.0, 0.1, stats=True)   # p, b, sum f, status
+    grad, dk = lt.backward(scores, g, res.b, 0.1)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import numpy as np
+
+__all__ = [
+    "Params", "ForwardResult", "forward", "backward", "forward_into", "backward_into", "soft_topk", "SoftTopK", "workspace_size",
+    "status_string", "launch_count", "trace_enable", "trace_collect", "library_path", "STATS_DTYPE", "ROW_CERTIFIED", "ROW_WIDENED",
+    "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "FORCE_NONE", "FORCE_FALLBACK",
+    "FORCE_STREAMING", "LapsumError",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "liblapsum_topk.so")
+
+LAPSUM_OK, LAPSUM_EINVAL, LAPSUM_EBADK, LAPSUM_EBADALPHA, LAPSUM_EWORKSPACE, LAPSUM_ECUDA = range(6)
+ROW_CERTIFIED, ROW_WIDENED, ROW_FALLBACK = 0x01, 0x02, 0x04
+ROW_NONFINITE, ROW_TIMEOUT, ROW_OVERFLOW = 0x08, 0x10, 0x20
+FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
+
+
+class LapsumError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+        self.code = code
+
+
+class _CParams(ctypes.Structure):
+    _fields_ = [
+        ("sample_m", ctypes.c_uint32),
+        ("force_path", ctypes.c_uint32),
+        ("z", ctypes.c_double),
+        ("seed", ctypes.c_uint64),
+        ("band_capacity", ctypes.c_int64),
+        ("max_widen", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+
+STATS_DTYPE = np.dtype([
+    ("a_L", np.float32), ("a_R", np.float32),
+    ("n_L", np.int64), ("n_R", np.int64), ("band", np.int64),
+    ("S_L", np.float64), ("S_R", np.float64),
+    ("b", np.float64), ("sum_p", np.float64), ("sum_f", np.float64),
+    ("sample_m", np.int32), ("buckets", np.int32),
+    ("status", np.uint32), ("reserved", np.int32),
+], align=True)
+assert STATS_DTYPE.itemsize == 88
+
+
+@dataclass
+class Params:
+    """Tuning and test knobs (lapsum_params).  Zero / negative = automatic."""
+    sample_m: int = 0
+    force_path: int = FORCE_NONE
+    z: float = 5.0
+    seed: int = 0
+    band_capacity: int = 0
+    max_widen: int = -1
+
+    def _c(self) -> _CParams:
+        return _CParams(int(self.sample_m), int(self.force_path), float(self.z),
+                        int(self.seed) & (2**64 - 1), int(self.band_capacity), int(self.max_widen), 0)
+
+
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lib_lock:
+        if _lib is None:
+            from . import _build
+            if _build.stale(_LIB_PATH):
+                _build.build()
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(f"native library missing: {_LIB_PATH}")
+            lib = ctypes.CDLL(_LIB_PATH)
+            P, i64, dbl, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+            lib.lapsum_default_params.argtypes = [P]
+            lib.lapsum_default_params.restype = None
+            lib.lapsum_topk_workspace_size.argtypes = [i64, i64, P]
+            lib.lapsum_topk_workspace_size.restype = sz
+            lib.lapsum_topk_fwd.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, sz, P, P]
+            lib.lapsum_topk_fwd.restype = ctypes.c_int
+            lib.lapsum_topk_bwd.argtypes = [P, P, P, P, i64, i64, i64, dbl, P, P, P, sz, P]
+            lib.lapsum_topk_bwd.restype = ctypes.c_int
+            lib.lapsum_status_string.argtypes = [ctypes.c_int]
+            lib.lapsum_status_string.restype = ctypes.c_char_p
+            lib.lapsum_launch_count.argtypes = []
+            lib.lapsum_launch_count.restype = ctypes.c_uint64
+            lib.lapsum_trace_enable.argtypes = [ctypes.c_int]
+            lib.lapsum_trace_enable.restype = None
+            lib.lapsum_trace_collect.argtypes = [ctypes.c_char_p, sz]
+            lib.lapsum_trace_collect.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return _load().lapsum_status_string(int(code)).decode()
+
+
+def launch_count() -> int:
+    """Kernels the native library has launched in this process."""
+    return int(_load().lapsum_launch_count())
+
+
+def trace_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events (see trace_collect)."""
+    _load().lapsum_trace_enable(1 if on else 0)
+
+
+def trace_collect() -> dict:
+    """{kernel: (launches, total_ms)} of the launches traced since the last call."""
+    import json
+    lib = _load()
+    need = lib.lapsum_trace_collect(None, 0)
+    buf = ctypes.create_string_buffer(max(need, 2) + 64)
+    n = lib.lapsum_trace_collect(buf, len(buf))
+    if n < 0:
+        raise RuntimeError("lapsum_trace_collect failed")
+    return {k: (int(v[0]), float(v[1])) for k, v in json.loads(buf.value.decode()).items()}
+
+
+def _params_ptr(params: Params | None):
+    if params is None:
+        return None, None
+    c = params._c()
+    return c, ctypes.byref(c)
+
+
+def workspace_size(rows: int, n: int, params: Params | None = None) -> int:
+    c, ptr = _params_ptr(params)
+    return int(_load().lapsum_topk_workspace_size(int(rows), int(n), ptr))
+
+
+# ---------------------------------------------------------------------------
+# tensor marshalling (torch is only the owner of device memory and streams)
+# ---------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+_ws_cache: dict = {}
+
+
+def _workspace(device, nbytes: int):
+    torch = _torch()
+    stream = torch.cuda.current_stream(device).cuda_stream
+    key = (device.index if device.index is not None else torch.cuda.current_device(), stream)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def _as_rows(t, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (this library has no CPU path)")
+    if t.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32")
+    if t.dim() == 1:
+        t2 = t.view(1, -1)
+    elif t.dim() == 2:
+        t2 = t
+    else:
+        raise ValueError(f"{name} must be 1-D or 2-D")
+    if t2.stride(1) != 1:
+        t2 = t2.contiguous()
+    return t2
+
+
+@dataclass
+class ForwardResult:
+    p: object          # torch.Tensor, same shape as scores
+    b: object          # torch.Tensor float64 [rows]
+    sumf: object       # torch.Tensor float64 [rows]
+    status: object     # torch.Tensor int32 view of uint32 [rows]
+    stats: np.ndarray | None = None  # STATS_DTYPE [rows], when requested
+
+
+def forward(scores, k: float, alpha: float, *, params: Params | None = None, workspace=None,
+            stats: bool = False, p_out=None) -> ForwardResult:
+    """Thresholds and memberships for every row of `scores` (CUDA fp32)."""
+    torch = _torch()
+    lib = _load()
+    x = _as_rows(scores, "scores")
+    rows, n = x.shape
+    dev = x.device
+    p = torch.empty_like(x) if p_out is None else _as_rows(p_out, "p_out")
+    b = torch.empty(rows, dtype=torch.float64, device=dev)
+    sumf = torch.empty(rows, dtype=torch.float64, device=dev)
+    status = torch.empty(rows, dtype=torch.int32, device=dev)
+    st = torch.empty(rows * STATS_DTYPE.itemsize, dtype=torch.uint8, device=dev) if stats else None
+    c, pptr = _params_ptr(params)
+    need = int(lib.lapsum_topk_workspace_size(rows, n, pptr))
+    ws = workspace if workspace is not None else _workspace(dev, need)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = lib.lapsum_topk_fwd(x.data_ptr(), rows, n, x.stride(0), float(k), float(alpha), p.data_ptr(),
+                             b.data_ptr(), sumf.data_ptr(), status.data_ptr(),
+                             st.data_ptr() if st is not None else None, ws.data_ptr(), ws.numel(), pptr,
+                             stream)
+    if rc != LAPSUM_OK:
+        raise LapsumError(rc, "lapsum_topk_fwd")
+    stats_np = st.cpu().numpy().view(STATS_DTYPE) if st is not None else None
+    return ForwardResult(p.view(scores.shape) if p_out is None else p_out, b, sumf, status, stats_np)
+
+
+def backward(scores, grad_p, b, alpha: float, *, sumf=None, workspace=None, grad_out=None):
+    """dL/dscores and dL/dk for upstream gradient `grad_p` at thresholds `b`."""
+    torch = _torch()
+    lib = _load()
+    x = _as_rows(scores, "scores")
+    g = _as_rows(grad_p, "grad_p")
+    rows, n = x.shape
+    if g.shape != x.shape or g.stride(0) != x.stride(0):
+        g = g.reshape(rows, n).contiguous()
+        if x.stride(0) != n:
+            x = x.contiguous()
+    dev = x.device
+    out = torch.empty_like(x) if grad_out is None else _as_rows(grad_out, "grad_out")
+    gk = torch.empty(rows, dtype=torch.float64, device=dev)
+    bb = b.to(device=dev, dtype=torch.float64).contiguous()
+    sf = sumf.to(device=dev, dtype=torch.float64).contiguous() if sumf is not None else None
+    need = int(lib.lapsum_topk_workspace_size(rows, n, None))
+    ws = workspace if workspace is not None else _workspace(dev, need)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = lib.lapsum_topk_bwd(x.data_ptr(), g.data_ptr(), bb.data_ptr(), sf.data_ptr() if sf is not None else None,
+                             rows, n, x.stride(0), float(alpha), out.data_ptr(), gk.data_ptr(), ws.data_ptr(),
+                             ws.numel(), stream)
+    if rc != LAPSUM_OK:
+        raise LapsumError(rc, "lapsum_topk_bwd")
+    return (out.view(scores.shape) if grad_out is None else grad_out), gk
+
+
+def forward_into(scores, k: float, alpha: float, p, b, sumf, status, workspace, params: Params | None = None,
+                 stats=None) -> None:
+    """forward() with every output preallocated (no allocation in the call)."""
+    torch = _torch()
+    lib = _load()
+    rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
+    stride = scores.stride(0) if scores.dim() == 2 else n
+    c, pptr = _params_ptr(params)
+    rc = lib.lapsum_topk_fwd(scores.data_ptr(), rows, n, stride, float(k), float(alpha), p.data_ptr(), b.data_ptr(),
+                             sumf.data_ptr() if sumf is not None else None,
+                             status.data_ptr() if status is not None else None,
+                             stats.data_ptr() if stats is not None else None, workspace.data_ptr(),
+                             workspace.numel(), pptr, torch.cuda.current_stream(scores.device).cuda_stream)
+    if rc != LAPSUM_OK:
+        raise LapsumError(rc, "lapsum_topk_fwd")
+
+
+def backward_into(scores, grad_p, b, alpha: float, grad, workspace, sumf=None, grad_k=None) -> None:
+    """backward() with every output preallocated (no allocation in the call)."""
+    torch = _torch()
+    lib = _load()
+    rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
+    stride = scores.stride(0) if scores.dim() == 2 else n
+    rc = lib.lapsum_topk_bwd(scores.data_ptr(), grad_p.data_ptr(), b.data_ptr(),
+                             sumf.data_ptr() if sumf is not None else None, rows, n, stride, float(alpha),
+                             grad.data_ptr(), grad_k.data_ptr() if grad_k is not None else None,
+                             workspace.data_ptr(), workspace.numel(),
+                             torch.cuda.current_stream(scores.device).cuda_stream)
+    if rc != LAPSUM_OK:
+        raise LapsumError(rc, "lapsum_topk_bwd")
+
+
+class SoftTopK:
+    """torch.autograd.Function wrapper: p = soft_topk(scores, k, alpha)."""
+
+    _fn = None
+
+    @classmethod
+    def fn(cls):
+        if cls._fn is None:
+            torch = _torch()
+
+            class _F(torch.autograd.Function):
+                @staticmethod
+                def forward(ctx, scores, k, alpha, params):
+                    res = forward(scores, k, alpha, params=params)
+                    ctx.save_for_backward(scores, res.b, res.sumf)
+                    ctx.alpha = alpha
+                    return res.p
+
+                @staticmethod
+                def backward(ctx, gp):
+                    scores, b, sumf = ctx.saved_tensors
+                    gs, gk = backward(scores, gp.contiguous(), b, ctx.alpha, sumf=sumf)
+                    return gs, None, None, None
+
+            cls._fn = _F
+        return cls._fn
+
+
+def soft_topk(scores, k: float, alpha: float, params: Params | None = None):
+    """Differentiable exact-budget soft top-k memberships of `scores` (CUDA fp32)."""
+    return SoftTopK.fn().apply(scores, float(k), float(alpha), params)

@@ -1,0 +1,376 @@
+// abi.cu -- the C ABI of lapsum_topk.h: argument checks, the localization
+// plan, workspace layout and dispatch to the resident (one block per row) or
+// streaming (many blocks per row) kernels.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+#include "lapsum_topk.h"
+
+namespace lapsum {
+
+cudaError_t resident_init();
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+struct DevInfo {
+  bool ready = false;
+  int sm_count = 0;
+  StreamOcc occ{};  // for C = kBucketMax
+};
+DevInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+cudaError_t device_info(DevInfo** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DevInfo* d = &g_dev[dev];
+  if (!d->ready) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!d->ready) {
+      e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      e = resident_init();
+      if (e != cudaSuccess) return e;
+      e = stream_occupancy(kBucketMax, &d->occ);
+      if (e != cudaSuccess) return e;
+      d->ready = true;
+    }
+  }
+  *out = d;
+  return cudaSuccess;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Resolved {
+  double z;
+  uint64_t seed;
+  int max_widen;
+  uint32_t force;
+  uint32_t m_user;
+  int64_t bcap_user;
+};
+
+Resolved resolve(const lapsum_params* p) {
+  Resolved r;
+  r.z = (p && p->z > 0.0 && std::isfinite(p->z)) ? p->z : 5.0;
+  r.seed = p ? p->seed : 0;
+  r.max_widen = (p && p->max_widen >= 0) ? std::min(p->max_widen, 1) : 1;
+  r.force = p ? p->force_path : 0u;
+  r.m_user = p ? p->sample_m : 0u;
+  r.bcap_user = p ? p->band_capacity : 0;
+  return r;
+}
+
+// Localization ranks (section 2.2): #{Y > b} ~ Binomial(m, k/n); the bracket
+// edges are the c_lo-th and (c_hi+1)-th largest samples, c_lo/hi = mq -/+ z sigma.
+struct Ranks {
+  int rank_lo, rank_hi;  // ascending indices into the sorted sample
+  int valid_lo, valid_hi;
+  int widen_delta;
+};
+Ranks sample_ranks(int64_t n, double k, int m, double z) {
+  const double q = k / (double)n;
+  const double mq = (double)m * q;
+  const double sigma = std::sqrt(mq * (1.0 - q));
+  const int64_t c_lo = (int64_t)std::floor(mq - z * sigma);
+  const int64_t c_hi = (int64_t)std::ceil(mq + z * sigma);
+  Ranks R;
+  R.valid_hi = c_lo >= 1;
+  R.rank_hi = R.valid_hi ? (int)(m - c_lo) : m - 1;
+  R.valid_lo = (c_hi + 1) <= m;
+  R.rank_lo = R.valid_lo ? (int)(m - c_hi - 1) : 0;
+  R.widen_delta = (int)std::ceil(2.0 * z * sigma) + 1;
+  return R;
+}
+
+int round_up(int64_t x, int64_t a) { return (int)(((x + a - 1) / a) * a); }
+
+bool resident_path(int64_t n, const Resolved& R) {
+  return n <= kResidentMaxN && !(R.force & LAPSUM_FORCE_STREAMING);
+}
+
+// ---- resident plan -------------------------------------------------------
+struct ResPlan {
+  int m, bcap;
+  Ranks rk;
+};
+ResPlan resident_plan(int64_t n, double k, const Resolved& R) {
+  ResPlan p;
+  const double q = k / (double)n;
+  if (R.m_user) {
+    p.m = (int)std::min<uint32_t>(R.m_user, 4096u);
+  } else {
+    const double opt = std::pow(R.z * (double)n * std::sqrt(q * (1.0 - q)), 2.0 / 3.0);
+    p.m = std::min(2048, std::max(128, round_up((int64_t)std::ceil(opt), 32)));
+  }
+  p.rk = sample_ranks(n, k, p.m, R.z);
+  const double M_est = (double)(p.rk.rank_hi - p.rk.rank_lo + 1) * (double)n / (double)p.m;
+  int64_t bcap = R.bcap_user > 0 ? R.bcap_user : (int64_t)(2.0 * M_est) + 256;
+  bcap = std::max<int64_t>(1, std::min<int64_t>(bcap, std::min<int64_t>(n, 8192)));
+  p.bcap = round_up(bcap, 4);
+  return p;
+}
+
+// ---- streaming plan and workspace ---------------------------------------
+struct StreamSizes {
+  int m;
+  Ranks rk;
+  int T, C, T_max;
+  int64_t band_cap;
+};
+StreamSizes stream_sizes(int64_t n, double k, const Resolved& R) {
+  StreamSizes s;
+  s.m = R.m_user ? (int)std::min<uint32_t>(R.m_user, 1u << 20)
+                 : (int)std::min<int64_t>(1 << 17, std::max<int64_t>(2048, round_up(n / 8, 1024)));
+  s.rk = sample_ranks(n, k, s.m, R.z);
+  const double M_est = (double)(s.rk.rank_hi - s.rk.rank_lo + 1) * (double)n / (double)s.m;
+  int64_t cap = R.bcap_user > 0 ? R.bcap_user : (int64_t)(8.0 * M_est) + 65536;
+  cap = std::max<int64_t>(1024, std::min<int64_t>(cap, (int64_t)round_up(n, 1024)));
+  s.band_cap = round_up(cap, 4);
+  s.T_max = (int)std::max<int64_t>(1, std::min<int64_t>(4096, s.band_cap / 256));
+  plan_buckets(n, s.m, s.rk.rank_lo, s.rk.rank_hi, s.T_max, s.band_cap, &s.T, &s.C);
+  return s;
+}
+
+struct StreamLayout {
+  size_t ctl, h1, h2, h3, cursor, zero_end, samp, fpart, band, aggs, mpart, fb_keys, fb_aggs, rcount, total;
+};
+StreamLayout stream_layout(int64_t rows, int64_t n, const StreamSizes& s) {
+  StreamLayout L;
+  size_t o = 0;
+  L.ctl = o;     o = align256(o + sizeof(RowCtl) * (size_t)rows);
+  L.h1 = o;      o = align256(o + 4 * 2048 * (size_t)rows);
+  L.h2 = o;      o = align256(o + 4 * 4096 * (size_t)rows);
+  L.h3 = o;      o = align256(o + 4 * 2048 * (size_t)rows);
+  L.cursor = o;  o = align256(o + 4 * (size_t)s.T_max * (size_t)rows);
+  L.zero_end = o;
+  L.samp = o;    o = align256(o + 4 * (size_t)s.m * (size_t)rows);
+  L.fpart = o;   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
+  L.band = o;    o = align256(o + 4 * (size_t)s.band_cap * (size_t)rows);
+  L.aggs = o;    o = align256(o + sizeof(GroupAgg) * (size_t)s.T_max * (size_t)rows);
+  L.mpart = o;   o = align256(o + 16 * (size_t)kMaxGridPerRow * (size_t)rows);
+  L.fb_keys = o; o = align256(o + 4 * (size_t)n);
+  L.fb_aggs = o; o = align256(o + sizeof(GroupAgg) * (size_t)(n / kFallbackGroup + 2));
+  L.rcount = o;  o = align256(o + 4 * (256 * (size_t)kMaxGridPerRow + 512));
+  L.total = o;
+  return L;
+}
+
+size_t resident_ws_bytes(int64_t rows) { return align256(4 * (size_t)rows) + 256 + align256(4 * (size_t)rows); }
+
+size_t bwd_ws_bytes(int64_t rows, int64_t n) {
+  if (n <= kResidentMaxN) return 0;
+  return align256(16 * (size_t)kMaxGridPerRow * (size_t)rows) + align256(4 * (size_t)rows) +
+         align256(8 * (size_t)rows);
+}
+
+size_t fwd_ws_bytes(int64_t rows, int64_t n, double k, const Resolved& R) {
+  if (resident_path(n, R)) return resident_ws_bytes(rows);
+  return stream_layout(rows, n, stream_sizes(n, k, R)).total;
+}
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + bn && y < x + an;
+}
+
+}  // namespace
+}  // namespace lapsum
+
+using namespace lapsum;
+
+extern "C" {
+
+void lapsum_default_params(lapsum_params* p) {
+  if (!p) return;
+  std::memset(p, 0, sizeof(*p));
+  p->z = 5.0;
+  p->max_widen = -1;
+}
+
+const char* lapsum_status_string(int code) {
+  switch (code) {
+    case LAPSUM_OK: return "ok";
+    case LAPSUM_EINVAL: return "invalid argument (null or misaligned pointer, bad shape, or overlapping buffers)";
+    case LAPSUM_EBADK: return "k must be finite with 0 < k < n";
+    case LAPSUM_EBADALPHA: return "alpha must be finite and in [1e-30, 1e30]";
+    case LAPSUM_EWORKSPACE: return "workspace missing or smaller than lapsum_topk_workspace_size()";
+    case LAPSUM_ECUDA: return "a CUDA call or kernel launch failed";
+    default: return "unknown status";
+  }
+}
+
+size_t lapsum_topk_workspace_size(int64_t rows, int64_t n, const lapsum_params* params) {
+  if (rows < 1 || n < 1 || n > INT32_MAX) return 0;
+  const Resolved R = resolve(params);
+  // k only shapes the band estimate; size for the widest case (k = n/2)
+  const size_t fwd = std::max(fwd_ws_bytes(rows, n, 0.5 * (double)n, R),
+                              std::max(fwd_ws_bytes(rows, n, 1.0, R), fwd_ws_bytes(rows, n, (double)n - 1.0, R)));
+  return std::max(fwd, bwd_ws_bytes(rows, n));
+}
+
+int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k, double alpha,
+                    float* p_out, double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
+                    void* workspace, size_t workspace_bytes, const lapsum_params* params, void* stream) {
+  if (!scores || !p_out || !b_out) return LAPSUM_EINVAL;
+  if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
+  if (((uintptr_t)scores & 3u) || ((uintptr_t)p_out & 3u) || ((uintptr_t)b_out & 7u)) return LAPSUM_EINVAL;
+  if (sumf_out && ((uintptr_t)sumf_out & 7u)) return LAPSUM_EINVAL;
+  if (!std::isfinite(k) || !(k > 0.0) || !(k < (double)n)) return LAPSUM_EBADK;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
+  if (overlaps(scores, span, p_out, span)) return LAPSUM_EINVAL;
+  const Resolved R = resolve(params);
+  const bool res = resident_path(n, R);
+  if (!res && rows > 65535) return LAPSUM_EINVAL;
+  const size_t need = fwd_ws_bytes(rows, n, k, R);
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)) return LAPSUM_EWORKSPACE;
+
+  DevInfo* dev = nullptr;
+  if (device_info(&dev) != cudaSuccess) return LAPSUM_ECUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+
+  if (res) {
+    const ResPlan rp = resident_plan(n, k, R);
+    ResidentFwd a{};
+    a.scores = scores;
+    a.rows = rows;
+    a.n = n;
+    a.stride = row_stride;
+    a.k = k;
+    a.alpha = alpha;
+    a.p_out = p_out;
+    a.b_out = b_out;
+    a.sumf_out = sumf_out;
+    a.status_out = row_status;
+    a.stats = stats;
+    a.m = rp.m;
+    a.rank_lo = rp.rk.rank_lo;
+    a.rank_hi = rp.rk.rank_hi;
+    a.valid_lo = rp.rk.valid_lo;
+    a.valid_hi = rp.rk.valid_hi;
+    a.widen_delta = rp.rk.widen_delta;
+    a.max_widen = R.max_widen;
+    a.bcap = rp.bcap;
+    a.seed = R.seed;
+    a.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+    a.vec = vec;
+    a.ws_status = reinterpret_cast<uint32_t*>(ws);
+    a.fb_count = reinterpret_cast<uint32_t*>(ws + align256(4 * (size_t)rows));
+    a.fb_list = reinterpret_cast<int32_t*>(ws + align256(4 * (size_t)rows) + 256);
+    if (resident_fwd_smem(a) > 227 * 1024) return LAPSUM_EINVAL;
+    return launch_resident_fwd(a, dev->sm_count, st) == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA;
+  }
+
+  const StreamSizes s = stream_sizes(n, k, R);
+  const StreamLayout L = stream_layout(rows, n, s);
+  StreamOcc occ{};
+  if (stream_occupancy(s.C, &occ) != cudaSuccess) return LAPSUM_ECUDA;
+  StreamPlan P{};
+  P.rows = rows;
+  P.n = n;
+  P.stride = row_stride;
+  P.k = k;
+  P.alpha = alpha;
+  P.m = s.m;
+  P.rank_lo = s.rk.rank_lo;
+  P.rank_hi = s.rk.rank_hi;
+  P.valid_lo = s.rk.valid_lo;
+  P.valid_hi = s.rk.valid_hi;
+  P.widen_delta = s.rk.widen_delta;
+  P.max_widen = R.max_widen;
+  P.T = s.T;
+  P.C = s.C;
+  P.T_max = s.T_max;
+  P.band_cap = s.band_cap;
+  P.seed = R.seed;
+  P.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+  P.vec = vec;
+  const int sm = dev->sm_count;
+  const int64_t per_row = std::max<int64_t>(1, (int64_t)sm * occ.filter_blocks / rows);
+  const int64_t chunks = std::max<int64_t>(1, (n / 4 + 1023) / 1024);
+  P.Gs = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (s.m + 1023) / 1024));
+  P.Gf = (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
+  P.Gm = P.Gf;
+  P.G3 = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)s.T, std::max<int64_t>(1, (int64_t)sm * occ.band_blocks / rows)));
+  P.Gr = std::min(kMaxGridPerRow, sm * occ.recover_blocks);
+  P.ctl = ws + L.ctl;
+  P.zero_bytes = L.zero_end - L.ctl;
+  P.hist1 = reinterpret_cast<uint32_t*>(ws + L.h1);
+  P.hist2 = reinterpret_cast<uint32_t*>(ws + L.h2);
+  P.hist3 = reinterpret_cast<uint32_t*>(ws + L.h3);
+  P.cursor = reinterpret_cast<uint32_t*>(ws + L.cursor);
+  P.samp = reinterpret_cast<uint32_t*>(ws + L.samp);
+  P.fpart = ws + L.fpart;
+  P.band = reinterpret_cast<float*>(ws + L.band);
+  P.aggs = ws + L.aggs;
+  P.mpart = ws + L.mpart;
+  P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
+  P.fb_aggs = ws + L.fb_aggs;
+  P.rcount = reinterpret_cast<uint32_t*>(ws + L.rcount);
+  return launch_stream_fwd(P, scores, p_out, b_out, sumf_out, row_status, stats, sm, st) == cudaSuccess
+             ? LAPSUM_OK
+             : LAPSUM_ECUDA;
+}
+
+int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, const double* sumf, int64_t rows,
+                    int64_t n, int64_t row_stride, double alpha, float* grad_scores, double* grad_k,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (!scores || !grad_p || !b || !grad_scores) return LAPSUM_EINVAL;
+  if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
+  if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)grad_scores & 3u) ||
+      ((uintptr_t)b & 7u))
+    return LAPSUM_EINVAL;
+  if ((sumf && ((uintptr_t)sumf & 7u)) || (grad_k && ((uintptr_t)grad_k & 7u))) return LAPSUM_EINVAL;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
+  if (overlaps(scores, span, grad_scores, span) || overlaps(grad_p, span, grad_scores, span)) return LAPSUM_EINVAL;
+  const size_t need = bwd_ws_bytes(rows, n);
+  if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))) return LAPSUM_EWORKSPACE;
+  if (n > kResidentMaxN && rows > 65535) return LAPSUM_EINVAL;
+  DevInfo* dev = nullptr;
+  if (device_info(&dev) != cudaSuccess) return LAPSUM_ECUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
+  if (n <= kResidentMaxN) {
+    RowBwd a{scores, grad_p, b, sumf, rows, n, row_stride, alpha, grad_scores, grad_k, vec};
+    return launch_resident_bwd(a, dev->sm_count, st) == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA;
+  }
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  StreamBwd a{};
+  a.scores = scores;
+  a.grad_p = grad_p;
+  a.b = b;
+  a.sumf = sumf;
+  a.rows = rows;
+  a.n = n;
+  a.stride = row_stride;
+  a.alpha = alpha;
+  a.grad = grad_scores;
+  a.grad_k = grad_k;
+  a.vec = vec;
+  const int64_t per_row = std::max<int64_t>(1, (int64_t)dev->sm_count * dev->occ.filter_blocks / rows);
+  const int64_t chunks = std::max<int64_t>(1, (n / 4 + 1023) / 1024);
+  a.Gb = (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
+  size_t o = 0;
+  a.part = ws + o;
+  o = align256(o + 16 * (size_t)kMaxGridPerRow * (size_t)rows);
+  a.done = reinterpret_cast<uint32_t*>(ws + o);
+  o = align256(o + 4 * (size_t)rows);
+  a.lam = reinterpret_cast<double*>(ws + o);
+  return launch_stream_bwd(a, st) == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA;
+}
+
+}  // extern "C"

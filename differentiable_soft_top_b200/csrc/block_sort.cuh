@@ -1,0 +1,116 @@
+// block_sort.cuh -- stable LSD radix sort of uint32 keys in shared memory.
+//
+// Used for the band (section 2.2 of the Fast LapSum technical summary: only
+// the band around the threshold is sorted), for the localization sample, and
+// for whole rows in the full-sort fallback.
+//
+// 8-bit digits, four passes.  Each warp owns one contiguous segment of the
+// keys and walks it 32 keys at a time; __match_any_sync groups the lanes that
+// share a digit, so ranks inside a warp follow key order and the pass is
+// stable.  Offsets are laid out digit-major, warp-minor.  A pass whose digit
+// is the same for every key is skipped (band keys usually share their top
+// byte).
+#pragma once
+
+#include "common.cuh"
+
+namespace lapsum {
+
+// shared scratch for the radix routines: NT/32 * 256 counters, a flag word,
+// NT/32 scan words, and 2 * 256 digit words for radix_pass's outputs
+template <int NT>
+struct SortScratch {
+  static constexpr int kWords = (NT / 32) * 256 + 64 + 512;
+};
+
+// One stable pass: keys[0, n) -> tmp[0, n) ordered by digit (key >> shift) & 255.
+// If the digit is the same for every key, nothing is moved and the function
+// returns false (uniformly in all threads); otherwise it returns true.
+// On return hist[NW*256 + 64 + d] holds the count of digit d and
+// hist[NW*256 + 64 + 256 + d] its first position in tmp.
+template <int NT>
+__device__ bool radix_pass(const uint32_t* keys, uint32_t* tmp, int n, uint32_t* hist, int shift,
+                           bool allow_skip = true) {
+  static_assert(NT >= 256 && NT % 32 == 0, "radix_pass needs >= 256 threads");
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int per = (n + NW - 1) / NW;
+  const int seg_lo = min(n, warp * per);
+  const int seg_hi = min(n, seg_lo + per);
+  uint32_t* whist = hist + warp * 256;
+  uint32_t* flag = hist + NW * 256;
+  uint32_t* scan_scr = flag + 1;  // NW words
+  uint32_t* dcount = hist + NW * 256 + 64;
+  uint32_t* dstart = dcount + 256;
+
+  __syncthreads();  // previous users of hist are done
+  for (int i = threadIdx.x; i < NW * 256; i += NT) hist[i] = 0u;
+  if (threadIdx.x == 0) flag[0] = 0u;
+  __syncthreads();
+  for (int base = seg_lo; base < seg_hi; base += 32) {
+    const int i = base + lane;
+    const bool act = i < seg_hi;
+    const uint32_t d = act ? ((keys[i] >> shift) & 255u) : 0u;
+    const uint32_t amask = __ballot_sync(0xffffffffu, act);
+    if (act) {
+      const uint32_t peers = __match_any_sync(amask, d);
+      if (lane == __ffs(peers) - 1) whist[d] += __popc(peers);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  uint32_t tot = 0;
+  if (threadIdx.x < 256) {
+    const uint32_t d = threadIdx.x;
+    for (int w = 0; w < NW; ++w) {
+      const uint32_t c = hist[w * 256 + d];
+      hist[w * 256 + d] = tot;
+      tot += c;
+    }
+    if (tot == (uint32_t)n) flag[0] = 1u;
+  }
+  const uint32_t base_d = block_excl_prefix_u32<NT>(threadIdx.x < 256 ? tot : 0u, scan_scr, nullptr);
+  if (threadIdx.x < 256) {
+    for (int w = 0; w < NW; ++w) hist[w * 256 + threadIdx.x] += base_d;
+    dcount[threadIdx.x] = tot;
+    dstart[threadIdx.x] = base_d;
+  }
+  __syncthreads();
+  const bool skip = allow_skip && flag[0] != 0u;
+  if (skip) return false;
+  for (int base = seg_lo; base < seg_hi; base += 32) {
+    const int i = base + lane;
+    const bool act = i < seg_hi;
+    const uint32_t k = act ? keys[i] : 0u;
+    const uint32_t d = (k >> shift) & 255u;
+    const uint32_t amask = __ballot_sync(0xffffffffu, act);
+    uint32_t peers = 0u;
+    if (act) {
+      peers = __match_any_sync(amask, d);
+      tmp[whist[d] + __popc(peers & lt_mask)] = k;
+    }
+    __syncwarp();
+    if (act && lane == __ffs(peers) - 1) whist[d] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  return true;
+}
+
+// Sorts keys[0, n) ascending.  `tmp` must hold n keys; `hist` must hold
+// SortScratch<NT>::kWords words.  Returns the buffer (keys or tmp) that holds
+// the result.  All NT threads of the block must call it.
+template <int NT>
+__device__ uint32_t* block_radix_sort(uint32_t* keys, uint32_t* tmp, int n, uint32_t* hist) {
+  for (int shift = 0; shift < 32; shift += 8) {
+    if (radix_pass<NT>(keys, tmp, n, hist, shift)) {
+      uint32_t* t = keys;
+      keys = tmp;
+      tmp = t;
+    }
+  }
+  return keys;
+}
+
+}  // namespace lapsum

@@ -1,0 +1,394 @@
+// common.cuh -- device building blocks of the B200 LapSum soft top-k.
+//
+// Method: "Fast LapSum: Exact Differentiable Top-k at Million Scale"
+// (Technical Summary sections 2.1-2.2; arXiv abstract of the same paper).
+#pragma once
+
+#include <cstdint>
+#include <cstring>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+namespace lapsum {
+
+// ---------------------------------------------------------------------------
+// row status bits.  The low byte mirrors LAPSUM_ROW_* of lapsum_topk.h; the
+// rest are internal hand-offs between kernels and never reach the caller.
+// ---------------------------------------------------------------------------
+constexpr uint32_t ROW_CERTIFIED = 0x01u;
+constexpr uint32_t ROW_WIDENED = 0x02u;
+constexpr uint32_t ROW_FALLBACK = 0x04u;
+constexpr uint32_t ROW_NONFINITE = 0x08u;
+constexpr uint32_t ROW_TIMEOUT = 0x10u;
+constexpr uint32_t ROW_OVERFLOW = 0x20u;
+constexpr uint32_t ROW_PUBLIC = 0xFFu;
+constexpr uint32_t ROW_MISS_LEFT = 0x100u;   // S(a_L) < k: b lies below a_L
+constexpr uint32_t ROW_MISS_RIGHT = 0x200u;  // S(a_R) >= k: b lies at or above a_R
+constexpr uint32_t ROW_FORCE_FB = 0x400u;    // test knob: take the full sort
+constexpr uint32_t ROW_NEEDS_RECOVERY = ROW_MISS_LEFT | ROW_MISS_RIGHT | ROW_OVERFLOW | ROW_FORCE_FB;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// splitmix64 (Steele, Lea & Flood, OOPSLA 2014), used counter-style: the i-th
+// output (i >= 1) of a generator whose state starts at s is mix(s + i*gamma).
+// ---------------------------------------------------------------------------
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+
+__host__ __device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+__host__ __device__ __forceinline__ uint64_t sm64_out(uint64_t s, uint64_t i) {
+  return sm64_mix(s + i * kGamma);
+}
+// stream of one row: the (row+1)-th output of a generator seeded with `seed`
+__host__ __device__ __forceinline__ uint64_t row_stream(uint64_t seed, uint64_t row) {
+  return sm64_out(seed, row + 1);
+}
+
+// Localization sample j of a row (section 2.2: scores with Laplace noise):
+// draw 2j+1 picks an index uniformly in [0, n) (high word of draw * n), draw
+// 2j+2 gives u in (0,1) and Laplace(0, alpha) noise by the inverse CDF.
+// Y = r[I] + eps is formed in fp64 and rounded to fp32.
+__device__ __forceinline__ uint64_t sample_index(uint64_t s, uint64_t j, uint64_t n) {
+  return __umul64hi(sm64_out(s, 2 * j + 1), n);
+}
+__device__ __forceinline__ double laplace_noise(uint64_t s, uint64_t j, double alpha) {
+  const uint64_t d = sm64_out(s, 2 * j + 2);
+  const double u = ((double)(d >> 11) + 0.5) * 0x1p-53;
+  const double e = (u < 0.5) ? log(2.0 * u) : -log(2.0 - 2.0 * u);
+  return alpha * e;
+}
+
+// ---------------------------------------------------------------------------
+// order-preserving map between fp32 values and uint32 keys (-0 < +0)
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ uint32_t f2key(float f) {
+#ifdef __CUDA_ARCH__
+  const uint32_t u = __float_as_uint(f);
+#else
+  uint32_t u;
+  memcpy(&u, &f, 4);
+#endif
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+}
+__host__ __device__ __forceinline__ float key2f(uint32_t k) {
+  const uint32_t u = k ^ ((k & 0x80000000u) ? 0x80000000u : 0xFFFFFFFFu);
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(u);
+#else
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+#endif
+}
+
+// ---------------------------------------------------------------------------
+// per-row control block kept in the workspace (256 bytes per row)
+// ---------------------------------------------------------------------------
+struct alignas(256) RowCtl {
+  // bracket and band plan, written by the selection step
+  float aL, aR;        // bracket [aL, aR); -inf / +inf when open
+  float lo, inv_w;     // band bucket of x: floor((x - lo) * inv_w), clamped
+  int32_t T, C;        // buckets and slots per bucket
+  int32_t rank_lo, rank_hi;  // ascending sample ranks of the two edges
+  uint32_t valid_lo, valid_hi;
+  int32_t widen_count, m;
+  // aggregates and result
+  int64_t nL, nR, M;
+  double SL, SR;
+  double b;
+  double sumf, sump;
+  uint32_t status;     // ROW_* bits
+  uint32_t flags;      // atomicOr target of the streaming pass
+  uint32_t done_sel, done_solve, done_memb, done_bwd;
+  uint32_t bar_count, bar_gen;
+  uint32_t sel_key[2];
+  double lam;
+  uint32_t timeout;    // set when a bounded grid-wide wait gives up
+};
+static_assert(sizeof(RowCtl) == 256, "RowCtl must stay one 256-byte slot");
+
+// aggregates of one sorted group of band values (a bucket, or a slice of a
+// fully sorted row): count, min, max, P = sum exp((y - ymax)/alpha),
+// Q = sum exp((ymin - y)/alpha); plus scan results filled in by the solver.
+struct alignas(16) GroupAgg {
+  int32_t cnt;
+  float ymin, ymax;
+  int32_t pad;
+  double P, Q;
+  double Apre;           // prefix anchored at ymax (left tail + groups <= t)
+  double Bx, Bs;         // suffix state of everything after the group
+  long long after;       // number of values after the group (incl. right tail)
+};
+
+// ---------------------------------------------------------------------------
+// anchored exponential sums: a state (x, s) means sum_v exp(+-(v - x)/alpha)
+// over a run of sorted values.  s == 0 is the empty run.
+// Prefix states are anchored at the run's maximum (terms exp((v - x)/alpha)),
+// suffix states at its minimum (terms exp((x - v)/alpha)); all terms <= 1.
+// ---------------------------------------------------------------------------
+struct Anch {
+  double x, s;
+};
+__device__ __forceinline__ Anch anch_empty() { return Anch{-CUDART_INF, 0.0}; }
+
+// earlier run a, later run b -> prefix state of a followed by b
+__device__ __forceinline__ Anch comb_pre(Anch a, Anch b, double inva) {
+  if (b.s == 0.0) return a;
+  if (a.s == 0.0) return b;
+  return Anch{b.x, fma(a.s, exp((a.x - b.x) * inva), b.s)};
+}
+// earlier run a, later run b -> suffix state of a followed by b
+__device__ __forceinline__ Anch comb_suf(Anch a, Anch b, double inva) {
+  if (a.s == 0.0) return b;
+  if (b.s == 0.0) return a;
+  return Anch{a.x, fma(b.s, exp((a.x - b.x) * inva), a.s)};
+}
+// value of a prefix state re-anchored at y >= st.x
+__device__ __forceinline__ double pre_at(Anch st, double y, double inva) {
+  return st.s == 0.0 ? 0.0 : st.s * exp((st.x - y) * inva);
+}
+// value of a suffix state re-anchored at y <= st.x
+__device__ __forceinline__ double suf_at(Anch st, double y, double inva) {
+  return st.s == 0.0 ? 0.0 : st.s * exp((y - st.x) * inva);
+}
+
+// ln(m + sqrt(m^2 + e^L)) for m >= 0, without overflow or underflow
+__device__ __forceinline__ double lnsum(double m, double L) {
+  if (m == 0.0) return 0.5 * L;
+  const double lm = log(m);
+  const double D = L - 2.0 * lm;
+  if (D > 0.0) return 0.5 * L + log(exp(-0.5 * D) + sqrt(exp(-D) + 1.0));
+  return lm + log(1.0 + sqrt(1.0 + exp(D)));
+}
+
+// Closed-form root on one interval [xj, xj1] of the threshold curve
+// (section 2.2: once the interval holding b is known, b has a closed form).
+// A  = prefix sum anchored at xj  (values <= xj, the left tail included),
+// Bp = suffix sum anchored at xj1 (values >= xj1, the right tail included),
+// c  = number of values above xj.  With u = exp((b - xj)/alpha) the budget
+// equation is B u^2 - 2 mu u - A = 0, mu = c - k, B = Bp exp(-(xj1-xj)/alpha).
+// The root is taken from the right knot when mu >= 0, from the left otherwise,
+// in log form; the result is clamped into the interval.
+__device__ __forceinline__ double closed_form_root(double xj, double xj1, double A, double Bp,
+                                                   double c, double k, double alpha) {
+  const double mu = c - k;
+  const double lnA = A > 0.0 ? log(A) : -CUDART_INF;
+  const double lnB = Bp > 0.0 ? log(Bp) : -CUDART_INF;
+  double L = -CUDART_INF;
+  if (A > 0.0 && Bp > 0.0) L = lnA + lnB - (xj1 - xj) / alpha;
+  double b;
+  if (mu >= 0.0) {
+    b = (Bp > 0.0) ? xj1 + alpha * (lnsum(mu, L) - lnB) : xj1;
+  } else {
+    b = (A > 0.0) ? xj + alpha * (lnA - lnsum(-mu, L)) : xj;
+  }
+  if (b < xj) b = xj;
+  if (b > xj1) b = xj1;
+  return b;
+}
+
+// ---------------------------------------------------------------------------
+// deterministic block reductions (fixed xor trees; scratch >= NT/32 slots)
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <int NT, typename T>
+__device__ __forceinline__ T block_sum(T v, T* scratch) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_sum(v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  T t = (lane < NW) ? scratch[lane] : T(0);
+  t = warp_sum(t);
+  return t;  // every thread holds the total
+}
+
+template <int NT>
+__device__ __forceinline__ int block_max_int(int v, int* scratch) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  int t = (lane < NW) ? scratch[lane] : INT32_MIN;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t = max(t, __shfl_xor_sync(0xffffffffu, t, o));
+  return t;
+}
+
+template <int NT>
+__device__ __forceinline__ uint32_t block_or(uint32_t v, uint32_t* scratch) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = __reduce_or_sync(0xffffffffu, v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  uint32_t t = (lane < NW) ? scratch[lane] : 0u;
+  return __reduce_or_sync(0xffffffffu, t);
+}
+
+// Block-wide exclusive scan of anchored states (prefix or suffix direction),
+// one state per thread, deterministic.  `scr` needs 2*NT/32 doubles.
+// Forward (prefix): thread t receives the combination of threads < t.
+// Backward (suffix): thread t receives the combination of threads > t.
+template <int NT, bool kPrefix>
+__device__ __forceinline__ Anch block_excl_scan_anch(Anch v, double inva, double* scr) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Anch inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    Anch oth;
+    if (kPrefix) {
+      oth.x = __shfl_up_sync(0xffffffffu, inc.x, o);
+      oth.s = __shfl_up_sync(0xffffffffu, inc.s, o);
+      if (lane >= o) inc = comb_pre(oth, inc, inva);
+    } else {
+      oth.x = __shfl_down_sync(0xffffffffu, inc.x, o);
+      oth.s = __shfl_down_sync(0xffffffffu, inc.s, o);
+      if (lane + o < 32) inc = comb_suf(inc, oth, inva);
+    }
+  }
+  Anch exl;
+  if (kPrefix) {
+    exl.x = __shfl_up_sync(0xffffffffu, inc.x, 1);
+    exl.s = __shfl_up_sync(0xffffffffu, inc.s, 1);
+    if (lane == 0) exl = anch_empty();
+  } else {
+    exl.x = __shfl_down_sync(0xffffffffu, inc.x, 1);
+    exl.s = __shfl_down_sync(0xffffffffu, inc.s, 1);
+    if (lane == 31) exl = anch_empty();
+  }
+  __syncthreads();
+  if ((kPrefix && lane == 31) || (!kPrefix && lane == 0)) {
+    scr[2 * warp] = inc.x;
+    scr[2 * warp + 1] = inc.s;
+  }
+  __syncthreads();
+  Anch wacc = anch_empty();
+  if (kPrefix) {
+    for (int w = 0; w < warp; ++w) wacc = comb_pre(wacc, Anch{scr[2 * w], scr[2 * w + 1]}, inva);
+    return comb_pre(wacc, exl, inva);
+  } else {
+    for (int w = NW - 1; w > warp; --w) wacc = comb_suf(Anch{scr[2 * w], scr[2 * w + 1]}, wacc, inva);
+    return comb_suf(exl, wacc, inva);
+  }
+}
+
+// block-wide exclusive scan of int64 counts in the suffix direction
+template <int NT>
+__device__ __forceinline__ long long block_excl_suffix_sum(long long v, long long* scr) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    long long oth = __shfl_down_sync(0xffffffffu, inc, o);
+    if (lane + o < 32) inc += oth;
+  }
+  long long exl = __shfl_down_sync(0xffffffffu, inc, 1);
+  if (lane == 31) exl = 0;
+  __syncthreads();
+  if (lane == 0) scr[warp] = inc;
+  __syncthreads();
+  long long wacc = 0;
+  for (int w = NW - 1; w > warp; --w) wacc += scr[w];
+  return exl + wacc;
+}
+
+// block-wide exclusive scan of uint32 values (prefix direction)
+template <int NT>
+__device__ __forceinline__ uint32_t block_excl_prefix_u32(uint32_t v, uint32_t* scr, uint32_t* total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t oth = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += oth;
+  }
+  __syncthreads();
+  if (lane == 31) scr[warp] = inc;
+  __syncthreads();
+  uint32_t wacc = 0, tot = 0;
+  for (int w = 0; w < NW; ++w) {
+    if (w < warp) wacc += scr[w];
+    tot += scr[w];
+  }
+  if (total) *total = tot;
+  return wacc + inc - v;
+}
+
+// ---------------------------------------------------------------------------
+// bounded waits.  Every spin in this library gives up after a fixed number
+// of polls, records ROW_TIMEOUT and returns, so a logic error can never hang
+// the GPU.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kSpinLimit = 1u << 22;  // x ~256 ns sleeps: about a second
+
+// Grid-wide barrier for a cooperatively launched grid (all blocks resident).
+// Returns false if the wait timed out; the caller must then stop.
+__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks,
+                                             uint32_t* timeout_flag) {
+  __shared__ uint32_t s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    s_ok = 1u;
+    volatile uint32_t* vgen = gen;
+    const uint32_t my_gen = *vgen;
+    __threadfence();
+    const uint32_t arrived = atomicAdd(count, 1u);
+    if (arrived == nblocks - 1) {
+      *count = 0u;
+      __threadfence();
+      atomicAdd(gen, 1u);
+    } else {
+      uint32_t polls = 0;
+      while (*vgen == my_gen) {
+        if (++polls > kSpinLimit || *((volatile uint32_t*)timeout_flag) != 0u) {
+          atomicOr(timeout_flag, 1u);
+          s_ok = 0u;
+          break;
+        }
+        __nanosleep(256);
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return s_ok != 0u;
+}
+
+// last-block-done: returns true in exactly one block (the last to arrive)
+__device__ __forceinline__ bool last_block_done(uint32_t* counter, uint32_t nblocks) {
+  __shared__ uint32_t s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == nblocks - 1) ? 1u : 0u;
+  __syncthreads();
+  if (s_last) __threadfence();
+  return s_last != 0u;
+}
+
+// ---------------------------------------------------------------------------
+// streaming loads/stores with cache hints
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float4 ldg_stream(const float4* p) { return __ldcs(p); }
+__device__ __forceinline__ float4 ldg_keep(const float4* p) { return __ldg(p); }
+__device__ __forceinline__ void stg_stream(float4* p, float4 v) { __stcs(p, v); }
+
+}  // namespace lapsum

@@ -1,0 +1,161 @@
+// launch.h -- host-side interface between the C ABI (abi.cu) and the kernel
+// translation units.  Not part of the public boundary.
+#pragma once
+
+#include <cmath>
+#include <cstddef>
+#include <cstdint>
+#include <cstring>
+#include <algorithm>
+#include <cuda_runtime.h>
+
+#include "lapsum_topk.h"
+
+namespace lapsum {
+
+void note_launch(int count);
+
+// Scope guard around one kernel launch: counts it and, while tracing is on,
+// brackets it with CUDA events on its stream (see trace.cu).
+class Launch {
+ public:
+  Launch(const char* name, cudaStream_t st);
+  ~Launch();
+  Launch(const Launch&) = delete;
+  Launch& operator=(const Launch&) = delete;
+
+ private:
+  const char* name_;
+  cudaStream_t st_;
+  cudaEvent_t a_ = nullptr, b_ = nullptr;
+};
+
+// rows of at most this many scores run on the resident path (one block per
+// row, the row held in shared memory)
+constexpr int64_t kResidentMaxN = 16384;
+constexpr int kResidentThreads = 256;
+
+struct ResidentFwd {
+  const float* scores;
+  int64_t rows, n, stride;
+  double k, alpha;
+  float* p_out;
+  double* b_out;
+  double* sumf_out;
+  uint32_t* status_out;
+  lapsum_row_stats* stats;
+  // localization plan (identical for every row)
+  int m;                 // sample size
+  int rank_lo, rank_hi;  // ascending sample ranks of a_L and a_R
+  int valid_lo, valid_hi;
+  int widen_delta;       // rank distance of one widening
+  int max_widen;
+  int bcap;              // band capacity
+  uint64_t seed;
+  int force_fallback;
+  int vec;               // scores and p_out rows 16-byte aligned
+  // workspace
+  uint32_t* ws_status;   // [rows]
+  uint32_t* fb_count;    // [1]
+  int32_t* fb_list;      // [rows]
+};
+
+size_t resident_fwd_smem(const ResidentFwd& a);
+size_t resident_fallback_smem(int64_t n);
+cudaError_t launch_resident_fwd(const ResidentFwd& a, int sm_count, cudaStream_t st);
+
+struct RowBwd {
+  const float* scores;
+  const float* grad_p;
+  const double* b;
+  const double* sumf;
+  int64_t rows, n, stride;
+  double alpha;
+  float* grad;
+  double* grad_k;
+  int vec;
+};
+cudaError_t launch_resident_bwd(const RowBwd& a, int sm_count, cudaStream_t st);
+
+// ---- multi-block (streaming) path ---------------------------------------
+struct StreamPlan {
+  int64_t rows, n, stride;
+  double k, alpha;
+  int m;
+  int rank_lo, rank_hi, valid_lo, valid_hi;
+  int widen_delta, max_widen;
+  int T, C;              // buckets and slots per bucket
+  int T_max;
+  int64_t band_cap;      // slots per row
+  uint64_t seed;
+  int force_fallback;
+  int vec;
+  int Gs, Gf, G3, Gm, Gr;  // grids: sampling, filter, band solve, membership, recovery
+  // workspace pieces
+  void* ctl;             // RowCtl[rows] followed by the zeroed per-row block
+  size_t zero_bytes;     // bytes to clear at the start of each forward
+  uint32_t* hist1;       // [rows][2048]
+  uint32_t* hist2;       // [rows][2][2048]
+  uint32_t* hist3;       // [rows][2][1024]
+  uint32_t* cursor;      // [rows][T_max]
+  uint32_t* samp;        // [rows][m]
+  void* fpart;           // filter partials [rows][Gf]
+  float* band;           // [rows][band_cap]
+  void* aggs;            // GroupAgg [rows][T_max]
+  void* mpart;           // membership partials [rows][Gm]
+  uint32_t* fb_keys;     // [n] keys for the full-sort fallback
+  void* fb_aggs;         // GroupAgg [n / kFallbackGroup + 1]
+  uint32_t* rcount;      // radix counts [256 * Gr] (+ scan space)
+};
+
+constexpr int kFallbackGroup = 4096;   // full-sort fallback: sorted values per group
+constexpr int kBucketTarget = 1024;    // expected band values per bucket
+constexpr int kBucketMax = 8192;       // largest bucket one block sorts in shared memory
+constexpr int kMaxGridPerRow = 4096;   // partial-sum slots per row
+constexpr int kStreamThreads = 256;
+
+// Buckets for a band that spans sample ranks [rank_lo, rank_hi]: the expected
+// band size is (rank_hi - rank_lo + 1) n / m values.
+__host__ __device__ inline void plan_buckets(int64_t n, int m, int rank_lo, int rank_hi, int T_max,
+                                             int64_t band_cap, int* T, int* C) {
+  const double M_est = (double)(rank_hi - rank_lo + 1) * (double)n / (double)m;
+  double tt = ceil(M_est / (double)kBucketTarget);
+  if (tt < 1.0) tt = 1.0;
+  if (tt > (double)T_max) tt = (double)T_max;
+  const int t = (int)tt;
+  int64_t c = band_cap / t;
+  if (c > kBucketMax) c = kBucketMax;
+  *T = t;
+  *C = (int)c;
+}
+
+cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p_out, double* b_out,
+                              double* sumf_out, uint32_t* status_out, lapsum_row_stats* stats,
+                              int sm_count, cudaStream_t st);
+
+struct StreamBwd {
+  const float* scores;
+  const float* grad_p;
+  const double* b;
+  const double* sumf;
+  int64_t rows, n, stride;
+  double alpha;
+  float* grad;
+  double* grad_k;
+  int vec;
+  int Gb;
+  void* part;        // [rows][Gb] partials
+  uint32_t* done;    // [rows] counters (zeroed by the launcher)
+  double* lam;       // [rows]
+};
+cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st);
+
+// occupancy facts of the streaming kernels on the current device
+struct StreamOcc {
+  int filter_blocks;    // resident blocks per SM of the streaming passes
+  int band_blocks;      // of the band sort kernel for the given bucket size
+  int recover_blocks;   // of the cooperative recovery kernel
+};
+cudaError_t stream_occupancy(int C, StreamOcc* out);
+
+}  // namespace lapsum

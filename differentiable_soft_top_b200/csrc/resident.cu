@@ -1,0 +1,459 @@
+// resident.cu -- rows that fit one block's shared memory (n <= 16384).
+//
+// One thread block owns a row.  The row is brought into shared memory once by
+// a bulk (TMA) copy; every step of the Fast LapSum pipeline (technical summary
+// section 2.2: localization sample, stream-and-filter, exact solve on the
+// band, certification with one widening) then runs on the copy, and the
+// memberships (section 2.1) are written straight from it.  HBM traffic is one
+// read of the row and one write of p.  Rows whose bracket cannot be certified
+// go to a full-sort fallback kernel (the worst-case branch of the arXiv
+// abstract).  The backward pass (section 2.1's analytic VJP) is one block per
+// row: a reduction for lambda and an elementwise pass.
+#include <algorithm>
+
+#include "block_sort.cuh"
+#include "common.cuh"
+#include "launch.h"
+#include "solve.cuh"
+#include "tma.cuh"
+
+namespace lapsum {
+namespace {
+
+constexpr int NT = kResidentThreads;
+constexpr int kFbGroup = 1024;  // fallback: sorted values per group
+
+struct ResLayout {
+  size_t row, samp, samp_tmp, band, band_tmp, dscr, hist, red, mbar, total;
+};
+
+__host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap) {
+  ResLayout L;
+  size_t o = 0;
+  L.row = o;      o = (o + 4 * (size_t)n + 15) & ~size_t(15);
+  L.samp = o;     o = (o + 4 * (size_t)m + 15) & ~size_t(15);
+  L.samp_tmp = o; o = (o + 4 * (size_t)m + 15) & ~size_t(15);
+  L.band = o;     o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
+  L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
+  L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
+  L.hist = o;     o = (o + 4 * (size_t)SortScratch<NT>::kWords + 15) & ~size_t(15);
+  L.red = o;      o = o + 8 * 64;
+  L.mbar = o;     o = o + 16;
+  L.total = o;
+  return L;
+}
+
+struct KeyRun {  // one group: the sorted band held as keys
+  const uint32_t* k;
+  __device__ float get(int, int i) const { return key2f(k[i]); }
+};
+struct KeyGroups {  // consecutive groups of `g` sorted keys
+  const uint32_t* k;
+  int g;
+  __device__ float get(int grp, int i) const { return key2f(k[grp * g + i]); }
+};
+
+struct Filtered {
+  long long nL, nR;
+  double SL, SR;
+  int M;
+  uint32_t bad;
+};
+
+// One pass over the row in shared memory (section 2.2 stream-and-filter):
+// scores below a_L and at/above a_R go into counts and anchored tail sums
+// (every term exp(-dist/alpha) <= 1, fp32 exp, fp64 sums); scores inside the
+// bracket are appended to the band with one shared atomic per warp.
+__device__ Filtered filter_row(const float* row, int n, float aL, float aR, float c2, uint32_t* band,
+                               int bcap, int* s_cnt, double* red) {
+  if (threadIdx.x == 0) *s_cnt = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  int nl = 0, nr = 0;
+  double sl = 0.0, sr = 0.0;
+  uint32_t bad = 0u;
+  for (int base = 0; base < n; base += NT) {
+    const int i = base + threadIdx.x;
+    const bool act = i < n;
+    const float x = act ? row[i] : 0.0f;
+    const bool isL = x < aL, isR = x >= aR;
+    const float e = exp2f(fminf(x - aL, aR - x) * c2);
+    if (act) {
+      if (isL) { sl += (double)e; ++nl; }
+      if (isR) { sr += (double)e; ++nr; }
+      if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;
+    }
+    const bool inb = act && !(isL || isR);
+    const uint32_t msk = __ballot_sync(0xffffffffu, inb);
+    if (msk) {
+      const int leader = __ffs(msk) - 1;
+      int wbase = 0;
+      if (lane == leader) wbase = atomicAdd(s_cnt, __popc(msk));
+      wbase = __shfl_sync(0xffffffffu, wbase, leader);
+      if (inb) {
+        const int pos = wbase + __popc(msk & lt);
+        if (pos < bcap) band[pos] = f2key(x);
+      }
+    }
+  }
+  Filtered f;
+  f.nL = block_sum<NT, long long>((long long)nl, reinterpret_cast<long long*>(red));
+  f.nR = block_sum<NT, long long>((long long)nr, reinterpret_cast<long long*>(red));
+  f.SL = block_sum<NT, double>(sl, red);
+  f.SR = block_sum<NT, double>(sr, red);
+  f.bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  f.M = *s_cnt;
+  __syncthreads();
+  return f;
+}
+
+// p_i = F((r_i - b)/alpha), with r_i - b formed from b split into two fp32
+// words (b = bh + bl) so that the difference keeps fp64-level accuracy.
+__device__ __forceinline__ float membership(float x, float bh, float bl, float c2, float& h) {
+  const float d = (x - bh) - bl;
+  h = 0.5f * exp2f(-fabsf(d) * c2);
+  return d < 0.0f ? h : 1.0f - h;
+}
+
+__device__ void write_stats(lapsum_row_stats* st, float aL, float aR, long long nL, long long nR, long long M,
+                            double SL, double SR, double b, double sump, double sumf, int m, int buckets,
+                            uint32_t status) {
+  st->a_L = aL;
+  st->a_R = aR;
+  st->n_L = nL;
+  st->n_R = nR;
+  st->band = M;
+  st->S_L = SL;
+  st->S_R = SR;
+  st->b = b;
+  st->sum_p = sump;
+  st->sum_f = sumf;
+  st->sample_m = m;
+  st->buckets = buckets;
+  st->status = status;
+  st->reserved = 0;
+}
+
+// Writes p for a row from `src` (shared or global) and finishes the row's
+// outputs.  Every thread must call it.
+__device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, double b, uint32_t status,
+                           float aL, float aR, long long nL, long long nR, long long M, double SL,
+                           double SR, int buckets, double* red) {
+  const int n = (int)a.n;
+  const double inva = 1.0 / a.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+  const float bh = __double2float_rn(b);
+  const float bl = __double2float_rn(b - (double)bh);
+  float* dst = a.p_out + r * a.stride;
+  double hs = 0.0, ps = 0.0;
+  const bool nonfinite = (status & ROW_NONFINITE) != 0u;
+  if (a.vec) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    float4* d4 = reinterpret_cast<float4*>(dst);
+    const int n4 = n >> 2;
+    for (int v = threadIdx.x; v < n4; v += NT) {
+      const float4 x = s4[v];
+      float4 p;
+      float h0, h1, h2, h3;
+      p.x = membership(x.x, bh, bl, c2, h0);
+      p.y = membership(x.y, bh, bl, c2, h1);
+      p.z = membership(x.z, bh, bl, c2, h2);
+      p.w = membership(x.w, bh, bl, c2, h3);
+      if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
+      hs += (double)((h0 + h1) + (h2 + h3));
+      ps += (double)((p.x + p.y) + (p.z + p.w));
+      stg_stream(d4 + v, p);
+    }
+    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
+      float h;
+      float p = membership(src[i], bh, bl, c2, h);
+      if (nonfinite) p = CUDART_NAN_F;
+      hs += (double)h;
+      ps += (double)p;
+      dst[i] = p;
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += NT) {
+      float h;
+      float p = membership(src[i], bh, bl, c2, h);
+      if (nonfinite) p = CUDART_NAN_F;
+      hs += (double)h;
+      ps += (double)p;
+      dst[i] = p;
+    }
+  }
+  hs = block_sum<NT, double>(hs, red);
+  ps = block_sum<NT, double>(ps, red);
+  if (threadIdx.x == 0) {
+    const double bo = nonfinite ? CUDART_NAN : b;
+    a.b_out[r] = bo;
+    if (a.sumf_out) a.sumf_out[r] = hs * inva;
+    if (a.status_out) a.status_out[r] = status & ROW_PUBLIC;
+    if (a.stats) write_stats(a.stats + r, aL, aR, nL, nR, M, SL, SR, bo, ps, hs * inva, a.m, buckets,
+                             status & ROW_PUBLIC);
+  }
+}
+
+__global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const ResLayout L = res_layout(a.n, a.m, a.bcap);
+  float* row = reinterpret_cast<float*>(smem + L.row);
+  uint32_t* samp = reinterpret_cast<uint32_t*>(smem + L.samp);
+  uint32_t* samp_tmp = reinterpret_cast<uint32_t*>(smem + L.samp_tmp);
+  uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
+  uint32_t* band_tmp = reinterpret_cast<uint32_t*>(smem + L.band_tmp);
+  double* dscr = reinterpret_cast<double*>(smem + L.dscr);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);
+  double* red = reinterpret_cast<double*>(smem + L.red);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
+  __shared__ int s_cnt;
+  __shared__ GroupAgg s_agg;
+  __shared__ SolveOut s_out;
+
+  const int64_t r = blockIdx.x;
+  const int n = (int)a.n;
+  const float* src = a.scores + r * a.stride;
+  const double inva = 1.0 / a.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+
+  // ---- bring the row into shared memory --------------------------------
+  uint32_t status = 0u;
+  if (a.vec) {
+    const uint32_t bytes = (uint32_t)(n >> 2) * 16u;
+    if (threadIdx.x == 0) {
+      mbar_init(mbar, 1);
+      fence_proxy_async_smem();
+      if (bytes > 0) {
+        mbar_arrive_expect_tx(mbar, bytes);
+        for (uint32_t off = 0; off < bytes; off += 16384u)
+          bulk_load(reinterpret_cast<unsigned char*>(row) + off, reinterpret_cast<const unsigned char*>(src) + off,
+                    min(16384u, bytes - off), mbar);
+      }
+    }
+    for (int i = (n & ~3) + threadIdx.x; i < n; i += NT) row[i] = src[i];
+    __syncthreads();
+    const int timed_out = (bytes > 0 && !mbar_wait_bounded(mbar, 0)) ? 1 : 0;
+    if (__syncthreads_or(timed_out)) status |= ROW_TIMEOUT;
+  } else {
+    for (int i = threadIdx.x; i < n; i += NT) row[i] = src[i];
+  }
+  __syncthreads();
+  if (status & ROW_TIMEOUT) {
+    // the copy never completed: wait once more, bounded, then give up on the row
+    mbar_wait_bounded(mbar, 0);
+    if (threadIdx.x == 0) {
+      a.b_out[r] = CUDART_NAN;
+      if (a.status_out) a.status_out[r] = ROW_TIMEOUT;
+    }
+    return;
+  }
+
+  // ---- localization (section 2.2, step 1) ---------------------------------
+  const int m = a.m;
+  const uint64_t s = row_stream(a.seed, (uint64_t)r);
+  for (int j = threadIdx.x; j < m; j += NT) {
+    const uint64_t I = sample_index(s, (uint64_t)j, (uint64_t)n);
+    const double Y = (double)row[I] + laplace_noise(s, (uint64_t)j, a.alpha);
+    samp[j] = f2key(__double2float_rn(Y));
+  }
+  __syncthreads();
+  const uint32_t* ss = block_radix_sort<NT>(samp, samp_tmp, m, hist);
+  __syncthreads();
+  int rlo = a.rank_lo, rhi = a.rank_hi;
+  bool vlo = a.valid_lo != 0, vhi = a.valid_hi != 0;
+  float aL = vlo ? key2f(ss[rlo]) : -CUDART_INF_F;
+  float aR = vhi ? key2f(ss[rhi]) : CUDART_INF_F;
+
+  // ---- filter, sort the band, solve, certify (steps 2-4) ------------------
+  bool solved = false;
+  Filtered f{};
+  if (!a.force_fallback) {
+    for (int attempt = 0;; ++attempt) {
+      f = filter_row(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
+      if (f.bad) { status |= ROW_NONFINITE; break; }
+      if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
+      const uint32_t* bs = block_radix_sort<NT>(band, band_tmp, f.M, hist);
+      __syncthreads();
+      aggregate_sorted_keys<NT, false>(bs, f.M, red, &s_agg, inva);
+      SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, a.k, a.alpha, inva};
+      solve_band<NT, false>(in, &s_agg, 1, KeyRun{bs}, dscr, red, &s_out);
+      if (s_out.status & ROW_CERTIFIED) { solved = true; break; }
+      if (attempt >= a.max_widen) break;
+      // widen once on the side that missed; the other edge moves to the old
+      // edge, which is now known to lie on the correct side of b
+      status |= ROW_WIDENED;
+      if (s_out.status & ROW_MISS_LEFT) {
+        rhi = rlo; vhi = true; aR = aL;
+        rlo -= a.widen_delta;
+        vlo = rlo >= 0;
+        if (!vlo) rlo = 0;
+        aL = vlo ? key2f(ss[rlo]) : -CUDART_INF_F;
+      } else {
+        rlo = rhi; vlo = true; aL = aR;
+        rhi += a.widen_delta;
+        vhi = rhi <= m - 1;
+        if (!vhi) rhi = m - 1;
+        aR = vhi ? key2f(ss[rhi]) : CUDART_INF_F;
+      }
+    }
+  }
+
+  if (solved) {
+    finish_row(a, r, row, s_out.b, status | ROW_CERTIFIED, aL, aR, f.nL, f.nR, f.M, f.SL, f.SR, 1, red);
+  } else if (status & ROW_NONFINITE) {
+    finish_row(a, r, row, CUDART_NAN, status, aL, aR, f.nL, f.nR, f.M, f.SL, f.SR, 1, red);
+  } else if (threadIdx.x == 0) {
+    const uint32_t idx = atomicAdd(a.fb_count, 1u);
+    a.fb_list[idx] = (int32_t)r;
+    a.ws_status[r] = status;
+  }
+}
+
+struct FbLayout {
+  size_t keys, tmp, hist, dscr, aggs, red, total;
+};
+__host__ __device__ inline FbLayout fb_layout(int64_t n) {
+  FbLayout L;
+  size_t o = 0;
+  const size_t groups = (size_t)((n + kFbGroup - 1) / kFbGroup);
+  L.keys = o; o = (o + 4 * (size_t)n + 15) & ~size_t(15);
+  L.tmp = o;  o = (o + 4 * (size_t)n + 15) & ~size_t(15);
+  L.hist = o; o = (o + 4 * (size_t)SortScratch<NT>::kWords + 15) & ~size_t(15);
+  L.dscr = o; o = (o + 8 * (size_t)kFbGroup + 15) & ~size_t(15);
+  L.aggs = o; o = (o + sizeof(GroupAgg) * groups + 15) & ~size_t(15);
+  L.red = o;  o = o + 8 * 64;
+  L.total = o;
+  return L;
+}
+
+// Full-sort fallback (arXiv abstract: covers the worst case; section 2.2:
+// the full-sort solver).  Rows queued by k_row_fwd are sorted whole in shared
+// memory and solved with no bracket.
+__global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  const FbLayout L = fb_layout(a.n);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem + L.keys);
+  uint32_t* tmp = reinterpret_cast<uint32_t*>(smem + L.tmp);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);
+  double* dscr = reinterpret_cast<double*>(smem + L.dscr);
+  GroupAgg* aggs = reinterpret_cast<GroupAgg*>(smem + L.aggs);
+  double* red = reinterpret_cast<double*>(smem + L.red);
+  __shared__ SolveOut s_out;
+  const int n = (int)a.n;
+  const double inva = 1.0 / a.alpha;
+  const uint32_t cnt = *reinterpret_cast<volatile uint32_t*>(a.fb_count);
+  for (uint32_t idx = blockIdx.x; idx < cnt; idx += gridDim.x) {
+    const int64_t r = a.fb_list[idx];
+    const float* src = a.scores + r * a.stride;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += NT) keys[i] = f2key(src[i]);
+    __syncthreads();
+    const uint32_t* sorted = block_radix_sort<NT>(keys, tmp, n, hist);
+    __syncthreads();
+    const int T = (n + kFbGroup - 1) / kFbGroup;
+    for (int g = 0; g < T; ++g)
+      aggregate_sorted_keys<NT, false>(sorted + g * kFbGroup, min(kFbGroup, n - g * kFbGroup), red, &aggs[g], inva);
+    SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, a.k, a.alpha, inva};
+    solve_band<NT, false>(in, aggs, T, KeyGroups{sorted, kFbGroup}, dscr, red, &s_out);
+    const uint32_t status = a.ws_status[r] | ROW_FALLBACK | ROW_CERTIFIED;
+    finish_row(a, r, src, s_out.b, status, -CUDART_INF_F, CUDART_INF_F, 0, 0, n, 0.0, 0.0, T, red);
+  }
+}
+
+// Backward for one row per block (section 2.1, analytic VJP):
+// lambda = sum g f / sum f, then grad = f (g - lambda).
+__device__ __forceinline__ float half_density(float x, float bh, float bl, float c2) {
+  const float d = (x - bh) - bl;
+  return 0.5f * exp2f(-fabsf(d) * c2);
+}
+
+__global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
+  __shared__ double red[64];
+  const int n = (int)a.n;
+  const double inva = 1.0 / a.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+  const float finva = (float)inva;
+  for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
+    const float* x = a.scores + r * a.stride;
+    const float* g = a.grad_p + r * a.stride;
+    float* o = a.grad + r * a.stride;
+    const double b = a.b[r];
+    const float bh = __double2float_rn(b);
+    const float bl = __double2float_rn(b - (double)bh);
+    double sh = 0.0, sgh = 0.0;
+    const int n4 = a.vec ? (n >> 2) : 0;
+    for (int v = threadIdx.x; v < n4; v += NT) {
+      const float4 xv = __ldg(reinterpret_cast<const float4*>(x) + v);
+      const float4 gv = __ldg(reinterpret_cast<const float4*>(g) + v);
+      const float h0 = half_density(xv.x, bh, bl, c2), h1 = half_density(xv.y, bh, bl, c2);
+      const float h2 = half_density(xv.z, bh, bl, c2), h3 = half_density(xv.w, bh, bl, c2);
+      sh += (double)((h0 + h1) + (h2 + h3));
+      sgh += (double)((gv.x * h0 + gv.y * h1) + (gv.z * h2 + gv.w * h3));
+    }
+    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
+      const float h = half_density(x[i], bh, bl, c2);
+      sh += (double)h;
+      sgh += (double)(g[i] * h);
+    }
+    sh = block_sum<NT, double>(sh, red);
+    sgh = block_sum<NT, double>(sgh, red);
+    const double lam = a.sumf ? (sgh * inva) / a.sumf[r] : sgh / sh;
+    const float lamf = (float)lam;
+    for (int v = threadIdx.x; v < n4; v += NT) {
+      const float4 xv = __ldcs(reinterpret_cast<const float4*>(x) + v);
+      const float4 gv = __ldcs(reinterpret_cast<const float4*>(g) + v);
+      float4 ov;
+      ov.x = half_density(xv.x, bh, bl, c2) * finva * (gv.x - lamf);
+      ov.y = half_density(xv.y, bh, bl, c2) * finva * (gv.y - lamf);
+      ov.z = half_density(xv.z, bh, bl, c2) * finva * (gv.z - lamf);
+      ov.w = half_density(xv.w, bh, bl, c2) * finva * (gv.w - lamf);
+      stg_stream(reinterpret_cast<float4*>(o) + v, ov);
+    }
+    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT)
+      o[i] = half_density(x[i], bh, bl, c2) * finva * (g[i] - lamf);
+    if (threadIdx.x == 0 && a.grad_k) a.grad_k[r] = lam;
+    __syncthreads();
+  }
+}
+
+}  // namespace
+
+size_t resident_fwd_smem(const ResidentFwd& a) { return res_layout(a.n, a.m, a.bcap).total; }
+size_t resident_fallback_smem(int64_t n) { return fb_layout(n).total; }
+
+// Lets both kernels use up to the 227 KB of shared memory a block may opt in
+// to; the size each launch actually requests decides its occupancy.
+cudaError_t resident_init() {
+  cudaError_t e = cudaFuncSetAttribute(k_row_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_row_fallback, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+}
+
+cudaError_t launch_resident_fwd(const ResidentFwd& a, int sm_count, cudaStream_t st) {
+  const size_t smem = resident_fwd_smem(a);
+  const size_t fsmem = resident_fallback_smem(a.n);
+  cudaError_t e = cudaMemsetAsync(a.fb_count, 0, sizeof(uint32_t), st);
+  if (e != cudaSuccess) return e;
+  {
+    Launch l("k_row_fwd", st);
+    k_row_fwd<<<(unsigned)a.rows, NT, smem, st>>>(a);
+  }
+  const unsigned fgrid = (unsigned)std::min<int64_t>(a.rows, (int64_t)sm_count);
+  {
+    Launch l("k_row_fallback", st);
+    k_row_fallback<<<fgrid, NT, fsmem, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_resident_bwd(const RowBwd& a, int sm_count, cudaStream_t st) {
+  const unsigned grid = (unsigned)std::min<int64_t>(a.rows, (int64_t)sm_count * 4);
+  {
+    Launch l("k_row_bwd", st);
+    k_row_bwd<<<grid, NT, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lapsum

@@ -1,0 +1,1020 @@
+// stream.cu -- rows longer than one block's shared memory (n > 16384).
+//
+// The Fast LapSum pipeline (technical summary section 2.2; arXiv abstract)
+// as a short sequence of grid-wide kernels per forward pass:
+//
+//   k_sample    localization sample: m Laplace-noised scores, level-1
+//               histogram of their fp32 keys
+//   k_select2/3 radix select of the two binomial order statistics that bound
+//               the bracket [a_L, a_R); the last block plans the band buckets
+//   k_filter    the HBM-bound stream-and-filter pass: 128-bit loads, tail
+//               counts and anchored tail sums (fp32 exp, fp64 partials), and
+//               in-band values appended to value buckets
+//   k_band      each bucket radix-sorted in shared memory; the last block
+//               runs the certified exact solve (solve.cuh)
+//   k_recover   cooperative, exits at once unless a row failed certification:
+//               widens the bracket once, then falls back to a full radix sort
+//               of the row (the worst-case branch of the abstract)
+//   k_memb      memberships p (section 2.1) plus sum f and sum p
+//
+// and two for the backward pass (section 2.1, analytic VJP): a reduction for
+// lambda = sum g f / sum f, then grad = f (g - lambda).  The HBM passes run in
+// alternating directions so that the part of the row the previous pass left in
+// L2 is read first.
+#include <algorithm>
+
+#include "block_sort.cuh"
+#include "common.cuh"
+#include "launch.h"
+#include "solve.cuh"
+
+namespace lapsum {
+namespace {
+
+constexpr int NT = kStreamThreads;
+constexpr int NW = NT / 32;
+constexpr int U = 4;              // float4 loads per thread per chunk
+constexpr int CHUNK4 = NT * U;    // float4 per chunk (4096 scores)
+constexpr int kTile = 2048;       // fallback scatter tile (keys)
+
+struct FPart {
+  long long nL;
+  double SL, SR;
+  uint32_t bad, pad;
+};
+struct MPart {
+  double a, b;
+};
+
+__device__ __forceinline__ RowCtl* ctl_of(const StreamPlan& P, int64_t r) {
+  return reinterpret_cast<RowCtl*>(P.ctl) + r;
+}
+__device__ __forceinline__ FPart* fpart_of(const StreamPlan& P, int64_t r) {
+  return reinterpret_cast<FPart*>(P.fpart) + r * kMaxGridPerRow;
+}
+__device__ __forceinline__ MPart* mpart_of(const StreamPlan& P, int64_t r) {
+  return reinterpret_cast<MPart*>(P.mpart) + r * kMaxGridPerRow;
+}
+__device__ __forceinline__ GroupAgg* aggs_of(const StreamPlan& P, int64_t r) {
+  return reinterpret_cast<GroupAgg*>(P.aggs) + r * P.T_max;
+}
+__device__ __forceinline__ uint32_t* cursor_of(const StreamPlan& P, int64_t r) { return P.cursor + r * P.T_max; }
+__device__ __forceinline__ float* band_of(const StreamPlan& P, int64_t r) { return P.band + r * P.band_cap; }
+__device__ __forceinline__ uint32_t* samp_of(const StreamPlan& P, int64_t r) { return P.samp + r * (int64_t)P.m; }
+__device__ __forceinline__ uint32_t* h1_of(const StreamPlan& P, int64_t r) { return P.hist1 + r * 2048; }
+__device__ __forceinline__ uint32_t* h2_of(const StreamPlan& P, int64_t r) { return P.hist2 + r * 4096; }
+__device__ __forceinline__ uint32_t* h3_of(const StreamPlan& P, int64_t r) { return P.hist3 + r * 2048; }
+
+// control words written earlier in the same kernel are read around L1
+template <typename T>
+__device__ __forceinline__ T vld(const T* p) {
+  return *reinterpret_cast<const volatile T*>(p);
+}
+
+// ===========================================================================
+// localization: sample keys and the radix select of two order statistics
+// ===========================================================================
+
+// bin holding ascending rank `rank` in a global histogram of NB bins; every
+// thread receives (bin, rank inside the bin)
+template <int NB>
+__device__ void find_bin(const uint32_t* gh, uint32_t rank, uint32_t* scr, int* bin, uint32_t* rem) {
+  constexpr int PER = NB / NT;
+  __shared__ int s_bin;
+  __shared__ uint32_t s_rem;
+  uint32_t v[PER];
+  uint32_t loc = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    v[i] = __ldcg(gh + threadIdx.x * PER + i);
+    loc += v[i];
+  }
+  if (threadIdx.x == 0) {
+    s_bin = NB - 1;
+    s_rem = 0;
+  }
+  const uint32_t base = block_excl_prefix_u32<NT>(loc, scr, nullptr);
+  if (rank >= base && rank < base + loc) {
+    uint32_t c = base;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      if (rank < c + v[i]) {
+        s_bin = threadIdx.x * PER + i;
+        s_rem = rank - c;
+        break;
+      }
+      c += v[i];
+    }
+  }
+  __syncthreads();
+  *bin = s_bin;
+  *rem = s_rem;
+  __syncthreads();
+}
+
+// warp-aggregated shared-memory histogram increment
+__device__ __forceinline__ void hist_add(uint32_t* h, uint32_t bin, bool act) {
+  const uint32_t amask = __ballot_sync(0xffffffffu, act);
+  if (act) {
+    const uint32_t peers = __match_any_sync(amask, bin);
+    if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(h + bin, __popc(peers));
+  }
+}
+
+__device__ void flush_hist(const uint32_t* sh, uint32_t* gh, int nb) {
+  __syncthreads();
+  for (int i = threadIdx.x; i < nb; i += NT)
+    if (sh[i]) atomicAdd(gh + i, sh[i]);
+  __syncthreads();
+}
+
+// level 1 over keys already stored (recovery path)
+__device__ void sel_level1(const uint32_t* samp, int m, int cta, int ncta, uint32_t* gh1, uint32_t* sh) {
+  for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
+  __syncthreads();
+  for (int j0 = cta * NT; j0 < m; j0 += ncta * NT) {
+    const int j = j0 + threadIdx.x;
+    const bool act = j < m;
+    const uint32_t key = act ? __ldcg(samp + j) : 0u;
+    hist_add(sh, key >> 21, act);
+  }
+  flush_hist(sh, gh1, 2048);
+}
+
+__device__ void sel_level2(const uint32_t* samp, int m, int cta, int ncta, const uint32_t* gh1, uint32_t* gh2,
+                           const int rk[2], uint32_t* sh, uint32_t* scr) {
+  int b1[2];
+  uint32_t r1[2];
+  find_bin<2048>(gh1, (uint32_t)rk[0], scr, &b1[0], &r1[0]);
+  find_bin<2048>(gh1, (uint32_t)rk[1], scr, &b1[1], &r1[1]);
+  for (int i = threadIdx.x; i < 4096; i += NT) sh[i] = 0u;
+  __syncthreads();
+  for (int j0 = cta * NT; j0 < m; j0 += ncta * NT) {
+    const int j = j0 + threadIdx.x;
+    const bool act = j < m;
+    const uint32_t key = act ? __ldcg(samp + j) : 0u;
+    const uint32_t top = key >> 21, d = (key >> 10) & 2047u;
+    hist_add(sh, d, act && top == (uint32_t)b1[0]);
+    hist_add(sh + 2048, d, act && top == (uint32_t)b1[1]);
+  }
+  flush_hist(sh, gh2, 4096);
+}
+
+__device__ void sel_level3(const uint32_t* samp, int m, int cta, int ncta, const uint32_t* gh1,
+                           const uint32_t* gh2, uint32_t* gh3, const int rk[2], uint32_t* sh, uint32_t* scr) {
+  uint32_t pre[2];
+  for (int t = 0; t < 2; ++t) {
+    int b1, b2;
+    uint32_t r1, r2;
+    find_bin<2048>(gh1, (uint32_t)rk[t], scr, &b1, &r1);
+    find_bin<2048>(gh2 + t * 2048, r1, scr, &b2, &r2);
+    pre[t] = ((uint32_t)b1 << 11) | (uint32_t)b2;
+  }
+  for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
+  __syncthreads();
+  for (int j0 = cta * NT; j0 < m; j0 += ncta * NT) {
+    const int j = j0 + threadIdx.x;
+    const bool act = j < m;
+    const uint32_t key = act ? __ldcg(samp + j) : 0u;
+    const uint32_t p = key >> 10, d = key & 1023u;
+    hist_add(sh, d, act && p == pre[0]);
+    hist_add(sh + 1024, d, act && p == pre[1]);
+  }
+  flush_hist(sh, gh3, 2048);
+}
+
+// exact keys of the two order statistics
+__device__ void sel_final(const uint32_t* gh1, const uint32_t* gh2, const uint32_t* gh3, const int rk[2],
+                          uint32_t* scr, uint32_t keys[2]) {
+  for (int t = 0; t < 2; ++t) {
+    int b1, b2, b3;
+    uint32_t r1, r2, r3;
+    find_bin<2048>(gh1, (uint32_t)rk[t], scr, &b1, &r1);
+    find_bin<2048>(gh2 + t * 2048, r1, scr, &b2, &r2);
+    find_bin<1024>(gh3 + t * 1024, r2, scr, &b3, &r3);
+    keys[t] = ((uint32_t)b1 << 21) | ((uint32_t)b2 << 10) | (uint32_t)b3;
+  }
+}
+
+// bracket and bucket plan for a row (one thread)
+__device__ void write_plan(RowCtl* c, int m, const uint32_t keys[2], int rlo, int rhi, bool vlo, bool vhi,
+                           int T, int C) {
+  const float vl = key2f(keys[0]), vh = key2f(keys[1]);
+  c->aL = vlo ? vl : -CUDART_INF_F;
+  c->aR = vhi ? vh : CUDART_INF_F;
+  c->lo = vl;
+  const double w = (double)vh - (double)vl;
+  double iw = (w > 0.0) ? (double)T / w : 0.0;
+  if (iw > 1e30) iw = 1e30;
+  c->inv_w = (float)iw;
+  c->T = T;
+  c->C = C;
+  c->rank_lo = rlo;
+  c->rank_hi = rhi;
+  c->valid_lo = vlo ? 1u : 0u;
+  c->valid_hi = vhi ? 1u : 0u;
+  c->m = m;
+  c->sel_key[0] = keys[0];
+  c->sel_key[1] = keys[1];
+}
+
+__global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* __restrict__ scores) {
+  __shared__ uint32_t sh[2048];
+  const int64_t r = blockIdx.y;
+  for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
+  __syncthreads();
+  const float* row = scores + r * P.stride;
+  const uint64_t s = row_stream(P.seed, (uint64_t)r);
+  uint32_t* samp = samp_of(P, r);
+  const int stride = gridDim.x * NT;
+  for (int j0 = blockIdx.x * NT; j0 < P.m; j0 += 4 * stride) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * stride + threadIdx.x;
+      v[u] = (j < P.m) ? __ldg(row + sample_index(s, (uint64_t)j, (uint64_t)P.n)) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * stride + threadIdx.x;
+      const bool act = j < P.m;
+      uint32_t key = 0u;
+      if (act) {
+        const double Y = (double)v[u] + laplace_noise(s, (uint64_t)j, P.alpha);
+        key = f2key(__double2float_rn(Y));
+        samp[j] = key;
+      }
+      hist_add(sh, key >> 21, act);
+    }
+  }
+  flush_hist(sh, h1_of(P, r), 2048);
+}
+
+__global__ void __launch_bounds__(NT) k_select2(const StreamPlan P) {
+  __shared__ uint32_t sh[4096];
+  __shared__ uint32_t scr[64];
+  const int64_t r = blockIdx.y;
+  const int rk[2] = {P.rank_lo, P.rank_hi};
+  sel_level2(samp_of(P, r), P.m, blockIdx.x, gridDim.x, h1_of(P, r), h2_of(P, r), rk, sh, scr);
+}
+
+__global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
+  __shared__ uint32_t sh[2048];
+  __shared__ uint32_t scr[64];
+  const int64_t r = blockIdx.y;
+  const int rk[2] = {P.rank_lo, P.rank_hi};
+  sel_level3(samp_of(P, r), P.m, blockIdx.x, gridDim.x, h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, sh, scr);
+  RowCtl* c = ctl_of(P, r);
+  if (last_block_done(&c->done_sel, gridDim.x)) {
+    uint32_t keys[2];
+    sel_final(h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, scr, keys);
+    if (threadIdx.x == 0) write_plan(c, P.m, keys, P.rank_lo, P.rank_hi, P.valid_lo, P.valid_hi, P.T, P.C);
+  }
+}
+
+// ===========================================================================
+// stream and filter (section 2.2, step 2)
+// ===========================================================================
+
+__device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
+                             int ncta, double* red) {
+  const float aL = vld(&c->aL), aR = vld(&c->aR), lo = vld(&c->lo), inv_w = vld(&c->inv_w);
+  const int T = vld(&c->T), C = vld(&c->C);
+  const float c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
+  uint32_t* cur = cursor_of(P, r);
+  float* band = band_of(P, r);
+  long long nl = 0;
+  double sl = 0.0, sr = 0.0;
+  uint32_t bad = 0u, ovf = 0u;
+
+  // an in-band value: append it to its value bucket (rare)
+  auto append = [&](float x) {
+    if (!(fabsf(x) < CUDART_INF_F)) {
+      bad = 1u;
+      return;
+    }
+    const float tf = (x - lo) * inv_w;
+    const int t = (tf >= (float)T) ? T - 1 : (tf > 0.0f ? (int)tf : 0);
+    const uint32_t slot = atomicAdd(cur + t, 1u);
+    if (slot < (uint32_t)C) band[(int64_t)t * C + slot] = x;
+    else ovf = 1u;
+  };
+  // one value, checked path
+  auto one = [&](float x) {
+    const bool isL = x < aL, isR = x >= aR;
+    const float e = exp2f(fminf(x - aL, aR - x) * c2);
+    if (isL) { sl += (double)e; ++nl; }
+    if (isR) sr += (double)e;
+    if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;
+    if (!(isL || isR)) append(x);
+  };
+
+  const int64_t n = P.n;
+  if (P.vec) {
+    const float4* x4 = reinterpret_cast<const float4*>(row);
+    const int64_t n4 = n >> 2;
+    const int64_t nchunks = n4 / CHUNK4;
+    for (int64_t q = cta; q < nchunks; q += ncta) {
+      const float4* base = x4 + q * CHUNK4 + threadIdx.x;
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = __ldg(base + u * NT);
+      float pl = 0.0f, pr = 0.0f;
+      int cl = 0;
+      uint32_t anyin = 0u, bd = 0u;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float x = xs[w];
+          const bool isL = x < aL, isR = x >= aR;
+          const float e = exp2f(fminf(x - aL, aR - x) * c2);
+          if (isL) { pl += e; ++cl; }
+          if (isR) pr += e;
+          bd |= (fabsf(x) < CUDART_INF_F) ? 0u : 1u;
+          anyin |= (isL || isR) ? 0u : 1u;
+        }
+      }
+      sl += (double)pl;
+      sr += (double)pr;
+      nl += cl;
+      bad |= bd;
+      if (__any_sync(0xffffffffu, anyin)) {
+        if (anyin) {
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+              if (!(xs[w] < aL) && !(xs[w] >= aR)) append(xs[w]);
+          }
+        }
+      }
+    }
+    for (int64_t i = nchunks * CHUNK4 + (int64_t)cta * NT + threadIdx.x; i < n4; i += (int64_t)ncta * NT) {
+      const float4 v = __ldg(x4 + i);
+      one(v.x);
+      one(v.y);
+      one(v.z);
+      one(v.w);
+    }
+    for (int64_t i = 4 * n4 + (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) one(row[i]);
+  } else {
+    for (int64_t i = (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) one(row[i]);
+  }
+  if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
+  nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
+  sl = block_sum<NT, double>(sl, red);
+  sr = block_sum<NT, double>(sr, red);
+  bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  if (threadIdx.x == 0) {
+    FPart p;
+    p.nL = nl;
+    p.SL = sl;
+    p.SR = sr;
+    p.bad = bad;
+    p.pad = 0u;
+    fpart_of(P, r)[cta] = p;
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(NT) k_filter(const StreamPlan P, const float* __restrict__ scores) {
+  __shared__ double red[64];
+  const int64_t r = blockIdx.y;
+  filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red);
+}
+
+// ===========================================================================
+// band: bucket sorts and the certified solve (section 2.2, steps 3-4)
+// ===========================================================================
+
+struct BandGroups {  // bucket g holds its sorted values at band + g*C
+  const float* band;
+  int C;
+  __device__ float get(int g, int i) const { return __ldcg(band + (int64_t)g * C + i); }
+};
+struct KeyGroupsG {  // consecutive groups of `g` sorted keys in global memory
+  const uint32_t* k;
+  int g;
+  __device__ float get(int grp, int i) const { return key2f(__ldcg(k + (int64_t)grp * g + i)); }
+};
+
+__device__ void band_sort_phase(const StreamPlan& P, int64_t r, RowCtl* c, int cta, int ncta, uint32_t* kbuf,
+                                uint32_t* tbuf, uint32_t* hist, double* red) {
+  const int T = vld(&c->T), C = vld(&c->C);
+  const double inva = 1.0 / P.alpha;
+  const uint32_t* cur = cursor_of(P, r);
+  float* band = band_of(P, r);
+  GroupAgg* ag = aggs_of(P, r);
+  for (int t = cta; t < T; t += ncta) {
+    const int cnt = (int)min(__ldcg(cur + t), (uint32_t)C);
+    float* vals = band + (int64_t)t * C;
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += NT) kbuf[i] = f2key(__ldcg(vals + i));
+    __syncthreads();
+    const uint32_t* sorted = block_radix_sort<NT>(kbuf, tbuf, cnt, hist);
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += NT) vals[i] = key2f(sorted[i]);
+    aggregate_sorted_keys<NT, false>(sorted, cnt, red, ag + t, inva);
+  }
+}
+
+// Reduces the filter partials and solves the row (one block).
+__device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int nparts, double* dscr,
+                                double* red) {
+  __shared__ SolveOut so;
+  const int T = vld(&c->T), C = vld(&c->C);
+  const double inva = 1.0 / P.alpha;
+  const FPart* parts = fpart_of(P, r);
+  const uint32_t* cur = cursor_of(P, r);
+  long long nl = 0, mt = 0;
+  double sl = 0.0, sr = 0.0;
+  uint32_t bad = 0u;
+  for (int i = threadIdx.x; i < nparts; i += NT) {
+    nl += __ldcg(&parts[i].nL);
+    sl += __ldcg(&parts[i].SL);
+    sr += __ldcg(&parts[i].SR);
+    bad |= __ldcg(&parts[i].bad);
+  }
+  for (int t = threadIdx.x; t < T; t += NT) mt += (long long)__ldcg(cur + t);
+  nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
+  mt = block_sum<NT, long long>(mt, reinterpret_cast<long long*>(red));
+  sl = block_sum<NT, double>(sl, red);
+  sr = block_sum<NT, double>(sr, red);
+  bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  const uint32_t flags = vld(&c->flags);
+  const long long nr = P.n - nl - mt;
+  uint32_t st = vld(&c->status) & ROW_WIDENED;
+  double b = 0.0;
+  if (bad) {
+    st |= ROW_NONFINITE;
+  } else if (flags & ROW_OVERFLOW) {
+    st |= ROW_OVERFLOW;
+  } else if (P.force_fallback) {
+    st |= ROW_FORCE_FB;
+  } else {
+    const SolveIn in{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, P.k, P.alpha, inva};
+    solve_band<NT, true>(in, aggs_of(P, r), T, BandGroups{band_of(P, r), C}, dscr, red, &so);
+    st |= so.status;
+    b = so.b;
+  }
+  if (threadIdx.x == 0) {
+    c->nL = nl;
+    c->nR = nr;
+    c->M = mt;
+    c->SL = sl;
+    c->SR = sr;
+    c->b = b;
+    c->status = st;
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(NT) k_band(const StreamPlan P) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* kbuf = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* tbuf = kbuf + P.C;
+  uint32_t* hist = tbuf + P.C;
+  double* red = reinterpret_cast<double*>(hist + SortScratch<NT>::kWords);
+  double* dscr = reinterpret_cast<double*>(smem);  // C doubles over kbuf + tbuf
+  const int64_t r = blockIdx.y;
+  RowCtl* c = ctl_of(P, r);
+  band_sort_phase(P, r, c, blockIdx.x, gridDim.x, kbuf, tbuf, hist, red);
+  if (last_block_done(&c->done_solve, gridDim.x)) band_solve_last(P, r, c, P.Gf, dscr, red);
+}
+
+// ===========================================================================
+// recovery: one widening, then the full-sort fallback (cooperative launch)
+// ===========================================================================
+
+struct RecSmem {
+  static constexpr size_t kKeys = 2 * (size_t)kBucketMax * 4;  // kbuf + tbuf; also dscr / selection hists
+  static constexpr size_t kHist = (size_t)SortScratch<NT>::kWords * 4;
+  static constexpr size_t kRed = 64 * 8;
+  static constexpr size_t kTotal = kKeys + kHist + kRed;
+};
+
+// exclusive prefix over `cnt` entries of a global array, in place; returns the total
+__device__ uint32_t block_scan_global_u32(uint32_t* a, int cnt, uint32_t* scr) {
+  const int q = (cnt + NT - 1) / NT;
+  const int i0 = min(cnt, (int)threadIdx.x * q), i1 = min(cnt, i0 + q);
+  uint32_t loc = 0;
+  for (int i = i0; i < i1; ++i) loc += __ldcg(a + i);
+  uint32_t tot;
+  uint32_t run = block_excl_prefix_u32<NT>(loc, scr, &tot);
+  for (int i = i0; i < i1; ++i) {
+    const uint32_t v = __ldcg(a + i);
+    a[i] = run;
+    run += v;
+  }
+  __syncthreads();
+  return tot;
+}
+
+__global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float* __restrict__ scores,
+                                                 float* __restrict__ p_out) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* kbuf = reinterpret_cast<uint32_t*>(smem);
+  uint32_t* tbuf = kbuf + kBucketMax;
+  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + RecSmem::kKeys);
+  double* red = reinterpret_cast<double*>(smem + RecSmem::kKeys + RecSmem::kHist);
+  double* dscr = reinterpret_cast<double*>(smem);
+  uint32_t* sh = kbuf;  // selection histograms (4096 words)
+  uint32_t* scr = reinterpret_cast<uint32_t*>(red);
+  __shared__ SolveOut so;
+  __shared__ int s_skip;
+
+  const int cta = blockIdx.x, ncta = gridDim.x;
+  RowCtl* c0 = ctl_of(P, 0);
+  const double inva = 1.0 / P.alpha;
+#define REC_BARRIER()                                                          \
+  do {                                                                         \
+    if (!grid_barrier(&c0->bar_count, &c0->bar_gen, (uint32_t)ncta, &c0->timeout)) { \
+      if (threadIdx.x == 0) atomicOr(&c->status, ROW_TIMEOUT);                 \
+      return;                                                                  \
+    }                                                                          \
+  } while (0)
+
+  for (int64_t r = 0; r < P.rows; ++r) {
+    RowCtl* c = ctl_of(P, r);
+    const uint32_t st0 = vld(&c->status);
+    if (!(st0 & ROW_NEEDS_RECOVERY) || (st0 & ROW_NONFINITE)) continue;
+    bool fallback = (st0 & (ROW_OVERFLOW | ROW_FORCE_FB)) != 0u || P.max_widen <= 0;
+
+    if (!fallback) {
+      // ---- widen once: the missed side moves out by widen_delta sample
+      // ranks, the other edge moves to the old edge (known to lie on the
+      // correct side of b) ----
+      const bool left = (st0 & ROW_MISS_LEFT) != 0u;
+      int rlo = vld(&c->rank_lo), rhi = vld(&c->rank_hi);
+      bool vlo = vld(&c->valid_lo) != 0u, vhi = vld(&c->valid_hi) != 0u;
+      if (left) {
+        rhi = rlo; vhi = true;
+        rlo -= P.widen_delta; vlo = rlo >= 0;
+        if (!vlo) rlo = 0;
+      } else {
+        rlo = rhi; vlo = true;
+        rhi += P.widen_delta; vhi = rhi <= P.m - 1;
+        if (!vhi) rhi = P.m - 1;
+      }
+      const int rk[2] = {rlo, rhi};
+      int T, Cc;
+      plan_buckets(P.n, P.m, rlo, rhi, P.T_max, P.band_cap, &T, &Cc);
+      for (int i = cta * NT + threadIdx.x; i < 2048; i += ncta * NT) { h1_of(P, r)[i] = 0u; h3_of(P, r)[i] = 0u; }
+      for (int i = cta * NT + threadIdx.x; i < 4096; i += ncta * NT) h2_of(P, r)[i] = 0u;
+      for (int i = cta * NT + threadIdx.x; i < P.T_max; i += ncta * NT) cursor_of(P, r)[i] = 0u;
+      REC_BARRIER();
+      sel_level1(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), sh);
+      REC_BARRIER();
+      sel_level2(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), h2_of(P, r), rk, sh, scr);
+      REC_BARRIER();
+      sel_level3(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, sh, scr);
+      REC_BARRIER();
+      if (cta == 0) {
+        uint32_t keys[2];
+        sel_final(h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, scr, keys);
+        if (threadIdx.x == 0) {
+          write_plan(c, P.m, keys, rlo, rhi, vlo, vhi, T, Cc);
+          c->flags = 0u;
+          c->status = ROW_WIDENED;
+          __threadfence();
+        }
+      }
+      REC_BARRIER();
+      filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red);
+      REC_BARRIER();
+      band_sort_phase(P, r, c, cta, ncta, kbuf, tbuf, hist, red);
+      REC_BARRIER();
+      if (cta == 0) {
+        band_solve_last(P, r, c, ncta, dscr, red);
+        if (threadIdx.x == 0) {
+          c->status |= ROW_WIDENED;
+          __threadfence();
+        }
+      }
+      REC_BARRIER();
+      const uint32_t st1 = vld(&c->status);
+      if (st1 & (ROW_CERTIFIED | ROW_NONFINITE)) continue;
+    }
+
+    // ---- full-sort fallback: LSD radix sort of the whole row, then the
+    // solver of section 2.2 with no bracket ----
+    {
+      const int64_t n = P.n;
+      const float* src = scores + r * P.stride;
+      uint32_t* A = P.fb_keys;
+      uint32_t* B = reinterpret_cast<uint32_t*>(p_out + r * P.stride);
+      uint32_t* cnts = P.rcount;                          // [256][ncta]
+      uint32_t* tots = P.rcount + 256 * (size_t)ncta;     // [256]
+      const int64_t L = (n + ncta - 1) / ncta;
+      const int64_t lo_i = min(n, (int64_t)cta * L), hi_i = min(n, lo_i + L);
+      uint32_t* cur = nullptr;  // pass 0 reads the scores themselves
+      uint32_t* sbuf = kbuf;
+      uint32_t* stmp = kbuf + kTile;
+      uint32_t* off = tbuf;
+      uint32_t* dig = tbuf + 256;
+      uint32_t* hh = tbuf + 512;
+      const uint32_t* dcount = hist + NW * 256 + 64;
+      const uint32_t* dstart = dcount + 256;
+      for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 8 * pass;
+        for (int i = threadIdx.x; i < 256; i += NT) hh[i] = 0u;
+        __syncthreads();
+        for (int64_t i0 = lo_i; i0 < hi_i; i0 += NT) {
+          const int64_t i = i0 + threadIdx.x;
+          const bool act = i < hi_i;
+          const uint32_t k = act ? (cur ? __ldcg(cur + i) : f2key(__ldg(src + i))) : 0u;
+          hist_add(hh, (k >> shift) & 255u, act);
+        }
+        __syncthreads();
+        for (int d = threadIdx.x; d < 256; d += NT) cnts[(size_t)d * ncta + cta] = hh[d];
+        REC_BARRIER();
+        for (int d = cta; d < 256; d += ncta) {
+          const uint32_t tot = block_scan_global_u32(cnts + (size_t)d * ncta, ncta, scr);
+          if (threadIdx.x == 0) tots[d] = tot;
+        }
+        REC_BARRIER();
+        if (threadIdx.x == 0) s_skip = 0;
+        __syncthreads();
+        uint32_t tv = 0u;
+        if (threadIdx.x < 256) {
+          tv = __ldcg(tots + threadIdx.x);
+          if ((int64_t)tv == n) s_skip = 1;
+        }
+        const uint32_t base_d = block_excl_prefix_u32<NT>(tv, scr, nullptr);
+        if (pass > 0 && s_skip) continue;  // every key shares this digit
+        uint32_t* dst = (cur == A) ? B : A;
+        if (threadIdx.x < 256) {
+          dig[threadIdx.x] = base_d;
+          off[threadIdx.x] = base_d + __ldcg(cnts + (size_t)threadIdx.x * ncta + cta);
+        }
+        __syncthreads();
+        for (int64_t t0 = lo_i; t0 < hi_i; t0 += kTile) {
+          const int tn = (int)min((int64_t)kTile, hi_i - t0);
+          for (int i = threadIdx.x; i < tn; i += NT)
+            sbuf[i] = cur ? __ldcg(cur + t0 + i) : f2key(__ldg(src + t0 + i));
+          __syncthreads();
+          radix_pass<NT>(sbuf, stmp, tn, hist, shift, false);
+          for (int q = threadIdx.x; q < tn; q += NT) {
+            const uint32_t k = stmp[q];
+            const uint32_t d = (k >> shift) & 255u;
+            dst[off[d] + (q - dstart[d])] = k;
+          }
+          __syncthreads();
+          if (threadIdx.x < 256) off[threadIdx.x] += dcount[threadIdx.x];
+          __syncthreads();
+        }
+        cur = dst;
+        REC_BARRIER();
+      }
+      const int ng = (int)((n + kFallbackGroup - 1) / kFallbackGroup);
+      GroupAgg* fa = reinterpret_cast<GroupAgg*>(P.fb_aggs);
+      for (int g = cta; g < ng; g += ncta)
+        aggregate_sorted_keys<NT, true>(cur + (int64_t)g * kFallbackGroup,
+                                        (int)min((int64_t)kFallbackGroup, n - (int64_t)g * kFallbackGroup), red,
+                                        fa + g, inva);
+      REC_BARRIER();
+      if (cta == 0) {
+        const SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, P.k, P.alpha, inva};
+        solve_band<NT, true>(in, fa, ng, KeyGroupsG{cur, kFallbackGroup}, dscr, red, &so);
+        if (threadIdx.x == 0) {
+          const uint32_t keep = (vld(&c->status) | st0) & (ROW_WIDENED | ROW_OVERFLOW);
+          c->b = so.b;
+          c->status = keep | ROW_FALLBACK | ROW_CERTIFIED;
+          c->aL = -CUDART_INF_F;
+          c->aR = CUDART_INF_F;
+          c->nL = 0;
+          c->nR = 0;
+          c->M = n;
+          c->SL = 0.0;
+          c->SR = 0.0;
+          c->T = ng;
+          __threadfence();
+        }
+      }
+      REC_BARRIER();
+    }
+  }
+#undef REC_BARRIER
+}
+
+// ===========================================================================
+// memberships (section 2.1) and the backward pass
+// ===========================================================================
+
+__device__ __forceinline__ float memb(float x, float bh, float bl, float c2, float& h) {
+  const float d = (x - bh) - bl;
+  h = 0.5f * exp2f(-fabsf(d) * c2);
+  return d < 0.0f ? h : 1.0f - h;
+}
+
+__global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __restrict__ scores,
+                                              float* __restrict__ p_out, double* b_out, double* sumf_out,
+                                              uint32_t* status_out, lapsum_row_stats* stats) {
+  __shared__ double red[64];
+  const int64_t r = blockIdx.y;
+  RowCtl* c = ctl_of(P, r);
+  const double b = c->b;
+  const uint32_t status = c->status;
+  const bool nonfinite = (status & ROW_NONFINITE) != 0u;
+  const double inva = 1.0 / P.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+  const float bh = __double2float_rn(b);
+  const float bl = __double2float_rn(b - (double)bh);
+  const float* row = scores + r * P.stride;
+  float* dst = p_out + r * P.stride;
+  const int64_t n = P.n;
+  double hs = 0.0, ps = 0.0;
+  auto one = [&](int64_t i) {
+    float h;
+    float p = memb(row[i], bh, bl, c2, h);
+    if (nonfinite) p = CUDART_NAN_F;
+    hs += (double)h;
+    ps += (double)p;
+    dst[i] = p;
+  };
+  if (P.vec) {
+    const float4* x4 = reinterpret_cast<const float4*>(row);
+    float4* d4 = reinterpret_cast<float4*>(dst);
+    const int64_t n4 = n >> 2;
+    const int64_t nchunks = n4 / CHUNK4;
+    for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
+      const int64_t qq = nchunks - 1 - q;  // reverse of the filter pass
+      const int64_t base = qq * CHUNK4 + threadIdx.x;
+      float4 v[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) v[u] = __ldg(x4 + base + u * NT);
+      float hl = 0.0f, pl = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float4 p;
+        float h0, h1, h2, h3;
+        p.x = memb(v[u].x, bh, bl, c2, h0);
+        p.y = memb(v[u].y, bh, bl, c2, h1);
+        p.z = memb(v[u].z, bh, bl, c2, h2);
+        p.w = memb(v[u].w, bh, bl, c2, h3);
+        if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
+        hl += (h0 + h1) + (h2 + h3);
+        pl += (p.x + p.y) + (p.z + p.w);
+        stg_stream(d4 + base + u * NT, p);
+      }
+      hs += (double)hl;
+      ps += (double)pl;
+    }
+    for (int64_t i = nchunks * CHUNK4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n4; i += (int64_t)gridDim.x * NT) {
+      one(4 * i);
+      one(4 * i + 1);
+      one(4 * i + 2);
+      one(4 * i + 3);
+    }
+    for (int64_t i = 4 * n4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) one(i);
+  } else {
+    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) one(i);
+  }
+  hs = block_sum<NT, double>(hs, red);
+  ps = block_sum<NT, double>(ps, red);
+  if (threadIdx.x == 0) mpart_of(P, r)[blockIdx.x] = MPart{hs, ps};
+  if (last_block_done(&c->done_memb, gridDim.x)) {
+    const MPart* mp = mpart_of(P, r);
+    double h = 0.0, p = 0.0;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
+      h += __ldcg(&mp[i].a);
+      p += __ldcg(&mp[i].b);
+    }
+    h = block_sum<NT, double>(h, red);
+    p = block_sum<NT, double>(p, red);
+    if (threadIdx.x == 0) {
+      const double bo = nonfinite ? CUDART_NAN : b;
+      const uint32_t pub = status & ROW_PUBLIC;
+      b_out[r] = bo;
+      if (sumf_out) sumf_out[r] = h * inva;
+      if (status_out) status_out[r] = pub;
+      c->sumf = h * inva;
+      c->sump = p;
+      if (stats) {
+        lapsum_row_stats* s = stats + r;
+        s->a_L = c->aL;
+        s->a_R = c->aR;
+        s->n_L = c->nL;
+        s->n_R = c->nR;
+        s->band = c->M;
+        s->S_L = c->SL;
+        s->S_R = c->SR;
+        s->b = bo;
+        s->sum_p = p;
+        s->sum_f = h * inva;
+        s->sample_m = P.m;
+        s->buckets = c->T;
+        s->status = pub;
+        s->reserved = 0;
+      }
+    }
+  }
+}
+
+struct BPart {
+  double sh, sgh;
+};
+
+__device__ __forceinline__ float half_dens(float x, float bh, float bl, float c2) {
+  const float d = (x - bh) - bl;
+  return 0.5f * exp2f(-fabsf(d) * c2);
+}
+
+__global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
+  __shared__ double red[64];
+  const int64_t r = blockIdx.y;
+  const double b = a.b[r];
+  const double inva = 1.0 / a.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+  const float bh = __double2float_rn(b);
+  const float bl = __double2float_rn(b - (double)bh);
+  const float* x = a.scores + r * a.stride;
+  const float* g = a.grad_p + r * a.stride;
+  const int64_t n = a.n;
+  double sh = 0.0, sgh = 0.0;
+  if (a.vec) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* g4 = reinterpret_cast<const float4*>(g);
+    const int64_t n4 = n >> 2;
+    const int64_t nchunks = n4 / CHUNK4;
+    for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
+      const int64_t base = q * CHUNK4 + threadIdx.x;
+      float4 xv[U], gv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        xv[u] = __ldg(x4 + base + u * NT);
+        gv[u] = __ldg(g4 + base + u * NT);
+      }
+      float hl = 0.0f, gl = 0.0f;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const float h0 = half_dens(xv[u].x, bh, bl, c2), h1 = half_dens(xv[u].y, bh, bl, c2);
+        const float h2 = half_dens(xv[u].z, bh, bl, c2), h3 = half_dens(xv[u].w, bh, bl, c2);
+        hl += (h0 + h1) + (h2 + h3);
+        gl += (gv[u].x * h0 + gv[u].y * h1) + (gv[u].z * h2 + gv[u].w * h3);
+      }
+      sh += (double)hl;
+      sgh += (double)gl;
+    }
+    for (int64_t i = 4 * nchunks * CHUNK4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
+      const float h = half_dens(x[i], bh, bl, c2);
+      sh += (double)h;
+      sgh += (double)(g[i] * h);
+    }
+  } else {
+    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
+      const float h = half_dens(x[i], bh, bl, c2);
+      sh += (double)h;
+      sgh += (double)(g[i] * h);
+    }
+  }
+  sh = block_sum<NT, double>(sh, red);
+  sgh = block_sum<NT, double>(sgh, red);
+  BPart* part = reinterpret_cast<BPart*>(a.part) + r * kMaxGridPerRow;
+  if (threadIdx.x == 0) part[blockIdx.x] = BPart{sh, sgh};
+  if (last_block_done(a.done + r, gridDim.x)) {
+    double h = 0.0, gh = 0.0;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
+      h += __ldcg(&part[i].sh);
+      gh += __ldcg(&part[i].sgh);
+    }
+    h = block_sum<NT, double>(h, red);
+    gh = block_sum<NT, double>(gh, red);
+    if (threadIdx.x == 0) {
+      const double lam = a.sumf ? (gh * inva) / a.sumf[r] : gh / h;
+      a.lam[r] = lam;
+      if (a.grad_k) a.grad_k[r] = lam;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
+  const int64_t r = blockIdx.y;
+  const double b = a.b[r];
+  const double inva = 1.0 / a.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+  const float finva = (float)inva;
+  const float bh = __double2float_rn(b);
+  const float bl = __double2float_rn(b - (double)bh);
+  const float lamf = (float)a.lam[r];
+  const float* x = a.scores + r * a.stride;
+  const float* g = a.grad_p + r * a.stride;
+  float* o = a.grad + r * a.stride;
+  const int64_t n = a.n;
+  if (a.vec) {
+    const float4* x4 = reinterpret_cast<const float4*>(x);
+    const float4* g4 = reinterpret_cast<const float4*>(g);
+    float4* o4 = reinterpret_cast<float4*>(o);
+    const int64_t n4 = n >> 2;
+    const int64_t nchunks = n4 / CHUNK4;
+    for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
+      const int64_t qq = nchunks - 1 - q;  // reverse of the reduction pass
+      const int64_t base = qq * CHUNK4 + threadIdx.x;
+      float4 xv[U], gv[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        xv[u] = __ldcs(x4 + base + u * NT);
+        gv[u] = __ldcs(g4 + base + u * NT);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float4 ov;
+        ov.x = half_dens(xv[u].x, bh, bl, c2) * finva * (gv[u].x - lamf);
+        ov.y = half_dens(xv[u].y, bh, bl, c2) * finva * (gv[u].y - lamf);
+        ov.z = half_dens(xv[u].z, bh, bl, c2) * finva * (gv[u].z - lamf);
+        ov.w = half_dens(xv[u].w, bh, bl, c2) * finva * (gv[u].w - lamf);
+        stg_stream(o4 + base + u * NT, ov);
+      }
+    }
+    for (int64_t i = 4 * nchunks * CHUNK4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
+      o[i] = half_dens(x[i], bh, bl, c2) * finva * (g[i] - lamf);
+  } else {
+    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
+      o[i] = half_dens(x[i], bh, bl, c2) * finva * (g[i] - lamf);
+  }
+}
+
+size_t band_smem(int C) { return (size_t)8 * C + (size_t)SortScratch<NT>::kWords * 4 + 64 * 8; }
+
+}  // namespace
+
+cudaError_t stream_occupancy(int C, StreamOcc* out) {
+  cudaError_t e = cudaFuncSetAttribute(k_band, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)band_smem(kBucketMax));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_recover, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RecSmem::kTotal);
+  if (e != cudaSuccess) return e;
+  int fb = 0, bb = 0, rb = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bb, k_band, NT, band_smem(C));
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&rb, k_recover, NT, RecSmem::kTotal);
+  if (e != cudaSuccess) return e;
+  out->filter_blocks = std::max(fb, 1);
+  out->band_blocks = std::max(bb, 1);
+  out->recover_blocks = std::max(rb, 1);
+  return cudaSuccess;
+}
+
+cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p_out, double* b_out,
+                              double* sumf_out, uint32_t* status_out, lapsum_row_stats* stats, int sm_count,
+                              cudaStream_t st) {
+  (void)sm_count;
+  cudaError_t e = cudaMemsetAsync(P.ctl, 0, P.zero_bytes, st);
+  if (e != cudaSuccess) return e;
+  const unsigned rows = (unsigned)P.rows;
+  {
+    Launch l("k_sample", st);
+    k_sample<<<dim3(P.Gs, rows), NT, 0, st>>>(P, scores);
+  }
+  {
+    Launch l("k_select2", st);
+    k_select2<<<dim3(P.Gs, rows), NT, 0, st>>>(P);
+  }
+  {
+    Launch l("k_select3", st);
+    k_select3<<<dim3(P.Gs, rows), NT, 0, st>>>(P);
+  }
+  {
+    Launch l("k_filter", st);
+    k_filter<<<dim3(P.Gf, rows), NT, 0, st>>>(P, scores);
+  }
+  {
+    Launch l("k_band", st);
+    k_band<<<dim3(P.G3, rows), NT, band_smem(P.C), st>>>(P);
+  }
+  {
+    StreamPlan Pc = P;
+    const float* sc = scores;
+    float* po = p_out;
+    void* args[] = {&Pc, &sc, &po};
+    Launch l("k_recover", st);
+    e = cudaLaunchCooperativeKernel((const void*)k_recover, dim3(P.Gr), dim3(NT), args, RecSmem::kTotal, st);
+    if (e != cudaSuccess) return e;
+  }
+  {
+    Launch l("k_memb", st);
+    k_memb<<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(a.done, 0, sizeof(uint32_t) * (size_t)a.rows, st);
+  if (e != cudaSuccess) return e;
+  {
+    Launch l("k_bwd_reduce", st);
+    k_bwd_reduce<<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+  }
+  {
+    Launch l("k_bwd_apply", st);
+    k_bwd_apply<<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lapsum

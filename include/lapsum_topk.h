@@ -1,0 +1,187 @@
+/*
+ * lapsum_topk.h -- C ABI of the B200 exact-budget LapSum soft top-k.
+ *
+ * The operator ("Fast LapSum: Exact Differentiable Top-k at Million Scale",
+ * Technical Summary section 2.1): for one row of scores r_1..r_n, a budget
+ * k (0 < k < n) and a Laplace scale alpha > 0,
+ *
+ *     p_i = F((r_i - b) / alpha),   F(z) = exp(z)/2 (z < 0), 1 - exp(-z)/2 (z >= 0),
+ *
+ * with the threshold b fixed by the exact budget  sum_i p_i = k.  The
+ * backward pass (same section: an analytic vector-Jacobian product) is
+ *
+ *     grad_j = f_j (g_j - lambda),  f_j = exp(-|r_j - b|/alpha) / (2 alpha),
+ *     lambda = sum_i g_i f_i / sum_i f_i   (which is also dL/dk).
+ *
+ * How b is found (section 2.2 of the same page, and the arXiv abstract of
+ * Fast LapSum): a sample of Laplace-noised scores and binomial order
+ * statistics give a bracket [a_L, a_R); one streaming pass keeps the scores
+ * inside it (the band) and folds the others into tail sums; the band is sorted
+ * and the budget equation is solved in closed form on it; a certification
+ * step proves b lies in the bracket, widening it once and falling back to a
+ * full sort of the row when it does not.
+ *
+ * Conventions for every entry point:
+ *   - All array pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory: scratch space is the caller's `workspace`.
+ *   - Scores are fp32, `rows` rows of `n` values, row i starting at
+ *     scores + i * row_stride (row-major when row_stride == n).  Outputs use
+ *     the same layout.  Outputs may not overlap inputs.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  All
+ *     work is enqueued on it; no entry point synchronises the host.
+ *   - Arguments are validated on the host before anything is launched; a
+ *     non-zero return code means nothing was enqueued.  Device-side outcomes
+ *     are reported per row in `row_status` (see LAPSUM_ROW_*), readable after
+ *     the stream has been synchronised.
+ *   - k and alpha are shared by all rows.  alpha must lie in [1e-30, 1e30]
+ *     (the fp32 exponent arithmetic needs 1/alpha finite).
+ *   - The first call on a device queries its properties and sets kernel
+ *     attributes; later calls on that device do not.
+ */
+#ifndef LAPSUM_TOPK_H
+#define LAPSUM_TOPK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LAPSUM_API __attribute__((visibility("default")))
+#else
+#define LAPSUM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- synchronous return codes ---------------------------------------- */
+#define LAPSUM_OK 0
+#define LAPSUM_EINVAL 1       /* null pointer, rows/n < 1, row_stride < n,
+                                 misaligned or overlapping buffers */
+#define LAPSUM_EBADK 2        /* k not finite or not in (0, n) */
+#define LAPSUM_EBADALPHA 3    /* alpha not finite or outside [1e-30, 1e30] */
+#define LAPSUM_EWORKSPACE 4   /* workspace NULL or smaller than required */
+#define LAPSUM_ECUDA 5        /* a CUDA call or launch failed */
+
+/* ---- per-row status bits (asynchronous, in row_status) ---------------- */
+#define LAPSUM_ROW_CERTIFIED 0x01u  /* b proven inside the final bracket */
+#define LAPSUM_ROW_WIDENED 0x02u    /* first bracket missed; widened once */
+#define LAPSUM_ROW_FALLBACK 0x04u   /* solved by the full-sort fallback */
+#define LAPSUM_ROW_NONFINITE 0x08u  /* NaN or +-inf in the row: outputs of
+                                       this row are unspecified */
+#define LAPSUM_ROW_TIMEOUT 0x10u    /* a bounded device wait gave up: outputs
+                                       of this row are unspecified */
+#define LAPSUM_ROW_OVERFLOW 0x20u   /* informational: a band bucket overflowed
+                                       (the row then took the fallback) */
+
+/* ---- tuning and test knobs --------------------------------------------- */
+typedef struct lapsum_params {
+    uint32_t sample_m;      /* localization sample size m; 0 = automatic */
+    uint32_t force_path;    /* 0 = normal; OR of LAPSUM_FORCE_* (tests) */
+    double z;               /* bracket half-width in binomial sigmas; 0 = 5 */
+    uint64_t seed;          /* seed of the sampling generator (splitmix64) */
+    int64_t band_capacity;  /* band slots per row; 0 = automatic */
+    int32_t max_widen;      /* widenings before the full sort: 0 or 1;
+                               negative = automatic (1) */
+    int32_t reserved;
+} lapsum_params;
+
+#define LAPSUM_FORCE_NONE 0u
+#define LAPSUM_FORCE_FALLBACK 1u   /* solve every row by the full-sort fallback */
+#define LAPSUM_FORCE_STREAMING 2u  /* use the multi-block path even for rows
+                                      that fit one block's shared memory */
+
+/* Fill *p with the defaults (all automatic, seed 0). */
+LAPSUM_API void lapsum_default_params(lapsum_params* p);
+
+/* ---- optional per-row diagnostics (device array of `rows` entries) ----- */
+typedef struct lapsum_row_stats {
+    float a_L, a_R;          /* final bracket; -inf / +inf when open */
+    int64_t n_L, n_R;        /* scores below a_L / at or above a_R */
+    int64_t band;            /* scores inside [a_L, a_R) */
+    double S_L, S_R;         /* sum exp((r - a_L)/alpha) over r < a_L and
+                                sum exp((a_R - r)/alpha) over r >= a_R */
+    double b;                /* the threshold */
+    double sum_p;            /* sum of the written p, accumulated in fp64 */
+    double sum_f;            /* sum_i f_i */
+    int32_t sample_m;        /* sample size used */
+    int32_t buckets;         /* band buckets used */
+    uint32_t status;         /* same bits as row_status */
+    int32_t reserved;
+} lapsum_row_stats;
+
+/*
+ * Bytes of workspace that lapsum_topk_fwd / lapsum_topk_bwd need for this
+ * shape and these parameters (params may be NULL for the defaults).  The
+ * value does not depend on the device.  Returns 0 for invalid shapes.
+ */
+LAPSUM_API size_t lapsum_topk_workspace_size(int64_t rows, int64_t n, const lapsum_params* params);
+
+/*
+ * Forward pass: threshold b and memberships p for every row.
+ *
+ *   scores      in   fp32 [rows, row_stride], at least 4-byte aligned
+ *   rows, n     in   rows >= 1, n >= 1, row_stride >= n (elements)
+ *   k, alpha    in   0 < k < n, alpha in [1e-30, 1e30]
+ *   p_out       out  fp32 [rows, row_stride] (only the first n of a row)
+ *   b_out       out  fp64 [rows]  threshold b of each row
+ *   sumf_out    out  fp64 [rows]  sum_i f_i of each row (may be NULL)
+ *   row_status  out  uint32 [rows] LAPSUM_ROW_* bits (may be NULL)
+ *   stats       out  lapsum_row_stats [rows] (may be NULL)
+ *   workspace   in   device scratch of workspace_bytes bytes, >= the size
+ *                    lapsum_topk_workspace_size returns; 256-byte aligned;
+ *                    contents on entry are ignored; may be reused by the next
+ *                    call on the same stream
+ *   params      in   host pointer or NULL
+ *   stream      in   cudaStream_t
+ * Returns LAPSUM_OK or an error code (nothing enqueued on error).
+ */
+LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                    double k, double alpha, float* p_out, double* b_out, double* sumf_out,
+                    uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
+                    size_t workspace_bytes, const lapsum_params* params, void* stream);
+
+/*
+ * Backward pass (vector-Jacobian product) for the b a forward pass returned.
+ *
+ *   scores      in   fp32 [rows, row_stride], the forward's input
+ *   grad_p      in   fp32 [rows, row_stride], upstream gradient dL/dp
+ *   b           in   fp64 [rows], the forward's b_out
+ *   sumf        in   fp64 [rows], the forward's sumf_out, or NULL to
+ *                    recompute sum_i f_i inside the reduction pass
+ *   alpha       in   the forward's alpha
+ *   grad_scores out  fp32 [rows, row_stride] dL/dr
+ *   grad_k      out  fp64 [rows] dL/dk = lambda (may be NULL)
+ *   workspace   in   as for the forward (the same buffer may be passed)
+ * Returns LAPSUM_OK or an error code (nothing enqueued on error).
+ */
+LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b,
+                    const double* sumf, int64_t rows, int64_t n, int64_t row_stride,
+                    double alpha, float* grad_scores, double* grad_k, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Static English text for a return code. */
+LAPSUM_API const char* lapsum_status_string(int code);
+
+/* Number of kernels this library has launched in this process (all devices,
+   all streams).  Used to count launches inside a timed region. */
+LAPSUM_API uint64_t lapsum_launch_count(void);
+
+/*
+ * Kernel timing without a profiler.  While enabled (on != 0), every kernel
+ * launch is bracketed by two CUDA events recorded on its stream; this adds two
+ * event records per launch and nothing else.  lapsum_trace_collect waits for
+ * the recorded events, writes a JSON object
+ *     {"<kernel>": [launches, total_milliseconds], ...}
+ * into buf (truncated to len-1 bytes, NUL-terminated), clears the record, and
+ * returns the number of bytes written (or the size needed when buf is NULL),
+ * or -1 if a CUDA call fails.  Both functions are thread-safe.
+ */
+LAPSUM_API void lapsum_trace_enable(int on);
+LAPSUM_API int lapsum_trace_collect(char* buf, size_t len);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAPSUM_TOPK_H */

@@ -10,8 +10,8 @@
  *   section 2.1 -- memberships p_i = F((r_i - b)/alpha), F the Laplace CDF,
  *                  with b fixed by  sum_i p_i = k;  an analytic VJP backward.
  *   section 2.2 -- full-sort solver: sort, one prefix/suffix pass over the
- *                  sorted scores ("threshold curve"), look up the interval where
- *                  the budget balances, closed-form root inside it.
+ *                  sorted scores, look up the interval where the budget
+ *                  balances, closed-form root inside it.
  *   section 2.2 -- localization: kernel-noised samples and binomial order
  *                  statistics give a bracket [a_L, a_R) around b; the stream
  *                  step aggregates the scores outside it into tail sums.

@@ -1,0 +1,154 @@
+"""CPU-only checks of the C-ABI boundary: the library builds and loads, it
+exports every entry point include/lapsum_topk.h declares, host-side argument
+validation rejects bad calls before any CUDA work, and the CUDA path shares no
+code with the oracle.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import differentiable_soft_top_b200 as lt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lapsum_topk.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"LAPSUM_API\s+[\w\s\*]+?\b(lapsum_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return lt._load()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    assert names == sorted([
+        "lapsum_default_params", "lapsum_launch_count", "lapsum_status_string",
+        "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_workspace_size",
+        "lapsum_trace_collect", "lapsum_trace_enable",
+    ])
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # nothing else leaks out of the library
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lt.library_path()], capture_output=True, text=True).stdout
+    exported = sorted(ln.split()[-1] for ln in out.splitlines() if " T " in ln)
+    assert exported == declared_functions()
+
+
+def test_params_struct_layout(lib):
+    assert ctypes.sizeof(lt._CParams) == 40
+    c = lt._CParams()
+    lib.lapsum_default_params(ctypes.byref(c))
+    assert c.z == 5.0 and c.max_widen == -1 and c.sample_m == 0 and c.seed == 0
+    assert lt.STATS_DTYPE.itemsize == 88
+
+
+def test_trace_collect_without_launches(lib):
+    lt.trace_enable(True)
+    assert lt.trace_collect() == {}
+    lt.trace_enable(False)
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert len(lt.status_string(code)) >= 2 and lt.status_string(code) != "unknown status"
+    assert lt.status_string(99) == "unknown status"
+
+
+def test_workspace_size(lib):
+    assert lt.workspace_size(0, 10) == 0
+    assert lt.workspace_size(1, 0) == 0
+    small = lt.workspace_size(1, 4096)
+    assert 0 < small < 1 << 20
+    assert lt.workspace_size(2048, 16384) >= lt.workspace_size(1024, 16384)
+    big = lt.workspace_size(1, 10**8)
+    assert 4 * 10**8 <= big < 2 * 10**9  # holds the fallback key buffer
+    forced = lt.workspace_size(1, 4096, lt.Params(force_path=lt.FORCE_STREAMING))
+    assert forced > small
+
+
+FAKE = 1 << 20  # aligned non-null placeholder; validation fails before any use
+
+
+def fwd(lib, scores=FAKE, rows=1, n=16, stride=16, k=4.0, alpha=0.5, p=FAKE * 4, b=FAKE * 8,
+        ws=FAKE * 16, wsb=1 << 30, params=None):
+    return lib.lapsum_topk_fwd(scores, rows, n, stride, k, alpha, p, b, None, None, None, ws, wsb, params, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(scores=None), lt.LAPSUM_EINVAL),
+    (dict(p=None), lt.LAPSUM_EINVAL),
+    (dict(b=None), lt.LAPSUM_EINVAL),
+    (dict(rows=0), lt.LAPSUM_EINVAL),
+    (dict(n=0), lt.LAPSUM_EINVAL),
+    (dict(stride=15), lt.LAPSUM_EINVAL),
+    (dict(scores=FAKE + 2), lt.LAPSUM_EINVAL),
+    (dict(p=FAKE + 8), lt.LAPSUM_EINVAL),  # overlaps the scores
+    (dict(k=0.0), lt.LAPSUM_EBADK),
+    (dict(k=-1.0), lt.LAPSUM_EBADK),
+    (dict(k=16.0), lt.LAPSUM_EBADK),
+    (dict(k=float("nan")), lt.LAPSUM_EBADK),
+    (dict(k=float("inf")), lt.LAPSUM_EBADK),
+    (dict(alpha=0.0), lt.LAPSUM_EBADALPHA),
+    (dict(alpha=-1.0), lt.LAPSUM_EBADALPHA),
+    (dict(alpha=1e-31), lt.LAPSUM_EBADALPHA),
+    (dict(alpha=float("nan")), lt.LAPSUM_EBADALPHA),
+    (dict(ws=None), lt.LAPSUM_EWORKSPACE),
+    (dict(wsb=8), lt.LAPSUM_EWORKSPACE),
+    (dict(ws=FAKE * 16 + 128), lt.LAPSUM_EWORKSPACE),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, code):
+    assert fwd(lib, **kw) == code
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    B = lib.lapsum_topk_bwd
+    ok = dict(s=FAKE, g=FAKE * 2, b=FAKE * 3, sf=None, rows=1, n=100000, stride=100000, a=0.5, out=FAKE * 4,
+              gk=None, ws=FAKE * 8, wsb=1 << 30)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return B(d["s"], d["g"], d["b"], d["sf"], d["rows"], d["n"], d["stride"], d["a"], d["out"], d["gk"],
+                 d["ws"], d["wsb"], None)
+
+    assert call(s=None) == lt.LAPSUM_EINVAL
+    assert call(out=None) == lt.LAPSUM_EINVAL
+    assert call(b=FAKE * 3 + 4) == lt.LAPSUM_EINVAL
+    assert call(n=0) == lt.LAPSUM_EINVAL
+    assert call(a=0.0) == lt.LAPSUM_EBADALPHA
+    assert call(out=FAKE + 64) == lt.LAPSUM_EINVAL  # overlaps the scores
+    assert call(wsb=16) == lt.LAPSUM_EWORKSPACE
+
+
+def test_binding_rejects_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    with pytest.raises(TypeError):
+        lt.forward(torch.zeros(8), 2.0, 1.0)
+
+
+def test_cuda_path_and_oracle_share_no_code():
+    """The oracle and the CUDA path neither include nor import each other; the
+    input generators (workloads.py) are the only module both sides use."""
+    csrc = os.path.join(ROOT, "differentiable_soft_top_b200", "csrc")
+    for f in os.listdir(csrc):
+        text = open(os.path.join(csrc, f)).read()
+        assert "oracle" not in text.lower(), f
+    imp = re.compile(r"^\s*(from|import)\s+(\S+)", re.M)
+    pkg = os.path.join(ROOT, "differentiable_soft_top_b200")
+    for f in os.listdir(pkg):
+        if f.endswith(".py"):
+            mods = [m[1] for m in imp.findall(open(os.path.join(pkg, f)).read())]
+            assert not any(m.startswith("oracle") for m in mods), f
+    text = open(os.path.join(ROOT, "oracle", "lapsum_oracle.c")).read()
+    assert '#include "' not in text
+    mods = [m[1] for m in imp.findall(open(os.path.join(ROOT, "oracle", "__init__.py")).read())]
+    assert not any(m.startswith("differentiable_soft_top_b200") for m in mods)

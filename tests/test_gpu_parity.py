@@ -1,0 +1,270 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (fp32 outputs):
+  max |p_gpu - p_ref|                          <= 1e-5
+  |sum p_gpu - k|                              <= 1e-3 max(1,k) sqrt(n/1e6)
+  ||grad_gpu - grad_ref||_2 / ||grad_ref||_2   <= 1e-4
+and, as a diagnostic of the threshold itself, |b_gpu - b_ref| small against
+alpha (the fp64 b must agree far below the p tolerance: dp/db <= 1/(2 alpha)).
+Every input is seeded and synthetic (differentiable_soft_top_b200.workloads).
+"""
+import math
+
+import numpy as np
+import pytest
+
+import differentiable_soft_top_b200 as lt
+from differentiable_soft_top_b200.workloads import WORKLOADS, make_grad, make_scores
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def tol_sum(k, n):
+    return 1e-3 * max(1.0, k) * math.sqrt(n / 1e6)
+
+
+def gpu_run(x_np, g_np, k, alpha, params=None, stats=False):
+    x = torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
+    g = torch.from_numpy(np.ascontiguousarray(g_np)).cuda()
+    res = lt.forward(x, k, alpha, params=params, stats=stats)
+    grad, gk = lt.backward(x, g, res.b, alpha, sumf=res.sumf)
+    torch.cuda.synchronize()
+    return dict(p=res.p.cpu().numpy(), b=res.b.cpu().numpy(), sumf=res.sumf.cpu().numpy(),
+                status=res.status.cpu().numpy().astype(np.uint32), stats=res.stats,
+                grad=grad.cpu().numpy(), gk=gk.cpu().numpy())
+
+
+def check_row(orc, r, g, p, grad, b, gk, k, alpha, label=""):
+    r = np.asarray(r, np.float32).reshape(-1)
+    n = r.size
+    p_ref, b_ref, _ = orc.forward(r, k, alpha)
+    grad_ref, lam, _ = orc.backward(r, np.asarray(g, np.float32).reshape(-1), b_ref, alpha)
+    p = np.asarray(p, np.float64).reshape(-1)
+    grad = np.asarray(grad, np.float64).reshape(-1)
+    dp = float(np.max(np.abs(p - p_ref)))
+    assert dp <= 1e-5, f"{label} max|dp|={dp:.3e} b_gpu={b!r} b_ref={b_ref!r}"
+    sp = math.fsum(p.tolist())
+    assert abs(sp - k) <= tol_sum(k, n), f"{label} sum p={sp} k={k}"
+    nref = float(np.linalg.norm(grad_ref))
+    if nref > 0:
+        rel = float(np.linalg.norm(grad - grad_ref)) / nref
+        assert rel <= 1e-4, f"{label} grad rel err {rel:.3e}"
+    assert abs(b - b_ref) <= 2e-6 * alpha + 1e-12 * abs(b_ref), f"{label} b {b!r} vs {b_ref!r}"
+    assert gk == pytest.approx(lam, rel=1e-4, abs=1e-8 * (1 + abs(lam)))
+    return b_ref
+
+
+def case(name, n=None, rows=None):
+    w = WORKLOADS[name]
+    if n is not None or rows is not None:
+        w = w.scaled(n=n, rows=rows)
+    return w, make_scores(w), make_grad(w.rows, w.n)
+
+
+# ---------------------------------------------------------------------------
+# the five workloads
+# ---------------------------------------------------------------------------
+def test_c1_single_row_4096(orc):
+    w, x, g = case("c1")
+    out = gpu_run(x, g, w.k, w.alpha, stats=True)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], w.k, w.alpha, "c1")
+    assert out["status"][0] & lt.ROW_CERTIFIED
+
+
+def test_c5_tied_batch(orc):
+    w, x, g = case("c5")
+    out = gpu_run(x, g, w.k, w.alpha)
+    assert np.all(out["status"] & lt.ROW_CERTIFIED)
+    for i in range(w.rows):
+        check_row(orc, x[i], g[i], out["p"][i], out["grad"][i], out["b"][i], out["gk"][i], w.k, w.alpha,
+                  f"c5 row {i}")
+
+
+def test_c2_1e6(orc):
+    w, x, g = case("c2")
+    out = gpu_run(x, g, w.k, w.alpha, stats=True)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], w.k, w.alpha, "c2")
+    assert out["status"][0] == lt.ROW_CERTIFIED
+
+
+def test_c3_1e7_mixture(orc):
+    w, x, g = case("c3")
+    out = gpu_run(x, g, w.k, w.alpha, stats=True)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], w.k, w.alpha, "c3")
+    assert out["status"][0] == lt.ROW_CERTIFIED
+
+
+@pytest.mark.slow
+def test_c4_1e8_uniform(orc):
+    """Full size, same launch configuration as bench.py; every output compared."""
+    w, x, g = case("c4")
+    out = gpu_run(x, g, w.k, w.alpha, stats=True)
+    assert out["status"][0] == lt.ROW_CERTIFIED
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], w.k, w.alpha, "c4")
+
+
+# ---------------------------------------------------------------------------
+# sizes spanning several tiles with ragged tails, strides, several rows
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n", [4097, 16383, 16385, 100_003, 1_000_001])
+def test_ragged_sizes(orc, n):
+    x = make_scores("normal", 1, n, seed=n)
+    g = make_grad(1, n, seed=n + 1)
+    k, alpha = n / 37.0, 0.3
+    out = gpu_run(x, g, k, alpha)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], k, alpha, f"n={n}")
+
+
+@pytest.mark.parametrize("n,force", [(5000, lt.FORCE_NONE), (5000, lt.FORCE_STREAMING), (70001, lt.FORCE_NONE)])
+def test_strided_unaligned_rows(orc, n, force):
+    rows, stride = 3, n + 3
+    base = make_scores("mixture", rows, stride, seed=7)
+    gb = make_grad(rows, stride, seed=8)
+    xt = torch.from_numpy(base).cuda()[:, 1:n + 1]  # 4-byte aligned only, row stride n+3
+    gt = torch.from_numpy(gb).cuda()[:, 1:n + 1]
+    k, alpha = 123.5, 0.07
+    params = lt.Params(force_path=force)
+    res = lt.forward(xt, k, alpha, params=params)
+    grad, gk = lt.backward(xt, gt, res.b, alpha)
+    torch.cuda.synchronize()
+    p, b = res.p.cpu().numpy(), res.b.cpu().numpy()
+    for i in range(rows):
+        check_row(orc, base[i, 1:n + 1], gb[i, 1:n + 1], p[i], grad.cpu().numpy()[i], b[i], gk.cpu().numpy()[i],
+                  k, alpha, f"strided row {i}")
+
+
+def test_many_rows_streaming(orc):
+    rows, n = 5, 40_000
+    x = make_scores("normal", rows, n, seed=3)
+    g = make_grad(rows, n, seed=4)
+    out = gpu_run(x, g, 400.0, 0.2)
+    for i in range(rows):
+        check_row(orc, x[i], g[i], out["p"][i], out["grad"][i], out["b"][i], out["gk"][i], 400.0, 0.2, f"row {i}")
+
+
+# ---------------------------------------------------------------------------
+# edge cases and degenerate inputs
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("n,k,alpha", [
+    (1, 0.5, 1.0), (1, 1e-6, 0.01), (2, 1.0, 0.5), (3, 2.999, 0.1), (7, 1e-4, 2.0),
+    (4096, 1e-3, 0.5), (4096, 4095.9, 0.5), (4096, 2048.0, 1e-6), (4096, 64.0, 1e6),
+    (100_000, 1.5, 1e-4), (100_000, 99_990.0, 0.3), (100_000, 50_000.0, 10.0),
+])
+def test_edge_budgets_and_temperatures(orc, n, k, alpha):
+    x = make_scores("normal", 1, n, seed=n + 17)
+    g = make_grad(1, n, seed=n + 18)
+    out = gpu_run(x, g, k, alpha)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], k, alpha, f"n={n} k={k}")
+
+
+@pytest.mark.parametrize("n", [5000, 300_000])
+def test_all_equal_scores(orc, n):
+    x = np.full((1, n), 0.25, np.float32)
+    g = make_grad(1, n, seed=2)
+    out = gpu_run(x, g, n / 3.0, 0.5)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], n / 3.0, 0.5, "all-equal")
+
+
+@pytest.mark.parametrize("n", [6000, 200_000])
+def test_signed_zeros_and_large_magnitudes(orc, n):
+    x = make_scores("normal", 1, n, seed=5)
+    x[0, ::7] = 0.0
+    x[0, 3::7] = -0.0
+    x[0, 5::97] = 3e30
+    x[0, 6::97] = -3e30
+    g = make_grad(1, n, seed=6)
+    k = n / 10.0
+    out = gpu_run(x, g, k, 0.05)
+    check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], k, 0.05, "zeros/large")
+
+
+@pytest.mark.parametrize("n", [3000, 50_000])
+def test_nonfinite_rows_flagged(orc, n):
+    x = make_scores("normal", 3, n, seed=9)
+    g = make_grad(3, n, seed=10)
+    x[1, n // 2] = np.nan
+    x[2, 7] = np.inf
+    out = gpu_run(x, g, 30.0, 0.5)
+    assert out["status"][1] & lt.ROW_NONFINITE
+    assert out["status"][2] & lt.ROW_NONFINITE
+    assert not (out["status"][0] & lt.ROW_NONFINITE)
+    check_row(orc, x[0], g[0], out["p"][0], out["grad"][0], out["b"][0], out["gk"][0], 30.0, 0.5, "finite row")
+
+
+# ---------------------------------------------------------------------------
+# the rare branches: widening, band overflow, full-sort fallback
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,n", [("c1", None), ("c2", None), ("c5", 2048)])
+@pytest.mark.parametrize("force", [lt.FORCE_NONE, lt.FORCE_STREAMING])
+def test_forced_paths_give_the_same_threshold(orc, name, n, force):
+    w, x, g = case(name, n=n) if name != "c5" else case("c5", rows=8)
+    x, g = x[:2], g[:2]
+    base = gpu_run(x, g, w.k, w.alpha, params=lt.Params(force_path=force))
+    fb = gpu_run(x, g, w.k, w.alpha, params=lt.Params(force_path=force | lt.FORCE_FALLBACK))
+    assert np.all(fb["status"] & lt.ROW_FALLBACK)
+    # a tiny z makes the bracket miss; one widening or the fallback recovers it
+    wid = gpu_run(x, g, w.k, w.alpha, params=lt.Params(force_path=force, z=0.02, seed=11))
+    ovf = gpu_run(x, g, w.k, w.alpha, params=lt.Params(force_path=force, band_capacity=8))
+    nowid = gpu_run(x, g, w.k, w.alpha, params=lt.Params(force_path=force, z=0.02, seed=11, max_widen=0))
+    for o in (base, fb, wid, ovf, nowid):
+        assert np.all(o["status"] & lt.ROW_CERTIFIED)
+        for i in range(x.shape[0]):
+            check_row(orc, x[i], g[i], o["p"][i], o["grad"][i], o["b"][i], o["gk"][i], w.k, w.alpha, name)
+            assert abs(o["b"][i] - base["b"][i]) <= 1e-9 * max(1.0, abs(base["b"][i])) + 1e-9 * w.alpha
+    assert np.any(wid["status"] & (lt.ROW_WIDENED | lt.ROW_FALLBACK))
+    assert np.all(((nowid["status"] & lt.ROW_FALLBACK) != 0) | (nowid["status"] == lt.ROW_CERTIFIED))
+    assert np.all(ovf["status"] & lt.ROW_FALLBACK)
+
+
+def test_widened_rows_report_it(orc):
+    w, x, g = case("c2")
+    seen = 0
+    for seed in range(6):
+        o = gpu_run(x, g, w.k, w.alpha, params=lt.Params(z=0.3, seed=seed))
+        check_row(orc, x[0], g[0], o["p"], o["grad"], o["b"][0], o["gk"][0], w.k, w.alpha, f"z=0.3 seed {seed}")
+        seen |= int(o["status"][0])
+    assert seen & (lt.ROW_WIDENED | lt.ROW_FALLBACK)
+
+
+# ---------------------------------------------------------------------------
+# the localization step against the oracle's own sample (same splitmix64)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,n", [("c1", None), ("c2", None), ("c3", 2_000_000), ("c5", None)])
+def test_bracket_and_tails_match_oracle(orc, name, n):
+    w, x, g = case(name, n=n) if name != "c5" else case("c5", rows=4)
+    out = gpu_run(x, g, w.k, w.alpha, stats=True, params=lt.Params(seed=123))
+    for i in range(x.shape[0]):
+        st = out["stats"][i]
+        aL, aR, _, _ = orc.bracket(x[i], w.k, w.alpha, int(st["sample_m"]), 5.0, 123, i)
+        assert np.float32(st["a_L"]) == np.float32(aL) and np.float32(st["a_R"]) == np.float32(aR)
+        nL, SL, nR, SR, M = orc.tails(x[i], aL, aR, w.alpha)
+        assert (st["n_L"], st["n_R"], st["band"]) == (nL, nR, M)
+        assert st["S_L"] == pytest.approx(SL, rel=2e-6, abs=1e-30)
+        assert st["S_R"] == pytest.approx(SR, rel=2e-6, abs=1e-30)
+        assert st["sum_p"] == pytest.approx(w.k, abs=tol_sum(w.k, w.n))
+        assert st["sum_f"] == pytest.approx(out["sumf"][i])
+
+
+def test_deterministic():
+    w, x, g = case("c3", n=3_000_000)
+    a = gpu_run(x, g, w.k, w.alpha)
+    b = gpu_run(x, g, w.k, w.alpha)
+    assert np.array_equal(a["p"], b["p"]) and np.array_equal(a["b"], b["b"])
+    assert np.array_equal(a["grad"], b["grad"])
+
+
+def test_autograd_wrapper_and_optional_sumf(orc):
+    w, x, g = case("c1")
+    xt = torch.from_numpy(x[0]).cuda().requires_grad_(True)
+    p = lt.soft_topk(xt, w.k, w.alpha)
+    p.backward(torch.from_numpy(g[0]).cuda())
+    res = lt.forward(xt.detach(), w.k, w.alpha)
+    g1, _ = lt.backward(xt.detach(), torch.from_numpy(g[0]).cuda(), res.b, w.alpha, sumf=res.sumf)
+    g2, _ = lt.backward(xt.detach(), torch.from_numpy(g[0]).cuda(), res.b, w.alpha)
+    assert torch.allclose(xt.grad, g1, rtol=0, atol=0)
+    assert float((g1 - g2).norm() / g1.norm()) < 1e-6
+    assert lt.launch_count() > 0
