@@ -151,6 +151,24 @@ def ncu_traffic(kernel: str, n_scores: int):
     return float(e["dram_bytes"]) * n_scores / float(e["scores"])
 
 
+def shard_rows(rows: int, world: int, rank: int) -> tuple[int, int]:
+    """Contiguous block of rows owned by `rank` when a batch is split across
+    `world` GPUs (rows are independent, so no collective is needed)."""
+    base, extra = divmod(rows, world)
+    lo = rank * base + min(rank, extra)
+    return lo, lo + base + (1 if rank < extra else 0)
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """The slowest rank's time: every rank takes the same collective step."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def cpu_baseline(x_row, g_row, w, budget_s: float = 20.0):
     """The fp64 oracle, as it stands, on a bounded prefix of the same row."""
     from oracle import oracle
@@ -251,7 +269,7 @@ def main():
 
     def step():
         lt.forward_into(x, w.k, w.alpha, p, b, sumf, status, ws)
-        lt.backward_into(x, g, b, w.alpha, grad, ws, sumf=sumf, grad_k=gk)
+        lt.backward_into(x, g, b, w.alpha, grad, ws, grad_k=gk)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -283,11 +301,7 @@ def main():
     lt.trace_enable(False)
     if dist is not None:
         dist.barrier()
-    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dist, dev)
     ms_per_step = total_ms / args.steps
     scores_per_step = rows * n
     value = world * scores_per_step / (ms_per_step * 1e-3)
@@ -319,11 +333,7 @@ def main():
             grad_h.copy_(grad, non_blocking=True)
             evs[i][1].record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = sum(s.elapsed_time(e) for s, e in evs[1:]) / n_e2e
-        if dist is not None:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in evs[1:]) / n_e2e, dist, dev)
         e2e = {"value": world * scores_per_step / (e2e_ms * 1e-3), "unit": "scores/s",
                "h2d_bytes_per_step": 8 * scores_per_step, "d2h_bytes_per_step": 8 * scores_per_step,
                "ms_per_step": e2e_ms, "note": "pinned host r,g -> device, fwd+bwd via the C ABI, p,grad -> host"}

@@ -43,7 +43,10 @@ FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
 
 class LapsumError(RuntimeError):
     def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {status_string(code)} (code {code})")
+        msg = f"{where}: {status_string(code)} (code {code})"
+        if code == LAPSUM_ECUDA:
+            msg += f": {_load().lapsum_last_cuda_error().decode()}"
+        super().__init__(msg)
         self.code = code
 
 
@@ -112,10 +115,12 @@ def _load():
             lib.lapsum_topk_workspace_size.restype = sz
             lib.lapsum_topk_fwd.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, sz, P, P]
             lib.lapsum_topk_fwd.restype = ctypes.c_int
-            lib.lapsum_topk_bwd.argtypes = [P, P, P, P, i64, i64, i64, dbl, P, P, P, sz, P]
+            lib.lapsum_topk_bwd.argtypes = [P, P, P, i64, i64, i64, dbl, P, P, P, sz, P]
             lib.lapsum_topk_bwd.restype = ctypes.c_int
             lib.lapsum_status_string.argtypes = [ctypes.c_int]
             lib.lapsum_status_string.restype = ctypes.c_char_p
+            lib.lapsum_last_cuda_error.argtypes = []
+            lib.lapsum_last_cuda_error.restype = ctypes.c_char_p
             lib.lapsum_launch_count.argtypes = []
             lib.lapsum_launch_count.restype = ctypes.c_uint64
             lib.lapsum_trace_enable.argtypes = [ctypes.c_int]
@@ -203,6 +208,14 @@ def _as_rows(t, name):
     return t2
 
 
+def _like_rows(x):
+    """An uninitialised [rows, n] tensor with the row stride of x (the C ABI
+    uses one row stride for inputs and outputs)."""
+    torch = _torch()
+    rows, n = x.shape
+    return torch.empty_strided((rows, n), (x.stride(0), 1), dtype=x.dtype, device=x.device)
+
+
 @dataclass
 class ForwardResult:
     p: object          # torch.Tensor, same shape as scores
@@ -220,7 +233,9 @@ def forward(scores, k: float, alpha: float, *, params: Params | None = None, wor
     x = _as_rows(scores, "scores")
     rows, n = x.shape
     dev = x.device
-    p = torch.empty_like(x) if p_out is None else _as_rows(p_out, "p_out")
+    p = _like_rows(x) if p_out is None else _as_rows(p_out, "p_out")
+    if p.stride(0) != x.stride(0):
+        raise ValueError("p_out must have the row stride of scores")
     b = torch.empty(rows, dtype=torch.float64, device=dev)
     sumf = torch.empty(rows, dtype=torch.float64, device=dev)
     status = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -236,31 +251,32 @@ def forward(scores, k: float, alpha: float, *, params: Params | None = None, wor
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_fwd")
     stats_np = st.cpu().numpy().view(STATS_DTYPE) if st is not None else None
-    return ForwardResult(p.view(scores.shape) if p_out is None else p_out, b, sumf, status, stats_np)
+    return ForwardResult(p.view(scores.shape) if p_out is None and scores.dim() == 1 else (p if p_out is None else p_out),
+                         b, sumf, status, stats_np)
 
 
-def backward(scores, grad_p, b, alpha: float, *, sumf=None, workspace=None, grad_out=None):
+def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None):
     """dL/dscores and dL/dk for upstream gradient `grad_p` at thresholds `b`."""
     torch = _torch()
     lib = _load()
     x = _as_rows(scores, "scores")
     g = _as_rows(grad_p, "grad_p")
     rows, n = x.shape
-    if g.shape != x.shape or g.stride(0) != x.stride(0):
-        g = g.reshape(rows, n).contiguous()
-        if x.stride(0) != n:
-            x = x.contiguous()
+    if g.shape != x.shape:
+        raise ValueError("grad_p must have the shape of scores")
+    if g.stride(0) != x.stride(0):  # the C ABI takes one row stride for all arrays
+        x, g = x.contiguous(), g.contiguous()
     dev = x.device
-    out = torch.empty_like(x) if grad_out is None else _as_rows(grad_out, "grad_out")
+    out = _like_rows(x) if grad_out is None else _as_rows(grad_out, "grad_out")
+    if out.stride(0) != x.stride(0):
+        raise ValueError("grad_out must have the row stride of scores")
     gk = torch.empty(rows, dtype=torch.float64, device=dev)
     bb = b.to(device=dev, dtype=torch.float64).contiguous()
-    sf = sumf.to(device=dev, dtype=torch.float64).contiguous() if sumf is not None else None
     need = int(lib.lapsum_topk_workspace_size(rows, n, None))
     ws = workspace if workspace is not None else _workspace(dev, need)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    rc = lib.lapsum_topk_bwd(x.data_ptr(), g.data_ptr(), bb.data_ptr(), sf.data_ptr() if sf is not None else None,
-                             rows, n, x.stride(0), float(alpha), out.data_ptr(), gk.data_ptr(), ws.data_ptr(),
-                             ws.numel(), stream)
+    rc = lib.lapsum_topk_bwd(x.data_ptr(), g.data_ptr(), bb.data_ptr(), rows, n, x.stride(0), float(alpha),
+                             out.data_ptr(), gk.data_ptr(), ws.data_ptr(), ws.numel(), stream)
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_bwd")
     return (out.view(scores.shape) if grad_out is None else grad_out), gk
@@ -283,14 +299,13 @@ def forward_into(scores, k: float, alpha: float, p, b, sumf, status, workspace, 
         raise LapsumError(rc, "lapsum_topk_fwd")
 
 
-def backward_into(scores, grad_p, b, alpha: float, grad, workspace, sumf=None, grad_k=None) -> None:
+def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None) -> None:
     """backward() with every output preallocated (no allocation in the call)."""
     torch = _torch()
     lib = _load()
     rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
     stride = scores.stride(0) if scores.dim() == 2 else n
-    rc = lib.lapsum_topk_bwd(scores.data_ptr(), grad_p.data_ptr(), b.data_ptr(),
-                             sumf.data_ptr() if sumf is not None else None, rows, n, stride, float(alpha),
+    rc = lib.lapsum_topk_bwd(scores.data_ptr(), grad_p.data_ptr(), b.data_ptr(), rows, n, stride, float(alpha),
                              grad.data_ptr(), grad_k.data_ptr() if grad_k is not None else None,
                              workspace.data_ptr(), workspace.numel(),
                              torch.cuda.current_stream(scores.device).cuda_stream)
@@ -312,15 +327,16 @@ class SoftTopK:
                 @staticmethod
                 def forward(ctx, scores, k, alpha, params):
                     res = forward(scores, k, alpha, params=params)
-                    ctx.save_for_backward(scores, res.b, res.sumf)
+                    ctx.save_for_backward(scores, res.b)
                     ctx.alpha = alpha
-                    return res.p
+                    return res.p.view(scores.shape)
 
                 @staticmethod
                 def backward(ctx, gp):
-                    scores, b, sumf = ctx.saved_tensors
-                    gs, gk = backward(scores, gp.contiguous(), b, ctx.alpha, sumf=sumf)
-                    return gs, None, None, None
+                    scores, b = ctx.saved_tensors
+                    sc = scores.contiguous()
+                    gs, gk = backward(sc, gp.contiguous().view(sc.shape), b, ctx.alpha)
+                    return gs.view(scores.shape), None, None, None
 
             cls._fn = _F
         return cls._fn

@@ -14,7 +14,7 @@
 
 namespace lapsum {
 
-cudaError_t resident_init();
+cudaError_t resident_init(int optin_bytes);
 
 namespace {
 
@@ -22,7 +22,8 @@ constexpr int kMaxDevices = 64;
 struct DevInfo {
   bool ready = false;
   int sm_count = 0;
-  StreamOcc occ{};  // for C = kBucketMax
+  int smem_optin = 0;  // bytes of shared memory a block may opt in to
+  StreamOcc occ{};     // for C = kBucketMax
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -38,7 +39,9 @@ cudaError_t device_info(DevInfo** out) {
     if (!d->ready) {
       e = cudaDeviceGetAttribute(&d->sm_count, cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
-      e = resident_init();
+      e = cudaDeviceGetAttribute(&d->smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+      if (e != cudaSuccess) return e;
+      e = resident_init(d->smem_optin);
       if (e != cudaSuccess) return e;
       e = stream_occupancy(kBucketMax, &d->occ);
       if (e != cudaSuccess) return e;
@@ -50,6 +53,14 @@ cudaError_t device_info(DevInfo** out) {
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// the text of the last failed CUDA call on this host thread
+thread_local const char* t_last_error = "no error";
+bool cuda_ok(cudaError_t e) {
+  if (e == cudaSuccess) return true;
+  t_last_error = cudaGetErrorString(e);
+  return false;
+}
 
 struct Resolved {
   double z;
@@ -170,7 +181,7 @@ size_t resident_ws_bytes(int64_t rows) { return align256(4 * (size_t)rows) + 256
 
 size_t bwd_ws_bytes(int64_t rows, int64_t n) {
   if (n <= kResidentMaxN) return 0;
-  return align256(16 * (size_t)kMaxGridPerRow * (size_t)rows) + align256(4 * (size_t)rows) +
+  return align256(32 * (size_t)kMaxGridPerRow * (size_t)rows) + align256(4 * (size_t)rows) +
          align256(8 * (size_t)rows);
 }
 
@@ -197,6 +208,8 @@ void lapsum_default_params(lapsum_params* p) {
   p->z = 5.0;
   p->max_widen = -1;
 }
+
+const char* lapsum_last_cuda_error(void) { return t_last_error; }
 
 const char* lapsum_status_string(int code) {
   switch (code) {
@@ -237,7 +250,7 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
   if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)) return LAPSUM_EWORKSPACE;
 
   DevInfo* dev = nullptr;
-  if (device_info(&dev) != cudaSuccess) return LAPSUM_ECUDA;
+  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -270,14 +283,14 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
     a.ws_status = reinterpret_cast<uint32_t*>(ws);
     a.fb_count = reinterpret_cast<uint32_t*>(ws + align256(4 * (size_t)rows));
     a.fb_list = reinterpret_cast<int32_t*>(ws + align256(4 * (size_t)rows) + 256);
-    if (resident_fwd_smem(a) > 227 * 1024) return LAPSUM_EINVAL;
-    return launch_resident_fwd(a, dev->sm_count, st) == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA;
+    if (resident_fwd_smem(a) + 1024 > (size_t)dev->smem_optin) return LAPSUM_EINVAL;
+    return cuda_ok(launch_resident_fwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
   }
 
   const StreamSizes s = stream_sizes(n, k, R);
   const StreamLayout L = stream_layout(rows, n, s);
   StreamOcc occ{};
-  if (stream_occupancy(s.C, &occ) != cudaSuccess) return LAPSUM_ECUDA;
+  if (!cuda_ok(stream_occupancy(s.C, &occ))) return LAPSUM_ECUDA;
   StreamPlan P{};
   P.rows = rows;
   P.n = n;
@@ -320,20 +333,19 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
   P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
   P.fb_aggs = ws + L.fb_aggs;
   P.rcount = reinterpret_cast<uint32_t*>(ws + L.rcount);
-  return launch_stream_fwd(P, scores, p_out, b_out, sumf_out, row_status, stats, sm, st) == cudaSuccess
-             ? LAPSUM_OK
-             : LAPSUM_ECUDA;
+  return cuda_ok(launch_stream_fwd(P, scores, p_out, b_out, sumf_out, row_status, stats, sm, st)) ? LAPSUM_OK
+                                                                                                : LAPSUM_ECUDA;
 }
 
-int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, const double* sumf, int64_t rows,
-                    int64_t n, int64_t row_stride, double alpha, float* grad_scores, double* grad_k,
-                    void* workspace, size_t workspace_bytes, void* stream) {
+int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
+                    int64_t row_stride, double alpha, float* grad_scores, double* grad_k, void* workspace,
+                    size_t workspace_bytes, void* stream) {
   if (!scores || !grad_p || !b || !grad_scores) return LAPSUM_EINVAL;
   if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
   if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)grad_scores & 3u) ||
       ((uintptr_t)b & 7u))
     return LAPSUM_EINVAL;
-  if ((sumf && ((uintptr_t)sumf & 7u)) || (grad_k && ((uintptr_t)grad_k & 7u))) return LAPSUM_EINVAL;
+  if (grad_k && ((uintptr_t)grad_k & 7u)) return LAPSUM_EINVAL;
   if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
   const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
   if (overlaps(scores, span, grad_scores, span) || overlaps(grad_p, span, grad_scores, span)) return LAPSUM_EINVAL;
@@ -341,19 +353,18 @@ int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, c
   if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))) return LAPSUM_EWORKSPACE;
   if (n > kResidentMaxN && rows > 65535) return LAPSUM_EINVAL;
   DevInfo* dev = nullptr;
-  if (device_info(&dev) != cudaSuccess) return LAPSUM_ECUDA;
+  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
   if (n <= kResidentMaxN) {
-    RowBwd a{scores, grad_p, b, sumf, rows, n, row_stride, alpha, grad_scores, grad_k, vec};
-    return launch_resident_bwd(a, dev->sm_count, st) == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA;
+    RowBwd a{scores, grad_p, b, rows, n, row_stride, alpha, grad_scores, grad_k, vec};
+    return cuda_ok(launch_resident_bwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
   }
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   StreamBwd a{};
   a.scores = scores;
   a.grad_p = grad_p;
   a.b = b;
-  a.sumf = sumf;
   a.rows = rows;
   a.n = n;
   a.stride = row_stride;
@@ -366,11 +377,11 @@ int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, c
   a.Gb = (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
   size_t o = 0;
   a.part = ws + o;
-  o = align256(o + 16 * (size_t)kMaxGridPerRow * (size_t)rows);
+  o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
   a.done = reinterpret_cast<uint32_t*>(ws + o);
   o = align256(o + 4 * (size_t)rows);
   a.lam = reinterpret_cast<double*>(ws + o);
-  return launch_stream_bwd(a, st) == cudaSuccess ? LAPSUM_OK : LAPSUM_ECUDA;
+  return cuda_ok(launch_stream_bwd(a, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
 }
 
 }  // extern "C"

@@ -191,6 +191,16 @@ __device__ __forceinline__ double closed_form_root(double xj, double xj1, double
   return b;
 }
 
+// sum_i f_i at the root b in [xj, xj1], f_i = exp(-|r_i - b|/alpha)/(2 alpha):
+// the values up to xj contribute A exp((xj - b)/alpha), those from xj1 on
+// contribute Bp exp((b - xj1)/alpha) (A, Bp anchored as in closed_form_root).
+// Exact in fp64, so it does not underflow with the fp32 per-score terms.
+__device__ __forceinline__ double sum_f_at(double xj, double xj1, double A, double Bp, double b, double inva) {
+  const double t1 = A > 0.0 ? A * exp((xj - b) * inva) : 0.0;
+  const double t2 = Bp > 0.0 ? Bp * exp((b - xj1) * inva) : 0.0;
+  return 0.5 * (t1 + t2) * inva;
+}
+
 // ---------------------------------------------------------------------------
 // deterministic block reductions (fixed xor trees; scratch >= NT/32 slots)
 // ---------------------------------------------------------------------------
@@ -331,6 +341,53 @@ __device__ __forceinline__ uint32_t block_excl_prefix_u32(uint32_t v, uint32_t* 
   }
   if (total) *total = tot;
   return wacc + inc - v;
+}
+
+// ---------------------------------------------------------------------------
+// backward reduction: lambda = sum g f / sum f with f = 2^{-a} up to a common
+// factor.  Terms are kept relative to the smallest a seen so far (the score
+// nearest to b), so neither sum underflows even when every f is below the
+// fp32 range; the shift cancels in the ratio.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void shift_add(float a, float g, float& m, float& ps, float& psg, double& S,
+                                          double& SG) {
+  if (a < m) {  // a new nearest score: rescale what was accumulated
+    const float sc = exp2f(a - m);
+    ps *= sc;
+    psg *= sc;
+    S *= (double)sc;
+    SG *= (double)sc;
+    m = a;
+  }
+  const float e = exp2f(m - a);
+  ps += e;
+  psg = fmaf(g, e, psg);
+}
+
+template <int NT>
+__device__ __forceinline__ float block_min_float(float v, float* scratch) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  float t = (lane < NW) ? scratch[lane] : CUDART_INF_F;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t = fminf(t, __shfl_xor_sync(0xffffffffu, t, o));
+  return t;
+}
+
+// Combines every thread's (m, S, SG) into the block's, relative to the block
+// minimum of m (returned in m of every thread).
+template <int NT>
+__device__ __forceinline__ void block_shift_reduce(float& m, double& S, double& SG, double* red) {
+  const float M = block_min_float<NT>(m, reinterpret_cast<float*>(red));
+  const double sc = (m == CUDART_INF_F) ? 0.0 : exp2((double)M - (double)m);
+  S = block_sum<NT, double>(S * sc, red);
+  SG = block_sum<NT, double>(SG * sc, red);
+  m = M;
 }
 
 // ---------------------------------------------------------------------------

@@ -68,7 +68,6 @@ struct RowBwd {
   const float* scores;
   const float* grad_p;
   const double* b;
-  const double* sumf;
   int64_t rows, n, stride;
   double alpha;
   float* grad;
@@ -137,14 +136,13 @@ struct StreamBwd {
   const float* scores;
   const float* grad_p;
   const double* b;
-  const double* sumf;
   int64_t rows, n, stride;
   double alpha;
   float* grad;
   double* grad_k;
   int vec;
   int Gb;
-  void* part;        // [rows][Gb] partials
+  void* part;        // [rows][kMaxGridPerRow] partials (32 bytes each)
   uint32_t* done;    // [rows] counters (zeroed by the launcher)
   double* lam;       // [rows]
 };

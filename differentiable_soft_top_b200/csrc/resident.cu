@@ -108,14 +108,6 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   return f;
 }
 
-// p_i = F((r_i - b)/alpha), with r_i - b formed from b split into two fp32
-// words (b = bh + bl) so that the difference keeps fp64-level accuracy.
-__device__ __forceinline__ float membership(float x, float bh, float bl, float c2, float& h) {
-  const float d = (x - bh) - bl;
-  h = 0.5f * exp2f(-fabsf(d) * c2);
-  return d < 0.0f ? h : 1.0f - h;
-}
-
 __device__ void write_stats(lapsum_row_stats* st, float aL, float aR, long long nL, long long nR, long long M,
                             double SL, double SR, double b, double sump, double sumf, int m, int buckets,
                             uint32_t status) {
@@ -135,18 +127,26 @@ __device__ void write_stats(lapsum_row_stats* st, float aL, float aR, long long 
   st->reserved = 0;
 }
 
+// p_i = F((r_i - b)/alpha) as an fp32 value; (r_i - b) is formed from b split
+// into two fp32 words (b = bh + bl), which keeps it accurate to fp64 level.
+__device__ __forceinline__ float membership(float x, float bh, float bl, float c2) {
+  const float d = (x - bh) - bl;
+  const float h = 0.5f * exp2f(-fabsf(d) * c2);
+  return d < 0.0f ? h : 1.0f - h;
+}
+
 // Writes p for a row from `src` (shared or global) and finishes the row's
-// outputs.  Every thread must call it.
-__device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, double b, uint32_t status,
-                           float aL, float aR, long long nL, long long nR, long long M, double SL,
-                           double SR, int buckets, double* red) {
+// outputs; sumf is the solver's exact sum of f.  Every thread must call it.
+__device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, double b, double sumf,
+                           uint32_t status, float aL, float aR, long long nL, long long nR, long long M,
+                           double SL, double SR, int buckets, double* red) {
   const int n = (int)a.n;
   const double inva = 1.0 / a.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
   float* dst = a.p_out + r * a.stride;
-  double hs = 0.0, ps = 0.0;
+  double ps = 0.0;
   const bool nonfinite = (status & ROW_NONFINITE) != 0u;
   if (a.vec) {
     const float4* s4 = reinterpret_cast<const float4*>(src);
@@ -155,43 +155,34 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
     for (int v = threadIdx.x; v < n4; v += NT) {
       const float4 x = s4[v];
       float4 p;
-      float h0, h1, h2, h3;
-      p.x = membership(x.x, bh, bl, c2, h0);
-      p.y = membership(x.y, bh, bl, c2, h1);
-      p.z = membership(x.z, bh, bl, c2, h2);
-      p.w = membership(x.w, bh, bl, c2, h3);
+      p.x = membership(x.x, bh, bl, c2);
+      p.y = membership(x.y, bh, bl, c2);
+      p.z = membership(x.z, bh, bl, c2);
+      p.w = membership(x.w, bh, bl, c2);
       if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
-      hs += (double)((h0 + h1) + (h2 + h3));
       ps += (double)((p.x + p.y) + (p.z + p.w));
       stg_stream(d4 + v, p);
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
-      float h;
-      float p = membership(src[i], bh, bl, c2, h);
-      if (nonfinite) p = CUDART_NAN_F;
-      hs += (double)h;
+      const float p = nonfinite ? CUDART_NAN_F : membership(src[i], bh, bl, c2);
       ps += (double)p;
       dst[i] = p;
     }
   } else {
     for (int i = threadIdx.x; i < n; i += NT) {
-      float h;
-      float p = membership(src[i], bh, bl, c2, h);
-      if (nonfinite) p = CUDART_NAN_F;
-      hs += (double)h;
+      const float p = nonfinite ? CUDART_NAN_F : membership(src[i], bh, bl, c2);
       ps += (double)p;
       dst[i] = p;
     }
   }
-  hs = block_sum<NT, double>(hs, red);
   ps = block_sum<NT, double>(ps, red);
   if (threadIdx.x == 0) {
     const double bo = nonfinite ? CUDART_NAN : b;
+    const double so = nonfinite ? CUDART_NAN : sumf;
     a.b_out[r] = bo;
-    if (a.sumf_out) a.sumf_out[r] = hs * inva;
+    if (a.sumf_out) a.sumf_out[r] = so;
     if (a.status_out) a.status_out[r] = status & ROW_PUBLIC;
-    if (a.stats) write_stats(a.stats + r, aL, aR, nL, nR, M, SL, SR, bo, ps, hs * inva, a.m, buckets,
-                             status & ROW_PUBLIC);
+    if (a.stats) write_stats(a.stats + r, aL, aR, nL, nR, M, SL, SR, bo, ps, so, a.m, buckets, status & ROW_PUBLIC);
   }
 }
 
@@ -300,9 +291,10 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   }
 
   if (solved) {
-    finish_row(a, r, row, s_out.b, status | ROW_CERTIFIED, aL, aR, f.nL, f.nR, f.M, f.SL, f.SR, 1, red);
+    finish_row(a, r, row, s_out.b, s_out.sumf, status | ROW_CERTIFIED, aL, aR, f.nL, f.nR, f.M, f.SL, f.SR, 1,
+               red);
   } else if (status & ROW_NONFINITE) {
-    finish_row(a, r, row, CUDART_NAN, status, aL, aR, f.nL, f.nR, f.M, f.SL, f.SR, 1, red);
+    finish_row(a, r, row, CUDART_NAN, CUDART_NAN, status, aL, aR, f.nL, f.nR, f.M, f.SL, f.SR, 1, red);
   } else if (threadIdx.x == 0) {
     const uint32_t idx = atomicAdd(a.fb_count, 1u);
     a.fb_list[idx] = (int32_t)r;
@@ -357,23 +349,21 @@ __global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
     SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, a.k, a.alpha, inva};
     solve_band<NT, false>(in, aggs, T, KeyGroups{sorted, kFbGroup}, dscr, red, &s_out);
     const uint32_t status = a.ws_status[r] | ROW_FALLBACK | ROW_CERTIFIED;
-    finish_row(a, r, src, s_out.b, status, -CUDART_INF_F, CUDART_INF_F, 0, 0, n, 0.0, 0.0, T, red);
+    finish_row(a, r, src, s_out.b, s_out.sumf, status, -CUDART_INF_F, CUDART_INF_F, 0, 0, n, 0.0, 0.0, T, red);
   }
 }
 
 // Backward for one row per block (section 2.1, analytic VJP):
-// lambda = sum g f / sum f, then grad = f (g - lambda).
-__device__ __forceinline__ float half_density(float x, float bh, float bl, float c2) {
-  const float d = (x - bh) - bl;
-  return 0.5f * exp2f(-fabsf(d) * c2);
-}
-
+// lambda = sum g f / sum f by the rescaled reduction of common.cuh, then
+// grad = f (g - lambda) with f = 2^(log2(1/(2 alpha)) - |r - b| log2(e)/alpha)
+// computed in one exponent, and lambda split into two fp32 words so that
+// g - lambda keeps its accuracy when g is close to lambda.
 __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
   __shared__ double red[64];
   const int n = (int)a.n;
   const double inva = 1.0 / a.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
-  const float finva = (float)inva;
+  const float lg = (float)log2(0.5 * inva);
   for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
     const float* x = a.scores + r * a.stride;
     const float* g = a.grad_p + r * a.stride;
@@ -381,37 +371,42 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     const double b = a.b[r];
     const float bh = __double2float_rn(b);
     const float bl = __double2float_rn(b - (double)bh);
-    double sh = 0.0, sgh = 0.0;
+    float m = CUDART_INF_F;
+    double S = 0.0, SG = 0.0;
     const int n4 = a.vec ? (n >> 2) : 0;
     for (int v = threadIdx.x; v < n4; v += NT) {
       const float4 xv = __ldg(reinterpret_cast<const float4*>(x) + v);
       const float4 gv = __ldg(reinterpret_cast<const float4*>(g) + v);
-      const float h0 = half_density(xv.x, bh, bl, c2), h1 = half_density(xv.y, bh, bl, c2);
-      const float h2 = half_density(xv.z, bh, bl, c2), h3 = half_density(xv.w, bh, bl, c2);
-      sh += (double)((h0 + h1) + (h2 + h3));
-      sgh += (double)((gv.x * h0 + gv.y * h1) + (gv.z * h2 + gv.w * h3));
+      float ps = 0.0f, psg = 0.0f;
+      shift_add(fabsf((xv.x - bh) - bl) * c2, gv.x, m, ps, psg, S, SG);
+      shift_add(fabsf((xv.y - bh) - bl) * c2, gv.y, m, ps, psg, S, SG);
+      shift_add(fabsf((xv.z - bh) - bl) * c2, gv.z, m, ps, psg, S, SG);
+      shift_add(fabsf((xv.w - bh) - bl) * c2, gv.w, m, ps, psg, S, SG);
+      S += (double)ps;
+      SG += (double)psg;
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
-      const float h = half_density(x[i], bh, bl, c2);
-      sh += (double)h;
-      sgh += (double)(g[i] * h);
+      float ps = 0.0f, psg = 0.0f;
+      shift_add(fabsf((x[i] - bh) - bl) * c2, g[i], m, ps, psg, S, SG);
+      S += (double)ps;
+      SG += (double)psg;
     }
-    sh = block_sum<NT, double>(sh, red);
-    sgh = block_sum<NT, double>(sgh, red);
-    const double lam = a.sumf ? (sgh * inva) / a.sumf[r] : sgh / sh;
-    const float lamf = (float)lam;
+    block_shift_reduce<NT>(m, S, SG, red);
+    const double lam = SG / S;
+    const float lh = __double2float_rn(lam);
+    const float ll = __double2float_rn(lam - (double)lh);
     for (int v = threadIdx.x; v < n4; v += NT) {
       const float4 xv = __ldcs(reinterpret_cast<const float4*>(x) + v);
       const float4 gv = __ldcs(reinterpret_cast<const float4*>(g) + v);
       float4 ov;
-      ov.x = half_density(xv.x, bh, bl, c2) * finva * (gv.x - lamf);
-      ov.y = half_density(xv.y, bh, bl, c2) * finva * (gv.y - lamf);
-      ov.z = half_density(xv.z, bh, bl, c2) * finva * (gv.z - lamf);
-      ov.w = half_density(xv.w, bh, bl, c2) * finva * (gv.w - lamf);
+      ov.x = exp2f(fmaf(-fabsf((xv.x - bh) - bl), c2, lg)) * ((gv.x - lh) - ll);
+      ov.y = exp2f(fmaf(-fabsf((xv.y - bh) - bl), c2, lg)) * ((gv.y - lh) - ll);
+      ov.z = exp2f(fmaf(-fabsf((xv.z - bh) - bl), c2, lg)) * ((gv.z - lh) - ll);
+      ov.w = exp2f(fmaf(-fabsf((xv.w - bh) - bl), c2, lg)) * ((gv.w - lh) - ll);
       stg_stream(reinterpret_cast<float4*>(o) + v, ov);
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT)
-      o[i] = half_density(x[i], bh, bl, c2) * finva * (g[i] - lamf);
+      o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
     if (threadIdx.x == 0 && a.grad_k) a.grad_k[r] = lam;
     __syncthreads();
   }
@@ -422,12 +417,20 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
 size_t resident_fwd_smem(const ResidentFwd& a) { return res_layout(a.n, a.m, a.bcap).total; }
 size_t resident_fallback_smem(int64_t n) { return fb_layout(n).total; }
 
-// Lets both kernels use up to the 227 KB of shared memory a block may opt in
-// to; the size each launch actually requests decides its occupancy.
-cudaError_t resident_init() {
-  cudaError_t e = cudaFuncSetAttribute(k_row_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+// Lets both kernels use all the shared memory a block may opt in to (less
+// their static shared memory); the size each launch actually requests decides
+// its occupancy.
+cudaError_t resident_init(int optin_bytes) {
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k_row_fwd);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_row_fallback, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  e = cudaFuncSetAttribute(k_row_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin_bytes - (int)fa.sharedSizeBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncGetAttributes(&fa, k_row_fallback);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_row_fallback, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              optin_bytes - (int)fa.sharedSizeBytes);
 }
 
 cudaError_t launch_resident_fwd(const ResidentFwd& a, int sm_count, cudaStream_t st) {

@@ -35,6 +35,7 @@ struct SolveIn {
 struct SolveOut {
   uint32_t status;  // ROW_CERTIFIED, or ROW_MISS_LEFT / ROW_MISS_RIGHT
   double b;
+  double sumf;      // sum_i f_i at b
   long long M;      // band size (sum of group counts)
   double S_aL, S_aR;
 };
@@ -138,6 +139,7 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
     if (tid == 0) {
       out->status = (!(S_aL >= in.k) ? ROW_MISS_LEFT : 0u) | (!(S_aR < in.k) ? ROW_MISS_RIGHT : 0u);
       out->b = 0.0;
+      out->sumf = 0.0;
       out->M = M;
       out->S_aL = S_aL;
       out->S_aR = S_aR;
@@ -159,7 +161,9 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
     // no values above the last knot: b in [x_in, a_R)
     if (tid == 0) {
       const double xj1 = finR ? (double)in.aR : CUDART_INF;
-      out->b = closed_form_root(inc.x, xj1, inc.s, finR ? in.SR : 0.0, (double)in.nR, in.k, in.alpha);
+      const double Bp = finR ? in.SR : 0.0;
+      out->b = closed_form_root(inc.x, xj1, inc.s, Bp, (double)in.nR, in.k, in.alpha);
+      out->sumf = sum_f_at(inc.x, xj1, inc.s, Bp, out->b, inva);
       out->status = ROW_CERTIFIED;
       out->M = M;
       out->S_aL = S_aL;
@@ -220,6 +224,7 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
     }
     const double cj = (double)((long long)(c - 1 - i_star) + g_after);
     out->b = closed_form_root(xj, xj1, A, Bp, cj, in.k, in.alpha);
+    out->sumf = sum_f_at(xj, xj1, A, Bp, out->b, inva);
     out->status = ROW_CERTIFIED;
     out->M = M;
     out->S_aL = S_aL;

@@ -447,7 +447,7 @@ __device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int n
   const uint32_t flags = vld(&c->flags);
   const long long nr = P.n - nl - mt;
   uint32_t st = vld(&c->status) & ROW_WIDENED;
-  double b = 0.0;
+  double b = 0.0, sumf = 0.0;
   if (bad) {
     st |= ROW_NONFINITE;
   } else if (flags & ROW_OVERFLOW) {
@@ -459,8 +459,10 @@ __device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int n
     solve_band<NT, true>(in, aggs_of(P, r), T, BandGroups{band_of(P, r), C}, dscr, red, &so);
     st |= so.status;
     b = so.b;
+    sumf = so.sumf;
   }
   if (threadIdx.x == 0) {
+    c->sumf = sumf;
     c->nL = nl;
     c->nR = nr;
     c->M = mt;
@@ -683,6 +685,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         if (threadIdx.x == 0) {
           const uint32_t keep = (vld(&c->status) | st0) & (ROW_WIDENED | ROW_OVERFLOW);
           c->b = so.b;
+          c->sumf = so.sumf;
           c->status = keep | ROW_FALLBACK | ROW_CERTIFIED;
           c->aL = -CUDART_INF_F;
           c->aR = CUDART_INF_F;
@@ -705,9 +708,10 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
 // memberships (section 2.1) and the backward pass
 // ===========================================================================
 
-__device__ __forceinline__ float memb(float x, float bh, float bl, float c2, float& h) {
+// p = F((x - b)/alpha), with x - b formed from b = bh + bl (two fp32 words)
+__device__ __forceinline__ float memb(float x, float bh, float bl, float c2) {
   const float d = (x - bh) - bl;
-  h = 0.5f * exp2f(-fabsf(d) * c2);
+  const float h = 0.5f * exp2f(-fabsf(d) * c2);
   return d < 0.0f ? h : 1.0f - h;
 }
 
@@ -727,12 +731,9 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
   const float* row = scores + r * P.stride;
   float* dst = p_out + r * P.stride;
   const int64_t n = P.n;
-  double hs = 0.0, ps = 0.0;
+  double ps = 0.0;
   auto one = [&](int64_t i) {
-    float h;
-    float p = memb(row[i], bh, bl, c2, h);
-    if (nonfinite) p = CUDART_NAN_F;
-    hs += (double)h;
+    const float p = nonfinite ? CUDART_NAN_F : memb(row[i], bh, bl, c2);
     ps += (double)p;
     dst[i] = p;
   };
@@ -747,52 +748,40 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
       float4 v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) v[u] = __ldg(x4 + base + u * NT);
-      float hl = 0.0f, pl = 0.0f;
+      float pl = 0.0f;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float4 p;
-        float h0, h1, h2, h3;
-        p.x = memb(v[u].x, bh, bl, c2, h0);
-        p.y = memb(v[u].y, bh, bl, c2, h1);
-        p.z = memb(v[u].z, bh, bl, c2, h2);
-        p.w = memb(v[u].w, bh, bl, c2, h3);
+        p.x = memb(v[u].x, bh, bl, c2);
+        p.y = memb(v[u].y, bh, bl, c2);
+        p.z = memb(v[u].z, bh, bl, c2);
+        p.w = memb(v[u].w, bh, bl, c2);
         if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
-        hl += (h0 + h1) + (h2 + h3);
         pl += (p.x + p.y) + (p.z + p.w);
         stg_stream(d4 + base + u * NT, p);
       }
-      hs += (double)hl;
       ps += (double)pl;
     }
-    for (int64_t i = nchunks * CHUNK4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n4; i += (int64_t)gridDim.x * NT) {
-      one(4 * i);
-      one(4 * i + 1);
-      one(4 * i + 2);
-      one(4 * i + 3);
-    }
-    for (int64_t i = 4 * n4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) one(i);
+    for (int64_t i = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * NT)
+      one(i);
   } else {
     for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) one(i);
   }
-  hs = block_sum<NT, double>(hs, red);
   ps = block_sum<NT, double>(ps, red);
-  if (threadIdx.x == 0) mpart_of(P, r)[blockIdx.x] = MPart{hs, ps};
+  if (threadIdx.x == 0) mpart_of(P, r)[blockIdx.x] = MPart{ps, 0.0};
   if (last_block_done(&c->done_memb, gridDim.x)) {
     const MPart* mp = mpart_of(P, r);
-    double h = 0.0, p = 0.0;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
-      h += __ldcg(&mp[i].a);
-      p += __ldcg(&mp[i].b);
-    }
-    h = block_sum<NT, double>(h, red);
+    double p = 0.0;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) p += __ldcg(&mp[i].a);
     p = block_sum<NT, double>(p, red);
     if (threadIdx.x == 0) {
       const double bo = nonfinite ? CUDART_NAN : b;
+      const double so = nonfinite ? CUDART_NAN : c->sumf;
       const uint32_t pub = status & ROW_PUBLIC;
       b_out[r] = bo;
-      if (sumf_out) sumf_out[r] = h * inva;
+      if (sumf_out) sumf_out[r] = so;
       if (status_out) status_out[r] = pub;
-      c->sumf = h * inva;
       c->sump = p;
       if (stats) {
         lapsum_row_stats* s = stats + r;
@@ -805,7 +794,7 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
         s->S_R = c->SR;
         s->b = bo;
         s->sum_p = p;
-        s->sum_f = h * inva;
+        s->sum_f = so;
         s->sample_m = P.m;
         s->buckets = c->T;
         s->status = pub;
@@ -816,14 +805,10 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
 }
 
 struct BPart {
-  double sh, sgh;
+  double m, S, SG, pad;
 };
 
-__device__ __forceinline__ float half_dens(float x, float bh, float bl, float c2) {
-  const float d = (x - bh) - bl;
-  return 0.5f * exp2f(-fabsf(d) * c2);
-}
-
+// lambda = sum g f / sum f by the rescaled reduction of common.cuh
 __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   __shared__ double red[64];
   const int64_t r = blockIdx.y;
@@ -835,12 +820,13 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   const float* x = a.scores + r * a.stride;
   const float* g = a.grad_p + r * a.stride;
   const int64_t n = a.n;
-  double sh = 0.0, sgh = 0.0;
+  float m = CUDART_INF_F;
+  double S = 0.0, SG = 0.0;
+  int64_t done = 0;
   if (a.vec) {
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const float4* g4 = reinterpret_cast<const float4*>(g);
-    const int64_t n4 = n >> 2;
-    const int64_t nchunks = n4 / CHUNK4;
+    const int64_t nchunks = (n >> 2) / CHUNK4;
     for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
       const int64_t base = q * CHUNK4 + threadIdx.x;
       float4 xv[U], gv[U];
@@ -849,68 +835,71 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
         xv[u] = __ldg(x4 + base + u * NT);
         gv[u] = __ldg(g4 + base + u * NT);
       }
-      float hl = 0.0f, gl = 0.0f;
+      float ps = 0.0f, psg = 0.0f;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const float h0 = half_dens(xv[u].x, bh, bl, c2), h1 = half_dens(xv[u].y, bh, bl, c2);
-        const float h2 = half_dens(xv[u].z, bh, bl, c2), h3 = half_dens(xv[u].w, bh, bl, c2);
-        hl += (h0 + h1) + (h2 + h3);
-        gl += (gv[u].x * h0 + gv[u].y * h1) + (gv[u].z * h2 + gv[u].w * h3);
+        shift_add(fabsf((xv[u].x - bh) - bl) * c2, gv[u].x, m, ps, psg, S, SG);
+        shift_add(fabsf((xv[u].y - bh) - bl) * c2, gv[u].y, m, ps, psg, S, SG);
+        shift_add(fabsf((xv[u].z - bh) - bl) * c2, gv[u].z, m, ps, psg, S, SG);
+        shift_add(fabsf((xv[u].w - bh) - bl) * c2, gv[u].w, m, ps, psg, S, SG);
       }
-      sh += (double)hl;
-      sgh += (double)gl;
+      S += (double)ps;
+      SG += (double)psg;
     }
-    for (int64_t i = 4 * nchunks * CHUNK4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
-      const float h = half_dens(x[i], bh, bl, c2);
-      sh += (double)h;
-      sgh += (double)(g[i] * h);
-    }
-  } else {
-    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
-      const float h = half_dens(x[i], bh, bl, c2);
-      sh += (double)h;
-      sgh += (double)(g[i] * h);
-    }
+    done = nchunks * CHUNK4 * 4;
   }
-  sh = block_sum<NT, double>(sh, red);
-  sgh = block_sum<NT, double>(sgh, red);
+  for (int64_t i = done + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
+    float ps = 0.0f, psg = 0.0f;
+    shift_add(fabsf((x[i] - bh) - bl) * c2, g[i], m, ps, psg, S, SG);
+    S += (double)ps;
+    SG += (double)psg;
+  }
+  block_shift_reduce<NT>(m, S, SG, red);
   BPart* part = reinterpret_cast<BPart*>(a.part) + r * kMaxGridPerRow;
-  if (threadIdx.x == 0) part[blockIdx.x] = BPart{sh, sgh};
+  if (threadIdx.x == 0) part[blockIdx.x] = BPart{(double)m, S, SG, 0.0};
   if (last_block_done(a.done + r, gridDim.x)) {
-    double h = 0.0, gh = 0.0;
+    double M = CUDART_INF;
+    for (int i = 0; i < (int)gridDim.x; ++i) M = fmin(M, __ldcg(&part[i].m));
+    double s = 0.0, sg = 0.0;
     for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
-      h += __ldcg(&part[i].sh);
-      gh += __ldcg(&part[i].sgh);
+      const double pm = __ldcg(&part[i].m);
+      const double sc = (pm == CUDART_INF) ? 0.0 : exp2(M - pm);
+      s += __ldcg(&part[i].S) * sc;
+      sg += __ldcg(&part[i].SG) * sc;
     }
-    h = block_sum<NT, double>(h, red);
-    gh = block_sum<NT, double>(gh, red);
+    s = block_sum<NT, double>(s, red);
+    sg = block_sum<NT, double>(sg, red);
     if (threadIdx.x == 0) {
-      const double lam = a.sumf ? (gh * inva) / a.sumf[r] : gh / h;
+      const double lam = sg / s;
       a.lam[r] = lam;
       if (a.grad_k) a.grad_k[r] = lam;
     }
   }
 }
 
+// grad = f (g - lambda), f = 2^(log2(1/(2 alpha)) - |x - b| log2(e)/alpha) in
+// one exponent, lambda split into two fp32 words
 __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
   const int64_t r = blockIdx.y;
   const double b = a.b[r];
   const double inva = 1.0 / a.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
-  const float finva = (float)inva;
+  const float lg = (float)log2(0.5 * inva);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
-  const float lamf = (float)a.lam[r];
+  const double lam = a.lam[r];
+  const float lh = __double2float_rn(lam);
+  const float ll = __double2float_rn(lam - (double)lh);
   const float* x = a.scores + r * a.stride;
   const float* g = a.grad_p + r * a.stride;
   float* o = a.grad + r * a.stride;
   const int64_t n = a.n;
+  int64_t done = 0;
   if (a.vec) {
     const float4* x4 = reinterpret_cast<const float4*>(x);
     const float4* g4 = reinterpret_cast<const float4*>(g);
     float4* o4 = reinterpret_cast<float4*>(o);
-    const int64_t n4 = n >> 2;
-    const int64_t nchunks = n4 / CHUNK4;
+    const int64_t nchunks = (n >> 2) / CHUNK4;
     for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
       const int64_t qq = nchunks - 1 - q;  // reverse of the reduction pass
       const int64_t base = qq * CHUNK4 + threadIdx.x;
@@ -923,19 +912,17 @@ __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float4 ov;
-        ov.x = half_dens(xv[u].x, bh, bl, c2) * finva * (gv[u].x - lamf);
-        ov.y = half_dens(xv[u].y, bh, bl, c2) * finva * (gv[u].y - lamf);
-        ov.z = half_dens(xv[u].z, bh, bl, c2) * finva * (gv[u].z - lamf);
-        ov.w = half_dens(xv[u].w, bh, bl, c2) * finva * (gv[u].w - lamf);
+        ov.x = exp2f(fmaf(-fabsf((xv[u].x - bh) - bl), c2, lg)) * ((gv[u].x - lh) - ll);
+        ov.y = exp2f(fmaf(-fabsf((xv[u].y - bh) - bl), c2, lg)) * ((gv[u].y - lh) - ll);
+        ov.z = exp2f(fmaf(-fabsf((xv[u].z - bh) - bl), c2, lg)) * ((gv[u].z - lh) - ll);
+        ov.w = exp2f(fmaf(-fabsf((xv[u].w - bh) - bl), c2, lg)) * ((gv[u].w - lh) - ll);
         stg_stream(o4 + base + u * NT, ov);
       }
     }
-    for (int64_t i = 4 * nchunks * CHUNK4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
-      o[i] = half_dens(x[i], bh, bl, c2) * finva * (g[i] - lamf);
-  } else {
-    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
-      o[i] = half_dens(x[i], bh, bl, c2) * finva * (g[i] - lamf);
+    done = nchunks * CHUNK4 * 4;
   }
+  for (int64_t i = done + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
+    o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
 }
 
 size_t band_smem(int C) { return (size_t)8 * C + (size_t)SortScratch<NT>::kWords * 4 + 64 * 8; }

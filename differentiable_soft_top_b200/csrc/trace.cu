@@ -94,11 +94,11 @@ int lapsum_trace_collect(char* buf, size_t len) {
     first = false;
   }
   out += "}";
-  g_acc.clear();
-  if (!buf || len == 0) return (int)out.size() + 1;
+  if (!buf || len == 0) return (int)out.size() + 1;  // size query: keep the record
   const size_t w = std::min(len - 1, out.size());
   std::memcpy(buf, out.data(), w);
   buf[w] = '\0';
+  g_acc.clear();
   return (int)w;
 }
 

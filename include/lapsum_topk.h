@@ -147,18 +147,21 @@ LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int
  *   scores      in   fp32 [rows, row_stride], the forward's input
  *   grad_p      in   fp32 [rows, row_stride], upstream gradient dL/dp
  *   b           in   fp64 [rows], the forward's b_out
- *   sumf        in   fp64 [rows], the forward's sumf_out, or NULL to
- *                    recompute sum_i f_i inside the reduction pass
  *   alpha       in   the forward's alpha
  *   grad_scores out  fp32 [rows, row_stride] dL/dr
  *   grad_k      out  fp64 [rows] dL/dk = lambda (may be NULL)
  *   workspace   in   as for the forward (the same buffer may be passed)
+ * sum_i f_i is not an input: the reduction pass forms sum g f and sum f
+ * together, relative to the score nearest b, so that neither underflows.
  * Returns LAPSUM_OK or an error code (nothing enqueued on error).
  */
-LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b,
-                    const double* sumf, int64_t rows, int64_t n, int64_t row_stride,
-                    double alpha, float* grad_scores, double* grad_k, void* workspace,
-                    size_t workspace_bytes, void* stream);
+LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows,
+                               int64_t n, int64_t row_stride, double alpha, float* grad_scores,
+                               double* grad_k, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Text of the CUDA error behind the last LAPSUM_ECUDA returned on the
+   calling host thread ("no error" if none). */
+LAPSUM_API const char* lapsum_last_cuda_error(void);
 
 /* Static English text for a return code. */
 LAPSUM_API const char* lapsum_status_string(int code);
@@ -174,8 +177,9 @@ LAPSUM_API uint64_t lapsum_launch_count(void);
  * the recorded events, writes a JSON object
  *     {"<kernel>": [launches, total_milliseconds], ...}
  * into buf (truncated to len-1 bytes, NUL-terminated), clears the record, and
- * returns the number of bytes written (or the size needed when buf is NULL),
- * or -1 if a CUDA call fails.  Both functions are thread-safe.
+ * returns the number of bytes written, or -1 if a CUDA call fails.  With
+ * buf == NULL it returns the size needed and keeps the record.  Both
+ * functions are thread-safe.
  */
 LAPSUM_API void lapsum_trace_enable(int on);
 LAPSUM_API int lapsum_trace_collect(char* buf, size_t len);

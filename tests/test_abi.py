@@ -28,7 +28,7 @@ def lib():
 def test_header_declares_the_boundary():
     names = declared_functions()
     assert names == sorted([
-        "lapsum_default_params", "lapsum_launch_count", "lapsum_status_string",
+        "lapsum_default_params", "lapsum_last_cuda_error", "lapsum_launch_count", "lapsum_status_string",
         "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_workspace_size",
         "lapsum_trace_collect", "lapsum_trace_enable",
     ])
@@ -112,12 +112,12 @@ def test_fwd_rejects_bad_arguments(lib, kw, code):
 
 def test_bwd_rejects_bad_arguments(lib):
     B = lib.lapsum_topk_bwd
-    ok = dict(s=FAKE, g=FAKE * 2, b=FAKE * 3, sf=None, rows=1, n=100000, stride=100000, a=0.5, out=FAKE * 4,
+    ok = dict(s=FAKE, g=FAKE * 2, b=FAKE * 3, rows=1, n=100000, stride=100000, a=0.5, out=FAKE * 4,
               gk=None, ws=FAKE * 8, wsb=1 << 30)
 
     def call(**kw):
         d = dict(ok, **kw)
-        return B(d["s"], d["g"], d["b"], d["sf"], d["rows"], d["n"], d["stride"], d["a"], d["out"], d["gk"],
+        return B(d["s"], d["g"], d["b"], d["rows"], d["n"], d["stride"], d["a"], d["out"], d["gk"],
                  d["ws"], d["wsb"], None)
 
     assert call(s=None) == lt.LAPSUM_EINVAL

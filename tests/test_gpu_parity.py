@@ -31,7 +31,7 @@ def gpu_run(x_np, g_np, k, alpha, params=None, stats=False):
     x = torch.from_numpy(np.ascontiguousarray(x_np)).cuda()
     g = torch.from_numpy(np.ascontiguousarray(g_np)).cuda()
     res = lt.forward(x, k, alpha, params=params, stats=stats)
-    grad, gk = lt.backward(x, g, res.b, alpha, sumf=res.sumf)
+    grad, gk = lt.backward(x, g, res.b, alpha)
     torch.cuda.synchronize()
     return dict(p=res.p.cpu().numpy(), b=res.b.cpu().numpy(), sumf=res.sumf.cpu().numpy(),
                 status=res.status.cpu().numpy().astype(np.uint32), stats=res.stats,
@@ -40,21 +40,26 @@ def gpu_run(x_np, g_np, k, alpha, params=None, stats=False):
 
 def check_row(orc, r, g, p, grad, b, gk, k, alpha, label=""):
     r = np.asarray(r, np.float32).reshape(-1)
+    gg = np.asarray(g, np.float32).reshape(-1)
     n = r.size
-    p_ref, b_ref, _ = orc.forward(r, k, alpha)
-    grad_ref, lam, _ = orc.backward(r, np.asarray(g, np.float32).reshape(-1), b_ref, alpha)
+    p_ref, b_ref, sumf_ref = orc.forward(r, k, alpha)
+    grad_ref, lam, _ = orc.backward(r, gg, b_ref, alpha)
     p = np.asarray(p, np.float64).reshape(-1)
     grad = np.asarray(grad, np.float64).reshape(-1)
     dp = float(np.max(np.abs(p - p_ref)))
     assert dp <= 1e-5, f"{label} max|dp|={dp:.3e} b_gpu={b!r} b_ref={b_ref!r}"
     sp = math.fsum(p.tolist())
     assert abs(sp - k) <= tol_sum(k, n), f"{label} sum p={sp} k={k}"
-    nref = float(np.linalg.norm(grad_ref))
-    if nref > 0:
-        rel = float(np.linalg.norm(grad - grad_ref)) / nref
-        assert rel <= 1e-4, f"{label} grad rel err {rel:.3e}"
+    # relative L2 error of the gradient, with the floor an fp32 output cannot
+    # beat: rounding of the terms f g (6e-8 each, 16x margin) and values below
+    # the smallest normal fp32 number
+    f = 0.5 * np.exp(-np.abs(r.astype(np.float64) - b_ref) / alpha) / alpha
+    err = float(np.linalg.norm(grad - grad_ref))
+    bound = 1e-4 * float(np.linalg.norm(grad_ref)) + 1e-6 * float(np.linalg.norm(f * gg)) + 1.2e-38 * math.sqrt(n)
+    assert err <= bound, f"{label} grad err {err:.3e} > {bound:.3e} (ref norm {np.linalg.norm(grad_ref):.3e})"
+    # b: far inside the p tolerance (dp/db <= 1/(2 alpha)); fp32 tail sums allow ~1e-6 alpha
     assert abs(b - b_ref) <= 2e-6 * alpha + 1e-12 * abs(b_ref), f"{label} b {b!r} vs {b_ref!r}"
-    assert gk == pytest.approx(lam, rel=1e-4, abs=1e-8 * (1 + abs(lam)))
+    assert gk == pytest.approx(lam, rel=1e-4, abs=1e-6 * (1 + abs(lam)))
     return b_ref
 
 
@@ -214,7 +219,8 @@ def test_forced_paths_give_the_same_threshold(orc, name, n, force):
         assert np.all(o["status"] & lt.ROW_CERTIFIED)
         for i in range(x.shape[0]):
             check_row(orc, x[i], g[i], o["p"][i], o["grad"][i], o["b"][i], o["gk"][i], w.k, w.alpha, name)
-            assert abs(o["b"][i] - base["b"][i]) <= 1e-9 * max(1.0, abs(base["b"][i])) + 1e-9 * w.alpha
+            # paths differ only in which sums use fp32 exp (tails) or fp64 (band, fallback)
+            assert abs(o["b"][i] - base["b"][i]) <= 4e-6 * w.alpha + 1e-12 * abs(base["b"][i])
     assert np.any(wid["status"] & (lt.ROW_WIDENED | lt.ROW_FALLBACK))
     assert np.all(((nowid["status"] & lt.ROW_FALLBACK) != 0) | (nowid["status"] == lt.ROW_CERTIFIED))
     assert np.all(ovf["status"] & lt.ROW_FALLBACK)
@@ -257,14 +263,34 @@ def test_deterministic():
     assert np.array_equal(a["grad"], b["grad"])
 
 
-def test_autograd_wrapper_and_optional_sumf(orc):
+def test_autograd_wrapper(orc):
     w, x, g = case("c1")
     xt = torch.from_numpy(x[0]).cuda().requires_grad_(True)
     p = lt.soft_topk(xt, w.k, w.alpha)
     p.backward(torch.from_numpy(g[0]).cuda())
     res = lt.forward(xt.detach(), w.k, w.alpha)
-    g1, _ = lt.backward(xt.detach(), torch.from_numpy(g[0]).cuda(), res.b, w.alpha, sumf=res.sumf)
-    g2, _ = lt.backward(xt.detach(), torch.from_numpy(g[0]).cuda(), res.b, w.alpha)
-    assert torch.allclose(xt.grad, g1, rtol=0, atol=0)
-    assert float((g1 - g2).norm() / g1.norm()) < 1e-6
+    g1, _ = lt.backward(xt.detach(), torch.from_numpy(g[0]).cuda(), res.b, w.alpha)
+    assert torch.equal(xt.grad, g1)
     assert lt.launch_count() > 0
+
+
+def test_sumf_matches_oracle(orc):
+    for name, n in (("c1", None), ("c2", None), ("c5", None)):
+        w, x, g = case(name, n=n) if name != "c5" else case("c5", rows=4)
+        out = gpu_run(x, g, w.k, w.alpha)
+        for i in range(x.shape[0]):
+            _, _, sf = orc.forward(x[i], w.k, w.alpha)
+            assert out["sumf"][i] == pytest.approx(sf, rel=1e-5)
+
+
+def test_deep_underflow_gradient_stays_finite(orc):
+    """alpha far below the score spacing: every f is below the fp32 range, yet
+    lambda (= dL/dk) is finite and the gradient is zero, not NaN."""
+    n = 4096
+    x = (np.arange(n, dtype=np.float64) * 1e-2).astype(np.float32).reshape(1, n)
+    g = make_grad(1, n, seed=3)
+    out = gpu_run(x, g, 100.0, 1e-5)  # integer k: b at the midpoint of two scores, 500 alpha from each
+    _, b_ref, _ = orc.forward(x[0], 100.0, 1e-5)
+    _, lam, _ = orc.backward(x[0], g[0], b_ref, 1e-5)
+    assert np.isfinite(out["gk"][0]) and out["gk"][0] == pytest.approx(lam, rel=1e-4, abs=1e-6)
+    assert np.all(np.isfinite(out["grad"]))
