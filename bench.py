@@ -62,6 +62,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true")
+    ap.add_argument("--n", type=int, default=0, help="scale the workload to n scores per row (k keeps its ratio)")
     return ap.parse_args()
 
 
@@ -249,6 +250,8 @@ def main():
     torch.cuda.set_device(dev)
 
     w = WORKLOADS[args.workload]
+    if args.n:
+        w = w.scaled(n=args.n)
     rows, n = w.rows, w.n
     x_np = make_scores(w)
     g_np = make_grad(rows, n)

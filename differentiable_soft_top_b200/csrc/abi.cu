@@ -190,6 +190,14 @@ size_t fwd_ws_bytes(int64_t rows, int64_t n, double k, const Resolved& R) {
   return stream_layout(rows, n, stream_sizes(n, k, R)).total;
 }
 
+// Blocks per row of a streaming pass: one full wave of the device shared by
+// the rows, but no more blocks than 4096-score chunks in a row.
+int stream_grid(int sm_count, int blocks_per_sm, int64_t rows, int64_t n) {
+  const int64_t per_row = std::max<int64_t>(1, (int64_t)sm_count * blocks_per_sm / rows);
+  const int64_t chunks = std::max<int64_t>(1, (n / 4 + 1023) / 1024);
+  return (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
+}
+
 bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
   return x < y + bn && y < x + an;
@@ -312,11 +320,9 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
   P.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
   P.vec = vec;
   const int sm = dev->sm_count;
-  const int64_t per_row = std::max<int64_t>(1, (int64_t)sm * occ.filter_blocks / rows);
-  const int64_t chunks = std::max<int64_t>(1, (n / 4 + 1023) / 1024);
   P.Gs = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (s.m + 1023) / 1024));
-  P.Gf = (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
-  P.Gm = P.Gf;
+  P.Gf = stream_grid(sm, occ.filter_blocks, rows, n);
+  P.Gm = stream_grid(sm, occ.memb_blocks, rows, n);
   P.G3 = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)s.T, std::max<int64_t>(1, (int64_t)sm * occ.band_blocks / rows)));
   P.Gr = std::min(kMaxGridPerRow, sm * occ.recover_blocks);
   P.ctl = ws + L.ctl;
@@ -372,9 +378,8 @@ int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, i
   a.grad = grad_scores;
   a.grad_k = grad_k;
   a.vec = vec;
-  const int64_t per_row = std::max<int64_t>(1, (int64_t)dev->sm_count * dev->occ.filter_blocks / rows);
-  const int64_t chunks = std::max<int64_t>(1, (n / 4 + 1023) / 1024);
-  a.Gb = (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
+  a.Gb = stream_grid(dev->sm_count, dev->occ.reduce_blocks, rows, n);
+  a.Ga = stream_grid(dev->sm_count, dev->occ.apply_blocks, rows, n);
   size_t o = 0;
   a.part = ws + o;
   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);

@@ -141,7 +141,7 @@ struct StreamBwd {
   float* grad;
   double* grad_k;
   int vec;
-  int Gb;
+  int Gb, Ga;        // grids of the reduction and elementwise passes
   void* part;        // [rows][kMaxGridPerRow] partials (32 bytes each)
   uint32_t* done;    // [rows] counters (zeroed by the launcher)
   double* lam;       // [rows]
@@ -150,7 +150,10 @@ cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st);
 
 // occupancy facts of the streaming kernels on the current device
 struct StreamOcc {
-  int filter_blocks;    // resident blocks per SM of the streaming passes
+  int filter_blocks;    // resident blocks per SM of the filter pass
+  int memb_blocks;      // of the membership pass
+  int reduce_blocks;    // of the backward reduction
+  int apply_blocks;     // of the backward elementwise pass
   int band_blocks;      // of the band sort kernel for the given bucket size
   int recover_blocks;   // of the cooperative recovery kernel
 };

@@ -276,8 +276,13 @@ __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
 // stream and filter (section 2.2, step 2)
 // ===========================================================================
 
+// In-band values are first staged in shared memory (a shared atomic per value,
+// no round trip to L2 inside the streaming loop) and appended to their global
+// buckets once per block at the end; a full stage spills to direct appends.
+constexpr int kStage = 3072;
+
 __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
-                             int ncta, double* red) {
+                             int ncta, double* red, float* stage, int* stage_n) {
   const float aL = vld(&c->aL), aR = vld(&c->aR), lo = vld(&c->lo), inv_w = vld(&c->inv_w);
   const int T = vld(&c->T), C = vld(&c->C);
   const float c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
@@ -286,8 +291,10 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   long long nl = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u, ovf = 0u;
+  if (threadIdx.x == 0) *stage_n = 0;
+  __syncthreads();
 
-  // an in-band value: append it to its value bucket (rare)
+  // an in-band value: append it to its value bucket
   auto append = [&](float x) {
     if (!(fabsf(x) < CUDART_INF_F)) {
       bad = 1u;
@@ -299,6 +306,16 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
     if (slot < (uint32_t)C) band[(int64_t)t * C + slot] = x;
     else ovf = 1u;
   };
+  // an in-band value met in the streaming loop: stage it
+  auto keep = [&](float x) {
+    if (!(fabsf(x) < CUDART_INF_F)) {
+      bad = 1u;
+      return;
+    }
+    const int pos = atomicAdd(stage_n, 1);
+    if (pos < kStage) stage[pos] = x;
+    else append(x);
+  };
   // one value, checked path
   auto one = [&](float x) {
     const bool isL = x < aL, isR = x >= aR;
@@ -306,7 +323,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
     if (isL) { sl += (double)e; ++nl; }
     if (isR) sr += (double)e;
     if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;
-    if (!(isL || isR)) append(x);
+    if (!(isL || isR)) keep(x);
   };
 
   const int64_t n = P.n;
@@ -347,7 +364,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
             const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
             for (int w = 0; w < 4; ++w)
-              if (!(xs[w] < aL) && !(xs[w] >= aR)) append(xs[w]);
+              if (!(xs[w] < aL) && !(xs[w] >= aR)) keep(xs[w]);
           }
         }
       }
@@ -363,6 +380,9 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   } else {
     for (int64_t i = (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) one(row[i]);
   }
+  __syncthreads();
+  const int ns = min(*stage_n, kStage);
+  for (int i = threadIdx.x; i < ns; i += NT) append(stage[i]);
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
   nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
   sl = block_sum<NT, double>(sl, red);
@@ -380,10 +400,12 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(NT) k_filter(const StreamPlan P, const float* __restrict__ scores) {
+__global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const float* __restrict__ scores) {
   __shared__ double red[64];
+  __shared__ float stage[kStage];
+  __shared__ int stage_n;
   const int64_t r = blockIdx.y;
-  filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red);
+  filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red, stage, &stage_n);
 }
 
 // ===========================================================================
@@ -586,7 +608,8 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         }
       }
       REC_BARRIER();
-      filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red);
+      filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(tbuf),
+                   reinterpret_cast<int*>(tbuf + kStage));
       REC_BARRIER();
       band_sort_phase(P, r, c, cta, ncta, kbuf, tbuf, hist, red);
       REC_BARRIER();
@@ -934,14 +957,23 @@ cudaError_t stream_occupancy(int C, StreamOcc* out) {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_recover, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RecSmem::kTotal);
   if (e != cudaSuccess) return e;
-  int fb = 0, bb = 0, rb = 0;
+  int fb = 0, bb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb, NT, 0);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&qb, k_bwd_reduce, NT, 0);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ab, k_bwd_apply, NT, 0);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bb, k_band, NT, band_smem(C));
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&rb, k_recover, NT, RecSmem::kTotal);
   if (e != cudaSuccess) return e;
   out->filter_blocks = std::max(fb, 1);
+  out->memb_blocks = std::max(mb, 1);
+  out->reduce_blocks = std::max(qb, 1);
+  out->apply_blocks = std::max(ab, 1);
   out->band_blocks = std::max(bb, 1);
   out->recover_blocks = std::max(rb, 1);
   return cudaSuccess;
@@ -999,7 +1031,7 @@ cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st) {
   }
   {
     Launch l("k_bwd_apply", st);
-    k_bwd_apply<<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+    k_bwd_apply<<<dim3(a.Ga, (unsigned)a.rows), NT, 0, st>>>(a);
   }
   return cudaGetLastError();
 }
