@@ -145,10 +145,12 @@ StreamSizes stream_sizes(int64_t n, double k, const Resolved& R) {
                  : (int)std::min<int64_t>(1 << 17, std::max<int64_t>(2048, round_up(n / 8, 1024)));
   s.rk = sample_ranks(n, k, s.m, R.z);
   const double M_est = (double)(s.rk.rank_hi - s.rk.rank_lo + 1) * (double)n / (double)s.m;
-  int64_t cap = R.bcap_user > 0 ? R.bcap_user : (int64_t)(8.0 * M_est) + 65536;
-  cap = std::max<int64_t>(1024, std::min<int64_t>(cap, (int64_t)round_up(n, 1024)));
+  // default capacity: four times the expected band plus slack, so a bucket
+  // holds about 4x its expected count (overflow sends the row to the fallback)
+  int64_t cap = R.bcap_user > 0 ? R.bcap_user : (int64_t)(4.0 * M_est) + 16384;
+  cap = std::max<int64_t>(R.bcap_user > 0 ? 4 : 1024, std::min<int64_t>(cap, (int64_t)round_up(n, 1024)));
   s.band_cap = round_up(cap, 4);
-  s.T_max = (int)std::max<int64_t>(1, std::min<int64_t>(4096, s.band_cap / 256));
+  s.T_max = (int)std::max<int64_t>(1, std::min<int64_t>(4096, s.band_cap / 1024));
   plan_buckets(n, s.m, s.rk.rank_lo, s.rk.rank_hi, s.T_max, s.band_cap, &s.T, &s.C);
   return s;
 }

@@ -108,6 +108,9 @@ struct alignas(256) RowCtl {
   uint32_t sel_key[2];
   double lam;
   uint32_t timeout;    // set when a bounded grid-wide wait gives up
+  uint32_t done_s1, done_s2;   // last-block counters of the selection levels
+  int32_t sel_bin[2][2];       // radix-select bins of levels 1 and 2, per edge
+  uint32_t sel_rem[2][2];      // rank left inside those bins
 };
 static_assert(sizeof(RowCtl) == 256, "RowCtl must stay one 256-byte slot");
 

@@ -54,14 +54,25 @@ __device__ __forceinline__ int block_min_int(int v, int* scratch) {
   return -block_max_int<NT>(-v, scratch);
 }
 
-// Elems: float get(int g, int i) returns value i of group g.
-// agg[0..T): cnt, ymin, ymax, P, Q filled in; Apre/Bx/Bs/after are written.
-// dscr: >= (largest group count) doubles of scratch (shared or global).
-// red:  >= 4 * NT/32 + 8 doubles of shared scratch.
-// The result is valid in every thread on return.
-template <int NT, bool kG, typename Elems>
-__device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& el,
-                           double* dscr, double* red, SolveOut* out) {
+// Result of the group-level step, shared by every thread of the block.
+struct GroupPick {
+  uint32_t status;     // ROW_CERTIFIED (go on) or ROW_MISS_LEFT / ROW_MISS_RIGHT
+  int tg;              // group holding knot j*+1, or -1: b lies in [x_in, a_R)
+  double inc_x, inc_s; // prefix state at the knot x_in (the last knot with S >= k
+                       // among a_L and the group maxima)
+  double out_x, out_s; // suffix state of everything after group tg
+  long long g_after;   // number of values after group tg (right tail included)
+  long long M;         // band size
+  double S_aL, S_aR;
+};
+
+// Group level: prefix sums at each group maximum, suffix sums at each group
+// minimum, knot values S(ymax_t), certification, and the group that holds the
+// knot after the root.  agg[0..T): cnt, ymin, ymax, P, Q filled in (Apre, Bx,
+// Bs, after are written).  red: >= 4 * NT/32 + 8 doubles of shared scratch.
+// The result is in *pk (shared) on return, in every thread.
+template <int NT, bool kG>
+__device__ void solve_groups(const SolveIn in, GroupAgg* agg, int T, double* red, GroupPick* pk) {
 #define AGG(t, f) ld<kG>(&agg[t].f)
   const double inva = in.inva;
   const int tid = threadIdx.x;
@@ -74,7 +85,7 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
   const Anch left = (finL && in.SL > 0.0) ? Anch{(double)in.aL, in.SL} : anch_empty();
   const Anch right = (finR && in.SR > 0.0) ? Anch{(double)in.aR, in.SR} : anch_empty();
 
-  // ---- group level, prefix direction: A at each group maximum ----------
+  // prefix direction: A at each group maximum
   const int q = (T + NT - 1) / NT;
   const int t0 = min(T, tid * q), t1 = min(T, t0 + q);
   Anch loc = anch_empty();
@@ -92,7 +103,7 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
     s_dbl[1] = st.s;
   }
 
-  // ---- group level, suffix direction, and the group knot values ---------
+  // suffix direction and the group knot values
   Anch sloc = anch_empty();
   long long cloc = 0;
   for (int t = t1 - 1; t >= t0; --t) {
@@ -103,7 +114,7 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
   }
   const Anch sexc = block_excl_scan_anch<NT, false>(sloc, inva, red);
   const long long cexc = block_excl_suffix_sum<NT>(cloc, lscr);
-  __syncthreads();  // agg[].Apre of every thread is visible below
+  __syncthreads();
   Anch ss = comb_suf(sexc, right, inva);
   long long after = cexc + in.nR;
   int cand = -1;
@@ -127,7 +138,7 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
   const int t_star = block_max_int<NT>(cand, iscr);
   __syncthreads();
 
-  // ---- certification (arXiv abstract: the bracket is proven, not trusted) --
+  // certification (arXiv abstract: the bracket is proven, not trusted)
   const Anch pre_all = Anch{s_dbl[0], s_dbl[1]};
   const Anch suf_all = Anch{s_dbl[2], s_dbl[3]};
   const long long M = s_ll[0] - in.nR;
@@ -135,65 +146,86 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
                            : CUDART_INF;
   const double S_aR = finR ? 0.5 * pre_at(pre_all, (double)in.aR, inva) + (double)in.nR - 0.5 * in.SR
                            : -CUDART_INF;
-  if (!(S_aL >= in.k) || !(S_aR < in.k)) {
-    if (tid == 0) {
-      out->status = (!(S_aL >= in.k) ? ROW_MISS_LEFT : 0u) | (!(S_aR < in.k) ? ROW_MISS_RIGHT : 0u);
-      out->b = 0.0;
-      out->sumf = 0.0;
-      out->M = M;
-      out->S_aL = S_aL;
-      out->S_aR = S_aR;
-    }
-    __syncthreads();
-    return;
-  }
+  const bool cert = (S_aL >= in.k) && (S_aR < in.k);
 
-  // ---- the group that holds knot j*+1 -----------------------------------
+  // the group that holds knot j*+1
   int tg_loc = INT32_MAX;
   for (int t = t0; t < t1; ++t)
     if (t > t_star && AGG(t, cnt) > 0) { tg_loc = t; break; }
   const int tg = block_min_int<NT>(tg_loc, iscr);
-  Anch inc;  // prefix state up to and including knot x_in (anchored there)
-  if (t_star >= 0) inc = Anch{(double)AGG(t_star, ymax), AGG(t_star, Apre)};
-  else inc = finL ? Anch{(double)in.aL, in.SL} : Anch{-CUDART_INF, 0.0};
-
-  if (tg == INT32_MAX) {
-    // no values above the last knot: b in [x_in, a_R)
-    if (tid == 0) {
-      const double xj1 = finR ? (double)in.aR : CUDART_INF;
-      const double Bp = finR ? in.SR : 0.0;
-      out->b = closed_form_root(inc.x, xj1, inc.s, Bp, (double)in.nR, in.k, in.alpha);
-      out->sumf = sum_f_at(inc.x, xj1, inc.s, Bp, out->b, inva);
-      out->status = ROW_CERTIFIED;
-      out->M = M;
-      out->S_aL = S_aL;
-      out->S_aR = S_aR;
+  if (tid == 0) {
+    pk->status = cert ? ROW_CERTIFIED
+                      : ((!(S_aL >= in.k) ? ROW_MISS_LEFT : 0u) | (!(S_aR < in.k) ? ROW_MISS_RIGHT : 0u));
+    pk->M = M;
+    pk->S_aL = S_aL;
+    pk->S_aR = S_aR;
+    if (t_star >= 0) {
+      pk->inc_x = (double)AGG(t_star, ymax);
+      pk->inc_s = AGG(t_star, Apre);
+    } else if (finL) {
+      pk->inc_x = (double)in.aL;
+      pk->inc_s = in.SL;
+    } else {
+      pk->inc_x = -CUDART_INF;
+      pk->inc_s = 0.0;
     }
-    __syncthreads();
-    return;
+    if (tg == INT32_MAX) {
+      pk->tg = -1;
+      pk->out_x = finR ? (double)in.aR : CUDART_INF;
+      pk->out_s = finR ? in.SR : 0.0;
+      pk->g_after = in.nR;
+    } else {
+      pk->tg = tg;
+      pk->out_x = AGG(tg, Bx);
+      pk->out_s = AGG(tg, Bs);
+      pk->g_after = AGG(tg, after);
+    }
   }
+  __syncthreads();
+#undef AGG
+}
 
-  // ---- value level inside group tg -------------------------------------
-  const int c = AGG(tg, cnt);
-  const Anch outg = Anch{AGG(tg, Bx), AGG(tg, Bs)};
-  const long long g_after = AGG(tg, after);
+// Root when no value lies above the last group knot: b in [x_in, a_R).
+__device__ inline void solve_tail_interval(const SolveIn& in, const GroupPick& pk, SolveOut* out) {
+  const double xj1 = isfinite(in.aR) ? (double)in.aR : CUDART_INF;
+  out->b = closed_form_root(pk.inc_x, xj1, pk.inc_s, pk.out_s, (double)pk.g_after, in.k, in.alpha);
+  out->sumf = sum_f_at(pk.inc_x, xj1, pk.inc_s, pk.out_s, out->b, in.inva);
+  out->status = ROW_CERTIFIED;
+  out->M = pk.M;
+  out->S_aL = pk.S_aL;
+  out->S_aR = pk.S_aR;
+}
+
+// Value level inside the picked group: its c values in ascending order are
+// el.get(i); A at each value, the knot after which S drops below k, the
+// closed-form root.  dscr: >= c doubles.  Every thread must call it.
+template <int NT, typename Vals>
+__device__ void solve_values(const SolveIn in, const GroupPick& pk, int c, const Vals& el, double* dscr,
+                             double* red, SolveOut* out) {
+  const double inva = in.inva;
+  const int tid = threadIdx.x;
+  __shared__ double s_bp;
+  int* iscr = reinterpret_cast<int*>(red);
+  const Anch inc = Anch{pk.inc_x, pk.inc_s};
+  const Anch outg = Anch{pk.out_x, pk.out_s};
+  const long long g_after = pk.g_after;
   const int qe = (c + NT - 1) / NT;
   const int i0 = min(c, tid * qe), i1 = min(c, i0 + qe);
   Anch lp = anch_empty();
-  for (int i = i0; i < i1; ++i) lp = comb_pre(lp, Anch{(double)el.get(tg, i), 1.0}, inva);
+  for (int i = i0; i < i1; ++i) lp = comb_pre(lp, Anch{(double)el.get(i), 1.0}, inva);
   Anch ps = comb_pre(inc, block_excl_scan_anch<NT, true>(lp, inva, red), inva);
   for (int i = i0; i < i1; ++i) {
-    ps = comb_pre(ps, Anch{(double)el.get(tg, i), 1.0}, inva);
+    ps = comb_pre(ps, Anch{(double)el.get(i), 1.0}, inva);
     dscr[i] = ps.s;  // A_i anchored at y_i
   }
   Anch ls = anch_empty();
-  for (int i = i1 - 1; i >= i0; --i) ls = comb_suf(Anch{(double)el.get(tg, i), 1.0}, ls, inva);
+  for (int i = i1 - 1; i >= i0; --i) ls = comb_suf(Anch{(double)el.get(i), 1.0}, ls, inva);
   const Anch chunk_in = comb_suf(block_excl_scan_anch<NT, false>(ls, inva, red), outg, inva);
   __syncthreads();  // dscr complete
   Anch sv = chunk_in;
   int icand = -1;
   for (int i = i1 - 1; i >= i0; --i) {
-    const double y = (double)el.get(tg, i);
+    const double y = (double)el.get(i);
     const double S = 0.5 * dscr[i] + (double)((long long)(c - 1 - i) + g_after) - 0.5 * suf_at(sv, y, inva);
     if (icand < 0 && S >= in.k) icand = i;
     sv = comb_suf(Anch{y, 1.0}, sv, inva);
@@ -202,8 +234,8 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
   const int jn = i_star + 1;  // right knot index inside the group (c = beyond)
   if (jn < c && jn >= i0 && jn < i1) {
     Anch w = chunk_in;
-    for (int i = i1 - 1; i >= jn; --i) w = comb_suf(Anch{(double)el.get(tg, i), 1.0}, w, inva);
-    s_dbl[4] = w.s;  // B' at y_jn, anchored there
+    for (int i = i1 - 1; i >= jn; --i) w = comb_suf(Anch{(double)el.get(i), 1.0}, w, inva);
+    s_bp = w.s;  // B' at y_jn, anchored there
   }
   __syncthreads();
   if (tid == 0) {
@@ -212,26 +244,104 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
       xj = inc.x;
       A = inc.s;
     } else {
-      xj = (double)el.get(tg, i_star);
+      xj = (double)el.get(i_star);
       A = dscr[i_star];
     }
     if (jn < c) {
-      xj1 = (double)el.get(tg, jn);
-      Bp = s_dbl[4];
+      xj1 = (double)el.get(jn);
+      Bp = s_bp;
     } else {
-      xj1 = (outg.s > 0.0) ? outg.x : (finR ? (double)in.aR : CUDART_INF);
+      xj1 = (outg.s > 0.0) ? outg.x : (isfinite(in.aR) ? (double)in.aR : CUDART_INF);
       Bp = outg.s;
     }
     const double cj = (double)((long long)(c - 1 - i_star) + g_after);
     out->b = closed_form_root(xj, xj1, A, Bp, cj, in.k, in.alpha);
     out->sumf = sum_f_at(xj, xj1, A, Bp, out->b, inva);
     out->status = ROW_CERTIFIED;
-    out->M = M;
-    out->S_aL = S_aL;
-    out->S_aR = S_aR;
+    out->M = pk.M;
+    out->S_aL = pk.S_aL;
+    out->S_aR = pk.S_aR;
   }
   __syncthreads();
-#undef AGG
+}
+
+// Both levels, for groups whose values are already sorted and readable
+// through el.get(g, i).
+template <int NT, bool kG, typename Elems>
+__device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& el, double* dscr, double* red,
+                           SolveOut* out) {
+  __shared__ GroupPick pk;
+  solve_groups<NT, kG>(in, agg, T, red, &pk);
+  if (pk.status != ROW_CERTIFIED) {
+    if (threadIdx.x == 0) {
+      out->status = pk.status;
+      out->b = 0.0;
+      out->sumf = 0.0;
+      out->M = pk.M;
+      out->S_aL = pk.S_aL;
+      out->S_aR = pk.S_aR;
+    }
+    __syncthreads();
+    return;
+  }
+  if (pk.tg < 0) {
+    if (threadIdx.x == 0) solve_tail_interval(in, pk, out);
+    __syncthreads();
+    return;
+  }
+  struct One {
+    const Elems& e;
+    int g;
+    __device__ float get(int i) const { return e.get(g, i); }
+  };
+  solve_values<NT>(in, pk, ld<kG>(&agg[pk.tg].cnt), One{el, pk.tg}, dscr, red, out);
+}
+
+template <int NT>
+__device__ __forceinline__ uint32_t block_minmax_u32(uint32_t v, bool is_max, uint32_t* scratch) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = is_max ? __reduce_max_sync(0xffffffffu, v) : __reduce_min_sync(0xffffffffu, v);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  uint32_t t = (lane < NW) ? scratch[lane] : (is_max ? 0u : 0xFFFFFFFFu);
+  return is_max ? __reduce_max_sync(0xffffffffu, t) : __reduce_min_sync(0xffffffffu, t);
+}
+
+// Aggregates of one unsorted group whose values other blocks wrote to global
+// memory (so they are read around L1): count, min, max, and the anchored sums
+// P = sum exp((y - ymax)/alpha), Q = sum exp((ymin - y)/alpha).  Every term
+// lies in (0, 1]; the sums are taken in 2^-40 fixed point, which makes them
+// independent of the order in which the values arrived (run-to-run
+// determinism) at an absolute error below cnt * 2^-41.
+template <int NT>
+__device__ void aggregate_unsorted(const float* vals, int cnt, double inva, double* red, GroupAgg* out) {
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = threadIdx.x; i < cnt; i += NT) {
+    const uint32_t k = f2key(__ldcg(vals + i));
+    kmin = min(kmin, k);
+    kmax = max(kmax, k);
+  }
+  kmin = block_minmax_u32<NT>(kmin, false, reinterpret_cast<uint32_t*>(red));
+  kmax = block_minmax_u32<NT>(kmax, true, reinterpret_cast<uint32_t*>(red));
+  const double ymin = (double)key2f(kmin), ymax = (double)key2f(kmax);
+  long long P = 0, Q = 0;
+  for (int i = threadIdx.x; i < cnt; i += NT) {
+    const double y = (double)__ldcg(vals + i);
+    P += llrint(exp((y - ymax) * inva) * 0x1p40);
+    Q += llrint(exp((ymin - y) * inva) * 0x1p40);
+  }
+  P = block_sum<NT, long long>(P, reinterpret_cast<long long*>(red));
+  Q = block_sum<NT, long long>(Q, reinterpret_cast<long long*>(red));
+  if (threadIdx.x == 0) {
+    out->cnt = cnt;
+    out->ymin = cnt > 0 ? (float)ymin : 0.0f;
+    out->ymax = cnt > 0 ? (float)ymax : 0.0f;
+    out->P = (double)P * 0x1p-40;
+    out->Q = (double)Q * 0x1p-40;
+  }
+  __syncthreads();
 }
 
 // Aggregates of an already sorted run held as keys.

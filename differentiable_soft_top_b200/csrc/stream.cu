@@ -128,8 +128,12 @@ __device__ void flush_hist(const uint32_t* sh, uint32_t* gh, int nb) {
   __syncthreads();
 }
 
-// level 1 over keys already stored (recovery path)
-__device__ void sel_level1(const uint32_t* samp, int m, int cta, int ncta, uint32_t* gh1, uint32_t* sh) {
+// Radix select of the two bracket edges over the stored sample keys, 11, 11
+// and 10 bits per level.  Each level is a histogram of the keys that share the
+// prefix found so far; one block then finds, for both edges, the bin holding
+// the wanted rank and the rank left inside it (sel_pick).
+
+__device__ void sel_hist1(const uint32_t* samp, int m, int cta, int ncta, uint32_t* gh1, uint32_t* sh) {
   for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
   __syncthreads();
   for (int j0 = cta * NT; j0 < m; j0 += ncta * NT) {
@@ -141,12 +145,8 @@ __device__ void sel_level1(const uint32_t* samp, int m, int cta, int ncta, uint3
   flush_hist(sh, gh1, 2048);
 }
 
-__device__ void sel_level2(const uint32_t* samp, int m, int cta, int ncta, const uint32_t* gh1, uint32_t* gh2,
-                           const int rk[2], uint32_t* sh, uint32_t* scr) {
-  int b1[2];
-  uint32_t r1[2];
-  find_bin<2048>(gh1, (uint32_t)rk[0], scr, &b1[0], &r1[0]);
-  find_bin<2048>(gh1, (uint32_t)rk[1], scr, &b1[1], &r1[1]);
+__device__ void sel_hist2(const uint32_t* samp, int m, int cta, int ncta, const int b1[2], uint32_t* gh2,
+                          uint32_t* sh) {
   for (int i = threadIdx.x; i < 4096; i += NT) sh[i] = 0u;
   __syncthreads();
   for (int j0 = cta * NT; j0 < m; j0 += ncta * NT) {
@@ -160,16 +160,8 @@ __device__ void sel_level2(const uint32_t* samp, int m, int cta, int ncta, const
   flush_hist(sh, gh2, 4096);
 }
 
-__device__ void sel_level3(const uint32_t* samp, int m, int cta, int ncta, const uint32_t* gh1,
-                           const uint32_t* gh2, uint32_t* gh3, const int rk[2], uint32_t* sh, uint32_t* scr) {
-  uint32_t pre[2];
-  for (int t = 0; t < 2; ++t) {
-    int b1, b2;
-    uint32_t r1, r2;
-    find_bin<2048>(gh1, (uint32_t)rk[t], scr, &b1, &r1);
-    find_bin<2048>(gh2 + t * 2048, r1, scr, &b2, &r2);
-    pre[t] = ((uint32_t)b1 << 11) | (uint32_t)b2;
-  }
+__device__ void sel_hist3(const uint32_t* samp, int m, int cta, int ncta, const uint32_t pre[2], uint32_t* gh3,
+                          uint32_t* sh) {
   for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
   __syncthreads();
   for (int j0 = cta * NT; j0 < m; j0 += ncta * NT) {
@@ -183,17 +175,28 @@ __device__ void sel_level3(const uint32_t* samp, int m, int cta, int ncta, const
   flush_hist(sh, gh3, 2048);
 }
 
-// exact keys of the two order statistics
-__device__ void sel_final(const uint32_t* gh1, const uint32_t* gh2, const uint32_t* gh3, const int rk[2],
-                          uint32_t* scr, uint32_t keys[2]) {
-  for (int t = 0; t < 2; ++t) {
-    int b1, b2, b3;
-    uint32_t r1, r2, r3;
-    find_bin<2048>(gh1, (uint32_t)rk[t], scr, &b1, &r1);
-    find_bin<2048>(gh2 + t * 2048, r1, scr, &b2, &r2);
-    find_bin<1024>(gh3 + t * 1024, r2, scr, &b3, &r3);
-    keys[t] = ((uint32_t)b1 << 21) | ((uint32_t)b2 << 10) | (uint32_t)b3;
+// one level's pick for both edges (one block): the bin of histogram gh (the
+// edge's own histogram at gh + t*NB when per_edge) that holds rank rk[t], and
+// the rank left inside it
+template <int NB>
+__device__ void sel_pick(const uint32_t* gh, bool per_edge, const uint32_t rk[2], uint32_t* scr, int bin[2],
+                         uint32_t rem[2]) {
+  for (int t = 0; t < 2; ++t) find_bin<NB>(gh + (per_edge ? t * NB : 0), rk[t], scr, &bin[t], &rem[t]);
+}
+
+__device__ void store_pick(RowCtl* c, int level, const int bin[2], const uint32_t rem[2]) {
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      c->sel_bin[level][t] = bin[t];
+      c->sel_rem[level][t] = rem[t];
+    }
+    __threadfence();
   }
+  __syncthreads();
+}
+
+__device__ __forceinline__ uint32_t level3_prefix(const RowCtl* c, int t) {
+  return ((uint32_t)vld(&c->sel_bin[0][t]) << 11) | (uint32_t)vld(&c->sel_bin[1][t]);
 }
 
 // bracket and bucket plan for a row (one thread)
@@ -220,6 +223,7 @@ __device__ void write_plan(RowCtl* c, int m, const uint32_t keys[2], int rlo, in
 
 __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* __restrict__ scores) {
   __shared__ uint32_t sh[2048];
+  __shared__ uint32_t scr[64];
   const int64_t r = blockIdx.y;
   for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
   __syncthreads();
@@ -248,26 +252,45 @@ __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* 
     }
   }
   flush_hist(sh, h1_of(P, r), 2048);
+  RowCtl* c = ctl_of(P, r);
+  if (last_block_done(&c->done_s1, gridDim.x)) {
+    const uint32_t rk[2] = {(uint32_t)P.rank_lo, (uint32_t)P.rank_hi};
+    int bin[2];
+    uint32_t rem[2];
+    sel_pick<2048>(h1_of(P, r), false, rk, scr, bin, rem);
+    store_pick(c, 0, bin, rem);
+  }
 }
 
 __global__ void __launch_bounds__(NT) k_select2(const StreamPlan P) {
   __shared__ uint32_t sh[4096];
   __shared__ uint32_t scr[64];
   const int64_t r = blockIdx.y;
-  const int rk[2] = {P.rank_lo, P.rank_hi};
-  sel_level2(samp_of(P, r), P.m, blockIdx.x, gridDim.x, h1_of(P, r), h2_of(P, r), rk, sh, scr);
+  RowCtl* c = ctl_of(P, r);
+  const int b1[2] = {c->sel_bin[0][0], c->sel_bin[0][1]};
+  sel_hist2(samp_of(P, r), P.m, blockIdx.x, gridDim.x, b1, h2_of(P, r), sh);
+  if (last_block_done(&c->done_s2, gridDim.x)) {
+    const uint32_t rk[2] = {c->sel_rem[0][0], c->sel_rem[0][1]};
+    int bin[2];
+    uint32_t rem[2];
+    sel_pick<2048>(h2_of(P, r), true, rk, scr, bin, rem);
+    store_pick(c, 1, bin, rem);
+  }
 }
 
 __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
   __shared__ uint32_t sh[2048];
   __shared__ uint32_t scr[64];
   const int64_t r = blockIdx.y;
-  const int rk[2] = {P.rank_lo, P.rank_hi};
-  sel_level3(samp_of(P, r), P.m, blockIdx.x, gridDim.x, h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, sh, scr);
   RowCtl* c = ctl_of(P, r);
+  const uint32_t pre[2] = {level3_prefix(c, 0), level3_prefix(c, 1)};
+  sel_hist3(samp_of(P, r), P.m, blockIdx.x, gridDim.x, pre, h3_of(P, r), sh);
   if (last_block_done(&c->done_sel, gridDim.x)) {
-    uint32_t keys[2];
-    sel_final(h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, scr, keys);
+    const uint32_t rk[2] = {c->sel_rem[1][0], c->sel_rem[1][1]};
+    int bin[2];
+    uint32_t rem[2];
+    sel_pick<1024>(h3_of(P, r), true, rk, scr, bin, rem);
+    const uint32_t keys[2] = {(pre[0] << 10) | (uint32_t)bin[0], (pre[1] << 10) | (uint32_t)bin[1]};
     if (threadIdx.x == 0) write_plan(c, P.m, keys, P.rank_lo, P.rank_hi, P.valid_lo, P.valid_hi, P.T, P.C);
   }
 }
@@ -281,64 +304,71 @@ __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
 // buckets once per block at the end; a full stage spills to direct appends.
 constexpr int kStage = 3072;
 
+struct FilterCtx {
+  float aL, aR, lo, inv_w, c2;
+  int T, C;
+  uint32_t* cur;
+  float* band;
+  float* stage;
+  int* stage_n;
+};
+
+// append an in-band value to its value bucket
+__device__ __noinline__ void band_append(const FilterCtx& f, float x, uint32_t& ovf) {
+  const float tf = (x - f.lo) * f.inv_w;
+  const int t = (tf >= (float)f.T) ? f.T - 1 : (tf > 0.0f ? (int)tf : 0);
+  const uint32_t slot = atomicAdd(f.cur + t, 1u);
+  if (slot < (uint32_t)f.C) f.band[(int64_t)t * f.C + slot] = x;
+  else ovf = 1u;
+}
+
+// an in-band value met in the streaming loop: stage it (NaN and inf are
+// flagged instead)
+__device__ __forceinline__ void band_keep(const FilterCtx& f, float x, uint32_t& bad, uint32_t& ovf) {
+  if (!(fabsf(x) < CUDART_INF_F)) {
+    bad = 1u;
+    return;
+  }
+  const int pos = atomicAdd(f.stage_n, 1);
+  if (pos < kStage) f.stage[pos] = x;
+  else band_append(f, x, ovf);
+}
+
 __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
                              int ncta, double* red, float* stage, int* stage_n) {
-  const float aL = vld(&c->aL), aR = vld(&c->aR), lo = vld(&c->lo), inv_w = vld(&c->inv_w);
-  const int T = vld(&c->T), C = vld(&c->C);
-  const float c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
-  uint32_t* cur = cursor_of(P, r);
-  float* band = band_of(P, r);
+  FilterCtx f;
+  f.aL = vld(&c->aL);
+  f.aR = vld(&c->aR);
+  f.lo = vld(&c->lo);
+  f.inv_w = vld(&c->inv_w);
+  f.T = vld(&c->T);
+  f.C = vld(&c->C);
+  f.c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
+  f.cur = cursor_of(P, r);
+  f.band = band_of(P, r);
+  f.stage = stage;
+  f.stage_n = stage_n;
+  const float aL = f.aL, aR = f.aR, c2 = f.c2;
   long long nl = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u, ovf = 0u;
+  float amax = 0.0f;
   if (threadIdx.x == 0) *stage_n = 0;
   __syncthreads();
 
-  // an in-band value: append it to its value bucket
-  auto append = [&](float x) {
-    if (!(fabsf(x) < CUDART_INF_F)) {
-      bad = 1u;
-      return;
-    }
-    const float tf = (x - lo) * inv_w;
-    const int t = (tf >= (float)T) ? T - 1 : (tf > 0.0f ? (int)tf : 0);
-    const uint32_t slot = atomicAdd(cur + t, 1u);
-    if (slot < (uint32_t)C) band[(int64_t)t * C + slot] = x;
-    else ovf = 1u;
-  };
-  // an in-band value met in the streaming loop: stage it
-  auto keep = [&](float x) {
-    if (!(fabsf(x) < CUDART_INF_F)) {
-      bad = 1u;
-      return;
-    }
-    const int pos = atomicAdd(stage_n, 1);
-    if (pos < kStage) stage[pos] = x;
-    else append(x);
-  };
-  // one value, checked path
-  auto one = [&](float x) {
-    const bool isL = x < aL, isR = x >= aR;
-    const float e = exp2f(fminf(x - aL, aR - x) * c2);
-    if (isL) { sl += (double)e; ++nl; }
-    if (isR) sr += (double)e;
-    if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;
-    if (!(isL || isR)) keep(x);
-  };
-
   const int64_t n = P.n;
+  int64_t done = 0;
   if (P.vec) {
     const float4* x4 = reinterpret_cast<const float4*>(row);
-    const int64_t n4 = n >> 2;
-    const int64_t nchunks = n4 / CHUNK4;
+    const int64_t nchunks = (n >> 2) / CHUNK4;
     for (int64_t q = cta; q < nchunks; q += ncta) {
       const float4* base = x4 + q * CHUNK4 + threadIdx.x;
       float4 v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) v[u] = __ldg(base + u * NT);
-      float pl = 0.0f, pr = 0.0f;
+      float pl = 0.0f, pr = 0.0f, am = 0.0f;
       int cl = 0;
-      uint32_t anyin = 0u, bd = 0u;
+      uint32_t mask = 0u;  // bit 4u+w: value w of float4 u lies in the band
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -347,42 +377,42 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
           const float x = xs[w];
           const bool isL = x < aL, isR = x >= aR;
           const float e = exp2f(fminf(x - aL, aR - x) * c2);
-          if (isL) { pl += e; ++cl; }
-          if (isR) pr += e;
-          bd |= (fabsf(x) < CUDART_INF_F) ? 0u : 1u;
-          anyin |= (isL || isR) ? 0u : 1u;
+          pl += isL ? e : 0.0f;
+          pr += isR ? e : 0.0f;
+          cl += isL ? 1 : 0;
+          mask |= (isL || isR) ? 0u : (1u << (4 * u + w));
+          am = fmaxf(am, fabsf(x));
         }
       }
       sl += (double)pl;
       sr += (double)pr;
       nl += cl;
-      bad |= bd;
-      if (__any_sync(0xffffffffu, anyin)) {
-        if (anyin) {
-#pragma unroll
-          for (int u = 0; u < U; ++u) {
-            const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-              if (!(xs[w] < aL) && !(xs[w] >= aR)) keep(xs[w]);
-          }
-        }
+      amax = fmaxf(amax, am);
+      while (mask) {  // rare: walk only this lane's in-band values
+        const int i = __ffs(mask) - 1;
+        mask &= mask - 1u;
+        const float x = __ldg(reinterpret_cast<const float*>(base + (i >> 2) * NT) + (i & 3));
+        band_keep(f, x, bad, ovf);
       }
     }
-    for (int64_t i = nchunks * CHUNK4 + (int64_t)cta * NT + threadIdx.x; i < n4; i += (int64_t)ncta * NT) {
-      const float4 v = __ldg(x4 + i);
-      one(v.x);
-      one(v.y);
-      one(v.z);
-      one(v.w);
-    }
-    for (int64_t i = 4 * n4 + (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) one(row[i]);
-  } else {
-    for (int64_t i = (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) one(row[i]);
+    done = nchunks * CHUNK4 * 4;
   }
+  for (int64_t i = done + (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) {
+    const float x = row[i];
+    const bool isL = x < aL, isR = x >= aR;
+    const float e = exp2f(fminf(x - aL, aR - x) * c2);
+    if (isL) {
+      sl += (double)e;
+      ++nl;
+    }
+    if (isR) sr += (double)e;
+    amax = fmaxf(amax, fabsf(x));
+    if (!(isL || isR)) band_keep(f, x, bad, ovf);
+  }
+  if (!(amax < CUDART_INF_F)) bad = 1u;
   __syncthreads();
   const int ns = min(*stage_n, kStage);
-  for (int i = threadIdx.x; i < ns; i += NT) append(stage[i]);
+  for (int i = threadIdx.x; i < ns; i += NT) band_append(f, stage[i], ovf);
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
   nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
   sl = block_sum<NT, double>(sl, red);
@@ -409,13 +439,13 @@ __global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const floa
 }
 
 // ===========================================================================
-// band: bucket sorts and the certified solve (section 2.2, steps 3-4)
+// band: bucket aggregates, then the certified solve on the one bucket that
+// holds the root (section 2.2, steps 3-4)
 // ===========================================================================
 
-struct BandGroups {  // bucket g holds its sorted values at band + g*C
-  const float* band;
-  int C;
-  __device__ float get(int g, int i) const { return __ldcg(band + (int64_t)g * C + i); }
+struct KeyVals {  // sorted keys in shared memory
+  const uint32_t* k;
+  __device__ float get(int i) const { return key2f(k[i]); }
 };
 struct KeyGroupsG {  // consecutive groups of `g` sorted keys in global memory
   const uint32_t* k;
@@ -423,30 +453,44 @@ struct KeyGroupsG {  // consecutive groups of `g` sorted keys in global memory
   __device__ float get(int grp, int i) const { return key2f(__ldcg(k + (int64_t)grp * g + i)); }
 };
 
-__device__ void band_sort_phase(const StreamPlan& P, int64_t r, RowCtl* c, int cta, int ncta, uint32_t* kbuf,
-                                uint32_t* tbuf, uint32_t* hist, double* red) {
+// Shared-memory layout of the band kernels for buckets of up to C values:
+// keys and radix scratch (4C + 4C bytes), per-value prefix sums of the solve
+// (8C bytes), the radix histograms and the reduction scratch.
+struct BandSmem {
+  uint32_t* kbuf;
+  uint32_t* tbuf;
+  double* dscr;
+  uint32_t* hist;
+  double* red;
+  __device__ BandSmem(unsigned char* smem, int C) {
+    kbuf = reinterpret_cast<uint32_t*>(smem);
+    tbuf = kbuf + C;
+    dscr = reinterpret_cast<double*>(tbuf + C);
+    hist = reinterpret_cast<uint32_t*>(dscr + C);
+    red = reinterpret_cast<double*>(hist + SortScratch<NT>::kWords);
+  }
+  static constexpr size_t bytes(int C) { return (size_t)16 * C + (size_t)SortScratch<NT>::kWords * 4 + 64 * 8; }
+};
+
+// every bucket's count, extremes and anchored sums; no sorting
+__device__ void band_aggregate_phase(const StreamPlan& P, int64_t r, RowCtl* c, int cta, int ncta, double* red) {
   const int T = vld(&c->T), C = vld(&c->C);
   const double inva = 1.0 / P.alpha;
   const uint32_t* cur = cursor_of(P, r);
-  float* band = band_of(P, r);
+  const float* band = band_of(P, r);
   GroupAgg* ag = aggs_of(P, r);
   for (int t = cta; t < T; t += ncta) {
     const int cnt = (int)min(__ldcg(cur + t), (uint32_t)C);
-    float* vals = band + (int64_t)t * C;
-    __syncthreads();
-    for (int i = threadIdx.x; i < cnt; i += NT) kbuf[i] = f2key(__ldcg(vals + i));
-    __syncthreads();
-    const uint32_t* sorted = block_radix_sort<NT>(kbuf, tbuf, cnt, hist);
-    __syncthreads();
-    for (int i = threadIdx.x; i < cnt; i += NT) vals[i] = key2f(sorted[i]);
-    aggregate_sorted_keys<NT, false>(sorted, cnt, red, ag + t, inva);
+    aggregate_unsorted<NT>(band + (int64_t)t * C, cnt, inva, red, ag + t);
   }
 }
 
-// Reduces the filter partials and solves the row (one block).
-__device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int nparts, double* dscr,
-                                double* red) {
+// Reduces the filter partials, certifies the bracket, sorts the bucket that
+// holds the root and solves the row (one block).
+__device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int nparts, const BandSmem& sm) {
   __shared__ SolveOut so;
+  __shared__ GroupPick pk;
+  double* red = sm.red;
   const int T = vld(&c->T), C = vld(&c->C);
   const double inva = 1.0 / P.alpha;
   const FPart* parts = fpart_of(P, r);
@@ -478,10 +522,27 @@ __device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int n
     st |= ROW_FORCE_FB;
   } else {
     const SolveIn in{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, P.k, P.alpha, inva};
-    solve_band<NT, true>(in, aggs_of(P, r), T, BandGroups{band_of(P, r), C}, dscr, red, &so);
-    st |= so.status;
-    b = so.b;
-    sumf = so.sumf;
+    GroupAgg* ag = aggs_of(P, r);
+    solve_groups<NT, true>(in, ag, T, red, &pk);
+    if (pk.status != ROW_CERTIFIED) {
+      st |= pk.status;
+    } else {
+      if (pk.tg < 0) {
+        if (threadIdx.x == 0) solve_tail_interval(in, pk, &so);
+        __syncthreads();
+      } else {
+        const int cnt = __ldcg(&ag[pk.tg].cnt);
+        const float* vals = band_of(P, r) + (int64_t)pk.tg * C;
+        for (int i = threadIdx.x; i < cnt; i += NT) sm.kbuf[i] = f2key(__ldcg(vals + i));
+        __syncthreads();
+        const uint32_t* sorted = block_radix_sort<NT>(sm.kbuf, sm.tbuf, cnt, sm.hist);
+        __syncthreads();
+        solve_values<NT>(in, pk, cnt, KeyVals{sorted}, sm.dscr, red, &so);
+      }
+      st |= so.status;
+      b = so.b;
+      sumf = so.sumf;
+    }
   }
   if (threadIdx.x == 0) {
     c->sumf = sumf;
@@ -499,15 +560,11 @@ __device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int n
 
 __global__ void __launch_bounds__(NT) k_band(const StreamPlan P) {
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* kbuf = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* tbuf = kbuf + P.C;
-  uint32_t* hist = tbuf + P.C;
-  double* red = reinterpret_cast<double*>(hist + SortScratch<NT>::kWords);
-  double* dscr = reinterpret_cast<double*>(smem);  // C doubles over kbuf + tbuf
+  const BandSmem sm(smem, P.C);
   const int64_t r = blockIdx.y;
   RowCtl* c = ctl_of(P, r);
-  band_sort_phase(P, r, c, blockIdx.x, gridDim.x, kbuf, tbuf, hist, red);
-  if (last_block_done(&c->done_solve, gridDim.x)) band_solve_last(P, r, c, P.Gf, dscr, red);
+  band_aggregate_phase(P, r, c, blockIdx.x, gridDim.x, sm.red);
+  if (last_block_done(&c->done_solve, gridDim.x)) band_solve_last(P, r, c, P.Gf, sm);
 }
 
 // ===========================================================================
@@ -515,10 +572,7 @@ __global__ void __launch_bounds__(NT) k_band(const StreamPlan P) {
 // ===========================================================================
 
 struct RecSmem {
-  static constexpr size_t kKeys = 2 * (size_t)kBucketMax * 4;  // kbuf + tbuf; also dscr / selection hists
-  static constexpr size_t kHist = (size_t)SortScratch<NT>::kWords * 4;
-  static constexpr size_t kRed = 64 * 8;
-  static constexpr size_t kTotal = kKeys + kHist + kRed;
+  static constexpr size_t kTotal = BandSmem::bytes(kBucketMax);
 };
 
 // exclusive prefix over `cnt` entries of a global array, in place; returns the total
@@ -541,11 +595,12 @@ __device__ uint32_t block_scan_global_u32(uint32_t* a, int cnt, uint32_t* scr) {
 __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float* __restrict__ scores,
                                                  float* __restrict__ p_out) {
   extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* kbuf = reinterpret_cast<uint32_t*>(smem);
-  uint32_t* tbuf = kbuf + kBucketMax;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + RecSmem::kKeys);
-  double* red = reinterpret_cast<double*>(smem + RecSmem::kKeys + RecSmem::kHist);
-  double* dscr = reinterpret_cast<double*>(smem);
+  const BandSmem sm(smem, kBucketMax);
+  uint32_t* kbuf = sm.kbuf;
+  uint32_t* tbuf = sm.tbuf;
+  uint32_t* hist = sm.hist;
+  double* red = sm.red;
+  double* dscr = sm.dscr;
   uint32_t* sh = kbuf;  // selection histograms (4096 words)
   uint32_t* scr = reinterpret_cast<uint32_t*>(red);
   __shared__ SolveOut so;
@@ -584,23 +639,45 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         rhi += P.widen_delta; vhi = rhi <= P.m - 1;
         if (!vhi) rhi = P.m - 1;
       }
-      const int rk[2] = {rlo, rhi};
       int T, Cc;
       plan_buckets(P.n, P.m, rlo, rhi, P.T_max, P.band_cap, &T, &Cc);
       for (int i = cta * NT + threadIdx.x; i < 2048; i += ncta * NT) { h1_of(P, r)[i] = 0u; h3_of(P, r)[i] = 0u; }
       for (int i = cta * NT + threadIdx.x; i < 4096; i += ncta * NT) h2_of(P, r)[i] = 0u;
       for (int i = cta * NT + threadIdx.x; i < P.T_max; i += ncta * NT) cursor_of(P, r)[i] = 0u;
       REC_BARRIER();
-      sel_level1(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), sh);
-      REC_BARRIER();
-      sel_level2(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), h2_of(P, r), rk, sh, scr);
-      REC_BARRIER();
-      sel_level3(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, sh, scr);
+      sel_hist1(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), sh);
       REC_BARRIER();
       if (cta == 0) {
-        uint32_t keys[2];
-        sel_final(h1_of(P, r), h2_of(P, r), h3_of(P, r), rk, scr, keys);
+        const uint32_t rk[2] = {(uint32_t)rlo, (uint32_t)rhi};
+        int bin[2];
+        uint32_t rem[2];
+        sel_pick<2048>(h1_of(P, r), false, rk, scr, bin, rem);
+        store_pick(c, 0, bin, rem);
+      }
+      REC_BARRIER();
+      {
+        const int b1[2] = {vld(&c->sel_bin[0][0]), vld(&c->sel_bin[0][1])};
+        sel_hist2(samp_of(P, r), P.m, cta, ncta, b1, h2_of(P, r), sh);
+      }
+      REC_BARRIER();
+      if (cta == 0) {
+        const uint32_t rk[2] = {vld(&c->sel_rem[0][0]), vld(&c->sel_rem[0][1])};
+        int bin[2];
+        uint32_t rem[2];
+        sel_pick<2048>(h2_of(P, r), true, rk, scr, bin, rem);
+        store_pick(c, 1, bin, rem);
+      }
+      REC_BARRIER();
+      const uint32_t pre[2] = {level3_prefix(c, 0), level3_prefix(c, 1)};
+      sel_hist3(samp_of(P, r), P.m, cta, ncta, pre, h3_of(P, r), sh);
+      REC_BARRIER();
+      if (cta == 0) {
+        const uint32_t rk[2] = {vld(&c->sel_rem[1][0]), vld(&c->sel_rem[1][1])};
+        int bin[2];
+        uint32_t rem[2];
+        sel_pick<1024>(h3_of(P, r), true, rk, scr, bin, rem);
         if (threadIdx.x == 0) {
+          const uint32_t keys[2] = {(pre[0] << 10) | (uint32_t)bin[0], (pre[1] << 10) | (uint32_t)bin[1]};
           write_plan(c, P.m, keys, rlo, rhi, vlo, vhi, T, Cc);
           c->flags = 0u;
           c->status = ROW_WIDENED;
@@ -611,10 +688,10 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(tbuf),
                    reinterpret_cast<int*>(tbuf + kStage));
       REC_BARRIER();
-      band_sort_phase(P, r, c, cta, ncta, kbuf, tbuf, hist, red);
+      band_aggregate_phase(P, r, c, cta, ncta, red);
       REC_BARRIER();
       if (cta == 0) {
-        band_solve_last(P, r, c, ncta, dscr, red);
+        band_solve_last(P, r, c, ncta, sm);
         if (threadIdx.x == 0) {
           c->status |= ROW_WIDENED;
           __threadfence();
@@ -948,7 +1025,7 @@ __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
     o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
 }
 
-size_t band_smem(int C) { return (size_t)8 * C + (size_t)SortScratch<NT>::kWords * 4 + 64 * 8; }
+size_t band_smem(int C) { return BandSmem::bytes(C); }
 
 }  // namespace
 
