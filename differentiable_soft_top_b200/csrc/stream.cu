@@ -361,11 +361,22 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   if (P.vec) {
     const float4* x4 = reinterpret_cast<const float4*>(row);
     const int64_t nchunks = (n >> 2) / CHUNK4;
+    // two chunks in flight per thread: the next chunk's loads are issued
+    // before the current one is processed
+    float4 nx[U];
+    if (cta < nchunks) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) nx[u] = __ldg(x4 + (int64_t)cta * CHUNK4 + threadIdx.x + u * NT);
+    }
     for (int64_t q = cta; q < nchunks; q += ncta) {
       const float4* base = x4 + q * CHUNK4 + threadIdx.x;
       float4 v[U];
 #pragma unroll
-      for (int u = 0; u < U; ++u) v[u] = __ldg(base + u * NT);
+      for (int u = 0; u < U; ++u) v[u] = nx[u];
+      if (q + ncta < nchunks) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) nx[u] = __ldg(base + (int64_t)ncta * CHUNK4 + u * NT);
+      }
       float pl = 0.0f, pr = 0.0f, am = 0.0f;
       int cl = 0;
       uint32_t mask = 0u;  // bit 4u+w: value w of float4 u lies in the band
@@ -958,8 +969,9 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   BPart* part = reinterpret_cast<BPart*>(a.part) + r * kMaxGridPerRow;
   if (threadIdx.x == 0) part[blockIdx.x] = BPart{(double)m, S, SG, 0.0};
   if (last_block_done(a.done + r, gridDim.x)) {
-    double M = CUDART_INF;
-    for (int i = 0; i < (int)gridDim.x; ++i) M = fmin(M, __ldcg(&part[i].m));
+    float mloc = CUDART_INF_F;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) mloc = fminf(mloc, (float)__ldcg(&part[i].m));
+    const double M = (double)block_min_float<NT>(mloc, reinterpret_cast<float*>(red));
     double s = 0.0, sg = 0.0;
     for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
       const double pm = __ldcg(&part[i].m);
