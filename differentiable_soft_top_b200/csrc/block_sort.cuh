@@ -113,4 +113,30 @@ __device__ uint32_t* block_radix_sort(uint32_t* keys, uint32_t* tmp, int n, uint
   return keys;
 }
 
+// Sorts buf[0, n) ascending in place with a bitonic network over N = the next
+// power of two >= n; buf must hold N keys (entries n..N-1 are overwritten with
+// the largest key, which no finite value maps to).  Order-independent and
+// insensitive to ties; about log2(N)^2 / 2 barrier stages.
+template <int NT>
+__device__ void block_bitonic_sort(uint32_t* buf, int n) {
+  int N = 1;
+  while (N < n) N <<= 1;
+  for (int i = n + threadIdx.x; i < N; i += NT) buf[i] = 0xFFFFFFFFu;
+  __syncthreads();
+  for (int k = 2; k <= N; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < (N >> 1); i += NT) {
+        const int lo = ((i & ~(j - 1)) << 1) | (i & (j - 1));
+        const int hi = lo | j;
+        const uint32_t a = buf[lo], b = buf[hi];
+        if ((a > b) == ((lo & k) == 0)) {
+          buf[lo] = b;
+          buf[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 }  // namespace lapsum

@@ -191,11 +191,8 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   const ResLayout L = res_layout(a.n, a.m, a.bcap);
   float* row = reinterpret_cast<float*>(smem + L.row);
   uint32_t* samp = reinterpret_cast<uint32_t*>(smem + L.samp);
-  uint32_t* samp_tmp = reinterpret_cast<uint32_t*>(smem + L.samp_tmp);
   uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
-  uint32_t* band_tmp = reinterpret_cast<uint32_t*>(smem + L.band_tmp);
   double* dscr = reinterpret_cast<double*>(smem + L.dscr);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + L.hist);
   double* red = reinterpret_cast<double*>(smem + L.red);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
@@ -249,8 +246,8 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
     samp[j] = f2key(__double2float_rn(Y));
   }
   __syncthreads();
-  const uint32_t* ss = block_radix_sort<NT>(samp, samp_tmp, m, hist);
-  __syncthreads();
+  block_bitonic_sort<NT>(samp, m);  // samp and samp_tmp form one buffer of 2m keys
+  const uint32_t* ss = samp;
   int rlo = a.rank_lo, rhi = a.rank_hi;
   bool vlo = a.valid_lo != 0, vhi = a.valid_hi != 0;
   float aL = vlo ? key2f(ss[rlo]) : -CUDART_INF_F;
@@ -264,8 +261,8 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
       f = filter_row(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
-      const uint32_t* bs = block_radix_sort<NT>(band, band_tmp, f.M, hist);
-      __syncthreads();
+      block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
+      const uint32_t* bs = band;
       aggregate_sorted_keys<NT, false>(bs, f.M, red, &s_agg, inva);
       SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, a.k, a.alpha, inva};
       solve_band<NT, false>(in, &s_agg, 1, KeyRun{bs}, dscr, red, &s_out);

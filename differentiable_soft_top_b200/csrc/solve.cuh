@@ -54,6 +54,100 @@ __device__ __forceinline__ int block_min_int(int v, int* scratch) {
   return -block_max_int<NT>(-v, scratch);
 }
 
+// ---------------------------------------------------------------------------
+// Anchored sums as affine maps.  Along sorted values y_0 <= y_1 <= ..., the
+// prefix sum anchored at the latest value obeys A_i = A_{i-1} f_i + w_i with
+// the link factor f_i = exp((y_{i-1} - y_i)/alpha) <= 1, which depends only on
+// the values.  Each step is the map v -> v F + S; a run of steps composes to
+// one such map, and composition is associative, so the scan across threads is
+// FMA-only and every exp is independent of every other.  The suffix direction
+// is the same with the roles of left and right swapped.
+// ---------------------------------------------------------------------------
+struct Aff {
+  double F, S;  // v -> v * F + S
+};
+__device__ __forceinline__ Aff aff_id() { return Aff{1.0, 0.0}; }
+// apply a first, then b
+__device__ __forceinline__ Aff aff_then(Aff a, Aff b) { return Aff{a.F * b.F, fma(a.S, b.F, b.S)}; }
+
+// Block-wide exclusive scan of affine maps.  kForward: thread t receives the
+// composition of threads 0..t-1 (applied in that order); otherwise of threads
+// NT-1..t+1 (applied from the right).  scr: >= 2*NT/32 doubles.
+template <int NT, bool kForward>
+__device__ __forceinline__ Aff block_excl_scan_aff(Aff v, double* scr) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  Aff inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    Aff oth;
+    if (kForward) {
+      oth.F = __shfl_up_sync(0xffffffffu, inc.F, o);
+      oth.S = __shfl_up_sync(0xffffffffu, inc.S, o);
+      if (lane >= o) inc = aff_then(oth, inc);
+    } else {
+      oth.F = __shfl_down_sync(0xffffffffu, inc.F, o);
+      oth.S = __shfl_down_sync(0xffffffffu, inc.S, o);
+      if (lane + o < 32) inc = aff_then(oth, inc);
+    }
+  }
+  Aff exl;
+  if (kForward) {
+    exl.F = __shfl_up_sync(0xffffffffu, inc.F, 1);
+    exl.S = __shfl_up_sync(0xffffffffu, inc.S, 1);
+    if (lane == 0) exl = aff_id();
+  } else {
+    exl.F = __shfl_down_sync(0xffffffffu, inc.F, 1);
+    exl.S = __shfl_down_sync(0xffffffffu, inc.S, 1);
+    if (lane == 31) exl = aff_id();
+  }
+  __syncthreads();
+  if ((kForward && lane == 31) || (!kForward && lane == 0)) {
+    scr[2 * warp] = inc.F;
+    scr[2 * warp + 1] = inc.S;
+  }
+  __syncthreads();
+  Aff wacc = aff_id();
+  if (kForward) {
+    for (int w = 0; w < warp; ++w) wacc = aff_then(wacc, Aff{scr[2 * w], scr[2 * w + 1]});
+  } else {
+    for (int w = NW - 1; w > warp; --w) wacc = aff_then(wacc, Aff{scr[2 * w], scr[2 * w + 1]});
+  }
+  return aff_then(wacc, exl);
+}
+
+// block-wide exclusive scans of anchors: forward max (the last anchor before
+// a thread's chunk), backward min (the first anchor after it)
+template <int NT, bool kForward>
+__device__ __forceinline__ double block_excl_scan_anchor(double v, double init, double* scr) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  double inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double oth = kForward ? __shfl_up_sync(0xffffffffu, inc, o) : __shfl_down_sync(0xffffffffu, inc, o);
+    if (kForward ? (lane >= o) : (lane + o < 32)) inc = kForward ? fmax(inc, oth) : fmin(inc, oth);
+  }
+  double exl = kForward ? __shfl_up_sync(0xffffffffu, inc, 1) : __shfl_down_sync(0xffffffffu, inc, 1);
+  if (kForward ? lane == 0 : lane == 31) exl = init;
+  __syncthreads();
+  if (kForward ? lane == 31 : lane == 0) scr[warp] = inc;
+  __syncthreads();
+  double acc = init;
+  if (kForward) {
+    for (int w = 0; w < warp; ++w) acc = fmax(acc, scr[w]);
+    return fmax(acc, exl);
+  } else {
+    for (int w = NW - 1; w > warp; --w) acc = fmin(acc, scr[w]);
+    return fmin(acc, exl);
+  }
+}
+
+// link factor exp((from - to)/alpha) for from <= to; 0 when from = -inf (or to = +inf)
+__device__ __forceinline__ double link(double from, double to, double inva) {
+  return isfinite(from) && isfinite(to) ? exp((from - to) * inva) : 0.0;
+}
+
 // Result of the group-level step, shared by every thread of the block.
 struct GroupPick {
   uint32_t status;     // ROW_CERTIFIED (go on) or ROW_MISS_LEFT / ROW_MISS_RIGHT
@@ -77,74 +171,108 @@ __device__ void solve_groups(const SolveIn in, GroupAgg* agg, int T, double* red
   const double inva = in.inva;
   const int tid = threadIdx.x;
   __shared__ double s_dbl[8];
-  __shared__ long long s_ll[4];
+  __shared__ long long s_ll[2];
   int* iscr = reinterpret_cast<int*>(red);
   long long* lscr = reinterpret_cast<long long*>(red);
-
   const bool finL = isfinite(in.aL), finR = isfinite(in.aR);
-  const Anch left = (finL && in.SL > 0.0) ? Anch{(double)in.aL, in.SL} : anch_empty();
-  const Anch right = (finR && in.SR > 0.0) ? Anch{(double)in.aR, in.SR} : anch_empty();
+  const double xL = finL ? (double)in.aL : -CUDART_INF;
+  const double xR = finR ? (double)in.aR : CUDART_INF;
+  const double A0 = finL ? in.SL : 0.0;  // prefix state at a_L
+  const double B0 = finR ? in.SR : 0.0;  // suffix state at a_R
 
-  // prefix direction: A at each group maximum
   const int q = (T + NT - 1) / NT;
   const int t0 = min(T, tid * q), t1 = min(T, t0 + q);
-  Anch loc = anch_empty();
-  for (int t = t0; t < t1; ++t)
-    if (AGG(t, cnt) > 0) loc = comb_pre(loc, Anch{(double)AGG(t, ymax), AGG(t, P)}, inva);
-  Anch st = comb_pre(left, block_excl_scan_anch<NT, true>(loc, inva, red), inva);
+
+  // anchors: the last group maximum before the chunk, the first group minimum after it
+  double lastmax = -CUDART_INF, firstmin = CUDART_INF;
+  long long cloc = 0;
   for (int t = t0; t < t1; ++t) {
-    if (AGG(t, cnt) > 0) {
-      st = comb_pre(st, Anch{(double)AGG(t, ymax), AGG(t, P)}, inva);
-      agg[t].Apre = st.s;
+    const int c = AGG(t, cnt);
+    if (c > 0) {
+      lastmax = (double)AGG(t, ymax);
+      if (firstmin == CUDART_INF) firstmin = (double)AGG(t, ymin);
+      cloc += c;
     }
   }
-  if (tid == NT - 1) {  // prefix over everything below a_R
-    s_dbl[0] = st.x;
-    s_dbl[1] = st.s;
+  const double Xin = block_excl_scan_anchor<NT, true>(lastmax, xL, red);
+  const double Yin = block_excl_scan_anchor<NT, false>(firstmin, xR, red);
+  const long long cexc = block_excl_suffix_sum<NT>(cloc, lscr);
+
+  // forward: chunk map, scan, then A at every group maximum
+  Aff m = aff_id();
+  {
+    double X = Xin;
+    for (int t = t0; t < t1; ++t) {
+      if (AGG(t, cnt) > 0) {
+        const double ym = (double)AGG(t, ymax);
+        m = aff_then(m, Aff{link(X, ym, inva), AGG(t, P)});
+        X = ym;
+      }
+    }
+  }
+  const Aff fe = block_excl_scan_aff<NT, true>(m, red);
+  double A = fma(A0, fe.F, fe.S);  // prefix state at Xin
+  {
+    double X = Xin;
+    for (int t = t0; t < t1; ++t) {
+      if (AGG(t, cnt) > 0) {
+        const double ym = (double)AGG(t, ymax);
+        A = fma(A, link(X, ym, inva), AGG(t, P));
+        agg[t].Apre = A;
+        X = ym;
+      }
+    }
+    if (tid == NT - 1) {  // prefix over everything below a_R, anchored at X
+      s_dbl[0] = X;
+      s_dbl[1] = A;
+    }
   }
 
-  // suffix direction and the group knot values
-  Anch sloc = anch_empty();
-  long long cloc = 0;
-  for (int t = t1 - 1; t >= t0; --t) {
-    if (AGG(t, cnt) > 0) {
-      sloc = comb_suf(Anch{(double)AGG(t, ymin), AGG(t, Q)}, sloc, inva);
-      cloc += AGG(t, cnt);
+  // backward: chunk map, scan, suffix states, knot values
+  Aff mb = aff_id();
+  {
+    double Y = Yin;
+    for (int t = t1 - 1; t >= t0; --t) {
+      if (AGG(t, cnt) > 0) {
+        const double yn = (double)AGG(t, ymin);
+        mb = aff_then(mb, Aff{link(yn, Y, inva), AGG(t, Q)});
+        Y = yn;
+      }
     }
   }
-  const Anch sexc = block_excl_scan_anch<NT, false>(sloc, inva, red);
-  const long long cexc = block_excl_suffix_sum<NT>(cloc, lscr);
-  __syncthreads();
-  Anch ss = comb_suf(sexc, right, inva);
+  const Aff be = block_excl_scan_aff<NT, false>(mb, red);
+  double B = fma(B0, be.F, be.S);  // suffix state at Yin
   long long after = cexc + in.nR;
   int cand = -1;
-  for (int t = t1 - 1; t >= t0; --t) {
-    agg[t].Bx = ss.x;
-    agg[t].Bs = ss.s;
-    agg[t].after = after;
-    if (AGG(t, cnt) > 0) {
-      const double ymax = (double)AGG(t, ymax);
-      const double S = 0.5 * AGG(t, Apre) + (double)after - 0.5 * suf_at(ss, ymax, inva);
-      if (cand < 0 && S >= in.k) cand = t;
-      ss = comb_suf(Anch{(double)AGG(t, ymin), AGG(t, Q)}, ss, inva);
-      after += AGG(t, cnt);
+  {
+    double Y = Yin;
+    for (int t = t1 - 1; t >= t0; --t) {
+      agg[t].Bx = Y;
+      agg[t].Bs = B;
+      agg[t].after = after;
+      if (AGG(t, cnt) > 0) {
+        const double ym = (double)AGG(t, ymax), yn = (double)AGG(t, ymin);
+        const double S = 0.5 * AGG(t, Apre) + (double)after - 0.5 * B * link(ym, Y, inva);
+        if (cand < 0 && S >= in.k) cand = t;
+        B = fma(B, link(yn, Y, inva), AGG(t, Q));
+        Y = yn;
+        after += AGG(t, cnt);
+      }
     }
-  }
-  if (tid == 0) {  // suffix over everything at or above a_L
-    s_dbl[2] = ss.x;
-    s_dbl[3] = ss.s;
-    s_ll[0] = after;  // M + n_R
+    if (tid == 0) {  // suffix over everything at or above a_L, anchored at Y
+      s_dbl[2] = Y;
+      s_dbl[3] = B;
+      s_ll[0] = after;  // M + n_R
+    }
   }
   const int t_star = block_max_int<NT>(cand, iscr);
   __syncthreads();
 
   // certification (arXiv abstract: the bracket is proven, not trusted)
-  const Anch pre_all = Anch{s_dbl[0], s_dbl[1]};
-  const Anch suf_all = Anch{s_dbl[2], s_dbl[3]};
   const long long M = s_ll[0] - in.nR;
-  const double S_aL = finL ? 0.5 * in.SL + (double)(M + in.nR) - 0.5 * suf_at(suf_all, (double)in.aL, inva)
+  const double S_aL = finL ? 0.5 * in.SL + (double)(M + in.nR) - 0.5 * s_dbl[3] * link(xL, s_dbl[2], inva)
                            : CUDART_INF;
-  const double S_aR = finR ? 0.5 * pre_at(pre_all, (double)in.aR, inva) + (double)in.nR - 0.5 * in.SR
+  const double S_aR = finR ? 0.5 * s_dbl[1] * link(s_dbl[0], xR, inva) + (double)in.nR - 0.5 * in.SR
                            : -CUDART_INF;
   const bool cert = (S_aL >= in.k) && (S_aR < in.k);
 
@@ -162,17 +290,14 @@ __device__ void solve_groups(const SolveIn in, GroupAgg* agg, int T, double* red
     if (t_star >= 0) {
       pk->inc_x = (double)AGG(t_star, ymax);
       pk->inc_s = AGG(t_star, Apre);
-    } else if (finL) {
-      pk->inc_x = (double)in.aL;
-      pk->inc_s = in.SL;
     } else {
-      pk->inc_x = -CUDART_INF;
-      pk->inc_s = 0.0;
+      pk->inc_x = xL;
+      pk->inc_s = A0;
     }
     if (tg == INT32_MAX) {
       pk->tg = -1;
-      pk->out_x = finR ? (double)in.aR : CUDART_INF;
-      pk->out_s = finR ? in.SR : 0.0;
+      pk->out_x = xR;
+      pk->out_s = B0;
       pk->g_after = in.nR;
     } else {
       pk->tg = tg;
@@ -187,9 +312,8 @@ __device__ void solve_groups(const SolveIn in, GroupAgg* agg, int T, double* red
 
 // Root when no value lies above the last group knot: b in [x_in, a_R).
 __device__ inline void solve_tail_interval(const SolveIn& in, const GroupPick& pk, SolveOut* out) {
-  const double xj1 = isfinite(in.aR) ? (double)in.aR : CUDART_INF;
-  out->b = closed_form_root(pk.inc_x, xj1, pk.inc_s, pk.out_s, (double)pk.g_after, in.k, in.alpha);
-  out->sumf = sum_f_at(pk.inc_x, xj1, pk.inc_s, pk.out_s, out->b, in.inva);
+  out->b = closed_form_root(pk.inc_x, pk.out_x, pk.inc_s, pk.out_s, (double)pk.g_after, in.k, in.alpha);
+  out->sumf = sum_f_at(pk.inc_x, pk.out_x, pk.inc_s, pk.out_s, out->b, in.inva);
   out->status = ROW_CERTIFIED;
   out->M = pk.M;
   out->S_aL = pk.S_aL;
@@ -206,43 +330,74 @@ __device__ void solve_values(const SolveIn in, const GroupPick& pk, int c, const
   const int tid = threadIdx.x;
   __shared__ double s_bp;
   int* iscr = reinterpret_cast<int*>(red);
-  const Anch inc = Anch{pk.inc_x, pk.inc_s};
-  const Anch outg = Anch{pk.out_x, pk.out_s};
   const long long g_after = pk.g_after;
   const int qe = (c + NT - 1) / NT;
   const int i0 = min(c, tid * qe), i1 = min(c, i0 + qe);
-  Anch lp = anch_empty();
-  for (int i = i0; i < i1; ++i) lp = comb_pre(lp, Anch{(double)el.get(i), 1.0}, inva);
-  Anch ps = comb_pre(inc, block_excl_scan_anch<NT, true>(lp, inva, red), inva);
-  for (int i = i0; i < i1; ++i) {
-    ps = comb_pre(ps, Anch{(double)el.get(i), 1.0}, inva);
-    dscr[i] = ps.s;  // A_i anchored at y_i
+  const double xprev = (i0 > 0) ? (double)el.get(i0 - 1) : pk.inc_x;   // anchor before the chunk
+  const double xnext = (i1 < c) ? (double)el.get(i1) : pk.out_x;       // anchor after the chunk
+
+  // forward: A_i = A_{i-1} f_i + 1
+  Aff m = aff_id();
+  {
+    double X = xprev;
+    for (int i = i0; i < i1; ++i) {
+      const double y = (double)el.get(i);
+      m = aff_then(m, Aff{link(X, y, inva), 1.0});
+      X = y;
+    }
   }
-  Anch ls = anch_empty();
-  for (int i = i1 - 1; i >= i0; --i) ls = comb_suf(Anch{(double)el.get(i), 1.0}, ls, inva);
-  const Anch chunk_in = comb_suf(block_excl_scan_anch<NT, false>(ls, inva, red), outg, inva);
+  const Aff fe = block_excl_scan_aff<NT, true>(m, red);
+  {
+    double A = fma(pk.inc_s, fe.F, fe.S);  // prefix state at xprev
+    double X = xprev;
+    for (int i = i0; i < i1; ++i) {
+      const double y = (double)el.get(i);
+      A = fma(A, link(X, y, inva), 1.0);
+      dscr[i] = A;  // A_i anchored at y_i
+      X = y;
+    }
+  }
+  // backward: B'_i = B'_{i+1} g_i + 1 (values >= y_i, anchored at y_i)
+  Aff mb = aff_id();
+  {
+    double Y = xnext;
+    for (int i = i1 - 1; i >= i0; --i) {
+      const double y = (double)el.get(i);
+      mb = aff_then(mb, Aff{link(y, Y, inva), 1.0});
+      Y = y;
+    }
+  }
+  const Aff be = block_excl_scan_aff<NT, false>(mb, red);
+  const double Bin = fma(pk.out_s, be.F, be.S);  // suffix state at xnext
   __syncthreads();  // dscr complete
-  Anch sv = chunk_in;
   int icand = -1;
-  for (int i = i1 - 1; i >= i0; --i) {
-    const double y = (double)el.get(i);
-    const double S = 0.5 * dscr[i] + (double)((long long)(c - 1 - i) + g_after) - 0.5 * suf_at(sv, y, inva);
-    if (icand < 0 && S >= in.k) icand = i;
-    sv = comb_suf(Anch{y, 1.0}, sv, inva);
+  {
+    double B = Bin, Y = xnext;
+    for (int i = i1 - 1; i >= i0; --i) {
+      const double y = (double)el.get(i);
+      const double S = 0.5 * dscr[i] + (double)((long long)(c - 1 - i) + g_after) - 0.5 * B * link(y, Y, inva);
+      if (icand < 0 && S >= in.k) icand = i;
+      B = fma(B, link(y, Y, inva), 1.0);
+      Y = y;
+    }
   }
   const int i_star = block_max_int<NT>(icand, iscr);
   const int jn = i_star + 1;  // right knot index inside the group (c = beyond)
   if (jn < c && jn >= i0 && jn < i1) {
-    Anch w = chunk_in;
-    for (int i = i1 - 1; i >= jn; --i) w = comb_suf(Anch{(double)el.get(i), 1.0}, w, inva);
-    s_bp = w.s;  // B' at y_jn, anchored there
+    double B = Bin, Y = xnext;
+    for (int i = i1 - 1; i >= jn; --i) {
+      const double y = (double)el.get(i);
+      B = fma(B, link(y, Y, inva), 1.0);
+      Y = y;
+    }
+    s_bp = B;  // B' at y_jn, anchored there
   }
   __syncthreads();
   if (tid == 0) {
     double xj, A, xj1, Bp;
     if (i_star < 0) {
-      xj = inc.x;
-      A = inc.s;
+      xj = pk.inc_x;
+      A = pk.inc_s;
     } else {
       xj = (double)el.get(i_star);
       A = dscr[i_star];
@@ -251,8 +406,8 @@ __device__ void solve_values(const SolveIn in, const GroupPick& pk, int c, const
       xj1 = (double)el.get(jn);
       Bp = s_bp;
     } else {
-      xj1 = (outg.s > 0.0) ? outg.x : (isfinite(in.aR) ? (double)in.aR : CUDART_INF);
-      Bp = outg.s;
+      xj1 = pk.out_x;
+      Bp = pk.out_s;
     }
     const double cj = (double)((long long)(c - 1 - i_star) + g_after);
     out->b = closed_form_root(xj, xj1, A, Bp, cj, in.k, in.alpha);

@@ -299,18 +299,18 @@ __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
 // stream and filter (section 2.2, step 2)
 // ===========================================================================
 
-// In-band values are first staged in shared memory (a shared atomic per value,
-// no round trip to L2 inside the streaming loop) and appended to their global
-// buckets once per block at the end; a full stage spills to direct appends.
-constexpr int kStage = 3072;
+// In-band values never leave the streaming loop through global memory: a
+// lane holding some writes its chunk to a shared scratch slot and copies the
+// flagged values into its own column of a shared stage (no atomics, no global
+// reload); columns are appended to the global buckets once per block, or
+// earlier when one is about to fill.
+constexpr int kLaneStage = 24;  // stage column per lane (floats)
 
 struct FilterCtx {
   float aL, aR, lo, inv_w, c2;
   int T, C;
   uint32_t* cur;
   float* band;
-  float* stage;
-  int* stage_n;
 };
 
 // append an in-band value to its value bucket
@@ -322,20 +322,19 @@ __device__ __noinline__ void band_append(const FilterCtx& f, float x, uint32_t& 
   else ovf = 1u;
 }
 
-// an in-band value met in the streaming loop: stage it (NaN and inf are
-// flagged instead)
-__device__ __forceinline__ void band_keep(const FilterCtx& f, float x, uint32_t& bad, uint32_t& ovf) {
-  if (!(fabsf(x) < CUDART_INF_F)) {
-    bad = 1u;
-    return;
+// empty this lane's stage column into the global buckets (NaN and inf are
+// flagged instead of appended)
+__device__ __noinline__ void flush_column(const FilterCtx& f, const float* col, int cnt, uint32_t& bad,
+                                          uint32_t& ovf) {
+  for (int j = 0; j < cnt; ++j) {
+    const float x = col[j * NT];
+    if (fabsf(x) < CUDART_INF_F) band_append(f, x, ovf);
+    else bad = 1u;
   }
-  const int pos = atomicAdd(f.stage_n, 1);
-  if (pos < kStage) f.stage[pos] = x;
-  else band_append(f, x, ovf);
 }
 
 __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
-                             int ncta, double* red, float* stage, int* stage_n) {
+                             int ncta, double* red, float* stage) {
   FilterCtx f;
   f.aL = vld(&c->aL);
   f.aR = vld(&c->aR);
@@ -346,15 +345,14 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   f.c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
   f.cur = cursor_of(P, r);
   f.band = band_of(P, r);
-  f.stage = stage;
-  f.stage_n = stage_n;
   const float aL = f.aL, aR = f.aR, c2 = f.c2;
+  float* col = stage + threadIdx.x;                             // this lane's column, stride NT
+  float4* scratch = reinterpret_cast<float4*>(stage + kLaneStage * NT) + threadIdx.x * U;  // U float4
+  int ncol = 0;
   long long nl = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u, ovf = 0u;
   float amax = 0.0f;
-  if (threadIdx.x == 0) *stage_n = 0;
-  __syncthreads();
 
   const int64_t n = P.n;
   int64_t done = 0;
@@ -399,11 +397,20 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
       sr += (double)pr;
       nl += cl;
       amax = fmaxf(amax, am);
-      while (mask) {  // rare: walk only this lane's in-band values
-        const int i = __ffs(mask) - 1;
-        mask &= mask - 1u;
-        const float x = __ldg(reinterpret_cast<const float*>(base + (i >> 2) * NT) + (i & 3));
-        band_keep(f, x, bad, ovf);
+      if (mask) {  // rare: copy this lane's in-band values into its column
+#pragma unroll
+        for (int u = 0; u < U; ++u) scratch[u] = v[u];
+        const float* sv = reinterpret_cast<const float*>(scratch);
+        do {
+          const int i = __ffs(mask) - 1;
+          mask &= mask - 1u;
+          col[ncol * NT] = sv[i];
+          ++ncol;
+        } while (mask);
+        if (ncol > kLaneStage - 4 * U) {
+          flush_column(f, col, ncol, bad, ovf);
+          ncol = 0;
+        }
       }
     }
     done = nchunks * CHUNK4 * 4;
@@ -418,12 +425,16 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
     }
     if (isR) sr += (double)e;
     amax = fmaxf(amax, fabsf(x));
-    if (!(isL || isR)) band_keep(f, x, bad, ovf);
+    if (!(isL || isR)) {
+      col[ncol * NT] = x;
+      if (++ncol == kLaneStage) {
+        flush_column(f, col, ncol, bad, ovf);
+        ncol = 0;
+      }
+    }
   }
+  flush_column(f, col, ncol, bad, ovf);
   if (!(amax < CUDART_INF_F)) bad = 1u;
-  __syncthreads();
-  const int ns = min(*stage_n, kStage);
-  for (int i = threadIdx.x; i < ns; i += NT) band_append(f, stage[i], ovf);
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
   nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
   sl = block_sum<NT, double>(sl, red);
@@ -441,12 +452,14 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   __syncthreads();
 }
 
+// shared memory of the filter pass: lane columns plus one scratch chunk per lane
+constexpr size_t kFilterStageBytes = (size_t)(kLaneStage * NT) * 4 + (size_t)NT * U * 16;
+
 __global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const float* __restrict__ scores) {
   __shared__ double red[64];
-  __shared__ float stage[kStage];
-  __shared__ int stage_n;
+  __shared__ __align__(16) float stage[kFilterStageBytes / 4];
   const int64_t r = blockIdx.y;
-  filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red, stage, &stage_n);
+  filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red, stage);
 }
 
 // ===========================================================================
@@ -546,9 +559,8 @@ __device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int n
         const float* vals = band_of(P, r) + (int64_t)pk.tg * C;
         for (int i = threadIdx.x; i < cnt; i += NT) sm.kbuf[i] = f2key(__ldcg(vals + i));
         __syncthreads();
-        const uint32_t* sorted = block_radix_sort<NT>(sm.kbuf, sm.tbuf, cnt, sm.hist);
-        __syncthreads();
-        solve_values<NT>(in, pk, cnt, KeyVals{sorted}, sm.dscr, red, &so);
+        block_bitonic_sort<NT>(sm.kbuf, cnt);  // kbuf and tbuf form one buffer of 2C keys
+        solve_values<NT>(in, pk, cnt, KeyVals{sm.kbuf}, sm.dscr, red, &so);
       }
       st |= so.status;
       b = so.b;
@@ -696,8 +708,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         }
       }
       REC_BARRIER();
-      filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(tbuf),
-                   reinterpret_cast<int*>(tbuf + kStage));
+      filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(kbuf));
       REC_BARRIER();
       band_aggregate_phase(P, r, c, cta, ncta, red);
       REC_BARRIER();
