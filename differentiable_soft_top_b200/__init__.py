@@ -35,7 +35,8 @@ __all__ = [
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "liblapsum_topk.so")
 
-LAPSUM_OK, LAPSUM_EINVAL, LAPSUM_EBADK, LAPSUM_EBADALPHA, LAPSUM_EWORKSPACE, LAPSUM_ECUDA = range(6)
+LAPSUM_OK, LAPSUM_EINVAL, LAPSUM_EBADK, LAPSUM_EBADALPHA, LAPSUM_EWORKSPACE, LAPSUM_ECUDA, LAPSUM_ETOOLARGE = range(7)
+NOALLOC_MAX_ROWS, NOALLOC_MAX_N = 65536, 16384  # limits of forward_noalloc_into
 ROW_CERTIFIED, ROW_WIDENED, ROW_FALLBACK = 0x01, 0x02, 0x04
 ROW_NONFINITE, ROW_TIMEOUT, ROW_OVERFLOW = 0x08, 0x10, 0x20
 FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
@@ -117,6 +118,8 @@ def _load():
             lib.lapsum_topk_fwd.restype = ctypes.c_int
             lib.lapsum_topk_bwd.argtypes = [P, P, P, i64, i64, i64, dbl, P, P, P, sz, P]
             lib.lapsum_topk_bwd.restype = ctypes.c_int
+            lib.lapsum_topk_fwd_noalloc.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, P]
+            lib.lapsum_topk_fwd_noalloc.restype = ctypes.c_int
             lib.lapsum_status_string.argtypes = [ctypes.c_int]
             lib.lapsum_status_string.restype = ctypes.c_char_p
             lib.lapsum_last_cuda_error.argtypes = []
@@ -297,6 +300,28 @@ def forward_into(scores, k: float, alpha: float, p, b, sumf, status, workspace, 
                              workspace.numel(), pptr, torch.cuda.current_stream(scores.device).cuda_stream)
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_fwd")
+
+
+def forward_noalloc_into(scores, k: float, alpha: float, p, b, sumf=None, status=None,
+                         params: Params | None = None, stats=None) -> None:
+    """forward_into() without a workspace, for callers that cannot allocate
+    device memory during the call (a fixed arena, a fully reserved pool, no
+    implicit synchronisation allowed).  Rows of at most NOALLOC_MAX_N scores,
+    at most NOALLOC_MAX_ROWS rows.  Its scratch is one static device array
+    inside the library, shared by all calls on a device: calls that overlap on
+    the GPU race, so serialise them."""
+    torch = _torch()
+    lib = _load()
+    rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
+    stride = scores.stride(0) if scores.dim() == 2 else n
+    c, pptr = _params_ptr(params)
+    rc = lib.lapsum_topk_fwd_noalloc(scores.data_ptr(), rows, n, stride, float(k), float(alpha), p.data_ptr(),
+                                     b.data_ptr(), sumf.data_ptr() if sumf is not None else None,
+                                     status.data_ptr() if status is not None else None,
+                                     stats.data_ptr() if stats is not None else None, pptr,
+                                     torch.cuda.current_stream(scores.device).cuda_stream)
+    if rc != LAPSUM_OK:
+        raise LapsumError(rc, "lapsum_topk_fwd_noalloc")
 
 
 def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None) -> None:

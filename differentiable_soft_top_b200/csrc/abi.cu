@@ -229,6 +229,7 @@ const char* lapsum_status_string(int code) {
     case LAPSUM_EBADALPHA: return "alpha must be finite and in [1e-30, 1e30]";
     case LAPSUM_EWORKSPACE: return "workspace missing or smaller than lapsum_topk_workspace_size()";
     case LAPSUM_ECUDA: return "a CUDA call or kernel launch failed";
+    case LAPSUM_ETOOLARGE: return "rows > LAPSUM_NOALLOC_MAX_ROWS or n > LAPSUM_NOALLOC_MAX_N for the allocation-free forward";
     default: return "unknown status";
   }
 }
@@ -392,3 +393,106 @@ int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, i
 }
 
 }  // extern "C"
+
+// ---- allocation-free forward --------------------------------------------
+// Some callers cannot allocate device memory at the moment they run the
+// operator: an inference engine that hands each plugin a fixed arena, a host
+// that has reserved all device memory for its own pool, or a framework that
+// must not synchronise (cudaMalloc may) in the middle of a step.  For rows
+// that one block holds (n <= 16384), the forward needs only 8 bytes of
+// scratch per row and one counter, so that scratch can live in a static
+// device array that the library owns.  The paper has no counterpart to this.
+
+// (2 * 256 KiB + 256 bytes: row statuses, the fallback counter, the fallback
+// row list for LAPSUM_NOALLOC_MAX_ROWS rows.)  Every GPU that loads the
+// library holds it until the process exits.  It is shared by every call on a
+// device and keeps the last call's contents; the only word that must start at
+// zero (the fallback row counter) is cleared on the caller's stream by each
+// call before the kernels that read it.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[2 * 4 * LAPSUM_NOALLOC_MAX_ROWS + 256];
+
+namespace lapsum {
+namespace {
+
+constexpr int64_t kNoAllocMaxRows = LAPSUM_NOALLOC_MAX_ROWS;
+constexpr size_t kNoAllocBytes = sizeof(g_noalloc_scratch);
+static_assert(4 * LAPSUM_NOALLOC_MAX_ROWS % 256 == 0, "row arrays must keep 256-byte alignment");
+static_assert(LAPSUM_NOALLOC_MAX_N == kResidentMaxN, "the allocation-free forward is the one-block-per-row path");
+
+unsigned char* g_noalloc_ptr[kMaxDevices];  // device address of the array, per device
+
+// The array's device address on the current device, looked up on the first
+// call there (in host code the symbol is only a stand-in, not an address).
+cudaError_t noalloc_scratch(unsigned char** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace lapsum
+
+extern "C" int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k,
+                                       double alpha, float* p_out, double* b_out, double* sumf_out,
+                                       uint32_t* row_status, lapsum_row_stats* stats, const lapsum_params* params,
+                                       void* stream) {
+  if (!scores || !p_out || !b_out) return LAPSUM_EINVAL;
+  if (rows < 1 || n < 1 || row_stride < n) return LAPSUM_EINVAL;
+  if (rows > kNoAllocMaxRows || n > LAPSUM_NOALLOC_MAX_N) return LAPSUM_ETOOLARGE;
+  if (((uintptr_t)scores & 3u) || ((uintptr_t)p_out & 3u) || ((uintptr_t)b_out & 7u)) return LAPSUM_EINVAL;
+  if (sumf_out && ((uintptr_t)sumf_out & 7u)) return LAPSUM_EINVAL;
+  if (!std::isfinite(k) || !(k > 0.0) || !(k < (double)n)) return LAPSUM_EBADK;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
+  if (overlaps(scores, span, p_out, span)) return LAPSUM_EINVAL;
+  const Resolved R = resolve(params);
+  if (!resident_path(n, R)) return LAPSUM_EINVAL;  // LAPSUM_FORCE_STREAMING is not available here
+  DevInfo* dev = nullptr;
+  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
+  unsigned char* ws = nullptr;
+  if (!cuda_ok(noalloc_scratch(&ws))) return LAPSUM_ECUDA;
+
+  const ResPlan rp = resident_plan(n, k, R);
+  ResidentFwd a{};
+  a.scores = scores;
+  a.rows = rows;
+  a.n = n;
+  a.stride = row_stride;
+  a.k = k;
+  a.alpha = alpha;
+  a.p_out = p_out;
+  a.b_out = b_out;
+  a.sumf_out = sumf_out;
+  a.status_out = row_status;
+  a.stats = stats;
+  a.m = rp.m;
+  a.rank_lo = rp.rk.rank_lo;
+  a.rank_hi = rp.rk.rank_hi;
+  a.valid_lo = rp.rk.valid_lo;
+  a.valid_hi = rp.rk.valid_hi;
+  a.widen_delta = rp.rk.widen_delta;
+  a.max_widen = R.max_widen;
+  a.bcap = rp.bcap;
+  a.seed = R.seed;
+  a.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+  a.vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  // same layout as the caller-workspace forward: statuses, counter, row list
+  const size_t list_off = align256(4 * (size_t)rows);
+  if (2 * list_off + 256 > kNoAllocBytes) return LAPSUM_ETOOLARGE;
+  a.ws_status = reinterpret_cast<uint32_t*>(ws);
+  a.fb_count = reinterpret_cast<uint32_t*>(ws + list_off);
+  a.fb_list = reinterpret_cast<int32_t*>(ws + list_off + 256);
+  if (resident_fwd_smem(a) + 1024 > (size_t)dev->smem_optin) return LAPSUM_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return cuda_ok(launch_resident_fwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
+}

@@ -23,7 +23,8 @@
  *
  * Conventions for every entry point:
  *   - All array pointers are DEVICE pointers owned by the caller.  The library
- *     allocates no memory: scratch space is the caller's `workspace`.
+ *     allocates no memory: scratch space is the caller's `workspace` (or,
+ *     for lapsum_topk_fwd_noalloc, a static array inside the library).
  *   - Scores are fp32, `rows` rows of `n` values, row i starting at
  *     scores + i * row_stride (row-major when row_stride == n).  Outputs use
  *     the same layout.  Outputs may not overlap inputs.
@@ -62,6 +63,8 @@ extern "C" {
 #define LAPSUM_EBADALPHA 3    /* alpha not finite or outside [1e-30, 1e30] */
 #define LAPSUM_EWORKSPACE 4   /* workspace NULL or smaller than required */
 #define LAPSUM_ECUDA 5        /* a CUDA call or launch failed */
+#define LAPSUM_ETOOLARGE 6    /* rows or n above the limits of
+                                 lapsum_topk_fwd_noalloc */
 
 /* ---- per-row status bits (asynchronous, in row_status) ---------------- */
 #define LAPSUM_ROW_CERTIFIED 0x01u  /* b proven inside the final bracket */
@@ -158,6 +161,37 @@ LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int
 LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows,
                                int64_t n, int64_t row_stride, double alpha, float* grad_scores,
                                double* grad_k, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Forward pass that allocates nothing and takes no workspace.  The paper has
+ * no counterpart: this entry point exists for callers that cannot allocate
+ * device memory when they run the operator -- an inference engine whose
+ * plugins get a fixed arena, a host that has reserved all device memory for
+ * its own pool, or a framework that must not risk the implicit
+ * synchronisation of cudaMalloc in the middle of a step.
+ *
+ * Arguments, results and per-row status are those of lapsum_topk_fwd, for
+ * the one-block-per-row path only:
+ *   rows <= LAPSUM_NOALLOC_MAX_ROWS and n <= LAPSUM_NOALLOC_MAX_N, else
+ *   LAPSUM_ETOOLARGE (nothing enqueued); LAPSUM_FORCE_STREAMING in params is
+ *   rejected with LAPSUM_EINVAL.
+ * Scratch: a static device array of 2 * 4 * LAPSUM_NOALLOC_MAX_ROWS + 256
+ * bytes (512.25 KiB) inside the library, which every GPU that loads the
+ * library holds until the process exits.  It is shared by all calls on a
+ * device and keeps the last call's contents; each call clears what must start
+ * at zero on its own stream.  Calls that overlap on the GPU (two streams, or
+ * two host threads) race on that array and may return wrong results:
+ * serialise them.
+ * The first call on a device looks up the array's device address and sets
+ * kernel attributes; make it before any stream capture on that device.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define LAPSUM_NOALLOC_MAX_ROWS 65536
+#define LAPSUM_NOALLOC_MAX_N 16384
+LAPSUM_API int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                                       double k, double alpha, float* p_out, double* b_out,
+                                       double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
+                                       const lapsum_params* params, void* stream);
 
 /* Text of the CUDA error behind the last LAPSUM_ECUDA returned on the
    calling host thread ("no error" if none). */

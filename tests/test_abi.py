@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     assert names == sorted([
         "lapsum_default_params", "lapsum_last_cuda_error", "lapsum_launch_count", "lapsum_status_string",
-        "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_workspace_size",
+        "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc", "lapsum_topk_workspace_size",
         "lapsum_trace_collect", "lapsum_trace_enable",
     ])
 
@@ -59,7 +59,7 @@ def test_trace_collect_without_launches(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert len(lt.status_string(code)) >= 2 and lt.status_string(code) != "unknown status"
     assert lt.status_string(99) == "unknown status"
 
