@@ -23,7 +23,7 @@ struct DevInfo {
   bool ready = false;
   int sm_count = 0;
   int smem_optin = 0;  // bytes of shared memory a block may opt in to
-  StreamOcc occ{};     // for C = kBucketMax
+  StreamOcc occ{};
 };
 DevInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -43,7 +43,7 @@ cudaError_t device_info(DevInfo** out) {
       if (e != cudaSuccess) return e;
       e = resident_init(d->smem_optin);
       if (e != cudaSuccess) return e;
-      e = stream_occupancy(kBucketMax, &d->occ);
+      e = stream_occupancy(&d->occ);
       if (e != cudaSuccess) return e;
       d->ready = true;
     }
@@ -136,7 +136,7 @@ ResPlan resident_plan(int64_t n, double k, const Resolved& R) {
 struct StreamSizes {
   int m;
   Ranks rk;
-  int T, C, T_max;
+  double M_est;  // expected band size
   int64_t band_cap;
 };
 StreamSizes stream_sizes(int64_t n, double k, const Resolved& R) {
@@ -144,19 +144,17 @@ StreamSizes stream_sizes(int64_t n, double k, const Resolved& R) {
   s.m = R.m_user ? (int)std::min<uint32_t>(R.m_user, 1u << 20)
                  : (int)std::min<int64_t>(1 << 17, std::max<int64_t>(2048, round_up(n / 8, 1024)));
   s.rk = sample_ranks(n, k, s.m, R.z);
-  const double M_est = (double)(s.rk.rank_hi - s.rk.rank_lo + 1) * (double)n / (double)s.m;
-  // default capacity: four times the expected band plus slack, so a bucket
-  // holds about 4x its expected count (overflow sends the row to the fallback)
-  int64_t cap = R.bcap_user > 0 ? R.bcap_user : (int64_t)(4.0 * M_est) + 16384;
+  s.M_est = (double)(s.rk.rank_hi - s.rk.rank_lo + 1) * (double)n / (double)s.m;
+  // default capacity: four times the expected band plus slack (overflow sends
+  // the row to the fallback)
+  int64_t cap = R.bcap_user > 0 ? R.bcap_user : (int64_t)(4.0 * s.M_est) + 16384;
   cap = std::max<int64_t>(R.bcap_user > 0 ? 4 : 1024, std::min<int64_t>(cap, (int64_t)round_up(n, 1024)));
   s.band_cap = round_up(cap, 4);
-  s.T_max = (int)std::max<int64_t>(1, std::min<int64_t>(4096, s.band_cap / 1024));
-  plan_buckets(n, s.m, s.rk.rank_lo, s.rk.rank_hi, s.T_max, s.band_cap, &s.T, &s.C);
   return s;
 }
 
 struct StreamLayout {
-  size_t ctl, h1, h2, h3, cursor, zero_end, samp, fpart, band, aggs, mpart, fb_keys, fb_aggs, rcount, total;
+  size_t ctl, h1, h2, h3, zero_end, samp, fpart, band, mpart, fb_keys, fb_aggs, rcount, total;
 };
 StreamLayout stream_layout(int64_t rows, int64_t n, const StreamSizes& s) {
   StreamLayout L;
@@ -165,12 +163,10 @@ StreamLayout stream_layout(int64_t rows, int64_t n, const StreamSizes& s) {
   L.h1 = o;      o = align256(o + 4 * 2048 * (size_t)rows);
   L.h2 = o;      o = align256(o + 4 * 4096 * (size_t)rows);
   L.h3 = o;      o = align256(o + 4 * 2048 * (size_t)rows);
-  L.cursor = o;  o = align256(o + 4 * (size_t)s.T_max * (size_t)rows);
   L.zero_end = o;
   L.samp = o;    o = align256(o + 4 * (size_t)s.m * (size_t)rows);
   L.fpart = o;   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
   L.band = o;    o = align256(o + 4 * (size_t)s.band_cap * (size_t)rows);
-  L.aggs = o;    o = align256(o + sizeof(GroupAgg) * (size_t)s.T_max * (size_t)rows);
   L.mpart = o;   o = align256(o + 16 * (size_t)kMaxGridPerRow * (size_t)rows);
   L.fb_keys = o; o = align256(o + 4 * (size_t)n);
   L.fb_aggs = o; o = align256(o + sizeof(GroupAgg) * (size_t)(n / kFallbackGroup + 2));
@@ -300,8 +296,7 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
 
   const StreamSizes s = stream_sizes(n, k, R);
   const StreamLayout L = stream_layout(rows, n, s);
-  StreamOcc occ{};
-  if (!cuda_ok(stream_occupancy(s.C, &occ))) return LAPSUM_ECUDA;
+  const StreamOcc& occ = dev->occ;
   StreamPlan P{};
   P.rows = rows;
   P.n = n;
@@ -315,9 +310,6 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
   P.valid_hi = s.rk.valid_hi;
   P.widen_delta = s.rk.widen_delta;
   P.max_widen = R.max_widen;
-  P.T = s.T;
-  P.C = s.C;
-  P.T_max = s.T_max;
   P.band_cap = s.band_cap;
   P.seed = R.seed;
   P.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
@@ -326,18 +318,20 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
   P.Gs = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (s.m + 1023) / 1024));
   P.Gf = stream_grid(sm, occ.filter_blocks, rows, n);
   P.Gm = stream_grid(sm, occ.memb_blocks, rows, n);
-  P.G3 = (int)std::max<int64_t>(1, std::min<int64_t>((int64_t)s.T, std::max<int64_t>(1, (int64_t)sm * occ.band_blocks / rows)));
   P.Gr = std::min(kMaxGridPerRow, sm * occ.recover_blocks);
+  // band cluster: about kBandValuesPerCta expected band values per CTA
+  // (with more than one CTA the leader holds no slice)
+  int cs = 1;
+  while (cs < occ.band_max_cluster && (double)(cs > 1 ? cs - 1 : 1) * kBandValuesPerCta < s.M_est) cs <<= 1;
+  P.band_cs = cs;
   P.ctl = ws + L.ctl;
   P.zero_bytes = L.zero_end - L.ctl;
   P.hist1 = reinterpret_cast<uint32_t*>(ws + L.h1);
   P.hist2 = reinterpret_cast<uint32_t*>(ws + L.h2);
   P.hist3 = reinterpret_cast<uint32_t*>(ws + L.h3);
-  P.cursor = reinterpret_cast<uint32_t*>(ws + L.cursor);
   P.samp = reinterpret_cast<uint32_t*>(ws + L.samp);
   P.fpart = ws + L.fpart;
   P.band = reinterpret_cast<float*>(ws + L.band);
-  P.aggs = ws + L.aggs;
   P.mpart = ws + L.mpart;
   P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
   P.fb_aggs = ws + L.fb_aggs;

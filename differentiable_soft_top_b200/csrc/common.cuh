@@ -25,6 +25,7 @@ constexpr uint32_t ROW_PUBLIC = 0xFFu;
 constexpr uint32_t ROW_MISS_LEFT = 0x100u;   // S(a_L) < k: b lies below a_L
 constexpr uint32_t ROW_MISS_RIGHT = 0x200u;  // S(a_R) >= k: b lies at or above a_R
 constexpr uint32_t ROW_FORCE_FB = 0x400u;    // test knob: take the full sort
+constexpr uint32_t ROW_PENDING = 0x800u;     // band solved up to its last step, left to the final kernel
 constexpr uint32_t ROW_NEEDS_RECOVERY = ROW_MISS_LEFT | ROW_MISS_RIGHT | ROW_OVERFLOW | ROW_FORCE_FB;
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -91,8 +92,10 @@ __host__ __device__ __forceinline__ float key2f(uint32_t k) {
 struct alignas(256) RowCtl {
   // bracket and band plan, written by the selection step
   float aL, aR;        // bracket [aL, aR); -inf / +inf when open
-  float lo, inv_w;     // band bucket of x: floor((x - lo) * inv_w), clamped
-  int32_t T, C;        // buckets and slots per bucket
+  uint32_t band_cnt;   // band values appended by the filter (may exceed the capacity)
+  uint32_t band_kmax;  // largest key appended
+  uint32_t band_nkmin; // bitwise complement of the smallest key appended
+  int32_t bins;        // key bins the band solve used (diagnostic)
   int32_t rank_lo, rank_hi;  // ascending sample ranks of the two edges
   uint32_t valid_lo, valid_hi;
   int32_t widen_count, m;

@@ -83,24 +83,21 @@ struct StreamPlan {
   int m;
   int rank_lo, rank_hi, valid_lo, valid_hi;
   int widen_delta, max_widen;
-  int T, C;              // buckets and slots per bucket
-  int T_max;
-  int64_t band_cap;      // slots per row
+  int64_t band_cap;      // band slots per row
   uint64_t seed;
   int force_fallback;
   int vec;
-  int Gs, Gf, G3, Gm, Gr;  // grids: sampling, filter, band solve, membership, recovery
+  int Gs, Gf, Gm, Gr;    // grids: sampling, filter, membership, recovery
+  int band_cs;           // CTAs in the cluster that solves one row's band
   // workspace pieces
   void* ctl;             // RowCtl[rows] followed by the zeroed per-row block
   size_t zero_bytes;     // bytes to clear at the start of each forward
   uint32_t* hist1;       // [rows][2048]
   uint32_t* hist2;       // [rows][2][2048]
   uint32_t* hist3;       // [rows][2][1024]
-  uint32_t* cursor;      // [rows][T_max]
   uint32_t* samp;        // [rows][m]
   void* fpart;           // filter partials [rows][Gf]
-  float* band;           // [rows][band_cap]
-  void* aggs;            // GroupAgg [rows][T_max]
+  float* band;           // [rows][band_cap], unsorted
   void* mpart;           // membership partials [rows][Gm]
   uint32_t* fb_keys;     // [n] keys for the full-sort fallback
   void* fb_aggs;         // GroupAgg [n / kFallbackGroup + 1]
@@ -108,25 +105,10 @@ struct StreamPlan {
 };
 
 constexpr int kFallbackGroup = 4096;   // full-sort fallback: sorted values per group
-constexpr int kBucketTarget = 1024;    // expected band values per bucket
-constexpr int kBucketMax = 8192;       // largest bucket one block sorts in shared memory
+constexpr int kBucketMax = 8192;       // keys of the fallback's shared-memory tiles
 constexpr int kMaxGridPerRow = 4096;   // partial-sum slots per row
 constexpr int kStreamThreads = 256;
-
-// Buckets for a band that spans sample ranks [rank_lo, rank_hi]: the expected
-// band size is (rank_hi - rank_lo + 1) n / m values.
-__host__ __device__ inline void plan_buckets(int64_t n, int m, int rank_lo, int rank_hi, int T_max,
-                                             int64_t band_cap, int* T, int* C) {
-  const double M_est = (double)(rank_hi - rank_lo + 1) * (double)n / (double)m;
-  double tt = ceil(M_est / (double)kBucketTarget);
-  if (tt < 1.0) tt = 1.0;
-  if (tt > (double)T_max) tt = (double)T_max;
-  const int t = (int)tt;
-  int64_t c = band_cap / t;
-  if (c > kBucketMax) c = kBucketMax;
-  *T = t;
-  *C = (int)c;
-}
+constexpr int kBandValuesPerCta = 16384;  // band values one CTA of the band cluster bins
 
 cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p_out, double* b_out,
                               double* sumf_out, uint32_t* status_out, lapsum_row_stats* stats,
@@ -154,9 +136,9 @@ struct StreamOcc {
   int memb_blocks;      // of the membership pass
   int reduce_blocks;    // of the backward reduction
   int apply_blocks;     // of the backward elementwise pass
-  int band_blocks;      // of the band sort kernel for the given bucket size
   int recover_blocks;   // of the cooperative recovery kernel
+  int band_max_cluster; // largest cluster of band CTAs (power of two, <= 16)
 };
-cudaError_t stream_occupancy(int C, StreamOcc* out);
+cudaError_t stream_occupancy(StreamOcc* out);
 
 }  // namespace lapsum

@@ -21,6 +21,8 @@
 // form of common.cuh.
 #pragma once
 
+#include <cstring>
+
 #include "common.cuh"
 
 namespace lapsum {
@@ -143,9 +145,13 @@ __device__ __forceinline__ double block_excl_scan_anchor(double v, double init, 
   }
 }
 
+// exp in fp64, called (not inlined) from the one-pass solver code: one copy
+// of the routine instead of one per call site keeps that code small
+static __device__ __noinline__ double exp_call(double x) { return exp(x); }
+
 // link factor exp((from - to)/alpha) for from <= to; 0 when from = -inf (or to = +inf)
 __device__ __forceinline__ double link(double from, double to, double inva) {
-  return isfinite(from) && isfinite(to) ? exp((from - to) * inva) : 0.0;
+  return isfinite(from) && isfinite(to) ? exp_call((from - to) * inva) : 0.0;
 }
 
 // Result of the group-level step, shared by every thread of the block.
@@ -416,6 +422,183 @@ __device__ void solve_values(const SolveIn in, const GroupPick& pk, int c, const
     out->M = pk.M;
     out->S_aL = pk.S_aL;
     out->S_aR = pk.S_aR;
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// The group level over key bins (the streaming band solve).  Bin t holds the
+// values in [e_t, e_{t+1}) of a key window (the top bin also its upper edge).
+// States are anchored at the bin edges:
+//   prefix  Ahat_{t+1} = sum over values below e_{t+1} of exp((y - e_{t+1})/a)
+//                      = Ahat_t s_t + P_t g_t
+//   suffix  Bhat_t     = sum over values from e_t on of exp((e_t - y)/a)
+//                      = Bhat_{t+1} s_t + Q_t r_t
+// with s_t = exp((e_t - e_{t+1})/a), g_t = exp((ymax_t - e_{t+1})/a),
+// r_t = exp((e_t - ymin_t)/a), and P_t, Q_t the bin's sums anchored at its own
+// maximum and minimum.  Every factor is computed beforehand (in parallel, by
+// whoever fills the table), so the solve is exps-free: two scans of affine
+// maps and the knot values
+//   S(ymax_t) = (Ahat_t h_t + P_t) / 2 + after_t - Bhat_{t+1} g_t / 2,
+// h_t = exp((e_t - ymax_t)/a).  Edge states are floating point, so a state
+// that underflows stands only for contributions that are negligible next to
+// the value-anchored sums (each of which is at least 1).
+// ---------------------------------------------------------------------------
+template <int NB>
+struct BinTable {
+  uint32_t cnt[NB];
+  float ymin[NB];
+  float ymax[NB];
+  float eup[NB];  // upper edge e_{t+1}
+  double s[NB];   // exp((e_t - e_{t+1})/a)
+  double g[NB];   // exp((ymax_t - e_{t+1})/a)
+  double h[NB];   // exp((e_t - ymax_t)/a)
+  double P[NB];   // sum exp((y - ymax_t)/a)
+  double Pg[NB];  // P_t g_t
+  double Qr[NB];  // Q_t r_t, Q_t = sum exp((ymin_t - y)/a)
+};
+
+template <int Q, typename T>
+__device__ __forceinline__ void load_chunk(T (&dst)[Q], const T* src) {
+  static_assert((Q * sizeof(T)) % 16 == 0, "chunk must be whole 16-byte words");
+  constexpr int V = (int)(Q * sizeof(T) / 16);
+  uint4 w[V];
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int v = 0; v < V; ++v) w[v] = s[v];
+  memcpy(dst, w, sizeof(dst));
+}
+
+// e0, eN: the first lower edge and the last upper edge of the window (every
+// band value of the level lies in [e0, eN]).  Same pick as solve_groups, with
+// out_x the upper edge of the picked bin.
+template <int NT, int NB>
+__device__ void solve_bins(const SolveIn in, const BinTable<NB>& tb, double e0, double eN, double* red,
+                           GroupPick* pk) {
+  constexpr int Q = NB / NT;
+  static_assert(Q >= 4 && NB % NT == 0, "at least four bins per thread");
+  const double inva = in.inva;
+  const int tid = threadIdx.x;
+  __shared__ double s_dbl[2];
+  __shared__ long long s_ll[1];
+  int* iscr = reinterpret_cast<int*>(red);
+  long long* lscr = reinterpret_cast<long long*>(red);
+  const bool finL = isfinite(in.aL), finR = isfinite(in.aR);
+  const double xL = finL ? (double)in.aL : -CUDART_INF;
+  const double xR = finR ? (double)in.aR : CUDART_INF;
+  const double tL = finL ? exp((xL - e0) * inva) : 0.0;  // a_L -> e0
+  const double tR = finR ? exp((eN - xR) * inva) : 0.0;  // eN -> a_R
+  const double Ah0 = finL ? in.SL * tL : 0.0;            // values below a_L, anchored at e0
+  const double BhN = finR ? in.SR * tR : 0.0;            // values from a_R on, anchored at eN
+  const int t0 = tid * Q;
+
+  uint32_t cn[Q];
+  double sv[Q], pg[Q], qr[Q];
+  load_chunk(cn, tb.cnt + t0);
+  load_chunk(sv, tb.s + t0);
+  load_chunk(pg, tb.Pg + t0);
+  load_chunk(qr, tb.Qr + t0);
+  long long cloc = 0;
+#pragma unroll
+  for (int j = 0; j < Q; ++j) cloc += cn[j];
+  const long long cexc = block_excl_suffix_sum<NT>(cloc, lscr);
+
+  // forward: edge prefix states
+  Aff m = aff_id();
+#pragma unroll
+  for (int j = 0; j < Q; ++j) m = aff_then(m, Aff{sv[j], pg[j]});
+  const Aff fe = block_excl_scan_aff<NT, true>(m, red);
+  const double Ah_in = fma(Ah0, fe.F, fe.S);  // at this chunk's lower edge
+  double Ah[Q];
+  {
+    double a = Ah_in;
+#pragma unroll
+    for (int j = 0; j < Q; ++j) {
+      Ah[j] = a;
+      a = fma(a, sv[j], pg[j]);
+    }
+    if (tid == NT - 1) s_dbl[0] = a;  // at eN
+  }
+
+  // backward: edge suffix states and the knot values S(ymax_t)
+  Aff mb = aff_id();
+#pragma unroll
+  for (int j = Q - 1; j >= 0; --j) mb = aff_then(mb, Aff{sv[j], qr[j]});
+  const Aff be = block_excl_scan_aff<NT, false>(mb, red);
+  const double Bh_in = fma(BhN, be.F, be.S);  // at this chunk's upper edge
+  double gv[Q], hv[Q], pv[Q];
+  load_chunk(gv, tb.g + t0);
+  load_chunk(hv, tb.h + t0);
+  load_chunk(pv, tb.P + t0);
+  int cand = -1;
+  {
+    double bb = Bh_in;
+    long long after = cexc + in.nR;
+#pragma unroll
+    for (int j = Q - 1; j >= 0; --j) {
+      if (cn[j]) {
+        const double A = fma(Ah[j], hv[j], pv[j]);
+        const double S = 0.5 * A + (double)after - 0.5 * bb * gv[j];
+        if (cand < 0 && S >= in.k) cand = t0 + j;
+      }
+      bb = fma(bb, sv[j], qr[j]);
+      after += cn[j];
+    }
+    if (tid == 0) {
+      s_dbl[1] = bb;     // at e0
+      s_ll[0] = after;   // M + n_R
+    }
+  }
+  const int t_star = block_max_int<NT>(cand, iscr);
+
+  const long long M = s_ll[0] - in.nR;
+  const double S_aL = finL ? 0.5 * in.SL + (double)(M + in.nR) - 0.5 * s_dbl[1] * tL : CUDART_INF;
+  const double S_aR = finR ? 0.5 * s_dbl[0] * tR + (double)in.nR - 0.5 * in.SR : -CUDART_INF;
+  const bool cert = (S_aL >= in.k) && (S_aR < in.k);
+
+  int tg_loc = INT32_MAX;
+#pragma unroll
+  for (int j = Q - 1; j >= 0; --j)
+    if (t0 + j > t_star && cn[j]) tg_loc = t0 + j;
+  const int tg = block_min_int<NT>(tg_loc, iscr);
+
+  // the owners of t* and tg rerun their chunk for the states they hand over
+  const bool own_st = t_star >= t0 && t_star < t0 + Q;
+  const bool own_tg = tg >= t0 && tg < t0 + Q;
+  if (own_st || own_tg) {
+    double bb = Bh_in;
+    long long after = cexc + in.nR;
+#pragma unroll
+    for (int j = Q - 1; j >= 0; --j) {
+      if (t0 + j == t_star) {
+        pk->inc_x = (double)tb.ymax[t0 + j];
+        pk->inc_s = fma(Ah[j], hv[j], pv[j]);
+      }
+      if (t0 + j == tg) {
+        pk->out_x = (double)tb.eup[t0 + j];
+        pk->out_s = bb;
+        pk->g_after = after;
+      }
+      bb = fma(bb, sv[j], qr[j]);
+      after += cn[j];
+    }
+  }
+  if (tid == 0) {
+    pk->status = cert ? ROW_CERTIFIED
+                      : ((!(S_aL >= in.k) ? ROW_MISS_LEFT : 0u) | (!(S_aR < in.k) ? ROW_MISS_RIGHT : 0u));
+    pk->M = M;
+    pk->S_aL = S_aL;
+    pk->S_aR = S_aR;
+    pk->tg = (tg == INT32_MAX) ? -1 : tg;
+    if (t_star < 0) {
+      pk->inc_x = xL;
+      pk->inc_s = finL ? in.SL : 0.0;
+    }
+    if (tg == INT32_MAX) {
+      pk->out_x = xR;
+      pk->out_s = finR ? in.SR : 0.0;
+      pk->g_after = in.nR;
+    }
   }
   __syncthreads();
 }

@@ -23,13 +23,18 @@
 // L2 is read first.
 #include <algorithm>
 
+#include <cooperative_groups.h>
+
 #include "block_sort.cuh"
 #include "common.cuh"
 #include "launch.h"
 #include "solve.cuh"
+#include "warp_solve.cuh"
 
 namespace lapsum {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr int NT = kStreamThreads;
 constexpr int NW = NT / 32;
@@ -55,10 +60,6 @@ __device__ __forceinline__ FPart* fpart_of(const StreamPlan& P, int64_t r) {
 __device__ __forceinline__ MPart* mpart_of(const StreamPlan& P, int64_t r) {
   return reinterpret_cast<MPart*>(P.mpart) + r * kMaxGridPerRow;
 }
-__device__ __forceinline__ GroupAgg* aggs_of(const StreamPlan& P, int64_t r) {
-  return reinterpret_cast<GroupAgg*>(P.aggs) + r * P.T_max;
-}
-__device__ __forceinline__ uint32_t* cursor_of(const StreamPlan& P, int64_t r) { return P.cursor + r * P.T_max; }
 __device__ __forceinline__ float* band_of(const StreamPlan& P, int64_t r) { return P.band + r * P.band_cap; }
 __device__ __forceinline__ uint32_t* samp_of(const StreamPlan& P, int64_t r) { return P.samp + r * (int64_t)P.m; }
 __device__ __forceinline__ uint32_t* h1_of(const StreamPlan& P, int64_t r) { return P.hist1 + r * 2048; }
@@ -199,19 +200,11 @@ __device__ __forceinline__ uint32_t level3_prefix(const RowCtl* c, int t) {
   return ((uint32_t)vld(&c->sel_bin[0][t]) << 11) | (uint32_t)vld(&c->sel_bin[1][t]);
 }
 
-// bracket and bucket plan for a row (one thread)
-__device__ void write_plan(RowCtl* c, int m, const uint32_t keys[2], int rlo, int rhi, bool vlo, bool vhi,
-                           int T, int C) {
+// bracket of a row (one thread)
+__device__ void write_plan(RowCtl* c, int m, const uint32_t keys[2], int rlo, int rhi, bool vlo, bool vhi) {
   const float vl = key2f(keys[0]), vh = key2f(keys[1]);
   c->aL = vlo ? vl : -CUDART_INF_F;
   c->aR = vhi ? vh : CUDART_INF_F;
-  c->lo = vl;
-  const double w = (double)vh - (double)vl;
-  double iw = (w > 0.0) ? (double)T / w : 0.0;
-  if (iw > 1e30) iw = 1e30;
-  c->inv_w = (float)iw;
-  c->T = T;
-  c->C = C;
   c->rank_lo = rlo;
   c->rank_hi = rhi;
   c->valid_lo = vlo ? 1u : 0u;
@@ -291,7 +284,7 @@ __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
     uint32_t rem[2];
     sel_pick<1024>(h3_of(P, r), true, rk, scr, bin, rem);
     const uint32_t keys[2] = {(pre[0] << 10) | (uint32_t)bin[0], (pre[1] << 10) | (uint32_t)bin[1]};
-    if (threadIdx.x == 0) write_plan(c, P.m, keys, P.rank_lo, P.rank_hi, P.valid_lo, P.valid_hi, P.T, P.C);
+    if (threadIdx.x == 0) write_plan(c, P.m, keys, P.rank_lo, P.rank_hi, P.valid_lo, P.valid_hi);
   }
 }
 
@@ -302,34 +295,63 @@ __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
 // In-band values never leave the streaming loop through global memory: a
 // lane holding some writes its chunk to a shared scratch slot and copies the
 // flagged values into its own column of a shared stage (no atomics, no global
-// reload); columns are appended to the global buckets once per block, or
-// earlier when one is about to fill.
+// reload).  A warp empties its 32 columns into the row's band with one atomic
+// for the whole warp, when one of them is about to fill and at the end.  The
+// band is one unsorted array per row; the band kernel bins it by key.
 constexpr int kLaneStage = 24;  // stage column per lane (floats)
 
 struct FilterCtx {
-  float aL, aR, lo, inv_w, c2;
-  int T, C;
-  uint32_t* cur;
+  float aL, aR, c2;
+  uint32_t* cnt;    // values appended to the band so far (may exceed cap)
+  uint32_t* kmax;   // largest key appended
+  uint32_t* nkmin;  // bitwise complement of the smallest key appended
   float* band;
+  uint32_t cap;
 };
 
-// append an in-band value to its value bucket
-__device__ __noinline__ void band_append(const FilterCtx& f, float x, uint32_t& ovf) {
-  const float tf = (x - f.lo) * f.inv_w;
-  const int t = (tf >= (float)f.T) ? f.T - 1 : (tf > 0.0f ? (int)tf : 0);
-  const uint32_t slot = atomicAdd(f.cur + t, 1u);
-  if (slot < (uint32_t)f.C) f.band[(int64_t)t * f.C + slot] = x;
-  else ovf = 1u;
-}
-
-// empty this lane's stage column into the global buckets (NaN and inf are
-// flagged instead of appended)
-__device__ __noinline__ void flush_column(const FilterCtx& f, const float* col, int cnt, uint32_t& bad,
-                                          uint32_t& ovf) {
-  for (int j = 0; j < cnt; ++j) {
+// Appends the staged values of all 32 lanes (col[j * NT], j < ncol) to the
+// band; NaN and inf are flagged instead.  All lanes of the warp call it.
+__device__ __noinline__ void flush_warp(const FilterCtx& f, const float* col, int ncol, uint32_t& bad,
+                                        uint32_t& ovf) {
+  const int lane = threadIdx.x & 31;
+  int good = 0;
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int j = 0; j < ncol; ++j) {
     const float x = col[j * NT];
-    if (fabsf(x) < CUDART_INF_F) band_append(f, x, ovf);
-    else bad = 1u;
+    if (fabsf(x) < CUDART_INF_F) {
+      ++good;
+      const uint32_t k = f2key(x);
+      kmin = min(kmin, k);
+      kmax = max(kmax, k);
+    } else {
+      bad = 1u;
+    }
+  }
+  int incl = good;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  if (total == 0) return;
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  uint32_t base = 0u;
+  if (lane == 0) {
+    base = atomicAdd(f.cnt, (uint32_t)total);
+    atomicMax(f.kmax, kmax);
+    atomicMax(f.nkmin, ~kmin);
+  }
+  base = __shfl_sync(0xffffffffu, base, 0);
+  uint32_t pos = base + (uint32_t)(incl - good);
+  for (int j = 0; j < ncol; ++j) {
+    const float x = col[j * NT];
+    if (fabsf(x) < CUDART_INF_F) {
+      if (pos < f.cap) f.band[pos] = x;
+      else ovf = 1u;
+      ++pos;
+    }
   }
 }
 
@@ -338,13 +360,12 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   FilterCtx f;
   f.aL = vld(&c->aL);
   f.aR = vld(&c->aR);
-  f.lo = vld(&c->lo);
-  f.inv_w = vld(&c->inv_w);
-  f.T = vld(&c->T);
-  f.C = vld(&c->C);
   f.c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
-  f.cur = cursor_of(P, r);
+  f.cnt = &c->band_cnt;
+  f.kmax = &c->band_kmax;
+  f.nkmin = &c->band_nkmin;
   f.band = band_of(P, r);
+  f.cap = (uint32_t)P.band_cap;
   const float aL = f.aL, aR = f.aR, c2 = f.c2;
   float* col = stage + threadIdx.x;                             // this lane's column, stride NT
   float4* scratch = reinterpret_cast<float4*>(stage + kLaneStage * NT) + threadIdx.x * U;  // U float4
@@ -407,33 +428,39 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
           col[ncol * NT] = sv[i];
           ++ncol;
         } while (mask);
-        if (ncol > kLaneStage - 4 * U) {
-          flush_column(f, col, ncol, bad, ovf);
-          ncol = 0;
-        }
+      }
+      if (__any_sync(0xffffffffu, ncol > kLaneStage - 4 * U)) {
+        flush_warp(f, col, ncol, bad, ovf);
+        ncol = 0;
       }
     }
     done = nchunks * CHUNK4 * 4;
   }
-  for (int64_t i = done + (int64_t)cta * NT + threadIdx.x; i < n; i += (int64_t)ncta * NT) {
-    const float x = row[i];
-    const bool isL = x < aL, isR = x >= aR;
-    const float e = exp2f(fminf(x - aL, aR - x) * c2);
-    if (isL) {
-      sl += (double)e;
-      ++nl;
-    }
-    if (isR) sr += (double)e;
-    amax = fmaxf(amax, fabsf(x));
-    if (!(isL || isR)) {
-      col[ncol * NT] = x;
-      if (++ncol == kLaneStage) {
-        flush_column(f, col, ncol, bad, ovf);
-        ncol = 0;
+  // the rest (or every score, for unaligned rows): one score per thread per
+  // step, the same trip count for the whole block
+  for (int64_t i0 = done + (int64_t)cta * NT; i0 < n; i0 += (int64_t)ncta * NT) {
+    const int64_t i = i0 + threadIdx.x;
+    if (i < n) {
+      const float x = row[i];
+      const bool isL = x < aL, isR = x >= aR;
+      const float e = exp2f(fminf(x - aL, aR - x) * c2);
+      if (isL) {
+        sl += (double)e;
+        ++nl;
+      }
+      if (isR) sr += (double)e;
+      amax = fmaxf(amax, fabsf(x));
+      if (!(isL || isR)) {
+        col[ncol * NT] = x;
+        ++ncol;
       }
     }
+    if (__any_sync(0xffffffffu, ncol >= kLaneStage)) {
+      flush_warp(f, col, ncol, bad, ovf);
+      ncol = 0;
+    }
   }
-  flush_column(f, col, ncol, bad, ovf);
+  if (__any_sync(0xffffffffu, ncol > 0)) flush_warp(f, col, ncol, bad, ovf);
   if (!(amax < CUDART_INF_F)) bad = 1u;
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
   nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
@@ -496,98 +523,527 @@ struct BandSmem {
   static constexpr size_t bytes(int C) { return (size_t)16 * C + (size_t)SortScratch<NT>::kWords * 4 + 64 * 8; }
 };
 
-// every bucket's count, extremes and anchored sums; no sorting
-__device__ void band_aggregate_phase(const StreamPlan& P, int64_t r, RowCtl* c, int cta, int ncta, double* red) {
-  const int T = vld(&c->T), C = vld(&c->C);
-  const double inva = 1.0 / P.alpha;
-  const uint32_t* cur = cursor_of(P, r);
-  const float* band = band_of(P, r);
-  GroupAgg* ag = aggs_of(P, r);
-  for (int t = cta; t < T; t += ncta) {
-    const int cnt = (int)min(__ldcg(cur + t), (uint32_t)C);
-    aggregate_unsorted<NT>(band + (int64_t)t * C, cnt, inva, red, ag + t);
+// ---------------------------------------------------------------------------
+// The band solve.  A cluster of CTAs (one CTA in the recovery kernel) owns a
+// row's unsorted band; with more than one CTA, the leader (rank 0) holds no
+// slice of it and is free for the solve.  Each level:
+//   A  every worker CTA copies its slice of the band into shared memory and
+//      bins it by key (2048 bins over the key window): count and extremes,
+//      then the sums P = sum exp((y - ymax)/a), Q = sum exp((ymin - y)/a)
+//      anchored at the bin's own extremes, in 2^-31 fixed point with exact
+//      64-bit sums (order-independent, hence deterministic);
+//   B  the CTAs merge the bins through distributed shared memory, in CTA
+//      order, into the leader's bin table;
+//   C  the leader runs the certified group solve (solve_bins): the bin that
+//      holds the knot after the root.
+// A single-key bin is solved at once; a bin of at most kTargetCap values is
+// gathered into the leader's shared memory, sorted and solved value by value
+// (by one warp when it has at most kWarpSortMax values); a larger one becomes
+// the key window of the next level (three levels reach single keys).
+// ---------------------------------------------------------------------------
+constexpr int kBins = 2048;
+constexpr int kTargetCap = 4096;
+constexpr int kMaxLevels = 4;
+constexpr int kMaxCluster = 16;
+constexpr int kBandThreads = 256;
+constexpr int kLimbBits = 11;                  // P, Q kept as three 11-bit limb sums
+constexpr int kLimbSliceMax = (1 << 21) - 1;   // slices up to this size cannot overflow a limb word
+
+struct BinPart {  // one CTA's bins
+  uint32_t cnt[kBins];
+  uint32_t kmin[kBins];
+  uint32_t kmax[kBins];
+  uint32_t P[3][kBins];  // limbs (or low word, high word when `wide`)
+  uint32_t Q[3][kBins];
+  uint32_t wide;         // 1: P, Q as two-word 64-bit sums (slices too long for limbs)
+};
+struct TargetBuf {
+  uint32_t keys[kTargetCap];
+  double dscr[kTargetCap];
+};
+enum : int { kBandDone = 0, kBandRefine = 1, kBandExtract = 2 };
+struct BandDecision {
+  int action, tg, shift, level;
+  uint32_t klo, khi;
+  uint32_t count;  // gathered values of the target bin
+};
+constexpr int kStageCap = (int)(sizeof(BinTable<kBins>) / 4);
+struct BandShared {
+  union {
+    BinTable<kBins> tab;     // the leader's merged bins
+    float stage[kStageCap];  // a worker's slice of the band
+  } tu;
+  union {
+    BinPart part;
+    TargetBuf tgt;
+  } u;
+  double red[64];
+  GroupPick pk;
+  SolveOut so;
+  SolveIn in;
+  BandDecision dec;
+};
+constexpr size_t kBandSmemBytes = sizeof(BandShared);
+
+template <typename T>
+__device__ __forceinline__ T* at_rank(T* p, int q, int cs) {
+  if (cs == 1) return p;
+  return cg::this_cluster().map_shared_rank(p, q);
+}
+__device__ __forceinline__ void cl_sync(int cs) {
+  if (cs > 1) cg::this_cluster().sync();
+  else __syncthreads();
+}
+
+// smallest shift that maps the key window onto kBins bins
+__device__ __forceinline__ int bin_shift(uint32_t klo, uint32_t khi) {
+  const uint32_t d = khi - klo;
+  int s = 0;
+  while ((d >> s) >= (uint32_t)kBins) ++s;
+  return s;
+}
+// key of edge e_t of the window (clamped to its top)
+__device__ __forceinline__ uint32_t edge_key(uint32_t klo, uint32_t khi, int shift, int t) {
+  const uint64_t e = (uint64_t)klo + ((uint64_t)t << shift);
+  return e > (uint64_t)khi ? khi : (uint32_t)e;
+}
+
+// one term exp(d/alpha) (d <= 0) in 2^-31 fixed point (at most 2^31)
+__device__ __forceinline__ uint32_t fx_term(float d, float c2) {
+  return __float2uint_rn(exp2f(d * c2) * 0x1p31f);
+}
+// a term into three limb words (no return value needed: plain reductions)
+__device__ __forceinline__ void add_limbs(uint32_t (*L)[kBins], int t, uint32_t v) {
+  constexpr uint32_t m = (1u << kLimbBits) - 1u;
+  atomicAdd(&L[0][t], v & m);
+  atomicAdd(&L[1][t], (v >> kLimbBits) & m);
+  atomicAdd(&L[2][t], v >> (2 * kLimbBits));
+}
+// exact 64-bit sum in two words: the add that wraps the low word carries
+__device__ __forceinline__ void add_wide(uint32_t (*L)[kBins], int t, uint32_t v) {
+  const uint32_t old = atomicAdd(&L[0][t], v);
+  if (old > 0xFFFFFFFFu - v) atomicAdd(&L[1][t], 1u);
+}
+__device__ __forceinline__ double fx_value(uint32_t w0, uint32_t w1, uint32_t w2, bool wide) {
+  const double v = wide ? (double)w1 * 4294967296.0 + (double)w0
+                        : ((double)w2 * (double)(1u << (2 * kLimbBits)) + (double)w1 * (double)(1u << kLimbBits)) +
+                              (double)w0;
+  return v * 0x1p-31;
+}
+
+// value j of a worker's slice: from the shared copy, or from L2
+__device__ __forceinline__ float slice_val(const float* src, const float* stage, bool staged, int j) {
+  return (staged && j < kStageCap) ? stage[j] : __ldcg(src + j);
+}
+
+constexpr int kSliceBatch = 8;  // loads in flight per thread
+
+// Bins the n values at src into bp.  write_stage: copy the first kStageCap of
+// them into `stage` on the way; read_stage: read them from there.  All
+// threads of the block call it.
+template <int NTX>
+__device__ void bin_slice(const float* src, int n, bool write_stage, bool read_stage, float* stage, uint32_t klo,
+                          uint32_t khi, int shift, float c2, BinPart& bp) {
+  const bool wide = n > kLimbSliceMax;
+  for (int t = threadIdx.x; t < kBins; t += NTX) {
+    bp.cnt[t] = 0u;
+    bp.kmin[t] = 0xFFFFFFFFu;
+    bp.kmax[t] = 0u;
+#pragma unroll
+    for (int l = 0; l < 3; ++l) {
+      bp.P[l][t] = 0u;
+      bp.Q[l][t] = 0u;
+    }
+  }
+  if (threadIdx.x == 0) bp.wide = wide ? 1u : 0u;
+  __syncthreads();
+  const bool first_from_stage = read_stage && !write_stage;
+  for (int j0 = 0; j0 < n; j0 += NTX * kSliceBatch) {
+    float v[kSliceBatch];
+#pragma unroll
+    for (int u = 0; u < kSliceBatch; ++u) {
+      const int j = j0 + u * NTX + (int)threadIdx.x;
+      v[u] = 0.0f;
+      if (j < n) v[u] = slice_val(src, stage, first_from_stage, j);
+    }
+#pragma unroll
+    for (int u = 0; u < kSliceBatch; ++u) {
+      const int j = j0 + u * NTX + (int)threadIdx.x;
+      if (j < n) {
+        if (write_stage && j < kStageCap) stage[j] = v[u];
+        const uint32_t key = f2key(v[u]);
+        if (key >= klo && key <= khi) {
+          const int t = (int)((key - klo) >> shift);
+          atomicAdd(&bp.cnt[t], 1u);
+          atomicMin(&bp.kmin[t], key);
+          atomicMax(&bp.kmax[t], key);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int j0 = 0; j0 < n; j0 += NTX * kSliceBatch) {
+    float v[kSliceBatch];
+#pragma unroll
+    for (int u = 0; u < kSliceBatch; ++u) {
+      const int j = j0 + u * NTX + (int)threadIdx.x;
+      v[u] = (j < n) ? slice_val(src, stage, read_stage, j) : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kSliceBatch; ++u) {
+      const int j = j0 + u * NTX + (int)threadIdx.x;
+      if (j < n) {
+        const float y = v[u];
+        const uint32_t key = f2key(y);
+        if (key >= klo && key <= khi) {
+          const int t = (int)((key - klo) >> shift);
+          const uint32_t tp = fx_term(y - key2f(bp.kmax[t]), c2);
+          const uint32_t tq = fx_term(key2f(bp.kmin[t]) - y, c2);
+          if (!wide) {
+            add_limbs(bp.P, t, tp);
+            add_limbs(bp.Q, t, tq);
+          } else {
+            add_wide(bp.P, t, tp);
+            add_wide(bp.Q, t, tq);
+          }
+        }
+      }
+    }
   }
 }
 
-// Reduces the filter partials, certifies the bracket, sorts the bucket that
-// holds the root and solves the row (one block).
-__device__ void band_solve_last(const StreamPlan& P, int64_t r, RowCtl* c, int nparts, const BandSmem& sm) {
-  __shared__ SolveOut so;
-  __shared__ GroupPick pk;
-  double* red = sm.red;
-  const int T = vld(&c->T), C = vld(&c->C);
+// This CTA's share of the bins, merged over all CTAs (in CTA order) into the
+// leader's table together with the edge factors of solve_bins; L lanes per
+// bin, each taking every L-th CTA.  Every load of a CTA's bin is issued before
+// any is used.
+template <int NTX>
+__device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32_t khi, int shift, double inva) {
+  const int per = kBins / cs;
+  int L = NTX / per;
+  L = L < 1 ? 1 : (L > cs ? cs : L);
+  constexpr int QM = 8;  // CTAs per lane: cs <= 16 with L >= cs / 8 at NTX >= 256
+  static_assert(NTX >= 256 && kMaxCluster <= 16, "at most 8 CTAs per merge lane");
+  const int sub = (int)threadIdx.x & (L - 1);
+  BinTable<kBins>* tab0 = at_rank(&S.tu.tab, 0, cs);
+  for (int base = (int)threadIdx.x / L; base < per; base += NTX / L) {
+    const int t = rank * per + base;
+    uint32_t c[QM], mn[QM], mx[QM], p0[QM], p1[QM], p2[QM], q0[QM], q1[QM], q2[QM], wd[QM];
+#pragma unroll
+    for (int i = 0; i < QM; ++i) {
+      const int q = sub + i * L;
+      c[i] = 0u;
+      if (q < cs) {
+        const BinPart* pq = at_rank(&S.u.part, q, cs);
+        c[i] = pq->cnt[t];
+        mn[i] = pq->kmin[t];
+        mx[i] = pq->kmax[t];
+        p0[i] = pq->P[0][t];
+        p1[i] = pq->P[1][t];
+        p2[i] = pq->P[2][t];
+        q0[i] = pq->Q[0][t];
+        q1[i] = pq->Q[1][t];
+        q2[i] = pq->Q[2][t];
+        wd[i] = pq->wide;
+      }
+    }
+    uint32_t cnt = 0u, kmn = 0xFFFFFFFFu, kmx = 0u;
+#pragma unroll
+    for (int q = 0; q < QM; ++q) {
+      if (c[q]) {
+        cnt += c[q];
+        kmn = min(kmn, mn[q]);
+        kmx = max(kmx, mx[q]);
+      }
+    }
+    for (int o = 1; o < L; o <<= 1) {
+      cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+      kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+      kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    }
+    const double ymax = (double)key2f(kmx), ymin = (double)key2f(kmn);
+    double Ps = 0.0, Qs = 0.0;
+#pragma unroll
+    for (int q = 0; q < QM; ++q) {
+      if (c[q]) {
+        Ps += fx_value(p0[q], p1[q], p2[q], wd[q] != 0u) * exp(((double)key2f(mx[q]) - ymax) * inva);
+        Qs += fx_value(q0[q], q1[q], q2[q], wd[q] != 0u) * exp((ymin - (double)key2f(mn[q])) * inva);
+      }
+    }
+    for (int o = 1; o < L; o <<= 1) {
+      Ps += __shfl_xor_sync(0xffffffffu, Ps, o);
+      Qs += __shfl_xor_sync(0xffffffffu, Qs, o);
+    }
+    if (sub == 0) {
+      const double elo = (double)key2f(edge_key(klo, khi, shift, t));
+      const float eup = key2f(edge_key(klo, khi, shift, t + 1));
+      const double ehi = (double)eup;
+      BinTable<kBins>& T = *tab0;
+      T.cnt[t] = cnt;
+      T.ymin[t] = cnt ? (float)ymin : 0.0f;
+      T.ymax[t] = cnt ? (float)ymax : 0.0f;
+      T.eup[t] = eup;
+      T.s[t] = exp((elo - ehi) * inva);
+      if (cnt) {
+        const double g = exp((ymax - ehi) * inva);
+        T.g[t] = g;
+        T.h[t] = exp((elo - ymax) * inva);
+        T.P[t] = Ps;
+        T.Pg[t] = Ps * g;
+        T.Qr[t] = Qs * exp((elo - ymin) * inva);
+      } else {
+        T.g[t] = 0.0;
+        T.h[t] = 0.0;
+        T.P[t] = 0.0;
+        T.Pg[t] = 0.0;
+        T.Qr[t] = 0.0;
+      }
+    }
+  }
+}
+
+// What the band kernel hands to the final kernel for a row whose root lies
+// inside a gathered bin (kept in the row's membership-partial slots, which are
+// not used before the membership pass); the bin's keys go to the start of the
+// row's band buffer, which is no longer read by then.
+struct FinalRec {
+  SolveIn in;
+  GroupPick pk;
+  int cnt;
+};
+__device__ __forceinline__ FinalRec* final_of(const StreamPlan& P, int64_t r) {
+  return reinterpret_cast<FinalRec*>(reinterpret_cast<unsigned char*>(P.mpart) + r * (int64_t)kMaxGridPerRow * 16);
+}
+
+// Solves row r from its filter partials and band.  cs CTAs of one cluster
+// (rank = the CTA's rank in it) or, with cs == 1, one block alone; nparts:
+// filter partials of the row.  defer: leave the sort and solve of a gathered
+// bin to k_final (the row gets ROW_PENDING).  Every thread of every CTA calls it.
+template <int NTX>
+__device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned char* smem, int nparts, int cs,
+                           int rank, bool defer) {
+  BandShared& S = *reinterpret_cast<BandShared*>(smem);
+  double* red = S.red;
   const double inva = 1.0 / P.alpha;
+  const float c2 = (float)(inva * (double)kLog2e);
+  const bool leader = rank == 0;
+
+  // row totals from the filter partials (every CTA, same order)
   const FPart* parts = fpart_of(P, r);
-  const uint32_t* cur = cursor_of(P, r);
-  long long nl = 0, mt = 0;
+  long long nl = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
-  for (int i = threadIdx.x; i < nparts; i += NT) {
+  for (int i = threadIdx.x; i < nparts; i += NTX) {
     nl += __ldcg(&parts[i].nL);
     sl += __ldcg(&parts[i].SL);
     sr += __ldcg(&parts[i].SR);
     bad |= __ldcg(&parts[i].bad);
   }
-  for (int t = threadIdx.x; t < T; t += NT) mt += (long long)__ldcg(cur + t);
-  nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
-  mt = block_sum<NT, long long>(mt, reinterpret_cast<long long*>(red));
-  sl = block_sum<NT, double>(sl, red);
-  sr = block_sum<NT, double>(sr, red);
-  bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  nl = block_sum<NTX, long long>(nl, reinterpret_cast<long long*>(red));
+  sl = block_sum<NTX, double>(sl, red);
+  sr = block_sum<NTX, double>(sr, red);
+  bad = block_or<NTX>(bad, reinterpret_cast<uint32_t*>(red));
   const uint32_t flags = vld(&c->flags);
-  const long long nr = P.n - nl - mt;
+  const uint32_t mt = vld(&c->band_cnt);
+  const long long nr = P.n - nl - (long long)mt;
+  const int64_t M = min((int64_t)mt, P.band_cap);
   uint32_t st = vld(&c->status) & ROW_WIDENED;
   double b = 0.0, sumf = 0.0;
+  int levels = 0;
+
   if (bad) {
     st |= ROW_NONFINITE;
-  } else if (flags & ROW_OVERFLOW) {
+  } else if ((flags & ROW_OVERFLOW) || (int64_t)mt > P.band_cap) {
     st |= ROW_OVERFLOW;
   } else if (P.force_fallback) {
     st |= ROW_FORCE_FB;
   } else {
-    const SolveIn in{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, P.k, P.alpha, inva};
-    GroupAgg* ag = aggs_of(P, r);
-    solve_groups<NT, true>(in, ag, T, red, &pk);
-    if (pk.status != ROW_CERTIFIED) {
-      st |= pk.status;
-    } else {
-      if (pk.tg < 0) {
-        if (threadIdx.x == 0) solve_tail_interval(in, pk, &so);
-        __syncthreads();
-      } else {
-        const int cnt = __ldcg(&ag[pk.tg].cnt);
-        const float* vals = band_of(P, r) + (int64_t)pk.tg * C;
-        for (int i = threadIdx.x; i < cnt; i += NT) sm.kbuf[i] = f2key(__ldcg(vals + i));
-        __syncthreads();
-        block_bitonic_sort<NT>(sm.kbuf, cnt);  // kbuf and tbuf form one buffer of 2C keys
-        solve_values<NT>(in, pk, cnt, KeyVals{sm.kbuf}, sm.dscr, red, &so);
+    // this CTA's slice [lo, lo + n) of the band
+    const int workers = cs > 1 ? cs - 1 : 1;
+    const int w = cs > 1 ? rank - 1 : 0;
+    const int64_t lo = (w < 0) ? 0 : M * w / workers;
+    const int n = (w < 0) ? 0 : (int)(M * (w + 1) / workers - lo);
+    const float* src = band_of(P, r) + lo;
+    uint32_t klo = ~vld(&c->band_nkmin), khi = vld(&c->band_kmax);
+    if (M == 0) klo = khi = 0u;
+    int shift = bin_shift(klo, khi);
+    if (leader && threadIdx.x == 0) S.in = SolveIn{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, P.k, P.alpha, inva};
+    int action = kBandDone;
+    for (int level = 0; level < kMaxLevels; ++level) {
+      levels = level + 1;
+      // a worker keeps its slice in shared memory; a lone CTA (cs == 1) holds
+      // the table in the same place, so it rereads its slice from L2 past level 0
+      bin_slice<NTX>(src, n, level == 0, level == 0 || cs > 1, S.tu.stage, klo, khi, shift, c2, S.u.part);
+      cl_sync(cs);
+      merge_bins<NTX>(S, cs, rank, klo, khi, shift, inva);
+      cl_sync(cs);
+      if (leader) {
+        solve_bins<NTX, kBins>(S.in, S.tu.tab, (double)key2f(klo), (double)key2f(khi), red, &S.pk);
+        if (threadIdx.x == 0) {
+          const GroupPick& pk = S.pk;
+          BandDecision d{kBandDone, pk.tg, shift, level, klo, khi, 0u};
+          S.so.status = pk.status;
+          S.so.M = pk.M;
+          S.so.S_aL = pk.S_aL;
+          S.so.S_aR = pk.S_aR;
+          S.so.b = 0.0;
+          S.so.sumf = 0.0;
+          if (pk.status != ROW_CERTIFIED) {
+          } else if (pk.tg < 0) {
+            solve_tail_interval(S.in, pk, &S.so);
+          } else {
+            const uint32_t gcnt = S.tu.tab.cnt[pk.tg];
+            const float gmin = S.tu.tab.ymin[pk.tg], gmax = S.tu.tab.ymax[pk.tg];
+            const uint32_t gk0 = f2key(gmin), gk1 = f2key(gmax);
+            if (gk0 == gk1) {
+              // every value of the bin equals y: the root lies in [inc_x, y]
+              const double y = (double)gmax;
+              const double Bp = (double)gcnt + pk.out_s * link(y, pk.out_x, S.in.inva);
+              S.so.b = closed_form_root(pk.inc_x, y, pk.inc_s, Bp, (double)((long long)gcnt + pk.g_after), S.in.k,
+                                        S.in.alpha);
+              S.so.sumf = sum_f_at(pk.inc_x, y, pk.inc_s, Bp, S.so.b, S.in.inva);
+            } else if (gcnt <= (uint32_t)kTargetCap) {
+              d.action = kBandExtract;
+            } else if (level + 1 < kMaxLevels) {
+              d.action = kBandRefine;
+              d.klo = gk0;
+              d.khi = gk1;
+              d.shift = bin_shift(gk0, gk1);
+              // everything outside the bin becomes the two tails of the next level
+              S.in.aL = (float)pk.inc_x;
+              S.in.SL = pk.inc_s;
+              S.in.aR = (float)pk.out_x;
+              S.in.SR = pk.out_s;
+              S.in.nR = pk.g_after;
+            } else {
+              S.so.status = ROW_FORCE_FB;
+            }
+          }
+          S.dec = d;
+        }
       }
-      st |= so.status;
-      b = so.b;
-      sumf = so.sumf;
+      cl_sync(cs);
+      const BandDecision d = *at_rank(&S.dec, 0, cs);
+      action = d.action;
+      if (action != kBandRefine) break;
+      klo = d.klo;
+      khi = d.khi;
+      shift = d.shift;
+    }
+    if (action == kBandExtract) {
+      // gather the target bin into the leader's buffer, one atomic per warp
+      const BandDecision d = *at_rank(&S.dec, 0, cs);
+      uint32_t* cnt0 = &at_rank(&S.dec, 0, cs)->count;
+      uint32_t* keys0 = at_rank(S.u.tgt.keys, 0, cs);
+      const int lane = threadIdx.x & 31;
+      for (int j0 = 0; j0 < n; j0 += NTX) {
+        const int j = j0 + (int)threadIdx.x;
+        uint32_t key = 0u;
+        bool hit = false;
+        if (j < n) {
+          key = f2key(slice_val(src, S.tu.stage, cs > 1, j));
+          hit = key >= d.klo && key <= d.khi && (int)((key - d.klo) >> d.shift) == d.tg;
+        }
+        const uint32_t m = __ballot_sync(0xffffffffu, hit);
+        if (m) {
+          uint32_t pos = 0u;
+          if (lane == 0) pos = atomicAdd(cnt0, (uint32_t)__popc(m));
+          pos = __shfl_sync(0xffffffffu, pos, 0) + (uint32_t)__popc(m & ((1u << lane) - 1u));
+          if (hit && pos < (uint32_t)kTargetCap) keys0[pos] = key;
+        }
+      }
+      cl_sync(cs);
+      if (leader && defer) {
+        const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
+        uint32_t* dst = reinterpret_cast<uint32_t*>(band_of(P, r));
+        for (int i = threadIdx.x; i < cnt; i += NTX) dst[i] = S.u.tgt.keys[i];
+        if (threadIdx.x == 0) {
+          FinalRec* f = final_of(P, r);
+          f->in = S.in;
+          f->pk = S.pk;
+          f->cnt = cnt;
+          S.so.status = ROW_PENDING;
+          S.so.b = 0.0;
+          S.so.sumf = 0.0;
+        }
+      } else if (leader) {
+        const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
+        if (cnt <= kWarpSortMax) {
+          if (threadIdx.x < 32)
+            warp_solve_bin(S.in, S.pk, S.u.tgt.keys, cnt, reinterpret_cast<uint32_t*>(S.u.tgt.dscr), &S.so);
+        } else {
+          block_bitonic_sort<NTX>(S.u.tgt.keys, cnt);
+          solve_values<NTX>(S.in, S.pk, cnt, KeyVals{S.u.tgt.keys}, S.u.tgt.dscr, red, &S.so);
+        }
+      }
+    }
+    if (leader) {
+      __syncthreads();
+      st |= S.so.status;
+      b = S.so.b;
+      sumf = S.so.sumf;
     }
   }
-  if (threadIdx.x == 0) {
+  if (leader && threadIdx.x == 0) {
     c->sumf = sumf;
     c->nL = nl;
     c->nR = nr;
-    c->M = mt;
+    c->M = (long long)mt;
     c->SL = sl;
     c->SR = sr;
     c->b = b;
+    c->bins = kBins * levels;
     c->status = st;
     __threadfence();
   }
-  __syncthreads();
+  cl_sync(cs);  // no CTA leaves while another may still read its shared memory
 }
 
-__global__ void __launch_bounds__(NT) k_band(const StreamPlan P) {
+__global__ void __launch_bounds__(kBandThreads, 1) k_band(const StreamPlan P) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const BandSmem sm(smem, P.C);
   const int64_t r = blockIdx.y;
+  const int cs = (int)cg::this_cluster().num_blocks();
+  const int rank = (int)cg::this_cluster().block_rank();
+  band_solve<kBandThreads>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank, true);
+}
+
+// The last step of the band solve for the rows k_band left pending: sort the
+// gathered bin and solve on its values (one CTA per row; one warp when the bin
+// has at most kWarpSortMax values).
+constexpr size_t kFinalSmemBytes = (size_t)kTargetCap * (4 + 8);
+
+__global__ void __launch_bounds__(NT) k_final(const StreamPlan P) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
+  double* dscr = reinterpret_cast<double*>(keys + kTargetCap);
+  __shared__ double red[64];
+  __shared__ SolveOut so;
+  __shared__ SolveIn sin;
+  __shared__ GroupPick spk;
+  const int64_t r = blockIdx.x;
   RowCtl* c = ctl_of(P, r);
-  band_aggregate_phase(P, r, c, blockIdx.x, gridDim.x, sm.red);
-  if (last_block_done(&c->done_solve, gridDim.x)) band_solve_last(P, r, c, P.Gf, sm);
+  const uint32_t st = c->status;
+  if (!(st & ROW_PENDING)) return;
+  const FinalRec* f = final_of(P, r);
+  const int cnt = min(f->cnt, kTargetCap);
+  if (threadIdx.x == 0) {
+    sin = f->in;
+    spk = f->pk;
+  }
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(band_of(P, r));
+  for (int i = threadIdx.x; i < cnt; i += NT) keys[i] = src[i];
+  __syncthreads();
+  if (cnt <= kWarpSortMax) {
+    if (threadIdx.x < 32) warp_solve_bin(sin, spk, keys, cnt, reinterpret_cast<uint32_t*>(dscr), &so);
+  } else {
+    block_bitonic_sort<NT>(keys, cnt);
+    solve_values<NT>(sin, spk, cnt, KeyVals{keys}, dscr, red, &so);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    c->b = so.b;
+    c->sumf = so.sumf;
+    c->status = (st & ~ROW_PENDING) | so.status;
+  }
 }
 
 // ===========================================================================
@@ -595,7 +1051,8 @@ __global__ void __launch_bounds__(NT) k_band(const StreamPlan P) {
 // ===========================================================================
 
 struct RecSmem {
-  static constexpr size_t kTotal = BandSmem::bytes(kBucketMax);
+  static constexpr size_t kSort = BandSmem::bytes(kBucketMax);
+  static constexpr size_t kTotal = kSort > kBandSmemBytes ? kSort : kBandSmemBytes;
 };
 
 // exclusive prefix over `cnt` entries of a global array, in place; returns the total
@@ -662,11 +1119,8 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         rhi += P.widen_delta; vhi = rhi <= P.m - 1;
         if (!vhi) rhi = P.m - 1;
       }
-      int T, Cc;
-      plan_buckets(P.n, P.m, rlo, rhi, P.T_max, P.band_cap, &T, &Cc);
       for (int i = cta * NT + threadIdx.x; i < 2048; i += ncta * NT) { h1_of(P, r)[i] = 0u; h3_of(P, r)[i] = 0u; }
       for (int i = cta * NT + threadIdx.x; i < 4096; i += ncta * NT) h2_of(P, r)[i] = 0u;
-      for (int i = cta * NT + threadIdx.x; i < P.T_max; i += ncta * NT) cursor_of(P, r)[i] = 0u;
       REC_BARRIER();
       sel_hist1(samp_of(P, r), P.m, cta, ncta, h1_of(P, r), sh);
       REC_BARRIER();
@@ -701,8 +1155,11 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         sel_pick<1024>(h3_of(P, r), true, rk, scr, bin, rem);
         if (threadIdx.x == 0) {
           const uint32_t keys[2] = {(pre[0] << 10) | (uint32_t)bin[0], (pre[1] << 10) | (uint32_t)bin[1]};
-          write_plan(c, P.m, keys, rlo, rhi, vlo, vhi, T, Cc);
+          write_plan(c, P.m, keys, rlo, rhi, vlo, vhi);
           c->flags = 0u;
+          c->band_cnt = 0u;
+          c->band_kmax = 0u;
+          c->band_nkmin = 0u;
           c->status = ROW_WIDENED;
           __threadfence();
         }
@@ -710,10 +1167,8 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       REC_BARRIER();
       filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(kbuf));
       REC_BARRIER();
-      band_aggregate_phase(P, r, c, cta, ncta, red);
-      REC_BARRIER();
       if (cta == 0) {
-        band_solve_last(P, r, c, ncta, sm);
+        band_solve<NT>(P, r, c, smem, ncta, 1, 0, false);
         if (threadIdx.x == 0) {
           c->status |= ROW_WIDENED;
           __threadfence();
@@ -816,7 +1271,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
           c->M = n;
           c->SL = 0.0;
           c->SR = 0.0;
-          c->T = ng;
+          c->bins = ng;
           __threadfence();
         }
       }
@@ -918,7 +1373,7 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
         s->sum_p = p;
         s->sum_f = so;
         s->sample_m = P.m;
-        s->buckets = c->T;
+        s->buckets = c->bins;
         s->status = pub;
         s->reserved = 0;
       }
@@ -1048,16 +1503,18 @@ __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
     o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
 }
 
-size_t band_smem(int C) { return BandSmem::bytes(C); }
-
 }  // namespace
 
-cudaError_t stream_occupancy(int C, StreamOcc* out) {
-  cudaError_t e = cudaFuncSetAttribute(k_band, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)band_smem(kBucketMax));
+cudaError_t stream_occupancy(StreamOcc* out) {
+  cudaError_t e = cudaFuncSetAttribute(k_band, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBandSmemBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_band, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_recover, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RecSmem::kTotal);
   if (e != cudaSuccess) return e;
-  int fb = 0, bb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
+  e = cudaFuncSetAttribute(k_final, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmemBytes);
+  if (e != cudaSuccess) return e;
+  int fb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb, NT, 0);
@@ -1066,16 +1523,34 @@ cudaError_t stream_occupancy(int C, StreamOcc* out) {
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ab, k_bwd_apply, NT, 0);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bb, k_band, NT, band_smem(C));
-  if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&rb, k_recover, NT, RecSmem::kTotal);
   if (e != cudaSuccess) return e;
   out->filter_blocks = std::max(fb, 1);
   out->memb_blocks = std::max(mb, 1);
   out->reduce_blocks = std::max(qb, 1);
   out->apply_blocks = std::max(ab, 1);
-  out->band_blocks = std::max(bb, 1);
   out->recover_blocks = std::max(rb, 1);
+  // the largest cluster of band CTAs the device can hold at once
+  out->band_max_cluster = 1;
+  for (int cs = kMaxCluster; cs >= 2; cs >>= 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs, 1, 1);
+    cfg.blockDim = dim3(kBandThreads, 1, 1);
+    cfg.dynamicSmemBytes = kBandSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (cudaOccupancyMaxActiveClusters(&nc, k_band, &cfg) == cudaSuccess && nc >= 1) {
+      out->band_max_cluster = cs;
+      break;
+    }
+    (void)cudaGetLastError();
+  }
   return cudaSuccess;
 }
 
@@ -1103,8 +1578,25 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     k_filter<<<dim3(P.Gf, rows), NT, 0, st>>>(P, scores);
   }
   {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)P.band_cs, rows, 1);
+    cfg.blockDim = dim3(kBandThreads, 1, 1);
+    cfg.dynamicSmemBytes = kBandSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)P.band_cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
     Launch l("k_band", st);
-    k_band<<<dim3(P.G3, rows), NT, band_smem(P.C), st>>>(P);
+    e = cudaLaunchKernelEx(&cfg, k_band, P);
+    if (e != cudaSuccess) return e;
+  }
+  {
+    Launch l("k_final", st);
+    k_final<<<rows, NT, kFinalSmemBytes, st>>>(P);
   }
   {
     StreamPlan Pc = P;
