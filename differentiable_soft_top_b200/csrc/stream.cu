@@ -545,7 +545,7 @@ constexpr int kBins = 2048;
 constexpr int kTargetCap = 4096;
 constexpr int kMaxLevels = 4;
 constexpr int kMaxCluster = 16;
-constexpr int kBandThreads = 256;
+constexpr int kBandThreads = 512;
 constexpr int kLimbBits = 11;                  // P, Q kept as three 11-bit limb sums
 constexpr int kLimbSliceMax = (1 << 21) - 1;   // slices up to this size cannot overflow a limb word
 
@@ -721,8 +721,10 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
   const int per = kBins / cs;
   int L = NTX / per;
   L = L < 1 ? 1 : (L > cs ? cs : L);
-  constexpr int QM = 8;  // CTAs per lane: cs <= 16 with L >= cs / 8 at NTX >= 256
-  static_assert(NTX >= 256 && kMaxCluster <= 16, "at most 8 CTAs per merge lane");
+  // CTAs per lane: L = NTX cs / kBins (at least 1), so a lane takes at most
+  // max(cs / L) = kBins / NTX of them
+  constexpr int QM = kBins / NTX;
+  static_assert(QM >= 1 && QM * NTX == kBins && kMaxCluster <= 16, "lanes per bin must cover the cluster");
   const int sub = (int)threadIdx.x & (L - 1);
   BinTable<kBins>* tab0 = at_rank(&S.tu.tab, 0, cs);
   for (int base = (int)threadIdx.x / L; base < per; base += NTX / L) {
@@ -816,11 +818,11 @@ __device__ __forceinline__ FinalRec* final_of(const StreamPlan& P, int64_t r) {
 
 // Solves row r from its filter partials and band.  cs CTAs of one cluster
 // (rank = the CTA's rank in it) or, with cs == 1, one block alone; nparts:
-// filter partials of the row.  defer: leave the sort and solve of a gathered
+// filter partials of the row.  kDefer: leave the sort and solve of a gathered
 // bin to k_final (the row gets ROW_PENDING).  Every thread of every CTA calls it.
-template <int NTX>
+template <int NTX, bool kDefer>
 __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned char* smem, int nparts, int cs,
-                           int rank, bool defer) {
+                           int rank) {
   BandShared& S = *reinterpret_cast<BandShared*>(smem);
   double* red = S.red;
   const double inva = 1.0 / P.alpha;
@@ -952,27 +954,31 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
         }
       }
       cl_sync(cs);
-      if (leader && defer) {
-        const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
-        uint32_t* dst = reinterpret_cast<uint32_t*>(band_of(P, r));
-        for (int i = threadIdx.x; i < cnt; i += NTX) dst[i] = S.u.tgt.keys[i];
-        if (threadIdx.x == 0) {
-          FinalRec* f = final_of(P, r);
-          f->in = S.in;
-          f->pk = S.pk;
-          f->cnt = cnt;
-          S.so.status = ROW_PENDING;
-          S.so.b = 0.0;
-          S.so.sumf = 0.0;
+      if constexpr (kDefer) {
+        if (leader) {
+          const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
+          uint32_t* dst = reinterpret_cast<uint32_t*>(band_of(P, r));
+          for (int i = threadIdx.x; i < cnt; i += NTX) dst[i] = S.u.tgt.keys[i];
+          if (threadIdx.x == 0) {
+            FinalRec* f = final_of(P, r);
+            f->in = S.in;
+            f->pk = S.pk;
+            f->cnt = cnt;
+            S.so.status = ROW_PENDING;
+            S.so.b = 0.0;
+            S.so.sumf = 0.0;
+          }
         }
-      } else if (leader) {
-        const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
-        if (cnt <= kWarpSortMax) {
-          if (threadIdx.x < 32)
-            warp_solve_bin(S.in, S.pk, S.u.tgt.keys, cnt, reinterpret_cast<uint32_t*>(S.u.tgt.dscr), &S.so);
-        } else {
-          block_bitonic_sort<NTX>(S.u.tgt.keys, cnt);
-          solve_values<NTX>(S.in, S.pk, cnt, KeyVals{S.u.tgt.keys}, S.u.tgt.dscr, red, &S.so);
+      } else {
+        if (leader) {
+          const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
+          if (cnt <= kWarpSortMax) {
+            if (threadIdx.x < 32)
+              warp_solve_bin(S.in, S.pk, S.u.tgt.keys, cnt, reinterpret_cast<uint32_t*>(S.u.tgt.dscr), &S.so);
+          } else {
+            block_bitonic_sort<NTX>(S.u.tgt.keys, cnt);
+            solve_values<NTX>(S.in, S.pk, cnt, KeyVals{S.u.tgt.keys}, S.u.tgt.dscr, red, &S.so);
+          }
         }
       }
     }
@@ -1003,7 +1009,7 @@ __global__ void __launch_bounds__(kBandThreads, 1) k_band(const StreamPlan P) {
   const int64_t r = blockIdx.y;
   const int cs = (int)cg::this_cluster().num_blocks();
   const int rank = (int)cg::this_cluster().block_rank();
-  band_solve<kBandThreads>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank, true);
+  band_solve<kBandThreads, true>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank);
 }
 
 // The last step of the band solve for the rows k_band left pending: sort the
@@ -1168,7 +1174,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(kbuf));
       REC_BARRIER();
       if (cta == 0) {
-        band_solve<NT>(P, r, c, smem, ncta, 1, 0, false);
+        band_solve<NT, false>(P, r, c, smem, ncta, 1, 0);
         if (threadIdx.x == 0) {
           c->status |= ROW_WIDENED;
           __threadfence();
