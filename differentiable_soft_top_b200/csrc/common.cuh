@@ -25,7 +25,6 @@ constexpr uint32_t ROW_PUBLIC = 0xFFu;
 constexpr uint32_t ROW_MISS_LEFT = 0x100u;   // S(a_L) < k: b lies below a_L
 constexpr uint32_t ROW_MISS_RIGHT = 0x200u;  // S(a_R) >= k: b lies at or above a_R
 constexpr uint32_t ROW_FORCE_FB = 0x400u;    // test knob: take the full sort
-constexpr uint32_t ROW_PENDING = 0x800u;     // band solved up to its last step, left to the final kernel
 constexpr uint32_t ROW_NEEDS_RECOVERY = ROW_MISS_LEFT | ROW_MISS_RIGHT | ROW_OVERFLOW | ROW_FORCE_FB;
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -29,7 +29,6 @@
 #include "common.cuh"
 #include "launch.h"
 #include "solve.cuh"
-#include "warp_solve.cuh"
 
 namespace lapsum {
 namespace {
@@ -542,7 +541,7 @@ struct BandSmem {
 // the key window of the next level (three levels reach single keys).
 // ---------------------------------------------------------------------------
 constexpr int kBins = 2048;
-constexpr int kTargetCap = 4096;
+constexpr int kTargetCap = kBins;  // a gathered bin becomes a table of its values
 constexpr int kMaxLevels = 4;
 constexpr int kMaxCluster = 16;
 constexpr int kBandThreads = 512;
@@ -559,7 +558,6 @@ struct BinPart {  // one CTA's bins
 };
 struct TargetBuf {
   uint32_t keys[kTargetCap];
-  double dscr[kTargetCap];
 };
 enum : int { kBandDone = 0, kBandRefine = 1, kBandExtract = 2 };
 struct BandDecision {
@@ -579,6 +577,7 @@ struct BandShared {
   } u;
   double red[64];
   GroupPick pk;
+  GroupPick pk2;  // the pick among the values of the gathered bin
   SolveOut so;
   SolveIn in;
   BandDecision dec;
@@ -803,24 +802,10 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
   }
 }
 
-// What the band kernel hands to the final kernel for a row whose root lies
-// inside a gathered bin (kept in the row's membership-partial slots, which are
-// not used before the membership pass); the bin's keys go to the start of the
-// row's band buffer, which is no longer read by then.
-struct FinalRec {
-  SolveIn in;
-  GroupPick pk;
-  int cnt;
-};
-__device__ __forceinline__ FinalRec* final_of(const StreamPlan& P, int64_t r) {
-  return reinterpret_cast<FinalRec*>(reinterpret_cast<unsigned char*>(P.mpart) + r * (int64_t)kMaxGridPerRow * 16);
-}
-
 // Solves row r from its filter partials and band.  cs CTAs of one cluster
 // (rank = the CTA's rank in it) or, with cs == 1, one block alone; nparts:
-// filter partials of the row.  kDefer: leave the sort and solve of a gathered
-// bin to k_final (the row gets ROW_PENDING).  Every thread of every CTA calls it.
-template <int NTX, bool kDefer>
+// filter partials of the row.  Every thread of every CTA calls it.
+template <int NTX>
 __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned char* smem, int nparts, int cs,
                            int rank) {
   BandShared& S = *reinterpret_cast<BandShared*>(smem);
@@ -954,30 +939,58 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
         }
       }
       cl_sync(cs);
-      if constexpr (kDefer) {
-        if (leader) {
-          const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
-          uint32_t* dst = reinterpret_cast<uint32_t*>(band_of(P, r));
-          for (int i = threadIdx.x; i < cnt; i += NTX) dst[i] = S.u.tgt.keys[i];
-          if (threadIdx.x == 0) {
-            FinalRec* f = final_of(P, r);
-            f->in = S.in;
-            f->pk = S.pk;
-            f->cnt = cnt;
-            S.so.status = ROW_PENDING;
-            S.so.b = 0.0;
-            S.so.sumf = 0.0;
+      if (leader) {
+        // the bin's values, sorted, each one entry of a bin table: the same
+        // group solve then picks the interval between two values that holds
+        // the root, and the closed form finishes
+        const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
+        uint32_t* keys = S.u.tgt.keys;
+        block_bitonic_sort<NTX>(keys, cnt);
+        BinTable<kBins>& T = S.tu.tab;
+        const float ylast = key2f(keys[cnt - 1]);
+        for (int i = threadIdx.x; i < kBins; i += NTX) {
+          if (i < cnt) {
+            const float y = key2f(keys[i]);
+            const float yn = (i + 1 < cnt) ? key2f(keys[i + 1]) : y;
+            const double sv = exp_call(((double)y - (double)yn) * inva);
+            T.cnt[i] = 1u;
+            T.ymin[i] = y;
+            T.ymax[i] = y;
+            T.eup[i] = yn;
+            T.s[i] = sv;
+            T.g[i] = sv;
+            T.h[i] = 1.0;
+            T.P[i] = 1.0;
+            T.Pg[i] = sv;
+            T.Qr[i] = 1.0;
+          } else {
+            T.cnt[i] = 0u;
+            T.ymin[i] = ylast;
+            T.ymax[i] = ylast;
+            T.eup[i] = ylast;
+            T.s[i] = 1.0;
+            T.g[i] = 0.0;
+            T.h[i] = 0.0;
+            T.P[i] = 0.0;
+            T.Pg[i] = 0.0;
+            T.Qr[i] = 0.0;
           }
         }
-      } else {
-        if (leader) {
-          const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
-          if (cnt <= kWarpSortMax) {
-            if (threadIdx.x < 32)
-              warp_solve_bin(S.in, S.pk, S.u.tgt.keys, cnt, reinterpret_cast<uint32_t*>(S.u.tgt.dscr), &S.so);
+        __syncthreads();
+        const GroupPick& pk = S.pk;
+        const SolveIn vin{(float)pk.inc_x, (float)pk.out_x, 0, pk.g_after, pk.inc_s, pk.out_s,
+                          S.in.k, S.in.alpha, S.in.inva};
+        solve_bins<NTX, kBins>(vin, T, (double)key2f(keys[0]), (double)ylast, red, &S.pk2);
+        if (threadIdx.x == 0) {
+          const GroupPick& q = S.pk2;
+          if (q.status != ROW_CERTIFIED || q.tg < 0) {
+            S.so.status = ROW_FORCE_FB;  // the two levels disagree at rounding level: full sort
           } else {
-            block_bitonic_sort<NTX>(S.u.tgt.keys, cnt);
-            solve_values<NTX>(S.in, S.pk, cnt, KeyVals{S.u.tgt.keys}, S.u.tgt.dscr, red, &S.so);
+            const double y = (double)T.ymax[q.tg];
+            const double Bp = 1.0 + q.out_s * link(y, q.out_x, inva);
+            S.so.b = closed_form_root(q.inc_x, y, q.inc_s, Bp, (double)(1 + q.g_after), S.in.k, S.in.alpha);
+            S.so.sumf = sum_f_at(q.inc_x, y, q.inc_s, Bp, S.so.b, inva);
+            S.so.status = ROW_CERTIFIED;
           }
         }
       }
@@ -1009,47 +1022,7 @@ __global__ void __launch_bounds__(kBandThreads, 1) k_band(const StreamPlan P) {
   const int64_t r = blockIdx.y;
   const int cs = (int)cg::this_cluster().num_blocks();
   const int rank = (int)cg::this_cluster().block_rank();
-  band_solve<kBandThreads, true>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank);
-}
-
-// The last step of the band solve for the rows k_band left pending: sort the
-// gathered bin and solve on its values (one CTA per row; one warp when the bin
-// has at most kWarpSortMax values).
-constexpr size_t kFinalSmemBytes = (size_t)kTargetCap * (4 + 8);
-
-__global__ void __launch_bounds__(NT) k_final(const StreamPlan P) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem);
-  double* dscr = reinterpret_cast<double*>(keys + kTargetCap);
-  __shared__ double red[64];
-  __shared__ SolveOut so;
-  __shared__ SolveIn sin;
-  __shared__ GroupPick spk;
-  const int64_t r = blockIdx.x;
-  RowCtl* c = ctl_of(P, r);
-  const uint32_t st = c->status;
-  if (!(st & ROW_PENDING)) return;
-  const FinalRec* f = final_of(P, r);
-  const int cnt = min(f->cnt, kTargetCap);
-  if (threadIdx.x == 0) {
-    sin = f->in;
-    spk = f->pk;
-  }
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(band_of(P, r));
-  for (int i = threadIdx.x; i < cnt; i += NT) keys[i] = src[i];
-  __syncthreads();
-  if (cnt <= kWarpSortMax) {
-    if (threadIdx.x < 32) warp_solve_bin(sin, spk, keys, cnt, reinterpret_cast<uint32_t*>(dscr), &so);
-  } else {
-    block_bitonic_sort<NT>(keys, cnt);
-    solve_values<NT>(sin, spk, cnt, KeyVals{keys}, dscr, red, &so);
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    c->b = so.b;
-    c->sumf = so.sumf;
-    c->status = (st & ~ROW_PENDING) | so.status;
-  }
+  band_solve<kBandThreads>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank);
 }
 
 // ===========================================================================
@@ -1174,7 +1147,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(kbuf));
       REC_BARRIER();
       if (cta == 0) {
-        band_solve<NT, false>(P, r, c, smem, ncta, 1, 0);
+        band_solve<NT>(P, r, c, smem, ncta, 1, 0);
         if (threadIdx.x == 0) {
           c->status |= ROW_WIDENED;
           __threadfence();
@@ -1518,8 +1491,6 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_recover, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RecSmem::kTotal);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_final, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFinalSmemBytes);
-  if (e != cudaSuccess) return e;
   int fb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
   if (e != cudaSuccess) return e;
@@ -1599,10 +1570,6 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     Launch l("k_band", st);
     e = cudaLaunchKernelEx(&cfg, k_band, P);
     if (e != cudaSuccess) return e;
-  }
-  {
-    Launch l("k_final", st);
-    k_final<<<rows, NT, kFinalSmemBytes, st>>>(P);
   }
   {
     StreamPlan Pc = P;
