@@ -116,7 +116,7 @@ struct alignas(256) RowCtl {
 };
 static_assert(sizeof(RowCtl) == 256, "RowCtl must stay one 256-byte slot");
 
-// aggregates of one sorted group of band values (a bucket, or a slice of a
+// aggregates of one sorted group of band values (a group of the resident band, or a slice of a
 // fully sorted row): count, min, max, P = sum exp((y - ymax)/alpha),
 // Q = sum exp((ymin - y)/alpha); plus scan results filled in by the solver.
 struct alignas(16) GroupAgg {

@@ -6,12 +6,12 @@
 //   k_sample    localization sample: m Laplace-noised scores, level-1
 //               histogram of their fp32 keys
 //   k_select2/3 radix select of the two binomial order statistics that bound
-//               the bracket [a_L, a_R); the last block plans the band buckets
+//               the bracket [a_L, a_R)
 //   k_filter    the HBM-bound stream-and-filter pass: 128-bit loads, tail
 //               counts and anchored tail sums (fp32 exp, fp64 partials), and
-//               in-band values appended to value buckets
-//   k_band      each bucket radix-sorted in shared memory; the last block
-//               runs the certified exact solve (solve.cuh)
+//               in-band values appended, unsorted, to the row's band
+//   k_band      a cluster of CTAs bins the band by key, certifies the bracket
+//               and solves on the one bin that holds the root (solve.cuh)
 //   k_recover   cooperative, exits at once unless a row failed certification:
 //               widens the bracket once, then falls back to a full radix sort
 //               of the row (the worst-case branch of the abstract)
@@ -489,7 +489,7 @@ __global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const floa
 }
 
 // ===========================================================================
-// band: bucket aggregates, then the certified solve on the one bucket that
+// band: key bins, certification, and the exact solve on the one bin that
 // holds the root (section 2.2, steps 3-4)
 // ===========================================================================
 
@@ -503,9 +503,9 @@ struct KeyGroupsG {  // consecutive groups of `g` sorted keys in global memory
   __device__ float get(int grp, int i) const { return key2f(__ldcg(k + (int64_t)grp * g + i)); }
 };
 
-// Shared-memory layout of the band kernels for buckets of up to C values:
-// keys and radix scratch (4C + 4C bytes), per-value prefix sums of the solve
-// (8C bytes), the radix histograms and the reduction scratch.
+// Shared-memory layout of the recovery kernel's full sort for tiles of up to
+// C keys: keys and radix scratch (4C + 4C bytes), per-value prefix sums of
+// the solve (8C bytes), the radix histograms and the reduction scratch.
 struct BandSmem {
   uint32_t* kbuf;
   uint32_t* tbuf;

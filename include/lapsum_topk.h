@@ -74,8 +74,8 @@ extern "C" {
                                        this row are unspecified */
 #define LAPSUM_ROW_TIMEOUT 0x10u    /* a bounded device wait gave up: outputs
                                        of this row are unspecified */
-#define LAPSUM_ROW_OVERFLOW 0x20u   /* informational: a band bucket overflowed
-                                       (the row then took the fallback) */
+#define LAPSUM_ROW_OVERFLOW 0x20u   /* informational: the band outgrew its
+                                       capacity (the row then took the fallback) */
 
 /* ---- tuning and test knobs --------------------------------------------- */
 typedef struct lapsum_params {
@@ -108,7 +108,8 @@ typedef struct lapsum_row_stats {
     double sum_p;            /* sum of the written p, accumulated in fp64 */
     double sum_f;            /* sum_i f_i */
     int32_t sample_m;        /* sample size used */
-    int32_t buckets;         /* band buckets used */
+    int32_t buckets;         /* band key bins used (all levels), or groups
+                                of the full-sort fallback */
     uint32_t status;         /* same bits as row_status */
     int32_t reserved;
 } lapsum_row_stats;
