@@ -129,6 +129,12 @@ struct alignas(16) GroupAgg {
   long long after;       // number of values after the group (incl. right tail)
 };
 
+// fp64 exp and log called (not inlined) from code that runs once per row:
+// one shared copy of each routine keeps that code small, which matters when
+// its instructions have to be fetched from HBM
+static __device__ __noinline__ double exp_call(double x) { return exp(x); }
+static __device__ __noinline__ double log_call(double x) { return log(x); }
+
 // ---------------------------------------------------------------------------
 // anchored exponential sums: a state (x, s) means sum_v exp(+-(v - x)/alpha)
 // over a run of sorted values.  s == 0 is the empty run.
@@ -164,25 +170,25 @@ __device__ __forceinline__ double suf_at(Anch st, double y, double inva) {
 // ln(m + sqrt(m^2 + e^L)) for m >= 0, without overflow or underflow
 __device__ __forceinline__ double lnsum(double m, double L) {
   if (m == 0.0) return 0.5 * L;
-  const double lm = log(m);
+  const double lm = log_call(m);
   const double D = L - 2.0 * lm;
-  if (D > 0.0) return 0.5 * L + log(exp(-0.5 * D) + sqrt(exp(-D) + 1.0));
-  return lm + log(1.0 + sqrt(1.0 + exp(D)));
+  if (D > 0.0) return 0.5 * L + log_call(exp_call(-0.5 * D) + sqrt(exp_call(-D) + 1.0));
+  return lm + log_call(1.0 + sqrt(1.0 + exp_call(D)));
 }
 
 // Closed-form root on one interval [xj, xj1] of the threshold curve
 // (section 2.2: once the interval holding b is known, b has a closed form).
 // A  = prefix sum anchored at xj  (values <= xj, the left tail included),
 // Bp = suffix sum anchored at xj1 (values >= xj1, the right tail included),
-// c  = number of values above xj.  With u = exp((b - xj)/alpha) the budget
-// equation is B u^2 - 2 mu u - A = 0, mu = c - k, B = Bp exp(-(xj1-xj)/alpha).
+// c  = number of values above xj.  With u = exp_call((b - xj)/alpha) the budget
+// equation is B u^2 - 2 mu u - A = 0, mu = c - k, B = Bp exp_call(-(xj1-xj)/alpha).
 // The root is taken from the right knot when mu >= 0, from the left otherwise,
 // in log form; the result is clamped into the interval.
 __device__ __forceinline__ double closed_form_root(double xj, double xj1, double A, double Bp,
                                                    double c, double k, double alpha) {
   const double mu = c - k;
-  const double lnA = A > 0.0 ? log(A) : -CUDART_INF;
-  const double lnB = Bp > 0.0 ? log(Bp) : -CUDART_INF;
+  const double lnA = A > 0.0 ? log_call(A) : -CUDART_INF;
+  const double lnB = Bp > 0.0 ? log_call(Bp) : -CUDART_INF;
   double L = -CUDART_INF;
   if (A > 0.0 && Bp > 0.0) L = lnA + lnB - (xj1 - xj) / alpha;
   double b;
@@ -196,13 +202,13 @@ __device__ __forceinline__ double closed_form_root(double xj, double xj1, double
   return b;
 }
 
-// sum_i f_i at the root b in [xj, xj1], f_i = exp(-|r_i - b|/alpha)/(2 alpha):
-// the values up to xj contribute A exp((xj - b)/alpha), those from xj1 on
-// contribute Bp exp((b - xj1)/alpha) (A, Bp anchored as in closed_form_root).
+// sum_i f_i at the root b in [xj, xj1], f_i = exp_call(-|r_i - b|/alpha)/(2 alpha):
+// the values up to xj contribute A exp_call((xj - b)/alpha), those from xj1 on
+// contribute Bp exp_call((b - xj1)/alpha) (A, Bp anchored as in closed_form_root).
 // Exact in fp64, so it does not underflow with the fp32 per-score terms.
 __device__ __forceinline__ double sum_f_at(double xj, double xj1, double A, double Bp, double b, double inva) {
-  const double t1 = A > 0.0 ? A * exp((xj - b) * inva) : 0.0;
-  const double t2 = Bp > 0.0 ? Bp * exp((b - xj1) * inva) : 0.0;
+  const double t1 = A > 0.0 ? A * exp_call((xj - b) * inva) : 0.0;
+  const double t2 = Bp > 0.0 ? Bp * exp_call((b - xj1) * inva) : 0.0;
   return 0.5 * (t1 + t2) * inva;
 }
 

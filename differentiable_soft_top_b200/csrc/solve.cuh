@@ -145,10 +145,6 @@ __device__ __forceinline__ double block_excl_scan_anchor(double v, double init, 
   }
 }
 
-// exp in fp64, called (not inlined) from the one-pass solver code: one copy
-// of the routine instead of one per call site keeps that code small
-static __device__ __noinline__ double exp_call(double x) { return exp(x); }
-
 // link factor exp((from - to)/alpha) for from <= to; 0 when from = -inf (or to = +inf)
 __device__ __forceinline__ double link(double from, double to, double inva) {
   return isfinite(from) && isfinite(to) ? exp_call((from - to) * inva) : 0.0;
@@ -473,7 +469,7 @@ __device__ __forceinline__ void load_chunk(T (&dst)[Q], const T* src) {
 // band value of the level lies in [e0, eN]).  Same pick as solve_groups, with
 // out_x the upper edge of the picked bin.
 template <int NT, int NB>
-__device__ void solve_bins(const SolveIn in, const BinTable<NB>& tb, double e0, double eN, double* red,
+__device__ __noinline__ void solve_bins(const SolveIn in, const BinTable<NB>& tb, double e0, double eN, double* red,
                            GroupPick* pk) {
   constexpr int Q = NB / NT;
   static_assert(Q >= 4 && NB % NT == 0, "at least four bins per thread");
@@ -486,8 +482,8 @@ __device__ void solve_bins(const SolveIn in, const BinTable<NB>& tb, double e0, 
   const bool finL = isfinite(in.aL), finR = isfinite(in.aR);
   const double xL = finL ? (double)in.aL : -CUDART_INF;
   const double xR = finR ? (double)in.aR : CUDART_INF;
-  const double tL = finL ? exp((xL - e0) * inva) : 0.0;  // a_L -> e0
-  const double tR = finR ? exp((eN - xR) * inva) : 0.0;  // eN -> a_R
+  const double tL = finL ? exp_call((xL - e0) * inva) : 0.0;  // a_L -> e0
+  const double tR = finR ? exp_call((eN - xR) * inva) : 0.0;  // eN -> a_R
   const double Ah0 = finL ? in.SL * tL : 0.0;            // values below a_L, anchored at e0
   const double BhN = finR ? in.SR * tR : 0.0;            // values from a_R on, anchored at eN
   const int t0 = tid * Q;

@@ -766,8 +766,8 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
 #pragma unroll
     for (int q = 0; q < QM; ++q) {
       if (c[q]) {
-        Ps += fx_value(p0[q], p1[q], p2[q], wd[q] != 0u) * exp(((double)key2f(mx[q]) - ymax) * inva);
-        Qs += fx_value(q0[q], q1[q], q2[q], wd[q] != 0u) * exp((ymin - (double)key2f(mn[q])) * inva);
+        Ps += fx_value(p0[q], p1[q], p2[q], wd[q] != 0u) * exp_call(((double)key2f(mx[q]) - ymax) * inva);
+        Qs += fx_value(q0[q], q1[q], q2[q], wd[q] != 0u) * exp_call((ymin - (double)key2f(mn[q])) * inva);
       }
     }
     for (int o = 1; o < L; o <<= 1) {
@@ -783,14 +783,14 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
       T.ymin[t] = cnt ? (float)ymin : 0.0f;
       T.ymax[t] = cnt ? (float)ymax : 0.0f;
       T.eup[t] = eup;
-      T.s[t] = exp((elo - ehi) * inva);
+      T.s[t] = exp_call((elo - ehi) * inva);
       if (cnt) {
-        const double g = exp((ymax - ehi) * inva);
+        const double g = exp_call((ymax - ehi) * inva);
         T.g[t] = g;
-        T.h[t] = exp((elo - ymax) * inva);
+        T.h[t] = exp_call((elo - ymax) * inva);
         T.P[t] = Ps;
         T.Pg[t] = Ps * g;
-        T.Qr[t] = Qs * exp((elo - ymin) * inva);
+        T.Qr[t] = Qs * exp_call((elo - ymin) * inva);
       } else {
         T.g[t] = 0.0;
         T.h[t] = 0.0;
