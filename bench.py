@@ -82,6 +82,53 @@ def workload_desc(w):
     return f"{w.name}: {w.rows} x {w.n} fp32 {dist}, k={w.k:g}, alpha={w.alpha:g}"
 
 
+class NvmlClockSampler:
+    """SM clock and clock-event reasons polled through NVML every ~2 ms while
+    the timed regions run (the same counters nvidia-smi reports, at a rate
+    that sees a region of a few milliseconds)."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown", 0x4: "sw_power_cap"}
+
+    def __init__(self, torch_device):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        props = __import__("torch").cuda.get_device_properties(torch_device)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            busid = "%08X:%02X:%02X.0" % (getattr(props, "pci_domain_id", 0), bus, getattr(props, "pci_device_id", 0))
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(busid)
+        else:
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_device.index or 0)
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.samples = []
+        self.stop_flag = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop_flag.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), int(get_reasons(self.h))))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        self.thread.start()
+
+    def stop(self):
+        self.stop_flag.set()
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return None
+        reasons = sorted({name for _, r in self.samples for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(c for c, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples), "source": "nvml, ~2 ms polling"}
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
 
@@ -348,31 +395,41 @@ def main():
     if not bool(((st & 1) != 0).all()):
         raise SystemExit(f"rows not certified: status {st.tolist()[:8]}")
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    clocks = ClockSampler(dev.index)
-    if dist is not None:
-        dist.barrier()
-    torch.cuda.synchronize(dev)
-    lt.trace_collect()
-    lt.trace_enable(True)
-    launches0 = lt.launch_count()
+    def timed(traced: bool):
+        """K steps, each after an L2 flush, bracketed by events on the launching
+        stream; with `traced`, every library kernel launch is also bracketed by
+        events (lapsum_trace_*), which adds time to the step itself."""
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        lt.trace_collect()
+        lt.trace_enable(traced)
+        l0 = lt.launch_count()
+        for i in range(args.steps):
+            if not args.no_flush:
+                flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        launched = lt.launch_count() - l0
+        tr = lt.trace_collect()
+        lt.trace_enable(False)
+        if dist is not None:
+            dist.barrier()
+        tot = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dist, dev)
+        return tot / args.steps, launched, tr
+
+    try:
+        clocks = NvmlClockSampler(dev)
+    except Exception:
+        clocks = ClockSampler(dev.index)
     clocks.start()
-    for i in range(args.steps):
-        if not args.no_flush:
-            flush.fill_(i & 0xFF)
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
+    ms_per_step, launches, _ = timed(False)       # the step time: no per-kernel events
+    traced_ms, _, trace = timed(True)             # per-kernel durations for the roofline
     clk = clocks.stop()
-    launches = lt.launch_count() - launches0
-    trace = lt.trace_collect()
-    lt.trace_enable(False)
-    if dist is not None:
-        dist.barrier()
-    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), dist, dev)
-    ms_per_step = total_ms / args.steps
     scores_per_step = rows * n
     value = world * scores_per_step / (ms_per_step * 1e-3)
 
@@ -419,7 +476,10 @@ def main():
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
-                     "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms},
+                     "bytes_per_launch": dom_bytes, "ms_per_launch": dom_ms,
+                     "note": "kernel durations from a second timed region of the same steps with per-launch "
+                             "CUDA events on the launching stream (%.3f ms/step there); the step time above is "
+                             "taken without them" % traced_ms},
         "step_roofline": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_bytes / (ms_per_step * 1e-3) / 1e9,
                           "frac_of_measured": step_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
                           "frac_of_8tbs": step_bytes / (ms_per_step * 1e-3) / 8e12},
