@@ -59,6 +59,8 @@ def _bind(lib):
         "lo_forward_f32": (ctypes.c_int, [_P, _i64, _dbl, _dbl, _P, _P, _P]),
         "lo_backward_f64": (ctypes.c_int, [_P, _P, _i64, _dbl, _dbl, _P, _P, _P]),
         "lo_backward_f32": (ctypes.c_int, [_P, _P, _i64, _dbl, _dbl, _P, _P, _P]),
+        "lo_backward_alpha_f64": (ctypes.c_int, [_P, _P, _i64, _dbl, _dbl, _P]),
+        "lo_backward_alpha_f32": (ctypes.c_int, [_P, _P, _i64, _dbl, _dbl, _P]),
         "lo_S_f64": (_dbl, [_P, _i64, _dbl, _dbl]),
         "lo_S_f32": (_dbl, [_P, _i64, _dbl, _dbl]),
         "lo_sm64_mix": (_u64, [_u64]),
@@ -154,6 +156,21 @@ class Oracle:
             fn = self.lib.lo_backward_f32
         _check(fn(pa, pc, n, float(b), float(alpha), gout.ctypes.data, ctypes.byref(lam), ctypes.byref(sf)))
         return gout.reshape(r.shape), lam.value, sf.value
+
+    def backward_alpha(self, r, g, b, alpha) -> float:
+        """dL/dalpha of L = sum g p at the threshold b (b moves with alpha)."""
+        r = np.asarray(r)
+        out = _dbl()
+        if r.dtype == np.float64:
+            a, pa = _vec(r, np.float64)
+            c, pc = _vec(g, np.float64)
+            fn = self.lib.lo_backward_alpha_f64
+        else:
+            a, pa = _vec(r, np.float32)
+            c, pc = _vec(g, np.float32)
+            fn = self.lib.lo_backward_alpha_f32
+        _check(fn(pa, pc, a.size, float(b), float(alpha), ctypes.byref(out)))
+        return out.value
 
     def S(self, r, b, alpha) -> float:
         r = np.asarray(r)

@@ -217,6 +217,42 @@ int lo_backward_f64(const double* r, const double* g, int64_t n, double b, doubl
     return LO_OK;
 }
 
+/*
+ * dL/dalpha for the loss L = sum_j g_j p_j (technical summary section 2.1:
+ * the budget constraint ties b to alpha).  Differentiating
+ * sum_i F((r_i - b)/alpha) = k with respect to alpha gives
+ *     db/dalpha = - sum_i f_i z_i / sum_i f_i,   z_i = (r_i - b)/alpha,
+ * and then, term by term,
+ *     dp_j/dalpha = f_j (-db/dalpha - z_j),
+ *     dL/dalpha   = sum_j g_j dp_j/dalpha.
+ */
+int lo_backward_alpha_f64(const double* r, const double* g, int64_t n, double b, double alpha,
+                          double* dalpha_out) {
+    if (n < 1) return LO_EINVAL;
+    if (!isfinite(alpha) || !(alpha > 0.0)) return LO_EBADALPHA;
+    nsum sf = {0.0, 0.0}, sfz = {0.0, 0.0};
+    for (int64_t i = 0; i < n; ++i) {
+        const double z = (r[i] - b) / alpha;
+        const double f = 0.5 * exp(-fabs(z)) / alpha;
+        nsum_add(&sf, f);
+        nsum_add(&sfz, f * z);
+    }
+    const double db = -nsum_get(&sfz) / nsum_get(&sf);
+    nsum dl = {0.0, 0.0};
+    for (int64_t i = 0; i < n; ++i) {
+        const double z = (r[i] - b) / alpha;
+        const double f = 0.5 * exp(-fabs(z)) / alpha;
+#if LO_MUTANT == 5
+        const double dp = f * (-z); /* dropped the move of b */
+#else
+        const double dp = f * (-db - z);
+#endif
+        nsum_add(&dl, g[i] * dp);
+    }
+    if (dalpha_out) *dalpha_out = nsum_get(&dl);
+    return LO_OK;
+}
+
 /* ------------------------------------------------------------------ */
 /* fp32-input wrappers (the GPU path reads fp32 scores)                */
 /* ------------------------------------------------------------------ */
@@ -251,6 +287,17 @@ int lo_backward_f32(const float* r, const float* g, int64_t n, double b, double 
     double* e = widen(g, n);
     if (!d || !e) { free(d); free(e); return LO_ENOMEM; }
     int rc = lo_backward_f64(d, e, n, b, alpha, grad_out, lambda_out, sumf_out);
+    free(d);
+    free(e);
+    return rc;
+}
+
+int lo_backward_alpha_f32(const float* r, const float* g, int64_t n, double b, double alpha,
+                          double* dalpha_out) {
+    double* d = widen(r, n);
+    double* e = widen(g, n);
+    if (!d || !e) { free(d); free(e); return LO_ENOMEM; }
+    int rc = lo_backward_alpha_f64(d, e, n, b, alpha, dalpha_out);
     free(d);
     free(e);
     return rc;

@@ -6,6 +6,7 @@ Mutants (see the LO_MUTANT blocks in oracle/lapsum_oracle.c):
   2  the suffix recurrence uses the wrong sign in its exponent
   3  the closed-form root ignores the sign of mu (one anchor for all cases)
   4  the backward pass drops the budget term lambda
+  5  dL/dalpha ignores that the threshold moves with alpha
 """
 import os
 
@@ -34,10 +35,13 @@ def _battery(o):
     run("bwd", lambda: pins.test_backward_invariants(o))
     for seed in range(2):
         run(f"fd{seed}", lambda s=seed: pins.test_vjp_finite_differences(o, s))
+        run(f"fda{seed}", lambda s=seed: pins.test_alpha_gradient_finite_differences(o, s))
+    run("apair", lambda: pins.test_alpha_gradient_symmetric_pair(o))
+    run("aconst", lambda: pins.test_alpha_gradient_constant_upstream_is_zero(o))
     return fails
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5])
 def test_pins_catch_mutant(tmp_path, mutant):
     path = oracle_mod.build(out=str(tmp_path / f"liblo_m{mutant}.so"), mutant=mutant, force=True)
     o = oracle_mod.Oracle(oracle_mod.load(path))

@@ -291,6 +291,47 @@ def test_vjp_finite_differences(orc, seed):
     assert fdk == pytest.approx(lam, rel=1e-6, abs=1e-9)
 
 
+# dL/dalpha: the threshold moves with alpha (section 2.1's constraint)
+@pytest.mark.parametrize("seed", range(6))
+def test_alpha_gradient_finite_differences(orc, seed):
+    rng = np.random.default_rng(300 + seed)
+    n = int(rng.integers(3, 65))
+    r = rng.standard_normal(n)
+    g = rng.standard_normal(n)
+    alpha = float(10 ** rng.uniform(-1, 0.5))
+    k = float(rng.uniform(0.5, n - 0.5))
+    _, b, _ = orc.forward(r, k, alpha)
+    da = orc.backward_alpha(r, g, b, alpha)
+
+    def L(a):
+        p, _, _ = orc.forward(r, k, a)
+        return float(np.dot(g, p))
+
+    h = 1e-6 * alpha
+    fd = (L(alpha + h) - L(alpha - h)) / (2 * h)
+    assert da == pytest.approx(fd, rel=1e-6, abs=1e-9)
+
+
+def test_alpha_gradient_symmetric_pair(orc):
+    """r = (-d, d), k = 1: b = 0 for every alpha, so p_1 = e^{-d/a}/2 and
+    p_2 = 1 - e^{-d/a}/2, and dL/da = (g_1 - g_2) e^{-d/a} d / (2 a^2)."""
+    d, a = 0.7, 0.3
+    r = np.array([-d, d])
+    g = np.array([1.3, -0.4])
+    _, b, _ = orc.forward(r, 1.0, a)
+    assert abs(b) < 1e-15
+    expect = (g[0] - g[1]) * math.exp(-d / a) * d / (2 * a * a)
+    assert orc.backward_alpha(r, g, b, a) == pytest.approx(expect, rel=1e-12)
+
+
+def test_alpha_gradient_constant_upstream_is_zero(orc):
+    """g = c: L = c * k does not depend on alpha."""
+    rng = np.random.default_rng(7)
+    r = rng.standard_normal(50)
+    _, b, _ = orc.forward(r, 12.5, 0.4)
+    assert abs(orc.backward_alpha(r, np.full(50, 2.5), b, 0.4)) < 1e-12
+
+
 # ---------------------------------------------------------------------------
 # localization step (section 2.2): samples, ranks, tails, coverage
 # ---------------------------------------------------------------------------
