@@ -116,7 +116,7 @@ def _load():
             lib.lapsum_topk_workspace_size.restype = sz
             lib.lapsum_topk_fwd.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, sz, P, P]
             lib.lapsum_topk_fwd.restype = ctypes.c_int
-            lib.lapsum_topk_bwd.argtypes = [P, P, P, i64, i64, i64, dbl, P, P, P, sz, P]
+            lib.lapsum_topk_bwd.argtypes = [P, P, P, i64, i64, i64, dbl, P, P, P, P, sz, P]
             lib.lapsum_topk_bwd.restype = ctypes.c_int
             lib.lapsum_topk_fwd_noalloc.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, P]
             lib.lapsum_topk_fwd_noalloc.restype = ctypes.c_int
@@ -258,8 +258,9 @@ def forward(scores, k: float, alpha: float, *, params: Params | None = None, wor
                          b, sumf, status, stats_np)
 
 
-def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None):
-    """dL/dscores and dL/dk for upstream gradient `grad_p` at thresholds `b`."""
+def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None, want_alpha: bool = False):
+    """dL/dscores and dL/dk (per row) for upstream gradient `grad_p` at
+    thresholds `b`; with want_alpha also dL/dalpha per row (a third result)."""
     torch = _torch()
     lib = _load()
     x = _as_rows(scores, "scores")
@@ -274,15 +275,18 @@ def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None):
     if out.stride(0) != x.stride(0):
         raise ValueError("grad_out must have the row stride of scores")
     gk = torch.empty(rows, dtype=torch.float64, device=dev)
+    ga = torch.empty(rows, dtype=torch.float64, device=dev) if want_alpha else None
     bb = b.to(device=dev, dtype=torch.float64).contiguous()
     need = int(lib.lapsum_topk_workspace_size(rows, n, None))
     ws = workspace if workspace is not None else _workspace(dev, need)
     stream = torch.cuda.current_stream(dev).cuda_stream
     rc = lib.lapsum_topk_bwd(x.data_ptr(), g.data_ptr(), bb.data_ptr(), rows, n, x.stride(0), float(alpha),
-                             out.data_ptr(), gk.data_ptr(), ws.data_ptr(), ws.numel(), stream)
+                             out.data_ptr(), gk.data_ptr(), ga.data_ptr() if ga is not None else None,
+                             ws.data_ptr(), ws.numel(), stream)
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_bwd")
-    return (out.view(scores.shape) if grad_out is None else grad_out), gk
+    res = (out.view(scores.shape) if grad_out is None else grad_out), gk
+    return res + (ga,) if want_alpha else res
 
 
 def forward_into(scores, k: float, alpha: float, p, b, sumf, status, workspace, params: Params | None = None,
@@ -324,7 +328,7 @@ def forward_noalloc_into(scores, k: float, alpha: float, p, b, sumf=None, status
         raise LapsumError(rc, "lapsum_topk_fwd_noalloc")
 
 
-def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None) -> None:
+def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None, grad_alpha=None) -> None:
     """backward() with every output preallocated (no allocation in the call)."""
     torch = _torch()
     lib = _load()
@@ -332,6 +336,7 @@ def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None)
     stride = scores.stride(0) if scores.dim() == 2 else n
     rc = lib.lapsum_topk_bwd(scores.data_ptr(), grad_p.data_ptr(), b.data_ptr(), rows, n, stride, float(alpha),
                              grad.data_ptr(), grad_k.data_ptr() if grad_k is not None else None,
+                             grad_alpha.data_ptr() if grad_alpha is not None else None,
                              workspace.data_ptr(), workspace.numel(),
                              torch.cuda.current_stream(scores.device).cuda_stream)
     if rc != LAPSUM_OK:
@@ -339,7 +344,9 @@ def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None)
 
 
 class SoftTopK:
-    """torch.autograd.Function wrapper: p = soft_topk(scores, k, alpha)."""
+    """torch.autograd.Function wrapper: p = soft_topk(scores, k, alpha).  k
+    and alpha may be Python numbers or 0-d tensors; tensors that require grad
+    receive dL/dk (= sum over rows of lambda) and dL/dalpha."""
 
     _fn = None
 
@@ -351,22 +358,33 @@ class SoftTopK:
             class _F(torch.autograd.Function):
                 @staticmethod
                 def forward(ctx, scores, k, alpha, params):
-                    res = forward(scores, k, alpha, params=params)
+                    kf, af = float(k), float(alpha)
+                    res = forward(scores, kf, af, params=params)
                     ctx.save_for_backward(scores, res.b)
-                    ctx.alpha = alpha
+                    ctx.alpha = af
+                    ctx.k_like = k if isinstance(k, torch.Tensor) else None
+                    ctx.a_like = alpha if isinstance(alpha, torch.Tensor) else None
                     return res.p.view(scores.shape)
 
                 @staticmethod
                 def backward(ctx, gp):
                     scores, b = ctx.saved_tensors
                     sc = scores.contiguous()
-                    gs, gk = backward(sc, gp.contiguous().view(sc.shape), b, ctx.alpha)
-                    return gs.view(scores.shape), None, None, None
+                    need_k, need_a = ctx.needs_input_grad[1], ctx.needs_input_grad[2]
+                    out = backward(sc, gp.contiguous().view(sc.shape), b, ctx.alpha, want_alpha=need_a)
+                    gs, gk = out[0], out[1]
+                    grad_k = gk.sum().to(ctx.k_like.dtype).view(ctx.k_like.shape) if need_k else None
+                    grad_a = out[2].sum().to(ctx.a_like.dtype).view(ctx.a_like.shape) if need_a else None
+                    return gs.view(scores.shape), grad_k, grad_a, None
 
             cls._fn = _F
         return cls._fn
 
 
-def soft_topk(scores, k: float, alpha: float, params: Params | None = None):
-    """Differentiable exact-budget soft top-k memberships of `scores` (CUDA fp32)."""
-    return SoftTopK.fn().apply(scores, float(k), float(alpha), params)
+def soft_topk(scores, k, alpha, params: Params | None = None):
+    """Differentiable exact-budget soft top-k memberships of `scores` (CUDA fp32).
+    k and alpha: numbers, or 0-d tensors when their gradients are wanted."""
+    torch = _torch()
+    k = k if isinstance(k, torch.Tensor) else float(k)
+    alpha = alpha if isinstance(alpha, torch.Tensor) else float(alpha)
+    return SoftTopK.fn().apply(scores, k, alpha, params)

@@ -179,7 +179,7 @@ size_t resident_ws_bytes(int64_t rows) { return align256(4 * (size_t)rows) + 256
 
 size_t bwd_ws_bytes(int64_t rows, int64_t n) {
   if (n <= kResidentMaxN) return 0;
-  return align256(32 * (size_t)kMaxGridPerRow * (size_t)rows) + align256(4 * (size_t)rows) +
+  return align256(48 * (size_t)kMaxGridPerRow * (size_t)rows) + align256(4 * (size_t)rows) +
          align256(8 * (size_t)rows);
 }
 
@@ -341,14 +341,15 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
 }
 
 int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
-                    int64_t row_stride, double alpha, float* grad_scores, double* grad_k, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+                    int64_t row_stride, double alpha, float* grad_scores, double* grad_k, double* grad_alpha,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   if (!scores || !grad_p || !b || !grad_scores) return LAPSUM_EINVAL;
   if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
   if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)grad_scores & 3u) ||
       ((uintptr_t)b & 7u))
     return LAPSUM_EINVAL;
   if (grad_k && ((uintptr_t)grad_k & 7u)) return LAPSUM_EINVAL;
+  if (grad_alpha && ((uintptr_t)grad_alpha & 7u)) return LAPSUM_EINVAL;
   if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
   const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
   if (overlaps(scores, span, grad_scores, span) || overlaps(grad_p, span, grad_scores, span)) return LAPSUM_EINVAL;
@@ -360,7 +361,7 @@ int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, i
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
   if (n <= kResidentMaxN) {
-    RowBwd a{scores, grad_p, b, rows, n, row_stride, alpha, grad_scores, grad_k, vec};
+    RowBwd a{scores, grad_p, b, rows, n, row_stride, alpha, grad_scores, grad_k, vec, grad_alpha};
     return cuda_ok(launch_resident_bwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
   }
   unsigned char* ws = static_cast<unsigned char*>(workspace);
@@ -374,12 +375,13 @@ int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, i
   a.alpha = alpha;
   a.grad = grad_scores;
   a.grad_k = grad_k;
+  a.grad_alpha = grad_alpha;
   a.vec = vec;
   a.Gb = stream_grid(dev->sm_count, dev->occ.reduce_blocks, rows, n);
   a.Ga = stream_grid(dev->sm_count, dev->occ.apply_blocks, rows, n);
   size_t o = 0;
   a.part = ws + o;
-  o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
+  o = align256(o + 48 * (size_t)kMaxGridPerRow * (size_t)rows);
   a.done = reinterpret_cast<uint32_t*>(ws + o);
   o = align256(o + 4 * (size_t)rows);
   a.lam = reinterpret_cast<double*>(ws + o);

@@ -375,6 +375,31 @@ __device__ __forceinline__ void shift_add(float a, float g, float& m, float& ps,
   psg = fmaf(g, e, psg);
 }
 
+// The same with two more sums weighted by z = r - b, for dL/dalpha:
+// sum f z and sum g f z, rescaled together with the other two.
+__device__ __forceinline__ void shift_add_z(float a, float g, float z, float& m, float& ps, float& psg,
+                                            float& psz, float& psgz, double& S, double& SG, double& SZ,
+                                            double& SGZ) {
+  if (a < m) {
+    const float sc = exp2f(a - m);
+    ps *= sc;
+    psg *= sc;
+    psz *= sc;
+    psgz *= sc;
+    S *= (double)sc;
+    SG *= (double)sc;
+    SZ *= (double)sc;
+    SGZ *= (double)sc;
+    m = a;
+  }
+  const float e = exp2f(m - a);
+  const float ez = e * z;
+  ps += e;
+  psg = fmaf(g, e, psg);
+  psz += ez;
+  psgz = fmaf(g, ez, psgz);
+}
+
 template <int NT>
 __device__ __forceinline__ float block_min_float(float v, float* scratch) {
   constexpr int NW = NT / 32;
@@ -399,6 +424,26 @@ __device__ __forceinline__ void block_shift_reduce(float& m, double& S, double& 
   S = block_sum<NT, double>(S * sc, red);
   SG = block_sum<NT, double>(SG * sc, red);
   m = M;
+}
+
+template <int NT>
+__device__ __forceinline__ void block_shift_reduce4(float& m, double& S, double& SG, double& SZ, double& SGZ,
+                                                    double* red) {
+  const float M = block_min_float<NT>(m, reinterpret_cast<float*>(red));
+  const double sc = (m == CUDART_INF_F) ? 0.0 : exp2((double)M - (double)m);
+  S = block_sum<NT, double>(S * sc, red);
+  SG = block_sum<NT, double>(SG * sc, red);
+  SZ = block_sum<NT, double>(SZ * sc, red);
+  SGZ = block_sum<NT, double>(SGZ * sc, red);
+  m = M;
+}
+
+// dL/dalpha from the rescaled sums: with a = |r - b| log2(e)/alpha and the
+// terms accumulated as 2^(m - a), sum f w = 2^(-m) / (2 alpha) sum 2^(m-a) w,
+// and dL/dalpha = -(1/alpha) sum (r - b) f (g - lambda).
+__device__ __forceinline__ double alpha_grad(double m, double SZ, double SGZ, double lam, double inva) {
+  if (!(m < 1e300)) return 0.0;  // no finite term
+  return -inva * 0.5 * inva * exp2(-m) * (SGZ - lam * SZ);
 }
 
 // ---------------------------------------------------------------------------

@@ -73,6 +73,7 @@ struct RowBwd {
   float* grad;
   double* grad_k;
   int vec;
+  double* grad_alpha;  // dL/dalpha per row, or null
 };
 cudaError_t launch_resident_bwd(const RowBwd& a, int sm_count, cudaStream_t st);
 
@@ -122,9 +123,10 @@ struct StreamBwd {
   double alpha;
   float* grad;
   double* grad_k;
+  double* grad_alpha;  // dL/dalpha per row, or null
   int vec;
   int Gb, Ga;        // grids of the reduction and elementwise passes
-  void* part;        // [rows][kMaxGridPerRow] partials (32 bytes each)
+  void* part;        // [rows][kMaxGridPerRow] partials (48 bytes each)
   uint32_t* done;    // [rows] counters (zeroed by the launcher)
   double* lam;       // [rows]
 };

@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
 // grad = f (g - lambda) with f = 2^(log2(1/(2 alpha)) - |r - b| log2(e)/alpha)
 // computed in one exponent, and lambda split into two fp32 words so that
 // g - lambda keeps its accuracy when g is close to lambda.
+template <bool kAlpha>
 __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
   __shared__ double red[64];
   const int n = (int)a.n;
@@ -369,26 +370,37 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     const float bh = __double2float_rn(b);
     const float bl = __double2float_rn(b - (double)bh);
     float m = CUDART_INF_F;
-    double S = 0.0, SG = 0.0;
+    double S = 0.0, SG = 0.0, SZ = 0.0, SGZ = 0.0;
+    // one score: the two sums of lambda, and with kAlpha the two of dL/dalpha
+    auto acc = [&](float xv, float gv, float& ps, float& psg, float& psz, float& psgz) {
+      const float z = (xv - bh) - bl;
+      if (kAlpha) shift_add_z(fabsf(z) * c2, gv, z, m, ps, psg, psz, psgz, S, SG, SZ, SGZ);
+      else shift_add(fabsf(z) * c2, gv, m, ps, psg, S, SG);
+    };
     const int n4 = a.vec ? (n >> 2) : 0;
     for (int v = threadIdx.x; v < n4; v += NT) {
       const float4 xv = __ldg(reinterpret_cast<const float4*>(x) + v);
       const float4 gv = __ldg(reinterpret_cast<const float4*>(g) + v);
-      float ps = 0.0f, psg = 0.0f;
-      shift_add(fabsf((xv.x - bh) - bl) * c2, gv.x, m, ps, psg, S, SG);
-      shift_add(fabsf((xv.y - bh) - bl) * c2, gv.y, m, ps, psg, S, SG);
-      shift_add(fabsf((xv.z - bh) - bl) * c2, gv.z, m, ps, psg, S, SG);
-      shift_add(fabsf((xv.w - bh) - bl) * c2, gv.w, m, ps, psg, S, SG);
+      float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
+      acc(xv.x, gv.x, ps, psg, psz, psgz);
+      acc(xv.y, gv.y, ps, psg, psz, psgz);
+      acc(xv.z, gv.z, ps, psg, psz, psgz);
+      acc(xv.w, gv.w, ps, psg, psz, psgz);
       S += (double)ps;
       SG += (double)psg;
+      SZ += (double)psz;
+      SGZ += (double)psgz;
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
-      float ps = 0.0f, psg = 0.0f;
-      shift_add(fabsf((x[i] - bh) - bl) * c2, g[i], m, ps, psg, S, SG);
+      float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
+      acc(x[i], g[i], ps, psg, psz, psgz);
       S += (double)ps;
       SG += (double)psg;
+      SZ += (double)psz;
+      SGZ += (double)psgz;
     }
-    block_shift_reduce<NT>(m, S, SG, red);
+    if (kAlpha) block_shift_reduce4<NT>(m, S, SG, SZ, SGZ, red);
+    else block_shift_reduce<NT>(m, S, SG, red);
     const double lam = SG / S;
     const float lh = __double2float_rn(lam);
     const float ll = __double2float_rn(lam - (double)lh);
@@ -405,6 +417,7 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT)
       o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
     if (threadIdx.x == 0 && a.grad_k) a.grad_k[r] = lam;
+    if (kAlpha && threadIdx.x == 0) a.grad_alpha[r] = alpha_grad((double)m, SZ, SGZ, lam, inva);
     __syncthreads();
   }
 }
@@ -451,7 +464,8 @@ cudaError_t launch_resident_bwd(const RowBwd& a, int sm_count, cudaStream_t st) 
   const unsigned grid = (unsigned)std::min<int64_t>(a.rows, (int64_t)sm_count * 4);
   {
     Launch l("k_row_bwd", st);
-    k_row_bwd<<<grid, NT, 0, st>>>(a);
+    if (a.grad_alpha) k_row_bwd<true><<<grid, NT, 0, st>>>(a);
+    else k_row_bwd<false><<<grid, NT, 0, st>>>(a);
   }
   return cudaGetLastError();
 }

@@ -1361,10 +1361,12 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
 }
 
 struct BPart {
-  double m, S, SG, pad;
+  double m, S, SG, SZ, SGZ, pad;
 };
 
-// lambda = sum g f / sum f by the rescaled reduction of common.cuh
+// lambda = sum g f / sum f by the rescaled reduction of common.cuh; with
+// kAlpha also sum f z and sum g f z (z = r - b) for dL/dalpha
+template <bool kAlpha>
 __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   __shared__ double red[64];
   const int64_t r = blockIdx.y;
@@ -1377,7 +1379,12 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   const float* g = a.grad_p + r * a.stride;
   const int64_t n = a.n;
   float m = CUDART_INF_F;
-  double S = 0.0, SG = 0.0;
+  double S = 0.0, SG = 0.0, SZ = 0.0, SGZ = 0.0;
+  auto acc = [&](float xv, float gv, float& ps, float& psg, float& psz, float& psgz) {
+    const float z = (xv - bh) - bl;
+    if (kAlpha) shift_add_z(fabsf(z) * c2, gv, z, m, ps, psg, psz, psgz, S, SG, SZ, SGZ);
+    else shift_add(fabsf(z) * c2, gv, m, ps, psg, S, SG);
+  };
   int64_t done = 0;
   if (a.vec) {
     const float4* x4 = reinterpret_cast<const float4*>(x);
@@ -1391,45 +1398,63 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
         xv[u] = __ldg(x4 + base + u * NT);
         gv[u] = __ldg(g4 + base + u * NT);
       }
-      float ps = 0.0f, psg = 0.0f;
+      float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        shift_add(fabsf((xv[u].x - bh) - bl) * c2, gv[u].x, m, ps, psg, S, SG);
-        shift_add(fabsf((xv[u].y - bh) - bl) * c2, gv[u].y, m, ps, psg, S, SG);
-        shift_add(fabsf((xv[u].z - bh) - bl) * c2, gv[u].z, m, ps, psg, S, SG);
-        shift_add(fabsf((xv[u].w - bh) - bl) * c2, gv[u].w, m, ps, psg, S, SG);
+        acc(xv[u].x, gv[u].x, ps, psg, psz, psgz);
+        acc(xv[u].y, gv[u].y, ps, psg, psz, psgz);
+        acc(xv[u].z, gv[u].z, ps, psg, psz, psgz);
+        acc(xv[u].w, gv[u].w, ps, psg, psz, psgz);
       }
       S += (double)ps;
       SG += (double)psg;
+      if (kAlpha) {
+        SZ += (double)psz;
+        SGZ += (double)psgz;
+      }
     }
     done = nchunks * CHUNK4 * 4;
   }
   for (int64_t i = done + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
-    float ps = 0.0f, psg = 0.0f;
-    shift_add(fabsf((x[i] - bh) - bl) * c2, g[i], m, ps, psg, S, SG);
+    float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
+    acc(x[i], g[i], ps, psg, psz, psgz);
     S += (double)ps;
     SG += (double)psg;
+    if (kAlpha) {
+      SZ += (double)psz;
+      SGZ += (double)psgz;
+    }
   }
-  block_shift_reduce<NT>(m, S, SG, red);
+  if (kAlpha) block_shift_reduce4<NT>(m, S, SG, SZ, SGZ, red);
+  else block_shift_reduce<NT>(m, S, SG, red);
   BPart* part = reinterpret_cast<BPart*>(a.part) + r * kMaxGridPerRow;
-  if (threadIdx.x == 0) part[blockIdx.x] = BPart{(double)m, S, SG, 0.0};
+  if (threadIdx.x == 0) part[blockIdx.x] = BPart{(double)m, S, SG, SZ, SGZ, 0.0};
   if (last_block_done(a.done + r, gridDim.x)) {
     float mloc = CUDART_INF_F;
     for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) mloc = fminf(mloc, (float)__ldcg(&part[i].m));
     const double M = (double)block_min_float<NT>(mloc, reinterpret_cast<float*>(red));
-    double s = 0.0, sg = 0.0;
+    double s = 0.0, sg = 0.0, sz = 0.0, sgz = 0.0;
     for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
       const double pm = __ldcg(&part[i].m);
       const double sc = (pm == CUDART_INF) ? 0.0 : exp2(M - pm);
       s += __ldcg(&part[i].S) * sc;
       sg += __ldcg(&part[i].SG) * sc;
+      if (kAlpha) {
+        sz += __ldcg(&part[i].SZ) * sc;
+        sgz += __ldcg(&part[i].SGZ) * sc;
+      }
     }
     s = block_sum<NT, double>(s, red);
     sg = block_sum<NT, double>(sg, red);
+    if (kAlpha) {
+      sz = block_sum<NT, double>(sz, red);
+      sgz = block_sum<NT, double>(sgz, red);
+    }
     if (threadIdx.x == 0) {
       const double lam = sg / s;
       a.lam[r] = lam;
       if (a.grad_k) a.grad_k[r] = lam;
+      if (kAlpha) a.grad_alpha[r] = alpha_grad(M, sz, sgz, lam, inva);
     }
   }
 }
@@ -1496,7 +1521,7 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb, NT, 0);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&qb, k_bwd_reduce, NT, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&qb, k_bwd_reduce<false>, NT, 0);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ab, k_bwd_apply, NT, 0);
   if (e != cudaSuccess) return e;
@@ -1592,7 +1617,8 @@ cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   {
     Launch l("k_bwd_reduce", st);
-    k_bwd_reduce<<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+    if (a.grad_alpha) k_bwd_reduce<true><<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+    else k_bwd_reduce<false><<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
   }
   {
     Launch l("k_bwd_apply", st);

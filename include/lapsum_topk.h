@@ -154,6 +154,10 @@ LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int
  *   alpha       in   the forward's alpha
  *   grad_scores out  fp32 [rows, row_stride] dL/dr
  *   grad_k      out  fp64 [rows] dL/dk = lambda (may be NULL)
+ *   grad_alpha  out  fp64 [rows] dL/dalpha (may be NULL; costs two more sums
+ *                    in the reduction pass).  With z_j = (r_j - b)/alpha the
+ *                    threshold moves as db/dalpha = -sum f z / sum f, and
+ *                    dL/dalpha = -(1/alpha) sum_j (r_j - b) grad_j.
  *   workspace   in   as for the forward (the same buffer may be passed)
  * sum_i f_i is not an input: the reduction pass forms sum g f and sum f
  * together, relative to the score nearest b, so that neither underflows.
@@ -161,7 +165,8 @@ LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int
  */
 LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows,
                                int64_t n, int64_t row_stride, double alpha, float* grad_scores,
-                               double* grad_k, void* workspace, size_t workspace_bytes, void* stream);
+                               double* grad_k, double* grad_alpha, void* workspace, size_t workspace_bytes,
+                               void* stream);
 
 /*
  * Forward pass that allocates nothing and takes no workspace.  The paper has

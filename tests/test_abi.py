@@ -113,11 +113,11 @@ def test_fwd_rejects_bad_arguments(lib, kw, code):
 def test_bwd_rejects_bad_arguments(lib):
     B = lib.lapsum_topk_bwd
     ok = dict(s=FAKE, g=FAKE * 2, b=FAKE * 3, rows=1, n=100000, stride=100000, a=0.5, out=FAKE * 4,
-              gk=None, ws=FAKE * 8, wsb=1 << 30)
+              gk=None, ga=None, ws=FAKE * 8, wsb=1 << 30)
 
     def call(**kw):
         d = dict(ok, **kw)
-        return B(d["s"], d["g"], d["b"], d["rows"], d["n"], d["stride"], d["a"], d["out"], d["gk"],
+        return B(d["s"], d["g"], d["b"], d["rows"], d["n"], d["stride"], d["a"], d["out"], d["gk"], d["ga"],
                  d["ws"], d["wsb"], None)
 
     assert call(s=None) == lt.LAPSUM_EINVAL
@@ -127,6 +127,7 @@ def test_bwd_rejects_bad_arguments(lib):
     assert call(a=0.0) == lt.LAPSUM_EBADALPHA
     assert call(out=FAKE + 64) == lt.LAPSUM_EINVAL  # overlaps the scores
     assert call(wsb=16) == lt.LAPSUM_EWORKSPACE
+    assert call(ga=FAKE * 5 + 4) == lt.LAPSUM_EINVAL  # misaligned dL/dalpha output
 
 
 def test_binding_rejects_cpu_tensors():

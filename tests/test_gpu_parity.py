@@ -318,3 +318,55 @@ def test_deep_underflow_gradient_stays_finite(orc):
     _, lam, _ = orc.backward(x[0], g[0], b_ref, 1e-5)
     assert np.isfinite(out["gk"][0]) and out["gk"][0] == pytest.approx(lam, rel=1e-4, abs=1e-6)
     assert np.all(np.isfinite(out["grad"]))
+
+
+# ---------------------------------------------------------------------------
+# dL/dalpha (the threshold moves with alpha): both paths, several rows, and
+# through autograd with k and alpha as tensors
+# ---------------------------------------------------------------------------
+def alpha_tol(r, g, b, alpha):
+    z = r.astype(np.float64) - b
+    f = 0.5 * np.exp(-np.abs(z) / alpha) / alpha
+    return 1e-6 * float(np.sum(np.abs(z) * f * np.abs(g.astype(np.float64)))) / alpha
+
+
+@pytest.mark.parametrize("name,n,rows,force", [
+    ("c1", None, None, 0),
+    ("c1", 4096, 3, lt.FORCE_STREAMING),
+    ("c2", None, None, 0),
+    ("c3", 2_000_003, None, 0),
+    ("c5", 16384, 4, 0),
+])
+def test_alpha_gradient_matches_oracle(orc, name, n, rows, force):
+    w, x, g = case(name, n=n, rows=rows)
+    xt = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    gt = torch.from_numpy(np.ascontiguousarray(g)).cuda()
+    params = lt.Params(force_path=force) if force else None
+    res = lt.forward(xt, w.k, w.alpha, params=params)
+    gs, gk, ga = lt.backward(xt, gt, res.b, w.alpha, want_alpha=True)
+    gs0, gk0 = lt.backward(xt, gt, res.b, w.alpha)
+    torch.cuda.synchronize()
+    # asking for dL/dalpha changes nothing else
+    assert torch.equal(gs, gs0) and torch.equal(gk, gk0)
+    ga = ga.cpu().numpy()
+    for i in range(x.shape[0]):
+        _, b_ref, _ = orc.forward(x[i], w.k, w.alpha)
+        ref = orc.backward_alpha(x[i], g[i], b_ref, w.alpha)
+        tol = 1e-4 * abs(ref) + alpha_tol(x[i], g[i], b_ref, w.alpha)
+        assert abs(ga[i] - ref) <= tol, f"{name} row {i}: {ga[i]!r} vs {ref!r} (tol {tol:.3e})"
+
+
+def test_autograd_k_and_alpha_tensors(orc):
+    w, x, g = case("c1")
+    xt = torch.from_numpy(x.copy()).cuda().requires_grad_(True)
+    kt = torch.tensor(w.k, dtype=torch.float64, device="cuda", requires_grad=True)
+    at = torch.tensor(w.alpha, dtype=torch.float32, device="cuda", requires_grad=True)
+    p = lt.soft_topk(xt, kt, at)
+    (p * torch.from_numpy(g).cuda()).sum().backward()
+    _, b_ref, _ = orc.forward(x[0], w.k, w.alpha)
+    _, lam, _ = orc.backward(x[0], g[0], b_ref, w.alpha)
+    ref_a = orc.backward_alpha(x[0], g[0], b_ref, w.alpha)
+    assert kt.grad.shape == kt.shape and at.grad.shape == at.shape and at.grad.dtype == torch.float32
+    assert float(kt.grad) == pytest.approx(lam, rel=1e-4, abs=1e-6 * (1 + abs(lam)))
+    assert float(at.grad) == pytest.approx(ref_a, rel=1e-4, abs=alpha_tol(x[0], g[0], b_ref, w.alpha) + 1e-6)
+    assert xt.grad is not None and torch.isfinite(xt.grad).all()
