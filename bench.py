@@ -60,6 +60,7 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="c4", choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sparse", action="store_true", help="skip the sparse-forward comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="scale the workload to n scores per row (k keeps its ratio)")
@@ -343,6 +344,56 @@ def e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step, n_s
                     "upload/compute/download on three streams, two buffer sets, %d steps" % n_steps}
 
 
+def sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, steps, eps=2.0 ** -24):
+    """The forward alone, dense p against the sparse (index, p) output of the
+    entries with p >= eps, on the same row: K untraced steps each, every step
+    after the L2 flush.  Returns a small dict for the JSON line."""
+    rows, n = x.shape
+    p = torch.empty_like(x)
+    b = torch.empty(rows, dtype=torch.float64, device=dev)
+    sumf = torch.empty(rows, dtype=torch.float64, device=dev)
+    status = torch.empty(rows, dtype=torch.int32, device=dev)
+    ws = torch.empty(lt.sparse_workspace_size(rows, n), dtype=torch.uint8, device=dev)
+    first = lt.forward_sparse(x, w.k, w.alpha, eps, workspace=ws)
+    cap = int(first.count.max() * 1.05) + 1024
+    res = lt.forward_sparse(x, w.k, w.alpha, eps, capacity=cap, workspace=ws)
+    lib = lt._load()
+    stream = torch.cuda.current_stream(dev)
+
+    def sparse_step():
+        rc = lib.lapsum_topk_fwd_sparse(x.data_ptr(), rows, n, x.stride(0), float(w.k), float(w.alpha), float(eps),
+                                        res.idx.data_ptr(), res.val.data_ptr(), cap, res.count.data_ptr(),
+                                        b.data_ptr(), sumf.data_ptr(), status.data_ptr(), None, ws.data_ptr(),
+                                        ws.numel(), None, stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(lt.status_string(rc))
+
+    def dense_step():
+        lt.forward_into(x, w.k, w.alpha, p, b, sumf, status, ws)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ev = []
+        for i in range(steps):
+            flush.fill_(i & 0xFF)
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            fn()
+            s1.record(stream)
+            ev.append((s0, s1))
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / steps, dist, dev)
+
+    ms_dense = timed(dense_step)
+    ms_sparse = timed(sparse_step)
+    entries = int(res.count.max())
+    return {"eps": eps, "entries_per_row": entries, "capacity": cap,
+            "dense_forward_ms": ms_dense, "sparse_forward_ms": ms_sparse,
+            "sparse_scores_per_s": rows * n / (ms_sparse * 1e-3),
+            "bytes_written_dense": 4 * rows * n, "bytes_written_sparse": 8 * rows * entries}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -445,6 +496,10 @@ def main():
     kernels = {k: {"launches": v[0], "ms_per_launch": v[1] / v[0], "share": v[1] / sum(t[1] for t in trace.values())}
                for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])}
 
+    sparse = None
+    if not args.no_sparse and n > 16384:
+        sparse = sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, args.steps)
+
     e2e = None
     if not args.no_e2e:
         e2e = e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step)
@@ -486,6 +541,7 @@ def main():
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "sparse_forward": sparse,
         "gpu_launches": launches,
         "clocks": clk,
     }

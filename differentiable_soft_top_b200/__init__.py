@@ -19,6 +19,7 @@ lambda = sum g f / sum f.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import threading
 from dataclasses import dataclass
@@ -28,7 +29,8 @@ import numpy as np
 __all__ = [
     "Params", "ForwardResult", "forward", "backward", "forward_into", "backward_into", "soft_topk", "SoftTopK", "workspace_size",
     "status_string", "launch_count", "trace_enable", "trace_collect", "library_path", "STATS_DTYPE", "ROW_CERTIFIED", "ROW_WIDENED",
-    "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "FORCE_NONE", "FORCE_FALLBACK",
+    "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "ROW_TRUNCATED",
+    "forward_sparse", "SparseResult", "sparse_workspace_size", "FORCE_NONE", "FORCE_FALLBACK",
     "FORCE_STREAMING", "LapsumError",
 ]
 
@@ -38,6 +40,7 @@ _LIB_PATH = os.path.join(_PKG, "liblapsum_topk.so")
 LAPSUM_OK, LAPSUM_EINVAL, LAPSUM_EBADK, LAPSUM_EBADALPHA, LAPSUM_EWORKSPACE, LAPSUM_ECUDA, LAPSUM_ETOOLARGE = range(7)
 NOALLOC_MAX_ROWS, NOALLOC_MAX_N = 65536, 16384  # limits of forward_noalloc_into
 ROW_CERTIFIED, ROW_WIDENED, ROW_FALLBACK = 0x01, 0x02, 0x04
+ROW_TRUNCATED = 0x40
 ROW_NONFINITE, ROW_TIMEOUT, ROW_OVERFLOW = 0x08, 0x10, 0x20
 FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
 
@@ -117,6 +120,11 @@ def _load():
             lib.lapsum_topk_fwd.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, sz, P, P]
             lib.lapsum_topk_fwd.restype = ctypes.c_int
             lib.lapsum_topk_bwd.argtypes = [P, P, P, i64, i64, i64, dbl, P, P, P, P, sz, P]
+            lib.lapsum_topk_fwd_sparse.argtypes = [P, i64, i64, i64, dbl, dbl, ctypes.c_float, P, P, i64, P, P, P,
+                                                   P, P, P, sz, P, P]
+            lib.lapsum_topk_fwd_sparse.restype = ctypes.c_int
+            lib.lapsum_topk_sparse_workspace_size.argtypes = [i64, i64, P]
+            lib.lapsum_topk_sparse_workspace_size.restype = sz
             lib.lapsum_topk_bwd.restype = ctypes.c_int
             lib.lapsum_topk_fwd_noalloc.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, P]
             lib.lapsum_topk_fwd_noalloc.restype = ctypes.c_int
@@ -256,6 +264,65 @@ def forward(scores, k: float, alpha: float, *, params: Params | None = None, wor
     stats_np = st.cpu().numpy().view(STATS_DTYPE) if st is not None else None
     return ForwardResult(p.view(scores.shape) if p_out is None and scores.dim() == 1 else (p if p_out is None else p_out),
                          b, sumf, status, stats_np)
+
+
+@dataclass
+class SparseResult:
+    idx: object        # torch.Tensor int32 [rows, capacity]
+    val: object        # torch.Tensor float32 [rows, capacity]
+    count: object      # torch.Tensor int64 [rows]: entries with p >= eps (may exceed capacity)
+    b: object          # torch.Tensor float64 [rows]
+    sumf: object       # torch.Tensor float64 [rows]
+    status: object     # torch.Tensor int32 [rows]
+
+    def row(self, r: int):
+        """(indices, p) of row r as tensors of its written entries."""
+        c = min(int(self.count[r]), self.idx.shape[1])
+        return self.idx[r, :c], self.val[r, :c]
+
+
+def sparse_workspace_size(rows: int, n: int, params: Params | None = None) -> int:
+    c, ptr = _params_ptr(params)
+    return int(_load().lapsum_topk_sparse_workspace_size(int(rows), int(n), ptr))
+
+
+def forward_sparse(scores, k: float, alpha: float, eps: float = 2.0 ** -24, *, capacity: int | None = None,
+                   params: Params | None = None, workspace=None) -> SparseResult:
+    """The entries with p >= eps of every row of `scores` (CUDA fp32) as
+    (index, p) pairs; the threshold is that of forward().  With no capacity
+    given, 2k + 4096 per row is tried first and, if a row has more entries,
+    the call is repeated with the exact count (one host synchronisation)."""
+    torch = _torch()
+    lib = _load()
+    x = _as_rows(scores, "scores")
+    rows, n = x.shape
+    dev = x.device
+    guess = capacity is None
+    cap = int(min(n, 2 * math.ceil(k) + 4096)) if guess else int(capacity)
+    c, pptr = _params_ptr(params)
+    need = int(lib.lapsum_topk_sparse_workspace_size(rows, n, pptr))
+    ws = workspace if workspace is not None else _workspace(dev, need)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    while True:
+        idx = torch.empty((rows, cap), dtype=torch.int32, device=dev)
+        val = torch.empty((rows, cap), dtype=torch.float32, device=dev)
+        cnt = torch.empty(rows, dtype=torch.int64, device=dev)
+        b = torch.empty(rows, dtype=torch.float64, device=dev)
+        sumf = torch.empty(rows, dtype=torch.float64, device=dev)
+        status = torch.empty(rows, dtype=torch.int32, device=dev)
+        rc = lib.lapsum_topk_fwd_sparse(x.data_ptr(), rows, n, x.stride(0), float(k), float(alpha), float(eps),
+                                        idx.data_ptr(), val.data_ptr(), cap, cnt.data_ptr(), b.data_ptr(),
+                                        sumf.data_ptr(), status.data_ptr(), None, ws.data_ptr(), ws.numel(),
+                                        pptr, stream)
+        if rc != LAPSUM_OK:
+            raise LapsumError(rc, "lapsum_topk_fwd_sparse")
+        if not guess:
+            break
+        top = int(cnt.max())
+        if top <= cap:
+            break
+        cap, guess = top, False
+    return SparseResult(idx, val, cnt, b, sumf, status)
 
 
 def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None, want_alpha: bool = False):

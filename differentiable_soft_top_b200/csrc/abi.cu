@@ -201,59 +201,35 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return x < y + bn && y < x + an;
 }
 
-}  // namespace
-}  // namespace lapsum
-
-using namespace lapsum;
-
-extern "C" {
-
-void lapsum_default_params(lapsum_params* p) {
-  if (!p) return;
-  std::memset(p, 0, sizeof(*p));
-  p->z = 5.0;
-  p->max_widen = -1;
-}
-
-const char* lapsum_last_cuda_error(void) { return t_last_error; }
-
-const char* lapsum_status_string(int code) {
-  switch (code) {
-    case LAPSUM_OK: return "ok";
-    case LAPSUM_EINVAL: return "invalid argument (null or misaligned pointer, bad shape, or overlapping buffers)";
-    case LAPSUM_EBADK: return "k must be finite with 0 < k < n";
-    case LAPSUM_EBADALPHA: return "alpha must be finite and in [1e-30, 1e30]";
-    case LAPSUM_EWORKSPACE: return "workspace missing or smaller than lapsum_topk_workspace_size()";
-    case LAPSUM_ECUDA: return "a CUDA call or kernel launch failed";
-    case LAPSUM_ETOOLARGE: return "rows > LAPSUM_NOALLOC_MAX_ROWS or n > LAPSUM_NOALLOC_MAX_N for the allocation-free forward";
-    default: return "unknown status";
-  }
-}
-
-size_t lapsum_topk_workspace_size(int64_t rows, int64_t n, const lapsum_params* params) {
-  if (rows < 1 || n < 1 || n > INT32_MAX) return 0;
-  const Resolved R = resolve(params);
-  // k only shapes the band estimate; size for the widest case (k = n/2)
-  const size_t fwd = std::max(fwd_ws_bytes(rows, n, 0.5 * (double)n, R),
-                              std::max(fwd_ws_bytes(rows, n, 1.0, R), fwd_ws_bytes(rows, n, (double)n - 1.0, R)));
-  return std::max(fwd, bwd_ws_bytes(rows, n));
-}
-
-int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k, double alpha,
-                    float* p_out, double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
-                    void* workspace, size_t workspace_bytes, const lapsum_params* params, void* stream) {
-  if (!scores || !p_out || !b_out) return LAPSUM_EINVAL;
+// The forward pass behind lapsum_topk_fwd (sp == null: dense p) and
+// lapsum_topk_fwd_sparse (sp: the entries with p >= eps).
+int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k, double alpha, float* p_out,
+             double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
+             size_t workspace_bytes, const lapsum_params* params, void* stream, const SparseOut* sp) {
+  if (!scores || !b_out || (!sp && !p_out)) return LAPSUM_EINVAL;
   if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
   if (((uintptr_t)scores & 3u) || ((uintptr_t)p_out & 3u) || ((uintptr_t)b_out & 7u)) return LAPSUM_EINVAL;
+  if (sp) {
+    if (!sp->idx || !sp->val || !sp->count || sp->cap < 0) return LAPSUM_EINVAL;
+    if (((uintptr_t)sp->idx & 3u) || ((uintptr_t)sp->val & 3u) || ((uintptr_t)sp->count & 7u)) return LAPSUM_EINVAL;
+    if (!std::isfinite(sp->eps) || !(sp->eps > 0.0f) || !(sp->eps <= 1.0f)) return LAPSUM_EINVAL;
+    p_out = nullptr;
+  }
   if (sumf_out && ((uintptr_t)sumf_out & 7u)) return LAPSUM_EINVAL;
   if (!std::isfinite(k) || !(k > 0.0) || !(k < (double)n)) return LAPSUM_EBADK;
   if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
   const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
-  if (overlaps(scores, span, p_out, span)) return LAPSUM_EINVAL;
+  if (p_out && overlaps(scores, span, p_out, span)) return LAPSUM_EINVAL;
+  if (sp) {
+    const size_t ob = 4 * (size_t)sp->cap * (size_t)rows;
+    if (ob && (overlaps(scores, span, sp->idx, ob) || overlaps(scores, span, sp->val, ob) ||
+               overlaps(sp->idx, ob, sp->val, ob)))
+      return LAPSUM_EINVAL;
+  }
   const Resolved R = resolve(params);
   const bool res = resident_path(n, R);
   if (!res && rows > 65535) return LAPSUM_EINVAL;
-  const size_t need = fwd_ws_bytes(rows, n, k, R);
+  const size_t need = fwd_ws_bytes(rows, n, k, R) + ((sp && !res) ? align256(4 * (size_t)n) : 0);
   if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)) return LAPSUM_EWORKSPACE;
 
   DevInfo* dev = nullptr;
@@ -290,6 +266,7 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
     a.ws_status = reinterpret_cast<uint32_t*>(ws);
     a.fb_count = reinterpret_cast<uint32_t*>(ws + align256(4 * (size_t)rows));
     a.fb_list = reinterpret_cast<int32_t*>(ws + align256(4 * (size_t)rows) + 256);
+    if (sp) a.sp = *sp;
     if (resident_fwd_smem(a) + 1024 > (size_t)dev->smem_optin) return LAPSUM_EINVAL;
     return cuda_ok(launch_resident_fwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
   }
@@ -335,9 +312,76 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
   P.mpart = ws + L.mpart;
   P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
   P.fb_aggs = ws + L.fb_aggs;
+  if (sp) {
+    P.sp = *sp;
+    P.fb_keys2 = reinterpret_cast<uint32_t*>(ws + L.total);  // past the dense layout
+    P.Gms = stream_grid(sm, occ.memb_sparse_blocks, rows, n);
+  }
   P.rcount = reinterpret_cast<uint32_t*>(ws + L.rcount);
   return cuda_ok(launch_stream_fwd(P, scores, p_out, b_out, sumf_out, row_status, stats, sm, st)) ? LAPSUM_OK
                                                                                                 : LAPSUM_ECUDA;
+}
+
+}  // namespace
+}  // namespace lapsum
+
+using namespace lapsum;
+
+extern "C" {
+
+void lapsum_default_params(lapsum_params* p) {
+  if (!p) return;
+  std::memset(p, 0, sizeof(*p));
+  p->z = 5.0;
+  p->max_widen = -1;
+}
+
+const char* lapsum_last_cuda_error(void) { return t_last_error; }
+
+const char* lapsum_status_string(int code) {
+  switch (code) {
+    case LAPSUM_OK: return "ok";
+    case LAPSUM_EINVAL: return "invalid argument (null or misaligned pointer, bad shape, or overlapping buffers)";
+    case LAPSUM_EBADK: return "k must be finite with 0 < k < n";
+    case LAPSUM_EBADALPHA: return "alpha must be finite and in [1e-30, 1e30]";
+    case LAPSUM_EWORKSPACE: return "workspace missing or smaller than lapsum_topk_workspace_size()";
+    case LAPSUM_ECUDA: return "a CUDA call or kernel launch failed";
+    case LAPSUM_ETOOLARGE: return "rows > LAPSUM_NOALLOC_MAX_ROWS or n > LAPSUM_NOALLOC_MAX_N for the allocation-free forward";
+    default: return "unknown status";
+  }
+}
+
+int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k, double alpha,
+                    float* p_out, double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
+                    void* workspace, size_t workspace_bytes, const lapsum_params* params, void* stream) {
+  return fwd_impl(scores, rows, n, row_stride, k, alpha, p_out, b_out, sumf_out, row_status, stats, workspace,
+                  workspace_bytes, params, stream, nullptr);
+}
+
+int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k,
+                           double alpha, float eps, int32_t* idx_out, float* val_out, int64_t capacity,
+                           uint64_t* count_out, double* b_out, double* sumf_out, uint32_t* row_status,
+                           lapsum_row_stats* stats, void* workspace, size_t workspace_bytes,
+                           const lapsum_params* params, void* stream) {
+  const SparseOut sp{eps, idx_out, val_out, capacity, count_out};
+  return fwd_impl(scores, rows, n, row_stride, k, alpha, nullptr, b_out, sumf_out, row_status, stats, workspace,
+                  workspace_bytes, params, stream, &sp);
+}
+
+size_t lapsum_topk_sparse_workspace_size(int64_t rows, int64_t n, const lapsum_params* params) {
+  const size_t dense = lapsum_topk_workspace_size(rows, n, params);
+  if (dense == 0) return 0;
+  const Resolved R = resolve(params);
+  return dense + (resident_path(n, R) ? 0 : align256(4 * (size_t)n));
+}
+
+size_t lapsum_topk_workspace_size(int64_t rows, int64_t n, const lapsum_params* params) {
+  if (rows < 1 || n < 1 || n > INT32_MAX) return 0;
+  const Resolved R = resolve(params);
+  // k only shapes the band estimate; size for the widest case (k = n/2)
+  const size_t fwd = std::max(fwd_ws_bytes(rows, n, 0.5 * (double)n, R),
+                              std::max(fwd_ws_bytes(rows, n, 1.0, R), fwd_ws_bytes(rows, n, (double)n - 1.0, R)));
+  return std::max(fwd, bwd_ws_bytes(rows, n));
 }
 
 int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,

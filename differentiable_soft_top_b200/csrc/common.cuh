@@ -21,6 +21,7 @@ constexpr uint32_t ROW_FALLBACK = 0x04u;
 constexpr uint32_t ROW_NONFINITE = 0x08u;
 constexpr uint32_t ROW_TIMEOUT = 0x10u;
 constexpr uint32_t ROW_OVERFLOW = 0x20u;
+constexpr uint32_t ROW_TRUNCATED = 0x40u;  // sparse output: more entries than its capacity
 constexpr uint32_t ROW_PUBLIC = 0xFFu;
 constexpr uint32_t ROW_MISS_LEFT = 0x100u;   // S(a_L) < k: b lies below a_L
 constexpr uint32_t ROW_MISS_RIGHT = 0x200u;  // S(a_R) >= k: b lies at or above a_R

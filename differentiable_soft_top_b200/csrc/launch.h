@@ -35,6 +35,18 @@ class Launch {
 constexpr int64_t kResidentMaxN = 16384;
 constexpr int kResidentThreads = 256;
 
+// Sparse output of a forward pass: the entries with p >= eps as (index, p)
+// pairs, row r at r * cap; count[r] receives the number of such entries
+// (which may exceed cap: then only cap of them are written).  idx == null
+// means the dense output p.
+struct SparseOut {
+  float eps;
+  int32_t* idx;
+  float* val;
+  int64_t cap;
+  uint64_t* count;
+};
+
 struct ResidentFwd {
   const float* scores;
   int64_t rows, n, stride;
@@ -58,6 +70,7 @@ struct ResidentFwd {
   uint32_t* ws_status;   // [rows]
   uint32_t* fb_count;    // [1]
   int32_t* fb_list;      // [rows]
+  SparseOut sp;          // sparse output instead of p_out (sp.idx != null)
 };
 
 size_t resident_fwd_smem(const ResidentFwd& a);
@@ -101,8 +114,11 @@ struct StreamPlan {
   float* band;           // [rows][band_cap], unsorted
   void* mpart;           // membership partials [rows][Gm]
   uint32_t* fb_keys;     // [n] keys for the full-sort fallback
+  uint32_t* fb_keys2;    // [n] its second buffer when there is no dense p to borrow
   void* fb_aggs;         // GroupAgg [n / kFallbackGroup + 1]
   uint32_t* rcount;      // radix counts [256 * Gr] (+ scan space)
+  SparseOut sp;          // sparse output instead of p (sp.idx != null)
+  int Gms;               // grid of the sparse membership pass
 };
 
 constexpr int kFallbackGroup = 4096;   // full-sort fallback: sorted values per group
@@ -138,6 +154,7 @@ struct StreamOcc {
   int memb_blocks;      // of the membership pass
   int reduce_blocks;    // of the backward reduction
   int apply_blocks;     // of the backward elementwise pass
+  int memb_sparse_blocks;  // of the sparse membership pass
   int recover_blocks;   // of the cooperative recovery kernel
   int band_max_cluster; // largest cluster of band CTAs (power of two, <= 16)
 };

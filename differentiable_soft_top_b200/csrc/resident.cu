@@ -145,10 +145,47 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
-  float* dst = a.p_out + r * a.stride;
   double ps = 0.0;
   const bool nonfinite = (status & ROW_NONFINITE) != 0u;
-  if (a.vec) {
+  if (a.sp.idx) {
+    // sparse output, in index order: each thread takes 4 consecutive scores
+    // of a 4*NT window, a block scan places its hits
+    int32_t* oi = a.sp.idx + r * a.sp.cap;
+    float* ov = a.sp.val + r * a.sp.cap;
+    uint64_t total = 0;
+    uint32_t* scr = reinterpret_cast<uint32_t*>(red);
+    for (int i0 = 0; i0 < n; i0 += 4 * NT) {
+      float pv[4];
+      uint32_t hits = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = i0 + 4 * (int)threadIdx.x + j;
+        pv[j] = 0.0f;
+        if (i < n) {
+          pv[j] = nonfinite ? CUDART_NAN_F : membership(src[i], bh, bl, c2);
+          ps += (double)pv[j];
+          if (pv[j] >= a.sp.eps) hits |= 1u << j;
+        }
+      }
+      uint32_t tot;
+      uint64_t pos = total + block_excl_prefix_u32<NT>((uint32_t)__popc(hits), scr, &tot);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (hits & (1u << j)) {
+          if (pos < (uint64_t)a.sp.cap) {
+            oi[pos] = i0 + 4 * (int)threadIdx.x + j;
+            ov[pos] = pv[j];
+          }
+          ++pos;
+        }
+      }
+      total += tot;
+    }
+    if (total > (uint64_t)a.sp.cap) status |= ROW_TRUNCATED;
+    if (threadIdx.x == 0) a.sp.count[r] = total;
+    __syncthreads();
+  } else if (a.vec) {
+    float* dst = a.p_out + r * a.stride;
     const float4* s4 = reinterpret_cast<const float4*>(src);
     float4* d4 = reinterpret_cast<float4*>(dst);
     const int n4 = n >> 2;
@@ -169,6 +206,7 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
       dst[i] = p;
     }
   } else {
+    float* dst = a.p_out + r * a.stride;
     for (int i = threadIdx.x; i < n; i += NT) {
       const float p = nonfinite ? CUDART_NAN_F : membership(src[i], bh, bl, c2);
       ps += (double)p;

@@ -1164,7 +1164,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       const int64_t n = P.n;
       const float* src = scores + r * P.stride;
       uint32_t* A = P.fb_keys;
-      uint32_t* B = reinterpret_cast<uint32_t*>(p_out + r * P.stride);
+      uint32_t* B = p_out ? reinterpret_cast<uint32_t*>(p_out + r * P.stride) : P.fb_keys2;
       uint32_t* cnts = P.rcount;                          // [256][ncta]
       uint32_t* tots = P.rcount + 256 * (size_t)ncta;     // [256]
       const int64_t L = (n + ncta - 1) / ncta;
@@ -1271,27 +1271,80 @@ __device__ __forceinline__ float memb(float x, float bh, float bl, float c2) {
   return d < 0.0f ? h : 1.0f - h;
 }
 
+// Sparse mode: each warp stages its entries with p >= eps in its own slice of
+// shared memory (ballots place them, no atomics) and, once it holds
+// kSpFlush of them, reserves room in the row's output with one global atomic
+// and copies them out; no block-wide barrier is involved.  The order of the
+// entries is unspecified.
+constexpr int kSpFlush = 128;
+constexpr int kSpWarpStage = kSpFlush + 32 * 4;  // a step adds at most 4 per lane
+
+template <bool kSparse>
 __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __restrict__ scores,
                                               float* __restrict__ p_out, double* b_out, double* sumf_out,
                                               uint32_t* status_out, lapsum_row_stats* stats) {
   __shared__ double red[64];
+  __shared__ int32_t s_idx[kSparse ? NW * kSpWarpStage : 1];
+  __shared__ float s_val[kSparse ? NW * kSpWarpStage : 1];
   const int64_t r = blockIdx.y;
   RowCtl* c = ctl_of(P, r);
   const double b = c->b;
-  const uint32_t status = c->status;
+  uint32_t status = c->status;
   const bool nonfinite = (status & ROW_NONFINITE) != 0u;
   const double inva = 1.0 / P.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
   const float* row = scores + r * P.stride;
-  float* dst = p_out + r * P.stride;
+  float* dst = kSparse ? nullptr : p_out + r * P.stride;
   const int64_t n = P.n;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  int32_t* widx = s_idx + (kSparse ? warp * kSpWarpStage : 0);
+  float* wval = s_val + (kSparse ? warp * kSpWarpStage : 0);
+  uint32_t wn = 0u;  // entries in this warp's stage (the same in every lane)
   double ps = 0.0;
-  auto one = [&](int64_t i) {
-    const float p = nonfinite ? CUDART_NAN_F : memb(row[i], bh, bl, c2);
-    ps += (double)p;
-    dst[i] = p;
+  // sparse: stage this lane's hits (bit j of `hits`: index i0 + j, value pv[j])
+  auto append = [&](uint32_t hits, int64_t i0, const float* pv, int cnt) {
+    for (int j = 0; j < cnt; ++j) {
+      const uint32_t m = __ballot_sync(0xffffffffu, (hits >> j) & 1u);
+      if ((hits >> j) & 1u) {
+        const uint32_t pos = wn + (uint32_t)__popc(m & lt_mask);
+        widx[pos] = (int32_t)(i0 + j);
+        wval[pos] = pv[j];
+      }
+      wn += (uint32_t)__popc(m);
+    }
+  };
+  auto flush = [&](bool force) {
+    if (wn >= (uint32_t)kSpFlush || (force && wn > 0u)) {
+      __syncwarp();
+      unsigned long long gb = 0ull;
+      if (lane == 0) gb = atomicAdd(reinterpret_cast<unsigned long long*>(P.sp.count + r), (unsigned long long)wn);
+      gb = __shfl_sync(0xffffffffu, gb, 0);
+      int32_t* oi = P.sp.idx + r * P.sp.cap;
+      float* ov = P.sp.val + r * P.sp.cap;
+      for (uint32_t j = lane; j < wn; j += 32) {
+        if (gb + j < (unsigned long long)P.sp.cap) {
+          oi[gb + j] = widx[j];
+          ov[gb + j] = wval[j];
+        }
+      }
+      __syncwarp();
+      wn = 0u;
+    }
+  };
+  auto one = [&](int64_t i, bool act) {  // the scalar loops: every thread of the block calls it
+    float p = 0.0f;
+    if (act) {
+      p = nonfinite ? CUDART_NAN_F : memb(row[i], bh, bl, c2);
+      ps += (double)p;
+      if (!kSparse) dst[i] = p;
+    }
+    if (kSparse) {
+      append((act && p >= P.sp.eps) ? 1u : 0u, i, &p, 1);
+      flush(false);
+    }
   };
   if (P.vec) {
     const float4* x4 = reinterpret_cast<const float4*>(row);
@@ -1314,16 +1367,26 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
         p.w = memb(v[u].w, bh, bl, c2);
         if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
         pl += (p.x + p.y) + (p.z + p.w);
-        stg_stream(d4 + base + u * NT, p);
+        if (kSparse) {
+          const float pv[4] = {p.x, p.y, p.z, p.w};
+          uint32_t hits = 0u;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) hits |= (pv[j] >= P.sp.eps) ? (1u << j) : 0u;
+          append(hits, (base + u * NT) * 4, pv, 4);
+          flush(false);
+        } else {
+          stg_stream(d4 + base + u * NT, p);
+        }
       }
       ps += (double)pl;
     }
-    for (int64_t i = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n;
-         i += (int64_t)gridDim.x * NT)
-      one(i);
+    for (int64_t i0 = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT; i0 < n; i0 += (int64_t)gridDim.x * NT)
+      one(i0 + threadIdx.x, i0 + threadIdx.x < n);
   } else {
-    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) one(i);
+    for (int64_t i0 = (int64_t)blockIdx.x * NT; i0 < n; i0 += (int64_t)gridDim.x * NT)
+      one(i0 + threadIdx.x, i0 + threadIdx.x < n);
   }
+  if (kSparse) flush(true);
   ps = block_sum<NT, double>(ps, red);
   if (threadIdx.x == 0) mpart_of(P, r)[blockIdx.x] = MPart{ps, 0.0};
   if (last_block_done(&c->done_memb, gridDim.x)) {
@@ -1332,6 +1395,8 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
     for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) p += __ldcg(&mp[i].a);
     p = block_sum<NT, double>(p, red);
     if (threadIdx.x == 0) {
+      if (kSparse && *reinterpret_cast<volatile unsigned long long*>(P.sp.count + r) > (unsigned long long)P.sp.cap)
+        status |= ROW_TRUNCATED;
       const double bo = nonfinite ? CUDART_NAN : b;
       const double so = nonfinite ? CUDART_NAN : c->sumf;
       const uint32_t pub = status & ROW_PUBLIC;
@@ -1519,7 +1584,10 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   int fb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb, NT, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb<false>, NT, 0);
+  if (e != cudaSuccess) return e;
+  int sb = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sb, k_memb<true>, NT, 0);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&qb, k_bwd_reduce<false>, NT, 0);
   if (e != cudaSuccess) return e;
@@ -1529,6 +1597,7 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   if (e != cudaSuccess) return e;
   out->filter_blocks = std::max(fb, 1);
   out->memb_blocks = std::max(mb, 1);
+  out->memb_sparse_blocks = std::max(sb, 1);
   out->reduce_blocks = std::max(qb, 1);
   out->apply_blocks = std::max(ab, 1);
   out->recover_blocks = std::max(rb, 1);
@@ -1606,8 +1675,15 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     if (e != cudaSuccess) return e;
   }
   {
-    Launch l("k_memb", st);
-    k_memb<<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+    if (P.sp.idx) {
+      e = cudaMemsetAsync(P.sp.count, 0, sizeof(uint64_t) * (size_t)P.rows, st);
+      if (e != cudaSuccess) return e;
+      Launch l("k_memb_sparse", st);
+      k_memb<true><<<dim3(P.Gms, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+    } else {
+      Launch l("k_memb", st);
+      k_memb<false><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+    }
   }
   return cudaGetLastError();
 }

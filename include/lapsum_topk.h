@@ -76,6 +76,9 @@ extern "C" {
                                        of this row are unspecified */
 #define LAPSUM_ROW_OVERFLOW 0x20u   /* informational: the band outgrew its
                                        capacity (the row then took the fallback) */
+#define LAPSUM_ROW_TRUNCATED 0x40u  /* sparse forward: the row has more entries
+                                       with p >= eps than the capacity; its
+                                       count is still the full number */
 
 /* ---- tuning and test knobs --------------------------------------------- */
 typedef struct lapsum_params {
@@ -144,6 +147,36 @@ LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int
                     double k, double alpha, float* p_out, double* b_out, double* sumf_out,
                     uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
                     size_t workspace_bytes, const lapsum_params* params, void* stream);
+
+/*
+ * Sparse forward pass: the same threshold b, but instead of the dense p only
+ * the entries with p_i >= eps, as (index, p_i) pairs.  Downstream top-k uses
+ * need about k + O(alpha * density) such entries per row instead of n, and
+ * the membership pass then writes those instead of 4n bytes per row.
+ *
+ *   eps         in   0 < eps <= 1 (e.g. 2^-24: every p_i below it is dropped)
+ *   idx_out     out  int32 [rows, capacity]: row-local indices, row r at
+ *                    r * capacity; ascending when the row takes the
+ *                    one-block path (n <= 16384), in unspecified order otherwise
+ *   val_out     out  fp32 [rows, capacity]: p at those indices
+ *   capacity    in   entries per row of idx_out / val_out (>= 0)
+ *   count_out   out  uint64 [rows]: the number of entries with p >= eps.  If it
+ *                    exceeds capacity, only capacity of them are written (which
+ *                    ones is unspecified) and the row gets LAPSUM_ROW_TRUNCATED
+ *   workspace   in   at least lapsum_topk_sparse_workspace_size() bytes
+ * The other arguments are those of lapsum_topk_fwd (there is no p_out).
+ * Returns LAPSUM_OK or an error code (nothing enqueued on error).
+ */
+LAPSUM_API int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                                      double k, double alpha, float eps, int32_t* idx_out, float* val_out,
+                                      int64_t capacity, uint64_t* count_out, double* b_out, double* sumf_out,
+                                      uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
+                                      size_t workspace_bytes, const lapsum_params* params, void* stream);
+
+/* Workspace bytes of lapsum_topk_fwd_sparse: that of the dense forward plus,
+   for rows longer than 16384 scores, 4n bytes the full-sort fallback uses in
+   place of the dense p row. */
+LAPSUM_API size_t lapsum_topk_sparse_workspace_size(int64_t rows, int64_t n, const lapsum_params* params);
 
 /*
  * Backward pass (vector-Jacobian product) for the b a forward pass returned.

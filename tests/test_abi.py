@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     assert names == sorted([
         "lapsum_default_params", "lapsum_last_cuda_error", "lapsum_launch_count", "lapsum_status_string",
-        "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc", "lapsum_topk_workspace_size",
+        "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc", "lapsum_topk_fwd_sparse",
+        "lapsum_topk_sparse_workspace_size", "lapsum_topk_workspace_size",
         "lapsum_trace_collect", "lapsum_trace_enable",
     ])
 
@@ -128,6 +129,31 @@ def test_bwd_rejects_bad_arguments(lib):
     assert call(out=FAKE + 64) == lt.LAPSUM_EINVAL  # overlaps the scores
     assert call(wsb=16) == lt.LAPSUM_EWORKSPACE
     assert call(ga=FAKE * 5 + 4) == lt.LAPSUM_EINVAL  # misaligned dL/dalpha output
+
+
+def test_sparse_fwd_rejects_bad_arguments(lib):
+    F = lib.lapsum_topk_fwd_sparse
+    ok = dict(s=FAKE, rows=1, n=100000, stride=100000, k=40.0, a=0.5, eps=2.0 ** -24, idx=FAKE * 64,
+              val=FAKE * 128, cap=1000, cnt=FAKE * 192, b=FAKE * 200, ws=FAKE * 256, wsb=1 << 31)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return F(d["s"], d["rows"], d["n"], d["stride"], d["k"], d["a"], d["eps"], d["idx"], d["val"], d["cap"],
+                 d["cnt"], d["b"], None, None, None, d["ws"], d["wsb"], None, None)
+
+    assert call(idx=None) == lt.LAPSUM_EINVAL
+    assert call(cnt=None) == lt.LAPSUM_EINVAL
+    assert call(cnt=FAKE * 192 + 4) == lt.LAPSUM_EINVAL
+    assert call(eps=0.0) == lt.LAPSUM_EINVAL
+    assert call(eps=1.5) == lt.LAPSUM_EINVAL
+    assert call(eps=float("nan")) == lt.LAPSUM_EINVAL
+    assert call(cap=-1) == lt.LAPSUM_EINVAL
+    assert call(idx=FAKE + 16) == lt.LAPSUM_EINVAL  # overlaps the scores
+    assert call(k=0.0) == lt.LAPSUM_EBADK
+    # the dense forward's workspace is too small: the fallback needs 4n more
+    assert call(wsb=lt.workspace_size(1, 100000)) == lt.LAPSUM_EWORKSPACE
+    assert lt.sparse_workspace_size(1, 100000) == lt.workspace_size(1, 100000) + 400128
+    assert lt.sparse_workspace_size(4, 4096) == lt.workspace_size(4, 4096)
 
 
 def test_binding_rejects_cpu_tensors():

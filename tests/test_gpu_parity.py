@@ -370,3 +370,73 @@ def test_autograd_k_and_alpha_tensors(orc):
     assert float(kt.grad) == pytest.approx(lam, rel=1e-4, abs=1e-6 * (1 + abs(lam)))
     assert float(at.grad) == pytest.approx(ref_a, rel=1e-4, abs=alpha_tol(x[0], g[0], b_ref, w.alpha) + 1e-6)
     assert xt.grad is not None and torch.isfinite(xt.grad).all()
+
+
+# ---------------------------------------------------------------------------
+# sparse forward: the entries with p >= eps as (index, p) pairs
+# ---------------------------------------------------------------------------
+EPS = 2.0 ** -24
+
+
+@pytest.mark.parametrize("name,n,rows,force", [
+    ("c1", None, None, 0),
+    ("c1", 4096, 3, lt.FORCE_STREAMING),
+    ("c2", None, None, 0),
+    ("c3", 2_000_003, None, 0),
+    ("c5", 16384, 4, 0),
+    ("c2", 100_003, 2, 0),
+])
+def test_sparse_forward_matches_dense_and_oracle(orc, name, n, rows, force):
+    w, x, _ = case(name, n=n, rows=rows)
+    xt = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    params = lt.Params(force_path=force) if force else None
+    dense = lt.forward(xt, w.k, w.alpha, params=params)
+    sp = lt.forward_sparse(xt, w.k, w.alpha, EPS, capacity=x.shape[1], params=params)
+    torch.cuda.synchronize()
+    assert torch.equal(sp.b, dense.b) and torch.equal(sp.status, dense.status)
+    p_dense = dense.p.view(x.shape).cpu().numpy()
+    resident = x.shape[1] <= 16384 and not force
+    for i in range(x.shape[0]):
+        idx, val = (t.cpu().numpy() for t in sp.row(i))
+        want = np.nonzero(p_dense[i] >= EPS)[0]
+        assert int(sp.count[i]) == want.size
+        assert np.array_equal(np.sort(idx), want), f"{name} row {i}: index sets differ"
+        assert np.array_equal(val, p_dense[i][idx])  # same arithmetic as the dense pass
+        if resident:
+            assert np.all(np.diff(idx) > 0)  # index order on the one-block path
+        p_ref, _, _ = orc.forward(x[i], w.k, w.alpha)
+        assert np.max(np.abs(val - p_ref[idx])) <= 1e-5
+        sure = np.nonzero(p_ref >= EPS * (1 + 1e-3) + 1e-5)[0]
+        assert np.all(np.isin(sure, idx))
+
+
+@pytest.mark.parametrize("name,n", [("c1", None), ("c2", None)])
+def test_sparse_forward_truncates_and_reports(orc, name, n):
+    w, x, _ = case(name, n=n)
+    xt = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    full = lt.forward_sparse(xt, w.k, w.alpha, EPS, capacity=x.shape[1])
+    torch.cuda.synchronize()
+    total = int(full.count[0])
+    cap = total // 3
+    part = lt.forward_sparse(xt, w.k, w.alpha, EPS, capacity=cap)
+    torch.cuda.synchronize()
+    assert int(part.count[0]) == total
+    assert int(part.status[0]) & lt.ROW_TRUNCATED
+    assert not int(full.status[0]) & lt.ROW_TRUNCATED
+    idx, val = (t.cpu().numpy() for t in part.row(0))
+    assert idx.size == cap and np.unique(idx).size == cap
+    fi, fv = (t.cpu().numpy() for t in full.row(0))
+    ref = dict(zip(fi.tolist(), fv.tolist()))
+    assert all(ref[int(j)] == v for j, v in zip(idx, val))
+
+
+def test_sparse_forward_default_capacity_retries(orc):
+    """The binding's default capacity (2k + 4096) is too small for a wide
+    transition; it then repeats the call with the exact count."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((1, 200_000)).astype(np.float32)
+    xt = torch.from_numpy(x).cuda()
+    sp = lt.forward_sparse(xt, 10.0, 5.0, EPS)  # alpha 5: most entries are non-negligible
+    torch.cuda.synchronize()
+    assert sp.idx.shape[1] == int(sp.count[0]) > 2 * 10 + 4096
+    assert not int(sp.status[0]) & lt.ROW_TRUNCATED
