@@ -71,6 +71,7 @@ def _bind(lib):
         "lo_bracket": (ctypes.c_int, [_P, _i64, _dbl, _dbl, _i64, _dbl, _u64, _i64, _P, _P, _P, _P]),
         "lo_tails": (None, [_P, _i64, ctypes.c_float, ctypes.c_float, _dbl, _P, _P, _P, _P, _P]),
         "lo_dftopk_threshold_f32": (ctypes.c_int, [_P, _i64, _i64, _P]),
+        "lo_dftopk_forward_f32": (ctypes.c_int, [_P, _i64, _i64, _dbl, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -219,6 +220,15 @@ class Oracle:
         self.lib.lo_tails(p, a.size, float(aL), float(aR), float(alpha), ctypes.byref(nL),
                           ctypes.byref(SL), ctypes.byref(nR), ctypes.byref(SR), ctypes.byref(M))
         return nL.value, SL.value, nR.value, SR.value, M.value
+
+    def dftopk_forward(self, r, k: int, alpha: float):
+        """DFTopK memberships (fp64), threshold (the midpoint) and mass sum p."""
+        a, pa = _vec(r, np.float32)
+        p = np.empty(a.size, np.float64)
+        b, mass = _dbl(), _dbl()
+        _check(self.lib.lo_dftopk_forward_f32(pa, a.size, int(k), float(alpha), p.ctypes.data, ctypes.byref(b),
+                                              ctypes.byref(mass)))
+        return p, b.value, mass.value
 
     def dftopk_threshold(self, r, k: int) -> float:
         a, p = _vec(r, np.float32)

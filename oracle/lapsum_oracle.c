@@ -418,3 +418,27 @@ int lo_dftopk_threshold_f32(const float* r, int64_t n, int64_t k, double* b_out)
     free(x);
     return LO_OK;
 }
+
+
+/*
+ * The DFTopK relaxation (technical summary section 2.3): the threshold is
+ * fixed at that midpoint instead of solving the budget, and the memberships
+ * are the same Laplace CDF at scale alpha; their mass sum_i p_i is then free
+ * to drift from k.
+ */
+int lo_dftopk_forward_f32(const float* r, int64_t n, int64_t k, double alpha, double* p_out, double* b_out,
+                          double* mass_out) {
+    if (!isfinite(alpha) || !(alpha > 0.0)) return LO_EBADALPHA;
+    double b;
+    int rc = lo_dftopk_threshold_f32(r, n, k, &b);
+    if (rc != LO_OK) return rc;
+    nsum mass = {0.0, 0.0};
+    for (int64_t i = 0; i < n; ++i) {
+        const double p = lap_cdf(((double)r[i] - b) / alpha);
+        if (p_out) p_out[i] = p;
+        nsum_add(&mass, p);
+    }
+    if (b_out) *b_out = b;
+    if (mass_out) *mass_out = nsum_get(&mass);
+    return LO_OK;
+}

@@ -262,6 +262,35 @@ def test_zero_temperature_limit(orc, n, k):
     assert np.max(np.abs(p - mask)) <= 1e-6
 
 
+# DFTopK (section 2.3): midpoint threshold, no budget; the mass drifts
+def test_dftopk_limits(orc):
+    rng = np.random.default_rng(11)
+    r = rng.standard_normal(3000).astype(np.float32)
+    k = 40
+    xs = np.sort(r.astype(np.float64))[::-1]
+    p, b, mass = orc.dftopk_forward(r, k, 1e-9)
+    assert b == 0.5 * (xs[k - 1] + xs[k])
+    assert mass == pytest.approx(k, abs=1e-6)           # zero temperature: the hard top-k
+    assert np.array_equal(p >= 0.5, r.astype(np.float64) > b)
+    _, _, mass_hot = orc.dftopk_forward(r, k, 1e9)
+    assert mass_hot == pytest.approx(r.size / 2, rel=1e-6)  # infinite temperature: every p -> 1/2
+    _, _, mass_mid = orc.dftopk_forward(r, k, 0.5)
+    assert mass_mid > k                                  # the drift the pages cite: mass above k here
+    # the LapSum threshold at the same alpha keeps the budget the midpoint loses
+    _, b_lap, _ = orc.forward(r, float(k), 0.5)
+    assert orc.S(r, b_lap, 0.5) == pytest.approx(k, rel=1e-12)
+
+
+def test_dftopk_symmetric_pair(orc):
+    """r = (-d, d), k = 1: b = 0, p = (e^{-d/a}/2, 1 - e^{-d/a}/2), mass 1."""
+    d, a = 0.8, 0.25
+    p, b, mass = orc.dftopk_forward(np.array([-d, d], np.float32), 1, a)
+    e = 0.5 * math.exp(-float(np.float32(d)) / a)
+    assert b == 0.0
+    assert p[0] == pytest.approx(e, rel=1e-14) and p[1] == pytest.approx(1 - e, rel=1e-14)
+    assert mass == pytest.approx(1.0, rel=1e-15)
+
+
 # ---------------------------------------------------------------------------
 # finite differences for the analytic VJP (section 2.1)
 # ---------------------------------------------------------------------------
