@@ -61,6 +61,7 @@ def parse():
     ap.add_argument("--workload", default="c4", choices=sorted(WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sparse", action="store_true", help="skip the sparse-forward comparison")
+    ap.add_argument("--no-dftopk", action="store_true", help="skip the DFTopK-relaxation comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="scale the workload to n scores per row (k keeps its ratio)")
@@ -344,6 +345,58 @@ def e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step, n_s
                     "upload/compute/download on three streams, two buffer sets, %d steps" % n_steps}
 
 
+def timed_calls(torch, fn, steps, flush, stream, dist, dev):
+    """Mean device ms of fn() over `steps` calls (3 untimed first), each after
+    the L2 flush, CUDA events on `stream`, max over ranks."""
+    for _ in range(3):
+        fn()
+    ev = []
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        fn()
+        s1.record(stream)
+        ev.append((s0, s1))
+    torch.cuda.synchronize(dev)
+    return max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / steps, dist, dev)
+
+
+def dftopk_vs_lapsum(lt, torch, w, x, dev, dist, flush, steps):
+    """The DFTopK relaxation (threshold at the midpoint of the k-th and
+    (k+1)-th largest, memberships at alpha) against the exact-budget forward on
+    the same rows: forward time of each and the mass sum p each keeps."""
+    rows, n = x.shape
+    k = int(round(w.k))
+    p = torch.empty_like(x)
+    b = torch.empty(rows, dtype=torch.float64, device=dev)
+    sumf = torch.empty(rows, dtype=torch.float64, device=dev)
+    mass = torch.empty(rows, dtype=torch.float64, device=dev)
+    status = torch.empty(rows, dtype=torch.int32, device=dev)
+    ws = torch.empty(lt.workspace_size(rows, n), dtype=torch.uint8, device=dev)
+    lib = lt._load()
+    stream = torch.cuda.current_stream(dev)
+
+    def df_step():
+        rc = lib.lapsum_dftopk_fwd(x.data_ptr(), rows, n, x.stride(0), k, float(w.alpha), p.data_ptr(), b.data_ptr(),
+                                   sumf.data_ptr(), mass.data_ptr(), status.data_ptr(), None, ws.data_ptr(),
+                                   ws.numel(), None, stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(lt.status_string(rc))
+
+    def exact_step():
+        lt.forward_into(x, float(k), w.alpha, p, b, sumf, status, ws)
+
+    ms_exact = timed_calls(torch, exact_step, steps, flush, stream, dist, dev)
+    mass_exact = float(p.double().sum())
+    ms_df = timed_calls(torch, df_step, steps, flush, stream, dist, dev)
+    mass_df = float(mass.sum())
+    return {"k": k * rows, "exact_forward_ms": ms_exact, "dftopk_forward_ms": ms_df,
+            "exact_mass": mass_exact, "dftopk_mass": mass_df,
+            "exact_mass_rel_err": abs(mass_exact - k * rows) / (k * rows),
+            "dftopk_mass_rel_err": abs(mass_df - k * rows) / (k * rows)}
+
+
 def sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, steps, eps=2.0 ** -24):
     """The forward alone, dense p against the sparse (index, p) output of the
     entries with p >= eps, on the same row: K untraced steps each, every step
@@ -371,22 +424,8 @@ def sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, steps, eps=2.0 **
     def dense_step():
         lt.forward_into(x, w.k, w.alpha, p, b, sumf, status, ws)
 
-    def timed(fn):
-        for _ in range(3):
-            fn()
-        ev = []
-        for i in range(steps):
-            flush.fill_(i & 0xFF)
-            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            s0.record(stream)
-            fn()
-            s1.record(stream)
-            ev.append((s0, s1))
-        torch.cuda.synchronize(dev)
-        return max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / steps, dist, dev)
-
-    ms_dense = timed(dense_step)
-    ms_sparse = timed(sparse_step)
+    ms_dense = timed_calls(torch, dense_step, steps, flush, stream, dist, dev)
+    ms_sparse = timed_calls(torch, sparse_step, steps, flush, stream, dist, dev)
     entries = int(res.count.max())
     return {"eps": eps, "entries_per_row": entries, "capacity": cap,
             "dense_forward_ms": ms_dense, "sparse_forward_ms": ms_sparse,
@@ -499,6 +538,9 @@ def main():
     sparse = None
     if not args.no_sparse and n > 16384:
         sparse = sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, args.steps)
+    dftopk = None
+    if not args.no_dftopk:
+        dftopk = dftopk_vs_lapsum(lt, torch, w, x, dev, dist, flush, args.steps)
 
     e2e = None
     if not args.no_e2e:
@@ -542,6 +584,7 @@ def main():
         "cpu_baseline": cpu,
         "e2e": e2e,
         "sparse_forward": sparse,
+        "dftopk_forward": dftopk,
         "gpu_launches": launches,
         "clocks": clk,
     }

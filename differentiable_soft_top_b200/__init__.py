@@ -31,7 +31,7 @@ __all__ = [
     "status_string", "launch_count", "trace_enable", "trace_collect", "library_path", "STATS_DTYPE", "ROW_CERTIFIED", "ROW_WIDENED",
     "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "ROW_TRUNCATED",
     "forward_sparse", "SparseResult", "sparse_workspace_size", "FORCE_NONE", "FORCE_FALLBACK",
-    "FORCE_STREAMING", "LapsumError",
+    "FORCE_STREAMING", "LapsumError", "dftopk_forward", "DFTopKResult",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -128,6 +128,8 @@ def _load():
             lib.lapsum_topk_bwd.restype = ctypes.c_int
             lib.lapsum_topk_fwd_noalloc.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, P]
             lib.lapsum_topk_fwd_noalloc.restype = ctypes.c_int
+            lib.lapsum_dftopk_fwd.argtypes = [P, i64, i64, i64, i64, dbl, P, P, P, P, P, P, P, sz, P, P]
+            lib.lapsum_dftopk_fwd.restype = ctypes.c_int
             lib.lapsum_status_string.argtypes = [ctypes.c_int]
             lib.lapsum_status_string.restype = ctypes.c_char_p
             lib.lapsum_last_cuda_error.argtypes = []
@@ -264,6 +266,44 @@ def forward(scores, k: float, alpha: float, *, params: Params | None = None, wor
     stats_np = st.cpu().numpy().view(STATS_DTYPE) if st is not None else None
     return ForwardResult(p.view(scores.shape) if p_out is None and scores.dim() == 1 else (p if p_out is None else p_out),
                          b, sumf, status, stats_np)
+
+
+@dataclass
+class DFTopKResult:
+    p: object          # torch.Tensor, same shape as scores
+    b: object          # torch.Tensor float64 [rows]: midpoint of the k-th and (k+1)-th largest
+    sumf: object       # torch.Tensor float64 [rows]: sum f at alpha
+    mass: object       # torch.Tensor float64 [rows]: sum p (drifts from k)
+    status: object     # torch.Tensor int32 [rows]
+
+
+def dftopk_forward(scores, k: int, alpha: float, *, params: Params | None = None,
+                   workspace=None) -> DFTopKResult:
+    """The DFTopK relaxation of every row of `scores` (CUDA fp32): threshold at
+    the midpoint of the k-th and (k+1)-th largest score, Laplace memberships
+    at scale alpha around it, and their drifted mass (integer 1 <= k < n)."""
+    torch = _torch()
+    lib = _load()
+    if int(k) != k:
+        raise ValueError("k must be an integer for the DFTopK relaxation")
+    x = _as_rows(scores, "scores")
+    rows, n = x.shape
+    dev = x.device
+    p = _like_rows(x)
+    b = torch.empty(rows, dtype=torch.float64, device=dev)
+    sumf = torch.empty(rows, dtype=torch.float64, device=dev)
+    mass = torch.empty(rows, dtype=torch.float64, device=dev)
+    status = torch.empty(rows, dtype=torch.int32, device=dev)
+    c, pptr = _params_ptr(params)
+    need = int(lib.lapsum_topk_workspace_size(rows, n, pptr))
+    ws = workspace if workspace is not None else _workspace(dev, need)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = lib.lapsum_dftopk_fwd(x.data_ptr(), rows, n, x.stride(0), int(k), float(alpha), p.data_ptr(),
+                               b.data_ptr(), sumf.data_ptr(), mass.data_ptr(), status.data_ptr(), None,
+                               ws.data_ptr(), ws.numel(), pptr, stream)
+    if rc != LAPSUM_OK:
+        raise LapsumError(rc, "lapsum_dftopk_fwd")
+    return DFTopKResult(p.view(scores.shape) if scores.dim() == 1 else p, b, sumf, mass, status)
 
 
 @dataclass

@@ -54,6 +54,8 @@ cudaError_t device_info(DevInfo** out) {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr double kDftopkSolveAlpha = 1e-30;  // the smallest scale the solver accepts
+
 // the text of the last failed CUDA call on this host thread
 thread_local const char* t_last_error = "no error";
 bool cuda_ok(cudaError_t e) {
@@ -167,7 +169,7 @@ StreamLayout stream_layout(int64_t rows, int64_t n, const StreamSizes& s) {
   L.samp = o;    o = align256(o + 4 * (size_t)s.m * (size_t)rows);
   L.fpart = o;   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
   L.band = o;    o = align256(o + 4 * (size_t)s.band_cap * (size_t)rows);
-  L.mpart = o;   o = align256(o + 16 * (size_t)kMaxGridPerRow * (size_t)rows);
+  L.mpart = o;   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
   L.fb_keys = o; o = align256(o + 4 * (size_t)n);
   L.fb_aggs = o; o = align256(o + sizeof(GroupAgg) * (size_t)(n / kFallbackGroup + 2));
   L.rcount = o;  o = align256(o + 4 * (256 * (size_t)kMaxGridPerRow + 512));
@@ -201,11 +203,13 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return x < y + bn && y < x + an;
 }
 
-// The forward pass behind lapsum_topk_fwd (sp == null: dense p) and
-// lapsum_topk_fwd_sparse (sp: the entries with p >= eps).
+// The forward pass behind lapsum_topk_fwd (sp == null: dense p),
+// lapsum_topk_fwd_sparse (sp: the entries with p >= eps) and lapsum_dftopk_fwd
+// (dftopk: b solved at the tiny scale `alpha`, memberships at alpha_p).
 int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k, double alpha, float* p_out,
              double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
-             size_t workspace_bytes, const lapsum_params* params, void* stream, const SparseOut* sp) {
+             size_t workspace_bytes, const lapsum_params* params, void* stream, const SparseOut* sp,
+             double alpha_p, bool dftopk, double* sump_out) {
   if (!scores || !b_out || (!sp && !p_out)) return LAPSUM_EINVAL;
   if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
   if (((uintptr_t)scores & 3u) || ((uintptr_t)p_out & 3u) || ((uintptr_t)b_out & 7u)) return LAPSUM_EINVAL;
@@ -216,6 +220,7 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
     p_out = nullptr;
   }
   if (sumf_out && ((uintptr_t)sumf_out & 7u)) return LAPSUM_EINVAL;
+  if (sump_out && ((uintptr_t)sump_out & 7u)) return LAPSUM_EINVAL;
   if (!std::isfinite(k) || !(k > 0.0) || !(k < (double)n)) return LAPSUM_EBADK;
   if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
   const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
@@ -267,6 +272,9 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
     a.fb_count = reinterpret_cast<uint32_t*>(ws + align256(4 * (size_t)rows));
     a.fb_list = reinterpret_cast<int32_t*>(ws + align256(4 * (size_t)rows) + 256);
     if (sp) a.sp = *sp;
+    a.alpha_p = alpha_p;
+    a.dftopk = dftopk ? 1 : 0;
+    a.sump_out = sump_out;
     if (resident_fwd_smem(a) + 1024 > (size_t)dev->smem_optin) return LAPSUM_EINVAL;
     return cuda_ok(launch_resident_fwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
   }
@@ -312,6 +320,9 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   P.mpart = ws + L.mpart;
   P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
   P.fb_aggs = ws + L.fb_aggs;
+  P.alpha_p = alpha_p;
+  P.dftopk = dftopk ? 1 : 0;
+  P.sump_out = sump_out;
   if (sp) {
     P.sp = *sp;
     P.fb_keys2 = reinterpret_cast<uint32_t*>(ws + L.total);  // past the dense layout
@@ -355,7 +366,7 @@ int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_st
                     float* p_out, double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
                     void* workspace, size_t workspace_bytes, const lapsum_params* params, void* stream) {
   return fwd_impl(scores, rows, n, row_stride, k, alpha, p_out, b_out, sumf_out, row_status, stats, workspace,
-                  workspace_bytes, params, stream, nullptr);
+                  workspace_bytes, params, stream, nullptr, alpha, false, nullptr);
 }
 
 int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k,
@@ -365,7 +376,19 @@ int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t n, int64_t
                            const lapsum_params* params, void* stream) {
   const SparseOut sp{eps, idx_out, val_out, capacity, count_out};
   return fwd_impl(scores, rows, n, row_stride, k, alpha, nullptr, b_out, sumf_out, row_status, stats, workspace,
-                  workspace_bytes, params, stream, &sp);
+                  workspace_bytes, params, stream, &sp, alpha, false, nullptr);
+}
+
+int lapsum_dftopk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t k, double alpha,
+                      float* p_out, double* b_out, double* sumf_out, double* mass_out, uint32_t* row_status,
+                      lapsum_row_stats* stats, void* workspace, size_t workspace_bytes, const lapsum_params* params,
+                      void* stream) {
+  if (k < 1 || k >= n) return LAPSUM_EBADK;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  // the budget solve at a vanishing scale lands on the midpoint of the k-th
+  // and (k+1)-th largest scores (closed form: mid + (a/2) ln(A/B), a -> 0)
+  return fwd_impl(scores, rows, n, row_stride, (double)k, kDftopkSolveAlpha, p_out, b_out, sumf_out, row_status,
+                  stats, workspace, workspace_bytes, params, stream, nullptr, alpha, true, mass_out);
 }
 
 size_t lapsum_topk_sparse_workspace_size(int64_t rows, int64_t n, const lapsum_params* params) {
@@ -526,6 +549,7 @@ extern "C" int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_
   a.seed = R.seed;
   a.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
   a.vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  a.alpha_p = alpha;
   // same layout as the caller-workspace forward: statuses, counter, row list
   const size_t list_off = align256(4 * (size_t)rows);
   if (2 * list_off + 256 > kNoAllocBytes) return LAPSUM_ETOOLARGE;

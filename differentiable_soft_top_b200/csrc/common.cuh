@@ -402,6 +402,57 @@ __device__ __forceinline__ void shift_add_z(float a, float g, float z, float& m,
 }
 
 template <int NT>
+__device__ __forceinline__ double block_min_double(double v, double* scratch) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmin(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  double t = (lane < NW) ? scratch[lane] : CUDART_INF;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) t = fmin(t, __shfl_xor_sync(0xffffffffu, t, o));
+  return t;
+}
+
+// Sum of exp(-|x - b|/alpha) over a set of scores, kept relative to the
+// nearest distance seen so far (d_min, S: the sum is exp(-d_min/alpha) S), so
+// that it underflows only where the fp64 sum itself does.  b = bh + bl as two
+// floats; each distance is formed as an unevaluated float pair (error-free
+// two-sum), so the differences to d_min that go through the fp32 exp2 are
+// exact to about 2^-48 of the distance even when distance/alpha is large.
+__device__ __forceinline__ void near_add(float x, float bh, float bl, float c2, float& mh, float& ml, double& S) {
+  const float s = x - bh;  // exact near b
+  const float nb = -bl;
+  float dh = s + nb;
+  const float bv = dh - s;
+  float dl = (s - (dh - bv)) + (nb - bv);
+  if (dh < 0.0f || (dh == 0.0f && dl < 0.0f)) {
+    dh = -dh;
+    dl = -dl;
+  }
+  if (dh < mh) {  // a new nearest score: rescale what was accumulated
+    S *= (double)exp2f(((dh - mh) + (dl - ml)) * c2);
+    mh = dh;
+    ml = dl;
+  }
+  S += (double)exp2f(((mh - dh) + (ml - dl)) * c2);
+}
+// the nearest distance of a thread's pair as one fp64 value (+inf if none)
+__device__ __forceinline__ double near_dist(float mh, float ml) {
+  return mh < CUDART_INF_F ? (double)mh + (double)ml : CUDART_INF;
+}
+// the same pair over a block: every thread gets the block's (d_min, S)
+template <int NT>
+__device__ __forceinline__ void block_near_reduce(double& dmin, double& S, double inva, double* red) {
+  const double M = block_min_double<NT>(dmin, red);
+  const double sc = (dmin < CUDART_INF) ? exp_call((M - dmin) * inva) : 0.0;
+  S = block_sum<NT, double>(S * sc, red);
+  dmin = M;
+}
+
+template <int NT>
 __device__ __forceinline__ float block_min_float(float v, float* scratch) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -71,6 +71,10 @@ struct ResidentFwd {
   uint32_t* fb_count;    // [1]
   int32_t* fb_list;      // [rows]
   SparseOut sp;          // sparse output instead of p_out (sp.idx != null)
+  double alpha_p;        // scale of the memberships (alpha except for DFTopK)
+  int dftopk;            // memberships around a threshold solved at a tiny alpha:
+                         // sum f is taken in the membership pass at alpha_p
+  double* sump_out;      // [rows] sum p (may be null)
 };
 
 size_t resident_fwd_smem(const ResidentFwd& a);
@@ -119,6 +123,9 @@ struct StreamPlan {
   uint32_t* rcount;      // radix counts [256 * Gr] (+ scan space)
   SparseOut sp;          // sparse output instead of p (sp.idx != null)
   int Gms;               // grid of the sparse membership pass
+  double alpha_p;        // scale of the memberships (alpha except for DFTopK)
+  int dftopk;            // sum f taken in the membership pass at alpha_p
+  double* sump_out;      // [rows] sum p (may be null)
 };
 
 constexpr int kFallbackGroup = 4096;   // full-sort fallback: sorted values per group

@@ -141,12 +141,21 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
                            uint32_t status, float aL, float aR, long long nL, long long nR, long long M,
                            double SL, double SR, int buckets, double* red) {
   const int n = (int)a.n;
-  const double inva = 1.0 / a.alpha;
+  const double inva = 1.0 / a.alpha_p;
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
   double ps = 0.0;
   const bool nonfinite = (status & ROW_NONFINITE) != 0u;
+  if (a.dftopk) {
+    // sum f at the membership scale alpha_p, relative to the score nearest b
+    float mh = CUDART_INF_F, ml = 0.0f;
+    double S = 0.0;
+    for (int i = threadIdx.x; i < n; i += NT) near_add(src[i], bh, bl, c2, mh, ml, S);
+    double dmin = near_dist(mh, ml);
+    block_near_reduce<NT>(dmin, S, inva, red);
+    sumf = (dmin < CUDART_INF) ? 0.5 * inva * exp_call(-dmin * inva) * S : 0.0;
+  }
   if (a.sp.idx) {
     // sparse output, in index order: each thread takes 4 consecutive scores
     // of a 4*NT window, a block scan places its hits
@@ -219,6 +228,7 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
     const double so = nonfinite ? CUDART_NAN : sumf;
     a.b_out[r] = bo;
     if (a.sumf_out) a.sumf_out[r] = so;
+    if (a.sump_out) a.sump_out[r] = nonfinite ? CUDART_NAN : ps;
     if (a.status_out) a.status_out[r] = status & ROW_PUBLIC;
     if (a.stats) write_stats(a.stats + r, aL, aR, nL, nR, M, SL, SR, bo, ps, so, a.m, buckets, status & ROW_PUBLIC);
   }

@@ -47,7 +47,7 @@ struct FPart {
   uint32_t bad, pad;
 };
 struct MPart {
-  double a, b;
+  double a, b, c, pad;
 };
 
 __device__ __forceinline__ RowCtl* ctl_of(const StreamPlan& P, int64_t r) {
@@ -1270,6 +1270,17 @@ __device__ __forceinline__ float memb(float x, float bh, float bl, float c2) {
   const float h = 0.5f * exp2f(-fabsf(d) * c2);
   return d < 0.0f ? h : 1.0f - h;
 }
+// the same, also returning h = exp(-|x - b|/alpha)/2 and |x - b|
+__device__ __forceinline__ float memb_h(float x, float bh, float bl, float c2, float& h, float& ad) {
+  const float d = (x - bh) - bl;
+  ad = fabsf(d);
+  h = 0.5f * exp2f(-ad * c2);
+  return d < 0.0f ? h : 1.0f - h;
+}
+// A block whose nearest |x - b| is above this many alpha_p / ln 2 has every
+// fp32 term exp(-|x - b|/alpha_p) below 2^-64: it counts its sum f again,
+// relative to its nearest score (near_add), instead of from the fp32 terms.
+constexpr float kDfDeepLog2 = 64.0f;
 
 // Sparse mode: each warp stages its entries with p >= eps in its own slice of
 // shared memory (ballots place them, no atomics) and, once it holds
@@ -1279,7 +1290,11 @@ __device__ __forceinline__ float memb(float x, float bh, float bl, float c2) {
 constexpr int kSpFlush = 128;
 constexpr int kSpWarpStage = kSpFlush + 32 * 4;  // a step adds at most 4 per lane
 
-template <bool kSparse>
+// kDf: the DFTopK relaxation; sum f is also taken here, at alpha_p, from the
+// fp32 terms of the memberships, or (blocks far from b) relative to the
+// block's nearest score.  Per block MPart holds (sum p, S, d): the block's
+// sum of exp(-|x - b|/alpha_p) is exp(-d/alpha_p) S.
+template <bool kSparse, bool kDf>
 __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __restrict__ scores,
                                               float* __restrict__ p_out, double* b_out, double* sumf_out,
                                               uint32_t* status_out, lapsum_row_stats* stats) {
@@ -1291,12 +1306,14 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
   const double b = c->b;
   uint32_t status = c->status;
   const bool nonfinite = (status & ROW_NONFINITE) != 0u;
-  const double inva = 1.0 / P.alpha;
+  const double inva = 1.0 / P.alpha_p;
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
   const float* row = scores + r * P.stride;
   float* dst = kSparse ? nullptr : p_out + r * P.stride;
+  double hs = 0.0;             // kDf: sum of h = exp(-|x - b|/alpha_p)/2
+  float amin = CUDART_INF_F;   // kDf: nearest |x - b| of this thread
   const int64_t n = P.n;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t lt_mask = (1u << lane) - 1u;
@@ -1337,8 +1354,14 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
   auto one = [&](int64_t i, bool act) {  // the scalar loops: every thread of the block calls it
     float p = 0.0f;
     if (act) {
-      p = nonfinite ? CUDART_NAN_F : memb(row[i], bh, bl, c2);
+      float h, ad;
+      p = memb_h(row[i], bh, bl, c2, h, ad);
+      if (nonfinite) p = CUDART_NAN_F;
       ps += (double)p;
+      if (kDf) {
+        hs += (double)h;
+        amin = fminf(amin, ad);
+      }
       if (!kSparse) dst[i] = p;
     }
     if (kSparse) {
@@ -1357,16 +1380,21 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
       float4 v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) v[u] = __ldg(x4 + base + u * NT);
-      float pl = 0.0f;
+      float pl = 0.0f, hl = 0.0f;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float4 p;
-        p.x = memb(v[u].x, bh, bl, c2);
-        p.y = memb(v[u].y, bh, bl, c2);
-        p.z = memb(v[u].z, bh, bl, c2);
-        p.w = memb(v[u].w, bh, bl, c2);
+        float h0, h1, h2, h3, a0, a1, a2, a3;
+        p.x = memb_h(v[u].x, bh, bl, c2, h0, a0);
+        p.y = memb_h(v[u].y, bh, bl, c2, h1, a1);
+        p.z = memb_h(v[u].z, bh, bl, c2, h2, a2);
+        p.w = memb_h(v[u].w, bh, bl, c2, h3, a3);
         if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
         pl += (p.x + p.y) + (p.z + p.w);
+        if (kDf) {
+          hl += (h0 + h1) + (h2 + h3);
+          amin = fminf(amin, fminf(fminf(a0, a1), fminf(a2, a3)));
+        }
         if (kSparse) {
           const float pv[4] = {p.x, p.y, p.z, p.w};
           uint32_t hits = 0u;
@@ -1379,6 +1407,7 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
         }
       }
       ps += (double)pl;
+      if (kDf) hs += (double)hl;
     }
     for (int64_t i0 = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT; i0 < n; i0 += (int64_t)gridDim.x * NT)
       one(i0 + threadIdx.x, i0 + threadIdx.x < n);
@@ -1388,13 +1417,59 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
   }
   if (kSparse) flush(true);
   ps = block_sum<NT, double>(ps, red);
-  if (threadIdx.x == 0) mpart_of(P, r)[blockIdx.x] = MPart{ps, 0.0};
+  double dmin = 0.0;
+  if (kDf) {
+    const float M = block_min_float<NT>(amin, reinterpret_cast<float*>(red));
+    if (M * c2 > kDfDeepLog2) {
+      // every fp32 term of this block is tiny: count again relative to its
+      // nearest score (its values are read a second time)
+      float mh = CUDART_INF_F, ml = 0.0f;
+      double S = 0.0;
+      if (P.vec) {
+        const float4* x4 = reinterpret_cast<const float4*>(row);
+        const int64_t nchunks = (n >> 2) / CHUNK4;
+        for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
+          const int64_t base = (nchunks - 1 - q) * CHUNK4 + threadIdx.x;
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const float4 v = __ldg(x4 + base + u * NT);
+            near_add(v.x, bh, bl, c2, mh, ml, S);
+            near_add(v.y, bh, bl, c2, mh, ml, S);
+            near_add(v.z, bh, bl, c2, mh, ml, S);
+            near_add(v.w, bh, bl, c2, mh, ml, S);
+          }
+        }
+        for (int64_t i = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n;
+             i += (int64_t)gridDim.x * NT)
+          near_add(row[i], bh, bl, c2, mh, ml, S);
+      } else {
+        for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
+          near_add(row[i], bh, bl, c2, mh, ml, S);
+      }
+      dmin = near_dist(mh, ml);
+      block_near_reduce<NT>(dmin, S, inva, red);
+      hs = S;
+    } else {
+      hs = 2.0 * block_sum<NT, double>(hs, red);  // anchored at distance 0
+    }
+  }
+  if (threadIdx.x == 0) mpart_of(P, r)[blockIdx.x] = MPart{ps, hs, dmin, 0.0};
   if (last_block_done(&c->done_memb, gridDim.x)) {
     const MPart* mp = mpart_of(P, r);
-    double p = 0.0;
+    double p = 0.0, h = 0.0, hm = CUDART_INF;
     for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) p += __ldcg(&mp[i].a);
     p = block_sum<NT, double>(p, red);
+    if (kDf) {
+      for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) hm = fmin(hm, __ldcg(&mp[i].c));
+      hm = block_min_double<NT>(hm, red);
+      for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
+        const double di = __ldcg(&mp[i].c);
+        if (di < CUDART_INF) h += __ldcg(&mp[i].b) * exp_call((hm - di) * inva);
+      }
+      h = block_sum<NT, double>(h, red);
+    }
     if (threadIdx.x == 0) {
+      if (kDf) c->sumf = (hm < CUDART_INF) ? 0.5 * inva * exp_call(-hm * inva) * h : 0.0;
       if (kSparse && *reinterpret_cast<volatile unsigned long long*>(P.sp.count + r) > (unsigned long long)P.sp.cap)
         status |= ROW_TRUNCATED;
       const double bo = nonfinite ? CUDART_NAN : b;
@@ -1402,6 +1477,7 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
       const uint32_t pub = status & ROW_PUBLIC;
       b_out[r] = bo;
       if (sumf_out) sumf_out[r] = so;
+      if (P.sump_out) P.sump_out[r] = nonfinite ? CUDART_NAN : p;
       if (status_out) status_out[r] = pub;
       c->sump = p;
       if (stats) {
@@ -1584,10 +1660,10 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   int fb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
   if (e != cudaSuccess) return e;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb<false>, NT, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb<false, false>, NT, 0);
   if (e != cudaSuccess) return e;
   int sb = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sb, k_memb<true>, NT, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&sb, k_memb<true, false>, NT, 0);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&qb, k_bwd_reduce<false>, NT, 0);
   if (e != cudaSuccess) return e;
@@ -1679,10 +1755,13 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
       e = cudaMemsetAsync(P.sp.count, 0, sizeof(uint64_t) * (size_t)P.rows, st);
       if (e != cudaSuccess) return e;
       Launch l("k_memb_sparse", st);
-      k_memb<true><<<dim3(P.Gms, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+      k_memb<true, false><<<dim3(P.Gms, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
     } else {
-      Launch l("k_memb", st);
-      k_memb<false><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+      Launch l(P.dftopk ? "k_memb_dftopk" : "k_memb", st);
+      if (P.dftopk)
+        k_memb<false, true><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+      else
+        k_memb<false, false><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
     }
   }
   return cudaGetLastError();

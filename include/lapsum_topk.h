@@ -173,6 +173,32 @@ LAPSUM_API int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t
                                       uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
                                       size_t workspace_bytes, const lapsum_params* params, void* stream);
 
+/*
+ * DFTopK relaxation (Fast LapSum technical summary, section 2.3 "Relation to
+ * DFTopK"): the threshold is not solved for the budget at alpha but fixed at
+ * the midpoint of the k-th and (k+1)-th largest scores of the row, which is
+ * the zero-temperature limit of the LapSum threshold; the memberships are the
+ * same Laplace CDF around it at scale alpha, so their mass sum_i p_i is free
+ * to drift away from k.  Computed as the LapSum threshold at alpha = 1e-30
+ * (exactly the midpoint at fp64 resolution for fp32 scores), then one
+ * membership pass at the caller's alpha.
+ *
+ *   k           in   integer, 1 <= k <= n - 1
+ *   alpha       in   membership scale, [1e-30, 1e30]
+ *   b_out       out  fp64 [rows]  the midpoint threshold
+ *   sumf_out    out  fp64 [rows]  sum_i f_i at alpha (may be NULL)
+ *   mass_out    out  fp64 [rows]  sum_i p_i, the drifted mass (may be NULL)
+ * The other arguments, the workspace size (lapsum_topk_workspace_size) and
+ * the per-row status are those of lapsum_topk_fwd.  lapsum_topk_bwd with this
+ * b and alpha is NOT the gradient of this map (its threshold does not move
+ * with the scores the way the budget constraint makes it move).
+ * Returns LAPSUM_OK or an error code (nothing enqueued on error).
+ */
+LAPSUM_API int lapsum_dftopk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t k,
+                                 double alpha, float* p_out, double* b_out, double* sumf_out, double* mass_out,
+                                 uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
+                                 size_t workspace_bytes, const lapsum_params* params, void* stream);
+
 /* Workspace bytes of lapsum_topk_fwd_sparse: that of the dense forward plus,
    for rows longer than 16384 scores, 4n bytes the full-sort fallback uses in
    place of the dense p row. */

@@ -28,8 +28,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = declared_functions()
     assert names == sorted([
-        "lapsum_default_params", "lapsum_last_cuda_error", "lapsum_launch_count", "lapsum_status_string",
-        "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc", "lapsum_topk_fwd_sparse",
+        "lapsum_default_params", "lapsum_dftopk_fwd", "lapsum_last_cuda_error", "lapsum_launch_count",
+        "lapsum_status_string", "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc", "lapsum_topk_fwd_sparse",
         "lapsum_topk_sparse_workspace_size", "lapsum_topk_workspace_size",
         "lapsum_trace_collect", "lapsum_trace_enable",
     ])
@@ -154,6 +154,32 @@ def test_sparse_fwd_rejects_bad_arguments(lib):
     assert call(wsb=lt.workspace_size(1, 100000)) == lt.LAPSUM_EWORKSPACE
     assert lt.sparse_workspace_size(1, 100000) == lt.workspace_size(1, 100000) + 400128
     assert lt.sparse_workspace_size(4, 4096) == lt.workspace_size(4, 4096)
+
+
+def test_dftopk_fwd_rejects_bad_arguments(lib):
+    """Argument checks of the DFTopK forward (integer 1 <= k <= n-1, alpha in
+    range, the dense forward's pointer rules); none of them reaches a GPU."""
+    F = lib.lapsum_dftopk_fwd
+    ok = dict(s=FAKE, rows=1, n=100000, stride=100000, k=40, a=0.5, out=FAKE * 64, b=FAKE * 128, mass=FAKE * 192,
+              ws=FAKE * 256, wsb=1 << 31)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return F(d["s"], d["rows"], d["n"], d["stride"], d["k"], d["a"], d["out"], d["b"], None, d["mass"], None,
+                 None, d["ws"], d["wsb"], None, None)
+
+    assert call(k=0) == lt.LAPSUM_EBADK
+    assert call(k=100000) == lt.LAPSUM_EBADK
+    assert call(k=-3) == lt.LAPSUM_EBADK
+    assert call(a=0.0) == lt.LAPSUM_EBADALPHA
+    assert call(a=float("inf")) == lt.LAPSUM_EBADALPHA
+    assert call(a=1e-31) == lt.LAPSUM_EBADALPHA
+    assert call(out=None) == lt.LAPSUM_EINVAL
+    assert call(mass=FAKE * 192 + 4) == lt.LAPSUM_EINVAL  # misaligned mass output
+    assert call(out=FAKE + 64) == lt.LAPSUM_EINVAL  # overlaps the scores
+    assert call(wsb=16) == lt.LAPSUM_EWORKSPACE
+    with pytest.raises(ValueError):
+        lt.dftopk_forward(None, 2.5, 1.0)
 
 
 def test_binding_rejects_cpu_tensors():

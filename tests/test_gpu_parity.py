@@ -440,3 +440,103 @@ def test_sparse_forward_default_capacity_retries(orc):
     torch.cuda.synchronize()
     assert sp.idx.shape[1] == int(sp.count[0]) > 2 * 10 + 4096
     assert not int(sp.status[0]) & lt.ROW_TRUNCATED
+
+
+# ---------------------------------------------------------------------------
+# DFTopK relaxation (Fast LapSum technical summary, section 2.3): threshold at
+# the midpoint of the k-th and (k+1)-th largest, memberships at alpha
+# ---------------------------------------------------------------------------
+def dftopk_check(orc, r, k, alpha, res, i, label):
+    r = np.asarray(r, np.float32).reshape(-1)
+    p_ref, b_ref, mass_ref = orc.dftopk_forward(r, k, alpha)
+    b = float(res.b[i])
+    # the solve at alpha = 1e-30 lands on the midpoint up to fp64 rounding of
+    # b = x_k - (x_k - x_k+1)/2 + O(1e-30)
+    gap = float(np.max(np.abs(r))) if r.size else 1.0
+    assert abs(b - b_ref) <= 8 * np.finfo(np.float64).eps * max(abs(b_ref), gap), f"{label} b {b!r} vs {b_ref!r}"
+    p = res.p.view(-1, r.size)[i].cpu().numpy().astype(np.float64)
+    dp = float(np.max(np.abs(p - p_ref)))
+    assert dp <= 1e-5, f"{label} max|dp|={dp:.3e}"
+    # the mass: sums of the same fp32 memberships (partial sums of up to 16 in
+    # fp32 on the streaming path, each rounded to 2^-24 relative; fp64 above)
+    mass = float(res.mass[i])
+    assert abs(mass - math.fsum(p.tolist())) <= 1e-6 * max(1.0, mass)
+    assert abs(mass - mass_ref) <= 1e-5 * max(1.0, k) * max(1.0, math.sqrt(r.size / 1e6)), f"{label} mass"
+    x = r.astype(np.float64)
+    sumf_ref = math.fsum((0.5 * np.exp(-np.abs(x - b_ref) / alpha) / alpha).tolist())
+    assert float(res.sumf[i]) == pytest.approx(sumf_ref, rel=1e-5, abs=1e-300)
+    return mass_ref
+
+
+@pytest.mark.parametrize("name,n,rows,force", [
+    ("c1", None, None, 0),
+    ("c1", 4096, 3, lt.FORCE_STREAMING),
+    ("c2", None, None, 0),
+    ("c3", 2_000_003, None, 0),
+    ("c5", 16384, 4, 0),
+    ("c2", 100_003, 2, 0),
+])
+def test_dftopk_matches_oracle(orc, name, n, rows, force):
+    w, x, _ = case(name, n=n, rows=rows)
+    k = int(round(w.k))
+    xt = torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    params = lt.Params(force_path=force) if force else None
+    res = lt.dftopk_forward(xt, k, w.alpha, params=params)
+    torch.cuda.synchronize()
+    assert np.all(res.status.cpu().numpy() & lt.ROW_NONFINITE == 0)
+    for i in range(x.shape[0]):
+        dftopk_check(orc, x[i], k, w.alpha, res, i, f"{name} row {i}")
+
+
+@pytest.mark.parametrize("n,k,alpha", [
+    (2, 1, 0.5), (3, 1, 1e-3), (3, 2, 10.0), (4096, 1, 0.01), (4096, 4095, 0.01),
+    (100_000, 1, 1e-4), (100_000, 99_999, 0.3), (100_000, 50_000, 10.0), (300_001, 7, 1e-6),
+    # half-gap / alpha of a few hundred: sum f far below fp32 range, still in fp64
+    (5000, 2500, 5e-7), (300_001, 150_000, 1e-8),
+])
+def test_dftopk_edge_budgets(orc, n, k, alpha):
+    x = make_scores("normal", 1, n, seed=n + 29)
+    res = lt.dftopk_forward(torch.from_numpy(x).cuda(), k, alpha)
+    torch.cuda.synchronize()
+    dftopk_check(orc, x[0], k, alpha, res, 0, f"n={n} k={k}")
+
+
+def test_dftopk_sumf_mixes_near_and_far_blocks(orc):
+    """Uniform scores with alpha far below the typical spacing of a block:
+    the block holding the scores next to b sums its fp32 terms, the others
+    (every term below 2^-64) recount relative to their nearest score."""
+    n, k, alpha = 1_000_000, 500_000, 3e-8
+    x = make_scores("uniform", 1, n, seed=77)
+    res = lt.dftopk_forward(torch.from_numpy(x).cuda(), k, alpha)
+    torch.cuda.synchronize()
+    dftopk_check(orc, x[0], k, alpha, res, 0, "mixed blocks")
+
+
+@pytest.mark.parametrize("n", [5000, 300_000])
+def test_dftopk_ties_at_the_boundary(orc, n):
+    """k-th and (k+1)-th largest equal: the midpoint is that value."""
+    rng = np.random.default_rng(n)
+    x = np.round(rng.standard_normal((1, n)) * 4).astype(np.float32)  # heavy ties
+    k = n // 3
+    res = lt.dftopk_forward(torch.from_numpy(x).cuda(), k, 0.05)
+    torch.cuda.synchronize()
+    s = np.sort(x[0].astype(np.float64))[::-1]
+    assert s[k - 1] == s[k] and float(res.b[0]) == s[k]
+    dftopk_check(orc, x[0], k, 0.05, res, 0, f"ties n={n}")
+
+
+def test_dftopk_is_the_zero_temperature_limit_of_lapsum(orc):
+    """The midpoint equals the LapSum threshold at alpha = 1e-30, and at a
+    finite alpha the LapSum mass is k while the DFTopK mass drifts."""
+    w, x, _ = case("c2")
+    k = int(round(w.k))
+    xt = torch.from_numpy(x).cuda()
+    cold = lt.forward(xt, float(k), 1e-30)
+    d = lt.dftopk_forward(xt, k, w.alpha)
+    exact = lt.forward(xt, float(k), w.alpha)
+    torch.cuda.synchronize()
+    assert float(cold.b[0]) == float(d.b[0])
+    mass_exact = math.fsum(exact.p.view(-1).double().cpu().numpy().tolist())
+    assert abs(mass_exact - k) <= tol_sum(k, x.shape[1])
+    mass_ref = orc.dftopk_forward(x[0], k, w.alpha)[2]
+    assert float(d.mass[0]) == pytest.approx(mass_ref, rel=1e-6)
