@@ -29,7 +29,7 @@ import numpy as np
 __all__ = [
     "Params", "ForwardResult", "forward", "backward", "forward_into", "backward_into", "soft_topk", "SoftTopK", "workspace_size",
     "status_string", "launch_count", "trace_enable", "trace_collect", "library_path", "STATS_DTYPE", "ROW_CERTIFIED", "ROW_WIDENED",
-    "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "ROW_TRUNCATED",
+    "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "ROW_TRUNCATED", "ROW_BADARG",
     "forward_sparse", "SparseResult", "sparse_workspace_size", "FORCE_NONE", "FORCE_FALLBACK",
     "FORCE_STREAMING", "LapsumError", "dftopk_forward", "DFTopKResult",
 ]
@@ -41,6 +41,7 @@ LAPSUM_OK, LAPSUM_EINVAL, LAPSUM_EBADK, LAPSUM_EBADALPHA, LAPSUM_EWORKSPACE, LAP
 NOALLOC_MAX_ROWS, NOALLOC_MAX_N = 65536, 16384  # limits of forward_noalloc_into
 ROW_CERTIFIED, ROW_WIDENED, ROW_FALLBACK = 0x01, 0x02, 0x04
 ROW_TRUNCATED = 0x40
+ROW_BADARG = 0x80  # per-row k or alpha out of range: the row's outputs are NaN
 ROW_NONFINITE, ROW_TIMEOUT, ROW_OVERFLOW = 0x08, 0x10, 0x20
 FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
 
@@ -128,6 +129,10 @@ def _load():
             lib.lapsum_topk_bwd.restype = ctypes.c_int
             lib.lapsum_topk_fwd_noalloc.argtypes = [P, i64, i64, i64, dbl, dbl, P, P, P, P, P, P, P]
             lib.lapsum_topk_fwd_noalloc.restype = ctypes.c_int
+            lib.lapsum_topk_fwd_rows.argtypes = [P, i64, i64, i64, P, P, P, P, P, P, P, P, sz, P, P]
+            lib.lapsum_topk_fwd_rows.restype = ctypes.c_int
+            lib.lapsum_topk_bwd_rows.argtypes = [P, P, P, i64, i64, i64, P, P, P, P, P, sz, P]
+            lib.lapsum_topk_bwd_rows.restype = ctypes.c_int
             lib.lapsum_dftopk_fwd.argtypes = [P, i64, i64, i64, i64, dbl, P, P, P, P, P, P, P, sz, P, P]
             lib.lapsum_dftopk_fwd.restype = ctypes.c_int
             lib.lapsum_status_string.argtypes = [ctypes.c_int]
@@ -229,6 +234,31 @@ def _like_rows(x):
     return torch.empty_strided((rows, n), (x.stride(0), 1), dtype=x.dtype, device=x.device)
 
 
+def _per_row(v, rows, dev):
+    """v as a contiguous fp64 [rows] CUDA tensor when it is a 1-D tensor with
+    one value per row; None when it is a number or a single-value tensor."""
+    torch = _torch()
+    if not isinstance(v, torch.Tensor) or v.dim() == 0:
+        return None
+    if v.dim() != 1 or v.shape[0] != rows:
+        raise ValueError(f"a per-row k or alpha must have shape [{rows}], got {tuple(v.shape)}")
+    return v.detach().to(device=dev, dtype=torch.float64).contiguous()
+
+
+def _rows_pair(k, alpha, rows, dev):
+    """(k_rows, alpha_rows) for the *_rows entry points, or None when both are
+    scalars (a scalar beside a vector is broadcast)."""
+    torch = _torch()
+    kr, ar = _per_row(k, rows, dev), _per_row(alpha, rows, dev)
+    if kr is None and ar is None:
+        return None
+    if kr is None:
+        kr = torch.full((rows,), float(k), dtype=torch.float64, device=dev)
+    if ar is None:
+        ar = torch.full((rows,), float(alpha), dtype=torch.float64, device=dev)
+    return kr, ar
+
+
 @dataclass
 class ForwardResult:
     p: object          # torch.Tensor, same shape as scores
@@ -238,9 +268,11 @@ class ForwardResult:
     stats: np.ndarray | None = None  # STATS_DTYPE [rows], when requested
 
 
-def forward(scores, k: float, alpha: float, *, params: Params | None = None, workspace=None,
+def forward(scores, k, alpha, *, params: Params | None = None, workspace=None,
             stats: bool = False, p_out=None) -> ForwardResult:
-    """Thresholds and memberships for every row of `scores` (CUDA fp32)."""
+    """Thresholds and memberships for every row of `scores` (CUDA fp32).  k
+    and alpha are numbers, or [rows] tensors giving each row its own value
+    (rows with an out-of-range value get ROW_BADARG and NaN outputs)."""
     torch = _torch()
     lib = _load()
     x = _as_rows(scores, "scores")
@@ -257,12 +289,19 @@ def forward(scores, k: float, alpha: float, *, params: Params | None = None, wor
     need = int(lib.lapsum_topk_workspace_size(rows, n, pptr))
     ws = workspace if workspace is not None else _workspace(dev, need)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    rc = lib.lapsum_topk_fwd(x.data_ptr(), rows, n, x.stride(0), float(k), float(alpha), p.data_ptr(),
-                             b.data_ptr(), sumf.data_ptr(), status.data_ptr(),
-                             st.data_ptr() if st is not None else None, ws.data_ptr(), ws.numel(), pptr,
-                             stream)
+    pr = _rows_pair(k, alpha, rows, dev)
+    if pr is None:
+        rc = lib.lapsum_topk_fwd(x.data_ptr(), rows, n, x.stride(0), float(k), float(alpha), p.data_ptr(),
+                                 b.data_ptr(), sumf.data_ptr(), status.data_ptr(),
+                                 st.data_ptr() if st is not None else None, ws.data_ptr(), ws.numel(), pptr,
+                                 stream)
+    else:
+        rc = lib.lapsum_topk_fwd_rows(x.data_ptr(), rows, n, x.stride(0), pr[0].data_ptr(), pr[1].data_ptr(),
+                                      p.data_ptr(), b.data_ptr(), sumf.data_ptr(), status.data_ptr(),
+                                      st.data_ptr() if st is not None else None, ws.data_ptr(), ws.numel(), pptr,
+                                      stream)
     if rc != LAPSUM_OK:
-        raise LapsumError(rc, "lapsum_topk_fwd")
+        raise LapsumError(rc, "lapsum_topk_fwd" if pr is None else "lapsum_topk_fwd_rows")
     stats_np = st.cpu().numpy().view(STATS_DTYPE) if st is not None else None
     return ForwardResult(p.view(scores.shape) if p_out is None and scores.dim() == 1 else (p if p_out is None else p_out),
                          b, sumf, status, stats_np)
@@ -365,9 +404,10 @@ def forward_sparse(scores, k: float, alpha: float, eps: float = 2.0 ** -24, *, c
     return SparseResult(idx, val, cnt, b, sumf, status)
 
 
-def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None, want_alpha: bool = False):
+def backward(scores, grad_p, b, alpha, *, workspace=None, grad_out=None, want_alpha: bool = False):
     """dL/dscores and dL/dk (per row) for upstream gradient `grad_p` at
-    thresholds `b`; with want_alpha also dL/dalpha per row (a third result)."""
+    thresholds `b`; with want_alpha also dL/dalpha per row (a third result).
+    alpha: a number, or a [rows] tensor (one per row)."""
     torch = _torch()
     lib = _load()
     x = _as_rows(scores, "scores")
@@ -387,11 +427,17 @@ def backward(scores, grad_p, b, alpha: float, *, workspace=None, grad_out=None, 
     need = int(lib.lapsum_topk_workspace_size(rows, n, None))
     ws = workspace if workspace is not None else _workspace(dev, need)
     stream = torch.cuda.current_stream(dev).cuda_stream
-    rc = lib.lapsum_topk_bwd(x.data_ptr(), g.data_ptr(), bb.data_ptr(), rows, n, x.stride(0), float(alpha),
-                             out.data_ptr(), gk.data_ptr(), ga.data_ptr() if ga is not None else None,
-                             ws.data_ptr(), ws.numel(), stream)
+    ar = _per_row(alpha, rows, dev)
+    if ar is None:
+        rc = lib.lapsum_topk_bwd(x.data_ptr(), g.data_ptr(), bb.data_ptr(), rows, n, x.stride(0), float(alpha),
+                                 out.data_ptr(), gk.data_ptr(), ga.data_ptr() if ga is not None else None,
+                                 ws.data_ptr(), ws.numel(), stream)
+    else:
+        rc = lib.lapsum_topk_bwd_rows(x.data_ptr(), g.data_ptr(), bb.data_ptr(), rows, n, x.stride(0),
+                                      ar.data_ptr(), out.data_ptr(), gk.data_ptr(),
+                                      ga.data_ptr() if ga is not None else None, ws.data_ptr(), ws.numel(), stream)
     if rc != LAPSUM_OK:
-        raise LapsumError(rc, "lapsum_topk_bwd")
+        raise LapsumError(rc, "lapsum_topk_bwd" if ar is None else "lapsum_topk_bwd_rows")
     res = (out.view(scores.shape) if grad_out is None else grad_out), gk
     return res + (ga,) if want_alpha else res
 
@@ -452,8 +498,9 @@ def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None,
 
 class SoftTopK:
     """torch.autograd.Function wrapper: p = soft_topk(scores, k, alpha).  k
-    and alpha may be Python numbers or 0-d tensors; tensors that require grad
-    receive dL/dk (= sum over rows of lambda) and dL/dalpha."""
+    and alpha may be Python numbers, 0-d tensors (shared by all rows) or
+    [rows] tensors (one per row); tensors that require grad receive dL/dk
+    (lambda per row, summed over the rows for a shared k) and dL/dalpha."""
 
     _fn = None
 
@@ -465,10 +512,12 @@ class SoftTopK:
             class _F(torch.autograd.Function):
                 @staticmethod
                 def forward(ctx, scores, k, alpha, params):
-                    kf, af = float(k), float(alpha)
+                    rows = scores.shape[0] if scores.dim() == 2 else 1
+                    kf = k if isinstance(k, torch.Tensor) and k.dim() == 1 else float(k)
+                    af = alpha if isinstance(alpha, torch.Tensor) and alpha.dim() == 1 else float(alpha)
                     res = forward(scores, kf, af, params=params)
                     ctx.save_for_backward(scores, res.b)
-                    ctx.alpha = af
+                    ctx.alpha = af if not isinstance(af, torch.Tensor) else _per_row(af, rows, scores.device)
                     ctx.k_like = k if isinstance(k, torch.Tensor) else None
                     ctx.a_like = alpha if isinstance(alpha, torch.Tensor) else None
                     return res.p.view(scores.shape)
@@ -480,8 +529,12 @@ class SoftTopK:
                     need_k, need_a = ctx.needs_input_grad[1], ctx.needs_input_grad[2]
                     out = backward(sc, gp.contiguous().view(sc.shape), b, ctx.alpha, want_alpha=need_a)
                     gs, gk = out[0], out[1]
-                    grad_k = gk.sum().to(ctx.k_like.dtype).view(ctx.k_like.shape) if need_k else None
-                    grad_a = out[2].sum().to(ctx.a_like.dtype).view(ctx.a_like.shape) if need_a else None
+
+                    def fold(g, like):  # per row for a [rows] input, summed for a shared one
+                        return (g if like.dim() == 1 else g.sum()).to(like.dtype).view(like.shape)
+
+                    grad_k = fold(gk, ctx.k_like) if need_k else None
+                    grad_a = fold(out[2], ctx.a_like) if need_a else None
                     return gs.view(scores.shape), grad_k, grad_a, None
 
             cls._fn = _F
@@ -490,7 +543,8 @@ class SoftTopK:
 
 def soft_topk(scores, k, alpha, params: Params | None = None):
     """Differentiable exact-budget soft top-k memberships of `scores` (CUDA fp32).
-    k and alpha: numbers, or 0-d tensors when their gradients are wanted."""
+    k and alpha: numbers, 0-d tensors, or [rows] tensors (one per row); tensors
+    receive their gradients."""
     torch = _torch()
     k = k if isinstance(k, torch.Tensor) else float(k)
     alpha = alpha if isinstance(alpha, torch.Tensor) else float(alpha)

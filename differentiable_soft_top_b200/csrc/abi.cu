@@ -209,7 +209,8 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
 int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, double k, double alpha, float* p_out,
              double* b_out, double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
              size_t workspace_bytes, const lapsum_params* params, void* stream, const SparseOut* sp,
-             double alpha_p, bool dftopk, double* sump_out) {
+             double alpha_p, bool dftopk, double* sump_out, const double* k_rows = nullptr,
+             const double* alpha_rows = nullptr) {
   if (!scores || !b_out || (!sp && !p_out)) return LAPSUM_EINVAL;
   if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
   if (((uintptr_t)scores & 3u) || ((uintptr_t)p_out & 3u) || ((uintptr_t)b_out & 7u)) return LAPSUM_EINVAL;
@@ -221,6 +222,11 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   }
   if (sumf_out && ((uintptr_t)sumf_out & 7u)) return LAPSUM_EINVAL;
   if (sump_out && ((uintptr_t)sump_out & 7u)) return LAPSUM_EINVAL;
+  if (((uintptr_t)k_rows & 7u) || ((uintptr_t)alpha_rows & 7u)) return LAPSUM_EINVAL;
+  // per-row values are checked on the device; the host plans for the widest
+  // bracket (k = n/2) and takes the ranks of each row from its own k there
+  if (k_rows) k = 0.5 * (double)n;
+  if (alpha_rows) alpha = alpha_p = 1.0;
   if (!std::isfinite(k) || !(k > 0.0) || !(k < (double)n)) return LAPSUM_EBADK;
   if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
   const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
@@ -275,6 +281,9 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
     a.alpha_p = alpha_p;
     a.dftopk = dftopk ? 1 : 0;
     a.sump_out = sump_out;
+    a.k_rows = k_rows;
+    a.alpha_rows = alpha_rows;
+    a.z = R.z;
     if (resident_fwd_smem(a) + 1024 > (size_t)dev->smem_optin) return LAPSUM_EINVAL;
     return cuda_ok(launch_resident_fwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
   }
@@ -323,6 +332,9 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   P.alpha_p = alpha_p;
   P.dftopk = dftopk ? 1 : 0;
   P.sump_out = sump_out;
+  P.k_rows = k_rows;
+  P.alpha_rows = alpha_rows;
+  P.z = R.z;
   if (sp) {
     P.sp = *sp;
     P.fb_keys2 = reinterpret_cast<uint32_t*>(ws + L.total);  // past the dense layout
@@ -331,6 +343,61 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   P.rcount = reinterpret_cast<uint32_t*>(ws + L.rcount);
   return cuda_ok(launch_stream_fwd(P, scores, p_out, b_out, sumf_out, row_status, stats, sm, st)) ? LAPSUM_OK
                                                                                                 : LAPSUM_ECUDA;
+}
+
+// The backward behind lapsum_topk_bwd (one alpha) and lapsum_topk_bwd_rows
+// (alpha_rows: one per row, checked on the device).
+int bwd_impl(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
+             int64_t row_stride, double alpha, const double* alpha_rows, float* grad_scores, double* grad_k,
+             double* grad_alpha, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!scores || !grad_p || !b || !grad_scores) return LAPSUM_EINVAL;
+  if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
+  if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)grad_scores & 3u) ||
+      ((uintptr_t)b & 7u))
+    return LAPSUM_EINVAL;
+  if (grad_k && ((uintptr_t)grad_k & 7u)) return LAPSUM_EINVAL;
+  if (grad_alpha && ((uintptr_t)grad_alpha & 7u)) return LAPSUM_EINVAL;
+  if (alpha_rows) {
+    if ((uintptr_t)alpha_rows & 7u) return LAPSUM_EINVAL;
+    alpha = 1.0;
+  }
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
+  if (overlaps(scores, span, grad_scores, span) || overlaps(grad_p, span, grad_scores, span)) return LAPSUM_EINVAL;
+  const size_t need = bwd_ws_bytes(rows, n);
+  if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))) return LAPSUM_EWORKSPACE;
+  if (n > kResidentMaxN && rows > 65535) return LAPSUM_EINVAL;
+  DevInfo* dev = nullptr;
+  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
+  if (n <= kResidentMaxN) {
+    RowBwd a{scores, grad_p, b, rows, n, row_stride, alpha, grad_scores, grad_k, vec, grad_alpha, alpha_rows};
+    return cuda_ok(launch_resident_bwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
+  }
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  StreamBwd a{};
+  a.scores = scores;
+  a.grad_p = grad_p;
+  a.b = b;
+  a.rows = rows;
+  a.n = n;
+  a.stride = row_stride;
+  a.alpha = alpha;
+  a.grad = grad_scores;
+  a.grad_k = grad_k;
+  a.grad_alpha = grad_alpha;
+  a.alpha_rows = alpha_rows;
+  a.vec = vec;
+  a.Gb = stream_grid(dev->sm_count, dev->occ.reduce_blocks, rows, n);
+  a.Ga = stream_grid(dev->sm_count, dev->occ.apply_blocks, rows, n);
+  size_t o = 0;
+  a.part = ws + o;
+  o = align256(o + 48 * (size_t)kMaxGridPerRow * (size_t)rows);
+  a.done = reinterpret_cast<uint32_t*>(ws + o);
+  o = align256(o + 4 * (size_t)rows);
+  a.lam = reinterpret_cast<double*>(ws + o);
+  return cuda_ok(launch_stream_bwd(a, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
 }
 
 }  // namespace
@@ -379,6 +446,15 @@ int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t n, int64_t
                   workspace_bytes, params, stream, &sp, alpha, false, nullptr);
 }
 
+int lapsum_topk_fwd_rows(const float* scores, int64_t rows, int64_t n, int64_t row_stride, const double* k,
+                         const double* alpha, float* p_out, double* b_out, double* sumf_out, uint32_t* row_status,
+                         lapsum_row_stats* stats, void* workspace, size_t workspace_bytes,
+                         const lapsum_params* params, void* stream) {
+  if (!k || !alpha) return LAPSUM_EINVAL;
+  return fwd_impl(scores, rows, n, row_stride, 1.0, 1.0, p_out, b_out, sumf_out, row_status, stats, workspace,
+                  workspace_bytes, params, stream, nullptr, 1.0, false, nullptr, k, alpha);
+}
+
 int lapsum_dftopk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t k, double alpha,
                       float* p_out, double* b_out, double* sumf_out, double* mass_out, uint32_t* row_status,
                       lapsum_row_stats* stats, void* workspace, size_t workspace_bytes, const lapsum_params* params,
@@ -410,49 +486,16 @@ size_t lapsum_topk_workspace_size(int64_t rows, int64_t n, const lapsum_params* 
 int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
                     int64_t row_stride, double alpha, float* grad_scores, double* grad_k, double* grad_alpha,
                     void* workspace, size_t workspace_bytes, void* stream) {
-  if (!scores || !grad_p || !b || !grad_scores) return LAPSUM_EINVAL;
-  if (rows < 1 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
-  if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)grad_scores & 3u) ||
-      ((uintptr_t)b & 7u))
-    return LAPSUM_EINVAL;
-  if (grad_k && ((uintptr_t)grad_k & 7u)) return LAPSUM_EINVAL;
-  if (grad_alpha && ((uintptr_t)grad_alpha & 7u)) return LAPSUM_EINVAL;
-  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
-  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
-  if (overlaps(scores, span, grad_scores, span) || overlaps(grad_p, span, grad_scores, span)) return LAPSUM_EINVAL;
-  const size_t need = bwd_ws_bytes(rows, n);
-  if (need > 0 && (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u))) return LAPSUM_EWORKSPACE;
-  if (n > kResidentMaxN && rows > 65535) return LAPSUM_EINVAL;
-  DevInfo* dev = nullptr;
-  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
-  if (n <= kResidentMaxN) {
-    RowBwd a{scores, grad_p, b, rows, n, row_stride, alpha, grad_scores, grad_k, vec, grad_alpha};
-    return cuda_ok(launch_resident_bwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
-  }
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  StreamBwd a{};
-  a.scores = scores;
-  a.grad_p = grad_p;
-  a.b = b;
-  a.rows = rows;
-  a.n = n;
-  a.stride = row_stride;
-  a.alpha = alpha;
-  a.grad = grad_scores;
-  a.grad_k = grad_k;
-  a.grad_alpha = grad_alpha;
-  a.vec = vec;
-  a.Gb = stream_grid(dev->sm_count, dev->occ.reduce_blocks, rows, n);
-  a.Ga = stream_grid(dev->sm_count, dev->occ.apply_blocks, rows, n);
-  size_t o = 0;
-  a.part = ws + o;
-  o = align256(o + 48 * (size_t)kMaxGridPerRow * (size_t)rows);
-  a.done = reinterpret_cast<uint32_t*>(ws + o);
-  o = align256(o + 4 * (size_t)rows);
-  a.lam = reinterpret_cast<double*>(ws + o);
-  return cuda_ok(launch_stream_bwd(a, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
+  return bwd_impl(scores, grad_p, b, rows, n, row_stride, alpha, nullptr, grad_scores, grad_k, grad_alpha, workspace,
+                  workspace_bytes, stream);
+}
+
+int lapsum_topk_bwd_rows(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
+                         int64_t row_stride, const double* alpha, float* grad_scores, double* grad_k,
+                         double* grad_alpha, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!alpha) return LAPSUM_EINVAL;
+  return bwd_impl(scores, grad_p, b, rows, n, row_stride, 1.0, alpha, grad_scores, grad_k, grad_alpha, workspace,
+                  workspace_bytes, stream);
 }
 
 }  // extern "C"

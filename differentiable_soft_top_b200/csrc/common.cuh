@@ -22,6 +22,7 @@ constexpr uint32_t ROW_NONFINITE = 0x08u;
 constexpr uint32_t ROW_TIMEOUT = 0x10u;
 constexpr uint32_t ROW_OVERFLOW = 0x20u;
 constexpr uint32_t ROW_TRUNCATED = 0x40u;  // sparse output: more entries than its capacity
+constexpr uint32_t ROW_BADARG = 0x80u;     // per-row k or alpha out of range: outputs NaN
 constexpr uint32_t ROW_PUBLIC = 0xFFu;
 constexpr uint32_t ROW_MISS_LEFT = 0x100u;   // S(a_L) < k: b lies below a_L
 constexpr uint32_t ROW_MISS_RIGHT = 0x200u;  // S(a_R) >= k: b lies at or above a_R
@@ -61,6 +62,85 @@ __device__ __forceinline__ double laplace_noise(uint64_t s, uint64_t j, double a
   const double u = ((double)(d >> 11) + 0.5) * 0x1p-53;
   const double e = (u < 0.5) ? log(2.0 * u) : -log(2.0 - 2.0 * u);
   return alpha * e;
+}
+
+// ---------------------------------------------------------------------------
+// per-row budget and scale.  The method is stated for one vector with one k
+// and one alpha (technical summary section 2.1); a batch may give every row
+// its own.  An out-of-range value marks the row ROW_BADARG and is replaced by
+// a harmless one (k = n/2, alpha = 1) so that every pass still runs; the
+// row's outputs are NaN.
+// ---------------------------------------------------------------------------
+struct RowArgs {
+  double k;        // budget
+  double alpha;    // scale of the threshold solve
+  double alpha_p;  // scale of the memberships (differs for the DFTopK form)
+  bool bad;
+};
+__device__ __forceinline__ RowArgs row_args(double k, double alpha, double alpha_p, int dftopk,
+                                            const double* k_rows, const double* alpha_rows, int64_t r,
+                                            int64_t n) {
+  RowArgs a{k, alpha, alpha_p, false};
+  if (k_rows) {
+    const double kr = __ldg(k_rows + r);
+    if (kr > 0.0 && kr < (double)n) a.k = kr;  // NaN fails the test
+    else a.bad = true;
+  }
+  if (alpha_rows) {
+    const double ar = __ldg(alpha_rows + r);
+    if (ar >= 1e-30 && ar <= 1e30) {
+      a.alpha_p = ar;
+      if (!dftopk) a.alpha = ar;
+    } else {
+      a.bad = true;
+    }
+  }
+  if (a.bad) {
+    a.k = 0.5 * (double)n;
+    a.alpha = 1.0;
+    a.alpha_p = 1.0;
+  }
+  return a;
+}
+template <class Plan>
+__device__ __forceinline__ RowArgs row_args(const Plan& P, int64_t r) {
+  return row_args(P.k, P.alpha, P.alpha_p, P.dftopk, P.k_rows, P.alpha_rows, r, P.n);
+}
+// alpha of row r for the backward (no k there)
+__device__ __forceinline__ double row_alpha(double alpha, const double* alpha_rows, int64_t r, bool* bad) {
+  if (!alpha_rows) return alpha;
+  const double ar = __ldg(alpha_rows + r);
+  if (ar >= 1e-30 && ar <= 1e30) return ar;
+  *bad = true;
+  return 1.0;
+}
+
+// Localization ranks (section 2.2): #{Y > b} ~ Binomial(m, q = k/n); the
+// bracket edges are the c_lo-th and (c_hi+1)-th largest samples with
+// c_lo/hi = mq -/+ z sigma, as ascending indices.  Every operation is rounded
+// on its own (no fused multiply-add), the order of the host's computation,
+// so a row that gets its k from a vector has the ranks a scalar call gets.
+struct RowRanks {
+  int rank_lo, rank_hi, valid_lo, valid_hi, widen_delta;
+};
+__device__ __forceinline__ RowRanks sample_ranks_dev(int64_t n, double k, int m, double z) {
+  const double q = __ddiv_rn(k, (double)n);
+  const double mq = __dmul_rn((double)m, q);
+  const double sigma = __dsqrt_rn(__dmul_rn(mq, __dsub_rn(1.0, q)));
+  const long long c_lo = (long long)floor(__dsub_rn(mq, __dmul_rn(z, sigma)));
+  const long long c_hi = (long long)ceil(__dadd_rn(mq, __dmul_rn(z, sigma)));
+  RowRanks R;
+  R.valid_hi = c_lo >= 1;
+  R.rank_hi = R.valid_hi ? (int)(m - c_lo) : m - 1;
+  R.valid_lo = (c_hi + 1) <= m;
+  R.rank_lo = R.valid_lo ? (int)(m - c_hi - 1) : 0;
+  R.widen_delta = (int)ceil(__dmul_rn(__dmul_rn(2.0, z), sigma)) + 1;
+  return R;
+}
+template <class Plan>
+__device__ __forceinline__ RowRanks row_ranks(const Plan& P, double k) {
+  if (!P.k_rows) return RowRanks{P.rank_lo, P.rank_hi, P.valid_lo, P.valid_hi, P.widen_delta};
+  return sample_ranks_dev(P.n, k, P.m, P.z);
 }
 
 // ---------------------------------------------------------------------------

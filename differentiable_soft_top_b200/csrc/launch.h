@@ -75,6 +75,11 @@ struct ResidentFwd {
   int dftopk;            // memberships around a threshold solved at a tiny alpha:
                          // sum f is taken in the membership pass at alpha_p
   double* sump_out;      // [rows] sum p (may be null)
+  // per-row budget and scale (device [rows], or null: k and alpha above for
+  // every row); the ranks are then computed per row from z and m
+  const double* k_rows;
+  const double* alpha_rows;
+  double z;
 };
 
 size_t resident_fwd_smem(const ResidentFwd& a);
@@ -91,6 +96,7 @@ struct RowBwd {
   double* grad_k;
   int vec;
   double* grad_alpha;  // dL/dalpha per row, or null
+  const double* alpha_rows;  // per-row alpha (device [rows]) or null
 };
 cudaError_t launch_resident_bwd(const RowBwd& a, int sm_count, cudaStream_t st);
 
@@ -126,6 +132,9 @@ struct StreamPlan {
   double alpha_p;        // scale of the memberships (alpha except for DFTopK)
   int dftopk;            // sum f taken in the membership pass at alpha_p
   double* sump_out;      // [rows] sum p (may be null)
+  const double* k_rows;      // per-row k (device [rows]) or null
+  const double* alpha_rows;  // per-row alpha (device [rows]) or null
+  double z;                  // rank half-width in standard deviations
 };
 
 constexpr int kFallbackGroup = 4096;   // full-sort fallback: sorted values per group
@@ -147,6 +156,7 @@ struct StreamBwd {
   float* grad;
   double* grad_k;
   double* grad_alpha;  // dL/dalpha per row, or null
+  const double* alpha_rows;  // per-row alpha (device [rows]) or null
   int vec;
   int Gb, Ga;        // grids of the reduction and elementwise passes
   void* part;        // [rows][kMaxGridPerRow] partials (48 bytes each)

@@ -141,12 +141,14 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
                            uint32_t status, float aL, float aR, long long nL, long long nR, long long M,
                            double SL, double SR, int buckets, double* red) {
   const int n = (int)a.n;
-  const double inva = 1.0 / a.alpha_p;
+  const RowArgs ra = row_args(a, r);
+  if (ra.bad) status |= ROW_BADARG;
+  const double inva = 1.0 / ra.alpha_p;
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
   double ps = 0.0;
-  const bool nonfinite = (status & ROW_NONFINITE) != 0u;
+  const bool nonfinite = (status & (ROW_NONFINITE | ROW_BADARG)) != 0u;
   if (a.dftopk) {
     // sum f at the membership scale alpha_p, relative to the score nearest b
     float mh = CUDART_INF_F, ml = 0.0f;
@@ -250,7 +252,9 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   const int64_t r = blockIdx.x;
   const int n = (int)a.n;
   const float* src = a.scores + r * a.stride;
-  const double inva = 1.0 / a.alpha;
+  const RowArgs ra = row_args(a, r);
+  const RowRanks rr = row_ranks(a, ra.k);
+  const double inva = 1.0 / ra.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
 
   // ---- bring the row into shared memory --------------------------------
@@ -290,14 +294,14 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   const uint64_t s = row_stream(a.seed, (uint64_t)r);
   for (int j = threadIdx.x; j < m; j += NT) {
     const uint64_t I = sample_index(s, (uint64_t)j, (uint64_t)n);
-    const double Y = (double)row[I] + laplace_noise(s, (uint64_t)j, a.alpha);
+    const double Y = (double)row[I] + laplace_noise(s, (uint64_t)j, ra.alpha);
     samp[j] = f2key(__double2float_rn(Y));
   }
   __syncthreads();
   block_bitonic_sort<NT>(samp, m);  // samp and samp_tmp form one buffer of 2m keys
   const uint32_t* ss = samp;
-  int rlo = a.rank_lo, rhi = a.rank_hi;
-  bool vlo = a.valid_lo != 0, vhi = a.valid_hi != 0;
+  int rlo = rr.rank_lo, rhi = rr.rank_hi;
+  bool vlo = rr.valid_lo != 0, vhi = rr.valid_hi != 0;
   float aL = vlo ? key2f(ss[rlo]) : -CUDART_INF_F;
   float aR = vhi ? key2f(ss[rhi]) : CUDART_INF_F;
 
@@ -312,7 +316,7 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
       block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
       const uint32_t* bs = band;
       aggregate_sorted_keys<NT, false>(bs, f.M, red, &s_agg, inva);
-      SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, a.k, a.alpha, inva};
+      SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, ra.k, ra.alpha, inva};
       solve_band<NT, false>(in, &s_agg, 1, KeyRun{bs}, dscr, red, &s_out);
       if (s_out.status & ROW_CERTIFIED) { solved = true; break; }
       if (attempt >= a.max_widen) break;
@@ -321,13 +325,13 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
       status |= ROW_WIDENED;
       if (s_out.status & ROW_MISS_LEFT) {
         rhi = rlo; vhi = true; aR = aL;
-        rlo -= a.widen_delta;
+        rlo -= rr.widen_delta;
         vlo = rlo >= 0;
         if (!vlo) rlo = 0;
         aL = vlo ? key2f(ss[rlo]) : -CUDART_INF_F;
       } else {
         rlo = rhi; vlo = true; aL = aR;
-        rhi += a.widen_delta;
+        rhi += rr.widen_delta;
         vhi = rhi <= m - 1;
         if (!vhi) rhi = m - 1;
         aR = vhi ? key2f(ss[rhi]) : CUDART_INF_F;
@@ -378,11 +382,12 @@ __global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
   double* red = reinterpret_cast<double*>(smem + L.red);
   __shared__ SolveOut s_out;
   const int n = (int)a.n;
-  const double inva = 1.0 / a.alpha;
   const uint32_t cnt = *reinterpret_cast<volatile uint32_t*>(a.fb_count);
   for (uint32_t idx = blockIdx.x; idx < cnt; idx += gridDim.x) {
     const int64_t r = a.fb_list[idx];
     const float* src = a.scores + r * a.stride;
+    const RowArgs ra = row_args(a, r);
+    const double inva = 1.0 / ra.alpha;
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += NT) keys[i] = f2key(src[i]);
     __syncthreads();
@@ -391,7 +396,7 @@ __global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
     const int T = (n + kFbGroup - 1) / kFbGroup;
     for (int g = 0; g < T; ++g)
       aggregate_sorted_keys<NT, false>(sorted + g * kFbGroup, min(kFbGroup, n - g * kFbGroup), red, &aggs[g], inva);
-    SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, a.k, a.alpha, inva};
+    SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, ra.k, ra.alpha, inva};
     solve_band<NT, false>(in, aggs, T, KeyGroups{sorted, kFbGroup}, dscr, red, &s_out);
     const uint32_t status = a.ws_status[r] | ROW_FALLBACK | ROW_CERTIFIED;
     finish_row(a, r, src, s_out.b, s_out.sumf, status, -CUDART_INF_F, CUDART_INF_F, 0, 0, n, 0.0, 0.0, T, red);
@@ -407,10 +412,11 @@ template <bool kAlpha>
 __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
   __shared__ double red[64];
   const int n = (int)a.n;
-  const double inva = 1.0 / a.alpha;
-  const float c2 = (float)(inva * (double)kLog2e);
-  const float lg = (float)log2(0.5 * inva);
   for (int64_t r = blockIdx.x; r < a.rows; r += gridDim.x) {
+    bool bad = false;
+    const double inva = 1.0 / row_alpha(a.alpha, a.alpha_rows, r, &bad);
+    const float c2 = (float)(inva * (double)kLog2e);
+    const float lg = (float)log2(0.5 * inva);
     const float* x = a.scores + r * a.stride;
     const float* g = a.grad_p + r * a.stride;
     float* o = a.grad + r * a.stride;
@@ -449,7 +455,7 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     }
     if (kAlpha) block_shift_reduce4<NT>(m, S, SG, SZ, SGZ, red);
     else block_shift_reduce<NT>(m, S, SG, red);
-    const double lam = SG / S;
+    const double lam = bad ? CUDART_NAN : SG / S;  // NaN also reaches every grad of the row
     const float lh = __double2float_rn(lam);
     const float ll = __double2float_rn(lam - (double)lh);
     for (int v = threadIdx.x; v < n4; v += NT) {
@@ -465,7 +471,7 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT)
       o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
     if (threadIdx.x == 0 && a.grad_k) a.grad_k[r] = lam;
-    if (kAlpha && threadIdx.x == 0) a.grad_alpha[r] = alpha_grad((double)m, SZ, SGZ, lam, inva);
+    if (kAlpha && threadIdx.x == 0) a.grad_alpha[r] = bad ? CUDART_NAN : alpha_grad((double)m, SZ, SGZ, lam, inva);
     __syncthreads();
   }
 }

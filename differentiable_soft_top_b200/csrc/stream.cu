@@ -222,6 +222,7 @@ __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* 
   const float* row = scores + r * P.stride;
   const uint64_t s = row_stream(P.seed, (uint64_t)r);
   uint32_t* samp = samp_of(P, r);
+  const RowArgs ra = row_args(P, r);
   const int stride = gridDim.x * NT;
   for (int j0 = blockIdx.x * NT; j0 < P.m; j0 += 4 * stride) {
     float v[4];
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* 
       const bool act = j < P.m;
       uint32_t key = 0u;
       if (act) {
-        const double Y = (double)v[u] + laplace_noise(s, (uint64_t)j, P.alpha);
+        const double Y = (double)v[u] + laplace_noise(s, (uint64_t)j, ra.alpha);
         key = f2key(__double2float_rn(Y));
         samp[j] = key;
       }
@@ -246,7 +247,8 @@ __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* 
   flush_hist(sh, h1_of(P, r), 2048);
   RowCtl* c = ctl_of(P, r);
   if (last_block_done(&c->done_s1, gridDim.x)) {
-    const uint32_t rk[2] = {(uint32_t)P.rank_lo, (uint32_t)P.rank_hi};
+    const RowRanks rr = row_ranks(P, ra.k);
+    const uint32_t rk[2] = {(uint32_t)rr.rank_lo, (uint32_t)rr.rank_hi};
     int bin[2];
     uint32_t rem[2];
     sel_pick<2048>(h1_of(P, r), false, rk, scr, bin, rem);
@@ -283,7 +285,8 @@ __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
     uint32_t rem[2];
     sel_pick<1024>(h3_of(P, r), true, rk, scr, bin, rem);
     const uint32_t keys[2] = {(pre[0] << 10) | (uint32_t)bin[0], (pre[1] << 10) | (uint32_t)bin[1]};
-    if (threadIdx.x == 0) write_plan(c, P.m, keys, P.rank_lo, P.rank_hi, P.valid_lo, P.valid_hi);
+    const RowRanks rr = row_ranks(P, row_args(P, r).k);
+    if (threadIdx.x == 0) write_plan(c, P.m, keys, rr.rank_lo, rr.rank_hi, rr.valid_lo, rr.valid_hi);
   }
 }
 
@@ -359,7 +362,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   FilterCtx f;
   f.aL = vld(&c->aL);
   f.aR = vld(&c->aR);
-  f.c2 = (float)((1.0 / P.alpha) * (double)kLog2e);
+  f.c2 = (float)((1.0 / row_args(P, r).alpha) * (double)kLog2e);
   f.cnt = &c->band_cnt;
   f.kmax = &c->band_kmax;
   f.nkmin = &c->band_nkmin;
@@ -810,7 +813,8 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
                            int rank) {
   BandShared& S = *reinterpret_cast<BandShared*>(smem);
   double* red = S.red;
-  const double inva = 1.0 / P.alpha;
+  const RowArgs ra = row_args(P, r);
+  const double inva = 1.0 / ra.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
   const bool leader = rank == 0;
 
@@ -853,7 +857,7 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
     uint32_t klo = ~vld(&c->band_nkmin), khi = vld(&c->band_kmax);
     if (M == 0) klo = khi = 0u;
     int shift = bin_shift(klo, khi);
-    if (leader && threadIdx.x == 0) S.in = SolveIn{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, P.k, P.alpha, inva};
+    if (leader && threadIdx.x == 0) S.in = SolveIn{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, ra.k, ra.alpha, inva};
     int action = kBandDone;
     for (int level = 0; level < kMaxLevels; ++level) {
       levels = level + 1;
@@ -1067,7 +1071,6 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
 
   const int cta = blockIdx.x, ncta = gridDim.x;
   RowCtl* c0 = ctl_of(P, 0);
-  const double inva = 1.0 / P.alpha;
 #define REC_BARRIER()                                                          \
   do {                                                                         \
     if (!grid_barrier(&c0->bar_count, &c0->bar_gen, (uint32_t)ncta, &c0->timeout)) { \
@@ -1080,6 +1083,9 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
     RowCtl* c = ctl_of(P, r);
     const uint32_t st0 = vld(&c->status);
     if (!(st0 & ROW_NEEDS_RECOVERY) || (st0 & ROW_NONFINITE)) continue;
+    const RowArgs ra = row_args(P, r);
+    const double inva = 1.0 / ra.alpha;
+    const int widen_delta = row_ranks(P, ra.k).widen_delta;
     bool fallback = (st0 & (ROW_OVERFLOW | ROW_FORCE_FB)) != 0u || P.max_widen <= 0;
 
     if (!fallback) {
@@ -1091,11 +1097,11 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       bool vlo = vld(&c->valid_lo) != 0u, vhi = vld(&c->valid_hi) != 0u;
       if (left) {
         rhi = rlo; vhi = true;
-        rlo -= P.widen_delta; vlo = rlo >= 0;
+        rlo -= widen_delta; vlo = rlo >= 0;
         if (!vlo) rlo = 0;
       } else {
         rlo = rhi; vlo = true;
-        rhi += P.widen_delta; vhi = rhi <= P.m - 1;
+        rhi += widen_delta; vhi = rhi <= P.m - 1;
         if (!vhi) rhi = P.m - 1;
       }
       for (int i = cta * NT + threadIdx.x; i < 2048; i += ncta * NT) { h1_of(P, r)[i] = 0u; h3_of(P, r)[i] = 0u; }
@@ -1236,7 +1242,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
                                         fa + g, inva);
       REC_BARRIER();
       if (cta == 0) {
-        const SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, P.k, P.alpha, inva};
+        const SolveIn in{-CUDART_INF_F, CUDART_INF_F, 0, 0, 0.0, 0.0, ra.k, ra.alpha, inva};
         solve_band<NT, true>(in, fa, ng, KeyGroupsG{cur, kFallbackGroup}, dscr, red, &so);
         if (threadIdx.x == 0) {
           const uint32_t keep = (vld(&c->status) | st0) & (ROW_WIDENED | ROW_OVERFLOW);
@@ -1304,9 +1310,10 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
   const int64_t r = blockIdx.y;
   RowCtl* c = ctl_of(P, r);
   const double b = c->b;
-  uint32_t status = c->status;
-  const bool nonfinite = (status & ROW_NONFINITE) != 0u;
-  const double inva = 1.0 / P.alpha_p;
+  const RowArgs ra = row_args(P, r);
+  uint32_t status = c->status | (ra.bad ? ROW_BADARG : 0u);
+  const bool nonfinite = (status & (ROW_NONFINITE | ROW_BADARG)) != 0u;
+  const double inva = 1.0 / ra.alpha_p;
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
@@ -1512,7 +1519,8 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   __shared__ double red[64];
   const int64_t r = blockIdx.y;
   const double b = a.b[r];
-  const double inva = 1.0 / a.alpha;
+  bool bad = false;
+  const double inva = 1.0 / row_alpha(a.alpha, a.alpha_rows, r, &bad);
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
@@ -1592,10 +1600,10 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
       sgz = block_sum<NT, double>(sgz, red);
     }
     if (threadIdx.x == 0) {
-      const double lam = sg / s;
+      const double lam = bad ? CUDART_NAN : sg / s;  // NaN also reaches every grad of the row
       a.lam[r] = lam;
       if (a.grad_k) a.grad_k[r] = lam;
-      if (kAlpha) a.grad_alpha[r] = alpha_grad(M, sz, sgz, lam, inva);
+      if (kAlpha) a.grad_alpha[r] = bad ? CUDART_NAN : alpha_grad(M, sz, sgz, lam, inva);
     }
   }
 }
@@ -1605,7 +1613,8 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
 __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
   const int64_t r = blockIdx.y;
   const double b = a.b[r];
-  const double inva = 1.0 / a.alpha;
+  bool bad = false;
+  const double inva = 1.0 / row_alpha(a.alpha, a.alpha_rows, r, &bad);
   const float c2 = (float)(inva * (double)kLog2e);
   const float lg = (float)log2(0.5 * inva);
   const float bh = __double2float_rn(b);

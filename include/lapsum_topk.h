@@ -34,8 +34,9 @@
  *     non-zero return code means nothing was enqueued.  Device-side outcomes
  *     are reported per row in `row_status` (see LAPSUM_ROW_*), readable after
  *     the stream has been synchronised.
- *   - k and alpha are shared by all rows.  alpha must lie in [1e-30, 1e30]
- *     (the fp32 exponent arithmetic needs 1/alpha finite).
+ *   - k and alpha are shared by all rows, except in the *_rows entry points,
+ *     which take one of each per row.  alpha must lie in [1e-30, 1e30] (the
+ *     fp32 exponent arithmetic needs 1/alpha finite).
  *   - The first call on a device queries its properties and sets kernel
  *     attributes; later calls on that device do not.
  */
@@ -79,6 +80,8 @@ extern "C" {
 #define LAPSUM_ROW_TRUNCATED 0x40u  /* sparse forward: the row has more entries
                                        with p >= eps than the capacity; its
                                        count is still the full number */
+#define LAPSUM_ROW_BADARG 0x80u    /* per-row k or alpha out of range
+                                      (lapsum_topk_fwd_rows): outputs NaN */
 
 /* ---- tuning and test knobs --------------------------------------------- */
 typedef struct lapsum_params {
@@ -172,6 +175,42 @@ LAPSUM_API int lapsum_topk_fwd_sparse(const float* scores, int64_t rows, int64_t
                                       int64_t capacity, uint64_t* count_out, double* b_out, double* sumf_out,
                                       uint32_t* row_status, lapsum_row_stats* stats, void* workspace,
                                       size_t workspace_bytes, const lapsum_params* params, void* stream);
+
+/*
+ * Batched forward with a budget and a scale per row.  The method is stated
+ * for one vector with one k and one alpha (Fast LapSum technical summary,
+ * section 2.1); here row r is solved with k[r] and alpha[r], read by the
+ * kernels from device memory, so the values may come straight from an earlier
+ * kernel or an autograd graph without a host round trip.
+ *
+ *   k           in   fp64 [rows], device, 8-byte aligned: 0 < k[r] < n
+ *   alpha       in   fp64 [rows], device, 8-byte aligned: 1e-30 <= alpha[r] <= 1e30
+ * A row whose k[r] or alpha[r] is out of range (or NaN) is not an error of the
+ * call: it gets LAPSUM_ROW_BADARG and NaN outputs, the other rows are solved.
+ * Every row's sample is drawn with the sample size the one-block path picks
+ * for k = n/2 (the widest bracket), so a row's b can differ from that of a
+ * lapsum_topk_fwd call with the same k and alpha by rounding (both are the
+ * exact root to fp64 accuracy); on the streaming path (n > 16384) the sample
+ * and the ranks are the same as there.
+ * The other arguments, the workspace size and the per-row status are those of
+ * lapsum_topk_fwd.  Returns LAPSUM_OK or an error code (nothing enqueued on
+ * error).
+ */
+LAPSUM_API int lapsum_topk_fwd_rows(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                                    const double* k, const double* alpha, float* p_out, double* b_out,
+                                    double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
+                                    void* workspace, size_t workspace_bytes, const lapsum_params* params,
+                                    void* stream);
+
+/*
+ * Backward of lapsum_topk_fwd_rows: lapsum_topk_bwd with alpha[r] (fp64
+ * [rows], device) for row r.  A row whose alpha[r] is out of range gets NaN
+ * in grad_scores, grad_k and grad_alpha.
+ */
+LAPSUM_API int lapsum_topk_bwd_rows(const float* scores, const float* grad_p, const double* b, int64_t rows,
+                                    int64_t n, int64_t row_stride, const double* alpha, float* grad_scores,
+                                    double* grad_k, double* grad_alpha, void* workspace, size_t workspace_bytes,
+                                    void* stream);
 
 /*
  * DFTopK relaxation (Fast LapSum technical summary, section 2.3 "Relation to

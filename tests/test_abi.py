@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     assert names == sorted([
         "lapsum_default_params", "lapsum_dftopk_fwd", "lapsum_last_cuda_error", "lapsum_launch_count",
-        "lapsum_status_string", "lapsum_topk_bwd", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc", "lapsum_topk_fwd_sparse",
+        "lapsum_status_string", "lapsum_topk_bwd", "lapsum_topk_bwd_rows", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc",
+        "lapsum_topk_fwd_rows", "lapsum_topk_fwd_sparse",
         "lapsum_topk_sparse_workspace_size", "lapsum_topk_workspace_size",
         "lapsum_trace_collect", "lapsum_trace_enable",
     ])
@@ -180,6 +181,46 @@ def test_dftopk_fwd_rejects_bad_arguments(lib):
     assert call(wsb=16) == lt.LAPSUM_EWORKSPACE
     with pytest.raises(ValueError):
         lt.dftopk_forward(None, 2.5, 1.0)
+
+
+def test_per_row_entry_points_reject_bad_arguments(lib):
+    """The *_rows entry points check pointers on the host (the values
+    themselves are checked per row on the device)."""
+    F = lib.lapsum_topk_fwd_rows
+    ok = dict(s=FAKE, rows=4, n=100000, stride=100000, k=FAKE * 128, a=FAKE * 130, out=FAKE * 64, b=FAKE * 132,
+              ws=FAKE * 256, wsb=1 << 31)
+
+    def call(**kw):
+        d = dict(ok, **kw)
+        return F(d["s"], d["rows"], d["n"], d["stride"], d["k"], d["a"], d["out"], d["b"], None, None, None,
+                 d["ws"], d["wsb"], None, None)
+
+    assert call(k=None) == lt.LAPSUM_EINVAL
+    assert call(a=None) == lt.LAPSUM_EINVAL
+    assert call(k=FAKE * 128 + 4) == lt.LAPSUM_EINVAL  # misaligned fp64 vector
+    assert call(a=FAKE * 130 + 2) == lt.LAPSUM_EINVAL
+    assert call(out=FAKE + 64) == lt.LAPSUM_EINVAL
+    assert call(wsb=16) == lt.LAPSUM_EWORKSPACE
+    B = lib.lapsum_topk_bwd_rows
+    bok = dict(s=FAKE, g=FAKE * 64, b=FAKE * 128, rows=4, n=100000, stride=100000, a=FAKE * 130, out=FAKE * 192,
+               ws=FAKE * 256, wsb=1 << 31)
+
+    def bcall(**kw):
+        d = dict(bok, **kw)
+        return B(d["s"], d["g"], d["b"], d["rows"], d["n"], d["stride"], d["a"], d["out"], None, None, d["ws"],
+                 d["wsb"], None)
+
+    assert bcall(a=None) == lt.LAPSUM_EINVAL
+    assert bcall(a=FAKE * 130 + 4) == lt.LAPSUM_EINVAL
+    assert bcall(out=FAKE + 8) == lt.LAPSUM_EINVAL  # overlaps the scores
+    assert bcall(wsb=16) == lt.LAPSUM_EWORKSPACE
+
+
+def test_binding_rejects_a_misshaped_per_row_vector():
+    torch = pytest.importorskip("torch")
+    with pytest.raises(ValueError):
+        lt._rows_pair(torch.ones(3), 1.0, 4, "cpu")
+    assert lt._rows_pair(2.0, torch.tensor(1.0), 4, "cpu") is None
 
 
 def test_binding_rejects_cpu_tensors():

@@ -540,3 +540,102 @@ def test_dftopk_is_the_zero_temperature_limit_of_lapsum(orc):
     assert abs(mass_exact - k) <= tol_sum(k, x.shape[1])
     mass_ref = orc.dftopk_forward(x[0], k, w.alpha)[2]
     assert float(d.mass[0]) == pytest.approx(mass_ref, rel=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# per-row k and alpha (one budget and one scale per row of a batch)
+# ---------------------------------------------------------------------------
+def per_row_values(rows, n, seed):
+    rng = np.random.default_rng(seed)
+    k = np.round(rng.uniform(0.5, n - 0.5, rows), 3)
+    k[0], k[-1] = 0.25, n - 0.75  # near both ends of (0, n)
+    alpha = 10.0 ** rng.uniform(-3, 0.5, rows)
+    return k, alpha
+
+
+@pytest.mark.parametrize("rows,n,force", [
+    (6, 4096, 0), (5, 16384, 0), (3, 4096, lt.FORCE_STREAMING), (3, 200_003, 0), (2, 1_000_000, 0),
+])
+def test_per_row_k_and_alpha_match_oracle(orc, rows, n, force):
+    x = make_scores("normal", rows, n, seed=rows * 1000 + n)
+    g = make_grad(rows, n, seed=rows + n)
+    k, alpha = per_row_values(rows, n, seed=n)
+    xt, gt = torch.from_numpy(x).cuda(), torch.from_numpy(g).cuda()
+    kt, at = torch.from_numpy(k).cuda(), torch.from_numpy(alpha).cuda()
+    params = lt.Params(force_path=force) if force else None
+    res = lt.forward(xt, kt, at, params=params)
+    gs, gk, ga = lt.backward(xt, gt, res.b, at, want_alpha=True)
+    torch.cuda.synchronize()
+    p, b, grad = res.p.cpu().numpy(), res.b.cpu().numpy(), gs.cpu().numpy()
+    gk, ga = gk.cpu().numpy(), ga.cpu().numpy()
+    assert np.all(res.status.cpu().numpy() & lt.ROW_CERTIFIED)
+    for i in range(rows):
+        b_ref = check_row(orc, x[i], g[i], p[i], grad[i], b[i], gk[i], float(k[i]), float(alpha[i]), f"row {i}")
+        ref = orc.backward_alpha(x[i], g[i], b_ref, float(alpha[i]))
+        tol = 1e-4 * abs(ref) + alpha_tol(x[i], g[i], b_ref, float(alpha[i]))
+        assert abs(ga[i] - ref) <= tol, f"row {i}: dL/dalpha {ga[i]!r} vs {ref!r}"
+
+
+@pytest.mark.parametrize("n", [3000, 100_000])
+def test_per_row_call_agrees_with_scalar_calls(orc, n):
+    """Each row of a per-row call against a scalar call with that row's k and
+    alpha: the same threshold to fp64 rounding (the streaming path draws the
+    same sample and ranks; the one-block path a larger sample)."""
+    rows = 4
+    x = make_scores("normal", rows, n, seed=n + 3)
+    k, alpha = per_row_values(rows, n, seed=n + 4)
+    xt = torch.from_numpy(x).cuda()
+    res = lt.forward(xt, torch.from_numpy(k).cuda(), torch.from_numpy(alpha).cuda())
+    torch.cuda.synchronize()
+    for i in range(rows):
+        one = lt.forward(xt[i:i + 1].contiguous(), float(k[i]), float(alpha[i]))
+        torch.cuda.synchronize()
+        bi, b1 = float(res.b[i]), float(one.b[0])
+        assert abs(bi - b1) <= 2e-6 * alpha[i] + 1e-12 * abs(b1), f"row {i}: {bi!r} vs {b1!r}"
+
+
+@pytest.mark.parametrize("n", [2048, 50_000])
+def test_per_row_bad_values_mark_only_their_rows(orc, n):
+    rows = 6
+    x = make_scores("normal", rows, n, seed=n + 5)
+    g = make_grad(rows, n, seed=n + 6)
+    k = np.array([0.0, n, 10.0, np.nan, 20.0, 5.0])
+    alpha = np.array([0.5, 0.5, 0.0, 0.5, np.inf, 0.2])
+    good = [5]
+    xt, gt = torch.from_numpy(x).cuda(), torch.from_numpy(g).cuda()
+    at = torch.from_numpy(alpha).cuda()
+    res = lt.forward(xt, torch.from_numpy(k).cuda(), at)
+    gs, gk, ga = lt.backward(xt, gt, res.b, at, want_alpha=True)
+    torch.cuda.synchronize()
+    st = res.status.cpu().numpy().astype(np.uint32)
+    b, p, grad = res.b.cpu().numpy(), res.p.cpu().numpy(), gs.cpu().numpy()
+    for i in range(rows):
+        if i in good:
+            assert not st[i] & lt.ROW_BADARG
+            check_row(orc, x[i], g[i], p[i], grad[i], b[i], float(gk[i]), float(k[i]), float(alpha[i]), f"row {i}")
+        else:
+            assert st[i] & lt.ROW_BADARG, f"row {i} status {st[i]:#x}"
+            assert np.isnan(b[i]) and np.all(np.isnan(p[i]))
+    # the backward flags only a bad alpha (it has no k)
+    for i in (2, 4):
+        assert np.all(np.isnan(grad[i])) and np.isnan(float(gk[i])) and np.isnan(float(ga[i]))
+
+
+def test_autograd_per_row_k_and_alpha(orc):
+    rows, n = 3, 5000
+    x = make_scores("normal", rows, n, seed=11)
+    g = make_grad(rows, n, seed=12)
+    k, alpha = per_row_values(rows, n, seed=13)
+    xt = torch.from_numpy(x).cuda().requires_grad_(True)
+    kt = torch.from_numpy(k).cuda().requires_grad_(True)
+    at = torch.from_numpy(alpha).float().cuda().requires_grad_(True)
+    p = lt.soft_topk(xt, kt, at)
+    (p * torch.from_numpy(g).cuda()).sum().backward()
+    assert kt.grad.shape == (rows,) and at.grad.shape == (rows,) and at.grad.dtype == torch.float32
+    for i in range(rows):
+        a = float(at[i].detach())  # the fp32 value the operator saw
+        _, b_ref, _ = orc.forward(x[i], float(k[i]), a)
+        _, lam, _ = orc.backward(x[i], g[i], b_ref, a)
+        ref_a = orc.backward_alpha(x[i], g[i], b_ref, a)
+        assert float(kt.grad[i]) == pytest.approx(lam, rel=1e-4, abs=1e-6 * (1 + abs(lam)))
+        assert float(at.grad[i]) == pytest.approx(ref_a, rel=1e-4, abs=alpha_tol(x[i], g[i], b_ref, a) + 1e-6)
