@@ -198,6 +198,55 @@ int stream_grid(int sm_count, int blocks_per_sm, int64_t rows, int64_t n) {
   return (int)std::min<int64_t>({(int64_t)kMaxGridPerRow, per_row, chunks});
 }
 
+// The plan of the streaming pipeline for rows of n scores (the band sized by
+// s), its pieces at the offsets L of the workspace ws.
+StreamPlan stream_plan(int64_t rows, int64_t n, int64_t row_stride, double k, double alpha, const StreamSizes& s,
+                       const StreamLayout& L, const Resolved& R, const DevInfo& dev, int vec, unsigned char* ws) {
+  const StreamOcc& occ = dev.occ;
+  StreamPlan P{};
+  P.rows = rows;
+  P.n = n;
+  P.stride = row_stride;
+  P.k = k;
+  P.alpha = alpha;
+  P.alpha_p = alpha;
+  P.m = s.m;
+  P.rank_lo = s.rk.rank_lo;
+  P.rank_hi = s.rk.rank_hi;
+  P.valid_lo = s.rk.valid_lo;
+  P.valid_hi = s.rk.valid_hi;
+  P.widen_delta = s.rk.widen_delta;
+  P.max_widen = R.max_widen;
+  P.band_cap = s.band_cap;
+  P.seed = R.seed;
+  P.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+  P.vec = vec;
+  const int sm = dev.sm_count;
+  P.Gs = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (s.m + 1023) / 1024));
+  P.Gf = stream_grid(sm, occ.filter_blocks, rows, n);
+  P.Gm = stream_grid(sm, occ.memb_blocks, rows, n);
+  P.Gr = std::min(kMaxGridPerRow, sm * occ.recover_blocks);
+  // band cluster: about kBandValuesPerCta expected band values per CTA
+  // (with more than one CTA the leader holds no slice)
+  int cs = 1;
+  while (cs < occ.band_max_cluster && (double)(cs > 1 ? cs - 1 : 1) * kBandValuesPerCta < s.M_est) cs <<= 1;
+  P.band_cs = cs;
+  P.ctl = ws + L.ctl;
+  P.zero_bytes = L.zero_end - L.ctl;
+  P.hist1 = reinterpret_cast<uint32_t*>(ws + L.h1);
+  P.hist2 = reinterpret_cast<uint32_t*>(ws + L.h2);
+  P.hist3 = reinterpret_cast<uint32_t*>(ws + L.h3);
+  P.samp = reinterpret_cast<uint32_t*>(ws + L.samp);
+  P.fpart = ws + L.fpart;
+  P.band = reinterpret_cast<float*>(ws + L.band);
+  P.mpart = ws + L.mpart;
+  P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
+  P.fb_aggs = ws + L.fb_aggs;
+  P.rcount = reinterpret_cast<uint32_t*>(ws + L.rcount);
+  P.z = R.z;
+  return P;
+}
+
 bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
   return x < y + bn && y < x + an;
@@ -291,44 +340,8 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   const StreamSizes s = stream_sizes(n, k, R);
   const StreamLayout L = stream_layout(rows, n, s);
   const StreamOcc& occ = dev->occ;
-  StreamPlan P{};
-  P.rows = rows;
-  P.n = n;
-  P.stride = row_stride;
-  P.k = k;
-  P.alpha = alpha;
-  P.m = s.m;
-  P.rank_lo = s.rk.rank_lo;
-  P.rank_hi = s.rk.rank_hi;
-  P.valid_lo = s.rk.valid_lo;
-  P.valid_hi = s.rk.valid_hi;
-  P.widen_delta = s.rk.widen_delta;
-  P.max_widen = R.max_widen;
-  P.band_cap = s.band_cap;
-  P.seed = R.seed;
-  P.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
-  P.vec = vec;
   const int sm = dev->sm_count;
-  P.Gs = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (s.m + 1023) / 1024));
-  P.Gf = stream_grid(sm, occ.filter_blocks, rows, n);
-  P.Gm = stream_grid(sm, occ.memb_blocks, rows, n);
-  P.Gr = std::min(kMaxGridPerRow, sm * occ.recover_blocks);
-  // band cluster: about kBandValuesPerCta expected band values per CTA
-  // (with more than one CTA the leader holds no slice)
-  int cs = 1;
-  while (cs < occ.band_max_cluster && (double)(cs > 1 ? cs - 1 : 1) * kBandValuesPerCta < s.M_est) cs <<= 1;
-  P.band_cs = cs;
-  P.ctl = ws + L.ctl;
-  P.zero_bytes = L.zero_end - L.ctl;
-  P.hist1 = reinterpret_cast<uint32_t*>(ws + L.h1);
-  P.hist2 = reinterpret_cast<uint32_t*>(ws + L.h2);
-  P.hist3 = reinterpret_cast<uint32_t*>(ws + L.h3);
-  P.samp = reinterpret_cast<uint32_t*>(ws + L.samp);
-  P.fpart = ws + L.fpart;
-  P.band = reinterpret_cast<float*>(ws + L.band);
-  P.mpart = ws + L.mpart;
-  P.fb_keys = reinterpret_cast<uint32_t*>(ws + L.fb_keys);
-  P.fb_aggs = ws + L.fb_aggs;
+  StreamPlan P = stream_plan(rows, n, row_stride, k, alpha, s, L, R, *dev, vec, ws);
   P.alpha_p = alpha_p;
   P.dftopk = dftopk ? 1 : 0;
   P.sump_out = sump_out;
@@ -343,6 +356,64 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   P.rcount = reinterpret_cast<uint32_t*>(ws + L.rcount);
   return cuda_ok(launch_stream_fwd(P, scores, p_out, b_out, sumf_out, row_status, stats, sm, st)) ? LAPSUM_OK
                                                                                                 : LAPSUM_ECUDA;
+}
+
+// ---- sharded rows ------------------------------------------------------------
+// The band of a sharded row is sized for the widest bracket (as the workspace
+// of the one-GPU forward is), so that the gathered exchange buffers have one
+// layout whatever k is.
+int64_t shard_band_cap(int64_t n_total, const Resolved& R) {
+  int64_t cap = 0;
+  for (double kk : {1.0, 0.5 * (double)n_total, (double)n_total - 1.0})
+    if (kk > 0.0 && kk < (double)n_total) cap = std::max(cap, stream_sizes(n_total, kk, R).band_cap);
+  return std::max<int64_t>(cap, 4);
+}
+
+void shard_layout(int64_t rows, int64_t n_total, const Resolved& R, lapsum_shard_layout* o) {
+  StreamSizes s = stream_sizes(n_total, 0.5 * (double)n_total, R);
+  s.band_cap = shard_band_cap(n_total, R);
+  const StreamLayout L = stream_layout(rows, 0, s);
+  o->sample_m = s.m;
+  o->band_cap = s.band_cap;
+  o->sample_bytes = 4 * (size_t)s.m * (size_t)rows;
+  o->hist_bytes = 4 * 2048 * (size_t)rows;
+  o->meta_bytes = 4 * (size_t)kShardMeta * (size_t)rows;
+  o->fpart_bytes = 32 * (size_t)kMaxGridPerRow * (size_t)rows;
+  o->band_bytes = 4 * (size_t)s.band_cap * (size_t)rows;
+  o->parts_bytes = 48 * (size_t)kMaxGridPerRow * (size_t)rows;
+  o->workspace_bytes = std::max(L.total, align256(8 * (size_t)rows) + align256(4 * (size_t)rows));
+}
+
+bool aligned16(const void* p) { return p && ((uintptr_t)p & 15u) == 0; }
+
+// Checks the arguments every sharded forward call shares and builds the plan
+// of this GPU's shard (P) and of the band step (Pb) in the workspace.
+int shard_fwd_plan(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t shard_lo,
+                   int64_t n_total, double k, double alpha, void* workspace, size_t workspace_bytes,
+                   const lapsum_params* params, const float* p_out, StreamPlan* P, StreamPlan* Pb, DevInfo** dev) {
+  if (!scores || ((uintptr_t)scores & 3u)) return LAPSUM_EINVAL;
+  if (rows < 1 || rows > 65535 || n < 1 || row_stride < n || shard_lo < 0 || n_total > INT32_MAX ||
+      shard_lo + n > n_total)
+    return LAPSUM_EINVAL;
+  if (!std::isfinite(k) || !(k > 0.0) || !(k < (double)n_total)) return LAPSUM_EBADK;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  const Resolved R = resolve(params);
+  lapsum_shard_layout lay;
+  shard_layout(rows, n_total, R, &lay);
+  if (!workspace || workspace_bytes < lay.workspace_bytes || ((uintptr_t)workspace & 255u)) return LAPSUM_EWORKSPACE;
+  if (!cuda_ok(device_info(dev))) return LAPSUM_ECUDA;
+  StreamSizes s = stream_sizes(n_total, k, R);  // ranks and cluster size from this k
+  s.band_cap = lay.band_cap;
+  StreamSizes sl = s;
+  const StreamLayout L = stream_layout(rows, 0, sl);
+  const int vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  *P = stream_plan(rows, n, row_stride, k, alpha, s, L, R, **dev, vec, static_cast<unsigned char*>(workspace));
+  P->shard = 1;
+  P->n_total = n_total;
+  P->shard_lo = shard_lo;
+  *Pb = *P;
+  Pb->Gf = 1;  // the gathered filter partials arrive summed into one per row
+  return LAPSUM_OK;
 }
 
 // The backward behind lapsum_topk_bwd (one alpha) and lapsum_topk_bwd_rows
@@ -496,6 +567,126 @@ int lapsum_topk_bwd_rows(const float* scores, const float* grad_p, const double*
   if (!alpha) return LAPSUM_EINVAL;
   return bwd_impl(scores, grad_p, b, rows, n, row_stride, 1.0, alpha, grad_scores, grad_k, grad_alpha, workspace,
                   workspace_bytes, stream);
+}
+
+void lapsum_shard_layout_get(int64_t rows, int64_t n_total, const lapsum_params* params, lapsum_shard_layout* out) {
+  if (!out) return;
+  std::memset(out, 0, sizeof(*out));
+  if (rows < 1 || n_total < 1 || n_total > INT32_MAX) return;
+  shard_layout(rows, n_total, resolve(params), out);
+}
+
+int lapsum_shard_fwd_sample(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t shard_lo,
+                            int64_t n_total, double k, double alpha, uint32_t* x_sample, uint32_t* x_hist,
+                            void* workspace, size_t workspace_bytes, const lapsum_params* params, void* stream) {
+  if (!aligned16(x_sample) || !aligned16(x_hist)) return LAPSUM_EINVAL;
+  StreamPlan P, Pb;
+  DevInfo* dev = nullptr;
+  const int rc = shard_fwd_plan(scores, rows, n, row_stride, shard_lo, n_total, k, alpha, workspace,
+                                workspace_bytes, params, nullptr, &P, &Pb, &dev);
+  if (rc != LAPSUM_OK) return rc;
+  P.samp = x_sample;
+  P.hist1 = x_hist;
+  return cuda_ok(launch_shard_sample(P, scores, reinterpret_cast<cudaStream_t>(stream))) ? LAPSUM_OK : LAPSUM_ECUDA;
+}
+
+int lapsum_shard_fwd_filter(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t shard_lo,
+                            int64_t n_total, double k, double alpha, const uint32_t* x_sample,
+                            const uint32_t* x_hist, uint32_t* x_meta, void* x_fpart, float* x_band,
+                            void* workspace, size_t workspace_bytes, const lapsum_params* params, void* stream) {
+  if (!aligned16(x_sample) || !aligned16(x_hist) || !aligned16(x_meta) || !aligned16(x_fpart) || !aligned16(x_band))
+    return LAPSUM_EINVAL;
+  StreamPlan P, Pb;
+  DevInfo* dev = nullptr;
+  const int rc = shard_fwd_plan(scores, rows, n, row_stride, shard_lo, n_total, k, alpha, workspace,
+                                workspace_bytes, params, nullptr, &P, &Pb, &dev);
+  if (rc != LAPSUM_OK) return rc;
+  P.samp = const_cast<uint32_t*>(x_sample);
+  P.hist1 = const_cast<uint32_t*>(x_hist);
+  P.fpart = x_fpart;
+  P.band = x_band;
+  return cuda_ok(launch_shard_filter(P, scores, x_meta, reinterpret_cast<cudaStream_t>(stream))) ? LAPSUM_OK
+                                                                                                  : LAPSUM_ECUDA;
+}
+
+int lapsum_shard_fwd_finish(const float* scores, int64_t rows, int64_t n, int64_t row_stride, int64_t shard_lo,
+                            int64_t n_total, double k, double alpha, int world, const uint32_t* g_meta,
+                            const void* g_fpart, const float* g_band, float* p_out, double* b_out, double* sumf_out,
+                            uint32_t* row_status, void* workspace, size_t workspace_bytes,
+                            const lapsum_params* params, void* stream) {
+  if (world < 1 || world > 1024 || !aligned16(g_meta) || !aligned16(g_fpart) || !aligned16(g_band)) return LAPSUM_EINVAL;
+  if (!p_out || !b_out || ((uintptr_t)p_out & 3u) || ((uintptr_t)b_out & 7u)) return LAPSUM_EINVAL;
+  if (sumf_out && ((uintptr_t)sumf_out & 7u)) return LAPSUM_EINVAL;
+  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
+  if (rows >= 1 && n >= 1 && overlaps(scores, span, p_out, span)) return LAPSUM_EINVAL;
+  StreamPlan P, Pb;
+  DevInfo* dev = nullptr;
+  const int rc = shard_fwd_plan(scores, rows, n, row_stride, shard_lo, n_total, k, alpha, workspace,
+                                workspace_bytes, params, p_out, &P, &Pb, &dev);
+  if (rc != LAPSUM_OK) return rc;
+  return cuda_ok(launch_shard_finish(P, Pb, scores, p_out, b_out, sumf_out, row_status, world, g_fpart, g_meta, g_band,
+                                     reinterpret_cast<cudaStream_t>(stream)))
+             ? LAPSUM_OK
+             : LAPSUM_ECUDA;
+}
+
+int lapsum_shard_bwd_partials(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
+                              int64_t row_stride, double alpha, int with_alpha, void* x_parts, void* stream) {
+  if (!scores || !grad_p || !b || !aligned16(x_parts)) return LAPSUM_EINVAL;
+  if (rows < 1 || rows > 65535 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
+  if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)b & 7u)) return LAPSUM_EINVAL;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  DevInfo* dev = nullptr;
+  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
+  StreamBwd a{};
+  a.scores = scores;
+  a.grad_p = grad_p;
+  a.b = b;
+  a.rows = rows;
+  a.n = n;
+  a.stride = row_stride;
+  a.alpha = alpha;
+  a.vec = (((uintptr_t)scores | (uintptr_t)grad_p) & 15u) == 0 && (row_stride & 3) == 0;
+  a.parts_only = 1;
+  a.part = x_parts;
+  a.Gb = stream_grid(dev->sm_count, dev->occ.reduce_blocks, rows, n);
+  return cuda_ok(launch_shard_bwd_partials(a, with_alpha != 0, reinterpret_cast<cudaStream_t>(stream))) ? LAPSUM_OK
+                                                                                                    : LAPSUM_ECUDA;
+}
+
+int lapsum_shard_bwd_finish(const float* scores, const float* grad_p, const double* b, int64_t rows, int64_t n,
+                            int64_t row_stride, double alpha, int world, const void* g_parts, float* grad_scores,
+                            double* grad_k, double* grad_alpha, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!scores || !grad_p || !b || !grad_scores || !aligned16(g_parts) || world < 1 || world > 1024)
+    return LAPSUM_EINVAL;
+  if (rows < 1 || rows > 65535 || n < 1 || n > INT32_MAX || row_stride < n) return LAPSUM_EINVAL;
+  if (((uintptr_t)scores & 3u) || ((uintptr_t)grad_p & 3u) || ((uintptr_t)grad_scores & 3u) || ((uintptr_t)b & 7u))
+    return LAPSUM_EINVAL;
+  if ((grad_k && ((uintptr_t)grad_k & 7u)) || (grad_alpha && ((uintptr_t)grad_alpha & 7u))) return LAPSUM_EINVAL;
+  if (!std::isfinite(alpha) || !(alpha >= 1e-30) || !(alpha <= 1e30)) return LAPSUM_EBADALPHA;
+  const size_t span = 4 * (size_t)((rows - 1) * row_stride + n);
+  if (overlaps(scores, span, grad_scores, span) || overlaps(grad_p, span, grad_scores, span)) return LAPSUM_EINVAL;
+  const size_t need = align256(8 * (size_t)rows);
+  if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255u)) return LAPSUM_EWORKSPACE;
+  DevInfo* dev = nullptr;
+  if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
+  StreamBwd a{};
+  a.scores = scores;
+  a.grad_p = grad_p;
+  a.b = b;
+  a.rows = rows;
+  a.n = n;
+  a.stride = row_stride;
+  a.alpha = alpha;
+  a.grad = grad_scores;
+  a.grad_k = grad_k;
+  a.grad_alpha = grad_alpha;
+  a.vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
+  a.lam = static_cast<double*>(workspace);
+  a.Ga = stream_grid(dev->sm_count, dev->occ.apply_blocks, rows, n);
+  return cuda_ok(launch_shard_bwd_finish(a, g_parts, world, reinterpret_cast<cudaStream_t>(stream))) ? LAPSUM_OK
+                                                                                                      : LAPSUM_ECUDA;
 }
 
 }  // extern "C"

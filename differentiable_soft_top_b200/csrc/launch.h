@@ -135,6 +135,11 @@ struct StreamPlan {
   const double* k_rows;      // per-row k (device [rows]) or null
   const double* alpha_rows;  // per-row alpha (device [rows]) or null
   double z;                  // rank half-width in standard deviations
+  // sharded rows (shard != 0): this GPU holds scores [shard_lo, shard_lo + n)
+  // of rows n_total long; the sample and the band solve see the whole row,
+  // the streaming passes the shard
+  int shard;
+  int64_t n_total, shard_lo;
 };
 
 constexpr int kFallbackGroup = 4096;   // full-sort fallback: sorted values per group
@@ -158,12 +163,32 @@ struct StreamBwd {
   double* grad_alpha;  // dL/dalpha per row, or null
   const double* alpha_rows;  // per-row alpha (device [rows]) or null
   int vec;
+  int parts_only;    // sharded rows: the reduction only writes this shard's partials
   int Gb, Ga;        // grids of the reduction and elementwise passes
   void* part;        // [rows][kMaxGridPerRow] partials (48 bytes each)
   uint32_t* done;    // [rows] counters (zeroed by the launcher)
   double* lam;       // [rows]
 };
 cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st);
+
+// ---- sharded rows: the streaming pipeline split at its three exchanges ----
+// Exchange 1 (sum over GPUs): the sample keys (P.samp; 0 where another GPU
+// holds the sampled score) and the level-1 histogram (P.hist1).
+// Exchange 2 (gather): per GPU and row, kShardMeta words (band count, largest
+// key, complement of the smallest key, flags, filter grid), the filter
+// partials (P.fpart, kMaxGridPerRow slots per row) and the band (P.band,
+// band_cap values per row).
+// Backward exchange (gather): the reduction partials, kMaxGridPerRow slots of
+// 48 bytes per row; slot 0 carries the number of valid slots.
+constexpr int kShardMeta = 8;
+cudaError_t launch_shard_sample(const StreamPlan& P, const float* scores, cudaStream_t st);
+cudaError_t launch_shard_filter(const StreamPlan& P, const float* scores, uint32_t* meta, cudaStream_t st);
+// Pb: the plan of the band step (local workspace for fpart and band)
+cudaError_t launch_shard_finish(const StreamPlan& P, const StreamPlan& Pb, const float* scores, float* p_out,
+                                double* b_out, double* sumf_out, uint32_t* status_out, int world,
+                                const void* g_fpart, const uint32_t* g_meta, const float* g_band, cudaStream_t st);
+cudaError_t launch_shard_bwd_partials(const StreamBwd& a, bool with_alpha, cudaStream_t st);
+cudaError_t launch_shard_bwd_finish(const StreamBwd& a, const void* parts_all, int world, cudaStream_t st);
 
 // occupancy facts of the streaming kernels on the current device
 struct StreamOcc {

@@ -224,27 +224,35 @@ __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* 
   uint32_t* samp = samp_of(P, r);
   const RowArgs ra = row_args(P, r);
   const int stride = gridDim.x * NT;
+  // a sharded row draws the indices of the whole row and gathers those of its
+  // shard; the others stay key 0 (no finite score has that key), so the sum
+  // of the GPUs' sample arrays is the full sample
+  const uint64_t nt = (uint64_t)(P.shard ? P.n_total : P.n);
+  const uint64_t lo = P.shard ? (uint64_t)P.shard_lo : 0u;
   for (int j0 = blockIdx.x * NT; j0 < P.m; j0 += 4 * stride) {
     float v[4];
+    bool own[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u * stride + threadIdx.x;
-      v[u] = (j < P.m) ? __ldg(row + sample_index(s, (uint64_t)j, (uint64_t)P.n)) : 0.0f;
+      const uint64_t I = (j < P.m) ? sample_index(s, (uint64_t)j, nt) : 0u;
+      own[u] = j < P.m && I >= lo && I - lo < (uint64_t)P.n;
+      v[u] = own[u] ? __ldg(row + (I - lo)) : 0.0f;
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int j = j0 + u * stride + threadIdx.x;
-      const bool act = j < P.m;
       uint32_t key = 0u;
-      if (act) {
+      if (own[u]) {
         const double Y = (double)v[u] + laplace_noise(s, (uint64_t)j, ra.alpha);
         key = f2key(__double2float_rn(Y));
-        samp[j] = key;
       }
-      hist_add(sh, key >> 21, act);
+      if (j < P.m) samp[j] = key;
+      hist_add(sh, key >> 21, own[u]);
     }
   }
   flush_hist(sh, h1_of(P, r), 2048);
+  if (P.shard) return;  // the pick waits for the other GPUs' histograms
   RowCtl* c = ctl_of(P, r);
   if (last_block_done(&c->done_s1, gridDim.x)) {
     const RowRanks rr = row_ranks(P, ra.k);
@@ -254,6 +262,18 @@ __global__ void __launch_bounds__(NT) k_sample(const StreamPlan P, const float* 
     sel_pick<2048>(h1_of(P, r), false, rk, scr, bin, rem);
     store_pick(c, 0, bin, rem);
   }
+}
+
+// sharded rows: the level-1 pick, once the histograms of all GPUs are summed
+__global__ void __launch_bounds__(NT) k_pick1(const StreamPlan P) {
+  __shared__ uint32_t scr[64];
+  const int64_t r = blockIdx.y;
+  const RowRanks rr = row_ranks(P, row_args(P, r).k);
+  const uint32_t rk[2] = {(uint32_t)rr.rank_lo, (uint32_t)rr.rank_hi};
+  int bin[2];
+  uint32_t rem[2];
+  sel_pick<2048>(h1_of(P, r), false, rk, scr, bin, rem);
+  store_pick(ctl_of(P, r), 0, bin, rem);
 }
 
 __global__ void __launch_bounds__(NT) k_select2(const StreamPlan P) {
@@ -835,7 +855,7 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
   bad = block_or<NTX>(bad, reinterpret_cast<uint32_t*>(red));
   const uint32_t flags = vld(&c->flags);
   const uint32_t mt = vld(&c->band_cnt);
-  const long long nr = P.n - nl - (long long)mt;
+  const long long nr = (P.shard ? P.n_total : P.n) - nl - (long long)mt;
   const int64_t M = min((int64_t)mt, P.band_cap);
   uint32_t st = vld(&c->status) & ROW_WIDENED;
   double b = 0.0, sumf = 0.0;
@@ -1512,6 +1532,52 @@ struct BPart {
   double m, S, SG, SZ, SGZ, pad;
 };
 
+// lambda (and dL/dalpha) of row r from `world` groups of reduction partials
+// (group w at parts + w * wstride; per partials in each, or the count a
+// sharded GPU left in slot 0 when per < 0), in a fixed order.  All threads of
+// one block call it.
+template <bool kAlpha>
+__device__ void combine_parts(const StreamBwd& a, int64_t r, const BPart* parts, int64_t wstride, int world, int per,
+                              bool bad, double inva, double* red) {
+  auto count = [&](int w) {
+    return per >= 0 ? per : (int)__ldcg(&parts[w * wstride].pad);
+  };
+  float mloc = CUDART_INF_F;
+  for (int w = 0; w < world; ++w) {
+    const BPart* pw = parts + w * wstride;
+    const int c = count(w);
+    for (int i = threadIdx.x; i < c; i += NT) mloc = fminf(mloc, (float)__ldcg(&pw[i].m));
+  }
+  const double M = (double)block_min_float<NT>(mloc, reinterpret_cast<float*>(red));
+  double s = 0.0, sg = 0.0, sz = 0.0, sgz = 0.0;
+  for (int w = 0; w < world; ++w) {
+    const BPart* pw = parts + w * wstride;
+    const int c = count(w);
+    for (int i = threadIdx.x; i < c; i += NT) {
+      const double pm = __ldcg(&pw[i].m);
+      const double sc = (pm == CUDART_INF) ? 0.0 : exp2(M - pm);
+      s += __ldcg(&pw[i].S) * sc;
+      sg += __ldcg(&pw[i].SG) * sc;
+      if (kAlpha) {
+        sz += __ldcg(&pw[i].SZ) * sc;
+        sgz += __ldcg(&pw[i].SGZ) * sc;
+      }
+    }
+  }
+  s = block_sum<NT, double>(s, red);
+  sg = block_sum<NT, double>(sg, red);
+  if (kAlpha) {
+    sz = block_sum<NT, double>(sz, red);
+    sgz = block_sum<NT, double>(sgz, red);
+  }
+  if (threadIdx.x == 0) {
+    const double lam = bad ? CUDART_NAN : sg / s;  // NaN also reaches every grad of the row
+    a.lam[r] = lam;
+    if (a.grad_k) a.grad_k[r] = lam;
+    if (kAlpha) a.grad_alpha[r] = bad ? CUDART_NAN : alpha_grad(M, sz, sgz, lam, inva);
+  }
+}
+
 // lambda = sum g f / sum f by the rescaled reduction of common.cuh; with
 // kAlpha also sum f z and sum g f z (z = r - b) for dL/dalpha
 template <bool kAlpha>
@@ -1578,34 +1644,23 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
   else block_shift_reduce<NT>(m, S, SG, red);
   BPart* part = reinterpret_cast<BPart*>(a.part) + r * kMaxGridPerRow;
   if (threadIdx.x == 0) part[blockIdx.x] = BPart{(double)m, S, SG, SZ, SGZ, 0.0};
-  if (last_block_done(a.done + r, gridDim.x)) {
-    float mloc = CUDART_INF_F;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) mloc = fminf(mloc, (float)__ldcg(&part[i].m));
-    const double M = (double)block_min_float<NT>(mloc, reinterpret_cast<float*>(red));
-    double s = 0.0, sg = 0.0, sz = 0.0, sgz = 0.0;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += NT) {
-      const double pm = __ldcg(&part[i].m);
-      const double sc = (pm == CUDART_INF) ? 0.0 : exp2(M - pm);
-      s += __ldcg(&part[i].S) * sc;
-      sg += __ldcg(&part[i].SG) * sc;
-      if (kAlpha) {
-        sz += __ldcg(&part[i].SZ) * sc;
-        sgz += __ldcg(&part[i].SGZ) * sc;
-      }
-    }
-    s = block_sum<NT, double>(s, red);
-    sg = block_sum<NT, double>(sg, red);
-    if (kAlpha) {
-      sz = block_sum<NT, double>(sz, red);
-      sgz = block_sum<NT, double>(sgz, red);
-    }
-    if (threadIdx.x == 0) {
-      const double lam = bad ? CUDART_NAN : sg / s;  // NaN also reaches every grad of the row
-      a.lam[r] = lam;
-      if (a.grad_k) a.grad_k[r] = lam;
-      if (kAlpha) a.grad_alpha[r] = bad ? CUDART_NAN : alpha_grad(M, sz, sgz, lam, inva);
-    }
+  if (a.parts_only) {
+    // sharded rows: slot 0 also carries this GPU's number of partials
+    if (threadIdx.x == 0 && blockIdx.x == 0) part[0].pad = (double)gridDim.x;
+    return;
   }
+  if (last_block_done(a.done + r, gridDim.x)) combine_parts<kAlpha>(a, r, part, 0, 1, (int)gridDim.x, bad, inva, red);
+}
+
+// sharded rows: lambda from the partials of all GPUs (gathered: GPU w's
+// [rows][kMaxGridPerRow] block at w * rows * kMaxGridPerRow)
+template <bool kAlpha>
+__global__ void __launch_bounds__(NT) k_bwd_combine(const StreamBwd a, const BPart* parts_all, int world) {
+  __shared__ double red[64];
+  const int64_t r = blockIdx.x;
+  bool bad = false;
+  const double inva = 1.0 / row_alpha(a.alpha, a.alpha_rows, r, &bad);
+  combine_parts<kAlpha>(a, r, parts_all + r * kMaxGridPerRow, a.rows * kMaxGridPerRow, world, -1, bad, inva, red);
 }
 
 // grad = f (g - lambda), f = 2^(log2(1/(2 alpha)) - |x - b| log2(e)/alpha) in
@@ -1655,6 +1710,91 @@ __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
   }
   for (int64_t i = done + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
     o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
+}
+
+
+// ===========================================================================
+// sharded rows: one long row split over GPUs in contiguous shards.  The
+// pipeline above runs per GPU on its shard; three exchanges, made by the
+// caller (NCCL), join the GPUs: the sample and level-1 histogram are summed,
+// the filter's partials, band and band statistics are gathered, and every GPU
+// then solves the same band for the same b.  Nothing here waits on another
+// GPU.
+// ===========================================================================
+
+// this GPU's band statistics for the gather
+__global__ void k_shard_pack(const StreamPlan P, uint32_t* meta) {
+  const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= P.rows) return;
+  const RowCtl* c = ctl_of(P, r);
+  uint32_t* m = meta + r * kShardMeta;
+  m[0] = c->band_cnt;
+  m[1] = c->band_kmax;
+  m[2] = c->band_nkmin;
+  m[3] = c->flags;
+  m[4] = (uint32_t)P.Gf;
+  m[5] = m[6] = m[7] = 0u;
+}
+
+// the gathered statistics and filter partials of all GPUs into this GPU's
+// row control and one filter partial per row (fixed order over GPUs)
+__global__ void __launch_bounds__(NT) k_shard_unpack(const StreamPlan Pb, int world, const FPart* g_fpart,
+                                                      const uint32_t* g_meta) {
+  __shared__ double red[64];
+  const int64_t r = blockIdx.x;
+  RowCtl* c = ctl_of(Pb, r);
+  long long nl = 0;
+  double sl = 0.0, sr = 0.0;
+  uint32_t bad = 0u;
+  for (int w = 0; w < world; ++w) {
+    const uint32_t* m = g_meta + ((int64_t)w * Pb.rows + r) * kShardMeta;
+    const int gf = min((int)m[4], kMaxGridPerRow);
+    const FPart* fp = g_fpart + ((int64_t)w * Pb.rows + r) * kMaxGridPerRow;
+    for (int i = threadIdx.x; i < gf; i += NT) {
+      nl += fp[i].nL;
+      sl += fp[i].SL;
+      sr += fp[i].SR;
+      bad |= fp[i].bad;
+    }
+  }
+  nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
+  sl = block_sum<NT, double>(sl, red);
+  sr = block_sum<NT, double>(sr, red);
+  bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  if (threadIdx.x == 0) {
+    unsigned long long cnt = 0ull;
+    uint32_t kmax = 0u, nkmin = 0u, flags = 0u;
+    for (int w = 0; w < world; ++w) {
+      const uint32_t* m = g_meta + ((int64_t)w * Pb.rows + r) * kShardMeta;
+      cnt += m[0];
+      kmax = max(kmax, m[1]);
+      nkmin = max(nkmin, m[2]);
+      flags |= m[3];
+    }
+    if (cnt > (unsigned long long)Pb.band_cap) flags |= ROW_OVERFLOW;
+    c->band_cnt = (uint32_t)min(cnt, 0xFFFFFFFFull);
+    c->band_kmax = kmax;
+    c->band_nkmin = nkmin;
+    c->flags = flags;
+    FPart* f = fpart_of(Pb, r);
+    f[0] = FPart{nl, sl, sr, bad, 0u};
+  }
+}
+
+// the gathered bands, one after the other, into this GPU's band of each row
+__global__ void __launch_bounds__(NT) k_shard_compact(const StreamPlan Pb, int world, const float* g_band,
+                                                       const uint32_t* g_meta) {
+  const int64_t r = blockIdx.y;
+  float* dst = band_of(Pb, r);
+  int64_t off = 0;
+  for (int w = 0; w < world; ++w) {
+    const int64_t cnt = min((int64_t)g_meta[((int64_t)w * Pb.rows + r) * kShardMeta], Pb.band_cap);
+    const float* src = g_band + ((int64_t)w * Pb.rows + r) * Pb.band_cap;
+    for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < cnt && off + i < Pb.band_cap;
+         i += (int64_t)gridDim.x * NT)
+      dst[off + i] = src[i];
+    off += cnt;
+  }
 }
 
 }  // namespace
@@ -1783,6 +1923,102 @@ cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st) {
     Launch l("k_bwd_reduce", st);
     if (a.grad_alpha) k_bwd_reduce<true><<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
     else k_bwd_reduce<false><<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+  }
+  {
+    Launch l("k_bwd_apply", st);
+    k_bwd_apply<<<dim3(a.Ga, (unsigned)a.rows), NT, 0, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_sample(const StreamPlan& P, const float* scores, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(P.ctl, 0, P.zero_bytes, st);
+  if (e != cudaSuccess) return e;
+  // the level-1 histogram is part of the exchange, outside the zeroed block
+  e = cudaMemsetAsync(P.hist1, 0, sizeof(uint32_t) * 2048 * (size_t)P.rows, st);
+  if (e != cudaSuccess) return e;
+  Launch l("k_sample", st);
+  k_sample<<<dim3(P.Gs, (unsigned)P.rows), NT, 0, st>>>(P, scores);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_filter(const StreamPlan& P, const float* scores, uint32_t* meta, cudaStream_t st) {
+  const unsigned rows = (unsigned)P.rows;
+  {
+    Launch l("k_pick1", st);
+    k_pick1<<<dim3(1, rows), NT, 0, st>>>(P);
+  }
+  {
+    Launch l("k_select2", st);
+    k_select2<<<dim3(P.Gs, rows), NT, 0, st>>>(P);
+  }
+  {
+    Launch l("k_select3", st);
+    k_select3<<<dim3(P.Gs, rows), NT, 0, st>>>(P);
+  }
+  {
+    Launch l("k_filter", st);
+    k_filter<<<dim3(P.Gf, rows), NT, 0, st>>>(P, scores);
+  }
+  {
+    Launch l("k_shard_pack", st);
+    k_shard_pack<<<(rows + 127) / 128, 128, 0, st>>>(P, meta);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_finish(const StreamPlan& P, const StreamPlan& Pb, const float* scores, float* p_out,
+                                double* b_out, double* sumf_out, uint32_t* status_out, int world,
+                                const void* g_fpart, const uint32_t* g_meta, const float* g_band, cudaStream_t st) {
+  const unsigned rows = (unsigned)P.rows;
+  cudaError_t e;
+  {
+    Launch l("k_shard_unpack", st);
+    k_shard_unpack<<<rows, NT, 0, st>>>(Pb, world, reinterpret_cast<const FPart*>(g_fpart), g_meta);
+  }
+  {
+    Launch l("k_shard_compact", st);
+    k_shard_compact<<<dim3(64, rows), NT, 0, st>>>(Pb, world, g_band, g_meta);
+  }
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)Pb.band_cs, rows, 1);
+    cfg.blockDim = dim3(kBandThreads, 1, 1);
+    cfg.dynamicSmemBytes = kBandSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)Pb.band_cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    Launch l("k_band", st);
+    e = cudaLaunchKernelEx(&cfg, k_band, Pb);
+    if (e != cudaSuccess) return e;
+  }
+  // no recovery here: a row the band does not certify keeps its miss bits and
+  // the caller solves it again from the whole row
+  {
+    Launch l("k_memb", st);
+    k_memb<false, false><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, nullptr);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_bwd_partials(const StreamBwd& a, bool with_alpha, cudaStream_t st) {
+  Launch l("k_bwd_reduce", st);
+  if (with_alpha) k_bwd_reduce<true><<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+  else k_bwd_reduce<false><<<dim3(a.Gb, (unsigned)a.rows), NT, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shard_bwd_finish(const StreamBwd& a, const void* parts_all, int world, cudaStream_t st) {
+  {
+    Launch l("k_bwd_combine", st);
+    const BPart* pa = reinterpret_cast<const BPart*>(parts_all);
+    if (a.grad_alpha) k_bwd_combine<true><<<(unsigned)a.rows, NT, 0, st>>>(a, pa, world);
+    else k_bwd_combine<false><<<(unsigned)a.rows, NT, 0, st>>>(a, pa, world);
   }
   {
     Launch l("k_bwd_apply", st);

@@ -297,6 +297,86 @@ LAPSUM_API int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_
                                        double* sumf_out, uint32_t* row_status, lapsum_row_stats* stats,
                                        const lapsum_params* params, void* stream);
 
+/*
+ * ---- sharded rows -----------------------------------------------------------
+ * One long row split over G GPUs in contiguous shards (GPU g holds scores
+ * [shard_lo, shard_lo + n) of a row n_total long; every GPU passes the same
+ * rows, n_total, k, alpha and params).  The probabilistic bracketing of the
+ * Fast LapSum technical summary (section 2.2) needs only small exchanges
+ * between the GPUs, which the caller makes between the calls below (NCCL
+ * through torch.distributed, for instance); no call waits on another GPU:
+ *
+ *   1. lapsum_shard_fwd_sample      writes x_sample, x_hist
+ *      SUM-reduce x_sample and x_hist over the GPUs, in place (int32 or
+ *      uint32 sums: every sample slot is non-zero on at most one GPU)
+ *   2. lapsum_shard_fwd_filter      reads them; writes x_meta, x_fpart, x_band
+ *      GATHER x_meta, x_fpart, x_band of all GPUs, GPU-major, into g_meta,
+ *      g_fpart, g_band (G times the size of each)
+ *   3. lapsum_shard_fwd_finish      every GPU solves the same band for the
+ *      same b, then writes the memberships of its shard
+ *
+ * The sample is the one a single GPU would draw for the whole row.  A row the
+ * band does not certify (its row_status lacks LAPSUM_ROW_CERTIFIED) is not
+ * widened here: the caller solves it again from the whole row.  The workspace
+ * keeps state from call 1 to call 3 and must not be shared meanwhile.
+ *
+ * Backward (analytic VJP, section 2.1): lapsum_shard_bwd_partials writes this
+ * shard's reduction partials into x_parts; GATHER them GPU-major into g_parts;
+ * lapsum_shard_bwd_finish forms lambda (and dL/dalpha when with_alpha was set
+ * in the partials call) from all of them and writes dL/dr of its shard.
+ *
+ * Exchange buffers are device memory, 16-byte aligned, of the sizes
+ * lapsum_shard_layout_get returns (per GPU; the gathered ones G times that).
+ */
+typedef struct lapsum_shard_layout {
+    int32_t sample_m;        /* localization sample size */
+    int32_t reserved;
+    int64_t band_cap;        /* band slots per row and GPU */
+    size_t sample_bytes;     /* x_sample: uint32 [rows][sample_m]  (summed) */
+    size_t hist_bytes;       /* x_hist:   uint32 [rows][2048]      (summed) */
+    size_t meta_bytes;       /* x_meta:   uint32 [rows][8]         (gathered) */
+    size_t fpart_bytes;      /* x_fpart:  [rows][4096] x 32 bytes  (gathered) */
+    size_t band_bytes;       /* x_band:   fp32 [rows][band_cap]    (gathered) */
+    size_t parts_bytes;      /* x_parts:  [rows][4096] x 48 bytes  (gathered) */
+    size_t workspace_bytes;  /* workspace of the forward and backward calls */
+} lapsum_shard_layout;
+
+/* Sizes for rows of n_total scores (zeros for an invalid shape). */
+LAPSUM_API void lapsum_shard_layout_get(int64_t rows, int64_t n_total, const lapsum_params* params,
+                                        lapsum_shard_layout* out);
+
+LAPSUM_API int lapsum_shard_fwd_sample(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                                       int64_t shard_lo, int64_t n_total, double k, double alpha,
+                                       uint32_t* x_sample, uint32_t* x_hist, void* workspace,
+                                       size_t workspace_bytes, const lapsum_params* params, void* stream);
+
+LAPSUM_API int lapsum_shard_fwd_filter(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                                       int64_t shard_lo, int64_t n_total, double k, double alpha,
+                                       const uint32_t* x_sample, const uint32_t* x_hist, uint32_t* x_meta,
+                                       void* x_fpart, float* x_band, void* workspace, size_t workspace_bytes,
+                                       const lapsum_params* params, void* stream);
+
+/* p_out: fp32 [rows, row_stride], this shard's memberships; b_out, sumf_out:
+   fp64 [rows], the same on every GPU; row_status as for lapsum_topk_fwd. */
+LAPSUM_API int lapsum_shard_fwd_finish(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
+                                       int64_t shard_lo, int64_t n_total, double k, double alpha, int world,
+                                       const uint32_t* g_meta, const void* g_fpart, const float* g_band,
+                                       float* p_out, double* b_out, double* sumf_out, uint32_t* row_status,
+                                       void* workspace, size_t workspace_bytes, const lapsum_params* params,
+                                       void* stream);
+
+LAPSUM_API int lapsum_shard_bwd_partials(const float* scores, const float* grad_p, const double* b, int64_t rows,
+                                         int64_t n, int64_t row_stride, double alpha, int with_alpha,
+                                         void* x_parts, void* stream);
+
+/* grad_scores: this shard's dL/dr; grad_k, grad_alpha (may be NULL): fp64
+   [rows], the same on every GPU. */
+LAPSUM_API int lapsum_shard_bwd_finish(const float* scores, const float* grad_p, const double* b, int64_t rows,
+                                       int64_t n, int64_t row_stride, double alpha, int world,
+                                       const void* g_parts, float* grad_scores, double* grad_k,
+                                       double* grad_alpha, void* workspace, size_t workspace_bytes,
+                                       void* stream);
+
 /* Text of the CUDA error behind the last LAPSUM_ECUDA returned on the
    calling host thread ("no error" if none). */
 LAPSUM_API const char* lapsum_last_cuda_error(void);

@@ -30,7 +30,8 @@ def test_header_declares_the_boundary():
     assert names == sorted([
         "lapsum_default_params", "lapsum_dftopk_fwd", "lapsum_last_cuda_error", "lapsum_launch_count",
         "lapsum_status_string", "lapsum_topk_bwd", "lapsum_topk_bwd_rows", "lapsum_topk_fwd", "lapsum_topk_fwd_noalloc",
-        "lapsum_topk_fwd_rows", "lapsum_topk_fwd_sparse",
+        "lapsum_topk_fwd_rows", "lapsum_topk_fwd_sparse", "lapsum_shard_bwd_finish", "lapsum_shard_bwd_partials",
+        "lapsum_shard_fwd_filter", "lapsum_shard_fwd_finish", "lapsum_shard_fwd_sample", "lapsum_shard_layout_get",
         "lapsum_topk_sparse_workspace_size", "lapsum_topk_workspace_size",
         "lapsum_trace_collect", "lapsum_trace_enable",
     ])
