@@ -87,7 +87,7 @@ extern "C" {
 typedef struct lapsum_params {
     uint32_t sample_m;      /* localization sample size m; 0 = automatic */
     uint32_t force_path;    /* 0 = normal; OR of LAPSUM_FORCE_* (tests) */
-    double z;               /* bracket half-width in binomial sigmas; 0 = 5 */
+    double z;               /* bracket half-width in binomial sigmas; 0 = 4 */
     uint64_t seed;          /* seed of the sampling generator (splitmix64) */
     int64_t band_capacity;  /* band slots per row; 0 = automatic */
     int32_t max_widen;      /* widenings before the full sort: 0 or 1;

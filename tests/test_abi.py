@@ -51,7 +51,7 @@ def test_params_struct_layout(lib):
     assert ctypes.sizeof(lt._CParams) == 40
     c = lt._CParams()
     lib.lapsum_default_params(ctypes.byref(c))
-    assert c.z == 5.0 and c.max_widen == -1 and c.sample_m == 0 and c.seed == 0
+    assert c.z == 4.0 and c.max_widen == -1 and c.sample_m == 0 and c.seed == 0
     assert lt.STATS_DTYPE.itemsize == 88
 
 
