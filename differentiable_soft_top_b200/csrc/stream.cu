@@ -568,16 +568,20 @@ constexpr int kTargetCap = kBins;  // a gathered bin becomes a table of its valu
 constexpr int kMaxLevels = 4;
 constexpr int kMaxCluster = 16;
 constexpr int kBandThreads = 512;
-constexpr int kLimbBits = 11;                  // P, Q kept as three 11-bit limb sums
-constexpr int kLimbSliceMax = (1 << 21) - 1;   // slices up to this size cannot overflow a limb word
+// P and Q are kept as exact integer sums of 2^-31 fixed-point terms (at most
+// 2^31 each), split into 32-bit words that cannot overflow for the slice:
+constexpr int kHalfSliceMax = 65535;          // two 16-bit limbs (two adds per term)
+constexpr int kLimbBits = 11;                 // or three 11-bit limbs (three adds)
+constexpr int kLimbSliceMax = (1 << 21) - 1;  // up to this many terms; beyond, a carried 64-bit sum
+enum : uint32_t { kSumHalves = 0, kSumLimbs = 1, kSumWide = 2 };
 
 struct BinPart {  // one CTA's bins
   uint32_t cnt[kBins];
   uint32_t kmin[kBins];
   uint32_t kmax[kBins];
-  uint32_t P[3][kBins];  // limbs (or low word, high word when `wide`)
+  uint32_t P[3][kBins];  // limb words, by `mode`
   uint32_t Q[3][kBins];
-  uint32_t wide;         // 1: P, Q as two-word 64-bit sums (slices too long for limbs)
+  uint32_t mode;         // kSumHalves, kSumLimbs or kSumWide (low word, high word)
 };
 struct TargetBuf {
   uint32_t keys[kTargetCap];
@@ -634,6 +638,11 @@ __device__ __forceinline__ uint32_t edge_key(uint32_t klo, uint32_t khi, int shi
 __device__ __forceinline__ uint32_t fx_term(float d, float c2) {
   return __float2uint_rn(exp2f(d * c2) * 0x1p31f);
 }
+// a term into two 16-bit limb words (plain reductions)
+__device__ __forceinline__ void add_halves(uint32_t (*L)[kBins], int t, uint32_t v) {
+  atomicAdd(&L[0][t], v & 0xFFFFu);
+  atomicAdd(&L[1][t], v >> 16);
+}
 // a term into three limb words (no return value needed: plain reductions)
 __device__ __forceinline__ void add_limbs(uint32_t (*L)[kBins], int t, uint32_t v) {
   constexpr uint32_t m = (1u << kLimbBits) - 1u;
@@ -646,10 +655,11 @@ __device__ __forceinline__ void add_wide(uint32_t (*L)[kBins], int t, uint32_t v
   const uint32_t old = atomicAdd(&L[0][t], v);
   if (old > 0xFFFFFFFFu - v) atomicAdd(&L[1][t], 1u);
 }
-__device__ __forceinline__ double fx_value(uint32_t w0, uint32_t w1, uint32_t w2, bool wide) {
-  const double v = wide ? (double)w1 * 4294967296.0 + (double)w0
-                        : ((double)w2 * (double)(1u << (2 * kLimbBits)) + (double)w1 * (double)(1u << kLimbBits)) +
-                              (double)w0;
+__device__ __forceinline__ double fx_value(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t mode) {
+  const double v = mode == kSumWide    ? (double)w1 * 4294967296.0 + (double)w0
+                   : mode == kSumHalves ? (double)w1 * 65536.0 + (double)w0
+                                        : ((double)w2 * (double)(1u << (2 * kLimbBits)) +
+                                           (double)w1 * (double)(1u << kLimbBits)) + (double)w0;
   return v * 0x1p-31;
 }
 
@@ -666,7 +676,7 @@ constexpr int kSliceBatch = 8;  // loads in flight per thread
 template <int NTX>
 __device__ void bin_slice(const float* src, int n, bool write_stage, bool read_stage, float* stage, uint32_t klo,
                           uint32_t khi, int shift, float c2, BinPart& bp) {
-  const bool wide = n > kLimbSliceMax;
+  const uint32_t mode = n <= kHalfSliceMax ? kSumHalves : (n <= kLimbSliceMax ? kSumLimbs : kSumWide);
   for (int t = threadIdx.x; t < kBins; t += NTX) {
     bp.cnt[t] = 0u;
     bp.kmin[t] = 0xFFFFFFFFu;
@@ -677,7 +687,7 @@ __device__ void bin_slice(const float* src, int n, bool write_stage, bool read_s
       bp.Q[l][t] = 0u;
     }
   }
-  if (threadIdx.x == 0) bp.wide = wide ? 1u : 0u;
+  if (threadIdx.x == 0) bp.mode = mode;
   __syncthreads();
   const bool first_from_stage = read_stage && !write_stage;
   for (int j0 = 0; j0 < n; j0 += NTX * kSliceBatch) {
@@ -721,7 +731,10 @@ __device__ void bin_slice(const float* src, int n, bool write_stage, bool read_s
           const int t = (int)((key - klo) >> shift);
           const uint32_t tp = fx_term(y - key2f(bp.kmax[t]), c2);
           const uint32_t tq = fx_term(key2f(bp.kmin[t]) - y, c2);
-          if (!wide) {
+          if (mode == kSumHalves) {
+            add_halves(bp.P, t, tp);
+            add_halves(bp.Q, t, tq);
+          } else if (mode == kSumLimbs) {
             add_limbs(bp.P, t, tp);
             add_limbs(bp.Q, t, tq);
           } else {
@@ -767,7 +780,7 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
         q0[i] = pq->Q[0][t];
         q1[i] = pq->Q[1][t];
         q2[i] = pq->Q[2][t];
-        wd[i] = pq->wide;
+        wd[i] = pq->mode;
       }
     }
     uint32_t cnt = 0u, kmn = 0xFFFFFFFFu, kmx = 0u;
@@ -789,8 +802,8 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
 #pragma unroll
     for (int q = 0; q < QM; ++q) {
       if (c[q]) {
-        Ps += fx_value(p0[q], p1[q], p2[q], wd[q] != 0u) * exp_call(((double)key2f(mx[q]) - ymax) * inva);
-        Qs += fx_value(q0[q], q1[q], q2[q], wd[q] != 0u) * exp_call((ymin - (double)key2f(mn[q])) * inva);
+        Ps += fx_value(p0[q], p1[q], p2[q], wd[q]) * exp_call(((double)key2f(mx[q]) - ymax) * inva);
+        Qs += fx_value(q0[q], q1[q], q2[q], wd[q]) * exp_call((ymin - (double)key2f(mn[q])) * inva);
       }
     }
     for (int o = 1; o < L; o <<= 1) {
