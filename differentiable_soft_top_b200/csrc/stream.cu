@@ -577,8 +577,10 @@ enum : uint32_t { kSumHalves = 0, kSumLimbs = 1, kSumWide = 2 };
 
 struct BinPart {  // one CTA's bins
   uint32_t cnt[kBins];
-  uint32_t kmin[kBins];
+  uint32_t kmin[kBins];  // this CTA's extreme keys per bin
   uint32_t kmax[kBins];
+  uint32_t gmin[kBins];  // the whole cluster's: the anchors of the sums, so that
+  uint32_t gmax[kBins];  // every CTA's terms are the same integers whatever its slice
   uint32_t P[3][kBins];  // limb words, by `mode`
   uint32_t Q[3][kBins];
   uint32_t mode;         // kSumHalves, kSumLimbs or kSumWide (low word, high word)
@@ -655,13 +657,6 @@ __device__ __forceinline__ void add_wide(uint32_t (*L)[kBins], int t, uint32_t v
   const uint32_t old = atomicAdd(&L[0][t], v);
   if (old > 0xFFFFFFFFu - v) atomicAdd(&L[1][t], 1u);
 }
-__device__ __forceinline__ double fx_value(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t mode) {
-  const double v = mode == kSumWide    ? (double)w1 * 4294967296.0 + (double)w0
-                   : mode == kSumHalves ? (double)w1 * 65536.0 + (double)w0
-                                        : ((double)w2 * (double)(1u << (2 * kLimbBits)) +
-                                           (double)w1 * (double)(1u << kLimbBits)) + (double)w0;
-  return v * 0x1p-31;
-}
 
 // value j of a worker's slice: from the shared copy, or from L2
 __device__ __forceinline__ float slice_val(const float* src, const float* stage, bool staged, int j) {
@@ -670,12 +665,13 @@ __device__ __forceinline__ float slice_val(const float* src, const float* stage,
 
 constexpr int kSliceBatch = 8;  // loads in flight per thread
 
-// Bins the n values at src into bp.  write_stage: copy the first kStageCap of
-// them into `stage` on the way; read_stage: read them from there.  All
-// threads of the block call it.
+// Pass 1 over the n values at src: count and extreme keys per bin into bp.
+// write_stage: copy the first kStageCap of them into `stage` on the way
+// (otherwise they come from `stage` when read_stage).  All threads of the
+// block call it.
 template <int NTX>
-__device__ void bin_slice(const float* src, int n, bool write_stage, bool read_stage, float* stage, uint32_t klo,
-                          uint32_t khi, int shift, float c2, BinPart& bp) {
+__device__ void bin_count(const float* src, int n, bool write_stage, bool read_stage, float* stage, uint32_t klo,
+                          uint32_t khi, int shift, BinPart& bp) {
   const uint32_t mode = n <= kHalfSliceMax ? kSumHalves : (n <= kLimbSliceMax ? kSumLimbs : kSumWide);
   for (int t = threadIdx.x; t < kBins; t += NTX) {
     bp.cnt[t] = 0u;
@@ -714,6 +710,46 @@ __device__ void bin_slice(const float* src, int n, bool write_stage, bool read_s
     }
   }
   __syncthreads();
+}
+
+// The cluster's extreme keys per bin, into every CTA's gmin / gmax: this CTA
+// merges its kBins / cs bins over all CTAs (L lanes per bin, each taking every
+// L-th CTA) and writes them to all CTAs.  A cluster barrier must follow
+// before they are read.
+template <int NTX>
+__device__ void merge_extremes(BandShared& S, int cs, int rank) {
+  const int per = kBins / cs;
+  int L = NTX / per;
+  L = L < 1 ? 1 : (L > cs ? cs : L);
+  const int sub = (int)threadIdx.x & (L - 1);
+  for (int base = (int)threadIdx.x / L; base < per; base += NTX / L) {
+    const int t = rank * per + base;
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    for (int q = sub; q < cs; q += L) {
+      const BinPart* pq = at_rank(&S.u.part, q, cs);
+      mn = min(mn, pq->kmin[t]);
+      mx = max(mx, pq->kmax[t]);
+    }
+    for (int o = 1; o < L; o <<= 1) {
+      mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    for (int q = sub; q < cs; q += L) {
+      BinPart* pq = at_rank(&S.u.part, q, cs);
+      pq->gmin[t] = mn;
+      pq->gmax[t] = mx;
+    }
+  }
+}
+
+// Pass 2: the sums P = sum exp((y - ymax)/a) and Q = sum exp((ymin - y)/a) per
+// bin, with ymax, ymin the cluster's extremes (bp.gmin / gmax), as integer
+// sums of 2^-31 fixed-point terms: the same integers whichever CTA holds a
+// value, so the merged sums do not depend on how the band was split.
+template <int NTX>
+__device__ void bin_sums(const float* src, int n, bool read_stage, const float* stage, uint32_t klo, uint32_t khi,
+                         int shift, float c2, BinPart& bp) {
+  const uint32_t mode = bp.mode;
   for (int j0 = 0; j0 < n; j0 += NTX * kSliceBatch) {
     float v[kSliceBatch];
 #pragma unroll
@@ -729,8 +765,8 @@ __device__ void bin_slice(const float* src, int n, bool write_stage, bool read_s
         const uint32_t key = f2key(y);
         if (key >= klo && key <= khi) {
           const int t = (int)((key - klo) >> shift);
-          const uint32_t tp = fx_term(y - key2f(bp.kmax[t]), c2);
-          const uint32_t tq = fx_term(key2f(bp.kmin[t]) - y, c2);
+          const uint32_t tp = fx_term(y - key2f(bp.gmax[t]), c2);
+          const uint32_t tq = fx_term(key2f(bp.gmin[t]) - y, c2);
           if (mode == kSumHalves) {
             add_halves(bp.P, t, tp);
             add_halves(bp.Q, t, tq);
@@ -747,10 +783,18 @@ __device__ void bin_slice(const float* src, int n, bool write_stage, bool read_s
   }
 }
 
-// This CTA's share of the bins, merged over all CTAs (in CTA order) into the
-// leader's table together with the edge factors of solve_bins; L lanes per
-// bin, each taking every L-th CTA.  Every load of a CTA's bin is issued before
-// any is used.
+// a CTA's limb words of one sum as the exact integer they stand for
+__device__ __forceinline__ unsigned long long fx_int(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t mode) {
+  if (mode == kSumWide) return ((unsigned long long)w1 << 32) | w0;
+  if (mode == kSumHalves) return ((unsigned long long)w1 << 16) + w0;
+  return ((unsigned long long)w2 << (2 * kLimbBits)) + ((unsigned long long)w1 << kLimbBits) + w0;
+}
+
+// This CTA's share of the bins, merged over all CTAs into the leader's table
+// together with the edge factors of solve_bins.  The sums are integers anchored
+// at the cluster's extremes, so merging is an exact integer addition (the same
+// result in any order).  L lanes per bin, each taking every L-th CTA; every
+// load of a CTA's bin is issued before any is used.
 template <int NTX>
 __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32_t khi, int shift, double inva) {
   const int per = kBins / cs;
@@ -764,7 +808,7 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
   BinTable<kBins>* tab0 = at_rank(&S.tu.tab, 0, cs);
   for (int base = (int)threadIdx.x / L; base < per; base += NTX / L) {
     const int t = rank * per + base;
-    uint32_t c[QM], mn[QM], mx[QM], p0[QM], p1[QM], p2[QM], q0[QM], q1[QM], q2[QM], wd[QM];
+    uint32_t c[QM], p0[QM], p1[QM], p2[QM], q0[QM], q1[QM], q2[QM], md[QM];
 #pragma unroll
     for (int i = 0; i < QM; ++i) {
       const int q = sub + i * L;
@@ -772,45 +816,34 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
       if (q < cs) {
         const BinPart* pq = at_rank(&S.u.part, q, cs);
         c[i] = pq->cnt[t];
-        mn[i] = pq->kmin[t];
-        mx[i] = pq->kmax[t];
         p0[i] = pq->P[0][t];
         p1[i] = pq->P[1][t];
         p2[i] = pq->P[2][t];
         q0[i] = pq->Q[0][t];
         q1[i] = pq->Q[1][t];
         q2[i] = pq->Q[2][t];
-        wd[i] = pq->mode;
+        md[i] = pq->mode;
       }
     }
-    uint32_t cnt = 0u, kmn = 0xFFFFFFFFu, kmx = 0u;
+    uint32_t cnt = 0u;
+    unsigned long long Pi = 0ull, Qi = 0ull;
 #pragma unroll
-    for (int q = 0; q < QM; ++q) {
-      if (c[q]) {
-        cnt += c[q];
-        kmn = min(kmn, mn[q]);
-        kmx = max(kmx, mx[q]);
+    for (int i = 0; i < QM; ++i) {
+      if (c[i]) {
+        cnt += c[i];
+        Pi += fx_int(p0[i], p1[i], p2[i], md[i]);
+        Qi += fx_int(q0[i], q1[i], q2[i], md[i]);
       }
     }
     for (int o = 1; o < L; o <<= 1) {
       cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-      kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
-      kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
-    }
-    const double ymax = (double)key2f(kmx), ymin = (double)key2f(kmn);
-    double Ps = 0.0, Qs = 0.0;
-#pragma unroll
-    for (int q = 0; q < QM; ++q) {
-      if (c[q]) {
-        Ps += fx_value(p0[q], p1[q], p2[q], wd[q]) * exp_call(((double)key2f(mx[q]) - ymax) * inva);
-        Qs += fx_value(q0[q], q1[q], q2[q], wd[q]) * exp_call((ymin - (double)key2f(mn[q])) * inva);
-      }
-    }
-    for (int o = 1; o < L; o <<= 1) {
-      Ps += __shfl_xor_sync(0xffffffffu, Ps, o);
-      Qs += __shfl_xor_sync(0xffffffffu, Qs, o);
+      Pi += __shfl_xor_sync(0xffffffffu, Pi, o);
+      Qi += __shfl_xor_sync(0xffffffffu, Qi, o);
     }
     if (sub == 0) {
+      const BinPart& own = S.u.part;
+      const double ymax = (double)key2f(own.gmax[t]), ymin = (double)key2f(own.gmin[t]);
+      const double Ps = (double)Pi * 0x1p-31, Qs = (double)Qi * 0x1p-31;
       const double elo = (double)key2f(edge_key(klo, khi, shift, t));
       const float eup = key2f(edge_key(klo, khi, shift, t + 1));
       const double ehi = (double)eup;
@@ -896,7 +929,12 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
       levels = level + 1;
       // a worker keeps its slice in shared memory; a lone CTA (cs == 1) holds
       // the table in the same place, so it rereads its slice from L2 past level 0
-      bin_slice<NTX>(src, n, level == 0, level == 0 || cs > 1, S.tu.stage, klo, khi, shift, c2, S.u.part);
+      const bool staged = level == 0 || cs > 1;
+      bin_count<NTX>(src, n, level == 0, staged, S.tu.stage, klo, khi, shift, S.u.part);
+      cl_sync(cs);
+      merge_extremes<NTX>(S, cs, rank);
+      cl_sync(cs);
+      bin_sums<NTX>(src, n, staged, S.tu.stage, klo, khi, shift, c2, S.u.part);
       cl_sync(cs);
       merge_bins<NTX>(S, cs, rank, klo, khi, shift, inva);
       cl_sync(cs);

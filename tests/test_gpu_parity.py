@@ -287,6 +287,24 @@ def test_deterministic():
     assert np.array_equal(a["grad"], b["grad"])
 
 
+def test_deterministic_with_a_band_cluster():
+    """A band split over a cluster of CTAs (the 1e8 workload's regime): the
+    band arrives in a different order each call and is sliced differently,
+    yet the bin sums are exact integers anchored at the cluster's extremes,
+    so every result is bit-identical."""
+    n = 30_000_000
+    x = make_scores("uniform", 1, n, seed=3)
+    g = make_grad(1, n, seed=4)
+    k, alpha = 3e5, 1e-3
+    runs = [gpu_run(x, g, k, alpha) for _ in range(3)]
+    st = runs[0]["stats"]
+    for r in runs[1:]:
+        assert np.array_equal(runs[0]["b"], r["b"]) and np.array_equal(runs[0]["sumf"], r["sumf"])
+        assert np.array_equal(runs[0]["p"], r["p"]) and np.array_equal(runs[0]["grad"], r["grad"])
+    res = lt.forward(torch.from_numpy(x).cuda(), k, alpha, stats=True)
+    assert int(res.stats[0]["band"]) > 2 * 16384  # more than one CTA of the cluster bins it
+
+
 def test_autograd_wrapper(orc):
     w, x, g = case("c1")
     xt = torch.from_numpy(x[0]).cuda().requires_grad_(True)
