@@ -62,6 +62,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-sparse", action="store_true", help="skip the sparse-forward comparison")
     ap.add_argument("--no-dftopk", action="store_true", help="skip the DFTopK-relaxation comparison")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="scale the workload to n scores per row (k keeps its ratio)")
@@ -362,6 +363,26 @@ def timed_calls(torch, fn, steps, flush, stream, dist, dev):
     return max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / steps, dist, dev)
 
 
+def graph_replay(torch, step, dev, dist, flush, steps):
+    """The same step captured once into a CUDA graph and replayed, as a
+    training loop with fixed shapes would run it (the library makes no host
+    synchronisation, so its launches capture as they are).  Each replay
+    after the L2 flush; CUDA events around the replay."""
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    torch.cuda.synchronize(dev)
+    ms = timed_calls(torch, graph.replay, steps, flush, torch.cuda.current_stream(dev), dist, dev)
+    del graph
+    return ms
+
+
 def dftopk_vs_lapsum(lt, torch, w, x, dev, dist, flush, steps):
     """The DFTopK relaxation (threshold at the midpoint of the k-th and
     (k+1)-th largest, memberships at alpha) against the exact-budget forward on
@@ -535,6 +556,12 @@ def main():
     kernels = {k: {"launches": v[0], "ms_per_launch": v[1] / v[0], "share": v[1] / sum(t[1] for t in trace.values())}
                for k, v in sorted(trace.items(), key=lambda kv: -kv[1][1])}
 
+    graph = None
+    if not args.no_graph:
+        gms = graph_replay(torch, step, dev, dist, flush, args.steps)
+        graph = {"ms_per_step": gms, "value": world * scores_per_step / (gms * 1e-3),
+                 "note": "the step captured once into a CUDA graph and replayed (flush outside the graph); "
+                         "the headline value above is the eager calls"}
     sparse = None
     if not args.no_sparse and n > 16384:
         sparse = sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, args.steps)
@@ -583,6 +610,7 @@ def main():
         "kernels": kernels,
         "cpu_baseline": cpu,
         "e2e": e2e,
+        "graph_replay": graph,
         "sparse_forward": sparse,
         "dftopk_forward": dftopk,
         "gpu_launches": launches,

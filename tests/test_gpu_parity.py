@@ -657,3 +657,40 @@ def test_autograd_per_row_k_and_alpha(orc):
         ref_a = orc.backward_alpha(x[i], g[i], b_ref, a)
         assert float(kt.grad[i]) == pytest.approx(lam, rel=1e-4, abs=1e-6 * (1 + abs(lam)))
         assert float(at.grad[i]) == pytest.approx(ref_a, rel=1e-4, abs=alpha_tol(x[i], g[i], b_ref, a) + 1e-6)
+
+
+@pytest.mark.parametrize("name,n,rows", [("c3", 2_000_000, None), ("c5", 16384, 8)])
+def test_capture_in_a_cuda_graph(name, n, rows):
+    """forward_into / backward_into make no host synchronisation, so a step
+    captures into a CUDA graph; its replays give the eager results bit for bit."""
+    w, x, g = case(name, n=n, rows=rows)
+    xt, gt = torch.from_numpy(x).cuda(), torch.from_numpy(g).cuda()
+    rws, nn = x.shape
+    p, grad = torch.empty_like(xt), torch.empty_like(xt)
+    b = torch.empty(rws, dtype=torch.float64, device="cuda")
+    sumf, gk = torch.empty_like(b), torch.empty_like(b)
+    st = torch.empty(rws, dtype=torch.int32, device="cuda")
+    ws = torch.empty(lt.workspace_size(rws, nn), dtype=torch.uint8, device="cuda")
+
+    def step():
+        lt.forward_into(xt, w.k, w.alpha, p, b, sumf, st, ws)
+        lt.backward_into(xt, gt, b, w.alpha, grad, ws, grad_k=gk)
+
+    step()
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (p, b, sumf, grad, gk)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for t in (p, b, grad):
+        t.zero_()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    for a, r in zip((p, b, sumf, grad, gk), ref):
+        assert torch.equal(a, r)
