@@ -73,7 +73,56 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   int nl = 0, nr = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
-  for (int base = 0; base < n; base += NT) {
+  // four scores per thread and step (the row is 16-byte aligned in shared
+  // memory); fp32 partial tail sums folded into fp64 once per step
+  const int n4 = n >> 2;
+  const float4* row4 = reinterpret_cast<const float4*>(row);
+  for (int base = 0; base < n4; base += NT) {
+    const int v = base + threadIdx.x;
+    const bool act = v < n4;
+    const float4 q = act ? row4[v] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const float xs[4] = {q.x, q.y, q.z, q.w};
+    float pl = 0.0f, pr = 0.0f;
+    uint32_t inb = 0u;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float x = xs[w];
+      const bool isL = x < aL, isR = x >= aR;
+      const float e = exp2f(fminf(x - aL, aR - x) * c2);
+      pl += isL ? e : 0.0f;
+      pr += isR ? e : 0.0f;
+      nl += (act && isL) ? 1 : 0;
+      nr += (act && isR) ? 1 : 0;
+      if (act && !(fabsf(x) < CUDART_INF_F)) bad = 1u;
+      inb |= (act && !(isL || isR)) ? (1u << w) : 0u;
+    }
+    if (act) {
+      sl += (double)pl;
+      sr += (double)pr;
+    }
+    if (__any_sync(0xffffffffu, inb != 0u)) {  // rare: this warp holds band values
+      const int c = __popc(inb);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      int wbase = 0;
+      if (lane == 0) wbase = atomicAdd(s_cnt, total);
+      wbase = __shfl_sync(0xffffffffu, wbase, 0);
+      int pos = wbase + incl - c;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        if ((inb >> w) & 1u) {
+          if (pos < bcap) band[pos] = f2key(xs[w]);
+          ++pos;
+        }
+      }
+    }
+  }
+  for (int base = n4 << 2; base < n; base += NT) {
     const int i = base + threadIdx.x;
     const bool act = i < n;
     const float x = act ? row[i] : 0.0f;
@@ -432,18 +481,29 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
       else shift_add(fabsf(z) * c2, gv, m, ps, psg, S, SG);
     };
     const int n4 = a.vec ? (n >> 2) : 0;
-    for (int v = threadIdx.x; v < n4; v += NT) {
-      const float4 xv = __ldg(reinterpret_cast<const float4*>(x) + v);
-      const float4 gv = __ldg(reinterpret_cast<const float4*>(g) + v);
-      float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
-      acc(xv.x, gv.x, ps, psg, psz, psgz);
-      acc(xv.y, gv.y, ps, psg, psz, psgz);
-      acc(xv.z, gv.z, ps, psg, psz, psgz);
-      acc(xv.w, gv.w, ps, psg, psz, psgz);
-      S += (double)ps;
-      SG += (double)psg;
-      SZ += (double)psz;
-      SGZ += (double)psgz;
+    // kB float4 of r and of g in flight per thread, then the sums
+    constexpr int kB = 4;
+    for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
+      float4 xv[kB], gv[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int v = v0 + u * NT;
+        xv[u] = v < n4 ? __ldg(reinterpret_cast<const float4*>(x) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[u] = v < n4 ? __ldg(reinterpret_cast<const float4*>(g) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        if (v0 + u * NT >= n4) break;
+        float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
+        acc(xv[u].x, gv[u].x, ps, psg, psz, psgz);
+        acc(xv[u].y, gv[u].y, ps, psg, psz, psgz);
+        acc(xv[u].z, gv[u].z, ps, psg, psz, psgz);
+        acc(xv[u].w, gv[u].w, ps, psg, psz, psgz);
+        S += (double)ps;
+        SG += (double)psg;
+        SZ += (double)psz;
+        SGZ += (double)psgz;
+      }
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
       float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
@@ -458,15 +518,25 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     const double lam = bad ? CUDART_NAN : SG / S;  // NaN also reaches every grad of the row
     const float lh = __double2float_rn(lam);
     const float ll = __double2float_rn(lam - (double)lh);
-    for (int v = threadIdx.x; v < n4; v += NT) {
-      const float4 xv = __ldcs(reinterpret_cast<const float4*>(x) + v);
-      const float4 gv = __ldcs(reinterpret_cast<const float4*>(g) + v);
-      float4 ov;
-      ov.x = exp2f(fmaf(-fabsf((xv.x - bh) - bl), c2, lg)) * ((gv.x - lh) - ll);
-      ov.y = exp2f(fmaf(-fabsf((xv.y - bh) - bl), c2, lg)) * ((gv.y - lh) - ll);
-      ov.z = exp2f(fmaf(-fabsf((xv.z - bh) - bl), c2, lg)) * ((gv.z - lh) - ll);
-      ov.w = exp2f(fmaf(-fabsf((xv.w - bh) - bl), c2, lg)) * ((gv.w - lh) - ll);
-      stg_stream(reinterpret_cast<float4*>(o) + v, ov);
+    for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
+      float4 xv[kB], gv[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int v = v0 + u * NT;
+        xv[u] = v < n4 ? __ldcs(reinterpret_cast<const float4*>(x) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[u] = v < n4 ? __ldcs(reinterpret_cast<const float4*>(g) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int v = v0 + u * NT;
+        if (v >= n4) break;
+        float4 ov;
+        ov.x = exp2f(fmaf(-fabsf((xv[u].x - bh) - bl), c2, lg)) * ((gv[u].x - lh) - ll);
+        ov.y = exp2f(fmaf(-fabsf((xv[u].y - bh) - bl), c2, lg)) * ((gv[u].y - lh) - ll);
+        ov.z = exp2f(fmaf(-fabsf((xv[u].z - bh) - bl), c2, lg)) * ((gv[u].z - lh) - ll);
+        ov.w = exp2f(fmaf(-fabsf((xv[u].w - bh) - bl), c2, lg)) * ((gv[u].w - lh) - ll);
+        stg_stream(reinterpret_cast<float4*>(o) + v, ov);
+      }
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT)
       o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
