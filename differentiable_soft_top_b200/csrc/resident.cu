@@ -27,10 +27,10 @@ struct ResLayout {
   size_t row, samp, samp_tmp, band, band_tmp, dscr, hist, red, mbar, total;
 };
 
-__host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap) {
+__host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool row_in_smem) {
   ResLayout L;
   size_t o = 0;
-  L.row = o;      o = (o + 4 * (size_t)n + 15) & ~size_t(15);
+  L.row = o;      o = (o + (row_in_smem ? 4 * (size_t)n : 0) + 15) & ~size_t(15);
   L.samp = o;     o = (o + 4 * (size_t)m + 15) & ~size_t(15);
   L.samp_tmp = o; o = (o + 4 * (size_t)m + 15) & ~size_t(15);
   L.band = o;     o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
@@ -64,8 +64,9 @@ struct Filtered {
 // scores below a_L and at/above a_R go into counts and anchored tail sums
 // (every term exp(-dist/alpha) <= 1, fp32 exp, fp64 sums); scores inside the
 // bracket are appended to the band with one shared atomic per warp.
+template <bool kGlobal>
 __device__ Filtered filter_row(const float* row, int n, float aL, float aR, float c2, uint32_t* band,
-                               int bcap, int* s_cnt, double* red) {
+                               int bcap, int* s_cnt, double* red, bool vec) {
   if (threadIdx.x == 0) *s_cnt = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -73,14 +74,24 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   int nl = 0, nr = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
-  // four scores per thread and step (the row is 16-byte aligned in shared
-  // memory); fp32 partial tail sums folded into fp64 once per step
-  const int n4 = n >> 2;
+  // four scores per thread and step (16-byte aligned rows); fp32 partial
+  // tail sums folded into fp64 once per step.  From global memory (L2) kB
+  // steps' loads are issued before any is used.
+  constexpr int kB = kGlobal ? 4 : 1;
+  const int n4 = vec ? (n >> 2) : 0;
   const float4* row4 = reinterpret_cast<const float4*>(row);
-  for (int base = 0; base < n4; base += NT) {
-    const int v = base + threadIdx.x;
+  for (int base0 = 0; base0 < n4; base0 += kB * NT) {
+  float4 qs[kB];
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int v = base0 + u * NT + threadIdx.x;
+    qs[u] = v < n4 ? (kGlobal ? __ldg(row4 + v) : row4[v]) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  }
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int v = base0 + u * NT + threadIdx.x;
     const bool act = v < n4;
-    const float4 q = act ? row4[v] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const float4 q = qs[u];
     const float xs[4] = {q.x, q.y, q.z, q.w};
     float pl = 0.0f, pr = 0.0f;
     uint32_t inb = 0u;
@@ -121,6 +132,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
         }
       }
     }
+  }
   }
   for (int base = n4 << 2; base < n; base += NT) {
     const int i = base + threadIdx.x;
@@ -249,16 +261,28 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
     const float4* s4 = reinterpret_cast<const float4*>(src);
     float4* d4 = reinterpret_cast<float4*>(dst);
     const int n4 = n >> 2;
-    for (int v = threadIdx.x; v < n4; v += NT) {
-      const float4 x = s4[v];
-      float4 p;
-      p.x = membership(x.x, bh, bl, c2);
-      p.y = membership(x.y, bh, bl, c2);
-      p.z = membership(x.z, bh, bl, c2);
-      p.w = membership(x.w, bh, bl, c2);
-      if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
-      ps += (double)((p.x + p.y) + (p.z + p.w));
-      stg_stream(d4 + v, p);
+    constexpr int kB = 4;  // loads in flight per thread (the row may be in global memory)
+    for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
+      float4 xs[kB];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int v = v0 + u * NT;
+        xs[u] = v < n4 ? s4[v] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      }
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int v = v0 + u * NT;
+        if (v >= n4) break;
+        const float4 x = xs[u];
+        float4 p;
+        p.x = membership(x.x, bh, bl, c2);
+        p.y = membership(x.y, bh, bl, c2);
+        p.z = membership(x.z, bh, bl, c2);
+        p.w = membership(x.w, bh, bl, c2);
+        if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
+        ps += (double)((p.x + p.y) + (p.z + p.w));
+        stg_stream(d4 + v, p);
+      }
     }
     for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
       const float p = nonfinite ? CUDART_NAN_F : membership(src[i], bh, bl, c2);
@@ -285,10 +309,15 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
   }
 }
 
+// Rows up to kRowSmemMaxN scores are copied into shared memory (one bulk copy)
+// and read there three times; longer ones are read from global memory (the
+// second and third reads hit L2), which leaves room for more rows per SM.
+constexpr int64_t kRowSmemMaxN = 8192;
+
+template <bool kSmemRow>
 __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   extern __shared__ __align__(16) unsigned char smem[];
-  const ResLayout L = res_layout(a.n, a.m, a.bcap);
-  float* row = reinterpret_cast<float*>(smem + L.row);
+  const ResLayout L = res_layout(a.n, a.m, a.bcap, kSmemRow);
   uint32_t* samp = reinterpret_cast<uint32_t*>(smem + L.samp);
   uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
   double* dscr = reinterpret_cast<double*>(smem + L.dscr);
@@ -301,6 +330,7 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   const int64_t r = blockIdx.x;
   const int n = (int)a.n;
   const float* src = a.scores + r * a.stride;
+  const float* row = kSmemRow ? reinterpret_cast<float*>(smem + L.row) : src;
   const RowArgs ra = row_args(a, r);
   const RowRanks rr = row_ranks(a, ra.k);
   const double inva = 1.0 / ra.alpha;
@@ -308,7 +338,9 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
 
   // ---- bring the row into shared memory --------------------------------
   uint32_t status = 0u;
-  if (a.vec) {
+  float* srow = reinterpret_cast<float*>(smem + L.row);
+  if (!kSmemRow) {
+  } else if (a.vec) {
     const uint32_t bytes = (uint32_t)(n >> 2) * 16u;
     if (threadIdx.x == 0) {
       mbar_init(mbar, 1);
@@ -316,16 +348,16 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
       if (bytes > 0) {
         mbar_arrive_expect_tx(mbar, bytes);
         for (uint32_t off = 0; off < bytes; off += 16384u)
-          bulk_load(reinterpret_cast<unsigned char*>(row) + off, reinterpret_cast<const unsigned char*>(src) + off,
+          bulk_load(reinterpret_cast<unsigned char*>(srow) + off, reinterpret_cast<const unsigned char*>(src) + off,
                     min(16384u, bytes - off), mbar);
       }
     }
-    for (int i = (n & ~3) + threadIdx.x; i < n; i += NT) row[i] = src[i];
+    for (int i = (n & ~3) + threadIdx.x; i < n; i += NT) srow[i] = src[i];
     __syncthreads();
     const int timed_out = (bytes > 0 && !mbar_wait_bounded(mbar, 0)) ? 1 : 0;
     if (__syncthreads_or(timed_out)) status |= ROW_TIMEOUT;
   } else {
-    for (int i = threadIdx.x; i < n; i += NT) row[i] = src[i];
+    for (int i = threadIdx.x; i < n; i += NT) srow[i] = src[i];
   }
   __syncthreads();
   if (status & ROW_TIMEOUT) {
@@ -359,7 +391,7 @@ __global__ void __launch_bounds__(NT) k_row_fwd(const ResidentFwd a) {
   Filtered f{};
   if (!a.force_fallback) {
     for (int attempt = 0;; ++attempt) {
-      f = filter_row(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
+      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red, kSmemRow ? true : a.vec != 0);
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
       block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
@@ -548,7 +580,9 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
 
 }  // namespace
 
-size_t resident_fwd_smem(const ResidentFwd& a) { return res_layout(a.n, a.m, a.bcap).total; }
+size_t resident_fwd_smem(const ResidentFwd& a) {
+  return res_layout(a.n, a.m, a.bcap, a.n <= kRowSmemMaxN).total;
+}
 size_t resident_fallback_smem(int64_t n) { return fb_layout(n).total; }
 
 // Lets both kernels use all the shared memory a block may opt in to (less
@@ -556,9 +590,14 @@ size_t resident_fallback_smem(int64_t n) { return fb_layout(n).total; }
 // its occupancy.
 cudaError_t resident_init(int optin_bytes) {
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, k_row_fwd);
+  cudaError_t e = cudaFuncGetAttributes(&fa, k_row_fwd<true>);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_row_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  e = cudaFuncSetAttribute(k_row_fwd<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin_bytes - (int)fa.sharedSizeBytes);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncGetAttributes(&fa, k_row_fwd<false>);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_row_fwd<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            optin_bytes - (int)fa.sharedSizeBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncGetAttributes(&fa, k_row_fallback);
@@ -574,7 +613,8 @@ cudaError_t launch_resident_fwd(const ResidentFwd& a, int sm_count, cudaStream_t
   if (e != cudaSuccess) return e;
   {
     Launch l("k_row_fwd", st);
-    k_row_fwd<<<(unsigned)a.rows, NT, smem, st>>>(a);
+    if (a.n <= kRowSmemMaxN) k_row_fwd<true><<<(unsigned)a.rows, NT, smem, st>>>(a);
+    else k_row_fwd<false><<<(unsigned)a.rows, NT, smem, st>>>(a);
   }
   const unsigned fgrid = (unsigned)std::min<int64_t>(a.rows, (int64_t)sm_count);
   {
