@@ -175,10 +175,15 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# the sources the streaming kernels and their launch plan are built from (the
+# one-block path's resident.cu does not touch the streaming kernels' traffic)
+STREAM_SOURCES = ("abi.cu", "block_sort.cuh", "common.cuh", "launch.h", "solve.cuh", "stream.cu", "tma.cuh")
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_soft_top_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in STREAM_SOURCES:
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode())
             h.update(fh.read())
