@@ -71,9 +71,10 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
-  int nl = 0, nr = 0;
+  int nl = 0;  // n_R is n - n_L - (band count): no per-score count for it
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
+  float amax = 0.0f;  // +-inf shows here; NaN falls in the band, checked there
   // four scores per thread and step (16-byte aligned rows); fp32 partial
   // tail sums folded into fp64 once per step.  From global memory (L2) kB
   // steps' loads are issued before any is used.
@@ -103,8 +104,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
       pl += isL ? e : 0.0f;
       pr += isR ? e : 0.0f;
       nl += (act && isL) ? 1 : 0;
-      nr += (act && isR) ? 1 : 0;
-      if (act && !(fabsf(x) < CUDART_INF_F)) bad = 1u;
+      amax = fmaxf(amax, fabsf(x));
       inb |= (act && !(isL || isR)) ? (1u << w) : 0u;
     }
     if (act) {
@@ -127,6 +127,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         if ((inb >> w) & 1u) {
+          if (!(fabsf(xs[w]) < CUDART_INF_F)) bad = 1u;  // NaN
           if (pos < bcap) band[pos] = f2key(xs[w]);
           ++pos;
         }
@@ -142,7 +143,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
     const float e = exp2f(fminf(x - aL, aR - x) * c2);
     if (act) {
       if (isL) { sl += (double)e; ++nl; }
-      if (isR) { sr += (double)e; ++nr; }
+      if (isR) sr += (double)e;
       if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;
     }
     const bool inb = act && !(isL || isR);
@@ -158,13 +159,14 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
       }
     }
   }
+  if (!(amax < CUDART_INF_F)) bad = 1u;
   Filtered f;
   f.nL = block_sum<NT, long long>((long long)nl, reinterpret_cast<long long*>(red));
-  f.nR = block_sum<NT, long long>((long long)nr, reinterpret_cast<long long*>(red));
   f.SL = block_sum<NT, double>(sl, red);
   f.SR = block_sum<NT, double>(sr, red);
   f.bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
   f.M = *s_cnt;
+  f.nR = (long long)n - f.nL - (long long)f.M;  // every score is left, right or in the band
   __syncthreads();
   return f;
 }
