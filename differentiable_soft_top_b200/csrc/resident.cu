@@ -10,6 +10,7 @@
 // abstract).  The backward pass (section 2.1's analytic VJP) is one block per
 // row: a reduction for lambda and an elementwise pass.
 #include <algorithm>
+#include <type_traits>
 
 #include "block_sort.cuh"
 #include "common.cuh"
@@ -88,52 +89,57 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
     const int v = base0 + u * NT + threadIdx.x;
     qs[u] = v < n4 ? (kGlobal ? __ldg(row4 + v) : row4[v]) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
+  // a step whose lanes all lie inside the row needs no per-score range check
+  auto step = [&](auto checked) {
 #pragma unroll
-  for (int u = 0; u < kB; ++u) {
-    const int v = base0 + u * NT + threadIdx.x;
-    const bool act = v < n4;
-    const float4 q = qs[u];
-    const float xs[4] = {q.x, q.y, q.z, q.w};
-    float pl = 0.0f, pr = 0.0f;
-    uint32_t inb = 0u;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float x = xs[w];
-      const bool isL = x < aL, isR = x >= aR;
-      const float e = exp2f(fminf(x - aL, aR - x) * c2);
-      pl += isL ? e : 0.0f;
-      pr += isR ? e : 0.0f;
-      nl += (act && isL) ? 1 : 0;
-      amax = fmaxf(amax, fabsf(x));
-      inb |= (act && !(isL || isR)) ? (1u << w) : 0u;
-    }
-    if (act) {
-      sl += (double)pl;
-      sr += (double)pr;
-    }
-    if (__any_sync(0xffffffffu, inb != 0u)) {  // rare: this warp holds band values
-      const int c = __popc(inb);
-      int incl = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      const int total = __shfl_sync(0xffffffffu, incl, 31);
-      int wbase = 0;
-      if (lane == 0) wbase = atomicAdd(s_cnt, total);
-      wbase = __shfl_sync(0xffffffffu, wbase, 0);
-      int pos = wbase + incl - c;
+    for (int u = 0; u < kB; ++u) {
+      const int v = base0 + u * NT + threadIdx.x;
+      const bool act = !decltype(checked)::value || v < n4;
+      const float4 q = qs[u];
+      const float xs[4] = {q.x, q.y, q.z, q.w};
+      float pl = 0.0f, pr = 0.0f;
+      uint32_t inb = 0u;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        if ((inb >> w) & 1u) {
-          if (!(fabsf(xs[w]) < CUDART_INF_F)) bad = 1u;  // NaN
-          if (pos < bcap) band[pos] = f2key(xs[w]);
-          ++pos;
+        const float x = xs[w];
+        const bool isL = x < aL, isR = x >= aR;
+        const float e = exp2f(fminf(x - aL, aR - x) * c2);
+        pl += isL ? e : 0.0f;
+        pr += isR ? e : 0.0f;
+        nl += (act && isL) ? 1 : 0;
+        amax = fmaxf(amax, fabsf(x));
+        inb |= (act && !(isL || isR)) ? (1u << w) : 0u;
+      }
+      if (act) {
+        sl += (double)pl;
+        sr += (double)pr;
+      }
+      if (__any_sync(0xffffffffu, inb != 0u)) {  // rare: this warp holds band values
+        const int c = __popc(inb);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        int wbase = 0;
+        if (lane == 0) wbase = atomicAdd(s_cnt, total);
+        wbase = __shfl_sync(0xffffffffu, wbase, 0);
+        int pos = wbase + incl - c;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          if ((inb >> w) & 1u) {
+            if (!(fabsf(xs[w]) < CUDART_INF_F)) bad = 1u;  // NaN
+            if (pos < bcap) band[pos] = f2key(xs[w]);
+            ++pos;
+          }
         }
       }
     }
-  }
+  };
+  if (base0 + kB * NT <= n4) step(std::false_type{});
+  else step(std::true_type{});
   }
   for (int base = n4 << 2; base < n; base += NT) {
     const int i = base + threadIdx.x;
