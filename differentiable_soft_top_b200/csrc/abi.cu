@@ -109,6 +109,15 @@ Ranks sample_ranks(int64_t n, double k, int m, double z) {
   return R;
 }
 
+// Arrays walked together as float4 must start at the same address mod 16:
+// every row of them then shares one head of 0-3 scores, which the kernels
+// take one at a time before the float4 body.  A null array (not written)
+// imposes nothing.
+int same_phase(const void* a, const void* b, const void* c = nullptr) {
+  const uintptr_t ph = (uintptr_t)a & 15u;
+  return (!b || ((uintptr_t)b & 15u) == ph) && (!c || ((uintptr_t)c & 15u) == ph);
+}
+
 int round_up(int64_t x, int64_t a) { return (int)(((x + a - 1) / a) * a); }
 
 bool resident_path(int64_t n, const Resolved& R) {
@@ -298,7 +307,7 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   DevInfo* dev = nullptr;
   if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  const int vec = same_phase(scores, p_out);
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
   if (res) {
@@ -409,7 +418,7 @@ int shard_fwd_plan(const float* scores, int64_t rows, int64_t n, int64_t row_str
   s.band_cap = lay.band_cap;
   StreamSizes sl = s;
   const StreamLayout L = stream_layout(rows, 0, sl);
-  const int vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  const int vec = same_phase(scores, p_out);
   *P = stream_plan(rows, n, row_stride, k, alpha, s, L, R, **dev, vec, static_cast<unsigned char*>(workspace));
   P->shard = 1;
   P->n_total = n_total;
@@ -444,7 +453,7 @@ int bwd_impl(const float* scores, const float* grad_p, const double* b, int64_t 
   DevInfo* dev = nullptr;
   if (!cuda_ok(device_info(&dev))) return LAPSUM_ECUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
+  const int vec = same_phase(scores, grad_p, grad_scores);
   if (n <= kResidentMaxN) {
     RowBwd a{scores, grad_p, b, rows, n, row_stride, alpha, grad_scores, grad_k, vec, grad_alpha, alpha_rows};
     return cuda_ok(launch_resident_bwd(a, dev->sm_count, st)) ? LAPSUM_OK : LAPSUM_ECUDA;
@@ -649,7 +658,7 @@ int lapsum_shard_bwd_partials(const float* scores, const float* grad_p, const do
   a.n = n;
   a.stride = row_stride;
   a.alpha = alpha;
-  a.vec = (((uintptr_t)scores | (uintptr_t)grad_p) & 15u) == 0 && (row_stride & 3) == 0;
+  a.vec = same_phase(scores, grad_p);
   a.parts_only = 1;
   a.part = x_parts;
   a.Gb = stream_grid(dev->sm_count, dev->occ.reduce_blocks, rows, n);
@@ -685,7 +694,7 @@ int lapsum_shard_bwd_finish(const float* scores, const float* grad_p, const doub
   a.grad = grad_scores;
   a.grad_k = grad_k;
   a.grad_alpha = grad_alpha;
-  a.vec = (((uintptr_t)scores | (uintptr_t)grad_p | (uintptr_t)grad_scores) & 15u) == 0 && (row_stride & 3) == 0;
+  a.vec = same_phase(scores, grad_p, grad_scores);
   a.lam = static_cast<double*>(workspace);
   a.Ga = stream_grid(dev->sm_count, dev->occ.apply_blocks, rows, n);
   return cuda_ok(launch_shard_bwd_finish(a, g_parts, world, reinterpret_cast<cudaStream_t>(stream))) ? LAPSUM_OK
@@ -785,7 +794,7 @@ extern "C" int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_
   a.bcap = rp.bcap;
   a.seed = R.seed;
   a.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
-  a.vec = (((uintptr_t)scores | (uintptr_t)p_out) & 15u) == 0 && (row_stride & 3) == 0;
+  a.vec = same_phase(scores, p_out);
   a.alpha_p = alpha;
   // same layout as the caller-workspace forward: statuses, counter, row list
   const size_t list_off = align256(4 * (size_t)rows);

@@ -167,6 +167,22 @@ __host__ __device__ __forceinline__ float key2f(uint32_t k) {
 }
 
 // ---------------------------------------------------------------------------
+// rows that do not start on a 16-byte boundary (odd n, offset views): the
+// first `head` (0-3) scores are taken one at a time and the body as float4
+// from row + head; arrays walked together (scores with p, g or grad) start at
+// the same address mod 16, so one head serves them all
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int row_head(const void* p, int64_t n) {
+  const int h = (int)(((0u - (uint32_t)(uintptr_t)p) & 15u) >> 2);
+  return n < h ? (int)n : h;
+}
+// index of the j-th score outside the body of n4 float4: [0, head), then
+// [head + 4 n4, n)
+__device__ __forceinline__ int64_t rest_index(int64_t j, int head, int64_t n4) {
+  return j < head ? j : j + 4 * n4;
+}
+
+// ---------------------------------------------------------------------------
 // per-row control block kept in the workspace (256 bytes per row)
 // ---------------------------------------------------------------------------
 struct alignas(256) RowCtl {

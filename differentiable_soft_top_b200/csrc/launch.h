@@ -65,7 +65,7 @@ struct ResidentFwd {
   int bcap;              // band capacity
   uint64_t seed;
   int force_fallback;
-  int vec;               // scores and p_out rows 16-byte aligned
+  int vec;               // scores and p_out start at the same address mod 16
   // workspace
   uint32_t* ws_status;   // [rows]
   uint32_t* fb_count;    // [1]
@@ -94,7 +94,7 @@ struct RowBwd {
   double alpha;
   float* grad;
   double* grad_k;
-  int vec;
+  int vec;             // scores, grad_p and grad start at the same address mod 16
   double* grad_alpha;  // dL/dalpha per row, or null
   const double* alpha_rows;  // per-row alpha (device [rows]) or null
 };
@@ -110,7 +110,7 @@ struct StreamPlan {
   int64_t band_cap;      // band slots per row
   uint64_t seed;
   int force_fallback;
-  int vec;
+  int vec;               // scores and p_out start at the same address mod 16
   int Gs, Gf, Gm, Gr;    // grids: sampling, filter, membership, recovery
   int band_cs;           // CTAs in the cluster that solves one row's band
   // workspace pieces
@@ -162,7 +162,7 @@ struct StreamBwd {
   double* grad_k;
   double* grad_alpha;  // dL/dalpha per row, or null
   const double* alpha_rows;  // per-row alpha (device [rows]) or null
-  int vec;
+  int vec;           // scores, grad_p and grad start at the same address mod 16
   int parts_only;    // sharded rows: the reduction only writes this shard's partials
   int Gb, Ga;        // grids of the reduction and elementwise passes
   void* part;        // [rows][kMaxGridPerRow] partials (48 bytes each)

@@ -31,7 +31,7 @@ struct ResLayout {
 __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool row_in_smem) {
   ResLayout L;
   size_t o = 0;
-  L.row = o;      o = (o + (row_in_smem ? 4 * (size_t)n : 0) + 15) & ~size_t(15);
+  L.row = o;      o = (o + (row_in_smem ? 4 * (size_t)n + 12 : 0) + 15) & ~size_t(15);
   L.samp = o;     o = (o + 4 * (size_t)m + 15) & ~size_t(15);
   L.samp_tmp = o; o = (o + 4 * (size_t)m + 15) & ~size_t(15);
   L.band = o;     o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
@@ -61,13 +61,14 @@ struct Filtered {
   uint32_t bad;
 };
 
-// One pass over the row in shared memory (section 2.2 stream-and-filter):
+// One pass over the row, in shared memory or (kGlobal) in global memory
+// (section 2.2 stream-and-filter):
 // scores below a_L and at/above a_R go into counts and anchored tail sums
 // (every term exp(-dist/alpha) <= 1, fp32 exp, fp64 sums); scores inside the
 // bracket are appended to the band with one shared atomic per warp.
 template <bool kGlobal>
 __device__ Filtered filter_row(const float* row, int n, float aL, float aR, float c2, uint32_t* band,
-                               int bcap, int* s_cnt, double* red, bool vec) {
+                               int bcap, int* s_cnt, double* red) {
   if (threadIdx.x == 0) *s_cnt = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -76,12 +77,13 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
   float amax = 0.0f;  // +-inf shows here; NaN falls in the band, checked there
-  // four scores per thread and step (16-byte aligned rows); fp32 partial
-  // tail sums folded into fp64 once per step.  From global memory (L2) kB
-  // steps' loads are issued before any is used.
+  // four scores per thread and step (the row's 16-byte aligned body); fp32
+  // partial tail sums folded into fp64 once per step.  From global memory
+  // (L2) kB steps' loads are issued before any is used.
   constexpr int kB = kGlobal ? 4 : 1;
-  const int n4 = vec ? (n >> 2) : 0;
-  const float4* row4 = reinterpret_cast<const float4*>(row);
+  const int head = row_head(row, n);
+  const int n4 = (n - head) >> 2;
+  const float4* row4 = reinterpret_cast<const float4*>(row + head);
   for (int base0 = 0; base0 < n4; base0 += kB * NT) {
   float4 qs[kB];
 #pragma unroll
@@ -141,10 +143,20 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   if (base0 + kB * NT <= n4) step(std::false_type{});
   else step(std::true_type{});
   }
-  for (int base = n4 << 2; base < n; base += NT) {
-    const int i = base + threadIdx.x;
-    const bool act = i < n;
-    const float x = act ? row[i] : 0.0f;
+  // the scores outside the body: one per thread and step, the loads of kB
+  // steps issued ahead from global memory
+  const int nrest = n - (n4 << 2);
+  for (int base0 = 0; base0 < nrest; base0 += kB * NT) {
+  float xq[kB];
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const int j = base0 + u * NT + threadIdx.x;
+    xq[u] = j < nrest ? row[rest_index(j, head, n4)] : 0.0f;
+  }
+#pragma unroll
+  for (int u = 0; u < kB; ++u) {
+    const bool act = base0 + u * NT + (int)threadIdx.x < nrest;
+    const float x = xq[u];
     const bool isL = x < aL, isR = x >= aR;
     const float e = exp2f(fminf(x - aL, aR - x) * c2);
     if (act) {
@@ -164,6 +176,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
         if (pos < bcap) band[pos] = f2key(x);
       }
     }
+  }
   }
   if (!(amax < CUDART_INF_F)) bad = 1u;
   Filtered f;
@@ -265,10 +278,13 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
     if (threadIdx.x == 0) a.sp.count[r] = total;
     __syncthreads();
   } else if (a.vec) {
+    // src and dst start at the same address mod 16 (a shared-memory copy is
+    // placed that way): one head, then float4 from both
     float* dst = a.p_out + r * a.stride;
-    const float4* s4 = reinterpret_cast<const float4*>(src);
-    float4* d4 = reinterpret_cast<float4*>(dst);
-    const int n4 = n >> 2;
+    const int head = row_head(src, n);
+    const float4* s4 = reinterpret_cast<const float4*>(src + head);
+    float4* d4 = reinterpret_cast<float4*>(dst + head);
+    const int n4 = (n - head) >> 2;
     constexpr int kB = 4;  // loads in flight per thread (the row may be in global memory)
     for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
       float4 xs[kB];
@@ -292,7 +308,8 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
         stg_stream(d4 + v, p);
       }
     }
-    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
+    for (int j = threadIdx.x; j < n - (n4 << 2); j += NT) {
+      const int i = (int)rest_index(j, head, n4);
       const float p = nonfinite ? CUDART_NAN_F : membership(src[i], bh, bl, c2);
       ps += (double)p;
       dst[i] = p;
@@ -338,7 +355,11 @@ __global__ void __launch_bounds__(NT, kSmemRow ? 1 : 4) k_row_fwd(const Resident
   const int64_t r = blockIdx.x;
   const int n = (int)a.n;
   const float* src = a.scores + r * a.stride;
-  const float* row = kSmemRow ? reinterpret_cast<float*>(smem + L.row) : src;
+  // the shared copy starts at src's address mod 16 when p is written with
+  // float4 (the region has 16 spare bytes), so that both walk one body
+  const int head = (kSmemRow && a.vec) ? row_head(src, n) : 0;
+  float* srow = reinterpret_cast<float*>(smem + L.row) + ((4 - head) & 3);
+  const float* row = kSmemRow ? srow : src;
   const RowArgs ra = row_args(a, r);
   const RowRanks rr = row_ranks(a, ra.k);
   const double inva = 1.0 / ra.alpha;
@@ -346,21 +367,24 @@ __global__ void __launch_bounds__(NT, kSmemRow ? 1 : 4) k_row_fwd(const Resident
 
   // ---- bring the row into shared memory --------------------------------
   uint32_t status = 0u;
-  float* srow = reinterpret_cast<float*>(smem + L.row);
   if (!kSmemRow) {
   } else if (a.vec) {
-    const uint32_t bytes = (uint32_t)(n >> 2) * 16u;
+    const int n4 = (n - head) >> 2;
+    const uint32_t bytes = (uint32_t)n4 * 16u;
     if (threadIdx.x == 0) {
       mbar_init(mbar, 1);
       fence_proxy_async_smem();
       if (bytes > 0) {
         mbar_arrive_expect_tx(mbar, bytes);
-        for (uint32_t off = 0; off < bytes; off += 16384u)
-          bulk_load(reinterpret_cast<unsigned char*>(srow) + off, reinterpret_cast<const unsigned char*>(src) + off,
-                    min(16384u, bytes - off), mbar);
+        unsigned char* d = reinterpret_cast<unsigned char*>(srow + head);
+        const unsigned char* s = reinterpret_cast<const unsigned char*>(src + head);
+        for (uint32_t off = 0; off < bytes; off += 16384u) bulk_load(d + off, s + off, min(16384u, bytes - off), mbar);
       }
     }
-    for (int i = (n & ~3) + threadIdx.x; i < n; i += NT) srow[i] = src[i];
+    for (int j = threadIdx.x; j < n - 4 * n4; j += NT) {
+      const int i = (int)rest_index(j, head, n4);
+      srow[i] = src[i];
+    }
     __syncthreads();
     const int timed_out = (bytes > 0 && !mbar_wait_bounded(mbar, 0)) ? 1 : 0;
     if (__syncthreads_or(timed_out)) status |= ROW_TIMEOUT;
@@ -399,7 +423,7 @@ __global__ void __launch_bounds__(NT, kSmemRow ? 1 : 4) k_row_fwd(const Resident
   Filtered f{};
   if (!a.force_fallback) {
     for (int attempt = 0;; ++attempt) {
-      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red, kSmemRow ? true : a.vec != 0);
+      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
       block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
@@ -520,16 +544,20 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
       if (kAlpha) shift_add_z(fabsf(z) * c2, gv, z, m, ps, psg, psz, psgz, S, SG, SZ, SGZ);
       else shift_add(fabsf(z) * c2, gv, m, ps, psg, S, SG);
     };
-    const int n4 = a.vec ? (n >> 2) : 0;
-    // kB float4 of r and of g in flight per thread, then the sums
+    // x, g and grad start at the same address mod 16: one head, then the
+    // body as float4, kB float4 of r and of g in flight per thread
+    const int head = a.vec ? row_head(x, n) : 0;
+    const int n4 = a.vec ? ((n - head) >> 2) : 0;
+    const float4* x4 = reinterpret_cast<const float4*>(x + head);
+    const float4* g4 = reinterpret_cast<const float4*>(g + head);
     constexpr int kB = 4;
     for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
       float4 xv[kB], gv[kB];
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
         const int v = v0 + u * NT;
-        xv[u] = v < n4 ? __ldg(reinterpret_cast<const float4*>(x) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-        gv[u] = v < n4 ? __ldg(reinterpret_cast<const float4*>(g) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        xv[u] = v < n4 ? __ldg(x4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[u] = v < n4 ? __ldg(g4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
@@ -545,7 +573,9 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
         SGZ += (double)psgz;
       }
     }
-    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT) {
+    const int nrest = n - (n4 << 2);
+    for (int j = threadIdx.x; j < nrest; j += NT) {
+      const int i = (int)rest_index(j, head, n4);
       float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
       acc(x[i], g[i], ps, psg, psz, psgz);
       S += (double)ps;
@@ -563,8 +593,8 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
         const int v = v0 + u * NT;
-        xv[u] = v < n4 ? __ldcs(reinterpret_cast<const float4*>(x) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
-        gv[u] = v < n4 ? __ldcs(reinterpret_cast<const float4*>(g) + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        xv[u] = v < n4 ? __ldcs(x4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[u] = v < n4 ? __ldcs(g4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
@@ -575,11 +605,13 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
         ov.y = exp2f(fmaf(-fabsf((xv[u].y - bh) - bl), c2, lg)) * ((gv[u].y - lh) - ll);
         ov.z = exp2f(fmaf(-fabsf((xv[u].z - bh) - bl), c2, lg)) * ((gv[u].z - lh) - ll);
         ov.w = exp2f(fmaf(-fabsf((xv[u].w - bh) - bl), c2, lg)) * ((gv[u].w - lh) - ll);
-        stg_stream(reinterpret_cast<float4*>(o) + v, ov);
+        stg_stream(reinterpret_cast<float4*>(o + head) + v, ov);
       }
     }
-    for (int i = (n4 << 2) + threadIdx.x; i < n; i += NT)
+    for (int j = threadIdx.x; j < nrest; j += NT) {
+      const int i = (int)rest_index(j, head, n4);
       o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
+    }
     if (threadIdx.x == 0 && a.grad_k) a.grad_k[r] = lam;
     if (kAlpha && threadIdx.x == 0) a.grad_alpha[r] = bad ? CUDART_NAN : alpha_grad((double)m, SZ, SGZ, lam, inva);
     __syncthreads();

@@ -398,10 +398,13 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   float amax = 0.0f;
 
   const int64_t n = P.n;
-  int64_t done = 0;
-  if (P.vec) {
-    const float4* x4 = reinterpret_cast<const float4*>(row);
-    const int64_t nchunks = (n >> 2) / CHUNK4;
+  // the 16-byte aligned body in chunks of CHUNK4 float4 (after a head of 0-3
+  // scores); the scores outside it go through the scalar loop below
+  const int head = row_head(row, n);
+  int64_t nb4 = 0;
+  {
+    const float4* x4 = reinterpret_cast<const float4*>(row + head);
+    const int64_t nchunks = ((n - head) >> 2) / CHUNK4;
     // two chunks in flight per thread: the next chunk's loads are issued
     // before the current one is processed
     float4 nx[U];
@@ -456,14 +459,15 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
         ncol = 0;
       }
     }
-    done = nchunks * CHUNK4 * 4;
+    nb4 = nchunks * CHUNK4;
   }
-  // the rest (or every score, for unaligned rows): one score per thread per
-  // step, the same trip count for the whole block
-  for (int64_t i0 = done + (int64_t)cta * NT; i0 < n; i0 += (int64_t)ncta * NT) {
-    const int64_t i = i0 + threadIdx.x;
-    if (i < n) {
-      const float x = row[i];
+  // the rest: one score per thread per step, the same trip count for the
+  // whole block
+  const int64_t nrest = n - 4 * nb4;
+  for (int64_t j0 = (int64_t)cta * NT; j0 < nrest; j0 += (int64_t)ncta * NT) {
+    const int64_t j = j0 + threadIdx.x;
+    if (j < nrest) {
+      const float x = row[rest_index(j, head, nb4)];
       const bool isL = x < aL, isR = x >= aR;
       const float e = exp2f(fminf(x - aL, aR - x) * c2);
       if (isL) {
@@ -516,10 +520,6 @@ __global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const floa
 // holds the root (section 2.2, steps 3-4)
 // ===========================================================================
 
-struct KeyVals {  // sorted keys in shared memory
-  const uint32_t* k;
-  __device__ float get(int i) const { return key2f(k[i]); }
-};
 struct KeyGroupsG {  // consecutive groups of `g` sorted keys in global memory
   const uint32_t* k;
   int g;
@@ -1341,13 +1341,8 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
 // memberships (section 2.1) and the backward pass
 // ===========================================================================
 
-// p = F((x - b)/alpha), with x - b formed from b = bh + bl (two fp32 words)
-__device__ __forceinline__ float memb(float x, float bh, float bl, float c2) {
-  const float d = (x - bh) - bl;
-  const float h = 0.5f * exp2f(-fabsf(d) * c2);
-  return d < 0.0f ? h : 1.0f - h;
-}
-// the same, also returning h = exp(-|x - b|/alpha)/2 and |x - b|
+// p = F((x - b)/alpha), with x - b formed from b = bh + bl (two fp32 words);
+// also returns h = exp(-|x - b|/alpha)/2 and |x - b|
 __device__ __forceinline__ float memb_h(float x, float bh, float bl, float c2, float& h, float& ad) {
   const float d = (x - bh) - bl;
   ad = fabsf(d);
@@ -1447,11 +1442,15 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
       flush(false);
     }
   };
-  if (P.vec) {
-    const float4* x4 = reinterpret_cast<const float4*>(row);
-    float4* d4 = reinterpret_cast<float4*>(dst);
-    const int64_t n4 = n >> 2;
-    const int64_t nchunks = n4 / CHUNK4;
+  // the body as float4 after a head of 0-3 scores (p starts at the scores'
+  // address mod 16 when vec; the sparse form writes no p)
+  const bool vec = kSparse || P.vec;
+  const int head = vec ? row_head(row, n) : 0;
+  const int64_t nb4 = vec ? ((n - head) >> 2) / CHUNK4 * CHUNK4 : 0;
+  {
+    const float4* x4 = reinterpret_cast<const float4*>(row + head);
+    float4* d4 = reinterpret_cast<float4*>(kSparse ? nullptr : dst + head);
+    const int64_t nchunks = nb4 / CHUNK4;
     for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
       const int64_t qq = nchunks - 1 - q;  // reverse of the filter pass
       const int64_t base = qq * CHUNK4 + threadIdx.x;
@@ -1478,7 +1477,7 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
           uint32_t hits = 0u;
 #pragma unroll
           for (int j = 0; j < 4; ++j) hits |= (pv[j] >= P.sp.eps) ? (1u << j) : 0u;
-          append(hits, (base + u * NT) * 4, pv, 4);
+          append(hits, head + (base + u * NT) * 4, pv, 4);
           flush(false);
         } else {
           stg_stream(d4 + base + u * NT, p);
@@ -1487,11 +1486,11 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
       ps += (double)pl;
       if (kDf) hs += (double)hl;
     }
-    for (int64_t i0 = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT; i0 < n; i0 += (int64_t)gridDim.x * NT)
-      one(i0 + threadIdx.x, i0 + threadIdx.x < n);
-  } else {
-    for (int64_t i0 = (int64_t)blockIdx.x * NT; i0 < n; i0 += (int64_t)gridDim.x * NT)
-      one(i0 + threadIdx.x, i0 + threadIdx.x < n);
+  }
+  const int64_t nrest = n - 4 * nb4;  // [0, head) and the tail; every score when !vec
+  for (int64_t j0 = (int64_t)blockIdx.x * NT; j0 < nrest; j0 += (int64_t)gridDim.x * NT) {
+    const int64_t j = j0 + threadIdx.x;
+    one(rest_index(j < nrest ? j : 0, head, nb4), j < nrest);
   }
   if (kSparse) flush(true);
   ps = block_sum<NT, double>(ps, red);
@@ -1503,9 +1502,9 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
       // nearest score (its values are read a second time)
       float mh = CUDART_INF_F, ml = 0.0f;
       double S = 0.0;
-      if (P.vec) {
-        const float4* x4 = reinterpret_cast<const float4*>(row);
-        const int64_t nchunks = (n >> 2) / CHUNK4;
+      {
+        const float4* x4 = reinterpret_cast<const float4*>(row + head);
+        const int64_t nchunks = nb4 / CHUNK4;
         for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
           const int64_t base = (nchunks - 1 - q) * CHUNK4 + threadIdx.x;
 #pragma unroll
@@ -1517,13 +1516,9 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
             near_add(v.w, bh, bl, c2, mh, ml, S);
           }
         }
-        for (int64_t i = nchunks * CHUNK4 * 4 + (int64_t)blockIdx.x * NT + threadIdx.x; i < n;
-             i += (int64_t)gridDim.x * NT)
-          near_add(row[i], bh, bl, c2, mh, ml, S);
-      } else {
-        for (int64_t i = (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
-          near_add(row[i], bh, bl, c2, mh, ml, S);
       }
+      for (int64_t j = (int64_t)blockIdx.x * NT + threadIdx.x; j < nrest; j += (int64_t)gridDim.x * NT)
+        near_add(row[rest_index(j, head, nb4)], bh, bl, c2, mh, ml, S);
       dmin = near_dist(mh, ml);
       block_near_reduce<NT>(dmin, S, inva, red);
       hs = S;
@@ -1651,11 +1646,14 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
     if (kAlpha) shift_add_z(fabsf(z) * c2, gv, z, m, ps, psg, psz, psgz, S, SG, SZ, SGZ);
     else shift_add(fabsf(z) * c2, gv, m, ps, psg, S, SG);
   };
-  int64_t done = 0;
-  if (a.vec) {
-    const float4* x4 = reinterpret_cast<const float4*>(x);
-    const float4* g4 = reinterpret_cast<const float4*>(g);
-    const int64_t nchunks = (n >> 2) / CHUNK4;
+  // x and g start at the same address mod 16 when vec: a head of 0-3
+  // scores, the body as float4, then the tail
+  const int head = a.vec ? row_head(x, n) : 0;
+  const int64_t nb4 = a.vec ? ((n - head) >> 2) / CHUNK4 * CHUNK4 : 0;
+  {
+    const float4* x4 = reinterpret_cast<const float4*>(x + head);
+    const float4* g4 = reinterpret_cast<const float4*>(g + head);
+    const int64_t nchunks = nb4 / CHUNK4;
     for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
       const int64_t base = q * CHUNK4 + threadIdx.x;
       float4 xv[U], gv[U];
@@ -1679,9 +1677,10 @@ __global__ void __launch_bounds__(NT) k_bwd_reduce(const StreamBwd a) {
         SGZ += (double)psgz;
       }
     }
-    done = nchunks * CHUNK4 * 4;
   }
-  for (int64_t i = done + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT) {
+  const int64_t nrest = n - 4 * nb4;
+  for (int64_t j = (int64_t)blockIdx.x * NT + threadIdx.x; j < nrest; j += (int64_t)gridDim.x * NT) {
+    const int64_t i = rest_index(j, head, nb4);
     float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
     acc(x[i], g[i], ps, psg, psz, psgz);
     S += (double)ps;
@@ -1732,12 +1731,14 @@ __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
   const float* g = a.grad_p + r * a.stride;
   float* o = a.grad + r * a.stride;
   const int64_t n = a.n;
-  int64_t done = 0;
-  if (a.vec) {
-    const float4* x4 = reinterpret_cast<const float4*>(x);
-    const float4* g4 = reinterpret_cast<const float4*>(g);
-    float4* o4 = reinterpret_cast<float4*>(o);
-    const int64_t nchunks = (n >> 2) / CHUNK4;
+  // x, g and grad start at the same address mod 16 when vec
+  const int head = a.vec ? row_head(x, n) : 0;
+  const int64_t nb4 = a.vec ? ((n - head) >> 2) / CHUNK4 * CHUNK4 : 0;
+  {
+    const float4* x4 = reinterpret_cast<const float4*>(x + head);
+    const float4* g4 = reinterpret_cast<const float4*>(g + head);
+    float4* o4 = reinterpret_cast<float4*>(o + head);
+    const int64_t nchunks = nb4 / CHUNK4;
     for (int64_t q = blockIdx.x; q < nchunks; q += gridDim.x) {
       const int64_t qq = nchunks - 1 - q;  // reverse of the reduction pass
       const int64_t base = qq * CHUNK4 + threadIdx.x;
@@ -1757,10 +1758,12 @@ __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
         stg_stream(o4 + base + u * NT, ov);
       }
     }
-    done = nchunks * CHUNK4 * 4;
   }
-  for (int64_t i = done + (int64_t)blockIdx.x * NT + threadIdx.x; i < n; i += (int64_t)gridDim.x * NT)
+  const int64_t nrest = n - 4 * nb4;
+  for (int64_t j = (int64_t)blockIdx.x * NT + threadIdx.x; j < nrest; j += (int64_t)gridDim.x * NT) {
+    const int64_t i = rest_index(j, head, nb4);
     o[i] = exp2f(fmaf(-fabsf((x[i] - bh) - bl), c2, lg)) * ((g[i] - lh) - ll);
+  }
 }
 
 

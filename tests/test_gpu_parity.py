@@ -124,8 +124,11 @@ def test_ragged_sizes(orc, n):
     check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], k, alpha, f"n={n}")
 
 
-@pytest.mark.parametrize("n,force", [(5000, lt.FORCE_NONE), (5000, lt.FORCE_STREAMING), (70001, lt.FORCE_NONE)])
+@pytest.mark.parametrize("n,force", [(5000, lt.FORCE_NONE), (5000, lt.FORCE_STREAMING), (12001, lt.FORCE_NONE),
+                                     (70001, lt.FORCE_NONE)])
 def test_strided_unaligned_rows(orc, n, force):
+    # scores start 4 bytes past the 16-byte grid, p and grad on it: the
+    # passes that write take every score one at a time
     rows, stride = 3, n + 3
     base = make_scores("mixture", rows, stride, seed=7)
     gb = make_grad(rows, stride, seed=8)
@@ -140,6 +143,22 @@ def test_strided_unaligned_rows(orc, n, force):
     for i in range(rows):
         check_row(orc, base[i, 1:n + 1], gb[i, 1:n + 1], p[i], grad.cpu().numpy()[i], b[i], gk.cpu().numpy()[i],
                   k, alpha, f"strided row {i}")
+
+
+@pytest.mark.parametrize("n,force", [(5001, lt.FORCE_NONE), (12001, lt.FORCE_NONE), (16383, lt.FORCE_NONE),
+                                     (5001, lt.FORCE_STREAMING), (70001, lt.FORCE_NONE)])
+def test_odd_n_rows_start_off_the_16_byte_grid(orc, n, force):
+    # contiguous rows of odd length start at every address mod 16 in turn
+    # (head of 0-3 scores before the float4 body); one-block rows in shared
+    # memory (n <= 8192) and in global memory, and streaming rows
+    rows = 5
+    x = make_scores("mixture", rows, n, seed=n + 11)
+    g = make_grad(rows, n, seed=n + 12)
+    k, alpha = n / 41.0, 0.05
+    out = gpu_run(x, g, k, alpha, params=lt.Params(force_path=force))
+    for i in range(rows):
+        check_row(orc, x[i], g[i], out["p"][i], out["grad"][i], out["b"][i], out["gk"][i], k, alpha,
+                  f"n={n} row {i}")
 
 
 def test_many_rows_streaming(orc):
@@ -354,6 +373,9 @@ def alpha_tol(r, g, b, alpha):
     ("c2", None, None, 0),
     ("c3", 2_000_003, None, 0),
     ("c5", 16384, 4, 0),
+    ("c5", 5001, 4, 0),
+    ("c5", 12001, 4, 0),
+    ("c2", 100_003, 3, 0),
 ])
 def test_alpha_gradient_matches_oracle(orc, name, n, rows, force):
     w, x, g = case(name, n=n, rows=rows)
@@ -403,6 +425,7 @@ EPS = 2.0 ** -24
     ("c3", 2_000_003, None, 0),
     ("c5", 16384, 4, 0),
     ("c2", 100_003, 2, 0),
+    ("c5", 12001, 4, 0),
 ])
 def test_sparse_forward_matches_dense_and_oracle(orc, name, n, rows, force):
     w, x, _ = case(name, n=n, rows=rows)
@@ -493,6 +516,8 @@ def dftopk_check(orc, r, k, alpha, res, i, label):
     ("c3", 2_000_003, None, 0),
     ("c5", 16384, 4, 0),
     ("c2", 100_003, 2, 0),
+    ("c5", 5001, 4, 0),
+    ("c5", 12001, 4, 0),
 ])
 def test_dftopk_matches_oracle(orc, name, n, rows, force):
     w, x, _ = case(name, n=n, rows=rows)
