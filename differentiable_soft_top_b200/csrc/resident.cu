@@ -1,9 +1,10 @@
-// resident.cu -- rows that fit one block's shared memory (n <= 16384).
+// resident.cu -- rows of at most 16384 scores, one thread block per row.
 //
-// One thread block owns a row.  The row is brought into shared memory once by
-// a bulk (TMA) copy; every step of the Fast LapSum pipeline (technical summary
-// section 2.2: localization sample, stream-and-filter, exact solve on the
-// band, certification with one widening) then runs on the copy, and the
+// One thread block owns a row.  Short rows are brought into shared memory
+// once by a bulk (TMA) copy, longer ones are read from global memory (L2
+// after the first pass); every step of the Fast LapSum pipeline (technical
+// summary section 2.2: localization sample, stream-and-filter, exact solve on
+// the band, certification with one widening) then runs on the row, and the
 // memberships (section 2.1) are written straight from it.  HBM traffic is one
 // read of the row and one write of p.  Rows whose bracket cannot be certified
 // go to a full-sort fallback kernel (the worst-case branch of the arXiv
@@ -25,7 +26,7 @@ constexpr int NT = kResidentThreads;
 constexpr int kFbGroup = 1024;  // fallback: sorted values per group
 
 struct ResLayout {
-  size_t row, samp, samp_tmp, band, band_tmp, dscr, hist, red, mbar, total;
+  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, red, mbar, total;
 };
 
 __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool row_in_smem) {
@@ -37,17 +38,13 @@ __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool
   L.band = o;     o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
-  L.hist = o;     o = (o + 4 * (size_t)SortScratch<NT>::kWords + 15) & ~size_t(15);
+  L.dlink = o;    o = (o + 8 * (size_t)bcap + 8 + 15) & ~size_t(15);
   L.red = o;      o = o + 8 * 64;
   L.mbar = o;     o = o + 16;
   L.total = o;
   return L;
 }
 
-struct KeyRun {  // one group: the sorted band held as keys
-  const uint32_t* k;
-  __device__ float get(int, int i) const { return key2f(k[i]); }
-};
 struct KeyGroups {  // consecutive groups of `g` sorted keys
   const uint32_t* k;
   int g;
@@ -336,20 +333,23 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
 
 // Rows up to kRowSmemMaxN scores are copied into shared memory (one bulk copy)
 // and read there three times; longer ones are read from global memory (the
-// second and third reads hit L2), which leaves room for more rows per SM.
-constexpr int64_t kRowSmemMaxN = 8192;
+// second and third reads hit L2).  Both forms run four rows per SM (64
+// registers a thread); a larger shared copy would leave room for fewer
+// (measured, 2048 rows of 8192: 148 us from global memory, 160 us from a
+// shared copy at three rows per SM).
+constexpr int64_t kRowSmemMaxN = 4096;
 
 template <bool kSmemRow>
-__global__ void __launch_bounds__(NT, kSmemRow ? 1 : 4) k_row_fwd(const ResidentFwd a) {
+__global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const ResLayout L = res_layout(a.n, a.m, a.bcap, kSmemRow);
   uint32_t* samp = reinterpret_cast<uint32_t*>(smem + L.samp);
   uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
   double* dscr = reinterpret_cast<double*>(smem + L.dscr);
+  double* dlink = reinterpret_cast<double*>(smem + L.dlink);
   double* red = reinterpret_cast<double*>(smem + L.red);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
-  __shared__ GroupAgg s_agg;
   __shared__ SolveOut s_out;
 
   const int64_t r = blockIdx.x;
@@ -427,10 +427,8 @@ __global__ void __launch_bounds__(NT, kSmemRow ? 1 : 4) k_row_fwd(const Resident
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
       block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
-      const uint32_t* bs = band;
-      aggregate_sorted_keys<NT, false>(bs, f.M, red, &s_agg, inva);
       SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, ra.k, ra.alpha, inva};
-      solve_band<NT, false>(in, &s_agg, 1, KeyRun{bs}, dscr, red, &s_out);
+      solve_run<NT>(in, band, f.M, dscr, dlink, red, &s_out);
       if (s_out.status & ROW_CERTIFIED) { solved = true; break; }
       if (attempt >= a.max_widen) break;
       // widen once on the side that missed; the other edge moves to the old

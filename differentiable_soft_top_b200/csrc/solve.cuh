@@ -631,6 +631,98 @@ __device__ void solve_band(const SolveIn in, GroupAgg* agg, int T, const Elems& 
   solve_values<NT>(in, pk, ld<kG>(&agg[pk.tg].cnt), One{el, pk.tg}, dscr, red, out);
 }
 
+// One sorted run (the one-block path's band, keys[0, M) in shared memory):
+// the value level over the whole band at once, with the certification taken
+// from the same two scans.  Writing y_{-1} = a_L and y_M = a_R, the link
+// factors l_i = exp((y_{i-1} - y_i)/alpha), i = 0..M, are computed once
+// (dL[0, M]); A_i = A_{i-1} l_i + 1 starts from S_L at a_L, and the suffix
+// B_i = B_{i+1} l_{i+1} + 1 (values >= y_i, anchored at y_i) from S_R at a_R.
+// Then S(y_i) = A_i/2 + (M - 1 - i + n_R) - B_{i+1} l_{i+1}/2, and at the
+// bracket edges S(a_L) = S_L/2 + M + n_R - B_0 l_0/2, S(a_R) = A_{M-1} l_M/2 +
+// n_R - S_R/2 (with B_0 = S_R, A_{M-1} = S_L when M = 0).  dA: >= M doubles,
+// dL: >= M + 1 doubles.  Every thread must call it; *out in shared memory.
+template <int NT>
+__device__ void solve_run(const SolveIn in, const uint32_t* keys, int M, double* dA, double* dL, double* red,
+                          SolveOut* out) {
+  const double inva = in.inva;
+  const int tid = threadIdx.x;
+  __shared__ double s_edge[2];  // B_0, A_{M-1}
+  __shared__ double s_bp;
+  int* iscr = reinterpret_cast<int*>(red);
+  const bool finL = isfinite(in.aL), finR = isfinite(in.aR);
+  const double xL = finL ? (double)in.aL : -CUDART_INF;
+  const double xR = finR ? (double)in.aR : CUDART_INF;
+  const double A0 = finL ? in.SL : 0.0;  // prefix state at a_L
+  const double B0 = finR ? in.SR : 0.0;  // suffix state at a_R
+  auto y = [&](int i) -> double { return i < 0 ? xL : (i >= M ? xR : (double)key2f(keys[i])); };
+  for (int i = tid; i <= M; i += NT) dL[i] = link(y(i - 1), y(i), inva);
+  if (tid == 0) {
+    s_edge[0] = B0;
+    s_edge[1] = A0;
+  }
+  __syncthreads();
+  const int qe = (M + NT - 1) / NT;
+  const int i0 = min(M, tid * qe), i1 = min(M, i0 + qe);
+
+  // forward: chunk map, scan, A at every value
+  Aff m = aff_id();
+  for (int i = i0; i < i1; ++i) m = aff_then(m, Aff{dL[i], 1.0});
+  const Aff fe = block_excl_scan_aff<NT, true>(m, red);
+  {
+    double A = fma(A0, fe.F, fe.S);  // prefix state at y_{i0 - 1}
+    for (int i = i0; i < i1; ++i) {
+      A = fma(A, dL[i], 1.0);
+      dA[i] = A;
+    }
+    if (i1 == M && i1 > i0) s_edge[1] = A;
+  }
+  // backward: chunk map, scan, knot values
+  Aff mb = aff_id();
+  for (int i = i1 - 1; i >= i0; --i) mb = aff_then(mb, Aff{dL[i + 1], 1.0});
+  const Aff be = block_excl_scan_aff<NT, false>(mb, red);
+  const double Bin = fma(B0, be.F, be.S);  // B_{i1}, anchored at y_{i1}
+  int icand = -1;
+  {
+    double B = Bin;
+    for (int i = i1 - 1; i >= i0; --i) {
+      const double S = 0.5 * dA[i] + (double)((long long)(M - 1 - i) + in.nR) - 0.5 * B * dL[i + 1];
+      if (icand < 0 && S >= in.k) icand = i;
+      B = fma(B, dL[i + 1], 1.0);
+    }
+    if (i0 == 0 && i1 > 0) s_edge[0] = B;
+  }
+  const int i_star = block_max_int<NT>(icand, iscr);  // its barriers publish s_edge
+  const int jn = i_star + 1;
+  if (jn < M && jn >= i0 && jn < i1) {
+    double B = Bin;
+    for (int i = i1 - 1; i >= jn; --i) B = fma(B, dL[i + 1], 1.0);
+    s_bp = B;  // B_jn
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const double S_aL = finL ? 0.5 * in.SL + (double)((long long)M + in.nR) - 0.5 * s_edge[0] * dL[0] : CUDART_INF;
+    const double S_aR = finR ? 0.5 * s_edge[1] * dL[M] + (double)in.nR - 0.5 * in.SR : -CUDART_INF;
+    out->M = M;
+    out->S_aL = S_aL;
+    out->S_aR = S_aR;
+    if (S_aL >= in.k && S_aR < in.k) {
+      const double xj = i_star < 0 ? xL : y(i_star);
+      const double A = i_star < 0 ? A0 : dA[i_star];
+      const double xj1 = jn < M ? y(jn) : xR;
+      const double Bp = jn < M ? s_bp : B0;
+      const double cj = (double)((long long)(M - 1 - i_star) + in.nR);
+      out->b = closed_form_root(xj, xj1, A, Bp, cj, in.k, in.alpha);
+      out->sumf = sum_f_at(xj, xj1, A, Bp, out->b, inva);
+      out->status = ROW_CERTIFIED;
+    } else {
+      out->b = 0.0;
+      out->sumf = 0.0;
+      out->status = (!(S_aL >= in.k) ? ROW_MISS_LEFT : 0u) | (!(S_aR < in.k) ? ROW_MISS_RIGHT : 0u);
+    }
+  }
+  __syncthreads();
+}
+
 template <int NT>
 __device__ __forceinline__ uint32_t block_minmax_u32(uint32_t v, bool is_max, uint32_t* scratch) {
   constexpr int NW = NT / 32;
