@@ -113,6 +113,87 @@ __device__ uint32_t* block_radix_sort(uint32_t* keys, uint32_t* tmp, int n, uint
   return keys;
 }
 
+// The keys of ascending ranks r[0] and r[1] among keys[0, n) (0 <= r < n),
+// without sorting: an MSD radix selection, 8 bits a level, one histogram per
+// rank over the keys that share its prefix so far.  Lanes of a warp that add
+// to the same bin are merged first (__match_any_sync), so equal keys cost one
+// atomic per warp.  scr: >= kSelectWords words of shared memory.  All NT
+// threads must call it; the result is returned in every thread.
+constexpr int kSelectWords = 2 * 256 + 4;
+template <int NT>
+__device__ void block_select2(const uint32_t* keys, int n, const int (&r)[2], uint32_t (&out)[2], uint32_t* scr) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t* st = scr + 512;  // prefix of rank 0 and 1, then the ranks left inside them
+  if (threadIdx.x == 0) {
+    st[0] = st[1] = 0u;
+    st[2] = (uint32_t)r[0];
+    st[3] = (uint32_t)r[1];
+  }
+  for (int level = 0; level < 4; ++level) {
+    const int shift = 24 - 8 * level;
+    const uint32_t pmask = level == 0 ? 0u : (0xFFFFFFFFu << (32 - 8 * level));
+    for (int i = threadIdx.x; i < 512; i += NT) scr[i] = 0u;
+    __syncthreads();
+    const uint32_t p0 = st[0], p1 = st[1];
+    for (int base = 0; base < n; base += NT) {
+      const int i = base + (int)threadIdx.x;
+      const bool act = i < n;
+      const uint32_t k = act ? keys[i] : 0u;
+      const uint32_t d = (k >> shift) & 255u;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const bool in = act && (k & pmask) == (t == 0 ? p0 : p1);
+        const uint32_t im = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const uint32_t peers = __match_any_sync(im, d);
+          if (lane == __ffs(peers) - 1) atomicAdd(&scr[256 * t + d], (uint32_t)__popc(peers));
+        }
+      }
+    }
+    __syncthreads();
+    if (warp < 2) {  // warp t finds the digit of rank t: lane l scans bins 8l .. 8l+7
+      const uint32_t* h = scr + 256 * warp;
+      const uint32_t rem = st[2 + warp];
+      uint32_t c[8], s = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = h[8 * lane + j];
+        s += c[j];
+      }
+      uint32_t incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      const uint32_t excl = incl - s;
+      __syncwarp();
+      if (rem >= excl && rem < incl) {
+        uint32_t acc = excl;  // keys of this prefix in lower bins
+        int d = 0;
+        bool found = false;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (!found) {
+            if (rem < acc + c[j]) {
+              d = j;
+              found = true;
+            } else {
+              acc += c[j];
+            }
+          }
+        }
+        st[warp] |= (uint32_t)(8 * lane + d) << shift;
+        st[2 + warp] = rem - acc;
+      }
+    }
+    __syncthreads();
+  }
+  out[0] = st[0];
+  out[1] = st[1];
+  __syncthreads();  // st may be reused by the caller
+}
+
 // Sorts buf[0, n) ascending in place with a bitonic network over N = the next
 // power of two >= n; buf must hold N keys (entries n..N-1 are overwritten with
 // the largest key, which no finite value maps to).  Order-independent and

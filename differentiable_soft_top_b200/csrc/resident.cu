@@ -351,6 +351,7 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
   __shared__ SolveOut s_out;
+  __shared__ uint32_t s_sel[kSelectWords];
 
   const int64_t r = blockIdx.x;
   const int n = (int)a.n;
@@ -365,58 +366,79 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   const double inva = 1.0 / ra.alpha;
   const float c2 = (float)(inva * (double)kLog2e);
 
-  // ---- bring the row into shared memory --------------------------------
+  // ---- start bringing the row in: a bulk copy into shared memory, or (rows
+  // read from global memory) an L2 prefetch; either overlaps the sample
   uint32_t status = 0u;
-  if (!kSmemRow) {
-  } else if (a.vec) {
-    const int n4 = (n - head) >> 2;
-    const uint32_t bytes = (uint32_t)n4 * 16u;
-    if (threadIdx.x == 0) {
-      mbar_init(mbar, 1);
-      fence_proxy_async_smem();
-      if (bytes > 0) {
-        mbar_arrive_expect_tx(mbar, bytes);
-        unsigned char* d = reinterpret_cast<unsigned char*>(srow + head);
-        const unsigned char* s = reinterpret_cast<const unsigned char*>(src + head);
-        for (uint32_t off = 0; off < bytes; off += 16384u) bulk_load(d + off, s + off, min(16384u, bytes - off), mbar);
+  const int n4c = (n - head) >> 2;
+  const uint32_t cbytes = (kSmemRow && a.vec) ? (uint32_t)n4c * 16u : 0u;
+  if (threadIdx.x == 0) {
+    if constexpr (kSmemRow) {
+      if (a.vec) {
+        mbar_init(mbar, 1);
+        fence_proxy_async_smem();
+        if (cbytes > 0) {
+          mbar_arrive_expect_tx(mbar, cbytes);
+          unsigned char* d = reinterpret_cast<unsigned char*>(srow + head);
+          const unsigned char* s = reinterpret_cast<const unsigned char*>(src + head);
+          for (uint32_t off = 0; off < cbytes; off += 16384u)
+            bulk_load(d + off, s + off, min(16384u, cbytes - off), mbar);
+        }
       }
+    } else {
+      const int h = row_head(src, n);
+      const uint32_t pb = (uint32_t)((n - h) >> 2) * 16u;
+      const unsigned char* s = reinterpret_cast<const unsigned char*>(src + h);
+      for (uint32_t off = 0; off < pb; off += 16384u) bulk_prefetch_l2(s + off, min(16384u, pb - off));
     }
-    for (int j = threadIdx.x; j < n - 4 * n4; j += NT) {
-      const int i = (int)rest_index(j, head, n4);
-      srow[i] = src[i];
-    }
-    __syncthreads();
-    const int timed_out = (bytes > 0 && !mbar_wait_bounded(mbar, 0)) ? 1 : 0;
-    if (__syncthreads_or(timed_out)) status |= ROW_TIMEOUT;
-  } else {
-    for (int i = threadIdx.x; i < n; i += NT) srow[i] = src[i];
-  }
-  __syncthreads();
-  if (status & ROW_TIMEOUT) {
-    // the copy never completed: wait once more, bounded, then give up on the row
-    mbar_wait_bounded(mbar, 0);
-    if (threadIdx.x == 0) {
-      a.b_out[r] = CUDART_NAN;
-      if (a.status_out) a.status_out[r] = ROW_TIMEOUT;
-    }
-    return;
   }
 
-  // ---- localization (section 2.2, step 1) ---------------------------------
+  // ---- localization (section 2.2, step 1), from global memory -------------
+  // Only the two order statistics of the bracket are needed: they are
+  // selected, not sorted for; the sample is sorted only if a widening needs
+  // other ranks.
   const int m = a.m;
   const uint64_t s = row_stream(a.seed, (uint64_t)r);
   for (int j = threadIdx.x; j < m; j += NT) {
     const uint64_t I = sample_index(s, (uint64_t)j, (uint64_t)n);
-    const double Y = (double)row[I] + laplace_noise(s, (uint64_t)j, ra.alpha);
+    const double Y = (double)src[I] + laplace_noise(s, (uint64_t)j, ra.alpha);
     samp[j] = f2key(__double2float_rn(Y));
   }
   __syncthreads();
-  block_bitonic_sort<NT>(samp, m);  // samp and samp_tmp form one buffer of 2m keys
-  const uint32_t* ss = samp;
   int rlo = rr.rank_lo, rhi = rr.rank_hi;
   bool vlo = rr.valid_lo != 0, vhi = rr.valid_hi != 0;
-  float aL = vlo ? key2f(ss[rlo]) : -CUDART_INF_F;
-  float aR = vhi ? key2f(ss[rhi]) : CUDART_INF_F;
+  float aL, aR;
+  {
+    const int want[2] = {vlo ? rlo : 0, vhi ? rhi : m - 1};
+    uint32_t got[2];
+    block_select2<NT>(samp, m, want, got, s_sel);
+    aL = vlo ? key2f(got[0]) : -CUDART_INF_F;
+    aR = vhi ? key2f(got[1]) : CUDART_INF_F;
+  }
+  bool samp_sorted = false;
+
+  // ---- finish the shared copy ----------------------------------------------
+  if constexpr (kSmemRow) {
+    if (a.vec) {
+      for (int j = threadIdx.x; j < n - 4 * n4c; j += NT) {
+        const int i = (int)rest_index(j, head, n4c);
+        srow[i] = src[i];
+      }
+      const int timed_out = (cbytes > 0 && !mbar_wait_bounded(mbar, 0)) ? 1 : 0;
+      if (__syncthreads_or(timed_out)) status |= ROW_TIMEOUT;
+    } else {
+      for (int i = threadIdx.x; i < n; i += NT) srow[i] = src[i];
+    }
+    __syncthreads();
+    if (status & ROW_TIMEOUT) {
+      // the copy never completed: wait once more, bounded, then give up on the row
+      mbar_wait_bounded(mbar, 0);
+      if (threadIdx.x == 0) {
+        a.b_out[r] = CUDART_NAN;
+        if (a.status_out) a.status_out[r] = ROW_TIMEOUT;
+      }
+      return;
+    }
+  }
 
   // ---- filter, sort the band, solve, certify (steps 2-4) ------------------
   bool solved = false;
@@ -434,6 +456,11 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
       // widen once on the side that missed; the other edge moves to the old
       // edge, which is now known to lie on the correct side of b
       status |= ROW_WIDENED;
+      if (!samp_sorted) {
+        block_bitonic_sort<NT>(samp, m);  // samp and samp_tmp form one buffer of 2m keys
+        samp_sorted = true;
+      }
+      const uint32_t* ss = samp;
       if (s_out.status & ROW_MISS_LEFT) {
         rhi = rlo; vhi = true; aR = aL;
         rlo -= rr.widen_delta;

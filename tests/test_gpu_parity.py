@@ -279,6 +279,18 @@ def test_widened_rows_report_it(orc):
     assert seen & (lt.ROW_WIDENED | lt.ROW_FALLBACK)
 
 
+@pytest.mark.parametrize("n", [3000, 16384])
+def test_widened_one_block_rows(orc, n):
+    # a narrow bracket (z = 0.3) misses often: the one-block path then sorts
+    # its sample and widens; rows in shared and in global memory
+    w, x, g = case("c5", n=n, rows=24)
+    o = gpu_run(x, g, w.k, w.alpha, params=lt.Params(z=0.3, seed=5))
+    for i in range(w.rows):
+        check_row(orc, x[i], g[i], o["p"][i], o["grad"][i], o["b"][i], o["gk"][i], w.k, w.alpha,
+                  f"n={n} z=0.3 row {i}")
+    assert np.any(o["status"] & lt.ROW_WIDENED)
+
+
 # ---------------------------------------------------------------------------
 # the localization step against the oracle's own sample (same splitmix64)
 # ---------------------------------------------------------------------------
