@@ -21,6 +21,9 @@ NVCC_FLAGS = [
     "-O3", "-std=c++17",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-lineinfo", "--ftz=true",
+    # a host-only function called from device code is an error, not a warning
+    # (the warning leaves a kernel that does nothing)
+    "--diag-error", "20011,20013,20014",
     "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
     "-I", INCLUDE, "-I", CSRC,
 ]

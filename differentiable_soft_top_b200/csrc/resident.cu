@@ -35,7 +35,8 @@ __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool
   L.row = o;      o = (o + (row_in_smem ? 4 * (size_t)n + 12 : 0) + 15) & ~size_t(15);
   L.samp = o;     o = (o + 4 * (size_t)m + 15) & ~size_t(15);
   L.samp_tmp = o; o = (o + 4 * (size_t)m + 15) & ~size_t(15);
-  L.band = o;     o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
+  // the band region also holds the selection's scratch before the filter
+  L.band = o;     o = (o + 4 * (size_t)(bcap > kSelectWords ? bcap : kSelectWords) + 15) & ~size_t(15);
   L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
   L.dlink = o;    o = (o + 8 * (size_t)bcap + 8 + 15) & ~size_t(15);
@@ -351,7 +352,6 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
   __shared__ SolveOut s_out;
-  __shared__ uint32_t s_sel[kSelectWords];
 
   const int64_t r = blockIdx.x;
   const int n = (int)a.n;
@@ -410,7 +410,7 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   {
     const int want[2] = {vlo ? rlo : 0, vhi ? rhi : m - 1};
     uint32_t got[2];
-    block_select2<NT>(samp, m, want, got, s_sel);
+    block_select2<NT>(samp, m, want, got, band);  // band is not written before the filter
     aL = vlo ? key2f(got[0]) : -CUDART_INF_F;
     aR = vhi ? key2f(got[1]) : CUDART_INF_F;
   }
