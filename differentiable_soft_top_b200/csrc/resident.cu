@@ -59,6 +59,32 @@ struct Filtered {
   uint32_t bad;
 };
 
+// The filter's four block reductions (n_L, S_L, S_R, the non-finite flag)
+// with one pair of barriers; the same xor trees as block_sum and block_or.
+__device__ __forceinline__ void block_reduce_filtered(long long& nl, double& sl, double& sr, uint32_t& bad,
+                                                      double* red) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  long long* rl = reinterpret_cast<long long*>(red + 2 * NW);
+  uint32_t* rb = reinterpret_cast<uint32_t*>(red + 3 * NW);
+  nl = warp_sum(nl);
+  sl = warp_sum(sl);
+  sr = warp_sum(sr);
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  __syncthreads();
+  if (lane == 0) {
+    red[warp] = sl;
+    red[NW + warp] = sr;
+    rl[warp] = nl;
+    rb[warp] = bad;
+  }
+  __syncthreads();
+  sl = warp_sum(lane < NW ? red[lane] : 0.0);
+  sr = warp_sum(lane < NW ? red[NW + lane] : 0.0);
+  nl = warp_sum(lane < NW ? rl[lane] : 0ll);
+  bad = __reduce_or_sync(0xffffffffu, lane < NW ? rb[lane] : 0u);
+}
+
 // One pass over the row, in shared memory or (kGlobal) in global memory
 // (section 2.2 stream-and-filter):
 // scores below a_L and at/above a_R go into counts and anchored tail sums
@@ -178,10 +204,12 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   }
   if (!(amax < CUDART_INF_F)) bad = 1u;
   Filtered f;
-  f.nL = block_sum<NT, long long>((long long)nl, reinterpret_cast<long long*>(red));
-  f.SL = block_sum<NT, double>(sl, red);
-  f.SR = block_sum<NT, double>(sr, red);
-  f.bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  long long nll = nl;
+  block_reduce_filtered(nll, sl, sr, bad, red);
+  f.nL = nll;
+  f.SL = sl;
+  f.SR = sr;
+  f.bad = bad;
   f.M = *s_cnt;
   f.nR = (long long)n - f.nL - (long long)f.M;  // every score is left, right or in the band
   __syncthreads();
