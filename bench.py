@@ -28,6 +28,7 @@ import io
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -180,13 +181,21 @@ class ClockSampler:
 STREAM_SOURCES = ("abi.cu", "block_sort.cuh", "common.cuh", "launch.h", "solve.cuh", "stream.cu", "tma.cuh")
 
 
+def code_only(text: str) -> str:
+    """C/C++/CUDA source without comments, trailing blanks or empty lines: the
+    DRAM counters depend on the code, not on how it is commented."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip())
+
+
 def source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "differentiable_soft_top_b200", "csrc")
     for f in STREAM_SOURCES:
-        with open(os.path.join(csrc, f), "rb") as fh:
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
             h.update(f.encode())
-            h.update(fh.read())
+            h.update(code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

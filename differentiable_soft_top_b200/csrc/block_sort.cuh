@@ -1,10 +1,14 @@
-// block_sort.cuh -- stable LSD radix sort of uint32 keys in shared memory.
+// block_sort.cuh -- sorting and selection of uint32 keys in shared memory,
+// by one thread block.
 //
-// Used for the band (section 2.2 of the Fast LapSum technical summary: only
-// the band around the threshold is sorted), for the localization sample, and
-// for whole rows in the full-sort fallback.
+// Section 2.2 of the Fast LapSum technical summary sorts only the band around
+// the threshold, and the bracket needs two order statistics of the
+// localization sample.  Here: a stable LSD radix sort (whole rows in the
+// full-sort fallback), an MSD radix selection of two ranks (the one-block
+// path's sample), and a bitonic network (the band, the streaming band's root
+// bin, and the sample when a widening needs other ranks).
 //
-// 8-bit digits, four passes.  Each warp owns one contiguous segment of the
+// Radix sort: 8-bit digits, four passes.  Each warp owns one contiguous segment of the
 // keys and walks it 32 keys at a time; __match_any_sync groups the lanes that
 // share a digit, so ranks inside a warp follow key order and the pass is
 // stable.  Offsets are laid out digit-major, warp-minor.  A pass whose digit

@@ -35,3 +35,13 @@ def test_reference_arm_prints_one_contract_line():
 def test_reference_arm_other_ranks_do_nothing():
     r = _run(["--impl", "reference", "--steps", "1", "--warmup", "0", "--workload", "c1"], env={"RANK": "1"})
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_traffic_key_ignores_comments_only():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = "int a; // note\n/* block\n   comment */ int b;  \n\n  // only a comment\nint c;\n"
+    assert bench.code_only(src) == "int a;\n int b;\nint c;"
+    assert bench.code_only(src.replace("note", "another note")) == bench.code_only(src)
+    assert bench.code_only(src.replace("int c;", "int d;")) != bench.code_only(src)
