@@ -145,6 +145,10 @@ LAPSUM_API size_t lapsum_topk_workspace_size(int64_t rows, int64_t n, const laps
  *   params      in   host pointer or NULL
  *   stream      in   cudaStream_t
  * Returns LAPSUM_OK or an error code (nothing enqueued on error).
+ * Speed, not results: every pass reads and writes rows 16 bytes at a time
+ * after a head of 0-3 scores, which needs scores and p_out to start at the
+ * same address mod 16 (contiguous tensors of one shape always do); when they
+ * do not, p is written one score at a time.
  */
 LAPSUM_API int lapsum_topk_fwd(const float* scores, int64_t rows, int64_t n, int64_t row_stride,
                     double k, double alpha, float* p_out, double* b_out, double* sumf_out,
@@ -260,6 +264,8 @@ LAPSUM_API size_t lapsum_topk_sparse_workspace_size(int64_t rows, int64_t n, con
  * sum_i f_i is not an input: the reduction pass forms sum g f and sum f
  * together, relative to the score nearest b, so that neither underflows.
  * Returns LAPSUM_OK or an error code (nothing enqueued on error).
+ * As for the forward, scores, grad_p and grad_scores take the 16-byte path
+ * when they start at the same address mod 16.
  */
 LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const double* b, int64_t rows,
                                int64_t n, int64_t row_stride, double alpha, float* grad_scores,
