@@ -124,8 +124,8 @@ def test_ragged_sizes(orc, n):
     check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], k, alpha, f"n={n}")
 
 
-@pytest.mark.parametrize("n,force", [(5000, lt.FORCE_NONE), (5000, lt.FORCE_STREAMING), (12001, lt.FORCE_NONE),
-                                     (70001, lt.FORCE_NONE)])
+@pytest.mark.parametrize("n,force", [(3000, lt.FORCE_NONE), (5000, lt.FORCE_NONE), (5000, lt.FORCE_STREAMING),
+                                     (12001, lt.FORCE_NONE), (70001, lt.FORCE_NONE)])
 def test_strided_unaligned_rows(orc, n, force):
     # scores start 4 bytes past the 16-byte grid, p and grad on it: the
     # passes that write take every score one at a time
@@ -145,12 +145,13 @@ def test_strided_unaligned_rows(orc, n, force):
                   k, alpha, f"strided row {i}")
 
 
-@pytest.mark.parametrize("n,force", [(5001, lt.FORCE_NONE), (12001, lt.FORCE_NONE), (16383, lt.FORCE_NONE),
-                                     (5001, lt.FORCE_STREAMING), (70001, lt.FORCE_NONE)])
+@pytest.mark.parametrize("n,force", [(3001, lt.FORCE_NONE), (4095, lt.FORCE_NONE), (5001, lt.FORCE_NONE),
+                                     (12001, lt.FORCE_NONE), (16383, lt.FORCE_NONE), (5001, lt.FORCE_STREAMING),
+                                     (70001, lt.FORCE_NONE)])
 def test_odd_n_rows_start_off_the_16_byte_grid(orc, n, force):
     # contiguous rows of odd length start at every address mod 16 in turn
-    # (head of 0-3 scores before the float4 body); one-block rows in shared
-    # memory (n <= 8192) and in global memory, and streaming rows
+    # (head of 0-3 scores before the float4 body); one-block rows copied to
+    # shared memory (n <= 4096) and read from global memory, and streaming rows
     rows = 5
     x = make_scores("mixture", rows, n, seed=n + 11)
     g = make_grad(rows, n, seed=n + 12)
