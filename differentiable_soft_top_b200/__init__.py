@@ -228,10 +228,17 @@ def _as_rows(t, name):
 
 def _like_rows(x):
     """An uninitialised [rows, n] tensor with the row stride of x (the C ABI
-    uses one row stride for inputs and outputs)."""
+    uses one row stride for inputs and outputs) that starts at x's address
+    mod 16, so that the kernels move both 16 bytes at a time even when x is
+    an offset view."""
     torch = _torch()
     rows, n = x.shape
-    return torch.empty_strided((rows, n), (x.stride(0), 1), dtype=x.dtype, device=x.device)
+    s = x.stride(0)
+    if rows == 0 or n == 0:  # rejected by the library; nothing to place
+        return torch.empty_strided((rows, n), (s, 1), dtype=x.dtype, device=x.device)
+    buf = torch.empty((rows - 1) * s + n + 3, dtype=x.dtype, device=x.device)
+    off = ((x.data_ptr() - buf.data_ptr()) // x.element_size()) % 4
+    return buf.as_strided((rows, n), (s, 1), storage_offset=off)
 
 
 def _per_row(v, rows, dev):

@@ -224,6 +224,22 @@ def test_binding_rejects_a_misshaped_per_row_vector():
     assert lt._rows_pair(2.0, torch.tensor(1.0), 4, "cpu") is None
 
 
+@pytest.mark.parametrize("rows,n,stride,off", [(3, 5000, 5003, 1), (1, 7, 7, 0), (5, 12001, 12001, 0),
+                                             (2, 10, 13, 3), (4, 9, 11, 2), (0, 5, 5, 0)])
+def test_outputs_start_at_the_scores_address_mod_16(rows, n, stride, off):
+    """Outputs the binding allocates share the scores' row stride and their
+    address mod 16 (the kernels then move both 16 bytes at a time)."""
+    torch = pytest.importorskip("torch")
+    base = torch.zeros(rows * stride + 8)
+    x = base.as_strided((rows, n), (stride, 1), storage_offset=off)
+    p = lt._like_rows(x)
+    assert p.shape == x.shape and p.stride() == x.stride()
+    if rows:
+        assert (p.data_ptr() - x.data_ptr()) % 16 == 0
+        assert p.storage_offset() + (rows - 1) * stride + n <= p.untyped_storage().nbytes() // 4
+        p.fill_(1.0)
+
+
 def test_binding_rejects_cpu_tensors():
     torch = pytest.importorskip("torch")
     with pytest.raises(TypeError):

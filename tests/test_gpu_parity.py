@@ -127,8 +127,8 @@ def test_ragged_sizes(orc, n):
 @pytest.mark.parametrize("n,force", [(3000, lt.FORCE_NONE), (5000, lt.FORCE_NONE), (5000, lt.FORCE_STREAMING),
                                      (12001, lt.FORCE_NONE), (70001, lt.FORCE_NONE)])
 def test_strided_unaligned_rows(orc, n, force):
-    # scores start 4 bytes past the 16-byte grid, p and grad on it: the
-    # passes that write take every score one at a time
+    # scores start 4 bytes past the 16-byte grid, row stride n + 3; the
+    # binding places p and grad at the same address mod 16
     rows, stride = 3, n + 3
     base = make_scores("mixture", rows, stride, seed=7)
     gb = make_grad(rows, stride, seed=8)
@@ -143,6 +143,28 @@ def test_strided_unaligned_rows(orc, n, force):
     for i in range(rows):
         check_row(orc, base[i, 1:n + 1], gb[i, 1:n + 1], p[i], grad.cpu().numpy()[i], b[i], gk.cpu().numpy()[i],
                   k, alpha, f"strided row {i}")
+
+
+@pytest.mark.parametrize("n,force", [(3000, lt.FORCE_NONE), (12001, lt.FORCE_NONE), (70001, lt.FORCE_NONE)])
+def test_outputs_off_the_scores_phase(orc, n, force):
+    # p and grad given by the caller 4 bytes further along the 16-byte grid
+    # than the scores: the passes that write take every score one at a time
+    rows, stride = 3, n + 3
+    base = make_scores("mixture", rows, stride, seed=9)
+    gb = make_grad(rows, stride, seed=10)
+    xt = torch.from_numpy(base).cuda()[:, 1:n + 1]
+    gt = torch.from_numpy(gb).cuda()[:, 1:n + 1]
+    p_out = torch.empty(rows * stride + 4, device="cuda").as_strided((rows, n), (stride, 1), storage_offset=2)
+    g_out = torch.empty(rows * stride + 4, device="cuda").as_strided((rows, n), (stride, 1), storage_offset=2)
+    assert (p_out.data_ptr() - xt.data_ptr()) % 16 != 0
+    k, alpha = 97.5, 0.07
+    res = lt.forward(xt, k, alpha, params=lt.Params(force_path=force), p_out=p_out)
+    grad, gk = lt.backward(xt, gt, res.b, alpha, grad_out=g_out)
+    torch.cuda.synchronize()
+    p, b = p_out.cpu().numpy(), res.b.cpu().numpy()
+    for i in range(rows):
+        check_row(orc, base[i, 1:n + 1], gb[i, 1:n + 1], p[i], g_out.cpu().numpy()[i], b[i],
+                  gk.cpu().numpy()[i], k, alpha, f"outputs off phase, row {i}")
 
 
 @pytest.mark.parametrize("n,force", [(3001, lt.FORCE_NONE), (4095, lt.FORCE_NONE), (5001, lt.FORCE_NONE),
