@@ -44,6 +44,7 @@ ROW_TRUNCATED = 0x40
 ROW_BADARG = 0x80  # per-row k or alpha out of range: the row's outputs are NaN
 ROW_NONFINITE, ROW_TIMEOUT, ROW_OVERFLOW = 0x08, 0x10, 0x20
 FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
+DEFAULT_Z = 4.0  # bracket half-width in binomial sigmas that Params.z = 0 selects
 
 
 class LapsumError(RuntimeError):
@@ -83,7 +84,7 @@ class Params:
     """Tuning and test knobs (lapsum_params).  Zero / negative = automatic."""
     sample_m: int = 0
     force_path: int = FORCE_NONE
-    z: float = 5.0
+    z: float = 0.0          # 0 = the library's default (4 binomial sigmas)
     seed: int = 0
     band_capacity: int = 0
     max_widen: int = -1
@@ -209,7 +210,11 @@ def _workspace(device, nbytes: int):
     return buf
 
 
-def _as_rows(t, name):
+def _rows_view(t, name, *, copy_ok=False):
+    """t (CUDA fp32, 1-D or 2-D) as a [rows, n] view with unit column stride.
+    An input may be copied to get that stride (copy_ok); an output may not,
+    since the kernels would then fill a temporary instead of the caller's
+    tensor."""
     torch = _torch()
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise TypeError(f"{name} must be a CUDA tensor (this library has no CPU path)")
@@ -221,9 +226,41 @@ def _as_rows(t, name):
         t2 = t
     else:
         raise ValueError(f"{name} must be 1-D or 2-D")
-    if t2.stride(1) != 1:
+    if t2.stride(1) != 1 and t2.shape[1] > 1:
+        if not copy_ok:
+            raise ValueError(f"{name} must have unit stride along its rows")
         t2 = t2.contiguous()
     return t2
+
+
+def _as_rows(t, name):
+    return _rows_view(t, name, copy_ok=True)
+
+
+def _check_like(x, t, name):
+    """t is laid out as the C ABI reads or writes it beside the scores x: the
+    same [rows, n] shape, the same device and x's row stride (one row stride
+    serves every array of a call).  Works on any device's tensors."""
+    if tuple(t.shape) != tuple(x.shape):
+        raise ValueError(f"{name} must have the shape of scores {tuple(x.shape)}, got {tuple(t.shape)}")
+    if t.device != x.device:
+        raise ValueError(f"{name} must be on the device of scores ({x.device}), got {t.device}")
+    if x.shape[0] > 1 and t.stride(0) != x.stride(0):
+        raise ValueError(f"{name} must have the row stride of scores ({x.stride(0)}), got {t.stride(0)}")
+
+
+def _check_vec(t, name, rows, dtype, device, optional=False):
+    """A per-row array: `rows` contiguous values of `dtype` on `device`."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous() or t.numel() < rows:
+        raise ValueError(f"{name} must be contiguous with at least {rows} values")
 
 
 def _like_rows(x):
@@ -285,9 +322,11 @@ def forward(scores, k, alpha, *, params: Params | None = None, workspace=None,
     x = _as_rows(scores, "scores")
     rows, n = x.shape
     dev = x.device
-    p = _like_rows(x) if p_out is None else _as_rows(p_out, "p_out")
-    if p.stride(0) != x.stride(0):
-        raise ValueError("p_out must have the row stride of scores")
+    if p_out is None:
+        p = _like_rows(x)
+    else:
+        p = _rows_view(p_out, "p_out")
+        _check_like(x, p, "p_out")
     b = torch.empty(rows, dtype=torch.float64, device=dev)
     sumf = torch.empty(rows, dtype=torch.float64, device=dev)
     status = torch.empty(rows, dtype=torch.int32, device=dev)
@@ -422,12 +461,18 @@ def backward(scores, grad_p, b, alpha, *, workspace=None, grad_out=None, want_al
     rows, n = x.shape
     if g.shape != x.shape:
         raise ValueError("grad_p must have the shape of scores")
+    if g.device != x.device:
+        raise ValueError("grad_p must be on the device of scores")
+    if b.numel() < rows:
+        raise ValueError(f"b must hold one threshold per row ({rows})")
     if g.stride(0) != x.stride(0):  # the C ABI takes one row stride for all arrays
         x, g = x.contiguous(), g.contiguous()
     dev = x.device
-    out = _like_rows(x) if grad_out is None else _as_rows(grad_out, "grad_out")
-    if out.stride(0) != x.stride(0):
-        raise ValueError("grad_out must have the row stride of scores")
+    if grad_out is None:
+        out = _like_rows(x)
+    else:
+        out = _rows_view(grad_out, "grad_out")
+        _check_like(x, out, "grad_out")
     gk = torch.empty(rows, dtype=torch.float64, device=dev)
     ga = torch.empty(rows, dtype=torch.float64, device=dev) if want_alpha else None
     bb = b.to(device=dev, dtype=torch.float64).contiguous()
@@ -449,19 +494,39 @@ def backward(scores, grad_p, b, alpha, *, workspace=None, grad_out=None, want_al
     return res + (ga,) if want_alpha else res
 
 
+def _into_args(scores, p, b, sumf, status, stats):
+    """Checks of the preallocated forward outputs against the scores; returns
+    the scores as a [rows, n] view."""
+    torch = _torch()
+    x = _rows_view(scores, "scores")
+    rows = x.shape[0]
+    pv = _rows_view(p, "p")
+    _check_like(x, pv, "p")
+    _check_vec(b, "b", rows, torch.float64, x.device)
+    _check_vec(sumf, "sumf", rows, torch.float64, x.device, optional=True)
+    _check_vec(status, "status", rows, torch.int32, x.device, optional=True)
+    if stats is not None:
+        _check_vec(stats, "stats", rows * STATS_DTYPE.itemsize, torch.uint8, x.device)
+    return x, pv
+
+
 def forward_into(scores, k: float, alpha: float, p, b, sumf, status, workspace, params: Params | None = None,
                  stats=None) -> None:
-    """forward() with every output preallocated (no allocation in the call)."""
+    """forward() with every output preallocated (no allocation in the call).
+    p has the shape, device and row stride of scores; b (float64), sumf
+    (float64) and status (int32) hold one value per row; stats, if given, is
+    a uint8 buffer of rows * STATS_DTYPE.itemsize bytes."""
     torch = _torch()
     lib = _load()
-    rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
-    stride = scores.stride(0) if scores.dim() == 2 else n
+    x, pv = _into_args(scores, p, b, sumf, status, stats)
+    rows, n = x.shape
+    _check_vec(workspace, "workspace", 1, torch.uint8, x.device)
     c, pptr = _params_ptr(params)
-    rc = lib.lapsum_topk_fwd(scores.data_ptr(), rows, n, stride, float(k), float(alpha), p.data_ptr(), b.data_ptr(),
+    rc = lib.lapsum_topk_fwd(x.data_ptr(), rows, n, x.stride(0), float(k), float(alpha), pv.data_ptr(), b.data_ptr(),
                              sumf.data_ptr() if sumf is not None else None,
                              status.data_ptr() if status is not None else None,
                              stats.data_ptr() if stats is not None else None, workspace.data_ptr(),
-                             workspace.numel(), pptr, torch.cuda.current_stream(scores.device).cuda_stream)
+                             workspace.numel(), pptr, torch.cuda.current_stream(x.device).cuda_stream)
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_fwd")
 
@@ -473,32 +538,43 @@ def forward_noalloc_into(scores, k: float, alpha: float, p, b, sumf=None, status
     implicit synchronisation allowed).  Rows of at most NOALLOC_MAX_N scores,
     at most NOALLOC_MAX_ROWS rows.  Its scratch is one static device array
     inside the library, shared by all calls on a device: calls that overlap on
-    the GPU race, so serialise them."""
+    the GPU race, so serialise them.  The outputs are checked as in
+    forward_into()."""
     torch = _torch()
     lib = _load()
-    rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
-    stride = scores.stride(0) if scores.dim() == 2 else n
+    x, pv = _into_args(scores, p, b, sumf, status, stats)
+    rows, n = x.shape
     c, pptr = _params_ptr(params)
-    rc = lib.lapsum_topk_fwd_noalloc(scores.data_ptr(), rows, n, stride, float(k), float(alpha), p.data_ptr(),
+    rc = lib.lapsum_topk_fwd_noalloc(x.data_ptr(), rows, n, x.stride(0), float(k), float(alpha), pv.data_ptr(),
                                      b.data_ptr(), sumf.data_ptr() if sumf is not None else None,
                                      status.data_ptr() if status is not None else None,
                                      stats.data_ptr() if stats is not None else None, pptr,
-                                     torch.cuda.current_stream(scores.device).cuda_stream)
+                                     torch.cuda.current_stream(x.device).cuda_stream)
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_fwd_noalloc")
 
 
 def backward_into(scores, grad_p, b, alpha: float, grad, workspace, grad_k=None, grad_alpha=None) -> None:
-    """backward() with every output preallocated (no allocation in the call)."""
+    """backward() with every output preallocated (no allocation in the call).
+    grad_p and grad have the shape, device and row stride of scores; b,
+    grad_k and grad_alpha are float64 with one value per row."""
     torch = _torch()
     lib = _load()
-    rows, n = scores.shape if scores.dim() == 2 else (1, scores.shape[0])
-    stride = scores.stride(0) if scores.dim() == 2 else n
-    rc = lib.lapsum_topk_bwd(scores.data_ptr(), grad_p.data_ptr(), b.data_ptr(), rows, n, stride, float(alpha),
-                             grad.data_ptr(), grad_k.data_ptr() if grad_k is not None else None,
+    x = _rows_view(scores, "scores")
+    rows, n = x.shape
+    gp = _rows_view(grad_p, "grad_p")
+    _check_like(x, gp, "grad_p")
+    gv = _rows_view(grad, "grad")
+    _check_like(x, gv, "grad")
+    _check_vec(b, "b", rows, torch.float64, x.device)
+    _check_vec(grad_k, "grad_k", rows, torch.float64, x.device, optional=True)
+    _check_vec(grad_alpha, "grad_alpha", rows, torch.float64, x.device, optional=True)
+    _check_vec(workspace, "workspace", 1, torch.uint8, x.device)
+    rc = lib.lapsum_topk_bwd(x.data_ptr(), gp.data_ptr(), b.data_ptr(), rows, n, x.stride(0), float(alpha),
+                             gv.data_ptr(), grad_k.data_ptr() if grad_k is not None else None,
                              grad_alpha.data_ptr() if grad_alpha is not None else None,
                              workspace.data_ptr(), workspace.numel(),
-                             torch.cuda.current_stream(scores.device).cuda_stream)
+                             torch.cuda.current_stream(x.device).cuda_stream)
     if rc != LAPSUM_OK:
         raise LapsumError(rc, "lapsum_topk_bwd")
 

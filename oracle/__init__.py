@@ -16,6 +16,9 @@ Parity status of each function (see the pin tests in tests/test_oracle_pins.py):
   sample / bracket / tails   pinned: published splitmix64 vectors, Laplace
                              noise distribution, exact-S identity of the tails,
                              bracket coverage
+  sample_ranks               pinned: exact binomial miss probability of the
+                             ranks against Phi(-z) (Berry-Esseen band), and
+                             the sampled bracket's miss rate per edge
 """
 from __future__ import annotations
 

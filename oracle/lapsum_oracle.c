@@ -358,9 +358,17 @@ void lo_sample(const float* r, int64_t n, double alpha, uint64_t seed, int64_t r
 void lo_sample_ranks(int64_t n, double k, int64_t m, double z, int64_t* c_lo, int64_t* c_hi) {
     double q = k / (double)n;
     double mq = (double)m * q;
+#if LO_MUTANT == 6
+    double sigma = sqrt(mq);  /* MUTANT: the (1 - q) factor of the variance dropped */
+#else
     double sigma = sqrt(mq * (1.0 - q));
+#endif
     *c_lo = (int64_t)floor(mq - z * sigma);
+#if LO_MUTANT == 7
+    *c_hi = (int64_t)ceil(mq);  /* MUTANT: the half-width applied on one side only */
+#else
     *c_hi = (int64_t)ceil(mq + z * sigma);
+#endif
 }
 
 /*

@@ -51,7 +51,7 @@ def test_params_struct_layout(lib):
     assert ctypes.sizeof(lt._CParams) == 40
     c = lt._CParams()
     lib.lapsum_default_params(ctypes.byref(c))
-    assert c.z == 4.0 and c.max_widen == -1 and c.sample_m == 0 and c.seed == 0
+    assert c.z == 4.0 == lt.DEFAULT_Z and c.max_widen == -1 and c.sample_m == 0 and c.seed == 0
     assert lt.STATS_DTYPE.itemsize == 88
 
 
@@ -238,6 +238,54 @@ def test_outputs_start_at_the_scores_address_mod_16(rows, n, stride, off):
         assert (p.data_ptr() - x.data_ptr()) % 16 == 0
         assert p.storage_offset() + (rows - 1) * stride + n <= p.untyped_storage().nbytes() // 4
         p.fill_(1.0)
+
+
+def test_caller_outputs_must_match_the_scores_layout():
+    """A caller-given output is written with the scores' row stride for every
+    row: a smaller, reshaped or differently strided buffer would be written
+    past its end, so the binding rejects it before any call."""
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(4, 1000)
+    lt._check_like(x, torch.zeros(4, 1000), "p")  # the natural case passes
+    with pytest.raises(ValueError, match="shape"):
+        lt._check_like(x, torch.zeros(1, 1000), "p")  # a 1-D p_out viewed as one row
+    with pytest.raises(ValueError, match="shape"):
+        lt._check_like(x, torch.zeros(4, 999), "p")
+    # strided scores (a column slice) beside a contiguous output of that shape
+    xs = torch.zeros(4, 1001)[:, 1:]
+    with pytest.raises(ValueError, match="row stride"):
+        lt._check_like(xs, torch.zeros(4, 1000), "p")
+    lt._check_like(xs, torch.zeros(4, 1001)[:, :1000], "p")
+    # one row: its stride is never used
+    lt._check_like(torch.zeros(1, 10), torch.zeros(1, 16)[:, :10], "p")
+    with pytest.raises(ValueError, match="device"):
+        lt._check_like(x, torch.zeros(4, 1000, device="meta"), "p")
+
+
+def test_per_row_outputs_must_hold_a_value_per_row():
+    torch = pytest.importorskip("torch")
+    lt._check_vec(torch.zeros(3, dtype=torch.float64), "b", 3, torch.float64, torch.device("cpu"))
+    with pytest.raises(TypeError):  # float32 b would be written as float64 past its end
+        lt._check_vec(torch.zeros(3), "b", 3, torch.float64, torch.device("cpu"))
+    with pytest.raises(ValueError):
+        lt._check_vec(torch.zeros(2, dtype=torch.float64), "b", 3, torch.float64, torch.device("cpu"))
+    with pytest.raises(ValueError):
+        lt._check_vec(torch.zeros(6, dtype=torch.float64)[::2], "b", 3, torch.float64, torch.device("cpu"))
+    lt._check_vec(None, "sumf", 3, torch.float64, torch.device("cpu"), optional=True)
+    with pytest.raises(ValueError):
+        lt._check_vec(None, "b", 3, torch.float64, torch.device("cpu"))
+
+
+def test_preallocated_entry_points_reject_cpu_tensors():
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(2, 8)
+    b = torch.zeros(2, dtype=torch.float64)
+    with pytest.raises(TypeError):
+        lt.forward_noalloc_into(x, 2.0, 1.0, torch.zeros(2, 8), b)
+    with pytest.raises(TypeError):
+        lt.forward_into(x, 2.0, 1.0, torch.zeros(2, 8), b, None, None, torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(TypeError):
+        lt.backward_into(x, x, b, 1.0, torch.zeros(2, 8), torch.zeros(16, dtype=torch.uint8))
 
 
 def test_binding_rejects_cpu_tensors():

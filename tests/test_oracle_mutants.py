@@ -7,6 +7,8 @@ Mutants (see the LO_MUTANT blocks in oracle/lapsum_oracle.c):
   3  the closed-form root ignores the sign of mu (one anchor for all cases)
   4  the backward pass drops the budget term lambda
   5  dL/dalpha ignores that the threshold moves with alpha
+  6  the bracket's rank half-width drops the (1 - q) factor of the binomial variance
+  7  the bracket's half-width is applied below the mean only
 """
 import os
 
@@ -38,10 +40,12 @@ def _battery(o):
         run(f"fda{seed}", lambda s=seed: pins.test_alpha_gradient_finite_differences(o, s))
     run("apair", lambda: pins.test_alpha_gradient_symmetric_pair(o))
     run("aconst", lambda: pins.test_alpha_gradient_constant_upstream_is_zero(o))
+    run("ranks", lambda: pins.check_rank_miss_probabilities(o))
+    run("misses", lambda: pins.check_bracket_miss_rates(o, cases=pins.MISS_CASES[2:]))
     return fails
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7])
 def test_pins_catch_mutant(tmp_path, mutant):
     path = oracle_mod.build(out=str(tmp_path / f"liblo_m{mutant}.so"), mutant=mutant, force=True)
     o = oracle_mod.Oracle(oracle_mod.load(path))

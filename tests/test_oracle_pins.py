@@ -380,12 +380,85 @@ def test_laplace_noise_distribution(orc):
     assert np.array_equal(Y, (r[idx].astype(np.float64) + eps).astype(np.float32))
 
 
-def test_sample_ranks_formula(orc):
-    for n, k, m, z in [(10**6, 1e4, 131072, 5.0), (4096, 64, 512, 5.0), (10**8, 1e6, 1 << 17, 3.0)]:
-        lo, hi = orc.sample_ranks(n, k, m, z)
+# ---------------------------------------------------------------------------
+# the bracket's ranks against the binomial law they must follow
+# ---------------------------------------------------------------------------
+# Technical summary section 2.2, step 1: with Laplace noise at the scale alpha,
+# P(Y_j > b) = (1/n) sum_i F((r_i - b)/alpha) = k/n exactly, so the number of
+# samples above b is X ~ Binomial(m, q = k/n).  The bracket edges are order
+# statistics at ranks placed z standard deviations either side of the mean,
+# so each edge misses b with probability close to Phi(-z):
+#   b >= a_R  <=>  X <= c_lo - 1,        b < a_L  <=>  X >= c_hi + 1.
+# Normal approximation with the Berry-Esseen bound for a binomial
+# (|P(X <= x) - Phi((x - mq)/s)| <= 0.4748 (q^2 + (1-q)^2) / s, s = sqrt(mq(1-q))),
+# and the rounding of the ranks to integers (at most one unit, 1/s in z):
+#   Phi(-z - 2/s) - BE  <=  P(miss on either side)  <=  Phi(-z) + BE.
+def _phi(x):
+    return 0.5 * math.erfc(-x / math.sqrt(2.0))
+
+
+def _miss_band(m, q, z):
+    s = math.sqrt(m * q * (1.0 - q))
+    be = 0.4748 * (q * q + (1.0 - q) ** 2) / s
+    return max(0.0, _phi(-z - 2.0 / s) - be), min(1.0, _phi(-z) + be)
+
+
+RANK_CASES = [  # (n, k, m): q = 1/64 (c1), 1/100 (c2), 1/2 and 9/10, where the (1 - q) factor matters
+    (4096, 64.0, 1 << 16), (10**6, 1e4, 1 << 17), (10**5, 5e4, 1 << 16), (10**5, 9e4, 1 << 16),
+]
+
+
+def check_rank_miss_probabilities(o):
+    from scipy.stats import binom
+    for n, k, m in RANK_CASES:
         q = k / n
-        s = math.sqrt(m * q * (1 - q))
-        assert lo == math.floor(m * q - z * s) and hi == math.ceil(m * q + z * s)
+        for z in (1.0, 2.0, 4.0):
+            lo, hi = o.sample_ranks(n, k, m, z)
+            p_right = float(binom.cdf(lo - 1, m, q))  # P(X <= c_lo - 1): b at or above a_R
+            p_left = float(binom.sf(hi, m, q))        # P(X >= c_hi + 1): b below a_L
+            band = _miss_band(m, q, z)
+            assert band[0] <= p_right <= band[1], (n, k, m, z, lo, p_right, band)
+            assert band[0] <= p_left <= band[1], (n, k, m, z, hi, p_left, band)
+
+
+def test_sample_ranks_reach_the_binomial_miss_probability(orc):
+    """Exact binomial tails at the oracle's ranks (scipy's binomial, not the
+    oracle's arithmetic) against the miss probability Phi(-z) the ranks are
+    meant to give; a variance without its (1 - q) factor, or a half-width on
+    one side only, lands far outside the band at q = 1/2 and 9/10."""
+    check_rank_miss_probabilities(orc)
+
+
+MISS_CASES = [  # (name, n, k, alpha, m): c1 as is, c2 scaled to 1e5, and a budget of half the row
+    ("c1", 4096, 64.0, 1.0, 8192), ("c2", 100_000, 1000.0, 0.1, 8192), ("half", 100_000, 50_000.0, 0.1, 8192),
+]
+
+
+def check_bracket_miss_rates(o, trials=1000, cases=MISS_CASES):
+    """Draw the bracket with `trials` seeds and count how often each edge
+    misses the oracle's threshold; each count must lie in the 99.9% binomial
+    range of `trials` draws at the miss probability band above."""
+    from scipy.stats import binom
+    for name, n, k, alpha, m in cases:
+        dist = "uniform" if name == "half" else ("normal" if name != "c3" else "mixture")
+        r = make_scores(dist, 1, n, seed=0)[0]
+        b = o.threshold(r, k, alpha)
+        for z in (1.0, 2.0):
+            miss_r = miss_l = 0
+            for seed in range(trials):
+                aL, aR, _, _ = o.bracket(r, k, alpha, m, z, seed)
+                miss_r += int(b >= aR)
+                miss_l += int(b < aL)
+            lo_p, hi_p = _miss_band(m, k / n, z)
+            lo_c, hi_c = binom.ppf(0.0005, trials, lo_p), binom.ppf(0.9995, trials, hi_p)
+            assert lo_c <= miss_r <= hi_c, (name, z, "right edge", miss_r, (lo_c, hi_c))
+            assert lo_c <= miss_l <= hi_c, (name, z, "left edge", miss_l, (lo_c, hi_c))
+
+
+def test_bracket_miss_rates_follow_the_binomial(orc):
+    """The sampled bracket (noise, indices, order statistics) misses b on
+    each side at the rate the binomial law of section 2.2 fixes."""
+    check_bracket_miss_rates(orc)
 
 
 @pytest.mark.parametrize("name,n", [("c1", None), ("c2", None), ("c3", 1_000_000), ("c4", 2_000_000)])
