@@ -31,7 +31,7 @@ __all__ = [
     "status_string", "launch_count", "trace_enable", "trace_collect", "library_path", "STATS_DTYPE", "ROW_CERTIFIED", "ROW_WIDENED",
     "ROW_FALLBACK", "ROW_NONFINITE", "ROW_TIMEOUT", "ROW_OVERFLOW", "ROW_TRUNCATED", "ROW_BADARG",
     "forward_sparse", "SparseResult", "sparse_workspace_size", "FORCE_NONE", "FORCE_FALLBACK",
-    "FORCE_STREAMING", "LapsumError", "dftopk_forward", "DFTopKResult",
+    "FORCE_STREAMING", "FORCE_TIMEOUT", "LapsumError", "dftopk_forward", "DFTopKResult",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -43,7 +43,7 @@ ROW_CERTIFIED, ROW_WIDENED, ROW_FALLBACK = 0x01, 0x02, 0x04
 ROW_TRUNCATED = 0x40
 ROW_BADARG = 0x80  # per-row k or alpha out of range: the row's outputs are NaN
 ROW_NONFINITE, ROW_TIMEOUT, ROW_OVERFLOW = 0x08, 0x10, 0x20
-FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING = 0, 1, 2
+FORCE_NONE, FORCE_FALLBACK, FORCE_STREAMING, FORCE_TIMEOUT = 0, 1, 2, 4
 DEFAULT_Z = 4.0  # bracket half-width in binomial sigmas that Params.z = 0 selects
 
 
@@ -64,7 +64,7 @@ class _CParams(ctypes.Structure):
         ("seed", ctypes.c_uint64),
         ("band_capacity", ctypes.c_int64),
         ("max_widen", ctypes.c_int32),
-        ("reserved", ctypes.c_int32),
+        ("spin_limit", ctypes.c_int32),
     ]
 
 
@@ -88,10 +88,12 @@ class Params:
     seed: int = 0
     band_capacity: int = 0
     max_widen: int = -1
+    spin_limit: int = 0     # polls before a bounded device wait gives up; 0 = about a second
 
     def _c(self) -> _CParams:
         return _CParams(int(self.sample_m), int(self.force_path), float(self.z),
-                        int(self.seed) & (2**64 - 1), int(self.band_capacity), int(self.max_widen), 0)
+                        int(self.seed) & (2**64 - 1), int(self.band_capacity), int(self.max_widen),
+                        int(self.spin_limit))
 
 
 _lib = None

@@ -71,6 +71,7 @@ struct Resolved {
   uint32_t force;
   uint32_t m_user;
   int64_t bcap_user;
+  uint32_t spin_limit;  // 0 = the kernels' default
 };
 
 Resolved resolve(const lapsum_params* p) {
@@ -84,6 +85,7 @@ Resolved resolve(const lapsum_params* p) {
   r.force = p ? p->force_path : 0u;
   r.m_user = p ? p->sample_m : 0u;
   r.bcap_user = p ? p->band_capacity : 0;
+  r.spin_limit = (p && p->spin_limit > 0) ? (uint32_t)p->spin_limit : 0u;
   return r;
 }
 
@@ -232,6 +234,8 @@ StreamPlan stream_plan(int64_t rows, int64_t n, int64_t row_stride, double k, do
   P.band_cap = s.band_cap;
   P.seed = R.seed;
   P.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+  P.force_timeout = (R.force & LAPSUM_FORCE_TIMEOUT) != 0;
+  P.spin_limit = R.spin_limit;
   P.vec = vec;
   const int sm = dev.sm_count;
   P.Gs = (int)std::min<int64_t>(1024, std::max<int64_t>(1, (s.m + 1023) / 1024));
@@ -334,6 +338,8 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
     a.bcap = rp.bcap;
     a.seed = R.seed;
     a.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+    a.force_timeout = (R.force & LAPSUM_FORCE_TIMEOUT) != 0;
+    a.spin_limit = R.spin_limit;
     a.vec = vec;
     a.ws_status = reinterpret_cast<uint32_t*>(ws);
     a.fb_count = reinterpret_cast<uint32_t*>(ws + align256(4 * (size_t)rows));
@@ -794,6 +800,8 @@ extern "C" int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_
   a.bcap = rp.bcap;
   a.seed = R.seed;
   a.force_fallback = (R.force & LAPSUM_FORCE_FALLBACK) != 0;
+  a.force_timeout = (R.force & LAPSUM_FORCE_TIMEOUT) != 0;
+  a.spin_limit = R.spin_limit;
   a.vec = same_phase(scores, p_out);
   a.alpha_p = alpha;
   // same layout as the caller-workspace forward: statuses, counter, row list

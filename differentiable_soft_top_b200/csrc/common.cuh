@@ -27,7 +27,10 @@ constexpr uint32_t ROW_PUBLIC = 0xFFu;
 constexpr uint32_t ROW_MISS_LEFT = 0x100u;   // S(a_L) < k: b lies below a_L
 constexpr uint32_t ROW_MISS_RIGHT = 0x200u;  // S(a_R) >= k: b lies at or above a_R
 constexpr uint32_t ROW_FORCE_FB = 0x400u;    // test knob: take the full sort
-constexpr uint32_t ROW_NEEDS_RECOVERY = ROW_MISS_LEFT | ROW_MISS_RIGHT | ROW_OVERFLOW | ROW_FORCE_FB;
+constexpr uint32_t ROW_FORCE_TO = 0x800u;    // test knob: the recovery barrier times out
+constexpr uint32_t ROW_NEEDS_RECOVERY = ROW_MISS_LEFT | ROW_MISS_RIGHT | ROW_OVERFLOW | ROW_FORCE_FB | ROW_FORCE_TO;
+// rows whose outputs are NaN
+constexpr uint32_t ROW_NAN_OUT = ROW_NONFINITE | ROW_BADARG | ROW_TIMEOUT;
 
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -599,12 +602,18 @@ __device__ __forceinline__ double alpha_grad(double m, double SZ, double SGZ, do
 // of polls, records ROW_TIMEOUT and returns, so a logic error can never hang
 // the GPU.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kSpinLimit = 1u << 22;  // x ~256 ns sleeps: about a second
+constexpr uint32_t kSpinLimitDefault = 1u << 22;  // x ~256 ns sleeps: about a second
 
-// Grid-wide barrier for a cooperatively launched grid (all blocks resident).
-// Returns false if the wait timed out; the caller must then stop.
+__host__ __device__ __forceinline__ uint32_t spin_limit_of(uint32_t requested) {
+  return requested ? requested : kSpinLimitDefault;
+}
+
+// Grid-wide barrier for a cooperatively launched grid (all blocks resident):
+// waits until `nblocks` blocks have arrived, polling at most `limit` times.
+// Returns false if the wait timed out (or another block's did); the caller
+// must then stop.
 __device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks,
-                                             uint32_t* timeout_flag) {
+                                             uint32_t* timeout_flag, uint32_t limit) {
   __shared__ uint32_t s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -620,7 +629,7 @@ __device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uin
     } else {
       uint32_t polls = 0;
       while (*vgen == my_gen) {
-        if (++polls > kSpinLimit || *((volatile uint32_t*)timeout_flag) != 0u) {
+        if (++polls > limit || *((volatile uint32_t*)timeout_flag) != 0u) {
           atomicOr(timeout_flag, 1u);
           s_ok = 0u;
           break;

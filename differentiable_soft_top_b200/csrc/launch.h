@@ -65,6 +65,8 @@ struct ResidentFwd {
   int bcap;              // band capacity
   uint64_t seed;
   int force_fallback;
+  int force_timeout;     // test knob: odd rows wait on a barrier no copy completes
+  uint32_t spin_limit;   // polls of a bounded wait; 0 = kSpinLimitDefault
   int vec;               // scores and p_out start at the same address mod 16
   // workspace
   uint32_t* ws_status;   // [rows]
@@ -110,6 +112,9 @@ struct StreamPlan {
   int64_t band_cap;      // band slots per row
   uint64_t seed;
   int force_fallback;
+  int force_timeout;     // test knob: odd rows go to the recovery kernel, whose
+                         // barrier then waits for one block more than it has
+  uint32_t spin_limit;   // polls of a bounded wait; 0 = kSpinLimitDefault
   int vec;               // scores and p_out start at the same address mod 16
   int Gs, Gf, Gm, Gr;    // grids: sampling, filter, membership, recovery
   int band_cs;           // CTAs in the cluster that solves one row's band

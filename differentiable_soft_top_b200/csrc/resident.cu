@@ -256,7 +256,7 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
   double ps = 0.0;
-  const bool nonfinite = (status & (ROW_NONFINITE | ROW_BADARG)) != 0u;
+  const bool nonfinite = (status & ROW_NAN_OUT) != 0u;
   if (a.dftopk) {
     // sum f at the membership scale alpha_p, relative to the score nearest b
     float mh = CUDART_INF_F, ml = 0.0f;
@@ -399,12 +399,15 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   uint32_t status = 0u;
   const int n4c = (n - head) >> 2;
   const uint32_t cbytes = (kSmemRow && a.vec) ? (uint32_t)n4c * 16u : 0u;
+  // test knob: odd rows issue no copy, so their bounded wait below runs out
+  const bool force_to = kSmemRow && a.vec && a.force_timeout && (r & 1);
+  const uint32_t limit = spin_limit_of(a.spin_limit);
   if (threadIdx.x == 0) {
     if constexpr (kSmemRow) {
       if (a.vec) {
         mbar_init(mbar, 1);
         fence_proxy_async_smem();
-        if (cbytes > 0) {
+        if (cbytes > 0 && !force_to) {
           mbar_arrive_expect_tx(mbar, cbytes);
           unsigned char* d = reinterpret_cast<unsigned char*>(srow + head);
           const unsigned char* s = reinterpret_cast<const unsigned char*>(src + head);
@@ -451,19 +454,20 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
         const int i = (int)rest_index(j, head, n4c);
         srow[i] = src[i];
       }
-      const int timed_out = (cbytes > 0 && !mbar_wait_bounded(mbar, 0)) ? 1 : 0;
+      const int timed_out = ((cbytes > 0 || force_to) && !mbar_wait_bounded(mbar, 0, limit)) ? 1 : 0;
       if (__syncthreads_or(timed_out)) status |= ROW_TIMEOUT;
     } else {
       for (int i = threadIdx.x; i < n; i += NT) srow[i] = src[i];
     }
     __syncthreads();
     if (status & ROW_TIMEOUT) {
-      // the copy never completed: wait once more, bounded, then give up on the row
-      mbar_wait_bounded(mbar, 0);
-      if (threadIdx.x == 0) {
-        a.b_out[r] = CUDART_NAN;
-        if (a.status_out) a.status_out[r] = ROW_TIMEOUT;
-      }
+      // the copy did not complete in time: wait once more, bounded, then give
+      // up on the row.  Its outputs are written as NaN from the global row
+      // (not the shared copy, which the bulk copy may still be filling).  If
+      // that copy is still in flight when the block exits, it may land in
+      // shared memory that a later block on this SM has been given.
+      mbar_wait_bounded(mbar, 0, limit);
+      finish_row(a, r, src, CUDART_NAN, CUDART_NAN, ROW_TIMEOUT, aL, aR, 0, 0, 0, 0.0, 0.0, 0, red);
       return;
     }
   }

@@ -54,9 +54,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* mbar, uint32_t phase) {
   return ok != 0u;
 }
 
-// Bounded wait on an mbarrier phase: false after kSpinLimit polls.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* mbar, uint32_t phase) {
-  for (uint32_t i = 0; i < kSpinLimit; ++i)
+// Bounded wait on an mbarrier phase: false after `limit` polls.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* mbar, uint32_t phase, uint32_t limit) {
+  for (uint32_t i = 0; i < limit; ++i)
     if (mbar_try_wait(mbar, phase)) return true;
   return false;
 }

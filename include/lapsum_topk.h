@@ -73,8 +73,8 @@ extern "C" {
 #define LAPSUM_ROW_FALLBACK 0x04u   /* solved by the full-sort fallback */
 #define LAPSUM_ROW_NONFINITE 0x08u  /* NaN or +-inf in the row: outputs of
                                        this row are unspecified */
-#define LAPSUM_ROW_TIMEOUT 0x10u    /* a bounded device wait gave up: outputs
-                                       of this row are unspecified */
+#define LAPSUM_ROW_TIMEOUT 0x10u    /* a bounded device wait gave up: the
+                                       row's p, b and sum f are NaN */
 #define LAPSUM_ROW_OVERFLOW 0x20u   /* informational: the band outgrew its
                                        capacity (the row then took the fallback) */
 #define LAPSUM_ROW_TRUNCATED 0x40u  /* sparse forward: the row has more entries
@@ -92,13 +92,28 @@ typedef struct lapsum_params {
     int64_t band_capacity;  /* band slots per row; 0 = automatic */
     int32_t max_widen;      /* widenings before the full sort: 0 or 1;
                                negative = automatic (1) */
-    int32_t reserved;
+    int32_t spin_limit;     /* polls before a bounded device wait gives up
+                               and sets LAPSUM_ROW_TIMEOUT; 0 or negative =
+                               the default (2^22 polls, about a second) */
 } lapsum_params;
 
 #define LAPSUM_FORCE_NONE 0u
 #define LAPSUM_FORCE_FALLBACK 1u   /* solve every row by the full-sort fallback */
 #define LAPSUM_FORCE_STREAMING 2u  /* use the multi-block path even for rows
                                       that fit one block's shared memory */
+/* Test knob: on every odd-numbered row, make one bounded device wait run out
+ * (pair it with a small spin_limit).  A one-block row that is copied into
+ * shared memory (n <= 4096) waits on a bulk-copy barrier that no copy
+ * targets (when scores and p start at the same address mod 16, as the copy
+ * needs); a streaming row is sent to the recovery kernel, whose first grid
+ * barrier then waits for one block more than the grid holds.  Such a row
+ * ends with LAPSUM_ROW_TIMEOUT and NaN outputs (p, b, sum f); on the
+ * streaming path every later row that needs the recovery kernel in that call
+ * ends the same way, since the kernel stops at its first timed-out barrier.
+ * Even-numbered rows are solved as usual, and the next call starts afresh.
+ * Nothing waits forever and no fault is raised.  Rows of 4097..16384 scores
+ * on the one-block path have no such wait and are not affected. */
+#define LAPSUM_FORCE_TIMEOUT 4u
 
 /* Fill *p with the defaults (all automatic, seed 0). */
 LAPSUM_API void lapsum_default_params(lapsum_params* p);
