@@ -65,6 +65,8 @@ def parse():
     ap.add_argument("--no-dftopk", action="store_true", help="skip the DFTopK-relaxation comparison")
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay of the step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' step times")
+    ap.add_argument("--no-full-sort", action="store_true", help="skip the full-sort branch comparison")
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="scale the workload to n scores per row (k keeps its ratio)")
     return ap.parse_args()
@@ -234,25 +236,19 @@ def max_over_ranks(value: float, dist, device) -> float:
     return float(t.item())
 
 
-def cpu_baseline(x_row, g_row, w, budget_s: float = 20.0):
-    """The fp64 oracle, as it stands, on a bounded prefix of the same row."""
+def cpu_baseline(x_row, g_row, w):
+    """The fp64 oracle, as it stands, on the whole row of the workload: one
+    run of forward + backward (at 1e8 scores about 40 s on one core)."""
     from oracle import oracle
     orc = oracle()
-    n_s = min(w.n, 10_000_000)
-    k_s = w.k * n_s / w.n
-    r = x_row[:n_s]
-    g = g_row[:n_s]
-    times = []
-    t_start = time.perf_counter()
-    while len(times) < 3 and (time.perf_counter() - t_start) < budget_s:
-        t0 = time.perf_counter()
-        _, b, _ = orc.forward(r, k_s, w.alpha)
-        orc.backward(r, g, b, w.alpha)
-        times.append(time.perf_counter() - t0)
-    t = statistics.median(times)
-    return {"value": n_s / t, "unit": "scores/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {n_s} scores of the same row, k scaled to {k_s:g}, fwd+bwd, "
-                      f"median of {len(times)} runs, single-threaded C"}
+    t0 = time.perf_counter()
+    _, b, _ = orc.forward(x_row, w.k, w.alpha)
+    orc.backward(x_row, g_row, b, w.alpha)
+    t = time.perf_counter() - t0
+    return {"value": w.n / t, "unit": "scores/s", "cores": 1, "host_cores": os.cpu_count(), "kind": "oracle",
+            "seconds": t,
+            "sample": f"the whole row ({w.n} scores, k={w.k:g}, alpha={w.alpha:g}), fwd+bwd, one run, "
+                      f"single-threaded C (sort, closed-form root, memberships, VJP)"}
 
 
 def run_reference(args):
@@ -262,7 +258,7 @@ def run_reference(args):
     from oracle import oracle
     orc = oracle()
     w = WORKLOADS[args.workload]
-    n_s = min(w.n, 2_000_000)
+    n_s = min(w.n, 10_000_000)
     k_s = w.k * n_s / w.n
     x = make_scores(w.dist, 1, n_s, seed=0)[0]
     g = make_grad(1, n_s, seed=1)[0]
@@ -286,7 +282,8 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(w), "rows": w.rows, "n": w.n, "k": w.k, "alpha": w.alpha},
-        "cpu_baseline": {"value": value, "unit": "scores/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "scores/s", "cores": 1, "host_cores": os.cpu_count(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "scores/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -468,6 +465,107 @@ def sparse_vs_dense_forward(lt, torch, w, x, dev, dist, flush, steps, eps=2.0 **
             "bytes_written_dense": 4 * rows * n, "bytes_written_sparse": 8 * rows * entries}
 
 
+def abi_step(lt, torch, w, x, g, dev, params=None, backward=True):
+    """One fwd(+bwd) step as direct calls of the C ABI on preallocated
+    buffers (no per-call Python checks, so short steps are not host-bound).
+    Returns (step, buffers)."""
+    import ctypes
+    lib = lt._load()
+    rows, n = x.shape
+    buf = dict(p=torch.empty_like(x), grad=torch.empty_like(x),
+               b=torch.empty(rows, dtype=torch.float64, device=dev),
+               sumf=torch.empty(rows, dtype=torch.float64, device=dev),
+               status=torch.empty(rows, dtype=torch.int32, device=dev),
+               gk=torch.empty(rows, dtype=torch.float64, device=dev),
+               ws=torch.empty(max(256, lt.workspace_size(rows, n, params)), dtype=torch.uint8, device=dev))
+    cp = params._c() if params is not None else None
+    pptr = ctypes.byref(cp) if cp is not None else None
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    fa = (x.data_ptr(), rows, n, x.stride(0), float(w.k), float(w.alpha), buf["p"].data_ptr(), buf["b"].data_ptr(),
+          buf["sumf"].data_ptr(), buf["status"].data_ptr(), None, buf["ws"].data_ptr(), buf["ws"].numel(), pptr, stream)
+    ba = (x.data_ptr(), g.data_ptr() if g is not None else None, buf["b"].data_ptr(), rows, n, x.stride(0),
+          float(w.alpha), buf["grad"].data_ptr(), buf["gk"].data_ptr(), None, buf["ws"].data_ptr(), buf["ws"].numel(),
+          stream)
+
+    def step():
+        rc = lib.lapsum_topk_fwd(*fa)
+        if rc == 0 and backward:
+            rc = lib.lapsum_topk_bwd(*ba)
+        if rc != 0:
+            raise RuntimeError(lt.status_string(rc))
+
+    step.keep = (cp, buf)  # the params struct must outlive the calls
+    return step, buf
+
+
+# the pages' median times (Fast LapSum arXiv abstract), other hardware, pass not stated
+PAGES_MS = {1_000_000: 0.92, 10_000_000: 1.39, 100_000_000: 7.24}
+
+
+def other_workloads(lt, torch, names, dev, dist, flush, steps, peak):
+    """fwd+bwd of each parity workload, K steps each after the L2 flush, CUDA
+    events on the launching stream: step time, scores/s and the fraction of
+    the HBM roofline at the path's algorithmic bytes per score (and at the
+    20 B/score floor of touching every byte once)."""
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for name in names:
+        w = WORKLOADS[name]
+        x = torch.from_numpy(make_scores(w)).to(dev)
+        g = torch.from_numpy(make_grad(w.rows, w.n)).to(dev)
+        step, buf = abi_step(lt, torch, w, x, g, dev)
+        step()
+        torch.cuda.synchronize(dev)
+        st = buf["status"].cpu()
+        certified = bool(((st & 1) != 0).all())
+        ms = timed_calls(torch, step, steps, flush, stream, dist, dev)
+        path = "resident" if w.n <= 16384 else "streaming"
+        scores = w.rows * w.n
+        gbs = STEP_BYTES_PER_SCORE[path] * scores / (ms * 1e-3) / 1e9
+        out[name] = {"workload": workload_desc(w), "path": path, "ms_per_step": ms,
+                     "scores_per_s": scores / (ms * 1e-3), "bytes_per_score": STEP_BYTES_PER_SCORE[path],
+                     "achieved_gbs": gbs, "frac_of_measured": gbs / peak, "frac_of_8tbs": gbs / 8000.0,
+                     "floor20_frac_of_measured": 20 * scores / (ms * 1e-3) / 1e9 / peak,
+                     "all_rows_certified": certified,
+                     "pages_ms": PAGES_MS.get(w.n) if w.rows == 1 else None}
+        del x, g, buf, step
+        torch.cuda.empty_cache()
+    return out
+
+
+# algorithmic bytes per score of the forward through the full-sort branch:
+# four 8-bit LSD passes, each reading and writing every key (32), the group
+# aggregation reading the sorted keys (4), the memberships reading r and
+# writing p (8)
+FULL_SORT_BYTES_PER_SCORE = 44
+
+
+def full_sort_branch(lt, torch, w, x, dev, dist, flush, steps, peak):
+    """The forward through the full-sort branch (every row sorted, technical
+    summary section 2.2) against the bracketed forward on the same row: the
+    pages quote the bracket up to 19x faster at 1e8 scores."""
+    stream = torch.cuda.current_stream(dev)
+    fb, fbuf = abi_step(lt, torch, w, x, None, dev, params=lt.Params(force_path=lt.FORCE_FALLBACK), backward=False)
+    br, bbuf = abi_step(lt, torch, w, x, None, dev, backward=False)
+    fb()
+    br()
+    torch.cuda.synchronize(dev)
+    ok = bool(((fbuf["status"].cpu() & lt.ROW_FALLBACK) != 0).all())
+    dp = float((fbuf["p"] - bbuf["p"]).abs().max())
+    db = float((fbuf["b"] - bbuf["b"]).abs().max())
+    ms_fb = timed_calls(torch, fb, steps, flush, stream, dist, dev)
+    ms_br = timed_calls(torch, br, steps, flush, stream, dist, dev)
+    scores = w.rows * w.n
+    gbs = FULL_SORT_BYTES_PER_SCORE * scores / (ms_fb * 1e-3) / 1e9
+    res = {"full_sort_forward_ms": ms_fb, "bracketed_forward_ms": ms_br, "ratio": ms_fb / ms_br,
+           "pages_ratio_up_to": 19.0, "all_rows_fallback": ok, "max_abs_dp_vs_bracketed": dp,
+           "max_abs_db_vs_bracketed": db, "bytes_per_score": FULL_SORT_BYTES_PER_SCORE, "achieved_gbs": gbs,
+           "frac_of_measured": gbs / peak}
+    del fb, br, fbuf, bbuf
+    torch.cuda.empty_cache()
+    return res
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -583,6 +681,14 @@ def main():
     if not args.no_dftopk:
         dftopk = dftopk_vs_lapsum(lt, torch, w, x, dev, dist, flush, args.steps)
 
+    full_sort = None
+    if not args.no_full_sort and n > 16384:
+        full_sort = full_sort_branch(lt, torch, w, x, dev, dist, flush, min(args.steps, 10), peak)
+    configs = None
+    if not args.no_configs and not args.n:
+        configs = other_workloads(lt, torch, [c for c in ("c1", "c2", "c3", "c5") if c != args.workload], dev,
+                                  dist, flush, args.steps, peak)
+
     e2e = None
     if not args.no_e2e:
         e2e = e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step)
@@ -627,6 +733,8 @@ def main():
         "graph_replay": graph,
         "sparse_forward": sparse,
         "dftopk_forward": dftopk,
+        "full_sort": full_sort,
+        "configs": configs,
         "gpu_launches": launches,
         "clocks": clk,
     }

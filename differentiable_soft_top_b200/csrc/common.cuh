@@ -598,6 +598,54 @@ __device__ __forceinline__ double alpha_grad(double m, double SZ, double SGZ, do
 }
 
 // ---------------------------------------------------------------------------
+// Classification of a score against the bracket [aL, aR) on the FMA pipe.
+// The streaming filter is bound by instruction issue, and compares, selects
+// and min/max run on the half-rate ALU pipe; here the left/right indicators
+// come from saturating multiplies instead (a saturated product of NaN is 0):
+//   L = sat(-(x - aL) 2^126)      1 if x < aL, else 0
+//   R = sat((x - aR) 2^126 + 1)   1 if x >= aR, else 0
+// Every normal difference is at least 2^-126 in magnitude, so the product
+// reaches 1; a difference below that is flushed to zero (--ftz), which places
+// a score within a subnormal step of an edge on the band's side of it.  A
+// score is in the band iff L + R == 0 (NaN lands there).  The tail term is
+//   e = exp2(-|min(x - aL, aR - x)| c2),
+// which is exp((x - aL)/alpha) on the left and exp((aR - x)/alpha) on the
+// right; the absolute value keeps the band's (unused) terms below 1, so that
+// 0 * e is never 0 * inf.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float mul_sat(float a, float b) {
+  float r;
+  asm("mul.rn.ftz.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float r;
+  asm("fma.rn.ftz.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+struct Side {
+  float L, R, e;
+};
+__device__ __forceinline__ Side classify(float x, float aL, float aR, float c2) {
+  const float dl = x - aL;
+  const float dr = x - aR;
+  Side s;
+  s.L = mul_sat(dl, -0x1p126f);
+  s.R = fma_sat(dr, 0x1p126f, 1.0f);
+  s.e = exp2f(-fabsf(fminf(dl, -dr)) * c2);
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  The short kernels of the forward pipeline
+// are launched with programmatic stream serialization, so that each can be
+// scheduled while the kernel ahead of it drains; it waits here, before it
+// reads anything that kernel wrote.  Launched without that attribute, this
+// returns at once.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // bounded waits.  Every spin in this library gives up after a fixed number
 // of polls, records ROW_TIMEOUT and returns, so a logic error can never hang
 // the GPU.

@@ -100,7 +100,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   int nl = 0;  // n_R is n - n_L - (band count): no per-score count for it
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
-  float amax = 0.0f;  // +-inf shows here; NaN falls in the band, checked there
+  float fsum = 0.0f;  // sum of the scores scaled by 2^-64: +-inf or NaN shows here
   // four scores per thread and step (the row's 16-byte aligned body); fp32
   // partial tail sums folded into fp64 once per step.  From global memory
   // (L2) kB steps' loads are issued before any is used.
@@ -123,24 +123,32 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
       const bool act = !decltype(checked)::value || v < n4;
       const float4 q = qs[u];
       const float xs[4] = {q.x, q.y, q.z, q.w};
-      float pl = 0.0f, pr = 0.0f;
-      uint32_t inb = 0u;
+      // classification and tail terms on the FMA pipe (classify)
+      float pl = 0.0f, pr = 0.0f, cl = 0.0f, cr = 0.0f;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const float x = xs[w];
-        const bool isL = x < aL, isR = x >= aR;
-        const float e = exp2f(fminf(x - aL, aR - x) * c2);
-        pl += isL ? e : 0.0f;
-        pr += isR ? e : 0.0f;
-        nl += (act && isL) ? 1 : 0;
-        amax = fmaxf(amax, fabsf(x));
-        inb |= (act && !(isL || isR)) ? (1u << w) : 0u;
+        const Side sd = classify(xs[w], aL, aR, c2);
+        pl = fmaf(sd.L, sd.e, pl);
+        pr = fmaf(sd.R, sd.e, pr);
+        cl += sd.L;
+        cr += sd.R;
+        fsum = fmaf(xs[w], 0x1p-64f, fsum);  // padding lanes hold 0
       }
       if (act) {
         sl += (double)pl;
         sr += (double)pr;
+        nl += (int)cl;
       }
-      if (__any_sync(0xffffffffu, inb != 0u)) {  // rare: this warp holds band values
+      const bool has_band = act && cl + cr < 4.0f;
+      if (__any_sync(0xffffffffu, has_band)) {  // rare: this warp holds band values
+        uint32_t inb = 0u;
+        if (has_band) {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const Side sd = classify(xs[w], aL, aR, c2);
+            inb |= (sd.L + sd.R == 0.0f) ? (1u << w) : 0u;
+          }
+        }
         const int c = __popc(inb);
         int incl = c;
 #pragma unroll
@@ -181,14 +189,13 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   for (int u = 0; u < kB; ++u) {
     const bool act = base0 + u * NT + (int)threadIdx.x < nrest;
     const float x = xq[u];
-    const bool isL = x < aL, isR = x >= aR;
-    const float e = exp2f(fminf(x - aL, aR - x) * c2);
+    const Side sd = classify(x, aL, aR, c2);
     if (act) {
-      if (isL) { sl += (double)e; ++nl; }
-      if (isR) sr += (double)e;
+      if (sd.L != 0.0f) { sl += (double)sd.e; ++nl; }
+      if (sd.R != 0.0f) sr += (double)sd.e;
       if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;
     }
-    const bool inb = act && !(isL || isR);
+    const bool inb = act && sd.L + sd.R == 0.0f;
     const uint32_t msk = __ballot_sync(0xffffffffu, inb);
     if (msk) {
       const int leader = __ffs(msk) - 1;
@@ -202,7 +209,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
     }
   }
   }
-  if (!(amax < CUDART_INF_F)) bad = 1u;
+  if (!(fabsf(fsum) < CUDART_INF_F)) bad = 1u;
   Filtered f;
   long long nll = nl;
   block_reduce_filtered(nll, sl, sr, bad, red);
@@ -237,10 +244,14 @@ __device__ void write_stats(lapsum_row_stats* st, float aL, float aR, long long 
 
 // p_i = F((r_i - b)/alpha) as an fp32 value; (r_i - b) is formed from b split
 // into two fp32 words (b = bh + bl), which keeps it accurate to fp64 level.
+// The side of b is taken as a saturated product on the FMA pipe (s = 1 at or
+// above b, 0 below), not a compare and select on the ALU pipe; 1 - h is then
+// formed as h + s (1 - 2h), within an ulp of 1 - h.
 __device__ __forceinline__ float membership(float x, float bh, float bl, float c2) {
   const float d = (x - bh) - bl;
   const float h = 0.5f * exp2f(-fabsf(d) * c2);
-  return d < 0.0f ? h : 1.0f - h;
+  const float s = fma_sat(d, 0x1p126f, 1.0f);
+  return fmaf(s, fmaf(-2.0f, h, 1.0f), h);
 }
 
 // Writes p for a row from `src` (shared or global) and finishes the row's

@@ -279,6 +279,7 @@ __global__ void __launch_bounds__(NT) k_pick1(const StreamPlan P) {
 __global__ void __launch_bounds__(NT) k_select2(const StreamPlan P) {
   __shared__ uint32_t sh[4096];
   __shared__ uint32_t scr[64];
+  wait_prior_grid();
   const int64_t r = blockIdx.y;
   RowCtl* c = ctl_of(P, r);
   const int b1[2] = {c->sel_bin[0][0], c->sel_bin[0][1]};
@@ -295,6 +296,7 @@ __global__ void __launch_bounds__(NT) k_select2(const StreamPlan P) {
 __global__ void __launch_bounds__(NT) k_select3(const StreamPlan P) {
   __shared__ uint32_t sh[2048];
   __shared__ uint32_t scr[64];
+  wait_prior_grid();
   const int64_t r = blockIdx.y;
   RowCtl* c = ctl_of(P, r);
   const uint32_t pre[2] = {level3_prefix(c, 0), level3_prefix(c, 1)};
@@ -379,6 +381,23 @@ __device__ __noinline__ void flush_warp(const FilterCtx& f, const float* col, in
 
 __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
                              int ncta, double* red, float* stage) {
+  const int64_t n = P.n;
+  // the 16-byte aligned body in chunks of CHUNK4 float4 (after a head of 0-3
+  // scores); the scores outside it go through the scalar loop below
+  const int head = row_head(row, n);
+  const float4* x4 = reinterpret_cast<const float4*>(row + head);
+  const int64_t nchunks = ((n - head) >> 2) / CHUNK4;
+  // two chunks in flight per thread: the next chunk's loads are issued
+  // before the current one is processed.  The scores are the caller's, so
+  // the first chunk is requested before waiting for the kernel that wrote
+  // the bracket.
+  float4 nx[U];
+  if (cta < nchunks) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) nx[u] = __ldg(x4 + (int64_t)cta * CHUNK4 + threadIdx.x + u * NT);
+  }
+  wait_prior_grid();
+
   FilterCtx f;
   f.aL = vld(&c->aL);
   f.aR = vld(&c->aR);
@@ -395,23 +414,12 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   long long nl = 0;
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u, ovf = 0u;
-  float amax = 0.0f;
+  // sum of the scores scaled by 2^-64: finite for any finite scores (at most
+  // 2^40 of them), inf or NaN as soon as one score is
+  float fsum = 0.0f;
 
-  const int64_t n = P.n;
-  // the 16-byte aligned body in chunks of CHUNK4 float4 (after a head of 0-3
-  // scores); the scores outside it go through the scalar loop below
-  const int head = row_head(row, n);
   int64_t nb4 = 0;
   {
-    const float4* x4 = reinterpret_cast<const float4*>(row + head);
-    const int64_t nchunks = ((n - head) >> 2) / CHUNK4;
-    // two chunks in flight per thread: the next chunk's loads are issued
-    // before the current one is processed
-    float4 nx[U];
-    if (cta < nchunks) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) nx[u] = __ldg(x4 + (int64_t)cta * CHUNK4 + threadIdx.x + u * NT);
-    }
     for (int64_t q = cta; q < nchunks; q += ncta) {
       const float4* base = x4 + q * CHUNK4 + threadIdx.x;
       float4 v[U];
@@ -421,38 +429,36 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
 #pragma unroll
         for (int u = 0; u < U; ++u) nx[u] = __ldg(base + (int64_t)ncta * CHUNK4 + u * NT);
       }
-      float pl = 0.0f, pr = 0.0f, am = 0.0f;
-      int cl = 0;
-      uint32_t mask = 0u;  // bit 4u+w: value w of float4 u lies in the band
+      // classification and tail terms on the FMA pipe (classify); the
+      // counts are exact small integers in fp32
+      float pl = 0.0f, pr = 0.0f, cl = 0.0f, cr = 0.0f;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-          const float x = xs[w];
-          const bool isL = x < aL, isR = x >= aR;
-          const float e = exp2f(fminf(x - aL, aR - x) * c2);
-          pl += isL ? e : 0.0f;
-          pr += isR ? e : 0.0f;
-          cl += isL ? 1 : 0;
-          mask |= (isL || isR) ? 0u : (1u << (4 * u + w));
-          am = fmaxf(am, fabsf(x));
+          const Side sd = classify(xs[w], aL, aR, c2);
+          pl = fmaf(sd.L, sd.e, pl);
+          pr = fmaf(sd.R, sd.e, pr);
+          cl += sd.L;
+          cr += sd.R;
+          fsum = fmaf(xs[w], 0x1p-64f, fsum);  // inf or NaN shows in this sum
         }
       }
       sl += (double)pl;
       sr += (double)pr;
-      nl += cl;
-      amax = fmaxf(amax, am);
-      if (mask) {  // rare: copy this lane's in-band values into its column
+      nl += (long long)cl;
+      if (cl + cr < (float)(4 * U)) {  // rare: copy this lane's in-band values into its column
 #pragma unroll
         for (int u = 0; u < U; ++u) scratch[u] = v[u];
         const float* sv = reinterpret_cast<const float*>(scratch);
-        do {
-          const int i = __ffs(mask) - 1;
-          mask &= mask - 1u;
-          col[ncol * NT] = sv[i];
-          ++ncol;
-        } while (mask);
+        for (int i = 0; i < 4 * U; ++i) {
+          const Side sd = classify(sv[i], aL, aR, c2);
+          if (sd.L + sd.R == 0.0f) {
+            col[ncol * NT] = sv[i];
+            ++ncol;
+          }
+        }
       }
       if (__any_sync(0xffffffffu, ncol > kLaneStage - 4 * U)) {
         flush_warp(f, col, ncol, bad, ovf);
@@ -468,15 +474,14 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
     const int64_t j = j0 + threadIdx.x;
     if (j < nrest) {
       const float x = row[rest_index(j, head, nb4)];
-      const bool isL = x < aL, isR = x >= aR;
-      const float e = exp2f(fminf(x - aL, aR - x) * c2);
-      if (isL) {
-        sl += (double)e;
+      const Side sd = classify(x, aL, aR, c2);
+      if (sd.L != 0.0f) {
+        sl += (double)sd.e;
         ++nl;
       }
-      if (isR) sr += (double)e;
-      amax = fmaxf(amax, fabsf(x));
-      if (!(isL || isR)) {
+      if (sd.R != 0.0f) sr += (double)sd.e;
+      fsum = fmaf(x, 0x1p-64f, fsum);
+      if (sd.L + sd.R == 0.0f) {
         col[ncol * NT] = x;
         ++ncol;
       }
@@ -487,7 +492,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
     }
   }
   if (__any_sync(0xffffffffu, ncol > 0)) flush_warp(f, col, ncol, bad, ovf);
-  if (!(amax < CUDART_INF_F)) bad = 1u;
+  if (!(fabsf(fsum) < CUDART_INF_F)) bad = 1u;
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
   nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
   sl = block_sum<NT, double>(sl, red);
@@ -511,7 +516,7 @@ constexpr size_t kFilterStageBytes = (size_t)(kLaneStage * NT) * 4 + (size_t)NT 
 __global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const float* __restrict__ scores) {
   __shared__ double red[64];
   __shared__ __align__(16) float stage[kFilterStageBytes / 4];
-  const int64_t r = blockIdx.y;
+  const int64_t r = blockIdx.y;  // filter_phase waits for the bracket's kernel
   filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red, stage);
 }
 
@@ -1096,6 +1101,7 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
 
 __global__ void __launch_bounds__(kBandThreads, 1) k_band(const StreamPlan P) {
   extern __shared__ __align__(16) unsigned char smem[];
+  wait_prior_grid();
   const int64_t r = blockIdx.y;
   const int cs = (int)cg::this_cluster().num_blocks();
   const int rank = (int)cg::this_cluster().block_rank();
@@ -1922,6 +1928,26 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   return cudaSuccess;
 }
 
+// Launches kern with programmatic stream serialization (kUsePdl): it may be
+// scheduled before the kernel ahead of it on the stream has finished, and
+// waits for it at entry (wait_prior_grid).
+constexpr bool kUsePdl = true;
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = kUsePdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p_out, double* b_out,
                               double* sumf_out, uint32_t* status_out, lapsum_row_stats* stats, int sm_count,
                               cudaStream_t st) {
@@ -1933,17 +1959,22 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     Launch l("k_sample", st);
     k_sample<<<dim3(P.Gs, rows), NT, 0, st>>>(P, scores);
   }
+  // the kernels below may be scheduled while the one ahead drains (each
+  // waits for it at entry: wait_prior_grid)
   {
     Launch l("k_select2", st);
-    k_select2<<<dim3(P.Gs, rows), NT, 0, st>>>(P);
+    e = launch_pdl(k_select2, dim3(P.Gs, rows), dim3(NT), 0, st, P);
+    if (e != cudaSuccess) return e;
   }
   {
     Launch l("k_select3", st);
-    k_select3<<<dim3(P.Gs, rows), NT, 0, st>>>(P);
+    e = launch_pdl(k_select3, dim3(P.Gs, rows), dim3(NT), 0, st, P);
+    if (e != cudaSuccess) return e;
   }
   {
     Launch l("k_filter", st);
-    k_filter<<<dim3(P.Gf, rows), NT, 0, st>>>(P, scores);
+    e = launch_pdl(k_filter, dim3(P.Gf, rows), dim3(NT), 0, st, P, scores);
+    if (e != cudaSuccess) return e;
   }
   {
     cudaLaunchConfig_t cfg = {};
@@ -1951,13 +1982,15 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     cfg.blockDim = dim3(kBandThreads, 1, 1);
     cfg.dynamicSmemBytes = kBandSmemBytes;
     cfg.stream = st;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = (unsigned)P.band_cs;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = kUsePdl ? 1 : 0;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     Launch l("k_band", st);
     e = cudaLaunchKernelEx(&cfg, k_band, P);
     if (e != cudaSuccess) return e;

@@ -38,7 +38,9 @@
  *     which take one of each per row.  alpha must lie in [1e-30, 1e30] (the
  *     fp32 exponent arithmetic needs 1/alpha finite).
  *   - The first call on a device queries its properties and sets kernel
- *     attributes; later calls on that device do not.
+ *     attributes; later calls on that device do not.  That set-up is kept
+ *     for the life of the process: after cudaDeviceReset, do not call the
+ *     library again in that process.
  */
 #ifndef LAPSUM_TOPK_H
 #define LAPSUM_TOPK_H
@@ -308,7 +310,11 @@ LAPSUM_API int lapsum_topk_bwd(const float* scores, const float* grad_p, const d
  * two host threads) race on that array and may return wrong results:
  * serialise them.
  * The first call on a device looks up the array's device address and sets
- * kernel attributes; make it before any stream capture on that device.
+ * kernel attributes; make it before any stream capture on that device.  The
+ * library keeps both for the life of the process: after cudaDeviceReset on
+ * that device they are stale, so do not call the library again in that
+ * process (this holds for every entry point, which cache the same per-device
+ * set-up).
  * Calls no cudaMalloc, cudaFree or other allocating routine.
  */
 #define LAPSUM_NOALLOC_MAX_ROWS 65536

@@ -296,7 +296,10 @@ def test_forced_paths_give_the_same_threshold(orc, name, n, force):
 @pytest.mark.parametrize("name,rows", [("c2", None), ("c5", 4)])
 def test_band_overflow_takes_the_fallback(orc, name, rows):
     w, x, g = case(name, rows=rows)
-    o = gpu_run(x, g, w.k, w.alpha, params=lt.Params(band_capacity=8))
+    # z = 5: a bracket wide enough that every row's band holds more than 8
+    # scores (at z = 4 a tied row's bracket can open above all its scores,
+    # with an empty band that certifies)
+    o = gpu_run(x, g, w.k, w.alpha, params=lt.Params(band_capacity=8, z=5.0))
     assert np.all(o["status"] & lt.ROW_OVERFLOW) and np.all(o["status"] & lt.ROW_FALLBACK)
     for i in range(x.shape[0]):
         check_row(orc, x[i], g[i], o["p"][i], o["grad"][i], o["b"][i], o["gk"][i], w.k, w.alpha, f"{name} row {i}")
