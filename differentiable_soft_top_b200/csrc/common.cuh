@@ -626,6 +626,9 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
 struct Side {
   float L, R, e;
 };
+struct Side2 {  // two scores (packed fp32x2 arithmetic where it exists)
+  float2 L, R, e;
+};
 __device__ __forceinline__ Side classify(float x, float aL, float aR, float c2) {
   const float dl = x - aL;
   const float dr = x - aR;
@@ -633,6 +636,19 @@ __device__ __forceinline__ Side classify(float x, float aL, float aR, float c2) 
   s.L = mul_sat(dl, -0x1p126f);
   s.R = fma_sat(dr, 0x1p126f, 1.0f);
   s.e = exp2f(-fabsf(fminf(dl, -dr)) * c2);
+  return s;
+}
+// classify for two scores: naL = (-aL, -aL), naR = (-aR, -aR), c22 = (c2, c2).
+// The same operations as classify (x - aL as x + (-aL) is the same rounded
+// value), so both give identical sides and terms.
+__device__ __forceinline__ Side2 classify2(float2 x, float2 naL, float2 naR, float2 c22) {
+  const float2 dl = __fadd2_rn(x, naL);
+  const float2 dr = __fadd2_rn(x, naR);
+  Side2 s;
+  s.L = make_float2(mul_sat(dl.x, -0x1p126f), mul_sat(dl.y, -0x1p126f));
+  s.R = make_float2(fma_sat(dr.x, 0x1p126f, 1.0f), fma_sat(dr.y, 0x1p126f, 1.0f));
+  const float2 a = __fmul2_rn(make_float2(fminf(dl.x, -dr.x), fminf(dl.y, -dr.y)), c22);
+  s.e = make_float2(exp2f(-fabsf(a.x)), exp2f(-fabsf(a.y)));
   return s;
 }
 

@@ -100,7 +100,10 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   int nl = 0;  // n_R is n - n_L - (band count): no per-score count for it
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
-  float fsum = 0.0f;  // sum of the scores scaled by 2^-64: +-inf or NaN shows here
+  // sum of the scores scaled by 2^-64: +-inf or NaN shows here
+  float2 fs2 = make_float2(0.0f, 0.0f);
+  const float2 naL2 = make_float2(-aL, -aL), naR2 = make_float2(-aR, -aR), c22 = make_float2(c2, c2);
+  const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
   // four scores per thread and step (the row's 16-byte aligned body); fp32
   // partial tail sums folded into fp64 once per step.  From global memory
   // (L2) kB steps' loads are issued before any is used.
@@ -123,32 +126,27 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
       const bool act = !decltype(checked)::value || v < n4;
       const float4 q = qs[u];
       const float xs[4] = {q.x, q.y, q.z, q.w};
-      // classification and tail terms on the FMA pipe (classify)
-      float pl = 0.0f, pr = 0.0f, cl = 0.0f, cr = 0.0f;
+      // classification and tail terms two scores at a time (classify2): tail
+      // sums, left count, and the positions outside the band as the bits of
+      // an exact fp32 sum
+      float2 pl2 = make_float2(0.0f, 0.0f), pr2 = pl2, cl2 = pl2, ob2 = pl2;
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const Side sd = classify(xs[w], aL, aR, c2);
-        pl = fmaf(sd.L, sd.e, pl);
-        pr = fmaf(sd.R, sd.e, pr);
-        cl += sd.L;
-        cr += sd.R;
-        fsum = fmaf(xs[w], 0x1p-64f, fsum);  // padding lanes hold 0
+      for (int h = 0; h < 2; ++h) {
+        const float2 x2 = h ? make_float2(q.z, q.w) : make_float2(q.x, q.y);
+        const Side2 sd = classify2(x2, naL2, naR2, c22);
+        pl2 = __ffma2_rn(sd.L, sd.e, pl2);
+        pr2 = __ffma2_rn(sd.R, sd.e, pr2);
+        cl2 = __fadd2_rn(cl2, sd.L);
+        ob2 = __ffma2_rn(__fadd2_rn(sd.L, sd.R), h ? make_float2(4.0f, 8.0f) : make_float2(1.0f, 2.0f), ob2);
+        fs2 = __ffma2_rn(x2, k64, fs2);  // padding lanes hold 0
       }
       if (act) {
-        sl += (double)pl;
-        sr += (double)pr;
-        nl += (int)cl;
+        sl += (double)(pl2.x + pl2.y);
+        sr += (double)(pr2.x + pr2.y);
+        nl += (int)(cl2.x + cl2.y);
       }
-      const bool has_band = act && cl + cr < 4.0f;
-      if (__any_sync(0xffffffffu, has_band)) {  // rare: this warp holds band values
-        uint32_t inb = 0u;
-        if (has_band) {
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const Side sd = classify(xs[w], aL, aR, c2);
-            inb |= (sd.L + sd.R == 0.0f) ? (1u << w) : 0u;
-          }
-        }
+      const uint32_t inb = act ? (~(uint32_t)(ob2.x + ob2.y) & 15u) : 0u;
+      if (__any_sync(0xffffffffu, inb != 0u)) {  // rare: this warp holds band values
         const int c = __popc(inb);
         int incl = c;
 #pragma unroll
@@ -209,7 +207,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
     }
   }
   }
-  if (!(fabsf(fsum) < CUDART_INF_F)) bad = 1u;
+  if (!(fabsf(fs2.x + fs2.y) < CUDART_INF_F)) bad = 1u;
   Filtered f;
   long long nll = nl;
   block_reduce_filtered(nll, sl, sr, bad, red);

@@ -29,6 +29,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "solve.cuh"
+#include "tma.cuh"
 
 namespace lapsum {
 namespace {
@@ -417,11 +418,18 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   // sum of the scores scaled by 2^-64: finite for any finite scores (at most
   // 2^40 of them), inf or NaN as soon as one score is
   float fsum = 0.0f;
+  float2 fs2 = make_float2(0.0f, 0.0f);
+  const float2 naL2 = make_float2(-aL, -aL), naR2 = make_float2(-aR, -aR), c22 = make_float2(c2, c2);
+  const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
 
   int64_t nb4 = 0;
   {
     for (int64_t q = cta; q < nchunks; q += ncta) {
       const float4* base = x4 + q * CHUNK4 + threadIdx.x;
+      // the chunk after the next one into L2 (its loads into registers are
+      // issued next iteration): more bytes in flight than registers hold
+      if (threadIdx.x == 0 && q + 2 * ncta < nchunks)
+        bulk_prefetch_l2(x4 + (q + 2 * ncta) * CHUNK4, CHUNK4 * 16u);
       float4 v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) v[u] = nx[u];
@@ -429,36 +437,39 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
 #pragma unroll
         for (int u = 0; u < U; ++u) nx[u] = __ldg(base + (int64_t)ncta * CHUNK4 + u * NT);
       }
-      // classification and tail terms on the FMA pipe (classify); the
-      // counts are exact small integers in fp32
-      float pl = 0.0f, pr = 0.0f, cl = 0.0f, cr = 0.0f;
+      // classification and tail terms two scores at a time (packed fp32x2
+      // arithmetic; the saturated side indicators of classify): tail sums,
+      // the left count, and the positions of the scores outside the band as
+      // bits of an exact fp32 sum
+      float2 pl2 = make_float2(0.0f, 0.0f), pr2 = pl2, cl2 = pl2, ob2 = pl2;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const float xs[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const Side sd = classify(xs[w], aL, aR, c2);
-          pl = fmaf(sd.L, sd.e, pl);
-          pr = fmaf(sd.R, sd.e, pr);
-          cl += sd.L;
-          cr += sd.R;
-          fsum = fmaf(xs[w], 0x1p-64f, fsum);  // inf or NaN shows in this sum
+        for (int h = 0; h < 2; ++h) {
+          const float2 x2 = h ? make_float2(v[u].z, v[u].w) : make_float2(v[u].x, v[u].y);
+          const Side2 sd = classify2(x2, naL2, naR2, c22);
+          const float bit = (float)(1u << (4 * u + 2 * h));
+          pl2 = __ffma2_rn(sd.L, sd.e, pl2);
+          pr2 = __ffma2_rn(sd.R, sd.e, pr2);
+          cl2 = __fadd2_rn(cl2, sd.L);
+          ob2 = __ffma2_rn(__fadd2_rn(sd.L, sd.R), make_float2(bit, 2.0f * bit), ob2);
+          fs2 = __ffma2_rn(x2, k64, fs2);
         }
       }
-      sl += (double)pl;
-      sr += (double)pr;
-      nl += (long long)cl;
-      if (cl + cr < (float)(4 * U)) {  // rare: copy this lane's in-band values into its column
+      sl += (double)(pl2.x + pl2.y);
+      sr += (double)(pr2.x + pr2.y);
+      nl += (long long)(cl2.x + cl2.y);
+      uint32_t mask = ~(uint32_t)(ob2.x + ob2.y) & ((1u << (4 * U)) - 1u);  // in-band positions
+      if (mask) {  // rare: copy this lane's in-band values into its column
 #pragma unroll
         for (int u = 0; u < U; ++u) scratch[u] = v[u];
         const float* sv = reinterpret_cast<const float*>(scratch);
-        for (int i = 0; i < 4 * U; ++i) {
-          const Side sd = classify(sv[i], aL, aR, c2);
-          if (sd.L + sd.R == 0.0f) {
-            col[ncol * NT] = sv[i];
-            ++ncol;
-          }
-        }
+        do {
+          const int i = __ffs(mask) - 1;
+          mask &= mask - 1u;
+          col[ncol * NT] = sv[i];
+          ++ncol;
+        } while (mask);
       }
       if (__any_sync(0xffffffffu, ncol > kLaneStage - 4 * U)) {
         flush_warp(f, col, ncol, bad, ovf);
@@ -466,6 +477,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
       }
     }
     nb4 = nchunks * CHUNK4;
+    fsum = fs2.x + fs2.y;
   }
   // the rest: one score per thread per step, the same trip count for the
   // whole block
