@@ -170,7 +170,7 @@ StreamSizes stream_sizes(int64_t n, double k, const Resolved& R) {
 }
 
 struct StreamLayout {
-  size_t ctl, h1, h2, h3, zero_end, samp, fpart, band, mpart, fb_keys, fb_aggs, rcount, total;
+  size_t ctl, h1, h2, h3, zero_end, samp, cand, fpart, band, mpart, fb_keys, fb_aggs, rcount, total;
 };
 StreamLayout stream_layout(int64_t rows, int64_t n, const StreamSizes& s) {
   StreamLayout L;
@@ -181,6 +181,7 @@ StreamLayout stream_layout(int64_t rows, int64_t n, const StreamSizes& s) {
   L.h3 = o;      o = align256(o + 4 * 2048 * (size_t)rows);
   L.zero_end = o;
   L.samp = o;    o = align256(o + 4 * (size_t)s.m * (size_t)rows);
+  L.cand = o;    o = align256(o + 4 * (size_t)((s.m + 3) & ~3) * (size_t)rows);
   L.fpart = o;   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
   L.band = o;    o = align256(o + 4 * (size_t)s.band_cap * (size_t)rows);
   L.mpart = o;   o = align256(o + 32 * (size_t)kMaxGridPerRow * (size_t)rows);
@@ -253,6 +254,7 @@ StreamPlan stream_plan(int64_t rows, int64_t n, int64_t row_stride, double k, do
   P.hist2 = reinterpret_cast<uint32_t*>(ws + L.h2);
   P.hist3 = reinterpret_cast<uint32_t*>(ws + L.h3);
   P.samp = reinterpret_cast<uint32_t*>(ws + L.samp);
+  P.cand = reinterpret_cast<uint32_t*>(ws + L.cand);
   P.fpart = ws + L.fpart;
   P.band = reinterpret_cast<float*>(ws + L.band);
   P.mpart = ws + L.mpart;

@@ -197,7 +197,8 @@ struct alignas(256) RowCtl {
   int32_t bins;        // key bins the band solve used (diagnostic)
   int32_t rank_lo, rank_hi;  // ascending sample ranks of the two edges
   uint32_t valid_lo, valid_hi;
-  int32_t widen_count, m;
+  uint32_t cand_cnt;   // keys in the row's level-3 candidate list
+  int32_t m;
   // aggregates and result
   int64_t nL, nR, M;
   double SL, SR;
@@ -623,6 +624,34 @@ __device__ __forceinline__ float fma_sat(float a, float b, float c) {
   asm("fma.rn.ftz.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
+// Packed fp32x2 arithmetic (two lanes per instruction on sm_100), with
+// denormals flushed like the scalar fp32 instructions under --ftz, so that a
+// packed and a scalar evaluation of the same formula agree bit for bit.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.ftz.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.ftz.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 struct Side {
   float L, R, e;
 };
@@ -642,12 +671,12 @@ __device__ __forceinline__ Side classify(float x, float aL, float aR, float c2) 
 // The same operations as classify (x - aL as x + (-aL) is the same rounded
 // value), so both give identical sides and terms.
 __device__ __forceinline__ Side2 classify2(float2 x, float2 naL, float2 naR, float2 c22) {
-  const float2 dl = __fadd2_rn(x, naL);
-  const float2 dr = __fadd2_rn(x, naR);
+  const float2 dl = add2(x, naL);
+  const float2 dr = add2(x, naR);
   Side2 s;
   s.L = make_float2(mul_sat(dl.x, -0x1p126f), mul_sat(dl.y, -0x1p126f));
   s.R = make_float2(fma_sat(dr.x, 0x1p126f, 1.0f), fma_sat(dr.y, 0x1p126f, 1.0f));
-  const float2 a = __fmul2_rn(make_float2(fminf(dl.x, -dr.x), fminf(dl.y, -dr.y)), c22);
+  const float2 a = mul2(make_float2(fminf(dl.x, -dr.x), fminf(dl.y, -dr.y)), c22);
   s.e = make_float2(exp2f(-fabsf(a.x)), exp2f(-fabsf(a.y)));
   return s;
 }

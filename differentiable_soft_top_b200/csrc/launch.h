@@ -30,6 +30,28 @@ class Launch {
   cudaEvent_t a_ = nullptr, b_ = nullptr;
 };
 
+// Launches kern on st; with `pdl`, with programmatic stream serialization:
+// the kernel may be scheduled before the one ahead of it on the stream has
+// finished, and must wait for it (griddepcontrol.wait) before it reads
+// anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+// kernels that follow a short or usually idle kernel are launched this way
+constexpr bool kPdlTail = true;
+
 // rows of at most this many scores run on the resident path (one block per
 // row, the row held in shared memory)
 constexpr int64_t kResidentMaxN = 16384;
@@ -125,6 +147,7 @@ struct StreamPlan {
   uint32_t* hist2;       // [rows][2][2048]
   uint32_t* hist3;       // [rows][2][1024]
   uint32_t* samp;        // [rows][m]
+  uint32_t* cand;        // [rows][m] sample keys of the two level-1 bins picked
   void* fpart;           // filter partials [rows][Gf]
   float* band;           // [rows][band_cap], unsorted
   void* mpart;           // membership partials [rows][Gm]

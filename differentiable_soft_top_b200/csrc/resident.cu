@@ -25,8 +25,10 @@ namespace {
 constexpr int NT = kResidentThreads;
 constexpr int kFbGroup = 1024;  // fallback: sorted values per group
 
+constexpr int kRowCol = 8;  // filter: staging column per lane (band keys)
+
 struct ResLayout {
-  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, red, mbar, total;
+  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, cols, red, mbar, total;
 };
 
 __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool row_in_smem) {
@@ -40,6 +42,7 @@ __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool
   L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
   L.dlink = o;    o = (o + 8 * (size_t)bcap + 8 + 15) & ~size_t(15);
+  L.cols = o;     o = o + 4 * (size_t)kRowCol * NT;
   L.red = o;      o = o + 8 * 64;
   L.mbar = o;     o = o + 16;
   L.total = o;
@@ -89,14 +92,33 @@ __device__ __forceinline__ void block_reduce_filtered(long long& nl, double& sl,
 // (section 2.2 stream-and-filter):
 // scores below a_L and at/above a_R go into counts and anchored tail sums
 // (every term exp(-dist/alpha) <= 1, fp32 exp, fp64 sums); scores inside the
-// bracket are appended to the band with one shared atomic per warp.
+// bracket are staged in a column per lane (cols: kRowCol keys per thread,
+// stride NT) and appended to the band with one shared atomic per warp when a
+// column is nearly full, and at the end.
 template <bool kGlobal>
 __device__ Filtered filter_row(const float* row, int n, float aL, float aR, float c2, uint32_t* band,
-                               int bcap, int* s_cnt, double* red) {
+                               int bcap, int* s_cnt, uint32_t* cols, double* red) {
   if (threadIdx.x == 0) *s_cnt = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
+  uint32_t* col = cols + threadIdx.x;
+  int ncol = 0;
+  auto flush = [&]() {  // every lane of the warp: its column into the band
+    int incl = ncol;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int wbase = 0;
+    if (lane == 0) wbase = atomicAdd(s_cnt, total);
+    int pos = __shfl_sync(0xffffffffu, wbase, 0) + incl - ncol;
+    for (int j = 0; j < ncol; ++j, ++pos)
+      if (pos < bcap) band[pos] = col[j * NT];
+    ncol = 0;
+  };
   int nl = 0;  // n_R is n - n_L - (band count): no per-score count for it
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
@@ -134,11 +156,11 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
       for (int h = 0; h < 2; ++h) {
         const float2 x2 = h ? make_float2(q.z, q.w) : make_float2(q.x, q.y);
         const Side2 sd = classify2(x2, naL2, naR2, c22);
-        pl2 = __ffma2_rn(sd.L, sd.e, pl2);
-        pr2 = __ffma2_rn(sd.R, sd.e, pr2);
-        cl2 = __fadd2_rn(cl2, sd.L);
-        ob2 = __ffma2_rn(__fadd2_rn(sd.L, sd.R), h ? make_float2(4.0f, 8.0f) : make_float2(1.0f, 2.0f), ob2);
-        fs2 = __ffma2_rn(x2, k64, fs2);  // padding lanes hold 0
+        pl2 = fma2(sd.L, sd.e, pl2);
+        pr2 = fma2(sd.R, sd.e, pr2);
+        cl2 = add2(cl2, sd.L);
+        ob2 = fma2(add2(sd.L, sd.R), h ? make_float2(4.0f, 8.0f) : make_float2(1.0f, 2.0f), ob2);
+        fs2 = fma2(x2, k64, fs2);  // padding lanes hold 0
       }
       if (act) {
         sl += (double)(pl2.x + pl2.y);
@@ -146,33 +168,23 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
         nl += (int)(cl2.x + cl2.y);
       }
       const uint32_t inb = act ? (~(uint32_t)(ob2.x + ob2.y) & 15u) : 0u;
-      if (__any_sync(0xffffffffu, inb != 0u)) {  // rare: this warp holds band values
-        const int c = __popc(inb);
-        int incl = c;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int t = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += t;
-        }
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        int wbase = 0;
-        if (lane == 0) wbase = atomicAdd(s_cnt, total);
-        wbase = __shfl_sync(0xffffffffu, wbase, 0);
-        int pos = wbase + incl - c;
+      if (inb) {  // rare: stage this lane's band values
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
           if ((inb >> w) & 1u) {
             if (!(fabsf(xs[w]) < CUDART_INF_F)) bad = 1u;  // NaN
-            if (pos < bcap) band[pos] = f2key(xs[w]);
-            ++pos;
+            col[ncol * NT] = f2key(xs[w]);
+            ++ncol;
           }
         }
       }
+      if (__any_sync(0xffffffffu, ncol > kRowCol - 4)) flush();
     }
   };
   if (base0 + kB * NT <= n4) step(std::false_type{});
   else step(std::true_type{});
   }
+  if (__any_sync(0xffffffffu, ncol > 0)) flush();
   // the scores outside the body: one per thread and step, the loads of kB
   // steps issued ahead from global memory
   const int nrest = n - (n4 << 2);
@@ -251,6 +263,15 @@ __device__ __forceinline__ float membership(float x, float bh, float bl, float c
   const float s = fma_sat(d, 0x1p126f, 1.0f);
   return fmaf(s, fmaf(-2.0f, h, 1.0f), h);
 }
+// membership for two scores with packed arithmetic: the same operations, so
+// the same values bit for bit (nbh = (-bh, -bh), nbl = (-bl, -bl))
+__device__ __forceinline__ float2 membership2(float2 x, float2 nbh, float2 nbl, float2 c22) {
+  const float2 d = add2(add2(x, nbh), nbl);
+  const float2 a = mul2(d, c22);
+  const float2 h = mul2(make_float2(exp2f(-fabsf(a.x)), exp2f(-fabsf(a.y))), make_float2(0.5f, 0.5f));
+  const float2 s = make_float2(fma_sat(d.x, 0x1p126f, 1.0f), fma_sat(d.y, 0x1p126f, 1.0f));
+  return fma2(s, fma2(make_float2(-2.0f, -2.0f), h, make_float2(1.0f, 1.0f)), h);
+}
 
 // Writes p for a row from `src` (shared or global) and finishes the row's
 // outputs; sumf is the solver's exact sum of f.  Every thread must call it.
@@ -264,6 +285,7 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
+  const float2 nbh2 = make_float2(-bh, -bh), nbl2 = make_float2(-bl, -bl), c22 = make_float2(c2, c2);
   double ps = 0.0;
   const bool nonfinite = (status & ROW_NAN_OUT) != 0u;
   if (a.dftopk) {
@@ -333,11 +355,9 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
         const int v = v0 + u * NT;
         if (v >= n4) break;
         const float4 x = xs[u];
-        float4 p;
-        p.x = membership(x.x, bh, bl, c2);
-        p.y = membership(x.y, bh, bl, c2);
-        p.z = membership(x.z, bh, bl, c2);
-        p.w = membership(x.w, bh, bl, c2);
+        const float2 p01 = membership2(make_float2(x.x, x.y), nbh2, nbl2, c22);
+        const float2 p23 = membership2(make_float2(x.z, x.w), nbh2, nbl2, c22);
+        float4 p = make_float4(p01.x, p01.y, p23.x, p23.y);
         if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
         ps += (double)((p.x + p.y) + (p.z + p.w));
         stg_stream(d4 + v, p);
@@ -385,6 +405,7 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
   double* dscr = reinterpret_cast<double*>(smem + L.dscr);
   double* dlink = reinterpret_cast<double*>(smem + L.dlink);
+  uint32_t* cols = reinterpret_cast<uint32_t*>(smem + L.cols);
   double* red = reinterpret_cast<double*>(smem + L.red);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
@@ -486,7 +507,7 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   Filtered f{};
   if (!a.force_fallback) {
     for (int attempt = 0;; ++attempt) {
-      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
+      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, cols, red);
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
       block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
@@ -560,6 +581,7 @@ __global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
   GroupAgg* aggs = reinterpret_cast<GroupAgg*>(smem + L.aggs);
   double* red = reinterpret_cast<double*>(smem + L.red);
   __shared__ SolveOut s_out;
+  wait_prior_grid();
   const int n = (int)a.n;
   const uint32_t cnt = *reinterpret_cast<volatile uint32_t*>(a.fb_count);
   for (uint32_t idx = blockIdx.x; idx < cnt; idx += gridDim.x) {
@@ -725,7 +747,8 @@ cudaError_t launch_resident_fwd(const ResidentFwd& a, int sm_count, cudaStream_t
   const unsigned fgrid = (unsigned)std::min<int64_t>(a.rows, (int64_t)sm_count);
   {
     Launch l("k_row_fallback", st);
-    k_row_fallback<<<fgrid, NT, fsmem, st>>>(a);
+    e = launch_ex(kPdlTail, k_row_fallback, dim3(fgrid), dim3(NT), fsmem, st, a);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

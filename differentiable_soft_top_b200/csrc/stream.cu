@@ -62,6 +62,10 @@ __device__ __forceinline__ MPart* mpart_of(const StreamPlan& P, int64_t r) {
 }
 __device__ __forceinline__ float* band_of(const StreamPlan& P, int64_t r) { return P.band + r * P.band_cap; }
 __device__ __forceinline__ uint32_t* samp_of(const StreamPlan& P, int64_t r) { return P.samp + r * (int64_t)P.m; }
+// the candidate list of a row starts 16-byte aligned (rows m rounded up to 4)
+__device__ __forceinline__ uint32_t* cand_of(const StreamPlan& P, int64_t r) {
+  return P.cand + r * (int64_t)((P.m + 3) & ~3);
+}
 __device__ __forceinline__ uint32_t* h1_of(const StreamPlan& P, int64_t r) { return P.hist1 + r * 2048; }
 __device__ __forceinline__ uint32_t* h2_of(const StreamPlan& P, int64_t r) { return P.hist2 + r * 4096; }
 __device__ __forceinline__ uint32_t* h3_of(const StreamPlan& P, int64_t r) { return P.hist3 + r * 2048; }
@@ -157,6 +161,42 @@ __device__ void sel_hist2(const uint32_t* samp, int m, int cta, int ncta, const 
     const uint32_t top = key >> 21, d = (key >> 10) & 2047u;
     hist_add(sh, d, act && top == (uint32_t)b1[0]);
     hist_add(sh + 2048, d, act && top == (uint32_t)b1[1]);
+  }
+  flush_hist(sh, gh2, 4096);
+}
+
+// sel_hist2, and the keys of the two level-1 bins appended to `cand` (one
+// atomic on *cnt per warp step that holds any)
+__device__ void sel_hist2_stash(const uint32_t* samp, int m, int cta, int ncta, const int b1[2], uint32_t* gh2,
+                                uint32_t* sh, uint32_t* cand, uint32_t* cnt) {
+  const int lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 4096; i += NT) sh[i] = 0u;
+  __syncthreads();
+  constexpr int kU = 4;  // keys loaded before any is used
+  const int step = ncta * NT;
+  for (int j0 = cta * NT; j0 < m; j0 += kU * step) {
+    uint32_t keys[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int j = j0 + u * step + (int)threadIdx.x;
+      keys[u] = j < m ? __ldcg(samp + j) : 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const bool act = j0 + u * step + (int)threadIdx.x < m;
+      const uint32_t key = keys[u];
+      const uint32_t top = key >> 21, d = (key >> 10) & 2047u;
+      const bool in0 = act && top == (uint32_t)b1[0], in1 = act && top == (uint32_t)b1[1];
+      hist_add(sh, d, in0);
+      hist_add(sh + 2048, d, in1);
+      const uint32_t cm = __ballot_sync(0xffffffffu, in0 || in1);
+      if (cm) {
+        uint32_t base = 0u;
+        if (lane == 0) base = atomicAdd(cnt, (uint32_t)__popc(cm));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (in0 || in1) cand[base + (uint32_t)__popc(cm & ((1u << lane) - 1u))] = key;
+      }
+    }
   }
   flush_hist(sh, gh2, 4096);
 }
@@ -291,6 +331,70 @@ __global__ void __launch_bounds__(NT) k_select2(const StreamPlan P) {
     uint32_t rem[2];
     sel_pick<2048>(h2_of(P, r), true, rk, scr, bin, rem);
     store_pick(c, 1, bin, rem);
+  }
+}
+
+// Levels 2 and 3 of the selection in one launch: every block histograms the
+// second level and stashes the keys of the two level-1 bins; the last block
+// picks level 2, then runs level 3 over the stash alone.
+__global__ void __launch_bounds__(NT) k_select23(const StreamPlan P) {
+  __shared__ uint32_t sh[4096];
+  __shared__ uint32_t scr[64];
+  wait_prior_grid();
+  const int64_t r = blockIdx.y;
+  RowCtl* c = ctl_of(P, r);
+  const int b1[2] = {c->sel_bin[0][0], c->sel_bin[0][1]};
+  uint32_t* cand = cand_of(P, r);
+  sel_hist2_stash(samp_of(P, r), P.m, blockIdx.x, gridDim.x, b1, h2_of(P, r), sh, cand, &c->cand_cnt);
+  if (last_block_done(&c->done_s2, gridDim.x)) {
+    uint32_t rk[2] = {c->sel_rem[0][0], c->sel_rem[0][1]};
+    int bin[2];
+    uint32_t rem[2];
+    sel_pick<2048>(h2_of(P, r), true, rk, scr, bin, rem);
+    const uint32_t pre[2] = {((uint32_t)b1[0] << 11) | (uint32_t)bin[0], ((uint32_t)b1[1] << 11) | (uint32_t)bin[1]};
+    // level 3 over the stashed keys (every key that can share a 22-bit prefix)
+    const uint32_t nc = vld(&c->cand_cnt);
+    for (int i = threadIdx.x; i < 2048; i += NT) sh[i] = 0u;
+    __syncthreads();
+    // 16-byte loads, kQ of them in flight per thread (one block walks the
+    // whole stash); the list starts 16-byte aligned (m is a multiple of 4)
+    constexpr int kQ = 4;
+    const uint4* c4 = reinterpret_cast<const uint4*>(cand);
+    const uint32_t nq = nc >> 2;
+    for (uint32_t q0 = 0; q0 < nq; q0 += kQ * NT) {
+      uint4 v[kQ];
+#pragma unroll
+      for (int u = 0; u < kQ; ++u) {
+        const uint32_t q = q0 + u * NT + threadIdx.x;
+        v[u] = q < nq ? __ldcg(c4 + q) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kQ; ++u) {
+        const bool act = q0 + u * NT + threadIdx.x < nq;
+        const uint32_t ks[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          hist_add(sh, ks[w] & 1023u, act && (ks[w] >> 10) == pre[0]);
+          hist_add(sh + 1024, ks[w] & 1023u, act && (ks[w] >> 10) == pre[1]);
+        }
+      }
+    }
+    for (uint32_t j = 4 * nq + threadIdx.x; j < 4 * nq + NT; j += NT) {  // the last 0-3 keys
+      const bool act = j < nc;
+      const uint32_t key = act ? __ldcg(cand + j) : 0u;
+      hist_add(sh, key & 1023u, act && (key >> 10) == pre[0]);
+      hist_add(sh + 1024, key & 1023u, act && (key >> 10) == pre[1]);
+    }
+    __syncthreads();
+    uint32_t* h3 = h3_of(P, r);
+    for (int i = threadIdx.x; i < 2048; i += NT) h3[i] = sh[i];
+    __syncthreads();
+    rk[0] = rem[0];
+    rk[1] = rem[1];
+    sel_pick<1024>(h3, true, rk, scr, bin, rem);
+    const uint32_t keys[2] = {(pre[0] << 10) | (uint32_t)bin[0], (pre[1] << 10) | (uint32_t)bin[1]};
+    const RowRanks rr = row_ranks(P, row_args(P, r).k);
+    if (threadIdx.x == 0) write_plan(c, P.m, keys, rr.rank_lo, rr.rank_hi, rr.valid_lo, rr.valid_hi);
   }
 }
 
@@ -449,11 +553,11 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
           const float2 x2 = h ? make_float2(v[u].z, v[u].w) : make_float2(v[u].x, v[u].y);
           const Side2 sd = classify2(x2, naL2, naR2, c22);
           const float bit = (float)(1u << (4 * u + 2 * h));
-          pl2 = __ffma2_rn(sd.L, sd.e, pl2);
-          pr2 = __ffma2_rn(sd.R, sd.e, pr2);
-          cl2 = __fadd2_rn(cl2, sd.L);
-          ob2 = __ffma2_rn(__fadd2_rn(sd.L, sd.R), make_float2(bit, 2.0f * bit), ob2);
-          fs2 = __ffma2_rn(x2, k64, fs2);
+          pl2 = fma2(sd.L, sd.e, pl2);
+          pr2 = fma2(sd.R, sd.e, pr2);
+          cl2 = add2(cl2, sd.L);
+          ob2 = fma2(add2(sd.L, sd.R), make_float2(bit, 2.0f * bit), ob2);
+          fs2 = fma2(x2, k64, fs2);
         }
       }
       sl += (double)(pl2.x + pl2.y);
@@ -1124,6 +1228,9 @@ __global__ void __launch_bounds__(kBandThreads, 1) k_band(const StreamPlan P) {
 // recovery: one widening, then the full-sort fallback (cooperative launch)
 // ===========================================================================
 
+// filter_phase in the recovery kernel uses the sort buffers kbuf, tbuf and
+// dscr (contiguous, 16 C bytes) as its stage
+static_assert(kFilterStageBytes <= (size_t)16 * kBucketMax, "the recovery kernel's filter stage does not fit");
 struct RecSmem {
   static constexpr size_t kSort = BandSmem::bytes(kBucketMax);
   static constexpr size_t kTotal = kSort > kBandSmemBytes ? kSort : kBandSmemBytes;
@@ -1408,6 +1515,7 @@ __global__ void __launch_bounds__(NT) k_memb(const StreamPlan P, const float* __
   __shared__ double red[64];
   __shared__ int32_t s_idx[kSparse ? NW * kSpWarpStage : 1];
   __shared__ float s_val[kSparse ? NW * kSpWarpStage : 1];
+  wait_prior_grid();
   const int64_t r = blockIdx.y;
   RowCtl* c = ctl_of(P, r);
   const double b = c->b;
@@ -1752,6 +1860,7 @@ __global__ void __launch_bounds__(NT) k_bwd_combine(const StreamBwd a, const BPa
 // grad = f (g - lambda), f = 2^(log2(1/(2 alpha)) - |x - b| log2(e)/alpha) in
 // one exponent, lambda split into two fp32 words
 __global__ void __launch_bounds__(NT) k_bwd_apply(const StreamBwd a) {
+  wait_prior_grid();
   const int64_t r = blockIdx.y;
   const double b = a.b[r];
   bool bad = false;
@@ -1940,24 +2049,13 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   return cudaSuccess;
 }
 
-// Launches kern with programmatic stream serialization (kUsePdl): it may be
-// scheduled before the kernel ahead of it on the stream has finished, and
-// waits for it at entry (wait_prior_grid).
+// the short kernels of the forward pipeline are launched with programmatic
+// stream serialization (each waits for the one ahead: wait_prior_grid)
 constexpr bool kUsePdl = true;
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                        Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  at[0].val.programmaticStreamSerializationAllowed = kUsePdl ? 1 : 0;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+  return launch_ex(kUsePdl, kern, grid, block, smem, st, args...);
 }
 
 cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p_out, double* b_out,
@@ -1974,13 +2072,8 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
   // the kernels below may be scheduled while the one ahead drains (each
   // waits for it at entry: wait_prior_grid)
   {
-    Launch l("k_select2", st);
-    e = launch_pdl(k_select2, dim3(P.Gs, rows), dim3(NT), 0, st, P);
-    if (e != cudaSuccess) return e;
-  }
-  {
-    Launch l("k_select3", st);
-    e = launch_pdl(k_select3, dim3(P.Gs, rows), dim3(NT), 0, st, P);
+    Launch l("k_select23", st);
+    e = launch_pdl(k_select23, dim3(P.Gs, rows), dim3(NT), 0, st, P);
     if (e != cudaSuccess) return e;
   }
   {
@@ -2025,9 +2118,12 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     } else {
       Launch l(P.dftopk ? "k_memb_dftopk" : "k_memb", st);
       if (P.dftopk)
-        k_memb<false, true><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+        e = launch_ex(kPdlTail, k_memb<false, true>, dim3(P.Gm, rows), dim3(NT), 0, st, P, scores, p_out, b_out,
+                      sumf_out, status_out, stats);
       else
-        k_memb<false, false><<<dim3(P.Gm, rows), NT, 0, st>>>(P, scores, p_out, b_out, sumf_out, status_out, stats);
+        e = launch_ex(kPdlTail, k_memb<false, false>, dim3(P.Gm, rows), dim3(NT), 0, st, P, scores, p_out, b_out,
+                      sumf_out, status_out, stats);
+      if (e != cudaSuccess) return e;
     }
   }
   return cudaGetLastError();
@@ -2043,7 +2139,8 @@ cudaError_t launch_stream_bwd(const StreamBwd& a, cudaStream_t st) {
   }
   {
     Launch l("k_bwd_apply", st);
-    k_bwd_apply<<<dim3(a.Ga, (unsigned)a.rows), NT, 0, st>>>(a);
+    e = launch_ex(kPdlTail, k_bwd_apply, dim3(a.Ga, (unsigned)a.rows), dim3(NT), 0, st, a);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -2139,7 +2236,8 @@ cudaError_t launch_shard_bwd_finish(const StreamBwd& a, const void* parts_all, i
   }
   {
     Launch l("k_bwd_apply", st);
-    k_bwd_apply<<<dim3(a.Ga, (unsigned)a.rows), NT, 0, st>>>(a);
+    const cudaError_t e = launch_ex(kPdlTail, k_bwd_apply, dim3(a.Ga, (unsigned)a.rows), dim3(NT), 0, st, a);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
