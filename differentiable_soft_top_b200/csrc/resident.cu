@@ -25,10 +25,8 @@ namespace {
 constexpr int NT = kResidentThreads;
 constexpr int kFbGroup = 1024;  // fallback: sorted values per group
 
-constexpr int kRowCol = 8;  // filter: staging column per lane (band keys)
-
 struct ResLayout {
-  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, cols, red, mbar, total;
+  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, red, mbar, total;
 };
 
 __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool row_in_smem) {
@@ -42,7 +40,6 @@ __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool
   L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
   L.dlink = o;    o = (o + 8 * (size_t)bcap + 8 + 15) & ~size_t(15);
-  L.cols = o;     o = o + 4 * (size_t)kRowCol * NT;
   L.red = o;      o = o + 8 * 64;
   L.mbar = o;     o = o + 16;
   L.total = o;
@@ -92,33 +89,18 @@ __device__ __forceinline__ void block_reduce_filtered(long long& nl, double& sl,
 // (section 2.2 stream-and-filter):
 // scores below a_L and at/above a_R go into counts and anchored tail sums
 // (every term exp(-dist/alpha) <= 1, fp32 exp, fp64 sums); scores inside the
-// bracket are staged in a column per lane (cols: kRowCol keys per thread,
-// stride NT) and appended to the band with one shared atomic per warp when a
-// column is nearly full, and at the end.
+// bracket are appended to the band with one shared atomic each.  A thread
+// takes 16 scores a step (four float4, their loads issued together) and
+// learns which of them lie in the band from the bits of an exact fp32 sum;
+// those few are read again by position (from L1 or shared memory), so the
+// common step has no branch per score.
 template <bool kGlobal>
 __device__ Filtered filter_row(const float* row, int n, float aL, float aR, float c2, uint32_t* band,
-                               int bcap, int* s_cnt, uint32_t* cols, double* red) {
+                               int bcap, int* s_cnt, double* red) {
   if (threadIdx.x == 0) *s_cnt = 0;
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
-  uint32_t* col = cols + threadIdx.x;
-  int ncol = 0;
-  auto flush = [&]() {  // every lane of the warp: its column into the band
-    int incl = ncol;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    int wbase = 0;
-    if (lane == 0) wbase = atomicAdd(s_cnt, total);
-    int pos = __shfl_sync(0xffffffffu, wbase, 0) + incl - ncol;
-    for (int j = 0; j < ncol; ++j, ++pos)
-      if (pos < bcap) band[pos] = col[j * NT];
-    ncol = 0;
-  };
   int nl = 0;  // n_R is n - n_L - (band count): no per-score count for it
   double sl = 0.0, sr = 0.0;
   uint32_t bad = 0u;
@@ -126,65 +108,56 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   float2 fs2 = make_float2(0.0f, 0.0f);
   const float2 naL2 = make_float2(-aL, -aL), naR2 = make_float2(-aR, -aR), c22 = make_float2(c2, c2);
   const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
-  // four scores per thread and step (the row's 16-byte aligned body); fp32
-  // partial tail sums folded into fp64 once per step.  From global memory
-  // (L2) kB steps' loads are issued before any is used.
-  constexpr int kB = kGlobal ? 4 : 1;
+  constexpr int kB = 4;
   const int head = row_head(row, n);
   const int n4 = (n - head) >> 2;
-  const float4* row4 = reinterpret_cast<const float4*>(row + head);
+  const float* rowh = row + head;
+  const float4* row4 = reinterpret_cast<const float4*>(rowh);
   for (int base0 = 0; base0 < n4; base0 += kB * NT) {
-  float4 qs[kB];
-#pragma unroll
-  for (int u = 0; u < kB; ++u) {
-    const int v = base0 + u * NT + threadIdx.x;
-    qs[u] = v < n4 ? (kGlobal ? __ldg(row4 + v) : row4[v]) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-  }
-  // a step whose lanes all lie inside the row needs no per-score range check
-  auto step = [&](auto checked) {
+    float4 qs[kB];
 #pragma unroll
     for (int u = 0; u < kB; ++u) {
       const int v = base0 + u * NT + threadIdx.x;
-      const bool act = !decltype(checked)::value || v < n4;
-      const float4 q = qs[u];
-      const float xs[4] = {q.x, q.y, q.z, q.w};
-      // classification and tail terms two scores at a time (classify2): tail
-      // sums, left count, and the positions outside the band as the bits of
-      // an exact fp32 sum
+      qs[u] = v < n4 ? (kGlobal ? __ldg(row4 + v) : row4[v]) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+    // a step whose lanes all lie inside the row needs no per-score range check
+    auto step = [&](auto checked) {
       float2 pl2 = make_float2(0.0f, 0.0f), pr2 = pl2, cl2 = pl2, ob2 = pl2;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float2 x2 = h ? make_float2(q.z, q.w) : make_float2(q.x, q.y);
-        const Side2 sd = classify2(x2, naL2, naR2, c22);
-        pl2 = fma2(sd.L, sd.e, pl2);
-        pr2 = fma2(sd.R, sd.e, pr2);
-        cl2 = add2(cl2, sd.L);
-        ob2 = fma2(add2(sd.L, sd.R), h ? make_float2(4.0f, 8.0f) : make_float2(1.0f, 2.0f), ob2);
-        fs2 = fma2(x2, k64, fs2);  // padding lanes hold 0
-      }
-      if (act) {
-        sl += (double)(pl2.x + pl2.y);
-        sr += (double)(pr2.x + pr2.y);
-        nl += (int)(cl2.x + cl2.y);
-      }
-      const uint32_t inb = act ? (~(uint32_t)(ob2.x + ob2.y) & 15u) : 0u;
-      if (inb) {  // rare: stage this lane's band values
+      for (int u = 0; u < kB; ++u) {
+        const bool act = !decltype(checked)::value || base0 + u * NT + (int)threadIdx.x < n4;
+        const float4 q = qs[u];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          if ((inb >> w) & 1u) {
-            if (!(fabsf(xs[w]) < CUDART_INF_F)) bad = 1u;  // NaN
-            col[ncol * NT] = f2key(xs[w]);
-            ++ncol;
-          }
+        for (int h = 0; h < 2; ++h) {
+          const float2 x2 = h ? make_float2(q.z, q.w) : make_float2(q.x, q.y);
+          const Side2 sd = classify2(x2, naL2, naR2, c22);
+          float2 L = sd.L, R = sd.R;
+          if (!act) L = R = make_float2(0.0f, 0.0f);
+          const float bit = (float)(1u << (4 * u + 2 * h));
+          pl2 = fma2(L, sd.e, pl2);
+          pr2 = fma2(R, sd.e, pr2);
+          cl2 = add2(cl2, L);
+          // positions outside the band (a padding position counts as outside)
+          ob2 = fma2(act ? add2(L, R) : make_float2(1.0f, 1.0f), make_float2(bit, 2.0f * bit), ob2);
+          fs2 = fma2(x2, k64, fs2);  // padding lanes hold 0
         }
       }
-      if (__any_sync(0xffffffffu, ncol > kRowCol - 4)) flush();
-    }
-  };
-  if (base0 + kB * NT <= n4) step(std::false_type{});
-  else step(std::true_type{});
+      sl += (double)(pl2.x + pl2.y);
+      sr += (double)(pr2.x + pr2.y);
+      nl += (int)(cl2.x + cl2.y);
+      uint32_t mask = ~(uint32_t)(ob2.x + ob2.y) & 0xFFFFu;  // in-band positions of this thread's 16
+      while (mask) {  // rare: read each again by position and append it
+        const int i = __ffs(mask) - 1;
+        mask &= mask - 1u;
+        const float x = rowh[4 * (base0 + (i >> 2) * NT + (int)threadIdx.x) + (i & 3)];
+        if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;  // NaN
+        const int pos = atomicAdd(s_cnt, 1);
+        if (pos < bcap) band[pos] = f2key(x);
+      }
+    };
+    if (base0 + kB * NT <= n4) step(std::false_type{});
+    else step(std::true_type{});
   }
-  if (__any_sync(0xffffffffu, ncol > 0)) flush();
   // the scores outside the body: one per thread and step, the loads of kB
   // steps issued ahead from global memory
   const int nrest = n - (n4 << 2);
@@ -336,32 +309,45 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
     __syncthreads();
   } else if (a.vec) {
     // src and dst start at the same address mod 16 (a shared-memory copy is
-    // placed that way): one head, then float4 from both
+    // placed that way): one head, then float4 from both.  sum p is only
+    // accumulated when the caller asked for it (sump_out, stats).
     float* dst = a.p_out + r * a.stride;
     const int head = row_head(src, n);
     const float4* s4 = reinterpret_cast<const float4*>(src + head);
     float4* d4 = reinterpret_cast<float4*>(dst + head);
     const int n4 = (n - head) >> 2;
     constexpr int kB = 4;  // loads in flight per thread (the row may be in global memory)
-    for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
-      float4 xs[kB];
+    auto pass = [&](auto want_ps) {
+      for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
+        float4 xs[kB];
 #pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int v = v0 + u * NT;
-        xs[u] = v < n4 ? s4[v] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      }
+        for (int u = 0; u < kB; ++u) {
+          const int v = v0 + u * NT;
+          xs[u] = v < n4 ? s4[v] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+        auto put = [&](auto checked) {
 #pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int v = v0 + u * NT;
-        if (v >= n4) break;
-        const float4 x = xs[u];
-        const float2 p01 = membership2(make_float2(x.x, x.y), nbh2, nbl2, c22);
-        const float2 p23 = membership2(make_float2(x.z, x.w), nbh2, nbl2, c22);
-        float4 p = make_float4(p01.x, p01.y, p23.x, p23.y);
-        if (nonfinite) p = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
-        ps += (double)((p.x + p.y) + (p.z + p.w));
-        stg_stream(d4 + v, p);
+          for (int u = 0; u < kB; ++u) {
+            const int v = v0 + u * NT;
+            if (decltype(checked)::value && v >= n4) break;
+            const float4 x = xs[u];
+            const float2 p01 = membership2(make_float2(x.x, x.y), nbh2, nbl2, c22);
+            const float2 p23 = membership2(make_float2(x.z, x.w), nbh2, nbl2, c22);
+            if (decltype(want_ps)::value) ps += (double)((p01.x + p01.y) + (p23.x + p23.y));
+            stg_stream(d4 + v, make_float4(p01.x, p01.y, p23.x, p23.y));
+          }
+        };
+        if (v0 - (int)threadIdx.x + kB * NT <= n4) put(std::false_type{});
+        else put(std::true_type{});
       }
+    };
+    if (nonfinite) {
+      const float4 nan4 = make_float4(CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F, CUDART_NAN_F);
+      for (int v = threadIdx.x; v < n4; v += NT) stg_stream(d4 + v, nan4);
+    } else if (a.sump_out || a.stats) {
+      pass(std::true_type{});
+    } else {
+      pass(std::false_type{});
     }
     for (int j = threadIdx.x; j < n - (n4 << 2); j += NT) {
       const int i = (int)rest_index(j, head, n4);
@@ -405,7 +391,6 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
   double* dscr = reinterpret_cast<double*>(smem + L.dscr);
   double* dlink = reinterpret_cast<double*>(smem + L.dlink);
-  uint32_t* cols = reinterpret_cast<uint32_t*>(smem + L.cols);
   double* red = reinterpret_cast<double*>(smem + L.red);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
@@ -507,7 +492,7 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   Filtered f{};
   if (!a.force_fallback) {
     for (int attempt = 0;; ++attempt) {
-      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, cols, red);
+      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
       block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
