@@ -26,7 +26,7 @@ constexpr int NT = kResidentThreads;
 constexpr int kFbGroup = 1024;  // fallback: sorted values per group
 
 struct ResLayout {
-  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, red, mbar, total;
+  size_t row, samp, samp_tmp, band, band_tmp, dscr, dlink, sortscr, red, mbar, total;
 };
 
 __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool row_in_smem) {
@@ -40,6 +40,7 @@ __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool
   L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
   L.dlink = o;    o = (o + 8 * (size_t)bcap + 8 + 15) & ~size_t(15);
+  L.sortscr = o;  o = o + 4 * 576;  // the band's bucket sort
   L.red = o;      o = o + 8 * 64;
   L.mbar = o;     o = o + 16;
   L.total = o;
@@ -57,6 +58,7 @@ struct Filtered {
   double SL, SR;
   int M;
   uint32_t bad;
+  uint32_t kmin, kmax;  // smallest and largest key appended to the band
 };
 
 // The filter's four block reductions (n_L, S_L, S_R, the non-finite flag)
@@ -96,8 +98,12 @@ __device__ __forceinline__ void block_reduce_filtered(long long& nl, double& sl,
 // common step has no branch per score.
 template <bool kGlobal>
 __device__ Filtered filter_row(const float* row, int n, float aL, float aR, float c2, uint32_t* band,
-                               int bcap, int* s_cnt, double* red) {
-  if (threadIdx.x == 0) *s_cnt = 0;
+                               int bcap, int* s_cnt, uint32_t* s_kr, double* red) {
+  if (threadIdx.x == 0) {
+    *s_cnt = 0;
+    s_kr[0] = 0xFFFFFFFFu;
+    s_kr[1] = 0u;
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31;
   const uint32_t lt = (1u << lane) - 1u;
@@ -151,8 +157,11 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
         mask &= mask - 1u;
         const float x = rowh[4 * (base0 + (i >> 2) * NT + (int)threadIdx.x) + (i & 3)];
         if (!(fabsf(x) < CUDART_INF_F)) bad = 1u;  // NaN
+        const uint32_t key = f2key(x);
         const int pos = atomicAdd(s_cnt, 1);
-        if (pos < bcap) band[pos] = f2key(x);
+        if (pos < bcap) band[pos] = key;
+        atomicMin(&s_kr[0], key);
+        atomicMax(&s_kr[1], key);
       }
     };
     if (base0 + kB * NT <= n4) step(std::false_type{});
@@ -187,7 +196,10 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
       wbase = __shfl_sync(0xffffffffu, wbase, leader);
       if (inb) {
         const int pos = wbase + __popc(msk & lt);
-        if (pos < bcap) band[pos] = f2key(x);
+        const uint32_t key = f2key(x);
+        if (pos < bcap) band[pos] = key;
+        atomicMin(&s_kr[0], key);
+        atomicMax(&s_kr[1], key);
       }
     }
   }
@@ -201,6 +213,8 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   f.SR = sr;
   f.bad = bad;
   f.M = *s_cnt;
+  f.kmin = s_kr[0];
+  f.kmax = s_kr[1];
   f.nR = (long long)n - f.nL - (long long)f.M;  // every score is left, right or in the band
   __syncthreads();
   return f;
@@ -391,9 +405,12 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   uint32_t* band = reinterpret_cast<uint32_t*>(smem + L.band);
   double* dscr = reinterpret_cast<double*>(smem + L.dscr);
   double* dlink = reinterpret_cast<double*>(smem + L.dlink);
+  uint32_t* band_tmp = reinterpret_cast<uint32_t*>(smem + L.band_tmp);
+  uint32_t* sortscr = reinterpret_cast<uint32_t*>(smem + L.sortscr);
   double* red = reinterpret_cast<double*>(smem + L.red);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + L.mbar);
   __shared__ int s_cnt;
+  __shared__ uint32_t s_kr[2];
   __shared__ SolveOut s_out;
 
   const int64_t r = blockIdx.x;
@@ -492,12 +509,18 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
   Filtered f{};
   if (!a.force_fallback) {
     for (int attempt = 0;; ++attempt) {
-      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, red);
+      f = filter_row<!kSmemRow>(row, n, aL, aR, c2, band, a.bcap, &s_cnt, s_kr, red);
       if (f.bad) { status |= ROW_NONFINITE; break; }
       if (f.M > a.bcap) { status |= ROW_OVERFLOW; break; }
-      block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
+      // one bucket pass over the band's key range; a band stretched by
+      // outliers into crowded buckets takes the bitonic network instead
+      const uint32_t* sorted = block_bucket_sort<NT>(band, band_tmp, f.M, f.kmin, f.kmax, sortscr);
+      if (!sorted) {
+        block_bitonic_sort<NT>(band, f.M);  // band and band_tmp form one buffer of 2 bcap keys
+        sorted = band;
+      }
       SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, ra.k, ra.alpha, inva};
-      solve_run<NT>(in, band, f.M, dscr, dlink, red, &s_out);
+      solve_run<NT>(in, sorted, f.M, dscr, dlink, red, &s_out);
       if (s_out.status & ROW_CERTIFIED) { solved = true; break; }
       if (attempt >= a.max_widen) break;
       // widen once on the side that missed; the other edge moves to the old
@@ -575,7 +598,24 @@ __global__ void __launch_bounds__(NT) k_row_fallback(const ResidentFwd a) {
     const RowArgs ra = row_args(a, r);
     const double inva = 1.0 / ra.alpha;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += NT) keys[i] = f2key(src[i]);
+    {
+      // eight loads a thread in flight (one block per SM: the loop would
+      // otherwise wait on every load)
+      constexpr int kLd = 8;
+      for (int i0 = 0; i0 < n; i0 += kLd * NT) {
+        float xx[kLd];
+#pragma unroll
+        for (int u = 0; u < kLd; ++u) {
+          const int i = i0 + u * NT + (int)threadIdx.x;
+          xx[u] = i < n ? src[i] : 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kLd; ++u) {
+          const int i = i0 + u * NT + (int)threadIdx.x;
+          if (i < n) keys[i] = f2key(xx[u]);
+        }
+      }
+    }
     __syncthreads();
     const uint32_t* sorted = block_radix_sort<NT>(keys, tmp, n, hist);
     __syncthreads();
@@ -624,6 +664,7 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     const float4* x4 = reinterpret_cast<const float4*>(x + head);
     const float4* g4 = reinterpret_cast<const float4*>(g + head);
     constexpr int kB = 4;
+    const float2 nbh2 = make_float2(-bh, -bh), nbl2 = make_float2(-bl, -bl), c22 = make_float2(c2, c2);
     for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
       float4 xv[kB], gv[kB];
 #pragma unroll
@@ -632,18 +673,63 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
         xv[u] = v < n4 ? __ldg(x4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
         gv[u] = v < n4 ? __ldg(g4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      // The step's 16 exponents a = |r - b| log2(e)/alpha in packed
+      // arithmetic; the terms 2^(m - a) are taken relative to the running
+      // minimum m, moved (and the sums rescaled) at most once a step rather
+      // than tested for every score.  Padding positions get a = +inf.  With
+      // kAlpha the z-weighted sums of dL/dalpha ride along; the two sums of
+      // lambda take the same operations either way.
+      float ae[4 * kB];
+      float2 zz[kAlpha ? 2 * kB : 1];
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
-        if (v0 + u * NT >= n4) break;
-        float ps = 0.0f, psg = 0.0f, psz = 0.0f, psgz = 0.0f;
-        acc(xv[u].x, gv[u].x, ps, psg, psz, psgz);
-        acc(xv[u].y, gv[u].y, ps, psg, psz, psgz);
-        acc(xv[u].z, gv[u].z, ps, psg, psz, psgz);
-        acc(xv[u].w, gv[u].w, ps, psg, psz, psgz);
-        S += (double)ps;
-        SG += (double)psg;
-        SZ += (double)psz;
-        SGZ += (double)psgz;
+        const bool act = v0 + u * NT < n4;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 x2 = h ? make_float2(xv[u].z, xv[u].w) : make_float2(xv[u].x, xv[u].y);
+          const float2 z = add2(add2(x2, nbh2), nbl2);
+          if (kAlpha) zz[2 * u + h] = z;
+          const float2 q = mul2(z, c22);
+          ae[4 * u + 2 * h] = act ? fabsf(q.x) : CUDART_INF_F;
+          ae[4 * u + 2 * h + 1] = act ? fabsf(q.y) : CUDART_INF_F;
+        }
+      }
+      float mstep = ae[0];
+#pragma unroll
+      for (int i = 1; i < 4 * kB; ++i) mstep = fminf(mstep, ae[i]);
+      if (mstep < m) {  // a new nearest score: rescale what was accumulated
+        const double sc = (double)exp2f(mstep - m);
+        S *= sc;
+        SG *= sc;
+        if (kAlpha) {
+          SZ *= sc;
+          SGZ *= sc;
+        }
+        m = mstep;
+      }
+      float2 ps2 = make_float2(0.0f, 0.0f), psg2 = ps2, psz2 = ps2, psgz2 = ps2;
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 g2 = h ? make_float2(gv[u].z, gv[u].w) : make_float2(gv[u].x, gv[u].y);
+          const float2 e2 = make_float2(exp2f(m - ae[4 * u + 2 * h]), exp2f(m - ae[4 * u + 2 * h + 1]));
+          ps2 = add2(ps2, e2);
+          psg2 = fma2(g2, e2, psg2);
+          if (kAlpha) {
+            const float2 ez = mul2(e2, zz[2 * u + h]);
+            psz2 = add2(psz2, ez);
+            psgz2 = fma2(g2, ez, psgz2);
+          }
+        }
+      }
+      if (m < CUDART_INF_F) {  // no finite exponent yet: nothing to add
+        S += (double)(ps2.x + ps2.y);
+        SG += (double)(psg2.x + psg2.y);
+        if (kAlpha) {
+          SZ += (double)(psz2.x + psz2.y);
+          SGZ += (double)(psgz2.x + psgz2.y);
+        }
       }
     }
     const int nrest = n - (n4 << 2);
@@ -661,6 +747,7 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
     const double lam = bad ? CUDART_NAN : SG / S;  // NaN also reaches every grad of the row
     const float lh = __double2float_rn(lam);
     const float ll = __double2float_rn(lam - (double)lh);
+    const float2 nlh2 = make_float2(-lh, -lh), nll2 = make_float2(-ll, -ll);
     for (int v0 = threadIdx.x; v0 < n4; v0 += kB * NT) {
       float4 xv[kB], gv[kB];
 #pragma unroll
@@ -673,12 +760,17 @@ __global__ void __launch_bounds__(NT) k_row_bwd(const RowBwd a) {
       for (int u = 0; u < kB; ++u) {
         const int v = v0 + u * NT;
         if (v >= n4) break;
-        float4 ov;
-        ov.x = exp2f(fmaf(-fabsf((xv[u].x - bh) - bl), c2, lg)) * ((gv[u].x - lh) - ll);
-        ov.y = exp2f(fmaf(-fabsf((xv[u].y - bh) - bl), c2, lg)) * ((gv[u].y - lh) - ll);
-        ov.z = exp2f(fmaf(-fabsf((xv[u].z - bh) - bl), c2, lg)) * ((gv[u].z - lh) - ll);
-        ov.w = exp2f(fmaf(-fabsf((xv[u].w - bh) - bl), c2, lg)) * ((gv[u].w - lh) - ll);
-        stg_stream(reinterpret_cast<float4*>(o + head) + v, ov);
+        // the same operations as the scalar form below, two scores at a time
+        float2 o2[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const float2 x2 = h ? make_float2(xv[u].z, xv[u].w) : make_float2(xv[u].x, xv[u].y);
+          const float2 g2 = h ? make_float2(gv[u].z, gv[u].w) : make_float2(gv[u].x, gv[u].y);
+          const float2 z = add2(add2(x2, nbh2), nbl2);
+          const float2 f = make_float2(exp2f(fmaf(-fabsf(z.x), c2, lg)), exp2f(fmaf(-fabsf(z.y), c2, lg)));
+          o2[h] = mul2(f, add2(add2(g2, nlh2), nll2));
+        }
+        stg_stream(reinterpret_cast<float4*>(o + head) + v, make_float4(o2[0].x, o2[0].y, o2[1].x, o2[1].y));
       }
     }
     for (int j = threadIdx.x; j < nrest; j += NT) {

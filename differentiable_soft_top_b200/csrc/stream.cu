@@ -708,6 +708,8 @@ struct BinPart {  // one CTA's bins
 };
 struct TargetBuf {
   uint32_t keys[kTargetCap];
+  uint32_t sorted[kTargetCap];  // the bucket sort's output
+  uint32_t scr[576];            // and its scratch
 };
 enum : int { kBandDone = 0, kBandRefine = 1, kBandExtract = 2 };
 struct BandDecision {
@@ -1140,9 +1142,15 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
         // group solve then picks the interval between two values that holds
         // the root, and the closed form finishes
         const int cnt = (int)min(S.dec.count, (uint32_t)kTargetCap);
-        uint32_t* keys = S.u.tgt.keys;
-        block_bitonic_sort<NTX>(keys, cnt);
         BinTable<kBins>& T = S.tu.tab;
+        // one bucket pass over the bin's key range (its extremes from the
+        // merge); a bin stretched by outliers takes the bitonic network
+        const uint32_t bk0 = f2key(T.ymin[S.pk.tg]), bk1 = f2key(T.ymax[S.pk.tg]);
+        const uint32_t* keys = block_bucket_sort<NTX>(S.u.tgt.keys, S.u.tgt.sorted, cnt, bk0, bk1, S.u.tgt.scr);
+        if (!keys) {
+          block_bitonic_sort<NTX>(S.u.tgt.keys, cnt);
+          keys = S.u.tgt.keys;
+        }
         const float ylast = key2f(keys[cnt - 1]);
         for (int i = threadIdx.x; i < kBins; i += NTX) {
           if (i < cnt) {
@@ -1400,11 +1408,18 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         const int shift = 8 * pass;
         for (int i = threadIdx.x; i < 256; i += NT) hh[i] = 0u;
         __syncthreads();
-        for (int64_t i0 = lo_i; i0 < hi_i; i0 += NT) {
-          const int64_t i = i0 + threadIdx.x;
-          const bool act = i < hi_i;
-          const uint32_t k = act ? (cur ? __ldcg(cur + i) : f2key(__ldg(src + i))) : 0u;
-          hist_add(hh, (k >> shift) & 255u, act);
+        // kLd keys a thread, their loads issued before any is used (one
+        // block per SM: the loop would otherwise wait on every load)
+        constexpr int kLd = 8;
+        for (int64_t i0 = lo_i; i0 < hi_i; i0 += kLd * NT) {
+          uint32_t kk[kLd];
+#pragma unroll
+          for (int u = 0; u < kLd; ++u) {
+            const int64_t i = i0 + u * NT + threadIdx.x;
+            kk[u] = i < hi_i ? (cur ? __ldcg(cur + i) : f2key(__ldg(src + i))) : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < kLd; ++u) hist_add(hh, (kk[u] >> shift) & 255u, i0 + u * NT + threadIdx.x < hi_i);
         }
         __syncthreads();
         for (int d = threadIdx.x; d < 256; d += NT) cnts[(size_t)d * ncta + cta] = hh[d];
@@ -1431,8 +1446,19 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
         __syncthreads();
         for (int64_t t0 = lo_i; t0 < hi_i; t0 += kTile) {
           const int tn = (int)min((int64_t)kTile, hi_i - t0);
-          for (int i = threadIdx.x; i < tn; i += NT)
-            sbuf[i] = cur ? __ldcg(cur + t0 + i) : f2key(__ldg(src + t0 + i));
+          for (int i0 = 0; i0 < tn; i0 += kLd * NT) {
+            uint32_t kk[kLd];
+#pragma unroll
+            for (int u = 0; u < kLd; ++u) {
+              const int i = i0 + u * NT + (int)threadIdx.x;
+              kk[u] = i < tn ? (cur ? __ldcg(cur + t0 + i) : f2key(__ldg(src + t0 + i))) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < kLd; ++u) {
+              const int i = i0 + u * NT + (int)threadIdx.x;
+              if (i < tn) sbuf[i] = kk[u];
+            }
+          }
           __syncthreads();
           radix_pass<NT>(sbuf, stmp, tn, hist, shift, false);
           for (int q = threadIdx.x; q < tn; q += NT) {
