@@ -297,7 +297,9 @@ def e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step, n_s
     on three streams with two device buffer sets, as a user would pipeline
     them: step i+1's uploads overlap step i's downloads, the upload of g
     overlaps the forward, the download of p overlaps the backward.  The time
-    is from the first upload to the last download, divided by the steps."""
+    is from the first upload to the last download, divided by the steps (the
+    pipeline's fill and drain included, so more steps approach its steady
+    state)."""
     rows, n = x_h.shape
     s_up, s_cmp, s_dn = (torch.cuda.Stream(dev) for _ in range(3))
     sets = []
@@ -693,7 +695,7 @@ def main():
 
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step)
+        e2e = e2e_pipelined(lt, torch, w, x_h, g_h, dev, dist, world, scores_per_step, n_steps=max(args.steps, 8))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
