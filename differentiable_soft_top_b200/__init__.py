@@ -232,6 +232,10 @@ def _rows_view(t, name, *, copy_ok=False):
         if not copy_ok:
             raise ValueError(f"{name} must have unit stride along its rows")
         t2 = t2.contiguous()
+    if t2.shape[0] == 1 and t2.stride(0) != t2.shape[1]:
+        # one row (a numpy [None, :] view has row stride 0): its row stride
+        # is never used, so give it the dense one the C ABI checks
+        t2 = t2.as_strided(t2.shape, (max(1, t2.shape[1]), 1))
     return t2
 
 

@@ -198,36 +198,36 @@ __device__ void block_select2(const uint32_t* keys, int n, const int (&r)[2], ui
   __syncthreads();  // st may be reused by the caller
 }
 
-// Sorts keys[0, n) ascending with one bucket pass: 256 buckets over the key
-// range [kmin, kmax] (the caller's bounds of the keys), a histogram, a scan,
-// a scatter into tmp, then one thread sorts each bucket by insertion (equal
-// keys cost no moves).  About five barriers instead of a network's log2(N)^2/2
-// stages.  If any bucket holds more than kMaxBucket keys (a range stretched by
-// outliers), it returns null and nothing is sorted: the caller falls back to
-// a network.  tmp must hold n keys; scr >= 2 * 256 + 64 words.  Returns tmp
-// (sorted) on success.  All NT threads must call it.
+// Sorts keys[0, n) ascending with one bucket pass: NT buckets over the key
+// range [kmin, kmax] (the caller's bounds of the keys; NT a power of two >=
+// 256), a histogram, a scan, a scatter into tmp, then one thread sorts each
+// bucket by insertion (equal keys cost no moves).  About five barriers
+// instead of a network's log2(N)^2/2 stages.  If any bucket holds more than
+// kMaxBucket keys (a range stretched by outliers), it returns null and nothing
+// is sorted: the caller falls back to a network.  tmp must hold n keys, scr
+// bucket_sort_scr_words(NT) words.  Returns tmp (sorted) on success.  All NT
+// threads must call it.
 constexpr int kMaxBucket = 48;
+__host__ __device__ constexpr int bucket_sort_scr_words(int nt) { return 2 * nt + 64; }
 template <int NT>
 __device__ uint32_t* block_bucket_sort(const uint32_t* keys, uint32_t* tmp, int n, uint32_t kmin, uint32_t kmax,
                                        uint32_t* scr) {
-  static_assert(NT >= 256, "one thread per bucket");
-  uint32_t* cnt = scr;          // 256 counts, then cursors
-  uint32_t* start = scr + 256;  // 256 bucket starts
-  uint32_t* big = scr + 512;    // flag: a crowded bucket
+  static_assert(NT >= 256 && (NT & (NT - 1)) == 0, "one thread per bucket");
+  uint32_t* cnt = scr;          // NT counts, then cursors
+  uint32_t* start = scr + NT;   // NT bucket starts
+  uint32_t* big = scr + 2 * NT; // flag: a crowded bucket
   int shift = 0;
-  while (((kmax - kmin) >> shift) >= 256u) ++shift;
-  if (threadIdx.x < 256) cnt[threadIdx.x] = 0u;
+  while (((kmax - kmin) >> shift) >= (uint32_t)NT) ++shift;
+  cnt[threadIdx.x] = 0u;
   if (threadIdx.x == 0) *big = 0u;
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += NT) atomicAdd(&cnt[(keys[i] - kmin) >> shift], 1u);
   __syncthreads();
-  const uint32_t c = threadIdx.x < 256 ? cnt[threadIdx.x] : 0u;
-  const uint32_t st = block_excl_prefix_u32<NT>(c, scr + 520, nullptr);
-  if (threadIdx.x < 256) {
-    start[threadIdx.x] = st;
-    cnt[threadIdx.x] = st;  // cursor
-    if (c > (uint32_t)kMaxBucket) *big = 1u;
-  }
+  const uint32_t c = cnt[threadIdx.x];
+  const uint32_t st = block_excl_prefix_u32<NT>(c, scr + 2 * NT + 8, nullptr);
+  start[threadIdx.x] = st;
+  cnt[threadIdx.x] = st;  // cursor
+  if (c > (uint32_t)kMaxBucket) *big = 1u;
   __syncthreads();
   if (*big) return nullptr;  // uniform: read after the barrier
   for (int i = threadIdx.x; i < n; i += NT) {
@@ -235,7 +235,7 @@ __device__ uint32_t* block_bucket_sort(const uint32_t* keys, uint32_t* tmp, int 
     tmp[atomicAdd(&cnt[(k - kmin) >> shift], 1u)] = k;
   }
   __syncthreads();
-  if (threadIdx.x < 256) {
+  {
     const int lo = (int)start[threadIdx.x], hi = lo + (int)c;
     for (int i = lo + 1; i < hi; ++i) {
       const uint32_t k = tmp[i];

@@ -40,7 +40,7 @@ __host__ __device__ inline ResLayout res_layout(int64_t n, int m, int bcap, bool
   L.band_tmp = o; o = (o + 4 * (size_t)bcap + 15) & ~size_t(15);
   L.dscr = o;     o = (o + 8 * (size_t)bcap + 15) & ~size_t(15);
   L.dlink = o;    o = (o + 8 * (size_t)bcap + 8 + 15) & ~size_t(15);
-  L.sortscr = o;  o = o + 4 * 576;  // the band's bucket sort
+  L.sortscr = o;  o = o + 4 * (size_t)bucket_sort_scr_words(NT);  // the band's bucket sort
   L.red = o;      o = o + 8 * 64;
   L.mbar = o;     o = o + 16;
   L.total = o;

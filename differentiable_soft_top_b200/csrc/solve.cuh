@@ -333,7 +333,7 @@ __device__ void solve_values(const SolveIn in, const GroupPick& pk, int c, const
   __shared__ double s_bp;
   int* iscr = reinterpret_cast<int*>(red);
   const long long g_after = pk.g_after;
-  const int qe = (c + NT - 1) / NT;
+  const int qe = ((c + NT - 1) / NT) | 1;  // odd: a warp's chunk starts fall in distinct banks
   const int i0 = min(c, tid * qe), i1 = min(c, i0 + qe);
   const double xprev = (i0 > 0) ? (double)el.get(i0 - 1) : pk.inc_x;   // anchor before the chunk
   const double xnext = (i1 < c) ? (double)el.get(i1) : pk.out_x;       // anchor after the chunk
@@ -661,7 +661,9 @@ __device__ void solve_run(const SolveIn in, const uint32_t* keys, int M, double*
     s_edge[1] = A0;
   }
   __syncthreads();
-  const int qe = (M + NT - 1) / NT;
+  // contiguous chunks of an odd length: the threads of a warp, stepping
+  // through their chunks together, touch distinct shared-memory banks
+  const int qe = ((M + NT - 1) / NT) | 1;
   const int i0 = min(M, tid * qe), i1 = min(M, i0 + qe);
 
   // forward: chunk map, scan, A at every value

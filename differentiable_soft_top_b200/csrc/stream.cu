@@ -484,25 +484,54 @@ __device__ __noinline__ void flush_warp(const FilterCtx& f, const float* col, in
   }
 }
 
-__device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
-                             int ncta, double* red, float* stage) {
-  const int64_t n = P.n;
-  // the 16-byte aligned body in chunks of CHUNK4 float4 (after a head of 0-3
-  // scores); the scores outside it go through the scalar loop below
-  const int head = row_head(row, n);
-  const float4* x4 = reinterpret_cast<const float4*>(row + head);
-  const int64_t nchunks = ((n - head) >> 2) / CHUNK4;
-  // two chunks in flight per thread: the next chunk's loads are issued
-  // before the current one is processed.  The scores are the caller's, so
-  // the first chunk is requested before waiting for the kernel that wrote
-  // the bracket.
-  float4 nx[U];
-  if (cta < nchunks) {
-#pragma unroll
-    for (int u = 0; u < U; ++u) nx[u] = __ldg(x4 + (int64_t)cta * CHUNK4 + threadIdx.x + u * NT);
-  }
-  wait_prior_grid();
+// The running sums of one lane of the filter.
+struct FilterAcc {
+  long long nl = 0;
+  double sl = 0.0, sr = 0.0;
+  // sum of the scores scaled by 2^-64: finite for any finite scores (at most
+  // 2^40 of them), inf or NaN as soon as one score is
+  float2 fs2 = make_float2(0.0f, 0.0f);
+  int ncol = 0;  // values staged in this lane's column
+};
 
+// One lane's U float4 of a chunk (v): classification and tail terms two
+// scores at a time (packed fp32x2 arithmetic; the saturated side indicators
+// of classify): tail sums, the left count, and the positions of the scores
+// outside the band as bits of an exact fp32 sum.  The rare in-band values are
+// copied into the lane's column (stride NT) from at(i), the lane's i-th score
+// of the chunk (i = 4u + component).
+template <typename At>
+__device__ __forceinline__ void filter_chunk(const float4 (&v)[U], float2 naL2, float2 naR2, float2 c22,
+                                             const At& at, float* col, FilterAcc& a) {
+  const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
+  float2 pl2 = make_float2(0.0f, 0.0f), pr2 = pl2, cl2 = pl2, ob2 = pl2;
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float2 x2 = h ? make_float2(v[u].z, v[u].w) : make_float2(v[u].x, v[u].y);
+      const Side2 sd = classify2(x2, naL2, naR2, c22);
+      const float bit = (float)(1u << (4 * u + 2 * h));
+      pl2 = fma2(sd.L, sd.e, pl2);
+      pr2 = fma2(sd.R, sd.e, pr2);
+      cl2 = add2(cl2, sd.L);
+      ob2 = fma2(add2(sd.L, sd.R), make_float2(bit, 2.0f * bit), ob2);
+      a.fs2 = fma2(x2, k64, a.fs2);
+    }
+  }
+  a.sl += (double)(pl2.x + pl2.y);
+  a.sr += (double)(pr2.x + pr2.y);
+  a.nl += (long long)(cl2.x + cl2.y);
+  uint32_t mask = ~(uint32_t)(ob2.x + ob2.y) & ((1u << (4 * U)) - 1u);  // in-band positions
+  while (mask) {  // rare
+    const int i = __ffs(mask) - 1;
+    mask &= mask - 1u;
+    col[a.ncol * NT] = at(i);
+    ++a.ncol;
+  }
+}
+
+__device__ __forceinline__ FilterCtx filter_ctx(const StreamPlan& P, int64_t r, RowCtl* c) {
   FilterCtx f;
   f.aL = vld(&c->aL);
   f.aR = vld(&c->aR);
@@ -512,107 +541,43 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   f.nkmin = &c->band_nkmin;
   f.band = band_of(P, r);
   f.cap = (uint32_t)P.band_cap;
-  const float aL = f.aL, aR = f.aR, c2 = f.c2;
-  float* col = stage + threadIdx.x;                             // this lane's column, stride NT
-  float4* scratch = reinterpret_cast<float4*>(stage + kLaneStage * NT) + threadIdx.x * U;  // U float4
-  int ncol = 0;
-  long long nl = 0;
-  double sl = 0.0, sr = 0.0;
-  uint32_t bad = 0u, ovf = 0u;
-  // sum of the scores scaled by 2^-64: finite for any finite scores (at most
-  // 2^40 of them), inf or NaN as soon as one score is
-  float fsum = 0.0f;
-  float2 fs2 = make_float2(0.0f, 0.0f);
-  const float2 naL2 = make_float2(-aL, -aL), naR2 = make_float2(-aR, -aR), c22 = make_float2(c2, c2);
-  const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
+  return f;
+}
 
-  int64_t nb4 = 0;
-  {
-    for (int64_t q = cta; q < nchunks; q += ncta) {
-      const float4* base = x4 + q * CHUNK4 + threadIdx.x;
-      // the chunk after the next one into L2 (its loads into registers are
-      // issued next iteration): more bytes in flight than registers hold
-      if (threadIdx.x == 0 && q + 2 * ncta < nchunks)
-        bulk_prefetch_l2(x4 + (q + 2 * ncta) * CHUNK4, CHUNK4 * 16u);
-      float4 v[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) v[u] = nx[u];
-      if (q + ncta < nchunks) {
-#pragma unroll
-        for (int u = 0; u < U; ++u) nx[u] = __ldg(base + (int64_t)ncta * CHUNK4 + u * NT);
-      }
-      // classification and tail terms two scores at a time (packed fp32x2
-      // arithmetic; the saturated side indicators of classify): tail sums,
-      // the left count, and the positions of the scores outside the band as
-      // bits of an exact fp32 sum
-      float2 pl2 = make_float2(0.0f, 0.0f), pr2 = pl2, cl2 = pl2, ob2 = pl2;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float2 x2 = h ? make_float2(v[u].z, v[u].w) : make_float2(v[u].x, v[u].y);
-          const Side2 sd = classify2(x2, naL2, naR2, c22);
-          const float bit = (float)(1u << (4 * u + 2 * h));
-          pl2 = fma2(sd.L, sd.e, pl2);
-          pr2 = fma2(sd.R, sd.e, pr2);
-          cl2 = add2(cl2, sd.L);
-          ob2 = fma2(add2(sd.L, sd.R), make_float2(bit, 2.0f * bit), ob2);
-          fs2 = fma2(x2, k64, fs2);
-        }
-      }
-      sl += (double)(pl2.x + pl2.y);
-      sr += (double)(pr2.x + pr2.y);
-      nl += (long long)(cl2.x + cl2.y);
-      uint32_t mask = ~(uint32_t)(ob2.x + ob2.y) & ((1u << (4 * U)) - 1u);  // in-band positions
-      if (mask) {  // rare: copy this lane's in-band values into its column
-#pragma unroll
-        for (int u = 0; u < U; ++u) scratch[u] = v[u];
-        const float* sv = reinterpret_cast<const float*>(scratch);
-        do {
-          const int i = __ffs(mask) - 1;
-          mask &= mask - 1u;
-          col[ncol * NT] = sv[i];
-          ++ncol;
-        } while (mask);
-      }
-      if (__any_sync(0xffffffffu, ncol > kLaneStage - 4 * U)) {
-        flush_warp(f, col, ncol, bad, ovf);
-        ncol = 0;
-      }
-    }
-    nb4 = nchunks * CHUNK4;
-    fsum = fs2.x + fs2.y;
-  }
-  // the rest: one score per thread per step, the same trip count for the
-  // whole block
-  const int64_t nrest = n - 4 * nb4;
+// The scores outside the float4 body (one per thread per step, the same trip
+// count for the whole block), the last flush, and the block's partial sums.
+__device__ void filter_finish(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
+                              int ncta, double* red, float* col, const FilterCtx& f, FilterAcc& a, int head,
+                              int64_t nb4, uint32_t bad, uint32_t ovf) {
+  float fsum = a.fs2.x + a.fs2.y;
+  const int64_t nrest = P.n - 4 * nb4;
   for (int64_t j0 = (int64_t)cta * NT; j0 < nrest; j0 += (int64_t)ncta * NT) {
     const int64_t j = j0 + threadIdx.x;
     if (j < nrest) {
       const float x = row[rest_index(j, head, nb4)];
-      const Side sd = classify(x, aL, aR, c2);
+      const Side sd = classify(x, f.aL, f.aR, f.c2);
       if (sd.L != 0.0f) {
-        sl += (double)sd.e;
-        ++nl;
+        a.sl += (double)sd.e;
+        ++a.nl;
       }
-      if (sd.R != 0.0f) sr += (double)sd.e;
+      if (sd.R != 0.0f) a.sr += (double)sd.e;
       fsum = fmaf(x, 0x1p-64f, fsum);
       if (sd.L + sd.R == 0.0f) {
-        col[ncol * NT] = x;
-        ++ncol;
+        col[a.ncol * NT] = x;
+        ++a.ncol;
       }
     }
-    if (__any_sync(0xffffffffu, ncol >= kLaneStage)) {
-      flush_warp(f, col, ncol, bad, ovf);
-      ncol = 0;
+    if (__any_sync(0xffffffffu, a.ncol >= kLaneStage)) {
+      flush_warp(f, col, a.ncol, bad, ovf);
+      a.ncol = 0;
     }
   }
-  if (__any_sync(0xffffffffu, ncol > 0)) flush_warp(f, col, ncol, bad, ovf);
+  if (__any_sync(0xffffffffu, a.ncol > 0)) flush_warp(f, col, a.ncol, bad, ovf);
   if (!(fabsf(fsum) < CUDART_INF_F)) bad = 1u;
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
-  nl = block_sum<NT, long long>(nl, reinterpret_cast<long long*>(red));
-  sl = block_sum<NT, double>(sl, red);
-  sr = block_sum<NT, double>(sr, red);
+  const long long nl = block_sum<NT, long long>(a.nl, reinterpret_cast<long long*>(red));
+  const double sl = block_sum<NT, double>(a.sl, red);
+  const double sr = block_sum<NT, double>(a.sr, red);
   bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
   if (threadIdx.x == 0) {
     FPart p;
@@ -626,14 +591,150 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   __syncthreads();
 }
 
-// shared memory of the filter pass: lane columns plus one scratch chunk per lane
+// The filter pass of the recovery kernel (a re-filter after a widening):
+// chunks loaded straight into registers, two in flight per thread (the next
+// chunk's loads are issued before the current one is processed).  stage:
+// the lane columns, then one scratch chunk per lane.
+__device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
+                             int ncta, double* red, float* stage) {
+  const int64_t n = P.n;
+  // the 16-byte aligned body in chunks of CHUNK4 float4 (after a head of 0-3
+  // scores); the scores outside it go through filter_finish
+  const int head = row_head(row, n);
+  const float4* x4 = reinterpret_cast<const float4*>(row + head);
+  const int64_t nchunks = ((n - head) >> 2) / CHUNK4;
+  float4 nx[U];
+  if (cta < nchunks) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) nx[u] = __ldg(x4 + (int64_t)cta * CHUNK4 + threadIdx.x + u * NT);
+  }
+  const FilterCtx f = filter_ctx(P, r, c);
+  float* col = stage + threadIdx.x;  // this lane's column, stride NT
+  float4* scratch = reinterpret_cast<float4*>(stage + kLaneStage * NT) + threadIdx.x * U;  // U float4
+  const float2 naL2 = make_float2(-f.aL, -f.aL), naR2 = make_float2(-f.aR, -f.aR), c22 = make_float2(f.c2, f.c2);
+  FilterAcc acc;
+  uint32_t bad = 0u, ovf = 0u;
+  for (int64_t q = cta; q < nchunks; q += ncta) {
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = nx[u];
+    if (q + ncta < nchunks) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) nx[u] = __ldg(x4 + (q + ncta) * CHUNK4 + threadIdx.x + u * NT);
+    }
+    // the lane's chunk goes to its scratch slot only when it holds in-band
+    // values (read back there by position)
+    bool spilled = false;
+    filter_chunk(v, naL2, naR2, c22,
+                 [&](int i) {
+                   if (!spilled) {
+#pragma unroll
+                     for (int u = 0; u < U; ++u) scratch[u] = v[u];
+                     spilled = true;
+                   }
+                   return reinterpret_cast<const float*>(scratch)[i];
+                 },
+                 col, acc);
+    if (__any_sync(0xffffffffu, acc.ncol > kLaneStage - 4 * U)) {
+      flush_warp(f, col, acc.ncol, bad, ovf);
+      acc.ncol = 0;
+    }
+  }
+  filter_finish(P, r, row, c, cta, ncta, red, col, f, acc, head, nchunks * CHUNK4, bad, ovf);
+}
+
+// shared memory of the recovery kernel's filter pass: lane columns plus one
+// scratch chunk per lane
 constexpr size_t kFilterStageBytes = (size_t)(kLaneStage * NT) * 4 + (size_t)NT * U * 16;
 
-__global__ void __launch_bounds__(NT, 4) k_filter(const StreamPlan P, const float* __restrict__ scores) {
-  __shared__ double red[64];
-  __shared__ __align__(16) float stage[kFilterStageBytes / 4];
-  const int64_t r = blockIdx.y;  // filter_phase waits for the bracket's kernel
-  filter_phase(P, r, scores + r * P.stride, ctl_of(P, r), blockIdx.x, gridDim.x, red, stage);
+// The filter kernel: the chunks of a block reach shared memory through bulk
+// copies (the Tensor Memory Accelerator) into a ring of kFilterRing stages,
+// issued by one thread, kFilterRing - 1 chunks ahead of the one being
+// classified: the bytes in flight per SM are the ring's, not what the
+// threads' registers can hold.  A stage is refilled once the whole block has
+// classified it (one barrier per chunk); the rare in-band values are copied
+// from the stage by position before that.
+constexpr int kFilterRing = 4;
+constexpr uint32_t kChunkBytes = CHUNK4 * 16u;
+struct FilterSmem {
+  float4 ring[kFilterRing][CHUNK4];
+  float stage[kLaneStage * NT];  // the lane columns
+  double red[64];
+  uint64_t full[kFilterRing];
+};
+constexpr size_t kFilterSmemBytes = sizeof(FilterSmem);
+
+__global__ void __launch_bounds__(NT, 2) k_filter(const StreamPlan P, const float* __restrict__ scores) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  FilterSmem& S = *reinterpret_cast<FilterSmem*>(smem_raw);
+  const int64_t r = blockIdx.y;
+  const int cta = blockIdx.x, ncta = gridDim.x;
+  const float* row = scores + r * P.stride;
+  RowCtl* c = ctl_of(P, r);
+  const int head = row_head(row, P.n);
+  const float4* x4 = reinterpret_cast<const float4*>(row + head);
+  const int64_t nchunks = ((P.n - head) >> 2) / CHUNK4;
+  const int mine = cta < nchunks ? (int)((nchunks - 1 - cta) / ncta) + 1 : 0;  // this block's chunks
+  // test knob: rows 1, 5, 9, ... issue no copy for their first chunk, so
+  // that its bounded wait runs out (rows 3, 7, ... time out in the recovery
+  // kernel instead)
+  const bool force_to = P.force_timeout && !P.shard && (r & 3) == 1;
+  // the scores are the caller's: the first stages are requested before
+  // waiting for the kernel that wrote the bracket
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFilterRing; ++s) mbar_init(&S.full[s], 1u);
+    for (int s = force_to ? 1 : 0; s < kFilterRing && s < mine; ++s) {
+      mbar_arrive_expect_tx(&S.full[s], kChunkBytes);
+      bulk_load(S.ring[s], x4 + (cta + (int64_t)s * ncta) * CHUNK4, kChunkBytes, &S.full[s]);
+    }
+  }
+  __syncthreads();
+  wait_prior_grid();
+  const FilterCtx f = filter_ctx(P, r, c);
+  float* col = S.stage + threadIdx.x;
+  const float2 naL2 = make_float2(-f.aL, -f.aL), naR2 = make_float2(-f.aR, -f.aR), c22 = make_float2(f.c2, f.c2);
+  const uint32_t limit = spin_limit_of(P.spin_limit);
+  FilterAcc acc;
+  uint32_t bad = 0u, ovf = 0u;
+  int it = 0;
+  bool late = false;
+  for (; it < mine; ++it) {
+    const int slot = it % kFilterRing;
+    const bool ok = mbar_wait_bounded(&S.full[slot], (uint32_t)(it / kFilterRing) & 1u, limit);
+    const float4* st = S.ring[slot] + threadIdx.x;
+    float4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) v[u] = st[u * NT];
+    filter_chunk(v, naL2, naR2, c22, [&](int i) { return reinterpret_cast<const float*>(st + (i >> 2) * NT)[i & 3]; },
+                 col, acc);
+    // every thread is done with the stage: refill it
+    if (!__syncthreads_and(ok)) {
+      late = true;  // a copy that did not complete in time: the row's results are void
+      break;
+    }
+    if (threadIdx.x == 0 && it + kFilterRing < mine) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&S.full[slot], kChunkBytes);
+      bulk_load(S.ring[slot], x4 + (cta + (int64_t)(it + kFilterRing) * ncta) * CHUNK4, kChunkBytes,
+                &S.full[slot]);
+    }
+    if (__any_sync(0xffffffffu, acc.ncol > kLaneStage - 4 * U)) {
+      flush_warp(f, col, acc.ncol, bad, ovf);
+      acc.ncol = 0;
+    }
+  }
+  if (late) {
+    // chunks it .. it + kFilterRing - 1 may still be in flight: let them land
+    // (again with a limit) before the block leaves; the band kernel reads
+    // the flag and solves nothing
+    if (threadIdx.x == 0) {
+      for (int j = it; j < mine && j < it + kFilterRing; ++j)
+        (void)mbar_wait_bounded(&S.full[j % kFilterRing], (uint32_t)(j / kFilterRing) & 1u, limit);
+      atomicOr(&c->flags, ROW_TIMEOUT);
+    }
+    __syncthreads();
+  }
+  filter_finish(P, r, row, c, cta, ncta, S.red, col, f, acc, head, nchunks * CHUNK4, bad, ovf);
 }
 
 // ===========================================================================
@@ -709,7 +810,7 @@ struct BinPart {  // one CTA's bins
 struct TargetBuf {
   uint32_t keys[kTargetCap];
   uint32_t sorted[kTargetCap];  // the bucket sort's output
-  uint32_t scr[576];            // and its scratch
+  uint32_t scr[bucket_sort_scr_words(kBandThreads)];  // and its scratch
 };
 enum : int { kBandDone = 0, kBandRefine = 1, kBandExtract = 2 };
 struct BandDecision {
@@ -735,6 +836,11 @@ struct BandShared {
   BandDecision dec;
 };
 constexpr size_t kBandSmemBytes = sizeof(BandShared);
+// A lone band CTA sorts a band of at most kRunCap values whole (keys, the
+// sort's output, then the prefix states and link factors of the one run, in
+// the stage area) and solves it without key bins.
+constexpr int kRunCap = 4096;
+static_assert((size_t)kRunCap * (4 + 4 + 8 + 8) + 8 <= sizeof(float) * kStageCap, "run fits the stage");
 
 template <typename T>
 __device__ __forceinline__ T* at_rank(T* p, int q, int cs) {
@@ -996,8 +1102,11 @@ __device__ void merge_bins(BandShared& S, int cs, int rank, uint32_t klo, uint32
 
 // Solves row r from its filter partials and band.  cs CTAs of one cluster
 // (rank = the CTA's rank in it) or, with cs == 1, one block alone; nparts:
-// filter partials of the row.  Every thread of every CTA calls it.
-template <int NTX>
+// filter partials of the row.  kRun: a lone CTA solves a band of at most
+// kRunCap values as one sorted run instead of binning it (a separate
+// instantiation, so that the cluster's bin path keeps its registers).  Every
+// thread of every CTA calls it.
+template <int NTX, bool kRun>
 __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned char* smem, int nparts, int cs,
                            int rank) {
   BandShared& S = *reinterpret_cast<BandShared*>(smem);
@@ -1030,7 +1139,9 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
   double b = 0.0, sumf = 0.0;
   int levels = 0;
 
-  if (bad) {
+  if (flags & ROW_TIMEOUT) {
+    st |= ROW_TIMEOUT;  // a filter block gave up waiting for its copies
+  } else if (bad) {
     st |= ROW_NONFINITE;
   } else if ((flags & ROW_OVERFLOW) || (int64_t)mt > P.band_cap) {
     st |= ROW_OVERFLOW;
@@ -1048,7 +1159,26 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
     int shift = bin_shift(klo, khi);
     if (leader && threadIdx.x == 0) S.in = SolveIn{vld(&c->aL), vld(&c->aR), nl, nr, sl, sr, ra.k, ra.alpha, inva};
     int action = kBandDone;
-    for (int level = 0; level < kMaxLevels; ++level) {
+    bool run = false;
+    if constexpr (kRun) {
+      if (cs == 1 && M > 0 && M <= kRunCap) {
+        // the whole band as one sorted run; a key range too stretched for
+        // the bucket pass leaves it to the bins.  [klo, khi] are the exact
+        // extremes of the appended keys.
+        uint32_t* keys = reinterpret_cast<uint32_t*>(S.tu.stage);
+        uint32_t* tmp = keys + kRunCap;
+        double* dA = reinterpret_cast<double*>(tmp + kRunCap);
+        double* dL = dA + kRunCap;
+        for (int i = threadIdx.x; i < n; i += NTX) keys[i] = f2key(__ldcg(src + i));
+        __syncthreads();
+        const uint32_t* sorted = block_bucket_sort<NTX>(keys, tmp, n, klo, khi, S.u.tgt.scr);
+        if (sorted) {
+          solve_run<NTX>(S.in, sorted, n, dA, dL, red, &S.so);
+          run = true;
+        }
+      }
+    }
+    for (int level = 0; level < kMaxLevels && !run; ++level) {
       levels = level + 1;
       // a worker keeps its slice in shared memory; a lone CTA (cs == 1) holds
       // the table in the same place, so it rereads its slice from L2 past level 0
@@ -1216,21 +1346,25 @@ __device__ void band_solve(const StreamPlan& P, int64_t r, RowCtl* c, unsigned c
     c->b = b;
     c->bins = kBins * levels;
     // test knob: odd rows go to the recovery kernel, whose barrier runs out
-    if (P.force_timeout && !P.shard && (r & 1) && !(st & ROW_NONFINITE)) st |= ROW_FORCE_TO;
+    if (P.force_timeout && !P.shard && (r & 1) && !(st & (ROW_NONFINITE | ROW_TIMEOUT))) st |= ROW_FORCE_TO;
     c->status = st;
     __threadfence();
   }
   cl_sync(cs);  // no CTA leaves while another may still read its shared memory
 }
 
+template <bool kRun>
 __global__ void __launch_bounds__(kBandThreads, 1) k_band(const StreamPlan P) {
   extern __shared__ __align__(16) unsigned char smem[];
   wait_prior_grid();
   const int64_t r = blockIdx.y;
   const int cs = (int)cg::this_cluster().num_blocks();
   const int rank = (int)cg::this_cluster().block_rank();
-  band_solve<kBandThreads>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank);
+  band_solve<kBandThreads, kRun>(P, r, ctl_of(P, r), smem, P.Gf, cs, rank);
 }
+// a lone band CTA may solve its band as one run; a cluster bins it
+using BandKernel = void (*)(const StreamPlan);
+BandKernel band_kernel(int cs) { return cs == 1 ? k_band<true> : k_band<false>; }
 
 // ===========================================================================
 // recovery: one widening, then the full-sort fallback (cooperative launch)
@@ -1374,7 +1508,7 @@ __global__ void __launch_bounds__(NT) k_recover(const StreamPlan P, const float*
       filter_phase(P, r, scores + r * P.stride, c, cta, ncta, red, reinterpret_cast<float*>(kbuf));
       REC_BARRIER();
       if (cta == 0) {
-        band_solve<NT>(P, r, c, smem, ncta, 1, 0);
+        band_solve<NT, false>(P, r, c, smem, ncta, 1, 0);
         if (threadIdx.x == 0) {
           c->status |= ROW_WIDENED;
           __threadfence();
@@ -2025,14 +2159,19 @@ __global__ void __launch_bounds__(NT) k_shard_compact(const StreamPlan Pb, int w
 }  // namespace
 
 cudaError_t stream_occupancy(StreamOcc* out) {
-  cudaError_t e = cudaFuncSetAttribute(k_band, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBandSmemBytes);
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_band, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaSuccess;
+  for (BandKernel kb : {k_band<false>, k_band<true>}) {
+    e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBandSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kb, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  e = cudaFuncSetAttribute(k_filter, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFilterSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_recover, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RecSmem::kTotal);
   if (e != cudaSuccess) return e;
   int fb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, 0);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, kFilterSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb<false, false>, NT, 0);
   if (e != cudaSuccess) return e;
@@ -2066,7 +2205,7 @@ cudaError_t stream_occupancy(StreamOcc* out) {
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int nc = 0;
-    if (cudaOccupancyMaxActiveClusters(&nc, k_band, &cfg) == cudaSuccess && nc >= 1) {
+    if (cudaOccupancyMaxActiveClusters(&nc, k_band<false>, &cfg) == cudaSuccess && nc >= 1) {
       out->band_max_cluster = cs;
       break;
     }
@@ -2104,7 +2243,7 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
   }
   {
     Launch l("k_filter", st);
-    e = launch_pdl(k_filter, dim3(P.Gf, rows), dim3(NT), 0, st, P, scores);
+    e = launch_pdl(k_filter, dim3(P.Gf, rows), dim3(NT), kFilterSmemBytes, st, P, scores);
     if (e != cudaSuccess) return e;
   }
   {
@@ -2123,7 +2262,7 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
     cfg.attrs = at;
     cfg.numAttrs = 2;
     Launch l("k_band", st);
-    e = cudaLaunchKernelEx(&cfg, k_band, P);
+    e = cudaLaunchKernelEx(&cfg, band_kernel(P.band_cs), P);
     if (e != cudaSuccess) return e;
   }
   {
@@ -2198,7 +2337,7 @@ cudaError_t launch_shard_filter(const StreamPlan& P, const float* scores, uint32
   }
   {
     Launch l("k_filter", st);
-    k_filter<<<dim3(P.Gf, rows), NT, 0, st>>>(P, scores);
+    k_filter<<<dim3(P.Gf, rows), NT, kFilterSmemBytes, st>>>(P, scores);
   }
   {
     Launch l("k_shard_pack", st);
@@ -2234,7 +2373,7 @@ cudaError_t launch_shard_finish(const StreamPlan& P, const StreamPlan& Pb, const
     cfg.attrs = at;
     cfg.numAttrs = 1;
     Launch l("k_band", st);
-    e = cudaLaunchKernelEx(&cfg, k_band, Pb);
+    e = cudaLaunchKernelEx(&cfg, band_kernel(Pb.band_cs), Pb);
     if (e != cudaSuccess) return e;
   }
   // no recovery here: a row the band does not certify keeps its miss bits and

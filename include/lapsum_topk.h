@@ -107,11 +107,15 @@ typedef struct lapsum_params {
  * (pair it with a small spin_limit).  A one-block row that is copied into
  * shared memory (n <= 4096) waits on a bulk-copy barrier that no copy
  * targets (when scores and p start at the same address mod 16, as the copy
- * needs); a streaming row is sent to the recovery kernel, whose first grid
- * barrier then waits for one block more than the grid holds.  Such a row
- * ends with LAPSUM_ROW_TIMEOUT and NaN outputs (p, b, sum f); on the
- * streaming path every later row that needs the recovery kernel in that call
- * ends the same way, since the kernel stops at its first timed-out barrier.
+ * needs).  On a streaming row numbered 1 mod 4 every filter block issues no
+ * bulk copy for its first chunk and its barrier wait for that chunk runs out
+ * (the block first waits, bounded, for its other copies in flight); any
+ * other odd streaming row (or one with no whole chunk of 4096 scores) is
+ * sent to the recovery kernel, whose first grid barrier then waits for one
+ * block more than the grid holds.  Such a row ends with LAPSUM_ROW_TIMEOUT
+ * and NaN outputs (p, b, sum f); on the streaming path every later row that
+ * needs the recovery kernel in that call ends the same way, since the kernel
+ * stops at its first timed-out barrier.
  * Even-numbered rows are solved as usual, and the next call starts afresh.
  * Nothing waits forever and no fault is raised.  Rows of 4097..16384 scores
  * on the one-block path have no such wait and are not affected. */
@@ -131,8 +135,9 @@ typedef struct lapsum_row_stats {
     double sum_p;            /* sum of the written p, accumulated in fp64 */
     double sum_f;            /* sum_i f_i */
     int32_t sample_m;        /* sample size used */
-    int32_t buckets;         /* band key bins used (all levels), or groups
-                                of the full-sort fallback */
+    int32_t buckets;         /* band key bins used (all levels; 0 when the
+                                band was sorted whole), or groups of the
+                                full-sort fallback */
     uint32_t status;         /* same bits as row_status */
     int32_t reserved;
 } lapsum_row_stats;

@@ -155,6 +155,22 @@ def test_strided_unaligned_rows(orc, n, force):
                   k, alpha, f"strided row {i}")
 
 
+@pytest.mark.parametrize("n", [3000, 70001])
+def test_one_row_with_any_row_stride(orc, n):
+    # a single row whose row stride is 0 (numpy's [None, :] view) or short
+    x = make_scores("normal", 1, n, seed=9)
+    g = make_grad(1, n, seed=10)
+    k, alpha = 77.0, 0.1
+    dense = gpu_run(x, g, k, alpha)
+    for s0 in (0, 1):
+        xt = torch.from_numpy(x).cuda().as_strided((1, n), (s0, 1))
+        gt = torch.from_numpy(g).cuda().as_strided((1, n), (s0, 1))
+        res = lt.forward(xt, k, alpha)
+        grad, gk = lt.backward(xt, gt, res.b, alpha)
+        assert np.array_equal(res.p.cpu().numpy(), dense["p"]) and np.array_equal(grad.cpu().numpy(), dense["grad"])
+    check_row(orc, x[0], g[0], dense["p"], dense["grad"], dense["b"][0], dense["gk"][0], k, alpha, f"one row n={n}")
+
+
 @pytest.mark.parametrize("n,force", [(3000, lt.FORCE_NONE), (12001, lt.FORCE_NONE), (70001, lt.FORCE_NONE)])
 def test_outputs_off_the_scores_phase(orc, n, force):
     # p and grad given by the caller 4 bytes further along the 16-byte grid
@@ -371,6 +387,24 @@ def test_deterministic_with_a_band_cluster():
         assert np.array_equal(runs[0]["p"], r["p"]) and np.array_equal(runs[0]["grad"], r["grad"])
     res = lt.forward(torch.from_numpy(x).cuda(), k, alpha, stats=True)
     assert int(res.stats[0]["band"]) > 2 * 16384  # more than one CTA of the cluster bins it
+
+
+def test_small_band_sorted_whole_or_binned(orc):
+    """A lone band CTA sorts a band of at most 4096 values whole and solves
+    it as one run (no key bins); a band whose ties crowd one bucket of the
+    bucket pass is binned instead.  Both give the oracle's result."""
+    n, k, alpha = 200_000, 2000.0, 0.05
+    rng = np.random.default_rng(11)
+    smooth = rng.standard_normal((1, n)).astype(np.float32)
+    tied = (np.round(smooth.astype(np.float64) * 64) / 64).astype(np.float32)  # ~80 ties a level at b
+    g = rng.standard_normal((1, n)).astype(np.float32)
+    for x, run in ((smooth, True), (tied, False)):
+        out = gpu_run(x, g, k, alpha, stats=True)
+        st = out["stats"][0]
+        assert 0 < int(st["band"]) <= 4096
+        assert (int(st["buckets"]) == 0) == run, f"buckets {int(st['buckets'])}, band {int(st['band'])}"
+        assert out["status"][0] & lt.ROW_CERTIFIED
+        check_row(orc, x[0], g[0], out["p"], out["grad"], out["b"][0], out["gk"][0], k, alpha, f"run={run}")
 
 
 def test_autograd_wrapper(orc):

@@ -1,14 +1,16 @@
 """Bounded device waits that run out (failure detection without a GPU fault).
 
 Every wait in the library's kernels -- the bulk-copy barrier of a one-block
-row copied into shared memory, the grid barrier of the cooperative recovery
-kernel -- gives up after a fixed number of polls, marks the row
+row copied into shared memory, the barriers of the filter's ring of bulk
+copies, the grid barrier of the cooperative recovery kernel -- gives up
+after a fixed number of polls, marks the row
 LAPSUM_ROW_TIMEOUT and returns (the pages' solver widens its bracket and falls
 back to a full sort, technical summary section 2.2 step 4; a wait that never
 ends would hang the GPU instead).  The LAPSUM_FORCE_TIMEOUT test knob makes
 the wait of every odd-numbered row run out: the one-block row waits on a
-barrier that no copy targets, the streaming row's recovery barrier waits for
-one block more than the grid holds.  Nothing faults or waits for good; a short
+barrier that no copy targets, so does each filter block of a streaming row
+numbered 1 mod 4 (for its first chunk), and the recovery barrier of a
+streaming row numbered 3 mod 4 waits for one block more than the grid holds.  Nothing faults or waits for good; a short
 spin_limit keeps each wait to a fraction of a millisecond.
 
 Checked: the forced rows report the timeout and carry NaN outputs, the other
@@ -62,18 +64,21 @@ def test_forced_waits_time_out_and_the_rest_is_solved(orc, n, force, rows):
 
 
 def test_timeout_with_the_fallback_forced_on_every_row(orc):
-    """FORCE_FALLBACK sends every row to the recovery kernel: the even rows'
-    full sorts run first and are certified, the first odd row's barrier runs
-    out, and the rows after it that still need recovery are marked too."""
-    rows, n = 4, 50_001
+    """FORCE_FALLBACK sends every row to the recovery kernel, except row 1,
+    whose filter wait already ran out (a row that timed out is not
+    recovered).  The full sorts of rows 0 and 2 run first and are certified,
+    row 3's barrier runs out, and the rows after it that still need recovery
+    are marked too (row 4, an even row); row 5 times out in its filter."""
+    rows, n = 6, 50_001
     x = make_scores("mixture", rows, n, seed=5)
     g = make_grad(rows, n, seed=6)
     k, alpha = 200.0, 0.05
     params = lt.Params(force_path=lt.FORCE_FALLBACK | lt.FORCE_TIMEOUT, spin_limit=2000)
     out = gpu_run(x, g, k, alpha, params=params)
     st = out["status"].astype(np.uint32)
-    assert st[0] & lt.ROW_FALLBACK and st[0] & lt.ROW_CERTIFIED
-    check_row(orc, x[0], g[0], out["p"][0], out["grad"][0], out["b"][0], out["gk"][0], k, alpha, "row 0")
-    for i in range(1, rows):
+    for i in (0, 2):
+        assert st[i] & lt.ROW_FALLBACK and st[i] & lt.ROW_CERTIFIED, f"row {i} status {st[i]:#x}"
+        check_row(orc, x[i], g[i], out["p"][i], out["grad"][i], out["b"][i], out["gk"][i], k, alpha, f"row {i}")
+    for i in (1, 3, 4, 5):
         assert st[i] & lt.ROW_TIMEOUT and not (st[i] & lt.ROW_CERTIFIED), f"row {i} status {st[i]:#x}"
         assert np.isnan(out["p"][i]).all() and np.isnan(out["b"][i])
