@@ -546,11 +546,13 @@ __device__ __forceinline__ FilterCtx filter_ctx(const StreamPlan& P, int64_t r, 
 
 // The scores outside the float4 body (one per thread per step, the same trip
 // count for the whole block), the last flush, and the block's partial sums.
+// NTB: the block's threads; the first NT of them take the tail.
+template <int NTB>
 __device__ void filter_finish(const StreamPlan& P, int64_t r, const float* __restrict__ row, RowCtl* c, int cta,
                               int ncta, double* red, float* col, const FilterCtx& f, FilterAcc& a, int head,
                               int64_t nb4, uint32_t bad, uint32_t ovf) {
   float fsum = a.fs2.x + a.fs2.y;
-  const int64_t nrest = P.n - 4 * nb4;
+  const int64_t nrest = threadIdx.x < NT ? P.n - 4 * nb4 : 0;
   for (int64_t j0 = (int64_t)cta * NT; j0 < nrest; j0 += (int64_t)ncta * NT) {
     const int64_t j = j0 + threadIdx.x;
     if (j < nrest) {
@@ -572,13 +574,13 @@ __device__ void filter_finish(const StreamPlan& P, int64_t r, const float* __res
       a.ncol = 0;
     }
   }
-  if (__any_sync(0xffffffffu, a.ncol > 0)) flush_warp(f, col, a.ncol, bad, ovf);
+  if (threadIdx.x < NT && __any_sync(0xffffffffu, a.ncol > 0)) flush_warp(f, col, a.ncol, bad, ovf);
   if (!(fabsf(fsum) < CUDART_INF_F)) bad = 1u;
   if (ovf) atomicOr(&c->flags, ROW_OVERFLOW);
-  const long long nl = block_sum<NT, long long>(a.nl, reinterpret_cast<long long*>(red));
-  const double sl = block_sum<NT, double>(a.sl, red);
-  const double sr = block_sum<NT, double>(a.sr, red);
-  bad = block_or<NT>(bad, reinterpret_cast<uint32_t*>(red));
+  const long long nl = block_sum<NTB, long long>(a.nl, reinterpret_cast<long long*>(red));
+  const double sl = block_sum<NTB, double>(a.sl, red);
+  const double sr = block_sum<NTB, double>(a.sr, red);
+  bad = block_or<NTB>(bad, reinterpret_cast<uint32_t*>(red));
   if (threadIdx.x == 0) {
     FPart p;
     p.nL = nl;
@@ -640,7 +642,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
       acc.ncol = 0;
     }
   }
-  filter_finish(P, r, row, c, cta, ncta, red, col, f, acc, head, nchunks * CHUNK4, bad, ovf);
+  filter_finish<NT>(P, r, row, c, cta, ncta, red, col, f, acc, head, nchunks * CHUNK4, bad, ovf);
 }
 
 // shared memory of the recovery kernel's filter pass: lane columns plus one
@@ -648,93 +650,119 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
 constexpr size_t kFilterStageBytes = (size_t)(kLaneStage * NT) * 4 + (size_t)NT * U * 16;
 
 // The filter kernel: the chunks of a block reach shared memory through bulk
-// copies (the Tensor Memory Accelerator) into a ring of kFilterRing stages,
-// issued by one thread, kFilterRing - 1 chunks ahead of the one being
-// classified: the bytes in flight per SM are the ring's, not what the
-// threads' registers can hold.  A stage is refilled once the whole block has
-// classified it (one barrier per chunk); the rare in-band values are copied
-// from the stage by position before that.
+// copies (the Tensor Memory Accelerator) into a ring of kFilterRing stages.
+// One producer warp (one lane of it) issues them, up to kFilterRing chunks
+// ahead: the bytes in flight per SM are the ring's, not what registers can
+// hold.  Eight consumer warps classify each chunk as it lands (full barrier of
+// its stage) and release the stage (empty barrier, one arrival per warp)
+// once they have copied out its rare in-band values; no block-wide barrier
+// per chunk, so the warps drift apart by up to the ring's depth.
 constexpr int kFilterRing = 4;
+constexpr int kFilterThreads = NT + 32;  // consumers + the producer warp
 constexpr uint32_t kChunkBytes = CHUNK4 * 16u;
 struct FilterSmem {
   float4 ring[kFilterRing][CHUNK4];
-  float stage[kLaneStage * NT];  // the lane columns
+  float stage[kLaneStage * NT];  // the consumer lanes' columns
   double red[64];
-  uint64_t full[kFilterRing];
+  uint64_t full[kFilterRing];   // a stage has landed (the copy's bytes)
+  uint64_t empty[kFilterRing];  // a stage has been read by every consumer warp
+  int issued;                   // chunks the producer issued
+  int late;                     // a wait ran out
 };
 constexpr size_t kFilterSmemBytes = sizeof(FilterSmem);
 
-__global__ void __launch_bounds__(NT, 2) k_filter(const StreamPlan P, const float* __restrict__ scores) {
+__global__ void __launch_bounds__(kFilterThreads, 2) k_filter(const StreamPlan P, const float* __restrict__ scores) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   FilterSmem& S = *reinterpret_cast<FilterSmem*>(smem_raw);
   const int64_t r = blockIdx.y;
   const int cta = blockIdx.x, ncta = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float* row = scores + r * P.stride;
   RowCtl* c = ctl_of(P, r);
   const int head = row_head(row, P.n);
   const float4* x4 = reinterpret_cast<const float4*>(row + head);
   const int64_t nchunks = ((P.n - head) >> 2) / CHUNK4;
   const int mine = cta < nchunks ? (int)((nchunks - 1 - cta) / ncta) + 1 : 0;  // this block's chunks
+  auto chunk = [&](int it) { return x4 + (cta + (int64_t)it * ncta) * CHUNK4; };
   // test knob: rows 1, 5, 9, ... issue no copy for their first chunk, so
-  // that its bounded wait runs out (rows 3, 7, ... time out in the recovery
+  // that the waits for it run out (rows 3, 7, ... time out in the recovery
   // kernel instead)
   const bool force_to = P.force_timeout && !P.shard && (r & 3) == 1;
   // the scores are the caller's: the first stages are requested before
   // waiting for the kernel that wrote the bracket
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kFilterRing; ++s) mbar_init(&S.full[s], 1u);
+    for (int s = 0; s < kFilterRing; ++s) {
+      mbar_init(&S.full[s], 1u);
+      mbar_init(&S.empty[s], (uint32_t)NW);
+    }
     for (int s = force_to ? 1 : 0; s < kFilterRing && s < mine; ++s) {
       mbar_arrive_expect_tx(&S.full[s], kChunkBytes);
-      bulk_load(S.ring[s], x4 + (cta + (int64_t)s * ncta) * CHUNK4, kChunkBytes, &S.full[s]);
+      bulk_load(S.ring[s], chunk(s), kChunkBytes, &S.full[s]);
     }
+    S.issued = min(kFilterRing, mine);
+    S.late = 0;
   }
   __syncthreads();
   wait_prior_grid();
-  const FilterCtx f = filter_ctx(P, r, c);
-  float* col = S.stage + threadIdx.x;
-  const float2 naL2 = make_float2(-f.aL, -f.aL), naR2 = make_float2(-f.aR, -f.aR), c22 = make_float2(f.c2, f.c2);
   const uint32_t limit = spin_limit_of(P.spin_limit);
+  const FilterCtx f = filter_ctx(P, r, c);
+  float* col = S.stage + (threadIdx.x < NT ? threadIdx.x : 0);
   FilterAcc acc;
   uint32_t bad = 0u, ovf = 0u;
-  int it = 0;
-  bool late = false;
-  for (; it < mine; ++it) {
-    const int slot = it % kFilterRing;
-    const bool ok = mbar_wait_bounded(&S.full[slot], (uint32_t)(it / kFilterRing) & 1u, limit);
-    const float4* st = S.ring[slot] + threadIdx.x;
-    float4 v[U];
+  if (warp == NW) {
+    // producer: refill a stage once every consumer warp has released it
+    if (lane == 0) {
+      int it = kFilterRing;
+      for (; it < mine; ++it) {
+        const int slot = it % kFilterRing;
+        if (!mbar_wait_bounded(&S.empty[slot], (uint32_t)(it / kFilterRing - 1) & 1u, limit)) {
+          S.late = 1;
+          break;
+        }
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&S.full[slot], kChunkBytes);
+        bulk_load(S.ring[slot], chunk(it), kChunkBytes, &S.full[slot]);
+      }
+      if (it > S.issued) S.issued = it;
+    }
+  } else {
+    const float2 naL2 = make_float2(-f.aL, -f.aL), naR2 = make_float2(-f.aR, -f.aR);
+    const float2 c22 = make_float2(f.c2, f.c2);
+    for (int it = 0; it < mine; ++it) {
+      const int slot = it % kFilterRing;
+      // a warp-uniform decision: every lane polls, the warp gives up together
+      const bool ok = mbar_wait_bounded(&S.full[slot], (uint32_t)(it / kFilterRing) & 1u, limit);
+      if (!__all_sync(0xffffffffu, ok)) {
+        S.late = 1;  // a copy that did not land in time: the row's results are void
+        break;
+      }
+      const float4* st = S.ring[slot] + threadIdx.x;
+      float4 v[U];
 #pragma unroll
-    for (int u = 0; u < U; ++u) v[u] = st[u * NT];
-    filter_chunk(v, naL2, naR2, c22, [&](int i) { return reinterpret_cast<const float*>(st + (i >> 2) * NT)[i & 3]; },
-                 col, acc);
-    // every thread is done with the stage: refill it
-    if (!__syncthreads_and(ok)) {
-      late = true;  // a copy that did not complete in time: the row's results are void
-      break;
-    }
-    if (threadIdx.x == 0 && it + kFilterRing < mine) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&S.full[slot], kChunkBytes);
-      bulk_load(S.ring[slot], x4 + (cta + (int64_t)(it + kFilterRing) * ncta) * CHUNK4, kChunkBytes,
-                &S.full[slot]);
-    }
-    if (__any_sync(0xffffffffu, acc.ncol > kLaneStage - 4 * U)) {
-      flush_warp(f, col, acc.ncol, bad, ovf);
-      acc.ncol = 0;
+      for (int u = 0; u < U; ++u) v[u] = st[u * NT];
+      filter_chunk(v, naL2, naR2, c22,
+                   [&](int i) { return reinterpret_cast<const float*>(st + (i >> 2) * NT)[i & 3]; }, col, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.empty[slot]);
+      if (__any_sync(0xffffffffu, acc.ncol > kLaneStage - 4 * U)) {
+        flush_warp(f, col, acc.ncol, bad, ovf);
+        acc.ncol = 0;
+      }
     }
   }
-  if (late) {
-    // chunks it .. it + kFilterRing - 1 may still be in flight: let them land
-    // (again with a limit) before the block leaves; the band kernel reads
-    // the flag and solves nothing
+  __syncthreads();
+  if (S.late) {
+    // the last chunks issued may still be in flight: let them land (again
+    // with a limit) before the block leaves; the band kernel reads the flag
+    // and solves nothing
     if (threadIdx.x == 0) {
-      for (int j = it; j < mine && j < it + kFilterRing; ++j)
+      for (int j = max(0, S.issued - kFilterRing); j < S.issued; ++j)
         (void)mbar_wait_bounded(&S.full[j % kFilterRing], (uint32_t)(j / kFilterRing) & 1u, limit);
       atomicOr(&c->flags, ROW_TIMEOUT);
     }
     __syncthreads();
   }
-  filter_finish(P, r, row, c, cta, ncta, S.red, col, f, acc, head, nchunks * CHUNK4, bad, ovf);
+  filter_finish<kFilterThreads>(P, r, row, c, cta, ncta, S.red, col, f, acc, head, nchunks * CHUNK4, bad, ovf);
 }
 
 // ===========================================================================
@@ -2171,7 +2199,7 @@ cudaError_t stream_occupancy(StreamOcc* out) {
   e = cudaFuncSetAttribute(k_recover, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RecSmem::kTotal);
   if (e != cudaSuccess) return e;
   int fb = 0, rb = 0, mb = 0, qb = 0, ab = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, NT, kFilterSmemBytes);
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fb, k_filter, kFilterThreads, kFilterSmemBytes);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&mb, k_memb<false, false>, NT, 0);
   if (e != cudaSuccess) return e;
@@ -2243,7 +2271,7 @@ cudaError_t launch_stream_fwd(const StreamPlan& P, const float* scores, float* p
   }
   {
     Launch l("k_filter", st);
-    e = launch_pdl(k_filter, dim3(P.Gf, rows), dim3(NT), kFilterSmemBytes, st, P, scores);
+    e = launch_pdl(k_filter, dim3(P.Gf, rows), dim3(kFilterThreads), kFilterSmemBytes, st, P, scores);
     if (e != cudaSuccess) return e;
   }
   {
@@ -2337,7 +2365,7 @@ cudaError_t launch_shard_filter(const StreamPlan& P, const float* scores, uint32
   }
   {
     Launch l("k_filter", st);
-    k_filter<<<dim3(P.Gf, rows), NT, kFilterSmemBytes, st>>>(P, scores);
+    k_filter<<<dim3(P.Gf, rows), kFilterThreads, kFilterSmemBytes, st>>>(P, scores);
   }
   {
     Launch l("k_shard_pack", st);
