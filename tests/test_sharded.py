@@ -2,7 +2,8 @@
 
 On CPU: the shard bounds, the lockstep driver, and the torch.distributed
 driver with two gloo ranks (the exchanges the GPU ranks would make with
-NCCL).  On a GPU: the sharded forward and backward, run as 2-4 ranks in
+NCCL), both on a toy program and on the real forward and backward programs
+with the library's buffer layout and the kernel calls stubbed.  On a GPU: the sharded forward and backward, run as 2-4 ranks in
 lockstep on one device, against the one-GPU operator and the oracle."""
 import math
 import os
@@ -94,6 +95,87 @@ def test_distributed_driver_with_two_gloo_ranks():
         assert p.exitcode == 0
     for _, r in res:
         assert tuple(r) == _expected(world)
+
+
+class _HostShard(sh.ShardedTopK):
+    """The real per-rank object (layout from the C library, exchange buffers
+    on the CPU) with its kernel calls replaced by rank-stamped fills: the real
+    forward and backward programs then make the real exchanges, and the
+    finish calls check what arrived."""
+
+    def _check_shard(self, x):
+        return x
+
+    def fwd_sample(self, x):
+        self.x_sample.zero_()
+        self.x_sample[self.rank::self.world] = self.rank + 1  # disjoint slots, as the sample keys
+        self.x_hist.fill_(self.rank + 1)
+
+    def fwd_filter(self, x):
+        self.x_meta.fill_(100 + self.rank)
+        self.x_fpart.fill_(50 + self.rank)
+        self.x_band.fill_(self.rank + 0.5)
+
+    def _ranks_of(self, t):
+        return [t.view(self.world, -1)[w] for w in range(self.world)]
+
+    def fwd_finish(self, x):
+        W = self.world
+        assert all(int(v) == (i % W) + 1 for i, v in enumerate(self.x_sample.tolist()))
+        assert bool((self.x_hist == W * (W + 1) // 2).all())
+        for w, (m, f, b) in enumerate(zip(self._ranks_of(self.g_meta), self._ranks_of(self.g_fpart),
+                                          self._ranks_of(self.g_band))):
+            assert bool((m == 100 + w).all()) and bool((f == 50 + w).all()) and bool((b == w + 0.5).all())
+        rows = self.rows
+        return sh.ShardResult(torch.zeros_like(x), torch.zeros(rows, dtype=torch.float64),
+                              torch.zeros(rows, dtype=torch.float64),
+                              torch.full((rows,), lt.ROW_CERTIFIED, dtype=torch.int32))
+
+    def bwd_partials(self, x, g, b, with_alpha):
+        self.x_parts.fill_(7 + self.rank)
+
+    def bwd_finish(self, x, g, b, with_alpha):
+        for w, t in enumerate(self._ranks_of(self.g_parts)):
+            assert bool((t == 7 + w).all())
+        return torch.zeros_like(x), torch.zeros(self.rows, dtype=torch.float64), None
+
+
+def _real_program_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rows, n_total = 2, 200_003
+        obj = _HostShard(rows, n_total, world, rank, 1000.0, 0.1, torch.device("cpu"))
+        x = torch.zeros(rows, obj.n)
+        res = sh.run_distributed(sh.forward_program(obj, x))
+        grad, gk, ga = sh.run_distributed(sh.backward_program(obj, x, x, res.b))
+        q.put((rank, bool((res.status == lt.ROW_CERTIFIED).all()), tuple(grad.shape)))
+    except Exception as e:  # the parent reports it
+        q.put((rank, repr(e), None))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_real_programs_exchange_over_two_gloo_ranks():
+    """The sharded forward and backward programs, with the library's own
+    layout and buffers, make their exchanges over torch.distributed (gloo
+    here, NCCL on GPUs): sums and rank-major gathers arrive as the kernels of
+    every rank wrote them."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_real_program_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, ok, shape in res:
+        assert ok is True, f"rank {rank}: {ok}"
+        lo, hi = sh.shard_bounds(200_003, world, rank)
+        assert shape == (2, hi - lo)
 
 
 # ---------------------------------------------------------------------------
