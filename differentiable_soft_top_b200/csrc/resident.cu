@@ -520,7 +520,7 @@ __global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
         sorted = band;
       }
       SolveIn in{aL, aR, f.nL, f.nR, f.SL, f.SR, ra.k, ra.alpha, inva};
-      solve_run<NT>(in, sorted, f.M, dscr, dlink, red, &s_out);
+      solve_run_warp<NT>(in, sorted, f.M, dscr, dlink, &s_out);
       if (s_out.status & ROW_CERTIFIED) { solved = true; break; }
       if (attempt >= a.max_widen) break;
       // widen once on the side that missed; the other edge moves to the old

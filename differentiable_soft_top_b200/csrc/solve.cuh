@@ -725,6 +725,121 @@ __device__ void solve_run(const SolveIn in, const uint32_t* keys, int M, double*
   __syncthreads();
 }
 
+// Warp-wide exclusive scan of affine maps (the shuffle part of
+// block_excl_scan_aff): lane l receives the composition of lanes 0..l-1
+// (kForward) or of lanes 31..l+1.
+template <bool kForward>
+__device__ __forceinline__ Aff warp_excl_scan_aff(Aff v) {
+  const int lane = threadIdx.x & 31;
+  Aff inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    Aff oth;
+    if (kForward) {
+      oth.F = __shfl_up_sync(0xffffffffu, inc.F, o);
+      oth.S = __shfl_up_sync(0xffffffffu, inc.S, o);
+      if (lane >= o) inc = aff_then(oth, inc);
+    } else {
+      oth.F = __shfl_down_sync(0xffffffffu, inc.F, o);
+      oth.S = __shfl_down_sync(0xffffffffu, inc.S, o);
+      if (lane + o < 32) inc = aff_then(oth, inc);
+    }
+  }
+  Aff exl;
+  if (kForward) {
+    exl.F = __shfl_up_sync(0xffffffffu, inc.F, 1);
+    exl.S = __shfl_up_sync(0xffffffffu, inc.S, 1);
+    if (lane == 0) exl = aff_id();
+  } else {
+    exl.F = __shfl_down_sync(0xffffffffu, inc.F, 1);
+    exl.S = __shfl_down_sync(0xffffffffu, inc.S, 1);
+    if (lane == 31) exl = aff_id();
+  }
+  return exl;
+}
+
+// solve_run with its scans taken by one warp: the whole block computes the
+// link factors (the exps), then warp 0 walks the run in 32 chunks, with
+// shuffles instead of block barriers between its phases.  The same
+// recurrences, knot values, certification and closed form as solve_run; only
+// the chunking, hence the rounding order of the compositions, differs.  For
+// the one-block rows, where other blocks on the SM keep the issue slots busy
+// while the other warps wait.  dA: >= M doubles, dL: >= M + 1 doubles.  Every
+// thread must call it; *out in shared memory.
+template <int NT>
+__device__ void solve_run_warp(const SolveIn in, const uint32_t* keys, int M, double* dA, double* dL,
+                               SolveOut* out) {
+  const double inva = in.inva;
+  const bool finL = isfinite(in.aL), finR = isfinite(in.aR);
+  const double xL = finL ? (double)in.aL : -CUDART_INF;
+  const double xR = finR ? (double)in.aR : CUDART_INF;
+  const double A0 = finL ? in.SL : 0.0;  // prefix state at a_L
+  const double B0 = finR ? in.SR : 0.0;  // suffix state at a_R
+  auto y = [&](int i) -> double { return i < 0 ? xL : (i >= M ? xR : (double)key2f(keys[i])); };
+  for (int i = threadIdx.x; i <= M; i += NT) dL[i] = link(y(i - 1), y(i), inva);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    // odd chunk lengths: the lanes' chunk starts fall in distinct banks
+    const int qe = ((M + 31) / 32) | 1;
+    const int i0 = min(M, lane * qe), i1 = min(M, i0 + qe);
+    // forward: chunk map, scan, A at every value
+    Aff m = aff_id();
+    for (int i = i0; i < i1; ++i) m = aff_then(m, Aff{dL[i], 1.0});
+    const Aff fe = warp_excl_scan_aff<true>(m);
+    double A = fma(A0, fe.F, fe.S);  // prefix state at y_{i0 - 1}
+    for (int i = i0; i < i1; ++i) {
+      A = fma(A, dL[i], 1.0);
+      dA[i] = A;
+    }
+    // A_{M-1} (A0 when M = 0) from the lane whose chunk ends the run
+    const double Alast = M > 0 ? __shfl_sync(0xffffffffu, A, (M - 1) / qe) : A0;
+    // backward: chunk map, scan, knot values
+    Aff mb = aff_id();
+    for (int i = i1 - 1; i >= i0; --i) mb = aff_then(mb, Aff{dL[i + 1], 1.0});
+    const Aff be = warp_excl_scan_aff<false>(mb);
+    const double Bin = fma(B0, be.F, be.S);  // B_{i1}, anchored at y_{i1}
+    int icand = -1;
+    double B = Bin;
+    for (int i = i1 - 1; i >= i0; --i) {
+      const double S = 0.5 * dA[i] + (double)((long long)(M - 1 - i) + in.nR) - 0.5 * B * dL[i + 1];
+      if (icand < 0 && S >= in.k) icand = i;
+      B = fma(B, dL[i + 1], 1.0);
+    }
+    const double Bfirst = M > 0 ? __shfl_sync(0xffffffffu, B, 0) : B0;  // B_0
+    const int i_star = __reduce_max_sync(0xffffffffu, icand);
+    const int jn = i_star + 1;
+    // B_jn from the lane whose chunk holds jn
+    double Bj = Bin;
+    if (jn < M && jn >= i0 && jn < i1)
+      for (int i = i1 - 1; i >= jn; --i) Bj = fma(Bj, dL[i + 1], 1.0);
+    const double Bp_run = __shfl_sync(0xffffffffu, Bj, jn < M ? jn / qe : 0);
+    __syncwarp();  // dA of every lane visible to lane 0
+    if (lane == 0) {
+      const double S_aL = finL ? 0.5 * in.SL + (double)((long long)M + in.nR) - 0.5 * Bfirst * dL[0] : CUDART_INF;
+      const double S_aR = finR ? 0.5 * Alast * dL[M] + (double)in.nR - 0.5 * in.SR : -CUDART_INF;
+      out->M = M;
+      out->S_aL = S_aL;
+      out->S_aR = S_aR;
+      if (S_aL >= in.k && S_aR < in.k) {
+        const double xj = i_star < 0 ? xL : y(i_star);
+        const double Ai = i_star < 0 ? A0 : dA[i_star];
+        const double xj1 = jn < M ? y(jn) : xR;
+        const double Bp = jn < M ? Bp_run : B0;
+        const double cj = (double)((long long)(M - 1 - i_star) + in.nR);
+        out->b = closed_form_root(xj, xj1, Ai, Bp, cj, in.k, in.alpha);
+        out->sumf = sum_f_at(xj, xj1, Ai, Bp, out->b, inva);
+        out->status = ROW_CERTIFIED;
+      } else {
+        out->b = 0.0;
+        out->sumf = 0.0;
+        out->status = (!(S_aL >= in.k) ? ROW_MISS_LEFT : 0u) | (!(S_aR < in.k) ? ROW_MISS_RIGHT : 0u);
+      }
+    }
+  }
+  __syncthreads();
+}
+
 template <int NT>
 __device__ __forceinline__ uint32_t block_minmax_u32(uint32_t v, bool is_max, uint32_t* scratch) {
   constexpr int NW = NT / 32;
