@@ -363,6 +363,26 @@ def test_bracket_and_tails_match_oracle(orc, name, n):
         assert st["sum_f"] == pytest.approx(out["sumf"][i])
 
 
+@pytest.mark.parametrize("dist,n,k", [
+    ("normal", 4096, 64.0),       # the two ranks in different first-level bins (~60 keys and 1)
+    ("uniform", 16384, 256.0),    # both ranks in one first-level bin of ~200 keys
+    ("uniform", 16384, 8192.0),   # ranks near the median, bins of ~370 and ~510 keys
+])
+def test_one_block_bracket_selection_matches_oracle(orc, dist, n, k):
+    """The one-block path selects the bracket's two sample ranks by a radix
+    selection in the block (no sort of the sample): the oracle's order
+    statistics exactly, whether the two ranks share first-level bins or not."""
+    rows, alpha = 3, 0.05
+    x = make_scores(dist, rows, n, seed=21)
+    g = make_grad(rows, n, seed=22)
+    out = gpu_run(x, g, k, alpha, stats=True, params=lt.Params(seed=7))
+    for i in range(rows):
+        st = out["stats"][i]
+        aL, aR, _, _ = orc.bracket(x[i], k, alpha, int(st["sample_m"]), lt.DEFAULT_Z, 7, i)
+        assert np.float32(st["a_L"]) == np.float32(aL) and np.float32(st["a_R"]) == np.float32(aR), f"row {i}"
+        check_row(orc, x[i], g[i], out["p"][i], out["grad"][i], out["b"][i], out["gk"][i], k, alpha, f"row {i}")
+
+
 def test_deterministic():
     w, x, g = case("c3", n=3_000_000)
     a = gpu_run(x, g, w.k, w.alpha)
