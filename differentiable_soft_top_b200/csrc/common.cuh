@@ -604,15 +604,18 @@ __device__ __forceinline__ double alpha_grad(double m, double SZ, double SGZ, do
 // and min/max run on the half-rate ALU pipe; here the left/right indicators
 // come from saturating multiplies instead (a saturated product of NaN is 0):
 //   L = sat(-(x - aL) 2^126)      1 if x < aL, else 0
-//   R = sat((x - aR) 2^126 + 1)   1 if x >= aR, else 0
+//   R = sat(-(aR - x) 2^126 + 1)  1 if x >= aR, else 0
 // Every normal difference is at least 2^-126 in magnitude, so the product
 // reaches 1; a difference below that is flushed to zero (--ftz), which places
 // a score within a subnormal step of an edge on the band's side of it.  A
 // score is in the band iff L + R == 0 (NaN lands there).  The tail term is
-//   e = exp2(-|min(x - aL, aR - x)| c2),
+//   e = exp2(min(min(x - aL, aR - x) c2, 0)),
 // which is exp((x - aL)/alpha) on the left and exp((aR - x)/alpha) on the
-// right; the absolute value keeps the band's (unused) terms below 1, so that
-// 0 * e is never 0 * inf.
+// right (where the inner min is not positive); the clamp at 0 makes the
+// band's (unused) terms 1, so that 0 * e is never 0 * inf.  Both differences
+// are formed as they are used (aR - x, not -(x - aR)) and the clamp replaces
+// an absolute value, so no operand needs a sign or magnitude change: the
+// min/max and exp2 instructions take none for free.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float mul_sat(float a, float b) {
   float r;
@@ -660,24 +663,24 @@ struct Side2 {  // two scores (packed fp32x2 arithmetic where it exists)
 };
 __device__ __forceinline__ Side classify(float x, float aL, float aR, float c2) {
   const float dl = x - aL;
-  const float dr = x - aR;
+  const float ndr = aR - x;
   Side s;
   s.L = mul_sat(dl, -0x1p126f);
-  s.R = fma_sat(dr, 0x1p126f, 1.0f);
-  s.e = exp2f(-fabsf(fminf(dl, -dr)) * c2);
+  s.R = fma_sat(ndr, -0x1p126f, 1.0f);
+  s.e = exp2f(fminf(fminf(dl, ndr) * c2, 0.0f));
   return s;
 }
-// classify for two scores: naL = (-aL, -aL), naR = (-aR, -aR), c22 = (c2, c2).
-// The same operations as classify (x - aL as x + (-aL) is the same rounded
-// value), so both give identical sides and terms.
-__device__ __forceinline__ Side2 classify2(float2 x, float2 naL, float2 naR, float2 c22) {
+// classify for two scores: naL = (-aL, -aL), aR2 = (aR, aR), c22 = (c2, c2).
+// The same rounded values as classify (x - aL as x + (-aL); aR - x as one
+// fused x * (-1) + aR), so both give identical sides and terms.
+__device__ __forceinline__ Side2 classify2(float2 x, float2 naL, float2 aR2, float2 c22) {
   const float2 dl = add2(x, naL);
-  const float2 dr = add2(x, naR);
+  const float2 ndr = fma2(x, make_float2(-1.0f, -1.0f), aR2);
   Side2 s;
   s.L = make_float2(mul_sat(dl.x, -0x1p126f), mul_sat(dl.y, -0x1p126f));
-  s.R = make_float2(fma_sat(dr.x, 0x1p126f, 1.0f), fma_sat(dr.y, 0x1p126f, 1.0f));
-  const float2 a = mul2(make_float2(fminf(dl.x, -dr.x), fminf(dl.y, -dr.y)), c22);
-  s.e = make_float2(exp2f(-fabsf(a.x)), exp2f(-fabsf(a.y)));
+  s.R = make_float2(fma_sat(ndr.x, -0x1p126f, 1.0f), fma_sat(ndr.y, -0x1p126f, 1.0f));
+  const float2 t = mul2(make_float2(fminf(dl.x, ndr.x), fminf(dl.y, ndr.y)), c22);
+  s.e = make_float2(exp2f(fminf(t.x, 0.0f)), exp2f(fminf(t.y, 0.0f)));
   return s;
 }
 

@@ -112,7 +112,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
   uint32_t bad = 0u;
   // sum of the scores scaled by 2^-64: +-inf or NaN shows here
   float2 fs2 = make_float2(0.0f, 0.0f);
-  const float2 naL2 = make_float2(-aL, -aL), naR2 = make_float2(-aR, -aR), c22 = make_float2(c2, c2);
+  const float2 naL2 = make_float2(-aL, -aL), aR2 = make_float2(aR, aR), c22 = make_float2(c2, c2);
   const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
   constexpr int kB = 4;
   const int head = row_head(row, n);
@@ -136,7 +136,7 @@ __device__ Filtered filter_row(const float* row, int n, float aL, float aR, floa
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const float2 x2 = h ? make_float2(q.z, q.w) : make_float2(q.x, q.y);
-          const Side2 sd = classify2(x2, naL2, naR2, c22);
+          const Side2 sd = classify2(x2, naL2, aR2, c22);
           float2 L = sd.L, R = sd.R;
           if (!act) L = R = make_float2(0.0f, 0.0f);
           const float bit = (float)(1u << (4 * u + 2 * h));

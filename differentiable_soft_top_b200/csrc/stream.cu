@@ -501,7 +501,7 @@ struct FilterAcc {
 // copied into the lane's column (stride NT) from at(i), the lane's i-th score
 // of the chunk (i = 4u + component).
 template <typename At>
-__device__ __forceinline__ void filter_chunk(const float4 (&v)[U], float2 naL2, float2 naR2, float2 c22,
+__device__ __forceinline__ void filter_chunk(const float4 (&v)[U], float2 naL2, float2 aR2, float2 c22,
                                              const At& at, float* col, FilterAcc& a) {
   const float2 k64 = make_float2(0x1p-64f, 0x1p-64f);
   float2 pl2 = make_float2(0.0f, 0.0f), pr2 = pl2, cl2 = pl2, ob2 = pl2;
@@ -510,7 +510,7 @@ __device__ __forceinline__ void filter_chunk(const float4 (&v)[U], float2 naL2, 
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const float2 x2 = h ? make_float2(v[u].z, v[u].w) : make_float2(v[u].x, v[u].y);
-      const Side2 sd = classify2(x2, naL2, naR2, c22);
+      const Side2 sd = classify2(x2, naL2, aR2, c22);
       const float bit = (float)(1u << (4 * u + 2 * h));
       pl2 = fma2(sd.L, sd.e, pl2);
       pr2 = fma2(sd.R, sd.e, pr2);
@@ -613,7 +613,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
   const FilterCtx f = filter_ctx(P, r, c);
   float* col = stage + threadIdx.x;  // this lane's column, stride NT
   float4* scratch = reinterpret_cast<float4*>(stage + kLaneStage * NT) + threadIdx.x * U;  // U float4
-  const float2 naL2 = make_float2(-f.aL, -f.aL), naR2 = make_float2(-f.aR, -f.aR), c22 = make_float2(f.c2, f.c2);
+  const float2 naL2 = make_float2(-f.aL, -f.aL), aR2 = make_float2(f.aR, f.aR), c22 = make_float2(f.c2, f.c2);
   FilterAcc acc;
   uint32_t bad = 0u, ovf = 0u;
   for (int64_t q = cta; q < nchunks; q += ncta) {
@@ -627,7 +627,7 @@ __device__ void filter_phase(const StreamPlan& P, int64_t r, const float* __rest
     // the lane's chunk goes to its scratch slot only when it holds in-band
     // values (read back there by position)
     bool spilled = false;
-    filter_chunk(v, naL2, naR2, c22,
+    filter_chunk(v, naL2, aR2, c22,
                  [&](int i) {
                    if (!spilled) {
 #pragma unroll
@@ -726,7 +726,7 @@ __global__ void __launch_bounds__(kFilterThreads, 2) k_filter(const StreamPlan P
       if (it > S.issued) S.issued = it;
     }
   } else {
-    const float2 naL2 = make_float2(-f.aL, -f.aL), naR2 = make_float2(-f.aR, -f.aR);
+    const float2 naL2 = make_float2(-f.aL, -f.aL), aR2 = make_float2(f.aR, f.aR);
     const float2 c22 = make_float2(f.c2, f.c2);
     for (int it = 0; it < mine; ++it) {
       const int slot = it % kFilterRing;
@@ -740,7 +740,7 @@ __global__ void __launch_bounds__(kFilterThreads, 2) k_filter(const StreamPlan P
       float4 v[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) v[u] = st[u * NT];
-      filter_chunk(v, naL2, naR2, c22,
+      filter_chunk(v, naL2, aR2, c22,
                    [&](int i) { return reinterpret_cast<const float*>(st + (i >> 2) * NT)[i & 3]; }, col, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.empty[slot]);
