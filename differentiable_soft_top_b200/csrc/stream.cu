@@ -723,7 +723,8 @@ __global__ void __launch_bounds__(kFilterThreads, 2) k_filter(const StreamPlan P
         mbar_arrive_expect_tx(&S.full[slot], kChunkBytes);
         bulk_load(S.ring[slot], chunk(it), kChunkBytes, &S.full[slot]);
       }
-      if (it > S.issued) S.issued = it;
+      const int issued = it < mine ? it : mine;  // chunks [0, issued) were requested
+      if (issued > S.issued) S.issued = issued;
     }
   } else {
     const float2 naL2 = make_float2(-f.aL, -f.aL), aR2 = make_float2(f.aR, f.aR);
