@@ -5,8 +5,10 @@
 // the threshold, and the bracket needs two order statistics of the
 // localization sample.  Here: a stable LSD radix sort (whole rows in the
 // full-sort fallback), an MSD radix selection of two ranks (the one-block
-// path's sample), and a bitonic network (the band, the streaming band's root
-// bin, and the sample when a widening needs other ranks).
+// path's sample), a one-pass bucket sort over a known key range (a band, a
+// small streaming band, the streaming band's root bin), and a bitonic network
+// (the bucket sort's fallback when outliers crowd a bucket, and the sample
+// when a widening needs other ranks).
 //
 // Radix sort: 8-bit digits, four passes.  Each warp owns one contiguous segment of the
 // keys and walks it 32 keys at a time; __match_any_sync groups the lanes that
