@@ -67,6 +67,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' step times")
     ap.add_argument("--no-full-sort", action="store_true", help="skip the full-sort branch comparison")
+    ap.add_argument("--no-context", action="store_true", help="skip the library read and copy timings")
     ap.add_argument("--no-flush", action="store_true")
     ap.add_argument("--n", type=int, default=0, help="scale the workload to n scores per row (k keeps its ratio)")
     return ap.parse_args()
@@ -374,6 +375,25 @@ def timed_calls(torch, fn, steps, flush, stream, dist, dev):
         ev.append((s0, s1))
     torch.cuda.synchronize(dev)
     return max_over_ranks(sum(a.elapsed_time(c) for a, c in ev) / steps, dist, dev)
+
+
+def bandwidth_context(torch, x, dev, dist, flush, steps, peak, filter_ms):
+    """Library kernels on the same scores, for the rate a pass that only reads
+    gets from HBM (the measured peak is a copy): torch's sum over the row
+    (reads 4n bytes) and a device copy of it (reads and writes 4n bytes),
+    each after the L2 flush, beside the filter pass (reads 4n bytes)."""
+    stream = torch.cuda.current_stream(dev)
+    y = torch.empty_like(x)
+    ms_sum = timed_calls(torch, lambda: x.sum(), steps, flush, stream, dist, dev)
+    ms_copy = timed_calls(torch, lambda: y.copy_(x), steps, flush, stream, dist, dev)
+    del y
+    nb = x.numel() * 4
+    out = {"torch_sum_ms": ms_sum, "torch_sum_gbs": nb / (ms_sum * 1e-3) / 1e9,
+           "copy_ms": ms_copy, "copy_gbs": 2 * nb / (ms_copy * 1e-3) / 1e9, "peak_gbs": peak}
+    if filter_ms:
+        out["k_filter_ms"] = filter_ms
+        out["k_filter_gbs"] = nb / (filter_ms * 1e-3) / 1e9
+    return out
 
 
 def graph_replay(torch, step, dev, dist, flush, steps):
@@ -685,6 +705,11 @@ def main():
     if not args.no_dftopk:
         dftopk = dftopk_vs_lapsum(lt, torch, w, x, dev, dist, flush, args.steps)
 
+    context = None
+    if path == "streaming" and not args.no_context:
+        fk = kernels.get("k_filter")
+        context = bandwidth_context(torch, x, dev, dist, flush, args.steps, peak,
+                                    fk["ms_per_launch"] if fk else None)
     full_sort = None
     if not args.no_full_sort:
         full_sort = full_sort_branch(lt, torch, w, x, dev, dist, flush, min(args.steps, 10), peak)
@@ -738,6 +763,7 @@ def main():
         "sparse_forward": sparse,
         "dftopk_forward": dftopk,
         "full_sort": full_sort,
+        "bandwidth_context": context,
         "configs": configs,
         "gpu_launches": launches,
         "clocks": clk,
