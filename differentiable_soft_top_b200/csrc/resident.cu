@@ -250,12 +250,13 @@ __device__ __forceinline__ float membership(float x, float bh, float bl, float c
   const float s = fma_sat(d, 0x1p126f, 1.0f);
   return fmaf(s, fmaf(-2.0f, h, 1.0f), h);
 }
-// membership for two scores with packed arithmetic: the same operations, so
-// the same values bit for bit (nbh = (-bh, -bh), nbl = (-bl, -bl))
-__device__ __forceinline__ float2 membership2(float2 x, float2 nbh, float2 nbl, float2 c22) {
+// membership for two scores with packed arithmetic: the same values bit for
+// bit (nbh = (-bh, -bh), nbl = (-bl, -bl), nc2 = -c2).  The exponent is the
+// scalar product |d| (-c2), which equals -|d c2| exactly and needs no
+// separate sign or magnitude change before the exp2.
+__device__ __forceinline__ float2 membership2(float2 x, float2 nbh, float2 nbl, float nc2) {
   const float2 d = add2(add2(x, nbh), nbl);
-  const float2 a = mul2(d, c22);
-  const float2 h = mul2(make_float2(exp2f(-fabsf(a.x)), exp2f(-fabsf(a.y))), make_float2(0.5f, 0.5f));
+  const float2 h = mul2(make_float2(exp2f(fabsf(d.x) * nc2), exp2f(fabsf(d.y) * nc2)), make_float2(0.5f, 0.5f));
   const float2 s = make_float2(fma_sat(d.x, 0x1p126f, 1.0f), fma_sat(d.y, 0x1p126f, 1.0f));
   return fma2(s, fma2(make_float2(-2.0f, -2.0f), h, make_float2(1.0f, 1.0f)), h);
 }
@@ -272,7 +273,7 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
   const float c2 = (float)(inva * (double)kLog2e);
   const float bh = __double2float_rn(b);
   const float bl = __double2float_rn(b - (double)bh);
-  const float2 nbh2 = make_float2(-bh, -bh), nbl2 = make_float2(-bl, -bl), c22 = make_float2(c2, c2);
+  const float2 nbh2 = make_float2(-bh, -bh), nbl2 = make_float2(-bl, -bl);
   double ps = 0.0;
   const bool nonfinite = (status & ROW_NAN_OUT) != 0u;
   if (a.dftopk) {
@@ -345,8 +346,8 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
             const int v = v0 + u * NT;
             if (decltype(checked)::value && v >= n4) break;
             const float4 x = xs[u];
-            const float2 p01 = membership2(make_float2(x.x, x.y), nbh2, nbl2, c22);
-            const float2 p23 = membership2(make_float2(x.z, x.w), nbh2, nbl2, c22);
+            const float2 p01 = membership2(make_float2(x.x, x.y), nbh2, nbl2, -c2);
+            const float2 p23 = membership2(make_float2(x.z, x.w), nbh2, nbl2, -c2);
             if (decltype(want_ps)::value) ps += (double)((p01.x + p01.y) + (p23.x + p23.y));
             stg_stream(d4 + v, make_float4(p01.x, p01.y, p23.x, p23.y));
           }
