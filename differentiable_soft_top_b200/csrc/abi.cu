@@ -131,7 +131,17 @@ struct ResPlan {
   int m, bcap;
   Ranks rk;
 };
-ResPlan resident_plan(int64_t n, double k, const Resolved& R) {
+// The sample size balances the sample and its selection (cost ~ m) against
+// the band (size ~ n / sqrt(m)): m ~ (z n sqrt(q (1 - q)))^(2/3).  A batch
+// of the longest rows (more rows than the GPU holds at once, `batch`, of
+// more than 8192 scores) is bound by the throughput of its rows rather than
+// the latency of one, and there a larger sample (2.5x, in whole multiples of
+// the block, at most 1024) shrinks the band and its sort and solve by more
+// than the longer sample costs: fwd+bwd of 2048 x 16384, 227.8 -> 223.9 us;
+// of 600 x 16384, 102.1 -> 97.6 us.  For rows of 4096 and 8192 scores the
+// same factor lost (107.6 -> 110.6 and 142.3 -> 146 us), and beyond 1024 the
+// sample's shared memory costs a resident row per SM.
+ResPlan resident_plan(int64_t n, double k, const Resolved& R, bool batch) {
   ResPlan p;
   const double q = k / (double)n;
   if (R.m_user) {
@@ -139,6 +149,8 @@ ResPlan resident_plan(int64_t n, double k, const Resolved& R) {
   } else {
     const double opt = std::pow(R.z * (double)n * std::sqrt(q * (1.0 - q)), 2.0 / 3.0);
     p.m = std::min(2048, std::max(128, round_up((int64_t)std::ceil(opt), 32)));
+    if (batch && n > 8192)
+      p.m = std::max(p.m, std::min(1024, round_up((int64_t)std::ceil(2.5 * opt), kResidentThreads)));
   }
   p.rk = sample_ranks(n, k, p.m, R.z);
   const double M_est = (double)(p.rk.rank_hi - p.rk.rank_lo + 1) * (double)n / (double)p.m;
@@ -317,7 +329,7 @@ int fwd_impl(const float* scores, int64_t rows, int64_t n, int64_t row_stride, d
   unsigned char* ws = static_cast<unsigned char*>(workspace);
 
   if (res) {
-    const ResPlan rp = resident_plan(n, k, R);
+    const ResPlan rp = resident_plan(n, k, R, rows > (int64_t)dev->sm_count * kResidentBlocksPerSm);
     ResidentFwd a{};
     a.scores = scores;
     a.rows = rows;
@@ -779,7 +791,7 @@ extern "C" int lapsum_topk_fwd_noalloc(const float* scores, int64_t rows, int64_
   unsigned char* ws = nullptr;
   if (!cuda_ok(noalloc_scratch(&ws))) return LAPSUM_ECUDA;
 
-  const ResPlan rp = resident_plan(n, k, R);
+  const ResPlan rp = resident_plan(n, k, R, rows > (int64_t)dev->sm_count * kResidentBlocksPerSm);
   ResidentFwd a{};
   a.scores = scores;
   a.rows = rows;

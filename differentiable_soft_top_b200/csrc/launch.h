@@ -56,6 +56,7 @@ constexpr bool kPdlTail = true;
 // row, the row held in shared memory)
 constexpr int64_t kResidentMaxN = 16384;
 constexpr int kResidentThreads = 256;
+constexpr int kResidentBlocksPerSm = 4;  // one-block forward rows resident per SM (its launch bound)
 
 // Sparse output of a forward pass: the entries with p >= eps as (index, p)
 // pairs, row r at r * cap; count[r] receives the number of such entries

@@ -399,7 +399,7 @@ __device__ void finish_row(const ResidentFwd& a, int64_t r, const float* src, do
 constexpr int64_t kRowSmemMaxN = 4096;
 
 template <bool kSmemRow>
-__global__ void __launch_bounds__(NT, 4) k_row_fwd(const ResidentFwd a) {
+__global__ void __launch_bounds__(NT, kResidentBlocksPerSm) k_row_fwd(const ResidentFwd a) {
   extern __shared__ __align__(16) unsigned char smem[];
   const ResLayout L = res_layout(a.n, a.m, a.bcap, kSmemRow);
   uint32_t* samp = reinterpret_cast<uint32_t*>(smem + L.samp);
