@@ -135,12 +135,15 @@ struct ResPlan {
 // the band (size ~ n / sqrt(m)): m ~ (z n sqrt(q (1 - q)))^(2/3).  A batch
 // of the longest rows (more rows than the GPU holds at once, `batch`, of
 // more than 8192 scores) is bound by the throughput of its rows rather than
-// the latency of one, and there a larger sample (2.5x, in whole multiples of
-// the block, at most 1024) shrinks the band and its sort and solve by more
-// than the longer sample costs: fwd+bwd of 2048 x 16384, 227.8 -> 223.9 us;
-// of 600 x 16384, 102.1 -> 97.6 us.  For rows of 4096 and 8192 scores the
-// same factor lost (107.6 -> 110.6 and 142.3 -> 146 us), and beyond 1024 the
-// sample's shared memory costs a resident row per SM.
+// the latency of one; where the balanced size is already at least 384 (the
+// band is large), a sample of 1024 shrinks the band and its sort and solve
+// by more than the longer sample costs.  Fwd+bwd of 2048 x 16384 (the tied
+// batch): k = 256, 228 -> 224 us; k = 1024, 394 -> 324 us; k = 4096, 560 ->
+// 556 us; k = 256 at alpha 0.05, 271 -> 268 us; 600 rows at k = 256, 102 ->
+// 98 us.  Where the balanced size is smaller the larger sample lost (k = 64:
+// 202 -> 206 us; 2048 x 12001 at k = 200: 195 -> 197 us; rows of 4096 and
+// 8192 scores: 108 -> 111 and 142 -> 146 us), and beyond 1024 the sample's
+// shared memory costs a resident row per SM.
 ResPlan resident_plan(int64_t n, double k, const Resolved& R, bool batch) {
   ResPlan p;
   const double q = k / (double)n;
@@ -149,8 +152,7 @@ ResPlan resident_plan(int64_t n, double k, const Resolved& R, bool batch) {
   } else {
     const double opt = std::pow(R.z * (double)n * std::sqrt(q * (1.0 - q)), 2.0 / 3.0);
     p.m = std::min(2048, std::max(128, round_up((int64_t)std::ceil(opt), 32)));
-    if (batch && n > 8192)
-      p.m = std::max(p.m, std::min(1024, round_up((int64_t)std::ceil(2.5 * opt), kResidentThreads)));
+    if (batch && n > 8192 && opt >= 384.0) p.m = std::max(p.m, 1024);
   }
   p.rk = sample_ranks(n, k, p.m, R.z);
   const double M_est = (double)(p.rk.rank_hi - p.rk.rank_lo + 1) * (double)n / (double)p.m;
